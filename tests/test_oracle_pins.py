@@ -1,0 +1,451 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each test checks an oracle function against a closed form, an invariant of the
+mathematics, an independent formulation built from library routines, brute
+force on tiny inputs, or central finite differences.  The mutation tests at the
+end plant plausible mistakes in the oracle (on the CPU) and confirm that these
+pins catch them.
+"""
+import itertools
+import math
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import slora_oracle as O
+from contextual_sparsity_lora_svd_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def tsilu(x):
+    """torch's SiLU on a float64 numpy array (an independent implementation)."""
+    return torch.nn.functional.silu(torch.from_numpy(x)).numpy()
+
+
+def colnorm(x):
+    return torch.linalg.vector_norm(torch.from_numpy(x), dim=0).numpy()
+
+
+# --------------------------------------------------------------------------- SVD
+@pytest.mark.parametrize("n,k,r", [(40, 24, 5), (24, 40, 8), (30, 30, 1)])
+def test_svd_prepare_closed_form(n, k, r):
+    sw = synth.decaying_weight(n, k, seed=7)
+    L, U = O.svd_prepare(sw.W, r)
+    # rank-r product equals the construction's leading triplets exactly
+    Wr = (sw.U[:, :r] * sw.s[None, :r]) @ sw.V[:, :r].T
+    np.testing.assert_allclose(U @ L.T, Wr, atol=1e-12 * np.abs(sw.W).max())
+    # L = V_r Sigma_r: column norms are the singular values
+    np.testing.assert_allclose(np.linalg.norm(L, axis=0), sw.s[:r], rtol=1e-12)
+    # U has orthonormal columns
+    np.testing.assert_allclose(U.T @ U, np.eye(r), atol=1e-12)
+    # Eckart-Young: residual energy is the tail of the spectrum
+    res = np.sum((sw.W - U @ L.T) ** 2)
+    np.testing.assert_allclose(res, np.sum(sw.s[r:] ** 2), rtol=1e-10)
+
+
+def test_decaying_weight_rms_and_spectrum():
+    sw = synth.decaying_weight(64, 48, seed=3)
+    assert abs(np.sqrt(np.mean(sw.W ** 2)) - 0.02) < 1e-12
+    sv = np.linalg.svd(sw.W, compute_uv=False)
+    np.testing.assert_allclose(sv, sw.c * np.arange(1, 49) ** -0.7, rtol=1e-10)
+
+
+# ---------------------------------------------------------------------- scores
+def _full_rank_factors(W):
+    m = min(W.shape)
+    return O.svd_prepare(W, m)
+
+
+def test_ffn_score_full_rank_equals_exact_activation_norm():
+    """With r = min(n, k) the estimate is exact, so the score is the true
+    SwiGLU activation norm over context tokens (computed with torch here)."""
+    tok = synth.Tokens(batch=3, seq=7, ctx_len=np.array([5, 7, 2], np.int32))
+    d, d_ff = 12, 18
+    X = synth.gaussian((tok.T, d), 1.0, 11)
+    Wg = synth.decaying_weight(d_ff, d, 12).W * 20
+    Wu = synth.decaying_weight(d_ff, d, 13).W * 20
+    Lg, Ug = _full_rank_factors(Wg)
+    Lu, Uu = _full_rank_factors(Wu)
+    C, _ = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    got = O.ffn_scores(O.project(X[C], Lg), O.project(X[C], Lu), Ug, Uu)
+    exact = colnorm(tsilu(X[C] @ Wg.T) * (X[C] @ Wu.T))
+    np.testing.assert_allclose(got, exact, rtol=1e-11)
+
+
+def test_ffn_score_rank_r_matches_factor_estimate():
+    """At rank r the score is the activation norm of the rank-r weights."""
+    tok = synth.Tokens.uniform(2, 8)
+    d, d_ff, r = 16, 20, 3
+    X = synth.gaussian((tok.T, d), 1.0, 21)
+    swg = synth.decaying_weight(d_ff, d, 22)
+    swu = synth.decaying_weight(d_ff, d, 23)
+    Lg, Ug = O.svd_prepare(swg.W, r)
+    Lu, Uu = O.svd_prepare(swu.W, r)
+    C, _ = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    Wg_r = (swg.U[:, :r] * swg.s[:r]) @ swg.V[:, :r].T
+    Wu_r = (swu.U[:, :r] * swu.s[:r]) @ swu.V[:, :r].T
+    exact = colnorm(tsilu(X[C] @ Wg_r.T) * (X[C] @ Wu_r.T))
+    got = O.ffn_scores(O.project(X[C], Lg), O.project(X[C], Lu), Ug, Uu)
+    np.testing.assert_allclose(got, exact, rtol=1e-10)
+
+
+def test_qk_score_full_rank_equals_exact_norm_product():
+    tok = synth.Tokens(batch=2, seq=6, ctx_len=np.array([4, 3], np.int32))
+    d, H, hd = 10, 2, 4
+    X = synth.gaussian((tok.T, d), 1.0, 31)
+    Wq = synth.decaying_weight(H * hd, d, 32).W
+    Wk = synth.decaying_weight(H * hd, d, 33).W
+    Lq, Uq = _full_rank_factors(Wq)
+    Lk, Uk = _full_rank_factors(Wk)
+    C, _ = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    got = O.qk_scores(O.project(X[C], Lq), O.project(X[C], Lk), Uq, Uk, H, H, hd)
+    exact = (colnorm(X[C] @ Wq.T) * colnorm(X[C] @ Wk.T)).reshape(H, hd)
+    np.testing.assert_allclose(got, exact, rtol=1e-11)
+
+
+def test_qk_score_gram_identity():
+    """||P U^T e_c||^2 = u_c^T (P^T P) u_c: the Gram form of the same score."""
+    rg = synth.rng(5)
+    P_q, P_k = rg.standard_normal((9, 3)), rg.standard_normal((9, 3))
+    U_q, U_k = rg.standard_normal((8, 3)), rg.standard_normal((8, 3))
+    Gq, Gk = P_q.T @ P_q, P_k.T @ P_k
+    nq = np.sqrt(np.einsum("cr,rs,cs->c", U_q, Gq, U_q))
+    nk = np.sqrt(np.einsum("cr,rs,cs->c", U_k, Gk, U_k))
+    got = O.qk_scores(P_q, P_k, U_q, U_k, 2, 2, 4)
+    np.testing.assert_allclose(got.ravel(), nq * nk, rtol=1e-12)
+
+
+def test_qk_gqa_equals_mha_on_replicated_keys():
+    """A GQA group score equals the sum of MHA scores of its query heads when
+    the shared key head is replicated once per query head."""
+    rg = synth.rng(6)
+    H, KV, hd, r, t = 4, 2, 3, 2, 7
+    P_q, P_k = rg.standard_normal((t, r)), rg.standard_normal((t, r))
+    U_q, U_k = rg.standard_normal((H * hd, r)), rg.standard_normal((KV * hd, r))
+    gqa = O.qk_scores(P_q, P_k, U_q, U_k, H, KV, hd)
+    U_k_rep = np.concatenate([U_k[(h // 2) * hd:(h // 2 + 1) * hd] for h in range(H)])
+    mha = O.qk_scores(P_q, P_k, U_q, U_k_rep, H, H, hd)
+    np.testing.assert_allclose(gqa, mha.reshape(KV, 2, hd).sum(axis=1), rtol=1e-12)
+
+
+def test_hand_worked_scores_closed_form():
+    """Two context tokens, rank 2, identity-like factors worked by hand:
+    P = [[1,0],[0,2]], U = [[1,0],[0,1],[1,1]] for gate and up alike, so
+    g_hat = u_hat = [[1,0,1],[0,2,2]] and act = g * sigmoid(g) * g.
+    score_0 = sigma(1), score_1 = 4 sigma(2), score_2 = sqrt(sigma(1)^2 + 16 sigma(2)^2)."""
+    P = np.array([[1.0, 0.0], [0.0, 2.0]])
+    U = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])
+    s1 = 1.0 / (1.0 + math.exp(-1.0))
+    s2 = 1.0 / (1.0 + math.exp(-2.0))
+    want = [s1, 4 * s2, math.sqrt(s1 * s1 + 16 * s2 * s2)]
+    got = O.ffn_scores(P, P, U, U)
+    np.testing.assert_allclose(got, want, rtol=1e-15)
+    assert O.topk_select(got, 2).tolist() == [1, 2]
+
+
+def test_golden_regression_fixture():
+    """Oracle outputs on a reduced workload-0 case, written by
+    tests/golden/make_golden.py (which calls only the oracle): guards against
+    unintended changes to the oracle's arithmetic."""
+    from tests.golden.make_golden import compute
+    with open(os.path.join(GOLDEN, "ffn_reduced_w0.json")) as f:
+        g = json.load(f)
+    cur = compute()
+    assert cur["idx"] == g["idx"]
+    for key in ("scores", "out_sum", "dX_sum", "grad_norms"):
+        np.testing.assert_allclose(cur[key], g[key], rtol=1e-12)
+
+
+# ------------------------------------------------------------------- selection
+def _brute_force_topk(score, k):
+    best = None
+    for sub in itertools.combinations(range(len(score)), k):
+        key = (sum(score[j] for j in sub), tuple(-j for j in sub))
+        if best is None or key > best[0]:
+            best = (key, sub)
+    return list(best[1])
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_brute_force_with_ties(seed):
+    rg = synth.rng(100 + seed)
+    N = int(rg.integers(1, 10))
+    k = int(rg.integers(0, N + 1))
+    score = rg.integers(0, 4, size=N).astype(float)   # integer scores: many exact ties
+    got = O.topk_select(score, k).tolist()
+    assert got == sorted(got)
+    assert got == _brute_force_topk(score.tolist(), k)
+
+
+def test_topk_separation_large():
+    rg = synth.rng(9)
+    score = rg.random(1000)
+    idx = O.topk_select(score, 137)
+    mask = np.zeros(1000, bool)
+    mask[idx] = True
+    assert mask.sum() == 137 and score[mask].min() >= score[~mask].max()
+
+
+@pytest.mark.parametrize("N,s,k", [(688, 0.5, 344), (11008, 0.5, 5504), (128, 0.5, 64),
+                                   (14336, 0.0, 14336), (14336, 0.3, 10036), (14336, 0.5, 7168),
+                                   (14336, 0.7, 4301), (14336, 0.9, 1434), (7, 0.99, 1)])
+def test_keep_count(N, s, k):
+    assert O.keep_count(N, s) == k
+
+
+def test_select_sparsity_zero_keeps_all():
+    score = synth.rng(2).random(33)
+    assert O.topk_select(score, O.keep_count(33, 0.0)).tolist() == list(range(33))
+
+
+# ---------------------------------------------------------------- LoRA linear
+def _lin_case(seed, n=9, k=7, r=3, tok=None):
+    tok = tok or synth.Tokens(batch=2, seq=5, ctx_len=np.array([3, 4], np.int32))
+    X = synth.gaussian((tok.T, k), 1.0, seed)
+    W0 = synth.gaussian((n, k), 0.3, seed + 1)
+    A = synth.gaussian((r, k), 0.3, seed + 2)
+    B = synth.gaussian((n, r), 0.3, seed + 3)
+    return tok, X, W0, A, B
+
+
+def _merged(W0, A, B, s):
+    return W0 + s * (B @ A)
+
+
+def test_linear_dense_equals_merged_weight():
+    tok, X, W0, A, B = _lin_case(40)
+    Y, _, _ = O.linear_fwd("none", X, None, tok.batch, tok.seq, tok.ctx_len, W0, A, B, 0.7, None)
+    np.testing.assert_allclose(Y, X @ _merged(W0, A, B, 0.7).T, rtol=1e-12)
+
+
+def test_linear_out_rows_all_channels_is_dense():
+    tok, X, W0, A, B = _lin_case(41)
+    C, Oo = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    idx = np.arange(W0.shape[0])
+    Yc, Yo, _ = O.linear_fwd("out_rows", X, None, tok.batch, tok.seq, tok.ctx_len, W0, A, B, 0.5, idx)
+    dense = X @ _merged(W0, A, B, 0.5).T
+    np.testing.assert_allclose(Yc, dense[C], rtol=1e-12)
+    np.testing.assert_allclose(Yo, dense[Oo], rtol=1e-12)
+
+
+def test_linear_out_rows_slice_equals_masked_dense():
+    tok, X, W0, A, B = _lin_case(42)
+    C, Oo = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    idx = np.array([1, 4, 5, 8])
+    Yc, Yo, _ = O.linear_fwd("out_rows", X, None, tok.batch, tok.seq, tok.ctx_len, W0, A, B, 0.5, idx)
+    dense = X @ _merged(W0, A, B, 0.5).T
+    np.testing.assert_allclose(Yc, dense[C][:, idx], rtol=1e-12)
+    np.testing.assert_allclose(Yo, dense[Oo], rtol=1e-12)
+
+
+def test_linear_in_cols_slice_equals_masked_dense():
+    tok, X, W0, A, B = _lin_case(43)
+    C, Oo = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    idx = np.array([0, 2, 3, 6])
+    Xc = X[C][:, idx]
+    Y, _, _ = O.linear_fwd("in_cols", Xc, X[Oo], tok.batch, tok.seq, tok.ctx_len, W0, A, B, 0.5, idx)
+    Xmask = np.zeros_like(X)
+    Xmask[np.ix_(C, idx)] = Xc
+    Xmask[Oo] = X[Oo]
+    np.testing.assert_allclose(Y, Xmask @ _merged(W0, A, B, 0.5).T, rtol=1e-12)
+
+
+def _fd(f, x, eps=1e-6):
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + eps
+        fp = f()
+        x[i] = old - eps
+        fm = f()
+        x[i] = old
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+@pytest.mark.parametrize("side", ["none", "out_rows", "in_cols"])
+def test_linear_bwd_finite_differences(side):
+    tok, X, W0, A, B = _lin_case(50 + len(side))
+    C, Oo = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    s = 0.8
+    idx = np.array([0, 3, 4]) if side == "in_cols" else np.array([1, 2, 6, 7])
+    if side == "in_cols":
+        Xin, Xout = X[C][:, idx].copy(), X[Oo].copy()
+    else:
+        Xin, Xout = X.copy(), None
+    rg = synth.rng(77)
+
+    def fwd():
+        return O.linear_fwd(side, Xin, Xout, tok.batch, tok.seq, tok.ctx_len, W0, A, B, s, idx)
+
+    Y1, Y2, XA = fwd()
+    dY1 = rg.standard_normal(Y1.shape)
+    dY2 = rg.standard_normal(Y2.shape) if Y2 is not None else None
+
+    def loss():
+        a, b, _ = fwd()
+        v = np.sum(a * dY1)
+        return v + (np.sum(b * dY2) if b is not None else 0.0)
+
+    dXc, dXo, dA, dB = O.linear_bwd(side, Xin, Xout, XA, dY1, dY2, tok.batch, tok.seq,
+                                    tok.ctx_len, W0, A, B, s, idx)
+    np.testing.assert_allclose(dA, _fd(loss, A), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dB, _fd(loss, B), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dXc, _fd(loss, Xin), rtol=1e-6, atol=1e-8)
+    if Xout is not None:
+        np.testing.assert_allclose(dXo, _fd(loss, Xout), rtol=1e-6, atol=1e-8)
+
+
+# ----------------------------------------------------------------------- FFN
+def _ffn_layer(seed, d=6, d_ff=10, r=2, scale=0.9, wscale=0.6):
+    g = lambda shape, k: synth.gaussian(shape, wscale, seed + k)
+    return dict(Wg=g((d_ff, d), 1), Wu=g((d_ff, d), 2), Wd=g((d, d_ff), 3),
+                Ag=g((r, d), 4), Bg=g((d_ff, r), 5), Au=g((r, d), 6), Bu=g((d_ff, r), 7),
+                Ad=g((r, d_ff), 8), Bd=g((d, r), 9), scale=scale)
+
+
+def _dense_swiglu(X, lay, mask=None):
+    """Textbook SwiGLU with merged LoRA weights, torch SiLU; ``mask`` zeroes
+    the gate/up rows (weight and LoRA-B) of skipped channels."""
+    s = lay["scale"]
+    Wg = _merged(lay["Wg"], lay["Ag"], lay["Bg"], s)
+    Wu = _merged(lay["Wu"], lay["Au"], lay["Bu"], s)
+    Wd = _merged(lay["Wd"], lay["Ad"], lay["Bd"], s)
+    if mask is not None:
+        Wg = Wg * mask[:, None]
+        Wu = Wu * mask[:, None]
+    return (tsilu(X @ Wg.T) * (X @ Wu.T)) @ Wd.T
+
+
+def test_ffn_all_channels_is_dense_swiglu():
+    tok = synth.Tokens(batch=2, seq=6, ctx_len=np.array([4, 5], np.int32))
+    lay = _ffn_layer(60)
+    X = synth.gaussian((tok.T, 6), 1.0, 61)
+    out, _ = O.ffn_fwd(X, tok.batch, tok.seq, tok.ctx_len, lay, np.arange(10))
+    np.testing.assert_allclose(out, _dense_swiglu(X, lay), rtol=1e-11)
+
+
+def test_ffn_slice_equals_masked_dense():
+    tok = synth.Tokens(batch=2, seq=6, ctx_len=np.array([4, 5], np.int32))
+    lay = _ffn_layer(62)
+    X = synth.gaussian((tok.T, 6), 1.0, 63)
+    idx = np.array([0, 2, 3, 7, 9])
+    mask = np.zeros(10)
+    mask[idx] = 1
+    out, _ = O.ffn_fwd(X, tok.batch, tok.seq, tok.ctx_len, lay, idx)
+    C, Oo = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    np.testing.assert_allclose(out[C], _dense_swiglu(X, lay, mask)[C], rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(out[Oo], _dense_swiglu(X, lay)[Oo], rtol=1e-11)
+
+
+def _ffn_fd_check(lay, X, tok, idx, tol=1e-6):
+    rg = synth.rng(88)
+    dOut = rg.standard_normal((tok.T, lay["Wd"].shape[0]))
+
+    def loss():
+        out, _ = O.ffn_fwd(X, tok.batch, tok.seq, tok.ctx_len, lay, idx)
+        return np.sum(out * dOut)
+
+    out, saved = O.ffn_fwd(X, tok.batch, tok.seq, tok.ctx_len, lay, idx)
+    gr = O.ffn_bwd(X, dOut, lay, idx, saved)
+    np.testing.assert_allclose(gr["dX"], _fd(loss, X), rtol=tol, atol=1e-8)
+    for name in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd"):
+        np.testing.assert_allclose(gr["d" + name], _fd(loss, lay[name]), rtol=tol, atol=1e-8)
+
+
+def test_ffn_bwd_finite_differences():
+    tok = synth.Tokens(batch=2, seq=6, ctx_len=np.array([4, 5], np.int32))
+    lay = _ffn_layer(64)
+    X = synth.gaussian((tok.T, 6), 1.0, 65)
+    _ffn_fd_check(lay, X, tok, np.array([1, 2, 5, 6, 8]))
+
+
+def test_ffn_zero_grad_rows_for_skipped_channels():
+    """No output tokens: skipped channels get exactly zero LoRA-B rows (gate,
+    up) and zero LoRA-A columns (down)."""
+    tok = synth.Tokens(batch=2, seq=5, ctx_len=np.array([5, 5], np.int32))
+    lay = _ffn_layer(66)
+    X = synth.gaussian((tok.T, 6), 1.0, 67)
+    dOut = synth.gaussian((tok.T, 6), 1.0, 68)
+    idx = np.array([0, 4, 5, 9])
+    skip = np.setdiff1d(np.arange(10), idx)
+    out, saved = O.ffn_fwd(X, tok.batch, tok.seq, tok.ctx_len, lay, idx)
+    gr = O.ffn_bwd(X, dOut, lay, idx, saved)
+    assert np.all(gr["dBg"][skip] == 0) and np.all(gr["dBu"][skip] == 0)
+    assert np.all(gr["dAd"][:, skip] == 0)
+    assert np.any(gr["dBg"][idx] != 0) and np.any(gr["dAd"][:, idx] != 0)
+
+
+def test_ffn_fwd_bwd_estimator_path_small_case():
+    """End-to-end oracle on a reduced workload-0 shape: the chosen set is the
+    top-k of the scores and equals the full-sparsity-0 dense result at s=0."""
+    tok = synth.Tokens.uniform(1, 32)
+    case = synth.ffn_case(tok, d=16, d_ff=40, r_svd=4, r_lora=4, sparsity=0.5)
+    lay = dict(Wg=case.Wg.W, Wu=case.Wu.W, Wd=case.Wd.W, Ag=case.Ag, Bg=case.Bg, Au=case.Au,
+               Bu=case.Bu, Ad=case.Ad, Bd=case.Bd, scale=1.0)
+    for nm, sw in (("g", case.Wg), ("u", case.Wu)):
+        lay["L" + nm], lay["U" + nm] = O.svd_prepare(sw.W, 4)
+    res = O.ffn_fwd_bwd(case.X, case.dOut, tok.batch, tok.seq, tok.ctx_len, lay, 0.5)
+    assert res["k"] == 20 and len(res["idx"]) == 20
+    sc = res["scores"]
+    mask = np.zeros(40, bool)
+    mask[res["idx"]] = True
+    assert sc[mask].min() >= sc[~mask].max()
+    dense = O.ffn_fwd_bwd(case.X, case.dOut, tok.batch, tok.seq, tok.ctx_len, lay, 0.0)
+    np.testing.assert_allclose(dense["out"], _dense_swiglu(case.X, lay), rtol=1e-10)
+
+
+def test_context_rows_layout():
+    C, Oo = O.context_rows(3, 4, [1, 4, 0])
+    assert C.tolist() == [0, 4, 5, 6, 7]
+    assert Oo.tolist() == [1, 2, 3, 8, 9, 10, 11]
+
+
+# --------------------------------------------------------- planted mistakes
+def test_planted_silu_grad_sign_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "silu_grad", lambda x: 1.0 / (1.0 + np.exp(x)) * (1 + x))
+    tok = synth.Tokens(batch=1, seq=4, ctx_len=np.array([3], np.int32))
+    lay = _ffn_layer(70, d=3, d_ff=4)
+    X = synth.gaussian((tok.T, 3), 1.0, 71)
+    with pytest.raises(AssertionError):
+        _ffn_fd_check(lay, X, tok, np.array([0, 2]))
+
+
+def test_planted_dropped_lora_term_is_caught(monkeypatch):
+    real = O.linear_fwd
+
+    def broken(side, X_ctx, X_out, b, s_, c, W0, A, B, scale, idx):
+        return real(side, X_ctx, X_out, b, s_, c, W0, A, B, 0.0 if side == "out_rows" else scale, idx)
+
+    monkeypatch.setattr(O, "linear_fwd", broken)
+    with pytest.raises(AssertionError):
+        test_linear_out_rows_slice_equals_masked_dense()
+
+
+def test_planted_transposed_factor_is_caught(monkeypatch):
+    real = O.ffn_scores
+    monkeypatch.setattr(O, "ffn_scores", lambda Pg, Pu, Ug, Uu: real(Pu, Pg, Ug, Uu))
+    with pytest.raises(AssertionError):
+        test_ffn_score_full_rank_equals_exact_activation_norm()
+
+
+def test_planted_tie_break_is_caught(monkeypatch):
+    def upper_wins(score, k):
+        order = np.lexsort((-np.arange(score.size), -np.asarray(score)))
+        return np.sort(order[:k])
+    monkeypatch.setattr(O, "topk_select", upper_wins)
+    with pytest.raises(AssertionError):
+        for seed in range(12):
+            test_topk_brute_force_with_ties(seed)
+
+
+def test_oracle_package_exports():
+    for name in O.__all__:
+        assert hasattr(oracle, name)
