@@ -1,0 +1,397 @@
+"""Benchmark of the contextually sparse LoRA hot path on one Llama-2-7B-shaped
+SwiGLU FFN layer (d=4096, d_ff=11008, batch 8 x seq 512, last 25% of each
+sequence dense output tokens, SVD rank 8, LoRA rank 16 on gate/up/down,
+sparsity 50%, bf16, forward + backward).
+
+One step = slora_ffn_fwd_bwd: estimate + select + sliced forward + sliced
+backward for one batch.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): data parallel, every rank runs its
+own batch (weak scaling); the six LoRA gradients, packed in one flat buffer,
+are summed across ranks with one NCCL all-reduce per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from contextual_sparsity_lora_svd_b200 import synth  # noqa: E402
+
+WORKLOAD = synth.WORKLOADS[1]
+METRIC = "sparse LoRA fwd+bwd tokens/s; sliced-GEMM % bf16 peak; estimator HBM GB/s"
+UNIT = "tokens/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return dict(hbm=m["hbm_gbs"], bf16=m["bf16_tflops"], bf16_sus=m["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every `period` s."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period: float = 0.002):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self.stop_ev = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": getattr(self, "max_mhz", None), "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ inputs
+_CASE = {}
+
+
+def make_case(batch=None, seq=None):
+    """The full workload (default) or its first `batch` sequences of length
+    `seq`: the same weights and the same leading rows of X and dOut."""
+    import dataclasses
+    w = WORKLOAD
+    if "full" not in _CASE:
+        tok = synth.Tokens.uniform(w["batch"], w["seq"], w["out_frac"])
+        _CASE["full"] = synth.ffn_case(tok, w["d"], w["d_ff"], w["r_svd"], w["r_lora"],
+                                       w["sparsity"], bf16=True, workload=1, fast=True)
+    full = _CASE["full"]
+    if batch is None and seq is None:
+        return full
+    assert seq == w["seq"]
+    tok = synth.Tokens.uniform(batch, seq, w["out_frac"])
+    return dataclasses.replace(full, tokens=tok, X=full.X[:tok.T], dOut=full.dOut[:tok.T])
+
+
+class GpuLayer:
+    """Device copies of one layer plus outputs/grads/workspace for bench steps."""
+
+    def __init__(self, case, L):
+        self.L, self.case = L, case
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(
+            torch.bfloat16).cuda()
+        w = WORKLOAD
+        d, F, r, rs = w["d"], w["d_ff"], w["r_lora"], w["r_svd"]
+        self.d, self.F, self.r = d, F, r
+        self.t = {k: bf(getattr(case, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+        for k in ("Wg", "Wu", "Wd"):
+            self.t[k] = bf(getattr(case, k).W)
+        # offline prepare (not timed): estimator factors of gate/up, Wd^T for the down proj
+        self.t["Wd_t"] = torch.empty(F, d, dtype=torch.bfloat16, device="cuda")
+        for nm, n, k in (("g", F, d), ("u", F, d)):
+            self.t["L" + nm] = torch.empty(k, rs, device="cuda")
+            self.t["U" + nm] = torch.empty(n, rs, device="cuda")
+            L.slora_svd_prepare(self.t["W" + nm], rs, self.t["L" + nm], self.t["U" + nm], seed=7)
+        Ld = torch.empty(F, rs, device="cuda")
+        Ud = torch.empty(d, rs, device="cuda")
+        L.slora_svd_prepare(self.t["Wd"], rs, Ld, Ud, W_t=self.t["Wd_t"], seed=7)
+        del self.t["Wd"]
+        T = case.tokens.T
+        self.X = bf(case.X)
+        self.dOut = bf(case.dOut)
+        self.out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        self.dX = torch.empty_like(self.out)
+        shapes = [(r, d), (F, r), (r, d), (F, r), (r, F), (d, r)]
+        self.gflat = torch.zeros(sum(a * b for a, b in shapes), device="cuda")
+        self.grads, o = [], 0
+        for a, b in shapes:
+            self.grads.append(self.gflat[o:o + a * b].view(a, b))
+            o += a * b
+        self.idx = torch.empty(F, dtype=torch.int32, device="cuda")
+        t = self.t
+        self.layer = L.ffn_layer_struct(d, F, rs, r, case.lora_scale, t["Wg"], t["Wu"], t["Wd_t"],
+                                        t["Ag"], t["Bg"], t["Au"], t["Bu"], t["Ad"], t["Bd"],
+                                        t["Lg"], t["Ug"], t["Lu"], t["Uu"])
+        self.gstruct = L.ffn_grads_struct(*self.grads)
+        tok = case.tokens
+        self.args, self.keep = L.ffn_args(L.BF16, self.layer, tok.batch, tok.seq, tok.ctx_len,
+                                          case.sparsity, self.X, self.dOut, self.out, self.dX,
+                                          self.gstruct, self.idx)
+        need = L.workspace_size("slora_ffn_fwd_bwd", self.args)
+        self.ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        self.ws_bytes = L.c_sz(need)
+
+    def step(self, stream):
+        import ctypes
+        L = self.L
+        st = L.lib().slora_ffn_fwd_bwd(*self.args, L.ptr(self.ws), ctypes.byref(self.ws_bytes),
+                                       stream.cuda_stream)
+        if st != 0:
+            raise L.SloraError("slora_ffn_fwd_bwd", st, L.lib().slora_last_error_string().decode())
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_step_time(case, reps=1):
+    """Seconds for the oracle's fwd+bwd of `case` (estimate, select, sliced
+    fwd/bwd), on this host's cores.  Estimator factors: the closed-form top-r
+    singular triplets of the construction."""
+    from oracle import slora_oracle as O
+    r = WORKLOAD["r_svd"]
+    lay = dict(Wg=case.Wg.W, Wu=case.Wu.W, Wd=case.Wd.W, Ag=case.Ag, Bg=case.Bg, Au=case.Au,
+               Bu=case.Bu, Ad=case.Ad, Bd=case.Bd, scale=case.lora_scale)
+    for nm, sw in (("g", case.Wg), ("u", case.Wu)):
+        lay["L" + nm] = sw.V[:, :r] * sw.s[None, :r]
+        lay["U" + nm] = sw.U[:, :r].copy()
+    tok = case.tokens
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        O.ffn_fwd_bwd(case.X, case.dOut, tok.batch, tok.seq, tok.ctx_len, lay, case.sparsity)
+    return (time.perf_counter() - t0) / reps
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def set_threads():
+    n = str(host_cores())
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ.setdefault(v, n)
+    torch.set_num_threads(int(n))
+
+
+CPU_SAMPLE = dict(batch=1, seq=512)  # one sequence: 384 context + 128 output tokens
+
+
+def cpu_baseline():
+    case = make_case(**CPU_SAMPLE)
+    oracle_step_time(case)  # warm the BLAS pools
+    t = oracle_step_time(case, reps=3)
+    T = case.tokens.T
+    return {"value": T / t, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+            "sample": f"{CPU_SAMPLE['batch']} x {CPU_SAMPLE['seq']} tokens of the same layer "
+                      f"(ctx 384 + out 128), fp64 NumPy oracle, 3 reps after 1 warm-up"}
+
+
+# ------------------------------------------------------------------- arms
+def config_dict(world):
+    w = WORKLOAD
+    return {"workload": w["name"], "model": "Llama-2-7B FFN layer (random init, decaying spectrum)",
+            "global_batch": w["batch"] * world, "seq_len": w["seq"], "d": w["d"],
+            "d_ff": w["d_ff"], "ctx_frac": 1 - w["out_frac"], "sparsity": w["sparsity"],
+            "r_svd": w["r_svd"], "r_lora": w["r_lora"],
+            "parallelism": f"dp{world}" if world > 1 else "single",
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    set_threads()
+    case = make_case(**CPU_SAMPLE)
+    for _ in range(args.warmup):
+        oracle_step_time(case)
+    ts = [oracle_step_time(case) for _ in range(args.steps)]
+    T = case.tokens.T
+    v = T / float(np.mean(ts))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(ts)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(world),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                             "sample": f"each step: {T} tokens ({CPU_SAMPLE['batch']} x "
+                                       f"{CPU_SAMPLE['seq']}) of the workload, fp64 NumPy oracle"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world):
+    from contextual_sparsity_lora_svd_b200 import _lib as L
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    case = make_case()
+    G = GpuLayer(case, L)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    T = case.tokens.T
+
+    def one_step():
+        G.step(stream)
+        if world > 1:
+            torch.distributed.all_reduce(G.gflat)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    L.profile_enable(True)
+    n0 = L.launch_count()
+    with ClockSampler(dev) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            one_step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    launches = L.launch_count() - n0
+    prof = {c: L.profile_read(c) for c in L.KERNEL_CLASSES}
+    L.profile_enable(False)
+    ms = float(sum(a.elapsed_time(b) for a, b in ev))
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * T / (ms_step / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    Xh = G.X.cpu().pin_memory()
+    dOh = G.dOut.cpu().pin_memory()
+    outh = torch.empty_like(G.out, device="cpu").pin_memory()
+    dXh = torch.empty_like(G.dX, device="cpu").pin_memory()
+    gh = torch.empty_like(G.gflat, device="cpu").pin_memory()
+    e2e_steps = max(1, min(args.steps, 10))
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        G.X.copy_(Xh, non_blocking=True)
+        G.dOut.copy_(dOh, non_blocking=True)
+        one_step()
+        outh.copy_(G.out, non_blocking=True)
+        dXh.copy_(G.dX, non_blocking=True)
+        gh.copy_(G.gflat, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = Xh.numel() * 2 + dOh.numel() * 2
+    d2h = outh.numel() * 2 + dXh.numel() * 2 + gh.numel() * 4
+
+    # ---- roofline of the dominant kernel class (by device time)
+    kernels = {}
+    for c, (n, kms, work) in prof.items():
+        if n:
+            kernels[c] = {"launches_per_step": n / args.steps, "ms_per_step": kms / args.steps,
+                          "share": kms / ms if ms > 0 else None}
+    gemm_cls = max(("gemm_tc", "gemm_simt"), key=lambda c: prof[c][1])
+    n_g, ms_g, fl_g = prof[gemm_cls]
+    achieved = fl_g / (ms_g / 1e3) / 1e12 if ms_g > 0 else 0.0
+    roof = {"kernel": gemm_cls, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"],
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16"], "traffic": None,
+            "peak_kind": f"bf16 burst, {pk['src']}",
+            "frac_of_sustained": achieved / pk["bf16_sus"],
+            "flops_per_launch": fl_g / max(n_g, 1), "ms_per_launch": ms_g / max(n_g, 1)}
+    n_e, ms_e, by_e = prof["estimate"]
+    n_s, ms_s, by_s = prof["select"]
+    est = {"ms_per_step": (ms_e + ms_s) / args.steps,
+           "GB/s": (by_e + by_s) / ((ms_e + ms_s) / 1e3) / 1e9 if ms_e + ms_s > 0 else None}
+    if est["GB/s"]:
+        est["frac_hbm"] = est["GB/s"] / pk["hbm"]
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Llama-2-7B-shaped inputs, random-init decaying-spectrum "
+                    "weights)",
+            "config": config_dict(world), "roofline": roof, "estimator": est,
+            "kernels": kernels, "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "impl": "ours"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        set_threads()
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,328 @@
+// C ABI entry points: argument validation, workspace planning and the launch
+// sequence of each call.  Every step of the hot path runs in this library's
+// kernels; the host only validates, carves the workspace and launches.
+#include <algorithm>
+#include <cmath>
+
+#include "estimator.cuh"
+#include "gemm_simt.cuh"
+#include "linear_ops.cuh"
+#include "swiglu.cuh"
+
+namespace slora {
+
+slora_status svd_prepare_impl(const void* W, int64_t n, int64_t k, int dt, int rank, int n_iter,
+                              uint64_t seed, float* L, float* U, void* W_t, Arena& ar,
+                              bool plan_only, cudaStream_t st);
+
+namespace {
+
+#define REQ_PTR(p)                                                                      \
+  do {                                                                                  \
+    if (!(p)) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: required pointer %s is NULL", fn, #p); \
+    if (!aligned16(p)) SLORA_FAIL(SLORA_ERR_ALIGN, "%s: %s is not 16-byte aligned", fn, #p); \
+  } while (0)
+
+#define OPT_PTR(p)                                                                      \
+  do {                                                                                  \
+    if ((p) && !aligned16(p)) SLORA_FAIL(SLORA_ERR_ALIGN, "%s: %s is not 16-byte aligned", fn, #p); \
+  } while (0)
+
+slora_status check_dtype(const char* fn, slora_dtype dt) {
+  if (dt != SLORA_F32 && dt != SLORA_BF16)
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: unknown dtype %d", fn, int(dt));
+  return SLORA_OK;
+}
+
+slora_status check_row(const char* fn, const char* what, int64_t len, int dt) {
+  const int64_t q = dt == kF32 ? 4 : 8;  // rows start on 16-byte boundaries
+  if (len <= 0) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: %s=%lld must be positive", fn, what, (long long)len);
+  if (len % q) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: %s=%lld must be a multiple of %lld", fn, what,
+                          (long long)len, (long long)q);
+  return SLORA_OK;
+}
+
+slora_status check_sparsity(const char* fn, float s) {
+  if (!(s >= 0.0f && s < 1.0f))
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: sparsity %g outside [0, 1)", fn, double(s));
+  return SLORA_OK;
+}
+
+// Channels kept at sparsity s: N - floor(s * N) (the skipped count rounds down).
+int64_t keep_count(int64_t N, float s) {
+  double skip = std::floor(double(s) * double(N) + 1e-9);
+  return N - int64_t(skip);
+}
+
+slora_status finish_ws(const char* fn, const Arena& ar, void* ws, size_t* ws_bytes) {
+  if (!ws_bytes) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: ws_bytes is NULL", fn);
+  if (!ws) {
+    *ws_bytes = ar.used;
+    return SLORA_OK;
+  }
+  if (*ws_bytes < ar.used)
+    SLORA_FAIL(SLORA_ERR_WORKSPACE, "%s: workspace of %zu bytes, %zu needed", fn, *ws_bytes,
+               ar.used);
+  return SLORA_OK;
+}
+
+}  // namespace
+}  // namespace slora
+
+using namespace slora;
+
+// --------------------------------------------------------------- prepare
+extern "C" slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, slora_dtype dt,
+                                          int rank, int n_iter, uint64_t seed, float* L,
+                                          float* U, void* W_t, void* ws, size_t* ws_bytes,
+                                          slora_stream_t stream) {
+  const char* fn = "slora_svd_prepare";
+  clear_error();
+  SLORA_TRY(check_dtype(fn, dt));
+  REQ_PTR(W); REQ_PTR(L); REQ_PTR(U); OPT_PTR(W_t); OPT_PTR(ws);
+  SLORA_TRY(check_row(fn, "k", k, dt));
+  SLORA_TRY(check_row(fn, "n", n, dt));
+  if (rank < 1 || rank > 48 || rank > std::min(n, k))
+    SLORA_FAIL(SLORA_ERR_SHAPE, "%s: rank %d outside [1, min(n, k, 48)]", fn, rank);
+  if (n_iter < 0 || n_iter > 100) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: n_iter %d", fn, n_iter);
+  Arena plan;
+  SLORA_TRY(svd_prepare_impl(W, n, k, dt, rank, n_iter, seed, L, U, W_t, plan, true, nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  return svd_prepare_impl(W, n, k, dt, rank, n_iter, seed, L, U, W_t, ar, false,
+                          static_cast<cudaStream_t>(stream));
+}
+
+// --------------------------------------------------------- estimate+select
+namespace slora {
+// Estimator body shared with the FFN call.  Writes idx (see slora.h layout).
+slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
+                                  const slora_tokens* tok, const TokenInfo& ti,
+                                  const int32_t* ctx_rows, int64_t d, const float* L0,
+                                  const float* U0, int64_t n0, const float* L1, const float* U1,
+                                  int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
+                                  int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
+                                  cudaStream_t st) {
+  (void)tok;
+  float* P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
+  const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
+  float* scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
+  const int nsplit = ffn_score_splits(ti.T_C, n0);
+  float* partial = nullptr;
+  double* gram = nullptr;
+  if (crit == SLORA_CRIT_FFN_SWIGLU_L2)
+    partial = ar.take<float>(size_t(nsplit) * n0);
+  else
+    gram = ar.take<double>(size_t(2) * rank * rank * 33);
+  if (plan) return SLORA_OK;
+  // P = X_C [L0 | L1]  (fp32 accumulate)
+  for (int p = 0; p < 2; ++p) {
+    GemmArgs g;
+    g.M = ti.T_C; g.N = rank; g.nseg = 1;
+    g.seg[0].a = rowmajor(X, dt, d, ctx_rows);
+    g.seg[0].b = colmajor(p == 0 ? L0 : L1, kF32, rank);
+    g.seg[0].K = d;
+    g.c = out_rowmajor(P + p * rank, kF32, 2 * rank);
+    SLORA_TRY(gemm_simt(g, st));
+  }
+  if (crit == SLORA_CRIT_FFN_SWIGLU_L2) {
+    SLORA_TRY(ffn_scores(P, 2 * rank, ti.T_C, U0, U1, n0, rank, partial, nsplit, scores, st));
+    SLORA_TRY(topk_select(scores, 1, int(n0), int(kkeep), 1, idx_out, nullptr, st));
+  } else {
+    SLORA_TRY(qk_scores(P, 2 * rank, ti.T_C, U0, U1, rank, heads, kv_heads, head_dim, gram,
+                        scores, st));
+    SLORA_TRY(topk_select(scores, kv_heads, head_dim, int(kkeep), heads / kv_heads, idx_out,
+                          idx_out + int64_t(heads) * kkeep, st));
+  }
+  return SLORA_OK;
+}
+}  // namespace slora
+
+extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dtype dt,
+                                              const slora_tokens* tok, int64_t d, const float* L0,
+                                              const float* U0, int64_t n0, const float* L1,
+                                              const float* U1, int64_t n1, int rank, int heads,
+                                              int kv_heads, int head_dim, float sparsity,
+                                              int32_t* idx_out, int32_t* k_out, float* scores_out,
+                                              void* ws, size_t* ws_bytes, slora_stream_t stream) {
+  const char* fn = "slora_estimate_select";
+  clear_error();
+  SLORA_TRY(check_dtype(fn, dt));
+  if (crit != SLORA_CRIT_FFN_SWIGLU_L2 && crit != SLORA_CRIT_QK_NORM)
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: unknown criterion %d", fn, int(crit));
+  REQ_PTR(X); REQ_PTR(L0); REQ_PTR(U0); REQ_PTR(L1); REQ_PTR(U1); REQ_PTR(idx_out);
+  OPT_PTR(scores_out); OPT_PTR(ws);
+  if (!k_out) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: k_out is NULL", fn);
+  SLORA_TRY(check_sparsity(fn, sparsity));
+  SLORA_TRY(check_row(fn, "d", d, dt));
+  if (rank < 1 || rank > 48) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: rank %d outside [1, 48]", fn, rank);
+  TokenInfo ti;
+  SLORA_TRY(parse_tokens(tok, &ti));
+  int64_t kkeep;
+  if (crit == SLORA_CRIT_FFN_SWIGLU_L2) {
+    if (n0 <= 0 || n0 != n1) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: FFN needs n0 == n1 > 0", fn);
+    if (n0 > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0 too large", fn);
+    kkeep = keep_count(n0, sparsity);
+  } else {
+    if (heads <= 0 || kv_heads <= 0 || head_dim <= 0 || heads % kv_heads)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: heads=%d kv_heads=%d head_dim=%d", fn, heads, kv_heads,
+                 head_dim);
+    if (n0 != int64_t(heads) * head_dim || n1 != int64_t(kv_heads) * head_dim)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0/n1 must be heads*head_dim / kv_heads*head_dim", fn);
+    kkeep = keep_count(head_dim, sparsity);
+  }
+  Arena plan;
+  plan.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  SLORA_TRY(estimate_select_body(crit, X, dt, tok, ti, nullptr, d, L0, U0, n0, L1, U1, rank,
+                                 heads, kv_heads, head_dim, kkeep, idx_out, scores_out, plan,
+                                 true, nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  *k_out = int32_t(kkeep);
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st));
+  return estimate_select_body(crit, X, dt, tok, ti, ctx_rows, d, L0, U0, n0, L1, U1, rank, heads,
+                              kv_heads, head_dim, kkeep, idx_out, scores_out, ar, false, st);
+}
+
+// ------------------------------------------------------------ linear calls
+namespace {
+slora_status linear_common_checks(const char* fn, slora_dtype dt, const slora_tokens* tok,
+                                  int64_t k, int64_t n, const void* W, const void* A,
+                                  const void* B, int r_lora, slora_slice side,
+                                  const int32_t* idx, int32_t n_idx, TokenInfo* ti) {
+  SLORA_TRY(check_dtype(fn, dt));
+  if (side != SLORA_SLICE_NONE && side != SLORA_SLICE_OUT_ROWS && side != SLORA_SLICE_IN_COLS)
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: unknown slice side %d", fn, int(side));
+  REQ_PTR(W); REQ_PTR(A); REQ_PTR(B);
+  SLORA_TRY(check_row(fn, "k", k, dt));
+  SLORA_TRY(check_row(fn, "n", n, dt));
+  if (r_lora < 1 || r_lora > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: r_lora %d outside [1, 64]", fn, r_lora);
+  SLORA_TRY(parse_tokens(tok, ti));
+  if (side != SLORA_SLICE_NONE) {
+    REQ_PTR(idx);
+    const int64_t lim = side == SLORA_SLICE_OUT_ROWS ? n : k;
+    if (n_idx < 0 || n_idx > lim)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n_idx=%d outside [0, %lld]", fn, n_idx, (long long)lim);
+  }
+  return SLORA_OK;
+}
+}  // namespace
+
+extern "C" slora_status slora_linear_fwd(slora_dtype dt, const slora_tokens* tok, int64_t k,
+                                         int64_t n, const void* W, const void* A, const void* B,
+                                         int r_lora, float lora_scale, slora_slice side,
+                                         const int32_t* idx, int32_t n_idx, const void* X_ctx,
+                                         const void* X_out, void* Y_ctx, void* Y_out,
+                                         float* XA_save, void* ws, size_t* ws_bytes,
+                                         slora_stream_t stream) {
+  const char* fn = "slora_linear_fwd";
+  clear_error();
+  TokenInfo ti;
+  SLORA_TRY(linear_common_checks(fn, dt, tok, k, n, W, A, B, r_lora, side, idx, n_idx, &ti));
+  REQ_PTR(X_ctx); REQ_PTR(Y_ctx); OPT_PTR(XA_save); OPT_PTR(ws);
+  if (side == SLORA_SLICE_OUT_ROWS && ti.T_O > 0) REQ_PTR(Y_out);
+  if (side == SLORA_SLICE_IN_COLS && ti.T_O > 0) REQ_PTR(X_out);
+  LinearDesc L{int(dt), ti, k, n, W, A, B, r_lora, lora_scale, side, idx, n_idx};
+  Arena plan;
+  SLORA_TRY(linear_fwd_run(L, nullptr, X_ctx, X_out, Y_ctx, Y_out, XA_save, plan, true, nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  return linear_fwd_run(L, tok, X_ctx, X_out, Y_ctx, Y_out, XA_save, ar, false,
+                        static_cast<cudaStream_t>(stream));
+}
+
+extern "C" slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok, int64_t k,
+                                         int64_t n, const void* W, const void* A, const void* B,
+                                         int r_lora, float lora_scale, slora_slice side,
+                                         const int32_t* idx, int32_t n_idx, const void* X_ctx,
+                                         const void* X_out, const float* XA_save,
+                                         const void* dY_ctx, const void* dY_out, void* dX_ctx,
+                                         void* dX_out, float* dA, float* dB, void* ws,
+                                         size_t* ws_bytes, slora_stream_t stream) {
+  const char* fn = "slora_linear_bwd";
+  clear_error();
+  TokenInfo ti;
+  SLORA_TRY(linear_common_checks(fn, dt, tok, k, n, W, A, B, r_lora, side, idx, n_idx, &ti));
+  REQ_PTR(X_ctx); REQ_PTR(XA_save); REQ_PTR(dY_ctx); REQ_PTR(dX_ctx); REQ_PTR(dA); REQ_PTR(dB);
+  OPT_PTR(ws);
+  if (side == SLORA_SLICE_OUT_ROWS && ti.T_O > 0) REQ_PTR(dY_out);
+  if (side == SLORA_SLICE_IN_COLS && ti.T_O > 0) { REQ_PTR(X_out); REQ_PTR(dX_out); }
+  LinearDesc L{int(dt), ti, k, n, W, A, B, r_lora, lora_scale, side, idx, n_idx};
+  Arena plan;
+  SLORA_TRY(linear_bwd_run(L, nullptr, X_ctx, X_out, XA_save, dY_ctx, dY_out, dX_ctx, dX_out, dA,
+                           dB, plan, true, nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  return linear_bwd_run(L, tok, X_ctx, X_out, XA_save, dY_ctx, dY_out, dX_ctx, dX_out, dA, dB, ar,
+                        false, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------- FFN
+extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
+                                          const slora_tokens* tok, float sparsity, const void* X,
+                                          const void* dOut, void* out, void* dX,
+                                          const slora_ffn_grads* grads, int32_t* idx_out,
+                                          int32_t* k_out, const int32_t* idx_force,
+                                          int32_t k_force, void* ws, size_t* ws_bytes,
+                                          slora_stream_t stream) {
+  const char* fn = "slora_ffn_fwd_bwd";
+  clear_error();
+  SLORA_TRY(check_dtype(fn, dt));
+  if (!layer || !grads) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: layer or grads is NULL", fn);
+  const slora_ffn_layer& Ly = *layer;
+  const slora_ffn_grads& Gr = *grads;
+  REQ_PTR(Ly.Wg); REQ_PTR(Ly.Wu); REQ_PTR(Ly.Wd_t);
+  REQ_PTR(Ly.Ag); REQ_PTR(Ly.Bg); REQ_PTR(Ly.Au); REQ_PTR(Ly.Bu); REQ_PTR(Ly.Ad); REQ_PTR(Ly.Bd);
+  REQ_PTR(X); REQ_PTR(dOut); REQ_PTR(out); REQ_PTR(dX); REQ_PTR(idx_out);
+  REQ_PTR(Gr.dAg); REQ_PTR(Gr.dBg); REQ_PTR(Gr.dAu); REQ_PTR(Gr.dBu); REQ_PTR(Gr.dAd);
+  REQ_PTR(Gr.dBd); OPT_PTR(ws); OPT_PTR(idx_force);
+  if (!k_out) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: k_out is NULL", fn);
+  SLORA_TRY(check_row(fn, "d", Ly.d, dt));
+  SLORA_TRY(check_row(fn, "d_ff", Ly.d_ff, dt));
+  if (Ly.r_lora < 1 || Ly.r_lora > 32)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "%s: r_lora %d outside [1, 32]", fn, Ly.r_lora);
+  int64_t kkeep;
+  if (idx_force) {
+    if (k_force < 0 || k_force > Ly.d_ff)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: k_force=%d outside [0, d_ff]", fn, k_force);
+    kkeep = k_force;
+  } else {
+    SLORA_TRY(check_sparsity(fn, sparsity));
+    REQ_PTR(Ly.Lg); REQ_PTR(Ly.Ug); REQ_PTR(Ly.Lu); REQ_PTR(Ly.Uu);
+    if (Ly.r_svd < 1 || Ly.r_svd > 48)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: r_svd %d outside [1, 48]", fn, Ly.r_svd);
+    kkeep = keep_count(Ly.d_ff, sparsity);
+  }
+  TokenInfo ti;
+  SLORA_TRY(parse_tokens(tok, &ti));
+  FfnDesc F{int(dt), ti, Ly, Gr, kkeep};
+  Arena plan;
+  SLORA_TRY(ffn_run(F, nullptr, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  *k_out = int32_t(kkeep);
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  return ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, ar, false,
+                 static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,116 @@
+// Shared internals of libslora: status reporting, workspace carving, element
+// access helpers.  Nothing here is part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "../../include/slora.h"
+
+namespace slora {
+
+enum DT : int { kF32 = 0, kBF16 = 1 };
+
+inline int dt_size(int dt) { return dt == kF32 ? 4 : 2; }
+
+// ---------------------------------------------------------------- errors
+void set_error(const char* fmt, ...);
+void clear_error();
+
+#define SLORA_FAIL(code, ...)      \
+  do {                             \
+    ::slora::set_error(__VA_ARGS__); \
+    return (code);                 \
+  } while (0)
+
+#define SLORA_CUDA(call)                                                              \
+  do {                                                                                \
+    cudaError_t e_ = (call);                                                          \
+    if (e_ != cudaSuccess)                                                            \
+      SLORA_FAIL(SLORA_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), \
+                 __FILE__, __LINE__);                                                 \
+  } while (0)
+
+#define SLORA_CHECK_LAUNCH()                                                          \
+  do {                                                                                \
+    cudaError_t e_ = cudaGetLastError();                                              \
+    if (e_ != cudaSuccess)                                                            \
+      SLORA_FAIL(SLORA_ERR_CUDA, "kernel launch failed: %s (%s:%d)",                  \
+                 cudaGetErrorString(e_), __FILE__, __LINE__);                         \
+  } while (0)
+
+#define SLORA_TRY(expr)                 \
+  do {                                  \
+    slora_status s_ = (expr);           \
+    if (s_ != SLORA_OK) return s_;      \
+  } while (0)
+
+// ------------------------------------------------------------- workspace
+// Bump allocator over the caller's workspace.  With base == nullptr it only
+// counts bytes (the workspace-size query).
+struct Arena {
+  char* base = nullptr;
+  size_t used = 0;
+  template <class T>
+  T* take(size_t count) {
+    size_t off = (used + 255) & ~size_t(255);
+    used = off + count * sizeof(T);
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+// ------------------------------------------------------------- devices
+slora_status check_device();  // sm_100 present and current
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------- tokens
+// Row maps of the context / output tokens of one call, built on the device.
+constexpr int kMaxBatch = 4096;
+struct TokenInfo {
+  int batch = 0, seq = 0;
+  int64_t T = 0, T_C = 0, T_O = 0;
+};
+slora_status parse_tokens(const slora_tokens* tok, TokenInfo* info);
+// Writes ctx_rows[T_C] and out_rows[T_O] (int32 row indices into the full layout).
+slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
+                            int32_t* out_rows, cudaStream_t st);
+
+// ------------------------------------------------------------- launches
+// Kernel classes for launch accounting (names in slora_profile_read).
+enum KClass : int { kGemmTC = 0, kGemmSimt, kEstimate, kSelect, kElementwise, kAux, kPrepare,
+                    kNumClasses };
+// Construct immediately before a kernel launch: counts it and, while
+// profiling is on, records CUDA events around it on `st`.
+struct LaunchScope {
+  LaunchScope(int cls, double work, cudaStream_t st);
+  ~LaunchScope();
+  int cls_;
+  cudaStream_t st_;
+  int slot_;
+};
+
+// ------------------------------------------------------------- elements
+__device__ __forceinline__ float ld_elem(const void* p, int64_t i, int dt) {
+  if (dt == kF32) return static_cast<const float*>(p)[i];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+__device__ __forceinline__ void st_elem(void* p, int64_t i, int dt, float v) {
+  if (dt == kF32)
+    static_cast<float*>(p)[i] = v;
+  else
+    static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+}
+
+// silu(x) = x * sigmoid(x) in fp32.  __expf is the fast exp2-based intrinsic
+// (relative error a few ulp); for x << 0 exp(-x) overflows to +inf and the
+// reciprocal gives 0, so silu -> 0 as it should.
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
+}  // namespace slora

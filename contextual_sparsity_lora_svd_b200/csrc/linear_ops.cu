@@ -1,0 +1,322 @@
+// Sliced LoRA linear and SwiGLU FFN: the sequence of gathered GEMMs.
+//
+// SparseLoRA article, section 1: only the selected channels are computed;
+// section 3: context tokens take the sparse path, output tokens stay dense;
+// sections 6-7: the sparsity is structured (whole channel slices) so the
+// GPU sees smaller dense GEMMs.  Forum post with the paper's abstract: the
+// loss and the gradients are computed on the selected weight subsets.
+//
+// Notation: W0 [n x k], A [r x k], B [n x r], s = lora_scale, C / O = context
+// and output rows, S = selected channel set (idx).
+#include <algorithm>
+
+#include "estimator.cuh"
+#include "gemm.cuh"
+#include "linear_ops.cuh"
+#include "swiglu.cuh"
+
+namespace slora {
+namespace {
+
+GemmArgs mk(int64_t M, int64_t N, OutRef c) {
+  GemmArgs g;
+  g.M = M; g.N = N; g.c = c; g.nseg = 0;
+  return g;
+}
+void add(GemmArgs& g, MatRef a, MatRef b, int64_t K, float alpha = 1.0f) {
+  Seg& s = g.seg[g.nseg++];
+  s.a = a; s.b = b; s.K = K; s.alpha = alpha;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ forward
+slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                            const void* X_out, void* Y_ctx, void* Y_out, float* XA_save,
+                            Arena& ar, bool plan, cudaStream_t st) {
+  const TokenInfo& ti = L.ti;
+  const int dt = L.dt, r = L.r;
+  const int64_t k = L.k, n = L.n, ni = L.n_idx;
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_O, 1)));
+  float* XA = XA_save ? XA_save : ar.take<float>(size_t(ti.T) * r);
+  if (plan) return SLORA_OK;
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
+
+  if (L.side == SLORA_SLICE_NONE) {
+    GemmArgs g = mk(ti.T, r, out_rowmajor(XA, kF32, r));  // XA = X A^T
+    add(g, rowmajor(X_ctx, dt, k), rowmajor(L.A, dt, k), k);
+    SLORA_TRY(gemm(g, st));
+    GemmArgs y = mk(ti.T, n, out_rowmajor(Y_ctx, dt, n));  // Y = X W0^T + s XA B^T
+    add(y, rowmajor(X_ctx, dt, k), rowmajor(L.W, dt, k), k);
+    add(y, rowmajor(XA, kF32, r), rowmajor(L.B, dt, r), r, L.s);
+    return gemm(y, st);
+  }
+  if (L.side == SLORA_SLICE_OUT_ROWS) {
+    GemmArgs g = mk(ti.T, r, out_rowmajor(XA, kF32, r));
+    add(g, rowmajor(X_ctx, dt, k), rowmajor(L.A, dt, k), k);
+    SLORA_TRY(gemm(g, st));
+    // context rows, output channels S
+    GemmArgs yc = mk(ti.T_C, ni, out_rowmajor(Y_ctx, dt, ni));
+    add(yc, rowmajor(X_ctx, dt, k, ctx_rows), rowmajor(L.W, dt, k, L.idx), k);
+    add(yc, rowmajor(XA, kF32, r, ctx_rows), rowmajor(L.B, dt, r, L.idx), r, L.s);
+    SLORA_TRY(gemm(yc, st));
+    // output rows, dense
+    GemmArgs yo = mk(ti.T_O, n, out_rowmajor(Y_out, dt, n));
+    add(yo, rowmajor(X_ctx, dt, k, out_rows), rowmajor(L.W, dt, k), k);
+    add(yo, rowmajor(XA, kF32, r, out_rows), rowmajor(L.B, dt, r), r, L.s);
+    return gemm(yo, st);
+  }
+  // IN_COLS: W is W0^T [k x n]; context rows read input channels S only.
+  {
+    GemmArgs gc = mk(ti.T_C, r, out_rowmajor(XA, kF32, r, ctx_rows));  // X_ctx A[:,S]^T
+    add(gc, rowmajor(X_ctx, dt, ni), rowmajor(L.A, dt, k, nullptr, L.idx), ni);
+    SLORA_TRY(gemm(gc, st));
+    GemmArgs go = mk(ti.T_O, r, out_rowmajor(XA, kF32, r, out_rows));  // X_out A^T
+    add(go, rowmajor(X_out, dt, k), rowmajor(L.A, dt, k), k);
+    SLORA_TRY(gemm(go, st));
+    GemmArgs yc = mk(ti.T_C, n, out_rowmajor(Y_ctx, dt, n, ctx_rows));
+    add(yc, rowmajor(X_ctx, dt, ni), colmajor(L.W, dt, n, nullptr, L.idx), ni);
+    add(yc, rowmajor(XA, kF32, r, ctx_rows), rowmajor(L.B, dt, r), r, L.s);
+    SLORA_TRY(gemm(yc, st));
+    GemmArgs yo = mk(ti.T_O, n, out_rowmajor(Y_ctx, dt, n, out_rows));
+    add(yo, rowmajor(X_out, dt, k), colmajor(L.W, dt, n), k);
+    add(yo, rowmajor(XA, kF32, r, out_rows), rowmajor(L.B, dt, r), r, L.s);
+    return gemm(yo, st);
+  }
+}
+
+// ----------------------------------------------------------------- backward
+slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                            const void* X_out, const float* XA, const void* dY_ctx,
+                            const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
+                            Arena& ar, bool plan, cudaStream_t st) {
+  const TokenInfo& ti = L.ti;
+  const int dt = L.dt, r = L.r;
+  const int64_t k = L.k, n = L.n, ni = L.n_idx;
+  const float s = L.s;
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_O, 1)));
+  float* dYB = ar.take<float>(size_t(ti.T) * r);  // dY B per row, full row layout
+  if (plan) return SLORA_OK;
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
+
+  if (L.side == SLORA_SLICE_NONE) {
+    GemmArgs g = mk(ti.T, r, out_rowmajor(dYB, kF32, r));
+    add(g, rowmajor(dY_ctx, dt, n), colmajor(L.B, dt, r), n);
+    SLORA_TRY(gemm(g, st));
+    GemmArgs x = mk(ti.T, k, out_rowmajor(dX_ctx, dt, k));  // dX = dY W0 + s dYB A
+    add(x, rowmajor(dY_ctx, dt, n), colmajor(L.W, dt, k), n);
+    add(x, rowmajor(dYB, kF32, r), colmajor(L.A, dt, k), r, s);
+    SLORA_TRY(gemm(x, st));
+    GemmArgs a = mk(r, k, out_rowmajor(dA, kF32, k));  // dA = s dYB^T X
+    add(a, colmajor(dYB, kF32, r), colmajor(X_ctx, dt, k), ti.T, s);
+    SLORA_TRY(gemm(a, st));
+    GemmArgs b = mk(n, r, out_rowmajor(dB, kF32, r));  // dB = s dY^T XA
+    add(b, colmajor(dY_ctx, dt, n), colmajor(XA, kF32, r), ti.T, s);
+    return gemm(b, st);
+  }
+  if (L.side == SLORA_SLICE_OUT_ROWS) {
+    GemmArgs bc = mk(ti.T_C, r, out_rowmajor(dYB, kF32, r, ctx_rows));  // dY_C B[S]
+    add(bc, rowmajor(dY_ctx, dt, ni), colmajor(L.B, dt, r, nullptr, L.idx), ni);
+    SLORA_TRY(gemm(bc, st));
+    GemmArgs bo = mk(ti.T_O, r, out_rowmajor(dYB, kF32, r, out_rows));  // dY_O B
+    add(bo, rowmajor(dY_out, dt, n), colmajor(L.B, dt, r), n);
+    SLORA_TRY(gemm(bo, st));
+    GemmArgs xc = mk(ti.T_C, k, out_rowmajor(dX_ctx, dt, k, ctx_rows));
+    add(xc, rowmajor(dY_ctx, dt, ni), colmajor(L.W, dt, k, nullptr, L.idx), ni);
+    add(xc, rowmajor(dYB, kF32, r, ctx_rows), colmajor(L.A, dt, k), r, s);
+    SLORA_TRY(gemm(xc, st));
+    GemmArgs xo = mk(ti.T_O, k, out_rowmajor(dX_ctx, dt, k, out_rows));
+    add(xo, rowmajor(dY_out, dt, n), colmajor(L.W, dt, k), n);
+    add(xo, rowmajor(dYB, kF32, r, out_rows), colmajor(L.A, dt, k), r, s);
+    SLORA_TRY(gemm(xo, st));
+    GemmArgs a = mk(r, k, out_rowmajor(dA, kF32, k));  // all rows
+    add(a, colmajor(dYB, kF32, r), colmajor(X_ctx, dt, k), ti.T, s);
+    SLORA_TRY(gemm(a, st));
+    GemmArgs b0 = mk(n, r, out_rowmajor(dB, kF32, r));  // output rows, every channel
+    add(b0, colmajor(dY_out, dt, n), colmajor(XA, kF32, r, nullptr, out_rows), ti.T_O, s);
+    SLORA_TRY(gemm(b0, st));
+    GemmArgs b1 = mk(ni, r, out_rowmajor(dB, kF32, r, L.idx, nullptr, 1));  // += ctx, rows S
+    add(b1, colmajor(dY_ctx, dt, ni), colmajor(XA, kF32, r, nullptr, ctx_rows), ti.T_C, s);
+    return gemm(b1, st);
+  }
+  // IN_COLS
+  {
+    GemmArgs g = mk(ti.T, r, out_rowmajor(dYB, kF32, r));  // dY B, every row
+    add(g, rowmajor(dY_ctx, dt, n), colmajor(L.B, dt, r), n);
+    SLORA_TRY(gemm(g, st));
+    GemmArgs xc = mk(ti.T_C, ni, out_rowmajor(dX_ctx, dt, ni));  // dY_C W0[:,S] + s dYB_C A[:,S]
+    add(xc, rowmajor(dY_ctx, dt, n, ctx_rows), rowmajor(L.W, dt, n, L.idx), n);
+    add(xc, rowmajor(dYB, kF32, r, ctx_rows), colmajor(L.A, dt, k, L.idx), r, s);
+    SLORA_TRY(gemm(xc, st));
+    GemmArgs xo = mk(ti.T_O, k, out_rowmajor(dX_out, dt, k));
+    add(xo, rowmajor(dY_ctx, dt, n, out_rows), rowmajor(L.W, dt, n), n);
+    add(xo, rowmajor(dYB, kF32, r, out_rows), colmajor(L.A, dt, k), r, s);
+    SLORA_TRY(gemm(xo, st));
+    GemmArgs a0 = mk(r, k, out_rowmajor(dA, kF32, k));  // output rows, every column
+    add(a0, colmajor(dYB, kF32, r, nullptr, out_rows), colmajor(X_out, dt, k), ti.T_O, s);
+    SLORA_TRY(gemm(a0, st));
+    GemmArgs a1 = mk(r, ni, out_rowmajor(dA, kF32, k, nullptr, L.idx, 1));  // += ctx, cols S
+    add(a1, colmajor(dYB, kF32, r, nullptr, ctx_rows), colmajor(X_ctx, dt, ni), ti.T_C, s);
+    SLORA_TRY(gemm(a1, st));
+    GemmArgs b = mk(n, r, out_rowmajor(dB, kF32, r));  // dB = s dY^T XA, every row
+    add(b, colmajor(dY_ctx, dt, n), colmajor(XA, kF32, r), ti.T, s);
+    return gemm(b, st);
+  }
+}
+
+// ---------------------------------------------------------------------- FFN
+slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
+                     void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
+                     bool plan, cudaStream_t st) {
+  const TokenInfo& ti = F.ti;
+  const slora_ffn_layer& L = F.L;
+  const slora_ffn_grads& G = F.G;
+  const int dt = F.dt, r = L.r_lora;
+  const int64_t d = L.d, Fd = L.d_ff, kk = F.kkeep, TC = ti.T_C, TO = ti.T_O, T = ti.T;
+  const float s = L.lora_scale;
+  const int es = dt_size(dt);
+  auto buf = [&](int64_t rows, int64_t cols) {
+    return static_cast<void*>(ar.take<char>(size_t(std::max<int64_t>(rows * cols, 1)) * es));
+  };
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TC, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TO, 1)));
+  float* XA = ar.take<float>(size_t(T) * 2 * r);   // [X Ag^T | X Au^T]
+  float* hA = ar.take<float>(size_t(T) * r);       // h Ad^T (on the channels used)
+  float* dOB = ar.take<float>(size_t(T) * r);      // dOut Bd
+  float* dGB = ar.take<float>(size_t(T) * 2 * r);  // [dG Bg | dU Bu] (on the channels used)
+  void* gC = buf(TC, kk);
+  void* uC = buf(TC, kk);
+  void* hC = buf(TC, kk);
+  void* dGC = buf(TC, kk);
+  void* dUC = buf(TC, kk);
+  void* gO = buf(TO, Fd);
+  void* uO = buf(TO, Fd);
+  void* hO = buf(TO, Fd);
+  void* dGO = buf(TO, Fd);
+  void* dUO = buf(TO, Fd);
+  if (!idx_force)
+    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
+                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
+                                   true, nullptr));
+  if (plan) return SLORA_OK;
+
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
+  if (idx_force) {
+    if (kk > 0)
+      SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
+                                 cudaMemcpyDeviceToDevice, st));
+  } else {
+    // same arena offsets as the plan: the estimator's scratch follows the buffers above
+    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
+                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
+                                   false, st));
+  }
+
+  // ---- forward
+  for (int p = 0; p < 2; ++p) {  // XA = X [Ag; Au]^T, every row
+    GemmArgs g = mk(T, r, out_rowmajor(XA + p * r, kF32, 2 * r));
+    add(g, rowmajor(X, dt, d), rowmajor(p ? L.Au : L.Ag, dt, d), d);
+    SLORA_TRY(gemm(g, st));
+  }
+  for (int p = 0; p < 2; ++p) {  // gate / up on context rows, channels S
+    const void* W = p ? L.Wu : L.Wg;
+    const void* Bm = p ? L.Bu : L.Bg;
+    GemmArgs gc = mk(TC, kk, out_rowmajor(p ? uC : gC, dt, kk));
+    add(gc, rowmajor(X, dt, d, ctx_rows), rowmajor(W, dt, d, idx), d);
+    add(gc, rowmajor(XA + p * r, kF32, 2 * r, ctx_rows), rowmajor(Bm, dt, r, idx), r, s);
+    SLORA_TRY(gemm(gc, st));
+    GemmArgs go = mk(TO, Fd, out_rowmajor(p ? uO : gO, dt, Fd));  // output rows, dense
+    add(go, rowmajor(X, dt, d, out_rows), rowmajor(W, dt, d), d);
+    add(go, rowmajor(XA + p * r, kF32, 2 * r, out_rows), rowmajor(Bm, dt, r), r, s);
+    SLORA_TRY(gemm(go, st));
+  }
+  SLORA_TRY(swiglu_fwd(gC, uC, hC, TC * kk, dt, st));
+  SLORA_TRY(swiglu_fwd(gO, uO, hO, TO * Fd, dt, st));
+  {
+    GemmArgs ac = mk(TC, r, out_rowmajor(hA, kF32, r, ctx_rows));  // h_S Ad[:,S]^T
+    add(ac, rowmajor(hC, dt, kk), rowmajor(L.Ad, dt, Fd, nullptr, idx), kk);
+    SLORA_TRY(gemm(ac, st));
+    GemmArgs ao = mk(TO, r, out_rowmajor(hA, kF32, r, out_rows));
+    add(ao, rowmajor(hO, dt, Fd), rowmajor(L.Ad, dt, Fd), Fd);
+    SLORA_TRY(gemm(ao, st));
+    // down projection: context rows read channels S only (rows S of Wd^T)
+    GemmArgs oc = mk(TC, d, out_rowmajor(out, dt, d, ctx_rows));
+    add(oc, rowmajor(hC, dt, kk), colmajor(L.Wd_t, dt, d, nullptr, idx), kk);
+    add(oc, rowmajor(hA, kF32, r, ctx_rows), rowmajor(L.Bd, dt, r), r, s);
+    SLORA_TRY(gemm(oc, st));
+    GemmArgs oo = mk(TO, d, out_rowmajor(out, dt, d, out_rows));
+    add(oo, rowmajor(hO, dt, Fd), colmajor(L.Wd_t, dt, d), Fd);
+    add(oo, rowmajor(hA, kF32, r, out_rows), rowmajor(L.Bd, dt, r), r, s);
+    SLORA_TRY(gemm(oo, st));
+  }
+
+  // ---- backward
+  {
+    GemmArgs g = mk(T, r, out_rowmajor(dOB, kF32, r));  // dOut Bd
+    add(g, rowmajor(dOut, dt, d), colmajor(L.Bd, dt, r), d);
+    SLORA_TRY(gemm(g, st));
+    // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]   (into dGC, then SwiGLU bwd in place)
+    GemmArgs hc = mk(TC, kk, out_rowmajor(dGC, dt, kk));
+    add(hc, rowmajor(dOut, dt, d, ctx_rows), rowmajor(L.Wd_t, dt, d, idx), d);
+    add(hc, rowmajor(dOB, kF32, r, ctx_rows), colmajor(L.Ad, dt, Fd, idx), r, s);
+    SLORA_TRY(gemm(hc, st));
+    GemmArgs ho = mk(TO, Fd, out_rowmajor(dGO, dt, Fd));
+    add(ho, rowmajor(dOut, dt, d, out_rows), rowmajor(L.Wd_t, dt, d), d);
+    add(ho, rowmajor(dOB, kF32, r, out_rows), colmajor(L.Ad, dt, Fd), r, s);
+    SLORA_TRY(gemm(ho, st));
+    // LoRA grads of the down projection
+    GemmArgs a0 = mk(r, Fd, out_rowmajor(G.dAd, kF32, Fd));
+    add(a0, colmajor(dOB, kF32, r, nullptr, out_rows), colmajor(hO, dt, Fd), TO, s);
+    SLORA_TRY(gemm(a0, st));
+    GemmArgs a1 = mk(r, kk, out_rowmajor(G.dAd, kF32, Fd, nullptr, idx, 1));
+    add(a1, colmajor(dOB, kF32, r, nullptr, ctx_rows), colmajor(hC, dt, kk), TC, s);
+    SLORA_TRY(gemm(a1, st));
+    GemmArgs b = mk(d, r, out_rowmajor(G.dBd, kF32, r));
+    add(b, colmajor(dOut, dt, d), colmajor(hA, kF32, r), T, s);
+    SLORA_TRY(gemm(b, st));
+  }
+  SLORA_TRY(swiglu_bwd(dGC, gC, uC, dGC, dUC, TC * kk, dt, st));
+  SLORA_TRY(swiglu_bwd(dGO, gO, uO, dGO, dUO, TO * Fd, dt, st));
+  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]
+    const void* Bm = p ? L.Bu : L.Bg;
+    GemmArgs bc = mk(TC, r, out_rowmajor(dGB + p * r, kF32, 2 * r, ctx_rows));
+    add(bc, rowmajor(p ? dUC : dGC, dt, kk), colmajor(Bm, dt, r, nullptr, idx), kk);
+    SLORA_TRY(gemm(bc, st));
+    GemmArgs bo = mk(TO, r, out_rowmajor(dGB + p * r, kF32, 2 * r, out_rows));
+    add(bo, rowmajor(p ? dUO : dGO, dt, Fd), colmajor(Bm, dt, r), Fd);
+    SLORA_TRY(gemm(bo, st));
+  }
+  {
+    GemmArgs xc = mk(TC, d, out_rowmajor(dX, dt, d, ctx_rows));
+    add(xc, rowmajor(dGC, dt, kk), colmajor(L.Wg, dt, d, nullptr, idx), kk);
+    add(xc, rowmajor(dUC, dt, kk), colmajor(L.Wu, dt, d, nullptr, idx), kk);
+    add(xc, rowmajor(dGB, kF32, 2 * r, ctx_rows), colmajor(L.Ag, dt, d), r, s);
+    add(xc, rowmajor(dGB + r, kF32, 2 * r, ctx_rows), colmajor(L.Au, dt, d), r, s);
+    SLORA_TRY(gemm(xc, st));
+    GemmArgs xo = mk(TO, d, out_rowmajor(dX, dt, d, out_rows));
+    add(xo, rowmajor(dGO, dt, Fd), colmajor(L.Wg, dt, d), Fd);
+    add(xo, rowmajor(dUO, dt, Fd), colmajor(L.Wu, dt, d), Fd);
+    add(xo, rowmajor(dGB, kF32, 2 * r, out_rows), colmajor(L.Ag, dt, d), r, s);
+    add(xo, rowmajor(dGB + r, kF32, 2 * r, out_rows), colmajor(L.Au, dt, d), r, s);
+    SLORA_TRY(gemm(xo, st));
+  }
+  for (int p = 0; p < 2; ++p) {
+    GemmArgs a = mk(r, d, out_rowmajor(p ? G.dAu : G.dAg, kF32, d));  // s dGB^T X, every row
+    add(a, colmajor(dGB + p * r, kF32, 2 * r), colmajor(X, dt, d), T, s);
+    SLORA_TRY(gemm(a, st));
+    float* dBm = p ? G.dBu : G.dBg;
+    GemmArgs b0 = mk(Fd, r, out_rowmajor(dBm, kF32, r));  // output rows, every channel
+    add(b0, colmajor(p ? dUO : dGO, dt, Fd), colmajor(XA + p * r, kF32, 2 * r, nullptr, out_rows),
+        TO, s);
+    SLORA_TRY(gemm(b0, st));
+    GemmArgs b1 = mk(kk, r, out_rowmajor(dBm, kF32, r, idx, nullptr, 1));  // += ctx, rows S
+    add(b1, colmajor(p ? dUC : dGC, dt, kk), colmajor(XA + p * r, kF32, 2 * r, nullptr, ctx_rows),
+        TC, s);
+    SLORA_TRY(gemm(b1, st));
+  }
+  return SLORA_OK;
+}
+
+}  // namespace slora

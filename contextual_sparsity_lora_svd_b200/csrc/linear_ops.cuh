@@ -1,0 +1,52 @@
+// Launch sequences of the sliced LoRA linear and the SwiGLU FFN layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace slora {
+
+struct LinearDesc {
+  int dt;
+  TokenInfo ti;
+  int64_t k, n;
+  const void* W;  // [n x k] (NONE, OUT_ROWS) or [k x n] (IN_COLS)
+  const void* A;  // [r x k]
+  const void* B;  // [n x r]
+  int r;
+  float s;
+  slora_slice side;
+  const int32_t* idx;
+  int32_t n_idx;
+};
+
+// With plan == true only the arena is sized (no pointer is touched).
+slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                            const void* X_out, void* Y_ctx, void* Y_out, float* XA_save,
+                            Arena& ar, bool plan, cudaStream_t st);
+slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                            const void* X_out, const float* XA, const void* dY_ctx,
+                            const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
+                            Arena& ar, bool plan, cudaStream_t st);
+
+struct FfnDesc {
+  int dt;
+  TokenInfo ti;
+  slora_ffn_layer L;
+  slora_ffn_grads G;
+  int64_t kkeep;
+};
+
+slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
+                     void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
+                     bool plan, cudaStream_t st);
+
+// Estimator body (estimate + select) shared by slora_estimate_select and the FFN call.
+slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
+                                  const slora_tokens* tok, const TokenInfo& ti,
+                                  const int32_t* ctx_rows, int64_t d, const float* L0,
+                                  const float* U0, int64_t n0, const float* L1, const float* U1,
+                                  int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
+                                  int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
+                                  cudaStream_t st);
+
+}  // namespace slora

@@ -1,0 +1,205 @@
+// Error text, device checks and token row maps.
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace slora {
+
+namespace {
+thread_local std::string g_error;
+
+struct RowmapParams {
+  int batch, seq;
+  int ctx_len[kMaxBatch];
+};
+
+// One block: scan ctx_len into per-sequence offsets, then every row t of the
+// full layout lands in ctx_rows or out_rows at its compact position.
+__global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
+                                                      int32_t* __restrict__ ctx_rows,
+                                                      int32_t* __restrict__ out_rows) {
+  __shared__ int ctx_off[kMaxBatch];
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = 0; b < p.batch; ++b) {
+      ctx_off[b] = acc;
+      acc += p.ctx_len[b];
+    }
+  }
+  __syncthreads();
+  const int64_t T = int64_t(p.batch) * p.seq;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+    const int b = int(t / p.seq), i = int(t % p.seq);
+    const int c = p.ctx_len[b];
+    if (i < c) {
+      if (ctx_rows) ctx_rows[ctx_off[b] + i] = int32_t(t);
+    } else {
+      // output rows before sequence b: b*seq - ctx_off[b]
+      if (out_rows) out_rows[int64_t(b) * p.seq - ctx_off[b] + (i - c)] = int32_t(t);
+    }
+  }
+}
+}  // namespace
+
+void set_error(const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_error = buf;
+}
+
+void clear_error() { g_error.clear(); }
+
+slora_status check_device() {
+  int dev = -1;
+  SLORA_CUDA(cudaGetDevice(&dev));
+  int major = 0, minor = 0;
+  SLORA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  SLORA_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+  if (major != 10 || minor != 0)
+    SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+               dev, major, minor);
+  return SLORA_OK;
+}
+
+slora_status parse_tokens(const slora_tokens* tok, TokenInfo* ti) {
+  if (!tok || !tok->ctx_len) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tokens or tokens->ctx_len is NULL");
+  if (tok->batch <= 0 || tok->seq <= 0)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "batch=%d seq=%d must be positive", tok->batch, tok->seq);
+  if (tok->batch > kMaxBatch)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "batch=%d exceeds the supported maximum %d", tok->batch, kMaxBatch);
+  int64_t T = int64_t(tok->batch) * tok->seq;
+  if (T > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "T=%lld rows too large", (long long)T);
+  int64_t tc = 0;
+  for (int b = 0; b < tok->batch; ++b) {
+    int c = tok->ctx_len[b];
+    if (c < 0 || c > tok->seq)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "ctx_len[%d]=%d outside [0, seq=%d]", b, c, tok->seq);
+    tc += c;
+  }
+  ti->batch = tok->batch;
+  ti->seq = tok->seq;
+  ti->T = T;
+  ti->T_C = tc;
+  ti->T_O = T - tc;
+  return SLORA_OK;
+}
+
+slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
+                            int32_t* out_rows, cudaStream_t st) {
+  RowmapParams p;
+  p.batch = ti.batch;
+  p.seq = ti.seq;
+  for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
+  LaunchScope ls(kAux, double(ti.T) * 4, st);
+  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+}  // namespace slora
+
+extern "C" const char* slora_last_error_string(void) { return slora::g_error.c_str(); }
+
+extern "C" int slora_version(void) { return 100; }
+
+// ------------------------------------------------------------ launch record
+namespace slora {
+namespace {
+const char* kClassNames[kNumClasses] = {"gemm_tc", "gemm_simt", "estimate", "select",
+                                        "elementwise", "aux", "prepare"};
+struct Rec {
+  int cls;
+  double work;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  std::mutex mu;
+  int64_t launches = 0;
+  bool on = false;
+  std::vector<Rec> recs;        // events of the current record
+  std::vector<cudaEvent_t> pool;  // free events
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+  void release_all() {
+    for (auto& r : recs) {
+      if (r.a) pool.push_back(r.a);
+      if (r.b) pool.push_back(r.b);
+    }
+    recs.clear();
+  }
+};
+Profiler& prof() {
+  static Profiler* p = new Profiler();
+  return *p;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(int cls, double work, cudaStream_t st) : cls_(cls), st_(st), slot_(-1) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  ++p.launches;
+  if (!p.on) return;
+  Rec r{cls, work, p.get(), p.get()};
+  if (r.a) cudaEventRecord(r.a, st);
+  p.recs.push_back(r);
+  slot_ = int(p.recs.size()) - 1;
+}
+
+LaunchScope::~LaunchScope() {
+  if (slot_ < 0) return;
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (slot_ < int(p.recs.size()) && p.recs[slot_].b) cudaEventRecord(p.recs[slot_].b, st_);
+}
+
+}  // namespace slora
+
+extern "C" int64_t slora_launch_count(void) { return slora::prof().launches; }
+
+extern "C" void slora_profile_enable(int on) {
+  slora::Profiler& p = slora::prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  cudaDeviceSynchronize();
+  p.release_all();
+  p.on = on != 0;
+}
+
+extern "C" slora_status slora_profile_read(const char* kernel_class, int64_t* launches,
+                                           double* total_ms, double* work) {
+  using namespace slora;
+  clear_error();
+  int cls = -1;
+  for (int i = 0; i < kNumClasses; ++i)
+    if (kernel_class && std::string(kernel_class) == kClassNames[i]) cls = i;
+  if (cls < 0) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "unknown kernel class '%s'",
+                          kernel_class ? kernel_class : "(null)");
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  int64_t n = 0;
+  double ms = 0.0, w = 0.0;
+  for (auto& r : p.recs) {
+    if (r.cls != cls || !r.a || !r.b) continue;
+    SLORA_CUDA(cudaEventSynchronize(r.b));
+    float e = 0.0f;
+    SLORA_CUDA(cudaEventElapsedTime(&e, r.a, r.b));
+    ++n;
+    ms += e;
+    w += r.work;
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  if (work) *work = w;
+  return SLORA_OK;
+}

@@ -1,0 +1,261 @@
+/*
+ * slora.h — C ABI of the contextually sparse LoRA hot path (SparseLoRA) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (page title, section):
+ *   [ART]  SparseLoRA news article (lsdiaocha.cn, ICML 2025 / arXiv 2506.16500),
+ *          sections 1 "dynamic sparsity design", 2 "SVD sparsity estimator",
+ *          3 "layer sensitivity" (context/output token split), 6 "compatibility"
+ *          (structured sparsity that real GPUs accelerate), 7 "implementation
+ *          details" (rank-8 estimator, slicing and compute order).
+ *   [ABS]  "SparseLoRA: accelerating LLM fine-tuning with contextual sparsity"
+ *          (xinfinite.net forum post), the paper's abstract: a training-free
+ *          SVD sparsity estimator dynamically selects sparse weight subsets for
+ *          the loss and gradient computation.
+ *
+ * Conventions shared by every call
+ *   - Layout follows PyTorch nn.Linear / PEFT: a frozen weight W0 is n x k
+ *     (out x in, row-major), y = x W0^T; LoRA A is r x k, B is n x r and the
+ *     LoRA output is lora_scale * (x A^T) B^T.  All matrices are row-major and
+ *     contiguous (leading dimension = number of columns).
+ *   - Tokens: X has T = batch * seq rows; in sequence b the first ctx_len[b]
+ *     rows are context tokens (sparse path), the other rows are output tokens
+ *     (dense path) [ART §3].  "Compact context" matrices hold the T_C context
+ *     rows in (sequence, position) order, "compact output" matrices the T_O
+ *     output rows in the same order.  ctx_len is a HOST array.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller and must be
+ *     16-byte aligned; the library never allocates device memory.  Scratch
+ *     space is the caller's workspace `ws`.  Workspace query: call with
+ *     ws == NULL; the call validates its arguments, stores the bytes it needs
+ *     in *ws_bytes, launches nothing and returns SLORA_OK.  Otherwise
+ *     *ws_bytes is the size of `ws` and must be at least that amount.
+ *   - dtype SLORA_F32 computes in fp32 throughout (CUDA-core FMA, for exact
+ *     parity work); SLORA_BF16 takes bf16 activations/weights, accumulates in
+ *     fp32 on the tensor cores and writes bf16 activations.  LoRA gradients
+ *     (dA, dB) and estimator factors (L, U) are always fp32.
+ *   - Calls are asynchronous on `stream` and return a slora_status.  A failed
+ *     call launches nothing (argument errors) or reports the first CUDA error
+ *     (SLORA_ERR_CUDA).  slora_last_error_string() gives a thread-local text.
+ *     Calls are re-entrant when given distinct workspaces and outputs.
+ *   - Requires an sm_100 device (SLORA_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef SLORA_H_
+#define SLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* slora_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  SLORA_OK = 0,
+  SLORA_ERR_INVALID_ARG = 1, /* null pointer, bad enum, sparsity outside [0,1) */
+  SLORA_ERR_SHAPE = 2,       /* inconsistent or unsupported sizes            */
+  SLORA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned             */
+  SLORA_ERR_WORKSPACE = 4,   /* *ws_bytes smaller than required              */
+  SLORA_ERR_UNSUPPORTED = 5, /* device is not sm_100                         */
+  SLORA_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed            */
+  SLORA_ERR_TIMEOUT = 7      /* reserved: bounded device wait expired        */
+} slora_status;
+
+typedef enum { SLORA_F32 = 0, SLORA_BF16 = 1 } slora_dtype;
+
+typedef enum {
+  SLORA_CRIT_FFN_SWIGLU_L2 = 0, /* SwiGLU FFN: L2 norm of the estimated activation */
+  SLORA_CRIT_QK_NORM = 1        /* attention q/k: QK-norm, top-k per head group     */
+} slora_criterion;
+
+typedef enum {
+  SLORA_SLICE_NONE = 0,     /* dense LoRA linear on every row                         */
+  SLORA_SLICE_OUT_ROWS = 1, /* context rows compute only output channels idx (q,k,gate,up) */
+  SLORA_SLICE_IN_COLS = 2   /* context rows read only input channels idx (down, o)    */
+} slora_slice;
+
+typedef struct {
+  int32_t batch;          /* number of sequences                          */
+  int32_t seq;            /* rows per sequence                            */
+  const int32_t* ctx_len; /* HOST array [batch], 0 <= ctx_len[b] <= seq   */
+} slora_tokens;
+
+/* Text of the last error on this thread ("" after success). */
+const char* slora_last_error_string(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int slora_version(void);
+
+/*
+ * Launch accounting and optional per-kernel timing (not part of the method;
+ * used to measure it).
+ *   slora_launch_count()   kernels this library has launched in this process.
+ *   slora_profile_enable() on != 0 clears the record and brackets every later
+ *                          launch with CUDA events on its stream; 0 stops.
+ *   slora_profile_read()   totals since enabling for one kernel class:
+ *                          "gemm_tc" (tcgen05 sliced GEMMs), "gemm_simt"
+ *                          (CUDA-core GEMMs), "estimate" (channel scores),
+ *                          "select" (top-k), "elementwise", "aux" (row maps,
+ *                          operand packing), "prepare".  It synchronizes the
+ *                          recorded events.  work = algorithmic FLOPs for the
+ *                          GEMM classes (2*M*N*K on the selected sizes), bytes
+ *                          moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
+ */
+int64_t slora_launch_count(void);
+void slora_profile_enable(int on);
+slora_status slora_profile_read(const char* kernel_class, int64_t* launches, double* total_ms,
+                                double* work);
+
+/*
+ * slora_svd_prepare — offline truncated SVD of one frozen weight, done once
+ * before training [ART §2: the weights are decomposed once, ahead of training,
+ * keeping the leading singular modes; §7: rank 8].
+ *
+ *   W      [n x k] dtype dt, the frozen weight W0.
+ *   rank   r, 1 <= r <= min(n, k, 48).
+ *   n_iter subspace iterations (0 = default 12).
+ *   seed   seed of the counter-based Gaussian start block.
+ *   L      out [k x r] fp32: V_r diag(sigma_r) (right factor times singular values).
+ *   U      out [n x r] fp32: U_r (orthonormal left factor), so X W0^T ~= (X L) U^T.
+ *   W_t    out [k x n] dtype dt, optional (NULL = skip): the transposed copy of W
+ *          that SLORA_SLICE_IN_COLS layers and the FFN down projection take.
+ * Singular-vector signs are arbitrary; only products such as L U^T are defined.
+ * Method: randomized block subspace iteration with Cholesky-QR
+ * re-orthonormalisation and an fp64 Jacobi eigen-solve of the small projected
+ * Gram matrix, all on the device.  Ordered on `stream`; not on the hot path.
+ */
+slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, slora_dtype dt, int rank,
+                               int n_iter, uint64_t seed, float* L, float* U, void* W_t,
+                               void* ws, size_t* ws_bytes, slora_stream_t stream);
+
+/*
+ * slora_estimate_select — online low-rank estimate on the context tokens,
+ * channel scores and top-k selection [ART §1 criteria (FFN: L2 norm of the
+ * neuron's activity; q/k: QK-norm from the query-key product), §2 estimator,
+ * §3 per-layer ratio; ABS].
+ *
+ *   crit     SLORA_CRIT_FFN_SWIGLU_L2 or SLORA_CRIT_QK_NORM.
+ *   X        [T x d] dtype dt, layer input, full row layout (context rows used).
+ *   (L0,U0)  factors of gate (FFN) or q (QK): L0 [d x rank], U0 [n0 x rank] fp32.
+ *   (L1,U1)  factors of up (FFN) or k (QK):   L1 [d x rank], U1 [n1 x rank] fp32.
+ *   FFN: n0 == n1 == d_ff; heads/kv_heads/head_dim ignored.  score_j is the L2
+ *        norm over context tokens of silu(g_hat_j) * u_hat_j with
+ *        g_hat = (X_C L0) U0^T, u_hat = (X_C L1) U1^T; k_keep = d_ff - floor(s*d_ff).
+ *        idx_out [k_keep] int32 receives the kept channels in ascending order.
+ *   QK:  n0 = heads*head_dim, n1 = kv_heads*head_dim, heads % kv_heads == 0.
+ *        Group g (one key head, heads/kv_heads query heads) scores channel c as
+ *        ||K_hat[:,g,c]|| * sum_h ||Q_hat[:,h,c]||; k_h = head_dim - floor(s*head_dim)
+ *        channels are kept per group.  idx_out [(heads + kv_heads) * k_h] int32:
+ *        first, for every query head h, its group's kept channels as
+ *        h*head_dim + c (ascending); then for every key head g, g*head_dim + c.
+ *   Ties: equal scores go to the lower index.
+ *   sparsity  s in [0, 1).
+ *   k_out     HOST int32*, receives k_keep (FFN) or k_h (QK).
+ *   scores_out optional [d_ff] (FFN) or [kv_heads*head_dim] (QK) fp32 scores.
+ */
+slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dtype dt,
+                                   const slora_tokens* tok, int64_t d, const float* L0,
+                                   const float* U0, int64_t n0, const float* L1, const float* U1,
+                                   int64_t n1, int rank, int heads, int kv_heads, int head_dim,
+                                   float sparsity, int32_t* idx_out, int32_t* k_out,
+                                   float* scores_out, void* ws, size_t* ws_bytes,
+                                   slora_stream_t stream);
+
+/*
+ * slora_linear_fwd — one LoRA linear on the selected slices, output tokens
+ * dense [ART §1, §3, §6, §7; ABS].
+ *
+ *   W       frozen weight in the layout whose ROWS are the sliced channels:
+ *           NONE / OUT_ROWS: W0 [n x k];  IN_COLS: W0^T [k x n].
+ *   A [r x k], B [n x r] dtype dt; lora_scale s.
+ *   idx     device int32 [n_idx], ascending, distinct, within [0, n) (OUT_ROWS)
+ *           or [0, k) (IN_COLS); ignored for NONE.
+ *   side NONE:     X_ctx = X [T x k];                  Y_ctx = Y [T x n].
+ *   side OUT_ROWS: X_ctx = X [T x k];                  Y_ctx [T_C x n_idx] compact,
+ *                  Y_ctx[:, j] = X_C W0[idx_j]^T + s (X_C A^T) B[idx_j]^T;
+ *                                                      Y_out [T_O x n] compact, dense.
+ *   side IN_COLS:  X_ctx [T_C x n_idx] compact (column j = input channel idx_j),
+ *                  X_out [T_O x k] compact;            Y_ctx = Y [T x n] full layout,
+ *                  Y[C] = X_ctx W0[:, idx]^T + s (X_ctx A[:, idx]^T) B^T.
+ *   XA_save [T x r] fp32 full row layout, optional: the LoRA down-projection of
+ *           each row as used above (unscaled), needed by slora_linear_bwd.
+ * Unused pointers may be NULL.  Channels outside idx are not computed for
+ * context rows (they are not stored: outputs are compact).
+ */
+slora_status slora_linear_fwd(slora_dtype dt, const slora_tokens* tok, int64_t k, int64_t n,
+                              const void* W, const void* A, const void* B, int r_lora,
+                              float lora_scale, slora_slice side, const int32_t* idx,
+                              int32_t n_idx, const void* X_ctx, const void* X_out, void* Y_ctx,
+                              void* Y_out, float* XA_save, void* ws, size_t* ws_bytes,
+                              slora_stream_t stream);
+
+/*
+ * slora_linear_bwd — backward of slora_linear_fwd with W0 frozen [ABS: loss
+ * and gradient computed on the selected subset].
+ *
+ *   Same layer arguments as the forward, plus
+ *   XA_save  [T x r] fp32 from the forward.
+ *   dY_ctx / dY_out  shaped like Y_ctx / Y_out of the forward.
+ *   dX_ctx / dX_out  shaped like X_ctx / X_out of the forward (written).
+ *   dA [r x k], dB [n x r] fp32, OVERWRITTEN.  Skipped channels of context rows
+ *   contribute nothing: with no output tokens, rows of dB (OUT_ROWS) or
+ *   columns of dA (IN_COLS) outside idx are exactly zero.
+ */
+slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok, int64_t k, int64_t n,
+                              const void* W, const void* A, const void* B, int r_lora,
+                              float lora_scale, slora_slice side, const int32_t* idx,
+                              int32_t n_idx, const void* X_ctx, const void* X_out,
+                              const float* XA_save, const void* dY_ctx, const void* dY_out,
+                              void* dX_ctx, void* dX_out, float* dA, float* dB, void* ws,
+                              size_t* ws_bytes, slora_stream_t stream);
+
+/* One SwiGLU FFN layer: out = (silu(X Wg^T) * (X Wu^T)) Wd^T, each projection
+ * with its LoRA pair.  All device pointers; weights and LoRA factors in the
+ * call's dtype, estimator factors fp32. */
+typedef struct {
+  int64_t d, d_ff;       /* model and intermediate width                       */
+  int32_t r_svd;         /* estimator rank (1..48)                             */
+  int32_t r_lora;        /* LoRA rank (1..32)                                  */
+  float lora_scale;      /* s                                                  */
+  const void* Wg;        /* [d_ff x d] gate                                    */
+  const void* Wu;        /* [d_ff x d] up                                      */
+  const void* Wd_t;      /* [d_ff x d] TRANSPOSED down weight (Wd is d x d_ff) */
+  const void *Ag, *Bg;   /* [r x d], [d_ff x r]                                */
+  const void *Au, *Bu;   /* [r x d], [d_ff x r]                                */
+  const void *Ad, *Bd;   /* [r x d_ff], [d x r]                                */
+  const float *Lg, *Ug;  /* gate estimator factors [d x r_svd], [d_ff x r_svd] */
+  const float *Lu, *Uu;  /* up estimator factors                               */
+} slora_ffn_layer;
+
+typedef struct {
+  float *dAg, *dBg, *dAu, *dBu, *dAd, *dBd; /* fp32, shapes of the factors; overwritten */
+} slora_ffn_grads;
+
+/*
+ * slora_ffn_fwd_bwd — the whole hot path of one FFN layer for one step:
+ * estimate + select (unless idx_force), sliced gate/up on the kept channels
+ * for context rows, down projection reading only those channels, dense
+ * output rows, then the matching sparse backward [ART §1-§3, §6-§7; ABS].
+ *
+ *   X, dOut   [T x d] dtype dt, full row layout.
+ *   sparsity  s in [0, 1): k_keep = d_ff - floor(s*d_ff).
+ *   out, dX   [T x d] dtype dt (written).
+ *   grads     the six LoRA gradients (written).
+ *   idx_out   device int32 [d_ff]: receives the k_keep channels used (ascending).
+ *   k_out     HOST int32*: receives k_keep.
+ *   idx_force optional device int32 [k_force] ascending channel set: skips the
+ *             estimator and uses this set (same-index parity runs); then
+ *             sparsity is ignored and k_keep = k_force.
+ */
+slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
+                               const slora_tokens* tok, float sparsity, const void* X,
+                               const void* dOut, void* out, void* dX, const slora_ffn_grads* grads,
+                               int32_t* idx_out, int32_t* k_out, const int32_t* idx_force,
+                               int32_t k_force, void* ws, size_t* ws_bytes,
+                               slora_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLORA_H_ */

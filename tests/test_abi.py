@@ -1,0 +1,122 @@
+"""The C-ABI library loads and exports what include/slora.h declares; host-side
+validation and workspace queries work without a GPU (no compute is called)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "slora.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(slora_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from contextual_sparsity_lora_svd_b200 import build
+    build.build()
+    from contextual_sparsity_lora_svd_b200 import _lib
+    return _lib
+
+
+def test_header_declares_the_five_calls():
+    names = _declared()
+    for n in ("slora_svd_prepare", "slora_estimate_select", "slora_linear_fwd",
+              "slora_linear_bwd", "slora_ffn_fwd_bwd"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (slora_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(L.lib(), n)
+    assert sorted(L.EXPORTS) == _declared()
+
+
+def test_version(L):
+    assert L.version() == 100
+
+
+FAKE = 0x10000  # 16-byte aligned dummy address: never dereferenced by validation/queries
+
+
+def _ffn_query(L, **over):
+    lay = L.ffn_layer_struct(256, 688, 8, 8, 1.0, *([FAKE] * 9), FAKE, FAKE, FAKE, FAKE)
+    g = L.ffn_grads_struct(*([FAKE] * 6))
+    args, keep = L.ffn_args(L.F32, lay, 1, 256, [192], over.get("s", 0.5), FAKE, FAKE, FAKE, FAKE,
+                            g, FAKE)
+    return L.workspace_size("slora_ffn_fwd_bwd", args), keep
+
+
+def test_ffn_workspace_query_and_k(L):
+    need, keep = _ffn_query(L)
+    assert need > 0
+    assert keep[2].value == 344
+
+
+@pytest.mark.parametrize("s", [-0.1, 1.0, float("nan")])
+def test_bad_sparsity_rejected(L, s):
+    with pytest.raises(L.SloraError) as e:
+        _ffn_query(L, s=s)
+    assert e.value.status == 1
+
+
+def test_misaligned_pointer_rejected(L):
+    lay = L.ffn_layer_struct(256, 688, 8, 8, 1.0, FAKE + 2, *([FAKE] * 8), FAKE, FAKE, FAKE, FAKE)
+    g = L.ffn_grads_struct(*([FAKE] * 6))
+    args, keep = L.ffn_args(L.F32, lay, 1, 256, [192], 0.5, FAKE, FAKE, FAKE, FAKE, g, FAKE)
+    with pytest.raises(L.SloraError) as e:
+        L.workspace_size("slora_ffn_fwd_bwd", args)
+    assert e.value.status == 3
+
+
+def test_bad_shapes_rejected(L):
+    tok, keep = L.make_tokens(2, 8, [3, 9])  # ctx_len > seq
+    args = [L.SLICE_OUT_ROWS, ctypes.byref(tok), 16, 32, FAKE, FAKE, FAKE, 4, 1.0, 1, FAKE, 4,
+            FAKE, FAKE, FAKE, FAKE, FAKE]
+    args = [L.F32] + args[1:]
+    with pytest.raises(L.SloraError) as e:
+        L.workspace_size("slora_linear_fwd", args)
+    assert e.value.status == 2
+    tok2, keep2 = L.make_tokens(2, 8, [3, 8])
+    ok = [L.F32, ctypes.byref(tok2), 16, 32, FAKE, FAKE, FAKE, 4, 1.0, L.SLICE_OUT_ROWS, FAKE, 4,
+          FAKE, FAKE, FAKE, FAKE, FAKE]
+    assert L.workspace_size("slora_linear_fwd", ok) > 0
+    bad_idx = list(ok)
+    bad_idx[11] = 33  # n_idx > n
+    with pytest.raises(L.SloraError):
+        L.workspace_size("slora_linear_fwd", bad_idx)
+    bad_row = list(ok)
+    bad_row[2] = 18  # k not a multiple of 4 (16-byte rows)
+    with pytest.raises(L.SloraError):
+        L.workspace_size("slora_linear_fwd", bad_row)
+
+
+def test_estimate_select_query_qk_layout(L):
+    tok, keep = L.make_tokens(4, 16, [12] * 4)
+    k_out = ctypes.c_int32(0)
+    args = [L.CRIT_QK, FAKE, L.BF16, ctypes.byref(tok), 64, FAKE, FAKE, 8 * 16, FAKE, FAKE, 2 * 16,
+            8, 8, 2, 16, 0.5, FAKE, ctypes.byref(k_out), None]
+    assert L.workspace_size("slora_estimate_select", args) > 0
+    assert k_out.value == 8
+    args[7] = 8 * 16 + 1  # n0 != heads*head_dim
+    with pytest.raises(L.SloraError):
+        L.workspace_size("slora_estimate_select", args)
+
+
+def test_prepare_rank_limits(L):
+    args = [FAKE, 64, 32, L.F32, 49, 0, 0, FAKE, FAKE, None]
+    with pytest.raises(L.SloraError):
+        L.workspace_size("slora_svd_prepare", args)
+    args[4] = 8
+    assert L.workspace_size("slora_svd_prepare", args) > 0
