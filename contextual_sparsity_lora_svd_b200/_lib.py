@@ -74,14 +74,15 @@ _sig("slora_svd_prepare", c_int,
      [c_vp, c_i64, c_i64, c_int, c_int, c_int, c_u64, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
 _sig("slora_estimate_select", c_int,
      [c_int, c_vp, c_int, ctypes.POINTER(Tokens), c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64,
-      c_int, c_int, c_int, c_int, c_f32, c_vp, P_I32, c_vp, c_vp, P_SZ, c_vp])
+      c_int, c_int, c_int, c_int, ctypes.c_double, c_vp, P_I32, c_vp, c_vp, P_SZ, c_vp])
 _LIN = [c_int, ctypes.POINTER(Tokens), c_i64, c_i64, c_vp, c_vp, c_vp, c_int, c_f32, c_int, c_vp,
         c_i32]
 _sig("slora_linear_fwd", c_int, _LIN + [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
 _sig("slora_linear_bwd", c_int,
      _LIN + [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
 _sig("slora_ffn_fwd_bwd", c_int,
-     [c_int, ctypes.POINTER(FfnLayer), ctypes.POINTER(Tokens), c_f32, c_vp, c_vp, c_vp, c_vp,
+     [c_int, ctypes.POINTER(FfnLayer), ctypes.POINTER(Tokens), ctypes.c_double, c_vp, c_vp, c_vp,
+      c_vp,
       ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 
 _sig("slora_launch_count", c_i64, [])

@@ -42,15 +42,15 @@ slora_status check_row(const char* fn, const char* what, int64_t len, int dt) {
   return SLORA_OK;
 }
 
-slora_status check_sparsity(const char* fn, float s) {
-  if (!(s >= 0.0f && s < 1.0f))
-    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: sparsity %g outside [0, 1)", fn, double(s));
+slora_status check_sparsity(const char* fn, double s) {
+  if (!(s >= 0.0 && s < 1.0))
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: sparsity %g outside [0, 1)", fn, s);
   return SLORA_OK;
 }
 
 // Channels kept at sparsity s: N - floor(s * N) (the skipped count rounds down).
-int64_t keep_count(int64_t N, float s) {
-  double skip = std::floor(double(s) * double(N) + 1e-9);
+int64_t keep_count(int64_t N, double s) {
+  double skip = std::floor(s * double(N) + 1e-9);
   return N - int64_t(skip);
 }
 
@@ -146,7 +146,7 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
                                               const slora_tokens* tok, int64_t d, const float* L0,
                                               const float* U0, int64_t n0, const float* L1,
                                               const float* U1, int64_t n1, int rank, int heads,
-                                              int kv_heads, int head_dim, float sparsity,
+                                              int kv_heads, int head_dim, double sparsity,
                                               int32_t* idx_out, int32_t* k_out, float* scores_out,
                                               void* ws, size_t* ws_bytes, slora_stream_t stream) {
   const char* fn = "slora_estimate_select";
@@ -277,7 +277,7 @@ extern "C" slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok
 
 // ------------------------------------------------------------------- FFN
 extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
-                                          const slora_tokens* tok, float sparsity, const void* X,
+                                          const slora_tokens* tok, double sparsity, const void* X,
                                           const void* dOut, void* out, void* dX,
                                           const slora_ffn_grads* grads, int32_t* idx_out,
                                           int32_t* k_out, const int32_t* idx_force,

@@ -158,7 +158,7 @@ slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dt
                                    const slora_tokens* tok, int64_t d, const float* L0,
                                    const float* U0, int64_t n0, const float* L1, const float* U1,
                                    int64_t n1, int rank, int heads, int kv_heads, int head_dim,
-                                   float sparsity, int32_t* idx_out, int32_t* k_out,
+                                   double sparsity, int32_t* idx_out, int32_t* k_out,
                                    float* scores_out, void* ws, size_t* ws_bytes,
                                    slora_stream_t stream);
 
@@ -249,7 +249,7 @@ typedef struct {
  *             sparsity is ignored and k_keep = k_force.
  */
 slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
-                               const slora_tokens* tok, float sparsity, const void* X,
+                               const slora_tokens* tok, double sparsity, const void* X,
                                const void* dOut, void* out, void* dX, const slora_ffn_grads* grads,
                                int32_t* idx_out, int32_t* k_out, const int32_t* idx_force,
                                int32_t k_force, void* ws, size_t* ws_bytes,
