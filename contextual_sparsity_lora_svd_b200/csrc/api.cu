@@ -234,7 +234,7 @@ extern "C" slora_status slora_linear_fwd(slora_dtype dt, const slora_tokens* tok
   if (side == SLORA_SLICE_IN_COLS && ti.T_O > 0) REQ_PTR(X_out);
   LinearDesc L{int(dt), ti, k, n, W, A, B, r_lora, lora_scale, side, idx, n_idx};
   Arena plan;
-  SLORA_TRY(linear_fwd_run(L, nullptr, X_ctx, X_out, Y_ctx, Y_out, XA_save, plan, true, nullptr));
+  SLORA_TRY(linear_fwd_run(L, tok, X_ctx, X_out, Y_ctx, Y_out, XA_save, plan, true, nullptr));
   const bool query = ws == nullptr;
   SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
   if (query) return SLORA_OK;
@@ -263,7 +263,7 @@ extern "C" slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok
   if (side == SLORA_SLICE_IN_COLS && ti.T_O > 0) { REQ_PTR(X_out); REQ_PTR(dX_out); }
   LinearDesc L{int(dt), ti, k, n, W, A, B, r_lora, lora_scale, side, idx, n_idx};
   Arena plan;
-  SLORA_TRY(linear_bwd_run(L, nullptr, X_ctx, X_out, XA_save, dY_ctx, dY_out, dX_ctx, dX_out, dA,
+  SLORA_TRY(linear_bwd_run(L, tok, X_ctx, X_out, XA_save, dY_ctx, dY_out, dX_ctx, dX_out, dA,
                            dB, plan, true, nullptr));
   const bool query = ws == nullptr;
   SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
@@ -315,7 +315,7 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   SLORA_TRY(parse_tokens(tok, &ti));
   FfnDesc F{int(dt), ti, Ly, Gr, kkeep};
   Arena plan;
-  SLORA_TRY(ffn_run(F, nullptr, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr));
+  SLORA_TRY(ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr));
   const bool query = ws == nullptr;
   SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
   *k_out = int32_t(kkeep);

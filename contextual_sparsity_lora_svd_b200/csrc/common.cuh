@@ -71,15 +71,22 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ------------------------------------------------------------- tokens
 // Row maps of the context / output tokens of one call, built on the device.
-constexpr int kMaxBatch = 4096;
+constexpr int kMaxBatch = 2048;
 struct TokenInfo {
   int batch = 0, seq = 0;
   int64_t T = 0, T_C = 0, T_O = 0;
 };
 slora_status parse_tokens(const slora_tokens* tok, TokenInfo* info);
-// Writes ctx_rows[T_C] and out_rows[T_O] (int32 row indices into the full layout).
+// Writes ctx_rows[T_C] and out_rows[T_O] (int32 row indices into the full
+// layout) and, when given, the 128-row M-tile lists of the context and output
+// rows: int4 {full_row0, compact_row0, nvalid, 0}, one list per row kind, a
+// tile never crossing a sequence.
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
-                            int32_t* out_rows, cudaStream_t st);
+                            int32_t* out_rows, cudaStream_t st, int4* ctx_tiles = nullptr,
+                            int4* out_tiles = nullptr);
+// Number of 128-row tiles of the context rows / output rows.
+int64_t count_tiles(const slora_tokens* tok, bool ctx);
+inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 
 // ------------------------------------------------------------- launches
 // Kernel classes for launch accounting (names in slora_profile_read).

@@ -99,6 +99,10 @@ __global__ void __launch_bounds__(NT) gemm_simt_kernel(const __grid_constant__ G
       float v = acc[a][b];
       if (c.accumulate) v += ld_elem(c.ptr, off, c.dt);
       st_elem(c.ptr, off, c.dt, v);
+      if (c.ptr2) {
+        const int64_t r2 = c.gm2 ? c.gm2[m] : m;
+        static_cast<__nv_bfloat16*>(c.ptr2)[r2 * c.ld2 + n] = __float2bfloat16_rn(c.scale2 * v);
+      }
     }
   }
 }

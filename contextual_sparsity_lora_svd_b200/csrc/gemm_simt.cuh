@@ -35,6 +35,11 @@ struct OutRef {
   const int32_t* gm = nullptr;
   const int32_t* gn = nullptr;
   int accumulate = 0;  // 1: C += result (read-modify-write in fp32)
+  // optional second copy: bf16(scale2 * C(m, n)) at ptr2[(gm2 ? gm2[m] : m) * ld2 + n]
+  void* ptr2 = nullptr;
+  int64_t ld2 = 0;
+  const int32_t* gm2 = nullptr;
+  float scale2 = 1.0f;
 };
 
 constexpr int kMaxSegs = 4;
@@ -63,6 +68,12 @@ inline OutRef out_rowmajor(void* p, int dt, int64_t ldc, const int32_t* gm = nul
                            const int32_t* gn = nullptr, int acc = 0) {
   OutRef o;
   o.ptr = p; o.dt = dt; o.ldc = ldc; o.gm = gm; o.gn = gn; o.accumulate = acc;
+  return o;
+}
+
+inline OutRef with_bf16_copy(OutRef o, void* p2, int64_t ld2, float scale2,
+                             const int32_t* gm2 = nullptr) {
+  o.ptr2 = p2; o.ld2 = ld2; o.scale2 = scale2; o.gm2 = gm2;
   return o;
 }
 

@@ -1,0 +1,587 @@
+// tcgen05 sliced GEMM for sm_100a (see gemm_tc.cuh for the operand forms).
+//
+// Persistent kernel, one 256-thread CTA per SM:
+//   warp 0      TMA producer: A tile (128 x 64) and B tile (256 x 64) per
+//               stage; gathered B rows arrive through cp.async.bulk.tensor
+//               tile::gather4 (4 rows per instruction, spread over the lanes)
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 x bf16 -> fp32) into a TMEM accumulator
+//   warp 2      TMEM allocator (512 columns = two 128x256 fp32 accumulators)
+//   warps 4..7  epilogue: tcgen05.ld rows of the finished accumulator, apply
+//               the epilogue, store bf16; the other accumulator is being
+//               filled meanwhile
+// Shared memory: 4 stages x (16 KB A + 32 KB B), 128-byte swizzle (the TMA
+// swizzle and the UMMA descriptor layout agree: 8-row / 1024-byte atoms).
+// Every mbarrier wait is bounded (clock64 budget); on expiry the CTA raises
+// an abort flag, waits (bounded) for its copies in flight, frees TMEM and
+// returns, and the host reads SLORA_ERR_TIMEOUT from the device flag.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm_tc.cuh"
+
+namespace slora {
+
+__device__ int g_tc_error = 0;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;               // 16 KB
+constexpr int B_BYTES = BN * BK * 2;               // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 48 KB
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr long long WAIT_BUDGET = 4000000000LL;    // ~2 s of SM clocks per wait
+
+struct alignas(64) TcParams {
+  CUtensorMap amap[4];
+  CUtensorMap bmap[4][2];
+  const int32_t* idx[4];
+  int nidx[4];
+  int nkb[4];
+  int bmode[4];
+  int bpair[4];
+  int nseg;
+  const int4* tiles;
+  int n_mtiles, n_ntiles;
+  int a_compact, out_compact;
+  int paired;
+  int N;
+  int epi;
+  void* out0;
+  void* out1;
+  void* out2;
+  long long ldo;
+  const void* in0;
+  const void* in1;
+  long long ldi;
+};
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase of parity `parity`; false on abort/expiry.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
+  if (mbar_try(b, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try(b, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > WAIT_BUDGET) {
+      *abort = 1;
+      atomicExch(&g_tc_error, 1);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
+                                         int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
+                                            int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;  // descriptor version (sm_100)
+  d |= uint64_t(2) << 61;  // SWIZZLE_128B
+  return d;
+}
+// Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, M=128, N=256.
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) |
+         (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          su32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Store 32 consecutive bf16 values (row-major, column c0..c0+31) with
+// per-column masking at the right edge.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* row, int c0, int N, const float* v) {
+  if (c0 + 32 <= N) {
+    uint4* dst = reinterpret_cast<uint4*>(row + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 h[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
+      dst[q] = *reinterpret_cast<uint4*>(h);
+    }
+  } else {
+    for (int j = 0; j < 32 && c0 + j < N; ++j) row[c0 + j] = __float2bfloat16_rn(v[j]);
+  }
+}
+__device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int c0, int N, float* v) {
+  if (c0 + 32 <= N) {
+    const uint4* src = reinterpret_cast<const uint4*>(row + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u = src[q];
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 f = __bfloat1622float2(h[e]);
+        v[q * 8 + 2 * e] = f.x;
+        v[q * 8 + 2 * e + 1] = f.y;
+      }
+    }
+  } else {
+    for (int j = 0; j < 32; ++j) v[j] = (c0 + j < N) ? __bfloat162float(row[c0 + j]) : 0.0f;
+  }
+}
+
+struct TileInfo {
+  int a_row, out_row, nvalid, n0;
+};
+__device__ __forceinline__ TileInfo tile_info(const TcParams& p, int t) {
+  const int mt = t % p.n_mtiles, nt = t / p.n_mtiles;
+  const int4 tl = p.tiles[mt];
+  TileInfo ti;
+  ti.a_row = p.a_compact ? tl.y : tl.x;
+  ti.out_row = p.out_compact ? tl.y : tl.x;
+  ti.nvalid = tl.z;
+  ti.n0 = nt * (p.paired ? BN / 2 : BN);
+  return ti;
+}
+
+__global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     su32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int total = p.n_mtiles * p.n_ntiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileInfo ti = tile_info(p, t);
+      const int nt = t / p.n_mtiles;
+      for (int s = 0; s < p.nseg && ok; ++s) {
+        const int mode = p.bmode[s];
+        const int32_t* idx = p.idx[s];
+        const int nidx = p.nidx[s];
+        // K-major gather: this lane's rows are fixed for the whole tile
+        int krow[2][4];
+        if (mode == B_K_GATHER) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int g = lane + 32 * j;  // 64 groups of 4 rows
+            const int h = g / 32, gi = g % 32;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              int n = p.bpair[s] ? (ti.n0 + 4 * gi + q) : (nt * BN + 128 * h + 4 * gi + q);
+              n = n < nidx ? n : nidx - 1;
+              krow[j][q] = __ldg(idx + n);
+            }
+          }
+        }
+        for (int kb = 0; kb < p.nkb[s]; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) { ok = false; break; }
+          if (lane == 0) mbar_expect_tx(&full[stage], STAGE_BYTES);
+          __syncwarp();
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          if (lane == 0) tma_load(sa, &p.amap[s], &full[stage], kb * BK, ti.a_row);
+          if (mode == B_K) {
+            if (lane < 2) {
+              const int h = lane;
+              const int row = p.bpair[s] ? ti.n0 : nt * BN + 128 * h;
+              tma_load(sb + h * (B_BYTES / 2), &p.bmap[s][p.bpair[s] ? h : 0], &full[stage],
+                       kb * BK, row);
+            }
+          } else if (mode == B_K_GATHER) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int g = lane + 32 * j;
+              const int h = g / 32;
+              tma_gather4(sb + g * 512, &p.bmap[s][p.bpair[s] ? h : 0], &full[stage], kb * BK,
+                          krow[j][0], krow[j][1], krow[j][2], krow[j][3]);
+            }
+          } else if (mode == B_MN) {
+            if (lane < 4)
+              tma_load(sb + lane * 8192, &p.bmap[s][0], &full[stage], ti.n0 + 64 * lane, kb * BK);
+          } else {  // B_MN_GATHER
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int g = lane + 32 * j;
+              const int a = g / 16, grp = g % 16;
+              int r[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                int k = kb * BK + 4 * grp + q;
+                k = k < nidx ? k : nidx - 1;
+                r[q] = __ldg(idx + k);
+              }
+              tma_gather4(sb + a * 8192 + grp * 512, &p.bmap[s][0], &full[stage],
+                          ti.n0 + 64 * a, r[0], r[1], r[2], r[3]);
+            }
+          }
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // let the copies already issued land before the CTA can exit
+      int st2 = stage;
+      uint32_t ph2 = phase;
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--st2 < 0) { st2 = STAGES - 1; ph2 ^= 1u; }
+        const long long t0 = clock64();
+        while (!mbar_try(&full[st2], ph2) && clock64() - t0 < WAIT_BUDGET) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = uint32_t(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort)) break;
+        fence_after();
+        const uint32_t d = tbase + uint32_t(acc * BN);
+        bool first = true;
+        for (int s = 0; s < p.nseg && ok; ++s) {
+          const int bmn = p.bmode[s] >= B_MN;
+          const uint32_t idesc = idesc_bf16(BM, BN, bmn);
+          for (int kb = 0; kb < p.nkb[s]; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
+            fence_after();
+            const uint32_t sa = su32(smem + stage * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = sdesc(sa + k * 32, 16, 1024);
+              const uint64_t bd = bmn ? sdesc(sb + k * 2048, 8192, 1024) : sdesc(sb + k * 32, 16, 1024);
+              mma_bf16(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+            }
+            first = false;
+            mma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        }
+        mma_commit(&tfull[acc]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - 4;
+    const int r = q * 32 + lane;  // row within the tile == TMEM lane
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = uint32_t(it >> 1) & 1u;
+      if (!mbar_wait(&tfull[acc], aph, abort)) break;
+      fence_after();
+      const TileInfo ti = tile_info(p, t);
+      const bool valid = r < ti.nvalid;
+      const int64_t orow = int64_t(ti.out_row) + r;
+      const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+      float v[32], w[32];
+      if (p.epi == EPI_SWIGLU_FWD) {
+        __nv_bfloat16* g = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+        __nv_bfloat16* u = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out2) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tl + c * 32, v);
+          tmem_ld32(tl + 128 + c * 32, w);
+          if (valid) {
+            const int c0 = ti.n0 + c * 32;
+            store_row32(g, c0, p.N, v);
+            store_row32(u, c0, p.N, w);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]) * w[j];
+            store_row32(h, c0, p.N, v);
+          }
+        }
+      } else if (p.epi == EPI_SWIGLU_BWD) {
+        const __nv_bfloat16* gi = static_cast<const __nv_bfloat16*>(p.in0) + orow * p.ldi;
+        const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
+        __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+        __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          tmem_ld32(tl + c * 32, v);  // dh
+          const int c0 = ti.n0 + c * 32;
+          if (valid && c0 < p.N) {
+            float gv[32];
+            load_row32(gi, c0, p.N, gv);
+            load_row32(ui, c0, p.N, w);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float sg = sigmoid_f(gv[j]);
+              const float dh = v[j];
+              v[j] = dh * w[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
+              w[j] = dh * gv[j] * sg;                                 // dU
+            }
+            store_row32(dg, c0, p.N, v);
+            store_row32(du, c0, p.N, w);
+          }
+        }
+      } else {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          tmem_ld32(tl + c * 32, v);
+          const int c0 = ti.n0 + c * 32;
+          if (valid && c0 < p.N) store_row32(o, c0, p.N, v);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tbase) : "memory");
+  }
+}
+
+// ----------------------------------------------------------- host helpers
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+slora_status get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  return SLORA_OK;
+}
+
+slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y) {
+  if (!t.ptr) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: null operand");
+  if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) || (t.ld % 8) || t.rows <= 0 || t.cols <= 0)
+    SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: operand not 16-byte aligned (ld=%lld)",
+               (long long)t.ld);
+  cuuint64_t dims[2] = {cuuint64_t(t.cols), cuuint64_t(t.rows)};
+  cuuint64_t strides[1] = {cuuint64_t(t.ld) * 2};
+  cuuint32_t box[2] = {cuuint32_t(box_x), cuuint32_t(box_y)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.ptr), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%lld cols=%lld ld=%lld",
+               int(r), (long long)t.rows, (long long)t.cols, (long long)t.ld);
+  return SLORA_OK;
+}
+
+bool g_attr_set = false;
+
+}  // namespace
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
+  if (g.N <= 0) return SLORA_OK;
+  if (g.tiles == nullptr) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: tile list missing");
+  if (g.n_mtiles <= 0) return SLORA_OK;
+  if (g.nseg < 1 || g.nseg > 4) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: nseg=%d", g.nseg);
+  if (g.ldo % 8 || (g.epi == EPI_SWIGLU_BWD && g.ldi % 8))
+    SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: output leading dimension not a multiple of 8");
+  if (g.N > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: N too large");
+  SLORA_TRY(get_encode());
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  int64_t ksum = 0;
+  for (int s = 0; s < g.nseg; ++s) {
+    const TcSeg& sg = g.seg[s];
+    if (sg.K <= 0) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: segment %d has K=%lld", s, (long long)sg.K);
+    SLORA_TRY(encode(&p.amap[s], sg.a, BK, BM));
+    const bool gather = sg.bmode == B_K_GATHER || sg.bmode == B_MN_GATHER;
+    if (gather && (!sg.idx || sg.nidx <= 0))
+      SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: gather without indices");
+    int by = 0;
+    switch (sg.bmode) {
+      case B_K: by = 128; break;
+      case B_MN: by = 64; break;
+      default: by = 1; break;
+    }
+    SLORA_TRY(encode(&p.bmap[s][0], sg.b0, BK, by));
+    if (sg.bpair) {
+      if (sg.bmode != B_K && sg.bmode != B_K_GATHER)
+        SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: paired halves need a K-major B");
+      SLORA_TRY(encode(&p.bmap[s][1], sg.b1, BK, by));
+    }
+    p.idx[s] = sg.idx;
+    p.nidx[s] = int(sg.nidx);
+    p.nkb[s] = int((sg.K + BK - 1) / BK);
+    p.bmode[s] = sg.bmode;
+    p.bpair[s] = sg.bpair;
+    ksum += sg.K;
+  }
+  p.nseg = g.nseg;
+  p.tiles = g.tiles;
+  p.n_mtiles = g.n_mtiles;
+  const int64_t ncols = g.paired ? BN / 2 : BN;
+  p.n_ntiles = int((g.N + ncols - 1) / ncols);
+  p.a_compact = g.a_compact;
+  p.out_compact = g.out_compact;
+  p.paired = g.paired;
+  p.N = int(g.N);
+  p.epi = g.epi;
+  p.out0 = g.out0;
+  p.out1 = g.out1;
+  p.out2 = g.out2;
+  p.ldo = g.ldo;
+  p.in0 = g.in0;
+  p.in1 = g.in1;
+  p.ldi = g.ldi;
+  if (!g_attr_set) {
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SMEM_BYTES));
+    g_attr_set = true;
+  }
+  const int64_t tiles = int64_t(p.n_mtiles) * p.n_ntiles;
+  const int grid = int(tiles < num_sms() ? tiles : num_sms());
+  // algorithmic FLOPs: 2 * valid rows (g.M) * computed columns * sum of K
+  LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum), st);
+  tc_gemm_kernel<<<grid, 256, SMEM_BYTES, st>>>(p);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status tc_check_error(bool clear) {
+  int v = 0;
+  SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(int)));
+  if (clear && v) {
+    int z = 0;
+    SLORA_CUDA(cudaMemcpyToSymbol(g_tc_error, &z, sizeof(int)));
+  }
+  if (v) SLORA_FAIL(SLORA_ERR_TIMEOUT, "a tcgen05 kernel's bounded wait expired");
+  return SLORA_OK;
+}
+
+}  // namespace slora

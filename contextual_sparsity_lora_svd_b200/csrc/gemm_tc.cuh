@@ -1,0 +1,72 @@
+// tcgen05 (5th-generation tensor core) GEMM for the bf16 sliced contractions.
+//
+//   C[M x N] = sum_seg A_seg[M x K_seg] . B_seg[N x K_seg]^T     (fp32 in TMEM)
+//
+// A operands are bf16 row-major (K-major) and loaded by TMA in 128 x 64
+// boxes.  B operands are bf16 and come in four forms:
+//   B_K          K-major, rows = output channels, contiguous rows
+//   B_K_GATHER   K-major, output channels = rows idx[n] (TMA tile::gather4)
+//   B_MN         MN-major, rows = reduction index k, contiguous
+//   B_MN_GATHER  MN-major, reduction index k -> row idx[k] (tile::gather4)
+// so a selected channel slice of a frozen weight is consumed in place, as
+// rows of W0 (output-side slice) or rows of W0^T (input-side slice), with no
+// compaction copy.  Up to four segments accumulate into one tile (the LoRA
+// branch is one more segment with K = rank).  Epilogues: plain bf16 store,
+// SwiGLU forward on paired gate/up halves (stores g, u and h = silu(g) u), and
+// SwiGLU backward (reads g, u; stores dG, dU).
+//
+// Rows: a list of 128-row M tiles {full_row0, compact_row0, nvalid}; a tile
+// never crosses a sequence, so a tile is contiguous both in the full token
+// layout and in the compact context/output layout.  Each operand picks which.
+#pragma once
+
+#include "common.cuh"
+
+namespace slora {
+
+enum TcBMode : int { B_K = 0, B_K_GATHER = 1, B_MN = 2, B_MN_GATHER = 3 };
+enum TcEpi : int { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2 };
+
+struct TcMat {  // bf16 row-major matrix in global memory
+  const void* ptr = nullptr;
+  int64_t rows = 0, cols = 0, ld = 0;  // ld in elements (multiple of 8)
+};
+
+struct TcSeg {
+  TcMat a;          // [rows x K]: row = tile row base + r, col = k
+  TcMat b0, b1;     // b1 only with bpair (second half of the N tile)
+  int bmode = B_K;
+  int bpair = 0;    // K-major only: half h of the 256-row tile reads b_h rows n0p + r
+  const int32_t* idx = nullptr;  // gather list (N index for B_K_GATHER, K index for B_MN_GATHER)
+  int64_t nidx = 0;              // valid entries of idx
+  int64_t K = 0;
+};
+
+struct TcGemm {
+  const int4* tiles = nullptr;  // {full_row0, compact_row0, nvalid, 0}; null: plain tiling of M
+  int n_mtiles = 0;
+  int a_compact = 0, out_compact = 0;
+  int64_t M = 0;      // plain tiling only
+  int64_t N = 0;      // valid output columns (channels)
+  int paired = 0;     // N tile = 128 channels as two 128-row halves (gate | up)
+  int nseg = 0;
+  TcSeg seg[4];
+  int epi = EPI_STORE;
+  void* out0 = nullptr;  // STORE: C; SWIGLU_FWD: g; SWIGLU_BWD: dG
+  void* out1 = nullptr;  // SWIGLU_FWD: u; SWIGLU_BWD: dU
+  void* out2 = nullptr;  // SWIGLU_FWD: h
+  int64_t ldo = 0;
+  const void* in0 = nullptr;  // SWIGLU_BWD: g
+  const void* in1 = nullptr;  // SWIGLU_BWD: u
+  int64_t ldi = 0;
+};
+
+slora_status gemm_tc(const TcGemm& g, cudaStream_t st);
+
+// Device error flag of the tcgen05 kernels (a bounded wait that expired).
+slora_status tc_check_error(bool clear);
+
+// Number of SMs of the current device (cached).
+int num_sms();
+
+}  // namespace slora

@@ -12,7 +12,9 @@
 
 #include "estimator.cuh"
 #include "gemm.cuh"
+#include "gemm_tc.cuh"
 #include "linear_ops.cuh"
+#include "lora_pack.cuh"
 #include "swiglu.cuh"
 
 namespace slora {
@@ -166,10 +168,239 @@ slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const 
   }
 }
 
+
+// ------------------------------------------------------- FFN, bf16, tcgen05
+// The eight large contractions (gate|up forward, down forward, dh backward,
+// dX backward; each once for the context rows on the selected channels and
+// once for the dense output rows) run on the tcgen05 kernel with the selected
+// slices gathered in place; the rank-r LoRA projections and the LoRA
+// gradients (HBM-bound, N or M = r) run on the CUDA-core GEMM.
+namespace {
+TcMat mat(const void* p, int64_t rows, int64_t cols, int64_t ld) {
+  TcMat m;
+  m.ptr = p; m.rows = rows; m.cols = cols; m.ld = ld;
+  return m;
+}
+struct TcBuilder {
+  TcGemm g;
+  TcBuilder(const int4* tiles, int64_t ntiles, int a_compact, int out_compact, int64_t M,
+            int64_t N, int paired, int epi) {
+    g.tiles = tiles; g.n_mtiles = int(ntiles); g.a_compact = a_compact;
+    g.out_compact = out_compact; g.M = M; g.N = N; g.paired = paired; g.epi = epi;
+  }
+  TcBuilder& seg(TcMat a, TcMat b0, int bmode, int64_t K, const int32_t* idx = nullptr,
+                 int64_t nidx = 0, int bpair = 0, TcMat b1 = TcMat()) {
+    if (K <= 0) return *this;  // an empty slice contributes nothing
+    TcSeg& s = g.seg[g.nseg++];
+    s.a = a; s.b0 = b0; s.b1 = b1; s.bmode = bmode; s.bpair = bpair; s.idx = idx;
+    s.nidx = nidx; s.K = K;
+    return *this;
+  }
+  TcBuilder& out(void* o0, void* o1, void* o2, int64_t ldo) {
+    g.out0 = o0; g.out1 = o1; g.out2 = o2; g.ldo = ldo;
+    return *this;
+  }
+  TcBuilder& in(const void* i0, const void* i1, int64_t ldi) {
+    g.in0 = i0; g.in1 = i1; g.ldi = ldi;
+    return *this;
+  }
+};
+}  // namespace
+
+slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X,
+                        const void* dOut, void* out, void* dX, int32_t* idx,
+                        const int32_t* idx_force, Arena& ar, bool plan, cudaStream_t st) {
+  const TokenInfo& ti = F.ti;
+  const slora_ffn_layer& L = F.L;
+  const slora_ffn_grads& G = F.G;
+  const int dt = kBF16, r = L.r_lora;
+  const int64_t d = L.d, Fd = L.d_ff, kk = F.kkeep, TC = ti.T_C, TO = ti.T_O, T = ti.T;
+  const float s = L.lora_scale;
+  const int64_t ldk = round8(std::max<int64_t>(kk, 1)), lr = round8(r), lr2 = round8(2 * r);
+  const int64_t nct = count_tiles(tok, true), nott = count_tiles(tok, false);
+  const int64_t nntC = (kk + 127) / 128, nntO = (Fd + 127) / 128;
+  auto bf = [&](int64_t rows, int64_t cols) {
+    return static_cast<void*>(
+        ar.take<__nv_bfloat16>(size_t(std::max<int64_t>(rows * cols, 1))));
+  };
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TC, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TO, 1)));
+  int4* ctiles = ar.take<int4>(size_t(std::max<int64_t>(nct, 1)));
+  int4* otiles = ar.take<int4>(size_t(std::max<int64_t>(nott, 1)));
+  float* XA = ar.take<float>(size_t(T) * 2 * r);
+  void* XAb = bf(T, lr2);
+  float* hA = ar.take<float>(size_t(T) * r);
+  void* hAbC = bf(TC, lr);
+  void* hAbO = bf(TO, lr);
+  float* dOB = ar.take<float>(size_t(T) * r);
+  void* dOBb = bf(T, lr);
+  float* dGB = ar.take<float>(size_t(T) * 2 * r);
+  void* dGBbC = bf(TC, lr2);
+  void* dGBbO = bf(TO, lr2);
+  void* BpC = bf(nntC * 256, lr2);
+  void* BpO = bf(nntO * 256, lr2);
+  void* Adt = bf(Fd, lr);
+  void* Bdp = bf(d, lr);
+  void* AgAu = bf(2 * r, d);
+  void* gC = bf(TC, ldk);
+  void* uC = bf(TC, ldk);
+  void* hC = bf(TC, ldk);
+  void* dGC = bf(TC, ldk);
+  void* dUC = bf(TC, ldk);
+  void* gO = bf(TO, Fd);
+  void* uO = bf(TO, Fd);
+  void* hO = bf(TO, Fd);
+  void* dGO = bf(TO, Fd);
+  void* dUO = bf(TO, Fd);
+  if (!idx_force)
+    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
+                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
+                                   true, nullptr));
+  if (plan) return SLORA_OK;
+
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  if (idx_force) {
+    if (kk > 0)
+      SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
+                                 cudaMemcpyDeviceToDevice, st));
+  } else {
+    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
+                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
+                                   false, st));
+  }
+  // LoRA operand packing (bf16, tiny)
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, st));
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, st));
+  SLORA_TRY(transpose_rows(L.Ad, r, Fd, lr, Adt, st));
+  SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
+  SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
+
+  // ---- forward
+  for (int p = 0; p < 2; ++p) {  // XA = X [Ag; Au]^T (fp32) and s*XA (bf16 operand)
+    GemmArgs g = mk(T, r, with_bf16_copy(out_rowmajor(XA + p * r, kF32, 2 * r),
+                                         static_cast<__nv_bfloat16*>(XAb) + p * r, lr2, s));
+    add(g, rowmajor(X, dt, d), rowmajor(p ? L.Au : L.Ag, dt, d), d);
+    SLORA_TRY(gemm_simt(g, st));
+  }
+  {  // gate|up, context rows, channels S: g, u, h = silu(g) u
+    TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
+    b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K_GATHER, d, idx, kk, 1, mat(L.Wu, Fd, d, d))
+        .seg(mat(XAb, T, 2 * r, lr2), mat(BpC, nntC * 256, 2 * r, lr2), B_K, 2 * r)
+        .out(gC, uC, hC, ldk);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // gate|up, output rows, every channel
+    TcBuilder b(otiles, nott, 0, 1, TO, Fd, 1, EPI_SWIGLU_FWD);
+    b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K, d, nullptr, 0, 1, mat(L.Wu, Fd, d, d))
+        .seg(mat(XAb, T, 2 * r, lr2), mat(BpO, nntO * 256, 2 * r, lr2), B_K, 2 * r)
+        .out(gO, uO, hO, Fd);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // hA = h Ad^T on the channels used (fp32, full rows) and s*hA (bf16, compact)
+    GemmArgs ac = mk(TC, r, with_bf16_copy(out_rowmajor(hA, kF32, r, ctx_rows), hAbC, lr, s));
+    add(ac, rowmajor(hC, dt, ldk), rowmajor(L.Ad, dt, Fd, nullptr, idx), kk);
+    SLORA_TRY(gemm_simt(ac, st));
+    GemmArgs ao = mk(TO, r, with_bf16_copy(out_rowmajor(hA, kF32, r, out_rows), hAbO, lr, s));
+    add(ao, rowmajor(hO, dt, Fd), rowmajor(L.Ad, dt, Fd), Fd);
+    SLORA_TRY(gemm_simt(ao, st));
+  }
+  {  // down projection, context rows: reads channels S only (rows S of Wd^T)
+    TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
+    b.seg(mat(hC, TC, kk, ldk), mat(L.Wd_t, Fd, d, d), B_MN_GATHER, kk, idx, kk)
+        .seg(mat(hAbC, TC, r, lr), mat(Bdp, d, r, lr), B_K, r)
+        .out(out, nullptr, nullptr, d);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // down projection, output rows, dense
+    TcBuilder b(otiles, nott, 1, 0, TO, d, 0, EPI_STORE);
+    b.seg(mat(hO, TO, Fd, Fd), mat(L.Wd_t, Fd, d, d), B_MN, Fd)
+        .seg(mat(hAbO, TO, r, lr), mat(Bdp, d, r, lr), B_K, r)
+        .out(out, nullptr, nullptr, d);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+
+  // ---- backward
+  {
+    GemmArgs g = mk(T, r, with_bf16_copy(out_rowmajor(dOB, kF32, r), dOBb, lr, s));  // dOut Bd
+    add(g, rowmajor(dOut, dt, d), colmajor(L.Bd, dt, r), d);
+    SLORA_TRY(gemm_simt(g, st));
+  }
+  {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
+    TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
+    b.seg(mat(dOut, T, d, d), mat(L.Wd_t, Fd, d, d), B_K_GATHER, d, idx, kk)
+        .seg(mat(dOBb, T, r, lr), mat(Adt, Fd, r, lr), B_K_GATHER, r, idx, kk)
+        .out(dGC, dUC, nullptr, ldk)
+        .in(gC, uC, ldk);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {
+    TcBuilder b(otiles, nott, 0, 1, TO, Fd, 0, EPI_SWIGLU_BWD);
+    b.seg(mat(dOut, T, d, d), mat(L.Wd_t, Fd, d, d), B_K, d)
+        .seg(mat(dOBb, T, r, lr), mat(Adt, Fd, r, lr), B_K, r)
+        .out(dGO, dUO, nullptr, Fd)
+        .in(gO, uO, Fd);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // LoRA grads of the down projection (CUDA cores, fp32)
+    GemmArgs a0 = mk(r, Fd, out_rowmajor(G.dAd, kF32, Fd));
+    add(a0, colmajor(dOB, kF32, r, nullptr, out_rows), colmajor(hO, dt, Fd), TO, s);
+    SLORA_TRY(gemm_simt(a0, st));
+    GemmArgs a1 = mk(r, kk, out_rowmajor(G.dAd, kF32, Fd, nullptr, idx, 1));
+    add(a1, colmajor(dOB, kF32, r, nullptr, ctx_rows), colmajor(hC, dt, ldk), TC, s);
+    SLORA_TRY(gemm_simt(a1, st));
+    GemmArgs b = mk(d, r, out_rowmajor(G.dBd, kF32, r));
+    add(b, colmajor(dOut, dt, d), colmajor(hA, kF32, r), T, s);
+    SLORA_TRY(gemm_simt(b, st));
+  }
+  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu] (fp32 full rows, s* bf16 compact)
+    const void* Bm = p ? L.Bu : L.Bg;
+    GemmArgs bc = mk(TC, r, with_bf16_copy(out_rowmajor(dGB + p * r, kF32, 2 * r, ctx_rows),
+                                           static_cast<__nv_bfloat16*>(dGBbC) + p * r, lr2, s));
+    add(bc, rowmajor(p ? dUC : dGC, dt, ldk), colmajor(Bm, dt, r, nullptr, idx), kk);
+    SLORA_TRY(gemm_simt(bc, st));
+    GemmArgs bo = mk(TO, r, with_bf16_copy(out_rowmajor(dGB + p * r, kF32, 2 * r, out_rows),
+                                           static_cast<__nv_bfloat16*>(dGBbO) + p * r, lr2, s));
+    add(bo, rowmajor(p ? dUO : dGO, dt, Fd), colmajor(Bm, dt, r), Fd);
+    SLORA_TRY(gemm_simt(bo, st));
+  }
+  {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
+    TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
+    b.seg(mat(dGC, TC, kk, ldk), mat(L.Wg, Fd, d, d), B_MN_GATHER, kk, idx, kk)
+        .seg(mat(dUC, TC, kk, ldk), mat(L.Wu, Fd, d, d), B_MN_GATHER, kk, idx, kk)
+        .seg(mat(dGBbC, TC, 2 * r, lr2), mat(AgAu, 2 * r, d, d), B_MN, 2 * r)
+        .out(dX, nullptr, nullptr, d);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // dX, output rows, dense
+    TcBuilder b(otiles, nott, 1, 0, TO, d, 0, EPI_STORE);
+    b.seg(mat(dGO, TO, Fd, Fd), mat(L.Wg, Fd, d, d), B_MN, Fd)
+        .seg(mat(dUO, TO, Fd, Fd), mat(L.Wu, Fd, d, d), B_MN, Fd)
+        .seg(mat(dGBbO, TO, 2 * r, lr2), mat(AgAu, 2 * r, d, d), B_MN, 2 * r)
+        .out(dX, nullptr, nullptr, d);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  for (int p = 0; p < 2; ++p) {  // LoRA grads of gate / up (CUDA cores, fp32)
+    GemmArgs a = mk(r, d, out_rowmajor(p ? G.dAu : G.dAg, kF32, d));
+    add(a, colmajor(dGB + p * r, kF32, 2 * r), colmajor(X, dt, d), T, s);
+    SLORA_TRY(gemm_simt(a, st));
+    float* dBm = p ? G.dBu : G.dBg;
+    GemmArgs b0 = mk(Fd, r, out_rowmajor(dBm, kF32, r));
+    add(b0, colmajor(p ? dUO : dGO, dt, Fd), colmajor(XA + p * r, kF32, 2 * r, nullptr, out_rows),
+        TO, s);
+    SLORA_TRY(gemm_simt(b0, st));
+    GemmArgs b1 = mk(kk, r, out_rowmajor(dBm, kF32, r, idx, nullptr, 1));
+    add(b1, colmajor(p ? dUC : dGC, dt, ldk), colmajor(XA + p * r, kF32, 2 * r, nullptr, ctx_rows),
+        TC, s);
+    SLORA_TRY(gemm_simt(b1, st));
+  }
+  return SLORA_OK;
+}
+
 // ---------------------------------------------------------------------- FFN
 slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
                      void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
                      bool plan, cudaStream_t st) {
+  if (F.dt == kBF16) return ffn_run_tc(F, tok, X, dOut, out, dX, idx, idx_force, ar, plan, st);
   const TokenInfo& ti = F.ti;
   const slora_ffn_layer& L = F.L;
   const slora_ffn_grads& G = F.G;

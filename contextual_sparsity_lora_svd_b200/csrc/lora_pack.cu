@@ -1,0 +1,104 @@
+// Small per-step packing of the LoRA factors into the operand layouts the
+// tcgen05 GEMM reads (all bf16, a few hundred KB per step):
+//   pack_gate_up_b : for every 256-row N tile of the paired gate|up GEMM, rows
+//                    0..127 = [B_g[c] | 0] and rows 128..255 = [0 | B_u[c]] for
+//                    the tile's 128 channels c (idx[c] when sliced), so the
+//                    LoRA up-projection of both halves is one K = 2r segment
+//   transpose_rows : out[c][q] = in[q][c]     (A_d^T, rows = channels)
+//   stack_rows     : out = [top; bottom]      ([A_g; A_u], MN-major operand)
+#include "lora_pack.cuh"
+
+namespace slora {
+namespace {
+
+__global__ void pack_gate_up_b_kernel(const __nv_bfloat16* __restrict__ Bg,
+                                      const __nv_bfloat16* __restrict__ Bu,
+                                      const int32_t* __restrict__ idx, int64_t N, int r,
+                                      int64_t rows, int64_t ldo, __nv_bfloat16* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= rows * ldo) return;
+  const int64_t R = e / ldo;
+  const int col = int(e % ldo);
+  const int64_t nt = R / 256;
+  const int h = int((R % 256) / 128);
+  const int64_t c = nt * 128 + (R % 128);
+  float v = 0.0f;
+  if (c < N && col >= h * r && col < (h + 1) * r) {
+    const int64_t src = idx ? idx[c] : c;
+    v = __bfloat162float((h ? Bu : Bg)[src * r + (col - h * r)]);
+  }
+  out[e] = __float2bfloat16_rn(v);
+}
+
+__global__ void transpose_rows_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows,
+                                      int64_t cols, int64_t ldo, __nv_bfloat16* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= cols * ldo) return;
+  const int64_t c = e / ldo, q = e % ldo;
+  out[e] = q < rows ? in[q * cols + c] : __float2bfloat16_rn(0.0f);
+}
+
+__global__ void stack_rows_kernel(const __nv_bfloat16* __restrict__ top,
+                                  const __nv_bfloat16* __restrict__ bottom, int64_t rows_top,
+                                  int64_t rows_bottom, int64_t cols,
+                                  __nv_bfloat16* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = (rows_top + rows_bottom) * cols;
+  if (e >= total) return;
+  const int64_t rr = e / cols, c = e % cols;
+  out[e] = rr < rows_top ? top[rr * cols + c] : bottom[(rr - rows_top) * cols + c];
+}
+
+__global__ void copy_pad_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows, int64_t cols,
+                                int64_t ldo, __nv_bfloat16* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= rows * ldo) return;
+  const int64_t rr = e / ldo, c = e % ldo;
+  out[e] = c < cols ? in[rr * cols + c] : __float2bfloat16_rn(0.0f);
+}
+
+unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
+
+}  // namespace
+
+slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, int64_t N, int r,
+                            int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st) {
+  const int64_t rows = n_ntiles * 256;
+  if (rows <= 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(rows) * ldo * 2 + double(N) * 2 * r * 2, st);
+  pack_gate_up_b_kernel<<<blocks(rows * ldo), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(Bg), static_cast<const __nv_bfloat16*>(Bu), idx, N, r,
+      rows, ldo, static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, int64_t ldo, void* out,
+                            cudaStream_t st) {
+  LaunchScope ls(kAux, double(rows) * cols * 2 + double(cols) * ldo * 2, st);
+  transpose_rows_kernel<<<blocks(cols * ldo), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(in), rows, cols, ldo, static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
+                        int64_t rows_bottom, int64_t cols, void* out, cudaStream_t st) {
+  LaunchScope ls(kAux, 4.0 * double(rows_top + rows_bottom) * cols, st);
+  stack_rows_kernel<<<blocks((rows_top + rows_bottom) * cols), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(top), static_cast<const __nv_bfloat16*>(bottom), rows_top,
+      rows_bottom, cols, static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status copy_pad(const void* in, int64_t rows, int64_t cols, int64_t ldo, void* out,
+                      cudaStream_t st) {
+  LaunchScope ls(kAux, double(rows) * (cols + ldo) * 2, st);
+  copy_pad_kernel<<<blocks(rows * ldo), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), rows,
+                                                      cols, ldo, static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+}  // namespace slora

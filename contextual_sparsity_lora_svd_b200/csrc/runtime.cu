@@ -15,16 +15,24 @@ struct RowmapParams {
 };
 
 // One block: scan ctx_len into per-sequence offsets, then every row t of the
-// full layout lands in ctx_rows or out_rows at its compact position.
+// full layout lands in ctx_rows or out_rows at its compact position, and every
+// sequence emits its context and output M tiles.
 __global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
                                                       int32_t* __restrict__ ctx_rows,
-                                                      int32_t* __restrict__ out_rows) {
-  __shared__ int ctx_off[kMaxBatch];
+                                                      int32_t* __restrict__ out_rows,
+                                                      int4* __restrict__ ctx_tiles,
+                                                      int4* __restrict__ out_tiles) {
+  __shared__ int ctx_off[kMaxBatch], ct_off[kMaxBatch], ot_off[kMaxBatch];
   if (threadIdx.x == 0) {
-    int acc = 0;
+    int acc = 0, ct = 0, ot = 0;
     for (int b = 0; b < p.batch; ++b) {
       ctx_off[b] = acc;
-      acc += p.ctx_len[b];
+      ct_off[b] = ct;
+      ot_off[b] = ot;
+      const int c = p.ctx_len[b];
+      acc += c;
+      ct += (c + 127) / 128;
+      ot += (p.seq - c + 127) / 128;
     }
   }
   __syncthreads();
@@ -38,6 +46,19 @@ __global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
       // output rows before sequence b: b*seq - ctx_off[b]
       if (out_rows) out_rows[int64_t(b) * p.seq - ctx_off[b] + (i - c)] = int32_t(t);
     }
+  }
+  for (int b = threadIdx.x; b < p.batch; b += blockDim.x) {
+    const int c = p.ctx_len[b];
+    const int full0 = b * p.seq;
+    if (ctx_tiles)
+      for (int j = 0; j * 128 < c; ++j)
+        ctx_tiles[ct_off[b] + j] = make_int4(full0 + 128 * j, ctx_off[b] + 128 * j,
+                                             min(128, c - 128 * j), 0);
+    const int o0 = b * p.seq - ctx_off[b];
+    if (out_tiles)
+      for (int j = 0; j * 128 < p.seq - c; ++j)
+        out_tiles[ot_off[b] + j] = make_int4(full0 + c + 128 * j, o0 + 128 * j,
+                                             min(128, p.seq - c - 128 * j), 0);
   }
 }
 }  // namespace
@@ -88,14 +109,24 @@ slora_status parse_tokens(const slora_tokens* tok, TokenInfo* ti) {
   return SLORA_OK;
 }
 
+int64_t count_tiles(const slora_tokens* tok, bool ctx) {
+  int64_t n = 0;
+  for (int b = 0; b < tok->batch; ++b) {
+    const int c = tok->ctx_len[b];
+    n += ctx ? (c + 127) / 128 : (tok->seq - c + 127) / 128;
+  }
+  return n;
+}
+
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
-                            int32_t* out_rows, cudaStream_t st) {
+                            int32_t* out_rows, cudaStream_t st, int4* ctx_tiles,
+                            int4* out_tiles) {
   RowmapParams p;
   p.batch = ti.batch;
   p.seq = ti.seq;
   for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
   LaunchScope ls(kAux, double(ti.T) * 4, st);
-  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows);
+  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
