@@ -283,6 +283,8 @@ def run_ours(args, rank, world):
           for _ in range(args.steps)]
     L.profile_enable(True)
     n0 = L.launch_count()
+    if args.profile_region:
+        torch.cuda.profiler.start()
     with ClockSampler(dev) as clk:
         for i in range(args.steps):
             flush.zero_()
@@ -290,6 +292,8 @@ def run_ours(args, rank, world):
             one_step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+    if args.profile_region:
+        torch.cuda.profiler.stop()
     launches = L.launch_count() - n0
     prof = {c: L.profile_read(c) for c in L.KERNEL_CLASSES}
     L.profile_enable(False)
@@ -376,6 +380,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-region", action="store_true",
+                    help="bracket the timed steps with cudaProfilerStart/Stop (for ncu "
+                         "--profile-from-start off)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
