@@ -120,7 +120,8 @@ def profile_read(kernel_class: str) -> tuple[int, float, float]:
     return int(n.value), float(ms.value), float(w.value)
 
 
-KERNEL_CLASSES = ["gemm_tc", "gemm_simt", "estimate", "select", "elementwise", "aux", "prepare"]
+KERNEL_CLASSES = ["gemm_tc", "gemm_simt", "estimate", "select", "elementwise", "aux", "prepare",
+                  "skinny", "compact"]
 
 
 def ptr(x) -> int | None:

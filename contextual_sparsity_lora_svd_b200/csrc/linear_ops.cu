@@ -15,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "linear_ops.cuh"
 #include "lora_pack.cuh"
+#include "skinny.cuh"
 #include "swiglu.cuh"
 
 namespace slora {
@@ -239,9 +240,13 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   void* dGBbO = bf(TO, lr2);
   void* BpC = bf(nntC * 256, lr2);
   void* BpO = bf(nntO * 256, lr2);
+  void* AdtS = bf(kk, lr);
   void* Adt = bf(Fd, lr);
   void* Bdp = bf(d, lr);
   void* AgAu = bf(2 * r, d);
+  void* WgS = bf(kk, d);  // selected rows of the frozen weights, compacted once per step
+  void* WuS = bf(kk, d);
+  void* WdS = bf(kk, d);  // rows S of Wd^T
   void* gC = bf(TC, ldk);
   void* uC = bf(TC, ldk);
   void* hC = bf(TC, ldk);
@@ -252,6 +257,14 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   void* hO = bf(TO, Fd);
   void* dGO = bf(TO, Fd);
   void* dUO = bf(TO, Fd);
+  // partial sums of the skinny contractions (reused sequentially)
+  int64_t npart = 1;
+  for (int64_t M : {T, TC, TO})
+    for (int64_t K : {d, kk, Fd}) {
+      npart = std::max(npart, rowdot_part_floats(M, K, 2 * r));
+      npart = std::max(npart, coldot_part_floats(M, K, 2 * r));
+    }
+  float* part = ar.take<float>(size_t(npart));
   if (!idx_force)
     SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
                                    L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
@@ -268,23 +281,34 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
                                    L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
                                    false, st));
   }
+  // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
+  SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st));
+  SLORA_TRY(gather_rows(L.Wu, d, idx, kk, d, WuS, d, st));
+  SLORA_TRY(gather_rows(L.Wd_t, d, idx, kk, d, WdS, d, st));
   // LoRA operand packing (bf16, tiny)
   SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, st));
   SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, st));
-  SLORA_TRY(transpose_rows(L.Ad, r, Fd, lr, Adt, st));
+  SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, st));
+  SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, st));
   SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
   SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
 
+  auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
+    SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
+  };
+  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
+    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
+  };
+
   // ---- forward
-  for (int p = 0; p < 2; ++p) {  // XA = X [Ag; Au]^T (fp32) and s*XA (bf16 operand)
-    GemmArgs g = mk(T, r, with_bf16_copy(out_rowmajor(XA + p * r, kF32, 2 * r),
-                                         static_cast<__nv_bfloat16*>(XAb) + p * r, lr2, s));
-    add(g, rowmajor(X, dt, d), rowmajor(p ? L.Au : L.Ag, dt, d), d);
-    SLORA_TRY(gemm_simt(g, st));
+  {  // XA = X [Ag; Au]^T: fp32 (gradients) and s*XA in bf16 (GEMM operand)
+    SkRowOut o;
+    o.out1 = XA; o.ld1 = 2 * r; o.out2 = XAb; o.ld2 = lr2; o.s2 = s;
+    SLORA_TRY(rowdot(Yv(X, d), T, d, Rv(AgAu, kBF16, 1, d), 2 * r, o, part, st));
   }
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
-    b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K_GATHER, d, idx, kk, 1, mat(L.Wu, Fd, d, d))
+    b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, nullptr, 0, 1, mat(WuS, kk, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpC, nntC * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gC, uC, hC, ldk);
     SLORA_TRY(gemm_tc(b.g, st));
@@ -296,17 +320,17 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .out(gO, uO, hO, Fd);
     SLORA_TRY(gemm_tc(b.g, st));
   }
-  {  // hA = h Ad^T on the channels used (fp32, full rows) and s*hA (bf16, compact)
-    GemmArgs ac = mk(TC, r, with_bf16_copy(out_rowmajor(hA, kF32, r, ctx_rows), hAbC, lr, s));
-    add(ac, rowmajor(hC, dt, ldk), rowmajor(L.Ad, dt, Fd, nullptr, idx), kk);
-    SLORA_TRY(gemm_simt(ac, st));
-    GemmArgs ao = mk(TO, r, with_bf16_copy(out_rowmajor(hA, kF32, r, out_rows), hAbO, lr, s));
-    add(ao, rowmajor(hO, dt, Fd), rowmajor(L.Ad, dt, Fd), Fd);
-    SLORA_TRY(gemm_simt(ao, st));
+  {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
+    SkRowOut oc;
+    oc.out1 = hA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = hAbC; oc.ld2 = lr; oc.s2 = s;
+    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, part, st));
+    SkRowOut oo;
+    oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
+    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, part, st));
   }
   {  // down projection, context rows: reads channels S only (rows S of Wd^T)
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
-    b.seg(mat(hC, TC, kk, ldk), mat(L.Wd_t, Fd, d, d), B_MN_GATHER, kk, idx, kk)
+    b.seg(mat(hC, TC, kk, ldk), mat(WdS, kk, d, d), B_MN, kk)
         .seg(mat(hAbC, TC, r, lr), mat(Bdp, d, r, lr), B_K, r)
         .out(out, nullptr, nullptr, d);
     SLORA_TRY(gemm_tc(b.g, st));
@@ -320,15 +344,18 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   }
 
   // ---- backward
-  {
-    GemmArgs g = mk(T, r, with_bf16_copy(out_rowmajor(dOB, kF32, r), dOBb, lr, s));  // dOut Bd
-    add(g, rowmajor(dOut, dt, d), colmajor(L.Bd, dt, r), d);
-    SLORA_TRY(gemm_simt(g, st));
+  {  // dOB = dOut Bd: fp32 and s*dOB bf16; dBd = s dOut^T hA (same stream of dOut)
+    SkRowOut o;
+    o.out1 = dOB; o.ld1 = r; o.out2 = dOBb; o.ld2 = lr; o.s2 = s;
+    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, part, st));
+    SkColOut c;
+    c.out = G.dBd; c.ldo = r; c.scale = s;
+    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, part, st));
   }
   {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
-    b.seg(mat(dOut, T, d, d), mat(L.Wd_t, Fd, d, d), B_K_GATHER, d, idx, kk)
-        .seg(mat(dOBb, T, r, lr), mat(Adt, Fd, r, lr), B_K_GATHER, r, idx, kk)
+    b.seg(mat(dOut, T, d, d), mat(WdS, kk, d, d), B_K, d)
+        .seg(mat(dOBb, T, r, lr), mat(AdtS, kk, r, lr), B_K, r)
         .out(dGC, dUC, nullptr, ldk)
         .in(gC, uC, ldk);
     SLORA_TRY(gemm_tc(b.g, st));
@@ -341,32 +368,37 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .in(gO, uO, Fd);
     SLORA_TRY(gemm_tc(b.g, st));
   }
-  {  // LoRA grads of the down projection (CUDA cores, fp32)
-    GemmArgs a0 = mk(r, Fd, out_rowmajor(G.dAd, kF32, Fd));
-    add(a0, colmajor(dOB, kF32, r, nullptr, out_rows), colmajor(hO, dt, Fd), TO, s);
-    SLORA_TRY(gemm_simt(a0, st));
-    GemmArgs a1 = mk(r, kk, out_rowmajor(G.dAd, kF32, Fd, nullptr, idx, 1));
-    add(a1, colmajor(dOB, kF32, r, nullptr, ctx_rows), colmajor(hC, dt, ldk), TC, s);
-    SLORA_TRY(gemm_simt(a1, st));
-    GemmArgs b = mk(d, r, out_rowmajor(G.dBd, kF32, r));
-    add(b, colmajor(dOut, dt, d), colmajor(hA, kF32, r), T, s);
-    SLORA_TRY(gemm_simt(b, st));
+  {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
+    SkColOut co;
+    co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
+    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, part, st));
+    SkColOut cc = co;
+    cc.kmap = idx; cc.accumulate = 1;
+    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, part, st));
   }
-  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu] (fp32 full rows, s* bf16 compact)
+  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]; dB = s dG^T XA on the same stream
     const void* Bm = p ? L.Bu : L.Bg;
-    GemmArgs bc = mk(TC, r, with_bf16_copy(out_rowmajor(dGB + p * r, kF32, 2 * r, ctx_rows),
-                                           static_cast<__nv_bfloat16*>(dGBbC) + p * r, lr2, s));
-    add(bc, rowmajor(p ? dUC : dGC, dt, ldk), colmajor(Bm, dt, r, nullptr, idx), kk);
-    SLORA_TRY(gemm_simt(bc, st));
-    GemmArgs bo = mk(TO, r, with_bf16_copy(out_rowmajor(dGB + p * r, kF32, 2 * r, out_rows),
-                                           static_cast<__nv_bfloat16*>(dGBbO) + p * r, lr2, s));
-    add(bo, rowmajor(p ? dUO : dGO, dt, Fd), colmajor(Bm, dt, r), Fd);
-    SLORA_TRY(gemm_simt(bo, st));
+    float* dBm = p ? G.dBu : G.dBg;
+    SkRowOut oo;
+    oo.out1 = dGB; oo.ld1 = 2 * r; oo.off1 = p * r; oo.map1 = out_rows;
+    oo.out2 = dGBbO; oo.ld2 = lr2; oo.off2 = p * r; oo.s2 = s;
+    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, part, st));
+    SkColOut bo;
+    bo.out = dBm; bo.ldo = r; bo.scale = s;
+    SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
+                     bo, part, st));
+    SkRowOut oc = oo;
+    oc.map1 = ctx_rows; oc.out2 = dGBbC;
+    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, part, st));
+    SkColOut bc = bo;
+    bc.kmap = idx; bc.accumulate = 1;
+    SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
+                     bc, part, st));
   }
   {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
-    b.seg(mat(dGC, TC, kk, ldk), mat(L.Wg, Fd, d, d), B_MN_GATHER, kk, idx, kk)
-        .seg(mat(dUC, TC, kk, ldk), mat(L.Wu, Fd, d, d), B_MN_GATHER, kk, idx, kk)
+    b.seg(mat(dGC, TC, kk, ldk), mat(WgS, kk, d, d), B_MN, kk)
+        .seg(mat(dUC, TC, kk, ldk), mat(WuS, kk, d, d), B_MN, kk)
         .seg(mat(dGBbC, TC, 2 * r, lr2), mat(AgAu, 2 * r, d, d), B_MN, 2 * r)
         .out(dX, nullptr, nullptr, d);
     SLORA_TRY(gemm_tc(b.g, st));
@@ -379,19 +411,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .out(dX, nullptr, nullptr, d);
     SLORA_TRY(gemm_tc(b.g, st));
   }
-  for (int p = 0; p < 2; ++p) {  // LoRA grads of gate / up (CUDA cores, fp32)
-    GemmArgs a = mk(r, d, out_rowmajor(p ? G.dAu : G.dAg, kF32, d));
-    add(a, colmajor(dGB + p * r, kF32, 2 * r), colmajor(X, dt, d), T, s);
-    SLORA_TRY(gemm_simt(a, st));
-    float* dBm = p ? G.dBu : G.dBg;
-    GemmArgs b0 = mk(Fd, r, out_rowmajor(dBm, kF32, r));
-    add(b0, colmajor(p ? dUO : dGO, dt, Fd), colmajor(XA + p * r, kF32, 2 * r, nullptr, out_rows),
-        TO, s);
-    SLORA_TRY(gemm_simt(b0, st));
-    GemmArgs b1 = mk(kk, r, out_rowmajor(dBm, kF32, r, idx, nullptr, 1));
-    add(b1, colmajor(p ? dUC : dGC, dt, ldk), colmajor(XA + p * r, kF32, 2 * r, nullptr, ctx_rows),
-        TC, s);
-    SLORA_TRY(gemm_simt(b1, st));
+  {  // dAg | dAu = s dGB^T X over every row, one stream of X
+    SkColOut c;
+    c.out = G.dAg; c.out_b = G.dAu; c.qsplit = r; c.ldo = d; c.trans = 1; c.scale = s;
+    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, part, st));
   }
   return SLORA_OK;
 }

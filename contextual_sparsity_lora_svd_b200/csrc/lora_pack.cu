@@ -31,11 +31,24 @@ __global__ void pack_gate_up_b_kernel(const __nv_bfloat16* __restrict__ Bg,
 }
 
 __global__ void transpose_rows_kernel(const __nv_bfloat16* __restrict__ in, int64_t rows,
-                                      int64_t cols, int64_t ldo, __nv_bfloat16* __restrict__ out) {
+                                      int64_t cols, const int32_t* __restrict__ idx, int64_t n,
+                                      int64_t ldo, __nv_bfloat16* __restrict__ out) {
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= cols * ldo) return;
+  if (e >= n * ldo) return;
   const int64_t c = e / ldo, q = e % ldo;
-  out[e] = q < rows ? in[q * cols + c] : __float2bfloat16_rn(0.0f);
+  const int64_t src = idx ? int64_t(idx[c]) : c;
+  out[e] = q < rows ? in[q * cols + src] : __float2bfloat16_rn(0.0f);
+}
+
+// One block per selected row and 2048-element column chunk; 16-byte copies.
+__global__ void gather_rows_kernel(const uint4* __restrict__ in, int64_t ld_in16,
+                                   const int32_t* __restrict__ idx, int64_t cols16,
+                                   uint4* __restrict__ out, int64_t ld_out16) {
+  const int64_t j = blockIdx.x;
+  const int64_t src = idx[j];
+  for (int64_t c = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; c < cols16;
+       c += int64_t(gridDim.y) * blockDim.x)
+    out[j * ld_out16 + c] = __ldg(in + src * ld_in16 + c);
 }
 
 __global__ void stack_rows_kernel(const __nv_bfloat16* __restrict__ top,
@@ -73,11 +86,28 @@ slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, 
   return SLORA_OK;
 }
 
-slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, int64_t ldo, void* out,
-                            cudaStream_t st) {
-  LaunchScope ls(kAux, double(rows) * cols * 2 + double(cols) * ldo * 2, st);
-  transpose_rows_kernel<<<blocks(cols * ldo), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(in), rows, cols, ldo, static_cast<__nv_bfloat16*>(out));
+slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const int32_t* idx,
+                            int64_t n, int64_t ldo, void* out, cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(rows) * n * 2 + double(n) * ldo * 2, st);
+  transpose_rows_kernel<<<blocks(n * ldo), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(in), rows, cols, idx, n, ldo,
+      static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
+                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  if (cols % 8 || ld_in % 8 || ld_out % 8)
+    SLORA_FAIL(SLORA_ERR_ALIGN, "gather_rows: rows must be whole 16-byte units");
+  const int64_t c16 = cols / 8;
+  const unsigned gy = unsigned((c16 + 255) / 256);
+  if (n > 2147483647) SLORA_FAIL(SLORA_ERR_SHAPE, "gather_rows: too many rows");
+  LaunchScope ls(kCompact, 2.0 * double(n) * cols * 2, st);
+  gather_rows_kernel<<<dim3(unsigned(n), gy), 256, 0, st>>>(
+      static_cast<const uint4*>(in), ld_in / 8, idx, c16, static_cast<uint4*>(out), ld_out / 8);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

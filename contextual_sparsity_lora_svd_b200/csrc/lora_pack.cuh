@@ -6,9 +6,14 @@ namespace slora {
 // [0 | Bu[c]] for channels c = nt*128 + j (idx[c] if idx), zero past N.
 slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, int64_t N, int r,
                             int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st);
-// out [cols x ldo] = in^T (in is rows x cols), zero columns past `rows`.
-slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, int64_t ldo, void* out,
-                            cudaStream_t st);
+// out [n x ldo] with out[c][q] = in[q][idx ? idx[c] : c] (in is rows x cols,
+// n = number of output rows), zero columns past `rows`.
+slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const int32_t* idx,
+                            int64_t n, int64_t ldo, void* out, cudaStream_t st);
+// Compaction of selected rows: out[j][:] = in[idx[j]][:] for j < n (bf16,
+// rows of `cols` elements, cols a multiple of 8, leading dimensions ld_in/ld_out).
+slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
+                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st);
 // out [(rows_top + rows_bottom) x cols] = [top; bottom].
 slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
                         int64_t rows_bottom, int64_t cols, void* out, cudaStream_t st);

@@ -141,7 +141,7 @@ extern "C" int slora_version(void) { return 100; }
 namespace slora {
 namespace {
 const char* kClassNames[kNumClasses] = {"gemm_tc", "gemm_simt", "estimate", "select",
-                                        "elementwise", "aux", "prepare"};
+                                        "elementwise", "aux", "prepare", "skinny", "compact"};
 struct Rec {
   int cls;
   double work;

@@ -1,0 +1,342 @@
+// Skinny (rank-sized) contractions, see skinny.cuh.
+//
+// 128-thread blocks over 64 x 64 tiles of Y staged in shared memory with
+// cp.async (zero-filled past the edges, optional row gather); the rank-sized
+// operand is staged transposed as 1 or 3 bf16 terms.  Each warp owns 16 rows
+// (rowdot) or 16 columns (coldot) of the tile and issues mma.sync m16n8k16
+// (bf16 in, fp32 accumulate).  Many small blocks per SM keep the HBM stream
+// of Y busy; partial sums over the split dimension go to a workspace and a
+// finalize kernel reduces them in a fixed order.
+#include "skinny.cuh"
+
+namespace slora {
+namespace {
+
+constexpr int TILE = 64, PAD = 72, NTH = 128;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3, const void* p) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
+__device__ __forceinline__ uint32_t lds32(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+__device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
+  const int64_t ii = R.map ? R.map[i] : i;
+  const int64_t off = ii * R.si + int64_t(q) * R.sq;
+  if (R.dt == kF32) return static_cast<const float*>(R.ptr)[off];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(R.ptr)[off]);
+}
+
+// Split v into NT bf16 terms whose sum reproduces v to ~2^-8 (NT=1) or ~2^-24 (NT=3).
+template <int NT>
+__device__ __forceinline__ void split_terms(float v, __nv_bfloat16* out) {
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  out[0] = h;
+  if (NT > 1) {
+    float r = v - __bfloat162float(h);
+    __nv_bfloat16 m = __float2bfloat16_rn(r);
+    out[1] = m;
+    r -= __bfloat162float(m);
+    out[2] = __float2bfloat16_rn(r);
+  }
+}
+
+// Stage the 64 x 64 tile of Y at (m0, k0) into Ys (rows m, columns k).
+__device__ __forceinline__ void stage_y(__nv_bfloat16 (*Ys)[PAD], const SkY& Y, int64_t M,
+                                        int64_t K, int64_t m0, int64_t k0, int tid) {
+  const __nv_bfloat16* base = static_cast<const __nv_bfloat16*>(Y.ptr);
+#pragma unroll
+  for (int i = 0; i < (TILE * TILE / 8) / NTH; ++i) {
+    const int seg = tid + NTH * i;
+    const int row = seg >> 3, c8 = (seg & 7) * 8;
+    const int64_t m = m0 + row, k = k0 + c8;
+    int bytes = 0;
+    const __nv_bfloat16* src = base;
+    if (m < M && k < K) {
+      const int64_t left = (K - k) * 2;
+      bytes = left < 16 ? int(left) : 16;
+      src = base + (Y.map ? int64_t(Y.map[m]) : m) * Y.ld + k;
+    }
+    cp_async16(&Ys[row][c8], src, bytes);
+  }
+}
+
+template <int NF, int NT>
+__global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int64_t K,
+                                                     const SkR R, int c, int chunks_per_split,
+                                                     float* __restrict__ part) {
+  constexpr int CP = NF * 8;
+  __shared__ __align__(16) __nv_bfloat16 Ys[TILE][PAD];
+  __shared__ __align__(16) __nv_bfloat16 Rs[NT][CP][PAD];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t m0 = int64_t(blockIdx.x) * TILE;
+  const int ks = blockIdx.y;
+  const int64_t nchunks = (K + TILE - 1) / TILE;
+  const int64_t kc0 = int64_t(ks) * chunks_per_split;
+  const int64_t kc1 = kc0 + chunks_per_split < nchunks ? kc0 + chunks_per_split : nchunks;
+  float acc[NF][4];
+#pragma unroll
+  for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
+  for (int64_t kc = kc0; kc < kc1; ++kc) {
+    const int64_t k0 = kc * TILE;
+    stage_y(Ys, Y, M, K, m0, k0, tid);
+    for (int e = tid; e < CP * TILE; e += NTH) {
+      const int q = e / TILE, kk = e % TILE;
+      const int64_t k = k0 + kk;
+      const float v = (q < c && k < K) ? load_r(R, k, q) : 0.0f;
+      __nv_bfloat16 tv[3];
+      split_terms<NT>(v, tv);
+#pragma unroll
+      for (int s = 0; s < NT; ++s) Rs[s][q][kk] = tv[s];
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    const int r0 = warp * 16 + g;
+#pragma unroll
+    for (int k16 = 0; k16 < TILE / 16; ++k16) {
+      const int kb = k16 * 16 + 2 * t;
+      const uint32_t a0 = lds32(&Ys[r0][kb]), a1 = lds32(&Ys[r0 + 8][kb]);
+      const uint32_t a2 = lds32(&Ys[r0][kb + 8]), a3 = lds32(&Ys[r0 + 8][kb + 8]);
+#pragma unroll
+      for (int f = 0; f < NF; ++f)
+#pragma unroll
+        for (int s = 0; s < NT; ++s)
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[s][f * 8 + g][kb]),
+                   lds32(&Rs[s][f * 8 + g][kb + 8]));
+    }
+    __syncthreads();
+  }
+  const int64_t row0 = m0 + warp * 16 + g;
+#pragma unroll
+  for (int f = 0; f < NF; ++f) {
+    const int col = f * 8 + 2 * t;
+    if (row0 < M) {
+      float* p = part + (int64_t(ks) * M + row0) * CP + col;
+      p[0] = acc[f][0];
+      p[1] = acc[f][1];
+    }
+    if (row0 + 8 < M) {
+      float* p = part + (int64_t(ks) * M + row0 + 8) * CP + col;
+      p[0] = acc[f][2];
+      p[1] = acc[f][3];
+    }
+  }
+}
+
+template <int NF, int NT>
+__global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int64_t K,
+                                                     const SkR R, int c, int chunks_per_split,
+                                                     float* __restrict__ part) {
+  constexpr int CP = NF * 8;
+  __shared__ __align__(16) __nv_bfloat16 Ys[TILE][PAD];
+  __shared__ __align__(16) __nv_bfloat16 Rs[NT][CP][PAD];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t k0 = int64_t(blockIdx.x) * TILE;
+  const int ms = blockIdx.y;
+  const int64_t nchunks = (M + TILE - 1) / TILE;
+  const int64_t mc0 = int64_t(ms) * chunks_per_split;
+  const int64_t mc1 = mc0 + chunks_per_split < nchunks ? mc0 + chunks_per_split : nchunks;
+  float acc[NF][4];
+#pragma unroll
+  for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
+  const int mq = lane >> 3, rr = lane & 7;  // ldmatrix: matrix index, row within it
+  for (int64_t mc = mc0; mc < mc1; ++mc) {
+    const int64_t m0 = mc * TILE;
+    stage_y(Ys, Y, M, K, m0, k0, tid);
+    for (int e = tid; e < CP * TILE; e += NTH) {
+      const int q = e / TILE, mm = e % TILE;
+      const int64_t m = m0 + mm;
+      const float v = (q < c && m < M) ? load_r(R, m, q) : 0.0f;
+      __nv_bfloat16 tv[3];
+      split_terms<NT>(v, tv);
+#pragma unroll
+      for (int s = 0; s < NT; ++s) Rs[s][q][mm] = tv[s];
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int m16 = 0; m16 < TILE / 16; ++m16) {
+      // A = Y^T fragment (16 k x 16 m) for columns warp*16.. of the tile
+      const int mb = m16 * 16 + (mq >> 1) * 8;
+      const int kb = warp * 16 + (mq & 1) * 8;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans(a0, a1, a2, a3, &Ys[mb + rr][kb]);
+      const int mcol = m16 * 16 + 2 * t;
+#pragma unroll
+      for (int f = 0; f < NF; ++f)
+#pragma unroll
+        for (int s = 0; s < NT; ++s)
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[s][f * 8 + g][mcol]),
+                   lds32(&Rs[s][f * 8 + g][mcol + 8]));
+    }
+    __syncthreads();
+  }
+  const int64_t kr = k0 + warp * 16 + g;
+#pragma unroll
+  for (int f = 0; f < NF; ++f) {
+    const int col = f * 8 + 2 * t;
+    if (kr < K) {
+      float* p = part + (int64_t(ms) * K + kr) * CP + col;
+      p[0] = acc[f][0];
+      p[1] = acc[f][1];
+    }
+    if (kr + 8 < K) {
+      float* p = part + (int64_t(ms) * K + kr + 8) * CP + col;
+      p[0] = acc[f][2];
+      p[1] = acc[f][3];
+    }
+  }
+}
+
+__global__ void rowdot_finalize(const float* __restrict__ part, int nsplit, int64_t M, int c,
+                                int CP, const SkRowOut o) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= M * c) return;
+  const int64_t m = e / c;
+  const int q = int(e % c);
+  float v = 0.0f;
+  for (int s = 0; s < nsplit; ++s) v += part[(int64_t(s) * M + m) * CP + q];
+  if (q < o.qsplit) {
+    if (o.out1) o.out1[(o.map1 ? int64_t(o.map1[m]) : m) * o.ld1 + o.off1 + q] = v;
+    if (o.out2)
+      static_cast<__nv_bfloat16*>(o.out2)[(o.map2 ? int64_t(o.map2[m]) : m) * o.ld2 + o.off2 + q] =
+          __float2bfloat16_rn(o.s2 * v);
+  } else if (o.out1b) {
+    o.out1b[(o.map1b ? int64_t(o.map1b[m]) : m) * o.ld1b + o.off1b + (q - o.qsplit)] = v;
+  }
+}
+
+__global__ void coldot_finalize(const float* __restrict__ part, int nsplit, int64_t K, int c,
+                                int CP, const SkColOut o) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= K * c) return;
+  const int64_t k = e / c;
+  const int q = int(e % c);
+  float v = 0.0f;
+  for (int s = 0; s < nsplit; ++s) v += part[(int64_t(s) * K + k) * CP + q];
+  v *= o.scale;
+  const int64_t kk = o.kmap ? int64_t(o.kmap[k]) : k;
+  float* base = q < o.qsplit ? o.out : o.out_b;
+  const int qq = q < o.qsplit ? q : q - o.qsplit;
+  float* dst = base + (o.trans ? int64_t(qq) * o.ldo + kk : kk * o.ldo + qq);
+  *dst = o.accumulate ? *dst + v : v;
+}
+
+constexpr int kTargetBlocks = 148 * 8;
+
+int64_t splits_for(int64_t nblocks, int64_t nchunks) {
+  int64_t s = (kTargetBlocks + nblocks - 1) / nblocks;
+  if (s > nchunks) s = nchunks;
+  if (s < 1) s = 1;
+  if (s > 64) s = 64;
+  return s;
+}
+
+int padded(int c) { return ((c + 15) / 16) * 16; }  // NF even keeps the templates few
+
+template <int NT>
+slora_status launch_rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, int cps,
+                           dim3 grid, float* part, cudaStream_t st) {
+  const int CP = padded(c);
+  switch (CP) {
+    case 16: rowdot_kernel<2, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    case 32: rowdot_kernel<4, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    case 48: rowdot_kernel<6, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    default: rowdot_kernel<8, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+  }
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+template <int NT>
+slora_status launch_coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, int cps,
+                           dim3 grid, float* part, cudaStream_t st) {
+  const int CP = padded(c);
+  switch (CP) {
+    case 16: coldot_kernel<2, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    case 32: coldot_kernel<4, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    case 48: coldot_kernel<6, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+    default: coldot_kernel<8, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+  }
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+}  // namespace
+
+int64_t rowdot_part_floats(int64_t M, int64_t K, int c) {
+  const int64_t mb = (M + TILE - 1) / TILE, nch = (K + TILE - 1) / TILE;
+  return splits_for(mb, nch) * M * padded(c);
+}
+
+int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
+  const int64_t kb = (K + TILE - 1) / TILE, nch = (M + TILE - 1) / TILE;
+  return splits_for(kb, nch) * K * padded(c);
+}
+
+slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkRowOut& o,
+                    float* part, cudaStream_t st) {
+  if (M <= 0 || c <= 0) return SLORA_OK;
+  if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "rowdot: %d columns (max 64)", c);
+  const int64_t mb = (M + TILE - 1) / TILE, nch = std::max<int64_t>((K + TILE - 1) / TILE, 1);
+  const int64_t ns = splits_for(mb, nch);
+  const int cps = int((nch + ns - 1) / ns);
+  const int nsplit = int((nch + cps - 1) / cps);
+  const dim3 grid = dim3(unsigned(mb), unsigned(nsplit), 1u);
+  {
+    LaunchScope ls(kSkinny, double(M) * K * 2 + double(K) * c * (R.dt == kF32 ? 4 : 2), st);
+    if (R.dt == kF32)
+      SLORA_TRY(launch_rowdot<3>(Y, M, K, R, c, cps, grid, part, st));
+    else
+      SLORA_TRY(launch_rowdot<1>(Y, M, K, R, c, cps, grid, part, st));
+  }
+  LaunchScope ls2(kSkinny, double(nsplit) * M * padded(c) * 4 + double(M) * c * 6, st);
+  rowdot_finalize<<<unsigned((M * c + 255) / 256), 256, 0, st>>>(part, nsplit, M, c, padded(c), o);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkColOut& o,
+                    float* part, cudaStream_t st) {
+  if (K <= 0 || c <= 0) return SLORA_OK;
+  if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "coldot: %d columns (max 64)", c);
+  const int64_t kb = (K + TILE - 1) / TILE, nch = std::max<int64_t>((M + TILE - 1) / TILE, 1);
+  const int64_t ns = splits_for(kb, nch);
+  const int cps = int((nch + ns - 1) / ns);
+  const int nsplit = int((nch + cps - 1) / cps);
+  const dim3 grid = dim3(unsigned(kb), unsigned(nsplit), 1u);
+  {
+    LaunchScope ls(kSkinny, double(M) * K * 2 + double(M) * c * (R.dt == kF32 ? 4 : 2), st);
+    if (R.dt == kF32)
+      SLORA_TRY(launch_coldot<3>(Y, M, K, R, c, cps, grid, part, st));
+    else
+      SLORA_TRY(launch_coldot<1>(Y, M, K, R, c, cps, grid, part, st));
+  }
+  LaunchScope ls2(kSkinny, double(nsplit) * K * padded(c) * 4 + double(K) * c * 4, st);
+  coldot_finalize<<<unsigned((K * c + 255) / 256), 256, 0, st>>>(part, nsplit, K, c, padded(c), o);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+}  // namespace slora

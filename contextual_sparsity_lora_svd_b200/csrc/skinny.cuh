@@ -1,0 +1,73 @@
+// Skinny contractions of the LoRA branch and of the estimator: one large
+// bf16 matrix Y [M x K] (activations or gradients, M = tokens) against a
+// rank-sized matrix with c <= 64 columns.  They are bound by the HBM stream of
+// Y, so they run on mma.sync bf16 tensor-core fragments inside CUDA-core
+// tiles (the tcgen05 tile shape would waste the machine on N = c), with fp32
+// operands split into three bf16 terms (hi + mid + lo, relative residual
+// 2^-24) so the result is fp32-accurate.
+//
+//   rowdot:  P1[m, q] = sum_k Y[m, k] R1(k, q)      (e.g. X A^T, h A_d^T, dOut B_d)
+//   coldot:  P2[k, q] = sum_m Y[m, k] R2(m, q)      (LoRA gradients, sums over tokens)
+//
+// Both write fixed-order partial sums (K or M split across blocks) that a
+// finalize pass reduces in order: results are bit-reproducible.
+#pragma once
+
+#include "common.cuh"
+
+namespace slora {
+
+struct SkY {  // Y(m, k) = ptr[(map ? map[m] : m) * ld + k], bf16, valid k < K
+  const void* ptr = nullptr;
+  int64_t ld = 0;
+  const int32_t* map = nullptr;
+};
+
+struct SkR {  // R(i, q) = ptr[(map ? map[i] : i) * si + q * sq], fp32 or bf16
+  const void* ptr = nullptr;
+  int dt = kF32;
+  int64_t si = 0, sq = 0;
+  const int32_t* map = nullptr;
+};
+
+// rowdot output: out1 fp32 at [(map1 ? map1[m] : m) * ld1 + off1 + q] and,
+// optionally, out2 bf16 at [(map2 ? map2[m] : m) * ld2 + off2 + q] scaled by s2.
+// Columns q are split at qsplit: q < qsplit go to (off1, off2), q >= qsplit
+// to (off1b + q - qsplit) of out1b / (off2b + q - qsplit) of out2b.
+struct SkRowOut {
+  float* out1 = nullptr;
+  int64_t ld1 = 0, off1 = 0;
+  const int32_t* map1 = nullptr;
+  void* out2 = nullptr;
+  int64_t ld2 = 0, off2 = 0;
+  const int32_t* map2 = nullptr;
+  float s2 = 1.0f;
+  int qsplit = 64;             // columns >= qsplit go to the second destination
+  float* out1b = nullptr;      // fp32 second destination (may be null)
+  int64_t ld1b = 0, off1b = 0;
+  const int32_t* map1b = nullptr;
+};
+
+// coldot output: v = scale * P2[k, q]; with kmap, column k is kmap[k].
+// dest = trans ? out[q' * ldo + k'] : out[k' * ldo + q'] where q' = q (or
+// q - qsplit into out_b); accumulate adds to the existing value.
+struct SkColOut {
+  float* out = nullptr;
+  float* out_b = nullptr;
+  int qsplit = 64;
+  int64_t ldo = 0;
+  int trans = 0;
+  const int32_t* kmap = nullptr;
+  float scale = 1.0f;
+  int accumulate = 0;
+};
+
+// c = number of R columns (1..64).  part: workspace of skinny_part_floats().
+int64_t rowdot_part_floats(int64_t M, int64_t K, int c);
+int64_t coldot_part_floats(int64_t M, int64_t K, int c);
+slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R1, int c,
+                    const SkRowOut& o, float* part, cudaStream_t st);
+slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R2, int c,
+                    const SkColOut& o, float* part, cudaStream_t st);
+
+}  // namespace slora

@@ -97,7 +97,9 @@ int slora_version(void);
  *                          "gemm_tc" (tcgen05 sliced GEMMs), "gemm_simt"
  *                          (CUDA-core GEMMs), "estimate" (channel scores),
  *                          "select" (top-k), "elementwise", "aux" (row maps,
- *                          operand packing), "prepare".  It synchronizes the
+ *                          operand packing), "prepare", "skinny" (rank-r
+ *                          LoRA projections and gradients), "compact"
+ *                          (selected-row gather).  It synchronizes the
  *                          recorded events.  work = algorithmic FLOPs for the
  *                          GEMM classes (2*M*N*K on the selected sizes), bytes
  *                          moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
