@@ -246,6 +246,8 @@ __global__ void coldot_finalize(const float* __restrict__ part, int nsplit, int6
 constexpr int kTargetBlocks = 148 * 8;
 
 int64_t splits_for(int64_t nblocks, int64_t nchunks) {
+  if (nblocks < 1) nblocks = 1;
+  if (nchunks < 1) nchunks = 1;
   int64_t s = (kTargetBlocks + nblocks - 1) / nblocks;
   if (s > nchunks) s = nchunks;
   if (s < 1) s = 1;

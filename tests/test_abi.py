@@ -5,6 +5,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -120,3 +121,16 @@ def test_prepare_rank_limits(L):
         L.workspace_size("slora_svd_prepare", args)
     args[4] = 8
     assert L.workspace_size("slora_svd_prepare", args) > 0
+
+
+@pytest.mark.parametrize("ctx", [[0, 0, 0], [90, 90, 90], [1, 0, 89], [70, 33, 90]])
+@pytest.mark.parametrize("s", [0.0, 0.3, 0.99])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_ffn_workspace_query_edge_layouts(L, ctx, s, bf16):
+    """Workspace planning handles empty context / output row sets and tiny k."""
+    lay = L.ffn_layer_struct(72, 152, 6, 5, 0.5, *([FAKE] * 13))
+    g = L.ffn_grads_struct(*([FAKE] * 6))
+    args, keep = L.ffn_args(L.BF16 if bf16 else L.F32, lay, 3, 90, ctx, s, FAKE, FAKE, FAKE,
+                            FAKE, g, FAKE)
+    assert L.workspace_size("slora_ffn_fwd_bwd", args) > 0
+    assert keep[2].value == 152 - int(np.floor(s * 152 + 1e-9))
