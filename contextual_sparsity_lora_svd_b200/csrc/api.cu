@@ -7,6 +7,7 @@
 #include "estimator.cuh"
 #include "gemm_simt.cuh"
 #include "linear_ops.cuh"
+#include "skinny.cuh"
 #include "swiglu.cuh"
 
 namespace slora {
@@ -100,15 +101,21 @@ extern "C" slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, s
 // --------------------------------------------------------- estimate+select
 namespace slora {
 // Estimator body shared with the FFN call.  Writes idx (see slora.h layout).
+// With P_pre the low-rank projection of the context rows is already
+// available (full row layout, row t of the context set at P_pre[ctx_rows[t]]).
 slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
                                   const slora_tokens* tok, const TokenInfo& ti,
                                   const int32_t* ctx_rows, int64_t d, const float* L0,
                                   const float* U0, int64_t n0, const float* L1, const float* U1,
                                   int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
                                   int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
-                                  cudaStream_t st) {
+                                  cudaStream_t st, bool has_pre, const float* P_pre,
+                                  int64_t ldp_pre) {
   (void)tok;
-  float* P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
+  float* P = has_pre ? nullptr : ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
+  float* ppart = (!has_pre && dt == kBF16)
+                     ? ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)))
+                     : nullptr;
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
   float* scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
   const int nsplit = ffn_score_splits(ti.T_C, n0);
@@ -119,21 +126,39 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
   else
     gram = ar.take<double>(size_t(2) * rank * rank * 33);
   if (plan) return SLORA_OK;
-  // P = X_C [L0 | L1]  (fp32 accumulate)
-  for (int p = 0; p < 2; ++p) {
-    GemmArgs g;
-    g.M = ti.T_C; g.N = rank; g.nseg = 1;
-    g.seg[0].a = rowmajor(X, dt, d, ctx_rows);
-    g.seg[0].b = colmajor(p == 0 ? L0 : L1, kF32, rank);
-    g.seg[0].K = d;
-    g.c = out_rowmajor(P + p * rank, kF32, 2 * rank);
-    SLORA_TRY(gemm_simt(g, st));
+  const float* Puse = P_pre;
+  int64_t ldp = ldp_pre;
+  const int32_t* pmap = has_pre ? ctx_rows : nullptr;
+  if (!has_pre) {
+    // P = X_C [L0 | L1]
+    if (dt == kBF16) {  // tensor-core stream over X_C, fp32 factors split in 3 bf16 terms
+      SkY y;
+      y.ptr = X; y.ld = d; y.map = ctx_rows;
+      SkR rr;
+      rr.ptr = L0; rr.dt = kF32; rr.si = rank; rr.sq = 1;
+      rr.qsplit = rank; rr.ptr_b = L1; rr.dt_b = kF32; rr.si_b = rank; rr.sq_b = 1;
+      SkRowOut o;
+      o.out1 = P; o.ld1 = 2 * rank;
+      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, st));
+    } else {  // fp32 activations: CUDA-core fp32 FMA
+      for (int p = 0; p < 2; ++p) {
+        GemmArgs g;
+        g.M = ti.T_C; g.N = rank; g.nseg = 1;
+        g.seg[0].a = rowmajor(X, dt, d, ctx_rows);
+        g.seg[0].b = colmajor(p == 0 ? L0 : L1, kF32, rank);
+        g.seg[0].K = d;
+        g.c = out_rowmajor(P + p * rank, kF32, 2 * rank);
+        SLORA_TRY(gemm_simt(g, st));
+      }
+    }
+    Puse = P;
+    ldp = 2 * rank;
   }
   if (crit == SLORA_CRIT_FFN_SWIGLU_L2) {
-    SLORA_TRY(ffn_scores(P, 2 * rank, ti.T_C, U0, U1, n0, rank, partial, nsplit, scores, st));
+    SLORA_TRY(ffn_scores(Puse, ldp, pmap, ti.T_C, U0, U1, n0, rank, partial, nsplit, scores, st));
     SLORA_TRY(topk_select(scores, 1, int(n0), int(kkeep), 1, idx_out, nullptr, st));
   } else {
-    SLORA_TRY(qk_scores(P, 2 * rank, ti.T_C, U0, U1, rank, heads, kv_heads, head_dim, gram,
+    SLORA_TRY(qk_scores(Puse, ldp, pmap, ti.T_C, U0, U1, rank, heads, kv_heads, head_dim, gram,
                         scores, st));
     SLORA_TRY(topk_select(scores, kv_heads, head_dim, int(kkeep), heads / kv_heads, idx_out,
                           idx_out + int64_t(heads) * kkeep, st));

@@ -16,8 +16,9 @@ namespace {
 // P rows through shared memory (broadcast reads).
 template <int RP>
 __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
-    const float* __restrict__ P, int64_t ldp, int64_t T_C, const float* __restrict__ Ug,
-    const float* __restrict__ Uu, int64_t n, int r, int64_t chunk, float* __restrict__ partial) {
+    const float* __restrict__ P, int64_t ldp, const int32_t* __restrict__ pmap, int64_t T_C,
+    const float* __restrict__ Ug, const float* __restrict__ Uu, int64_t n, int r, int64_t chunk,
+    float* __restrict__ partial) {
   constexpr int TT = 32;
   __shared__ float sp[TT][2 * RP];
   const int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -37,7 +38,10 @@ __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
       int tt = e / (2 * RP), q = e % (2 * RP);
       int half = q / RP, qq = q % RP;
       float v = 0.0f;
-      if (tt < nt && qq < r) v = P[(tb + tt) * ldp + half * r + qq];
+      if (tt < nt && qq < r) {
+        const int64_t row = pmap ? int64_t(pmap[tb + tt]) : tb + tt;
+        v = P[row * ldp + half * r + qq];
+      }
       sp[tt][q] = v;
     }
     __syncthreads();
@@ -66,15 +70,18 @@ __global__ void sumsq_finalize_kernel(const float* __restrict__ partial, int nsp
 
 // ----------------------------------------------------------------- QK score
 // Gram partials: block (p, split) sums P_p[t,a] P_p[t,b] over its token chunk.
-__global__ void qk_gram_partial_kernel(const float* __restrict__ P, int64_t ldp, int64_t T_C,
-                                       int r, int64_t chunk, double* __restrict__ part) {
+__global__ void qk_gram_partial_kernel(const float* __restrict__ P, int64_t ldp,
+                                       const int32_t* __restrict__ pmap, int64_t T_C, int r,
+                                       int64_t chunk, double* __restrict__ part) {
   const int p = blockIdx.x, sp = blockIdx.y, nsp = gridDim.y;
   const int64_t t0 = int64_t(sp) * chunk, t1 = min(T_C, t0 + chunk);
   for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
     int a = e / r, b = e % r;
     double s = 0.0;
-    for (int64_t t = t0; t < t1; ++t)
-      s += double(P[t * ldp + p * r + a]) * double(P[t * ldp + p * r + b]);
+    for (int64_t t = t0; t < t1; ++t) {
+      const int64_t row = pmap ? int64_t(pmap[t]) : t;
+      s += double(P[row * ldp + p * r + a]) * double(P[row * ldp + p * r + b]);
+    }
     part[(int64_t(p) * nsp + sp) * r * r + e] = s;
   }
 }
@@ -219,22 +226,26 @@ int ffn_score_splits(int64_t T_C, int64_t n) {
   return int(s);
 }
 
-slora_status ffn_scores(const float* P, int64_t ldp, int64_t T_C, const float* Ug,
-                        const float* Uu, int64_t n, int r, float* partial, int nsplit,
-                        float* scores, cudaStream_t st) {
+slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                        const float* Ug, const float* Uu, int64_t n, int r, float* partial,
+                        int nsplit, float* scores, cudaStream_t st) {
   if (n <= 0) return SLORA_OK;
   const int64_t chunk = T_C > 0 ? (T_C + nsplit - 1) / nsplit : 1;
   dim3 grid(unsigned((n + 127) / 128), unsigned(nsplit));
   {
   LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 + double(nsplit) * n * 4, st);
   if (r <= 8)
-    ffn_score_partial_kernel<8><<<grid, 128, 0, st>>>(P, ldp, T_C, Ug, Uu, n, r, chunk, partial);
+    ffn_score_partial_kernel<8><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
+                                                         partial);
   else if (r <= 16)
-    ffn_score_partial_kernel<16><<<grid, 128, 0, st>>>(P, ldp, T_C, Ug, Uu, n, r, chunk, partial);
+    ffn_score_partial_kernel<16><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
+                                                         partial);
   else if (r <= 32)
-    ffn_score_partial_kernel<32><<<grid, 128, 0, st>>>(P, ldp, T_C, Ug, Uu, n, r, chunk, partial);
+    ffn_score_partial_kernel<32><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
+                                                         partial);
   else
-    ffn_score_partial_kernel<48><<<grid, 128, 0, st>>>(P, ldp, T_C, Ug, Uu, n, r, chunk, partial);
+    ffn_score_partial_kernel<48><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
+                                                         partial);
   }
   SLORA_CHECK_LAUNCH();
   LaunchScope ls2(kEstimate, double(nsplit) * n * 4 + double(n) * 4, st);
@@ -243,7 +254,8 @@ slora_status ffn_scores(const float* P, int64_t ldp, int64_t T_C, const float* U
   return SLORA_OK;
 }
 
-slora_status qk_scores(const float* P, int64_t ldp, int64_t T_C, const float* Uq,
+slora_status qk_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                       const float* Uq,
                        const float* Uk, int r, int heads, int kv_heads, int head_dim,
                        double* gram, float* scores, cudaStream_t st) {
   constexpr int kSplits = 32;
@@ -251,7 +263,7 @@ slora_status qk_scores(const float* P, int64_t ldp, int64_t T_C, const float* Uq
   const int64_t chunk = T_C > 0 ? (T_C + kSplits - 1) / kSplits : 1;
   {
   LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4, st);
-  qk_gram_partial_kernel<<<dim3(2, kSplits), 256, 0, st>>>(P, ldp, T_C, r, chunk, part);
+  qk_gram_partial_kernel<<<dim3(2, kSplits), 256, 0, st>>>(P, ldp, pmap, T_C, r, chunk, part);
   SLORA_CHECK_LAUNCH();
   }
   SLORA_CHECK_LAUNCH();

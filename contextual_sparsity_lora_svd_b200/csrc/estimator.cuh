@@ -8,14 +8,16 @@ namespace slora {
 // FFN: sumsq partials over token chunks of (silu(P_g U_g^T) * (P_u U_u^T))^2,
 // then a fixed-order reduction and sqrt into scores[n].
 //   P [T_C x ldp] fp32 with P_g in columns [0, r) and P_u in [r, 2r).
-slora_status ffn_scores(const float* P, int64_t ldp, int64_t T_C, const float* Ug,
-                        const float* Uu, int64_t n, int r, float* partial, int nsplit,
-                        float* scores, cudaStream_t st);
+// P rows are read through pmap when given (row t of the context set is P[pmap[t]]).
+slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                        const float* Ug, const float* Uu, int64_t n, int r, float* partial,
+                        int nsplit, float* scores, cudaStream_t st);
 int ffn_score_splits(int64_t T_C, int64_t n);
 
 // QK: Gram matrices of P_q (cols [0,r)) and P_k (cols [r,2r)) in fp64, then
 // score[g, c] = ||K_hat[:, g, c]|| * sum_{h in g} ||Q_hat[:, h, c]||.
-slora_status qk_scores(const float* P, int64_t ldp, int64_t T_C, const float* Uq,
+slora_status qk_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                       const float* Uq,
                        const float* Uk, int r, int heads, int kv_heads, int head_dim,
                        double* gram /* [2 r r] */, float* scores, cudaStream_t st);
 

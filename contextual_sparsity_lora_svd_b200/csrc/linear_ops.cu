@@ -258,28 +258,54 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   void* dGO = bf(TO, Fd);
   void* dUO = bf(TO, Fd);
   // partial sums of the skinny contractions (reused sequentially)
+  const int rs = L.r_svd;
+  const bool fused = !idx_force && 2 * r + 2 * rs <= 64;  // one pass over X for XA and P
   int64_t npart = 1;
   for (int64_t M : {T, TC, TO})
     for (int64_t K : {d, kk, Fd}) {
-      npart = std::max(npart, rowdot_part_floats(M, K, 2 * r));
+      npart = std::max(npart, rowdot_part_floats(M, K, fused ? 2 * r + 2 * rs : 2 * r));
       npart = std::max(npart, coldot_part_floats(M, K, 2 * r));
     }
   float* part = ar.take<float>(size_t(npart));
+  float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
+  float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   if (!idx_force)
     SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
-                                   true, nullptr));
+                                   L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
+                                   true, nullptr, fused, Pfull, 2 * rs));
   if (plan) return SLORA_OK;
 
+  auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
+    SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
+  };
+  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
+    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
+  };
+
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
+  {  // one stream over X: XA = X [Ag; Au]^T (fp32 and s*XA bf16) and, for the
+     // estimator, P = X [Lg | Lu] (fp32-accurate, read for the context rows)
+    SkRowOut o;
+    o.out1 = XA; o.ld1 = 2 * r; o.out2 = XAb; o.ld2 = lr2; o.s2 = s;
+    SkR rr = Rv(AgAu, kBF16, 1, d);
+    int c = 2 * r;
+    if (fused) {
+      SLORA_TRY(concat_cols_f32(L.Lg, L.Lu, d, rs, rs, LgLu, st));
+      rr.qsplit = 2 * r; rr.ptr_b = LgLu; rr.dt_b = kF32; rr.si_b = 2 * rs; rr.sq_b = 1;
+      o.qsplit = 2 * r; o.out1b = Pfull; o.ld1b = 2 * rs;
+      c = 2 * r + 2 * rs;
+    }
+    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, part, st));
+  }
   if (idx_force) {
     if (kk > 0)
       SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
                                  cudaMemcpyDeviceToDevice, st));
   } else {
     SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
-                                   false, st));
+                                   L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
+                                   false, st, fused, Pfull, 2 * rs));
   }
   // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
   SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st));
@@ -291,21 +317,8 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, st));
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, st));
   SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
-  SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
-
-  auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
-    SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
-  };
-  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
-    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
-  };
 
   // ---- forward
-  {  // XA = X [Ag; Au]^T: fp32 (gradients) and s*XA in bf16 (GEMM operand)
-    SkRowOut o;
-    o.out1 = XA; o.ld1 = 2 * r; o.out2 = XAb; o.ld2 = lr2; o.s2 = s;
-    SLORA_TRY(rowdot(Yv(X, d), T, d, Rv(AgAu, kBF16, 1, d), 2 * r, o, part, st));
-  }
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
     b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, nullptr, 0, 1, mat(WuS, kk, d, d))

@@ -70,6 +70,15 @@ __global__ void copy_pad_kernel(const __nv_bfloat16* __restrict__ in, int64_t ro
   out[e] = c < cols ? in[rr * cols + c] : __float2bfloat16_rn(0.0f);
 }
 
+__global__ void concat_cols_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                                   int64_t rows, int64_t ca, int64_t cb, float* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t w = ca + cb;
+  if (e >= rows * w) return;
+  const int64_t rr = e / w, c = e % w;
+  out[e] = c < ca ? a[rr * ca + c] : b[rr * cb + (c - ca)];
+}
+
 unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
 
 }  // namespace
@@ -118,6 +127,14 @@ slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
   stack_rows_kernel<<<blocks((rows_top + rows_bottom) * cols), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(top), static_cast<const __nv_bfloat16*>(bottom), rows_top,
       rows_bottom, cols, static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64_t ca,
+                             int64_t cb, float* out, cudaStream_t st) {
+  LaunchScope ls(kAux, 8.0 * double(rows) * (ca + cb), st);
+  concat_cols_kernel<<<blocks(rows * (ca + cb)), 256, 0, st>>>(a, b, rows, ca, cb, out);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

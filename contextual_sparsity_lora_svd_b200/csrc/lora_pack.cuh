@@ -20,4 +20,7 @@ slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
 // out [rows x ldo] = in [rows x cols] with zero padding columns.
 slora_status copy_pad(const void* in, int64_t rows, int64_t cols, int64_t ldo, void* out,
                       cudaStream_t st);
+// out [rows x (ca + cb)] fp32 = [a | b] (a: rows x ca, b: rows x cb, both row-major).
+slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64_t ca,
+                             int64_t cb, float* out, cudaStream_t st);
 }  // namespace slora

@@ -41,13 +41,6 @@ __device__ __forceinline__ uint32_t lds32(const __nv_bfloat16* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-__device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
-  const int64_t ii = R.map ? R.map[i] : i;
-  const int64_t off = ii * R.si + int64_t(q) * R.sq;
-  if (R.dt == kF32) return static_cast<const float*>(R.ptr)[off];
-  return __bfloat162float(static_cast<const __nv_bfloat16*>(R.ptr)[off]);
-}
-
 // Split v into NT bf16 terms whose sum reproduces v to ~2^-8 (NT=1) or ~2^-24 (NT=3).
 template <int NT>
 __device__ __forceinline__ void split_terms(float v, __nv_bfloat16* out) {
@@ -59,6 +52,45 @@ __device__ __forceinline__ void split_terms(float v, __nv_bfloat16* out) {
     out[1] = m;
     r -= __bfloat162float(m);
     out[2] = __float2bfloat16_rn(r);
+  }
+}
+
+__device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
+  const int64_t ii = R.map ? R.map[i] : i;
+  const void* p = R.ptr;
+  int dt = R.dt;
+  int64_t off = ii * R.si + int64_t(q) * R.sq;
+  if (q >= R.qsplit) {
+    p = R.ptr_b;
+    dt = R.dt_b;
+    off = ii * R.si_b + int64_t(q - R.qsplit) * R.sq_b;
+  }
+  if (dt == kF32) return static_cast<const float*>(p)[off];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[off]);
+}
+
+// Stage the rank-sized operand for rows [i0, i0 + 64) as NT bf16 terms,
+// transposed (Rs[term][q][i]).  Lanes walk q when q is the contiguous index
+// of the source, otherwise i.
+template <int CP, int NT>
+__device__ __forceinline__ void stage_r(__nv_bfloat16 (*Rs)[CP][PAD], const SkR& R, int c,
+                                        int64_t i0, int64_t I, int tid) {
+  const bool q_fast = R.sq == 1 && (R.ptr_b == nullptr || R.sq_b == 1);
+  for (int e = tid; e < CP * TILE; e += NTH) {
+    int q, ii;
+    if (q_fast) {
+      q = e % CP;
+      ii = e / CP;
+    } else {
+      q = e / TILE;
+      ii = e % TILE;
+    }
+    const int64_t i = i0 + ii;
+    const float v = (q < c && i < I) ? load_r(R, i, q) : 0.0f;
+    __nv_bfloat16 tv[3];
+    split_terms<NT>(v, tv);
+#pragma unroll
+    for (int s = 0; s < NT; ++s) Rs[s][q][ii] = tv[s];
   }
 }
 
@@ -101,15 +133,7 @@ __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int
   for (int64_t kc = kc0; kc < kc1; ++kc) {
     const int64_t k0 = kc * TILE;
     stage_y(Ys, Y, M, K, m0, k0, tid);
-    for (int e = tid; e < CP * TILE; e += NTH) {
-      const int q = e / TILE, kk = e % TILE;
-      const int64_t k = k0 + kk;
-      const float v = (q < c && k < K) ? load_r(R, k, q) : 0.0f;
-      __nv_bfloat16 tv[3];
-      split_terms<NT>(v, tv);
-#pragma unroll
-      for (int s = 0; s < NT; ++s) Rs[s][q][kk] = tv[s];
-    }
+    stage_r<CP, NT>(Rs, R, c, k0, K, tid);
     cp_async_wait_all();
     __syncthreads();
     const int r0 = warp * 16 + g;
@@ -164,15 +188,7 @@ __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int
   for (int64_t mc = mc0; mc < mc1; ++mc) {
     const int64_t m0 = mc * TILE;
     stage_y(Ys, Y, M, K, m0, k0, tid);
-    for (int e = tid; e < CP * TILE; e += NTH) {
-      const int q = e / TILE, mm = e % TILE;
-      const int64_t m = m0 + mm;
-      const float v = (q < c && m < M) ? load_r(R, m, q) : 0.0f;
-      __nv_bfloat16 tv[3];
-      split_terms<NT>(v, tv);
-#pragma unroll
-      for (int s = 0; s < NT; ++s) Rs[s][q][mm] = tv[s];
-    }
+    stage_r<CP, NT>(Rs, R, c, m0, M, tid);
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll
@@ -243,7 +259,7 @@ __global__ void coldot_finalize(const float* __restrict__ part, int nsplit, int6
   *dst = o.accumulate ? *dst + v : v;
 }
 
-constexpr int kTargetBlocks = 148 * 8;
+constexpr int kTargetBlocks = 148 * 4;
 
 int64_t splits_for(int64_t nblocks, int64_t nchunks) {
   if (nblocks < 1) nblocks = 1;
@@ -308,7 +324,7 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
   const dim3 grid = dim3(unsigned(mb), unsigned(nsplit), 1u);
   {
     LaunchScope ls(kSkinny, double(M) * K * 2 + double(K) * c * (R.dt == kF32 ? 4 : 2), st);
-    if (R.dt == kF32)
+    if (R.dt == kF32 || (R.ptr_b && R.dt_b == kF32))
       SLORA_TRY(launch_rowdot<3>(Y, M, K, R, c, cps, grid, part, st));
     else
       SLORA_TRY(launch_rowdot<1>(Y, M, K, R, c, cps, grid, part, st));
@@ -330,7 +346,7 @@ slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
   const dim3 grid = dim3(unsigned(kb), unsigned(nsplit), 1u);
   {
     LaunchScope ls(kSkinny, double(M) * K * 2 + double(M) * c * (R.dt == kF32 ? 4 : 2), st);
-    if (R.dt == kF32)
+    if (R.dt == kF32 || (R.ptr_b && R.dt_b == kF32))
       SLORA_TRY(launch_coldot<3>(Y, M, K, R, c, cps, grid, part, st));
     else
       SLORA_TRY(launch_coldot<1>(Y, M, K, R, c, cps, grid, part, st));

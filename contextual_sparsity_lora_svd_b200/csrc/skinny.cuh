@@ -28,6 +28,11 @@ struct SkR {  // R(i, q) = ptr[(map ? map[i] : i) * si + q * sq], fp32 or bf16
   int dt = kF32;
   int64_t si = 0, sq = 0;
   const int32_t* map = nullptr;
+  // columns q >= qsplit come from a second source: ptr_b[i' * si_b + (q - qsplit) * sq_b]
+  int qsplit = 1 << 30;
+  const void* ptr_b = nullptr;
+  int dt_b = kF32;
+  int64_t si_b = 0, sq_b = 0;
 };
 
 // rowdot output: out1 fp32 at [(map1 ? map1[m] : m) * ld1 + off1 + q] and,
