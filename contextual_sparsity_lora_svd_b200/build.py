@@ -56,7 +56,8 @@ def build(verbose: bool = False, extra: list[str] | None = None) -> str:
         objs = list(ex.map(lambda s: _compile(s, extra, verbose), srcs))
     newest = max(os.path.getmtime(o) for o in objs)
     if not os.path.exists(OUT) or os.path.getmtime(OUT) < newest or extra:
-        cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-o", OUT, *objs]
+        cmd = [NVCC, *ARCH, "-shared", "-cudart", "static", "-Xlinker", "--no-undefined",
+               "-o", OUT, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -116,6 +116,9 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
   float* ppart = (!has_pre && dt == kBF16)
                      ? ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)))
                      : nullptr;
+  void* prs = (!has_pre && dt == kBF16)
+                  ? static_cast<void*>(ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(d))))
+                  : nullptr;
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
   float* scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
   const int nsplit = ffn_score_splits(ti.T_C, n0);
@@ -139,7 +142,7 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
       rr.qsplit = rank; rr.ptr_b = L1; rr.dt_b = kF32; rr.si_b = rank; rr.sq_b = 1;
       SkRowOut o;
       o.out1 = P; o.ld1 = 2 * rank;
-      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, st));
+      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, prs, st));
     } else {  // fp32 activations: CUDA-core fp32 FMA
       for (int p = 0; p < 2; ++p) {
         GemmArgs g;

@@ -267,6 +267,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       npart = std::max(npart, coldot_part_floats(M, K, 2 * r));
     }
   float* part = ar.take<float>(size_t(npart));
+  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, d, Fd}))));
   float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   if (!idx_force)
@@ -296,7 +297,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       o.qsplit = 2 * r; o.out1b = Pfull; o.ld1b = 2 * rs;
       c = 2 * r + 2 * rs;
     }
-    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, part, st));
+    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, part, rsp, st));
   }
   if (idx_force) {
     if (kk > 0)
@@ -336,10 +337,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
     SkRowOut oc;
     oc.out1 = hA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = hAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, part, st));
+    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, part, rsp, st));
     SkRowOut oo;
     oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, part, st));
+    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, part, rsp, st));
   }
   {  // down projection, context rows: reads channels S only (rows S of Wd^T)
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -360,10 +361,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dOB = dOut Bd: fp32 and s*dOB bf16; dBd = s dOut^T hA (same stream of dOut)
     SkRowOut o;
     o.out1 = dOB; o.ld1 = r; o.out2 = dOBb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, part, st));
+    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, part, rsp, st));
     SkColOut c;
     c.out = G.dBd; c.ldo = r; c.scale = s;
-    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, part, st));
+    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, part, rsp, st));
   }
   {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
@@ -384,10 +385,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
     SkColOut co;
     co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
-    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, part, st));
+    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, part, rsp, st));
     SkColOut cc = co;
     cc.kmap = idx; cc.accumulate = 1;
-    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, part, st));
+    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, part, rsp, st));
   }
   for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]; dB = s dG^T XA on the same stream
     const void* Bm = p ? L.Bu : L.Bg;
@@ -395,18 +396,18 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkRowOut oo;
     oo.out1 = dGB; oo.ld1 = 2 * r; oo.off1 = p * r; oo.map1 = out_rows;
     oo.out2 = dGBbO; oo.ld2 = lr2; oo.off2 = p * r; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, part, st));
+    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, part, rsp, st));
     SkColOut bo;
     bo.out = dBm; bo.ldo = r; bo.scale = s;
     SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
-                     bo, part, st));
+                     bo, part, rsp, st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
-    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, part, st));
+    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, part, rsp, st));
     SkColOut bc = bo;
     bc.kmap = idx; bc.accumulate = 1;
     SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
-                     bc, part, st));
+                     bc, part, rsp, st));
   }
   {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -427,7 +428,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAg | dAu = s dGB^T X over every row, one stream of X
     SkColOut c;
     c.out = G.dAg; c.out_b = G.dAu; c.qsplit = r; c.ldo = d; c.trans = 1; c.scale = s;
-    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, part, st));
+    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, part, rsp, st));
   }
   return SLORA_OK;
 }

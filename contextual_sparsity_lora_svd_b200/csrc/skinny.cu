@@ -69,28 +69,39 @@ __device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
   return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[off]);
 }
 
-// Stage the rank-sized operand for rows [i0, i0 + 64) as NT bf16 terms,
-// transposed (Rs[term][q][i]).  Lanes walk q when q is the contiguous index
-// of the source, otherwise i.
-template <int CP, int NT>
-__device__ __forceinline__ void stage_r(__nv_bfloat16 (*Rs)[CP][PAD], const SkR& R, int c,
-                                        int64_t i0, int64_t I, int tid) {
+// Pre-split of the rank-sized operand, once per call: RS[s][q][i] = term s of
+// R(i, q) (zero for q >= c or i >= I), rows of I64 = roundup(I, 64) elements.
+template <int NT>
+__global__ void prep_r_kernel(const SkR R, int c, int CP, int64_t I, int64_t I64,
+                              __nv_bfloat16* __restrict__ RS) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= int64_t(CP) * I64) return;
   const bool q_fast = R.sq == 1 && (R.ptr_b == nullptr || R.sq_b == 1);
-  for (int e = tid; e < CP * TILE; e += NTH) {
-    int q, ii;
-    if (q_fast) {
-      q = e % CP;
-      ii = e / CP;
-    } else {
-      q = e / TILE;
-      ii = e % TILE;
-    }
-    const int64_t i = i0 + ii;
-    const float v = (q < c && i < I) ? load_r(R, i, q) : 0.0f;
-    __nv_bfloat16 tv[3];
-    split_terms<NT>(v, tv);
+  int q;
+  int64_t i;
+  if (q_fast) {
+    q = int(e % CP);
+    i = e / CP;
+  } else {
+    q = int(e / I64);
+    i = e % I64;
+  }
+  const float v = (q < c && i < I) ? load_r(R, i, q) : 0.0f;
+  __nv_bfloat16 tv[3];
+  split_terms<NT>(v, tv);
 #pragma unroll
-    for (int s = 0; s < NT; ++s) Rs[s][q][ii] = tv[s];
+  for (int s = 0; s < NT; ++s) RS[(int64_t(s) * CP + q) * I64 + i] = tv[s];
+}
+
+// Stage RS[:, :, i0 .. i0+64) into Rs[s][q][0..64) with 16-byte async copies.
+template <int CP, int NT>
+__device__ __forceinline__ void stage_r(__nv_bfloat16 (*Rs)[CP][PAD],
+                                        const __nv_bfloat16* __restrict__ RS, int64_t I64,
+                                        int64_t i0, int tid) {
+  for (int e = tid; e < NT * CP * 8; e += NTH) {
+    const int seg = e & 7, row = e >> 3;  // row = s * CP + q
+    const int sidx = row / CP, q = row % CP;
+    cp_async16(&Rs[sidx][q][seg * 8], RS + int64_t(row) * I64 + i0 + seg * 8, 16);
   }
 }
 
@@ -114,13 +125,21 @@ __device__ __forceinline__ void stage_y(__nv_bfloat16 (*Ys)[PAD], const SkY& Y, 
   }
 }
 
+// cp.async double buffering: chunk j+1 is in flight while chunk j is consumed.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 template <int NF, int NT>
 __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int64_t K,
-                                                     const SkR R, int c, int chunks_per_split,
+                                                     const __nv_bfloat16* __restrict__ RS,
+                                                     int64_t I64, int chunks_per_split,
                                                      float* __restrict__ part) {
   constexpr int CP = NF * 8;
-  __shared__ __align__(16) __nv_bfloat16 Ys[TILE][PAD];
-  __shared__ __align__(16) __nv_bfloat16 Rs[NT][CP][PAD];
+  extern __shared__ __align__(16) unsigned char sk_smem[];
+  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [2][TILE][PAD]
+  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + 2 * TILE * PAD * 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t m0 = int64_t(blockIdx.x) * TILE;
   const int ks = blockIdx.y;
@@ -130,24 +149,32 @@ __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int
   float acc[NF][4];
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
-  for (int64_t kc = kc0; kc < kc1; ++kc) {
-    const int64_t k0 = kc * TILE;
-    stage_y(Ys, Y, M, K, m0, k0, tid);
-    stage_r<CP, NT>(Rs, R, c, k0, K, tid);
-    cp_async_wait_all();
+  if (kc0 < kc1) {
+    stage_y(Ys[0], Y, M, K, m0, kc0 * TILE, tid);
+    stage_r<CP, NT>(Rs[0], RS, I64, kc0 * TILE, tid);
+  }
+  cp_async_commit();
+  int buf = 0;
+  for (int64_t kc = kc0; kc < kc1; ++kc, buf ^= 1) {
+    if (kc + 1 < kc1) {
+      stage_y(Ys[buf ^ 1], Y, M, K, m0, (kc + 1) * TILE, tid);
+      stage_r<CP, NT>(Rs[buf ^ 1], RS, I64, (kc + 1) * TILE, tid);
+    }
+    cp_async_commit();
+    cp_async_wait_one();
     __syncthreads();
     const int r0 = warp * 16 + g;
 #pragma unroll
     for (int k16 = 0; k16 < TILE / 16; ++k16) {
       const int kb = k16 * 16 + 2 * t;
-      const uint32_t a0 = lds32(&Ys[r0][kb]), a1 = lds32(&Ys[r0 + 8][kb]);
-      const uint32_t a2 = lds32(&Ys[r0][kb + 8]), a3 = lds32(&Ys[r0 + 8][kb + 8]);
+      const uint32_t a0 = lds32(&Ys[buf][r0][kb]), a1 = lds32(&Ys[buf][r0 + 8][kb]);
+      const uint32_t a2 = lds32(&Ys[buf][r0][kb + 8]), a3 = lds32(&Ys[buf][r0 + 8][kb + 8]);
 #pragma unroll
       for (int f = 0; f < NF; ++f)
 #pragma unroll
         for (int s = 0; s < NT; ++s)
-          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[s][f * 8 + g][kb]),
-                   lds32(&Rs[s][f * 8 + g][kb + 8]));
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[buf][s][f * 8 + g][kb]),
+                   lds32(&Rs[buf][s][f * 8 + g][kb + 8]));
     }
     __syncthreads();
   }
@@ -170,11 +197,13 @@ __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int
 
 template <int NF, int NT>
 __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int64_t K,
-                                                     const SkR R, int c, int chunks_per_split,
+                                                     const __nv_bfloat16* __restrict__ RS,
+                                                     int64_t I64, int chunks_per_split,
                                                      float* __restrict__ part) {
   constexpr int CP = NF * 8;
-  __shared__ __align__(16) __nv_bfloat16 Ys[TILE][PAD];
-  __shared__ __align__(16) __nv_bfloat16 Rs[NT][CP][PAD];
+  extern __shared__ __align__(16) unsigned char sk_smem[];
+  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [2][TILE][PAD]
+  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + 2 * TILE * PAD * 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t k0 = int64_t(blockIdx.x) * TILE;
   const int ms = blockIdx.y;
@@ -185,11 +214,19 @@ __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
   const int mq = lane >> 3, rr = lane & 7;  // ldmatrix: matrix index, row within it
-  for (int64_t mc = mc0; mc < mc1; ++mc) {
-    const int64_t m0 = mc * TILE;
-    stage_y(Ys, Y, M, K, m0, k0, tid);
-    stage_r<CP, NT>(Rs, R, c, m0, M, tid);
-    cp_async_wait_all();
+  if (mc0 < mc1) {
+    stage_y(Ys[0], Y, M, K, mc0 * TILE, k0, tid);
+    stage_r<CP, NT>(Rs[0], RS, I64, mc0 * TILE, tid);
+  }
+  cp_async_commit();
+  int buf = 0;
+  for (int64_t mc = mc0; mc < mc1; ++mc, buf ^= 1) {
+    if (mc + 1 < mc1) {
+      stage_y(Ys[buf ^ 1], Y, M, K, (mc + 1) * TILE, k0, tid);
+      stage_r<CP, NT>(Rs[buf ^ 1], RS, I64, (mc + 1) * TILE, tid);
+    }
+    cp_async_commit();
+    cp_async_wait_one();
     __syncthreads();
 #pragma unroll
     for (int m16 = 0; m16 < TILE / 16; ++m16) {
@@ -197,14 +234,14 @@ __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int
       const int mb = m16 * 16 + (mq >> 1) * 8;
       const int kb = warp * 16 + (mq & 1) * 8;
       uint32_t a0, a1, a2, a3;
-      ldsm_x4_trans(a0, a1, a2, a3, &Ys[mb + rr][kb]);
+      ldsm_x4_trans(a0, a1, a2, a3, &Ys[buf][mb + rr][kb]);
       const int mcol = m16 * 16 + 2 * t;
 #pragma unroll
       for (int f = 0; f < NF; ++f)
 #pragma unroll
         for (int s = 0; s < NT; ++s)
-          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[s][f * 8 + g][mcol]),
-                   lds32(&Rs[s][f * 8 + g][mcol + 8]));
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[buf][s][f * 8 + g][mcol]),
+                   lds32(&Rs[buf][s][f * 8 + g][mcol + 8]));
     }
     __syncthreads();
   }
@@ -259,7 +296,7 @@ __global__ void coldot_finalize(const float* __restrict__ part, int nsplit, int6
   *dst = o.accumulate ? *dst + v : v;
 }
 
-constexpr int kTargetBlocks = 148 * 4;
+constexpr int kTargetBlocks = 148 * 8;
 
 int64_t splits_for(int64_t nblocks, int64_t nchunks) {
   if (nblocks < 1) nblocks = 1;
@@ -272,87 +309,108 @@ int64_t splits_for(int64_t nblocks, int64_t nchunks) {
 }
 
 int padded(int c) { return ((c + 15) / 16) * 16; }  // NF even keeps the templates few
+int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
+bool fp32_terms(const SkR& R) { return R.dt == kF32 || (R.ptr_b && R.dt_b == kF32); }
 
-template <int NT>
-slora_status launch_rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, int cps,
-                           dim3 grid, float* part, cudaStream_t st) {
-  const int CP = padded(c);
-  switch (CP) {
-    case 16: rowdot_kernel<2, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    case 32: rowdot_kernel<4, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    case 48: rowdot_kernel<6, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    default: rowdot_kernel<8, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-  }
+slora_status prep_r(const SkR& R, int c, int CP, int64_t I, int nt, __nv_bfloat16* RS,
+                    cudaStream_t st) {
+  const int64_t I64 = round64(std::max<int64_t>(I, 1));
+  const int64_t n = int64_t(CP) * I64;
+  LaunchScope ls(kSkinny, double(I) * c * (R.dt == kF32 ? 4 : 2) + double(nt) * n * 2, st);
+  if (nt == 3)
+    prep_r_kernel<3><<<unsigned((n + 255) / 256), 256, 0, st>>>(R, c, CP, I, I64, RS);
+  else
+    prep_r_kernel<1><<<unsigned((n + 255) / 256), 256, 0, st>>>(R, c, CP, I, I64, RS);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
 
-template <int NT>
-slora_status launch_coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, int cps,
-                           dim3 grid, float* part, cudaStream_t st) {
-  const int CP = padded(c);
-  switch (CP) {
-    case 16: coldot_kernel<2, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    case 32: coldot_kernel<4, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    case 48: coldot_kernel<6, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
-    default: coldot_kernel<8, NT><<<grid, NTH, 0, st>>>(Y, M, K, R, c, cps, part); break;
+int smem_bytes(int CP, int NT) { return 2 * TILE * PAD * 2 + 2 * NT * CP * PAD * 2; }
+
+#define SLORA_SKINNY_CASE(KERNEL, NF_, NT)                                              \
+  case NF_ * 8: {                                                                       \
+    auto kfn = KERNEL<NF_, NT>;                                                         \
+    const int sm = smem_bytes(NF_ * 8, NT);                                             \
+    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);         \
+    kfn<<<grid, NTH, sm, st>>>(Y, M, K, RS, I64, cps, part);                            \
+  } break;
+#define SLORA_SKINNY_SWITCH(KERNEL, NT)   \
+  switch (CP) {                           \
+    SLORA_SKINNY_CASE(KERNEL, 2, NT)      \
+    SLORA_SKINNY_CASE(KERNEL, 4, NT)      \
+    SLORA_SKINNY_CASE(KERNEL, 6, NT)      \
+    default:                              \
+    SLORA_SKINNY_CASE(KERNEL, 8, NT)      \
   }
-  SLORA_CHECK_LAUNCH();
-  return SLORA_OK;
-}
 
 }  // namespace
 
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c) {
   const int64_t mb = (M + TILE - 1) / TILE, nch = (K + TILE - 1) / TILE;
-  return splits_for(mb, nch) * M * padded(c);
+  return splits_for(mb, nch) * std::max<int64_t>(M, 1) * padded(c);
 }
 
 int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
   const int64_t kb = (K + TILE - 1) / TILE, nch = (M + TILE - 1) / TILE;
-  return splits_for(kb, nch) * K * padded(c);
+  return splits_for(kb, nch) * std::max<int64_t>(K, 1) * padded(c);
 }
 
+int64_t skinny_rsplit_elems(int64_t I) { return 3 * 64 * round64(std::max<int64_t>(I, 1)); }
+
 slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkRowOut& o,
-                    float* part, cudaStream_t st) {
+                    float* part, void* rsplit, cudaStream_t st) {
   if (M <= 0 || c <= 0) return SLORA_OK;
   if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "rowdot: %d columns (max 64)", c);
+  const int CP = padded(c);
+  const int nt = fp32_terms(R) ? 3 : 1;
+  const int64_t I64 = round64(std::max<int64_t>(K, 1));
+  __nv_bfloat16* RS = static_cast<__nv_bfloat16*>(rsplit);
+  SLORA_TRY(prep_r(R, c, CP, K, nt, RS, st));
   const int64_t mb = (M + TILE - 1) / TILE, nch = std::max<int64_t>((K + TILE - 1) / TILE, 1);
   const int64_t ns = splits_for(mb, nch);
   const int cps = int((nch + ns - 1) / ns);
   const int nsplit = int((nch + cps - 1) / cps);
   const dim3 grid = dim3(unsigned(mb), unsigned(nsplit), 1u);
   {
-    LaunchScope ls(kSkinny, double(M) * K * 2 + double(K) * c * (R.dt == kF32 ? 4 : 2), st);
-    if (R.dt == kF32 || (R.ptr_b && R.dt_b == kF32))
-      SLORA_TRY(launch_rowdot<3>(Y, M, K, R, c, cps, grid, part, st));
-    else
-      SLORA_TRY(launch_rowdot<1>(Y, M, K, R, c, cps, grid, part, st));
+    LaunchScope ls(kSkinny, double(M) * K * 2 + double(nsplit) * M * CP * 4, st);
+    if (nt == 3) {
+      SLORA_SKINNY_SWITCH(rowdot_kernel, 3)
+    } else {
+      SLORA_SKINNY_SWITCH(rowdot_kernel, 1)
+    }
+    SLORA_CHECK_LAUNCH();
   }
-  LaunchScope ls2(kSkinny, double(nsplit) * M * padded(c) * 4 + double(M) * c * 6, st);
-  rowdot_finalize<<<unsigned((M * c + 255) / 256), 256, 0, st>>>(part, nsplit, M, c, padded(c), o);
+  LaunchScope ls2(kSkinny, double(nsplit) * M * CP * 4 + double(M) * c * 6, st);
+  rowdot_finalize<<<unsigned((M * c + 255) / 256), 256, 0, st>>>(part, nsplit, M, c, CP, o);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
 
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkColOut& o,
-                    float* part, cudaStream_t st) {
+                    float* part, void* rsplit, cudaStream_t st) {
   if (K <= 0 || c <= 0) return SLORA_OK;
   if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "coldot: %d columns (max 64)", c);
+  const int CP = padded(c);
+  const int nt = fp32_terms(R) ? 3 : 1;
+  const int64_t I64 = round64(std::max<int64_t>(M, 1));
+  __nv_bfloat16* RS = static_cast<__nv_bfloat16*>(rsplit);
+  SLORA_TRY(prep_r(R, c, CP, M, nt, RS, st));
   const int64_t kb = (K + TILE - 1) / TILE, nch = std::max<int64_t>((M + TILE - 1) / TILE, 1);
   const int64_t ns = splits_for(kb, nch);
   const int cps = int((nch + ns - 1) / ns);
   const int nsplit = int((nch + cps - 1) / cps);
   const dim3 grid = dim3(unsigned(kb), unsigned(nsplit), 1u);
   {
-    LaunchScope ls(kSkinny, double(M) * K * 2 + double(M) * c * (R.dt == kF32 ? 4 : 2), st);
-    if (R.dt == kF32 || (R.ptr_b && R.dt_b == kF32))
-      SLORA_TRY(launch_coldot<3>(Y, M, K, R, c, cps, grid, part, st));
-    else
-      SLORA_TRY(launch_coldot<1>(Y, M, K, R, c, cps, grid, part, st));
+    LaunchScope ls(kSkinny, double(M) * K * 2 + double(nsplit) * K * CP * 4, st);
+    if (nt == 3) {
+      SLORA_SKINNY_SWITCH(coldot_kernel, 3)
+    } else {
+      SLORA_SKINNY_SWITCH(coldot_kernel, 1)
+    }
+    SLORA_CHECK_LAUNCH();
   }
-  LaunchScope ls2(kSkinny, double(nsplit) * K * padded(c) * 4 + double(K) * c * 4, st);
-  coldot_finalize<<<unsigned((K * c + 255) / 256), 256, 0, st>>>(part, nsplit, K, c, padded(c), o);
+  LaunchScope ls2(kSkinny, double(nsplit) * K * CP * 4 + double(K) * c * 4, st);
+  coldot_finalize<<<unsigned((K * c + 255) / 256), 256, 0, st>>>(part, nsplit, K, c, CP, o);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

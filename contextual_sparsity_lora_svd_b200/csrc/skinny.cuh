@@ -67,12 +67,15 @@ struct SkColOut {
   int accumulate = 0;
 };
 
-// c = number of R columns (1..64).  part: workspace of skinny_part_floats().
+// c = number of R columns (1..64).  part: fp32 workspace of *_part_floats();
+// rsplit: bf16 workspace of skinny_rsplit_elems(I) elements, I = K (rowdot) or
+// M (coldot), holding the pre-split rank-sized operand.
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c);
 int64_t coldot_part_floats(int64_t M, int64_t K, int c);
-slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R1, int c,
-                    const SkRowOut& o, float* part, cudaStream_t st);
-slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R2, int c,
-                    const SkColOut& o, float* part, cudaStream_t st);
+int64_t skinny_rsplit_elems(int64_t I);
+slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
+                    const SkRowOut& o, float* part, void* rsplit, cudaStream_t st);
+slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
+                    const SkColOut& o, float* part, void* rsplit, cudaStream_t st);
 
 }  // namespace slora

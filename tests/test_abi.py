@@ -134,3 +134,9 @@ def test_ffn_workspace_query_edge_layouts(L, ctx, s, bf16):
                             FAKE, g, FAKE)
     assert L.workspace_size("slora_ffn_fwd_bwd", args) > 0
     assert keep[2].value == 152 - int(np.floor(s * 152 + 1e-9))
+
+
+def test_library_has_no_unresolved_internal_symbols(L):
+    out = subprocess.run(["nm", "-D", "--undefined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    assert "slora" not in out, out
