@@ -85,6 +85,10 @@ _sig("slora_ffn_fwd_bwd", c_int,
       c_vp,
       ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 
+_sig("slora_noalloc_scratch_bytes", c_sz, [])
+_sig("slora_estimate_select_noalloc", c_int,
+     [c_int, c_vp, c_int, ctypes.POINTER(Tokens), c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64,
+      c_int, c_int, c_int, c_int, ctypes.c_double, c_vp, P_I32, c_vp, c_vp])
 _sig("slora_launch_count", c_i64, [])
 _sig("slora_profile_enable", None, [c_int])
 _sig("slora_profile_read", c_int, [ctypes.c_char_p, ctypes.POINTER(c_i64),
@@ -93,7 +97,8 @@ _sig("slora_profile_read", c_int, [ctypes.c_char_p, ctypes.POINTER(c_i64),
 EXPORTS = sorted(["slora_last_error_string", "slora_version", "slora_svd_prepare",
                   "slora_estimate_select", "slora_linear_fwd", "slora_linear_bwd",
                   "slora_ffn_fwd_bwd", "slora_launch_count", "slora_profile_enable",
-                  "slora_profile_read"])
+                  "slora_profile_read", "slora_noalloc_scratch_bytes",
+                  "slora_estimate_select_noalloc"])
 
 
 def lib():
@@ -198,6 +203,25 @@ def slora_estimate_select(crit, X, batch, seq, ctx_len, L0, U0, L1, U1, rank, sp
           float(sparsity), ptr(idx_out), ctypes.byref(k_out), ptr(scores_out)], ws, stream)
     del keep
     return int(k_out.value)
+
+
+def slora_estimate_select_noalloc(crit, X, batch, seq, ctx_len, L0, U0, L1, U1, rank, sparsity,
+                                  idx_out, heads=0, kv_heads=0, head_dim=0, scores_out=None,
+                                  stream=None):
+    """slora_estimate_select with the library's built-in scratch buffer (no
+    workspace argument, nothing allocated).  Returns k_keep (FFN) or k_h (QK)."""
+    tok, keep = make_tokens(batch, seq, ctx_len)
+    k_out = c_i32(0)
+    _check("slora_estimate_select_noalloc", _lib.slora_estimate_select_noalloc(
+        crit, ptr(X), dtype_code(X), ctypes.byref(tok), X.shape[1], ptr(L0), ptr(U0),
+        U0.shape[0], ptr(L1), ptr(U1), U1.shape[0], rank, heads, kv_heads, head_dim,
+        float(sparsity), ptr(idx_out), ctypes.byref(k_out), ptr(scores_out), _stream(stream)))
+    del keep
+    return int(k_out.value)
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(_lib.slora_noalloc_scratch_bytes())
 
 
 def slora_linear_fwd(side, batch, seq, ctx_len, k, n, W, A, B, lora_scale, idx, X_ctx,

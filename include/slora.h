@@ -165,6 +165,42 @@ slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dt
                                    slora_stream_t stream);
 
 /*
+ * slora_estimate_select_noalloc — slora_estimate_select for callers that
+ * cannot allocate device memory.  The pages have no counterpart of this call;
+ * it exists for integration only.
+ *
+ * Some callers have no way to give the library a workspace: a plugin
+ * interface of a framework that owns every device allocation through its own
+ * pool and hands a kernel only its input and output buffers; a process that
+ * reserved nearly all device memory at start-up, so a later cudaMalloc would
+ * fail; a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device synchronisation.  This entry point takes the same arguments as
+ * slora_estimate_select minus the workspace, and runs with a scratch buffer
+ * that the library itself holds in device memory: a fixed
+ * slora_noalloc_scratch_bytes() bytes (32 MiB) on every GPU that loads the
+ * library, kept until the process exits.  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - Problems whose scratch need exceeds the buffer are refused with
+ *     SLORA_ERR_WORKSPACE (the message states both sizes); use
+ *     slora_estimate_select with a workspace for those.
+ *   - The first call on a device resolves the buffer's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one buffer and it keeps the last
+ *     call's contents (nothing in it needs to start at zero).  Calls that
+ *     overlap on the GPU (different streams, or different host threads
+ *     without ordering) race on it: serialise them.
+ */
+size_t slora_noalloc_scratch_bytes(void);
+slora_status slora_estimate_select_noalloc(slora_criterion crit, const void* X, slora_dtype dt,
+                                           const slora_tokens* tok, int64_t d, const float* L0,
+                                           const float* U0, int64_t n0, const float* L1,
+                                           const float* U1, int64_t n1, int rank, int heads,
+                                           int kv_heads, int head_dim, double sparsity,
+                                           int32_t* idx_out, int32_t* k_out, float* scores_out,
+                                           slora_stream_t stream);
+
+/*
  * slora_linear_fwd — one LoRA linear on the selected slices, output tokens
  * dense [ART §1, §3, §6, §7; ABS].
  *
