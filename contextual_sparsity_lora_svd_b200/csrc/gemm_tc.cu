@@ -50,6 +50,7 @@ struct alignas(64) TcParams {
   int paired;
   int N;
   int epi;
+  int vec_out;  // output rows start on 16-byte boundaries (vector stores allowed)
   void* out0;
   void* out1;
   void* out2;
@@ -170,8 +171,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 
 // Store 32 consecutive bf16 values (row-major, column c0..c0+31) with
 // per-column masking at the right edge.
-__device__ __forceinline__ void store_row32(__nv_bfloat16* row, int c0, int N, const float* v) {
-  if (c0 + 32 <= N) {
+__device__ __forceinline__ void store_row32(__nv_bfloat16* row, int c0, int N, const float* v,
+                                            bool vec = true) {
+  if (vec && c0 + 32 <= N) {
     uint4* dst = reinterpret_cast<uint4*>(row + c0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -437,7 +439,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__
         for (int c = 0; c < 8; ++c) {
           tmem_ld32(tl + c * 32, v);
           const int c0 = ti.n0 + c * 32;
-          if (valid && c0 < p.N) store_row32(o, c0, p.N, v);
+          if (valid && c0 < p.N) store_row32(o, c0, p.N, v, p.vec_out != 0);
         }
       }
       fence_before();
@@ -509,8 +511,8 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   if (g.tiles == nullptr) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: tile list missing");
   if (g.n_mtiles <= 0) return SLORA_OK;
   if (g.nseg < 1 || g.nseg > 4) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: nseg=%d", g.nseg);
-  if (g.ldo % 8 || (g.epi == EPI_SWIGLU_BWD && g.ldi % 8))
-    SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: output leading dimension not a multiple of 8");
+  if (g.epi != EPI_STORE && (g.ldo % 8 || (g.epi == EPI_SWIGLU_BWD && g.ldi % 8)))
+    SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: SwiGLU operands need rows of whole 16 bytes");
   if (g.N > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: N too large");
   SLORA_TRY(get_encode());
   TcParams p;
@@ -552,6 +554,7 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   p.paired = g.paired;
   p.N = int(g.N);
   p.epi = g.epi;
+  p.vec_out = (g.ldo % 8 == 0) && ((reinterpret_cast<uintptr_t>(g.out0) & 15) == 0);
   p.out0 = g.out0;
   p.out1 = g.out1;
   p.out2 = g.out2;

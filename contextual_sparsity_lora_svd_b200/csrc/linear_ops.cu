@@ -33,10 +33,20 @@ void add(GemmArgs& g, MatRef a, MatRef b, int64_t K, float alpha = 1.0f) {
 
 }  // namespace
 
+slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                           const void* X_out, void* Y_ctx, void* Y_out, float* XA_save, Arena& ar,
+                           bool plan, cudaStream_t st);
+slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                           const void* X_out, const float* XA, const void* dY_ctx,
+                           const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
+                           Arena& ar, bool plan, cudaStream_t st);
+
 // ------------------------------------------------------------------ forward
 slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
                             const void* X_out, void* Y_ctx, void* Y_out, float* XA_save,
                             Arena& ar, bool plan, cudaStream_t st) {
+  if (L.dt == kBF16)
+    return linear_fwd_tc(L, tok, X_ctx, X_out, Y_ctx, Y_out, XA_save, ar, plan, st);
   const TokenInfo& ti = L.ti;
   const int dt = L.dt, r = L.r;
   const int64_t k = L.k, n = L.n, ni = L.n_idx;
@@ -94,6 +104,9 @@ slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const 
                             const void* X_out, const float* XA, const void* dY_ctx,
                             const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
                             Arena& ar, bool plan, cudaStream_t st) {
+  if (L.dt == kBF16)
+    return linear_bwd_tc(L, tok, X_ctx, X_out, XA, dY_ctx, dY_out, dX_ctx, dX_out, dA, dB, ar,
+                         plan, st);
   const TokenInfo& ti = L.ti;
   const int dt = L.dt, r = L.r;
   const int64_t k = L.k, n = L.n, ni = L.n_idx;
@@ -585,6 +598,258 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
     SLORA_TRY(gemm(b1, st));
   }
   return SLORA_OK;
+}
+
+// ------------------------------------------------------ linear, bf16, tcgen05
+// Same structure as the FFN: the selected slice of W0 is compacted into
+// contiguous rows once per call, the large contractions run on tcgen05
+// (context rows on the slice, output rows dense), the rank-r projections and
+// the LoRA gradients on the skinny tensor-core kernels.
+namespace {
+SkY ykv(const void* p, int64_t ld, const int32_t* map = nullptr) {
+  SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
+}
+SkR rkv(const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
+  SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
+}
+int64_t skinny_part_bound(const TokenInfo& ti, int64_t a, int64_t b, int64_t c2, int r) {
+  int64_t np = 1;
+  for (int64_t M : {ti.T, ti.T_C, ti.T_O})
+    for (int64_t K : {a, b, c2}) {
+      np = std::max(np, rowdot_part_floats(M, K, r));
+      np = std::max(np, coldot_part_floats(M, K, r));
+    }
+  return np;
+}
+}  // namespace
+
+slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                           const void* X_out, void* Y_ctx, void* Y_out, float* XA_save, Arena& ar,
+                           bool plan, cudaStream_t st) {
+  const TokenInfo& ti = L.ti;
+  const int r = L.r;
+  const int64_t k = L.k, n = L.n, ni = L.n_idx, T = ti.T, TC = ti.T_C, TO = ti.T_O;
+  const float s = L.s;
+  const int64_t lr = round8(r), ldi = round8(std::max<int64_t>(ni, 1));
+  const bool none = L.side == SLORA_SLICE_NONE, outr = L.side == SLORA_SLICE_OUT_ROWS;
+  const int64_t nct = count_tiles(tok, true), nott = count_tiles(tok, false);
+  auto bf = [&](int64_t rows, int64_t cols) {
+    return static_cast<void*>(ar.take<__nv_bfloat16>(size_t(std::max<int64_t>(rows * cols, 1))));
+  };
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TC, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TO, 1)));
+  int4* ctiles = ar.take<int4>(size_t(std::max<int64_t>(nct, 1)));
+  int4* otiles = ar.take<int4>(size_t(std::max<int64_t>(nott, 1)));
+  int4* ptiles = ar.take<int4>(size_t((T + 127) / 128));
+  float* XA = XA_save ? XA_save : ar.take<float>(size_t(T) * r);
+  void* XAb = bf(T, lr);      // s*XA, full rows (NONE, OUT_ROWS)
+  void* XAbC = bf(TC, lr);    // s*XA, compact context rows (IN_COLS)
+  void* XAbO = bf(TO, lr);    // s*XA, compact output rows (IN_COLS)
+  void* Bp = bf(n, lr);       // B padded
+  void* BS = bf(ni, lr);      // B[idx] padded (OUT_ROWS)
+  void* WS = bf(ni, outr ? k : n);  // rows idx of W (W0 or W0^T)
+  void* Xpad = (!none && !outr && ni % 8) ? bf(TC, ldi) : nullptr;  // X_ctx with 16-byte rows
+  float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
+  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  if (plan) return SLORA_OK;
+
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  SLORA_TRY(gather_pad(L.B, r, nullptr, n, r, Bp, lr, st));
+  if (none || outr) {
+    SkRowOut o;
+    o.out1 = XA; o.ld1 = r; o.out2 = XAb; o.ld2 = lr; o.s2 = s;
+    SLORA_TRY(rowdot(ykv(X_ctx, k), T, k, rkv(L.A, kBF16, 1, k), r, o, part, rsp, st));
+  }
+  if (none) {
+    SLORA_TRY(make_plain_tiles(ptiles, T, st));
+    TcBuilder b(ptiles, (T + 127) / 128, 0, 0, T, n, 0, EPI_STORE);
+    b.seg(mat(X_ctx, T, k, k), mat(L.W, n, k, k), B_K, k)
+        .seg(mat(XAb, T, r, lr), mat(Bp, n, r, lr), B_K, r)
+        .out(Y_ctx, nullptr, nullptr, n);
+    return gemm_tc(b.g, st);
+  }
+  if (outr) {
+    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st));
+    SLORA_TRY(gather_pad(L.B, r, L.idx, ni, r, BS, lr, st));
+    {  // context rows, output channels S
+      TcBuilder b(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
+      b.seg(mat(X_ctx, T, k, k), mat(WS, ni, k, k), B_K, k)
+          .seg(mat(XAb, T, r, lr), mat(BS, ni, r, lr), B_K, r)
+          .out(Y_ctx, nullptr, nullptr, ni);
+      SLORA_TRY(gemm_tc(b.g, st));
+    }
+    TcBuilder b(otiles, nott, 0, 1, TO, n, 0, EPI_STORE);  // output rows, dense
+    b.seg(mat(X_ctx, T, k, k), mat(L.W, n, k, k), B_K, k)
+        .seg(mat(XAb, T, r, lr), mat(Bp, n, r, lr), B_K, r)
+        .out(Y_out, nullptr, nullptr, n);
+    return gemm_tc(b.g, st);
+  }
+  // IN_COLS: W = W0^T [k x n]; context rows read input channels S only
+  const void* Xc = X_ctx;
+  int64_t ldxc = ni;
+  if (Xpad) {
+    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st));
+    Xc = Xpad;
+    ldxc = ldi;
+  }
+  {
+    SkRowOut oc;
+    oc.out1 = XA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = XAbC; oc.ld2 = lr; oc.s2 = s;
+    SLORA_TRY(rowdot(ykv(Xc, ldxc), TC, ni, rkv(L.A, kBF16, 1, k, L.idx), r, oc, part, rsp, st));
+    SkRowOut oo;
+    oo.out1 = XA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = XAbO; oo.ld2 = lr; oo.s2 = s;
+    SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, part, rsp, st));
+  }
+  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st));
+  {
+    TcBuilder b(ctiles, nct, 1, 0, TC, n, 0, EPI_STORE);
+    b.seg(mat(Xc, TC, ni, ldxc), mat(WS, ni, n, n), B_MN, ni)
+        .seg(mat(XAbC, TC, r, lr), mat(Bp, n, r, lr), B_K, r)
+        .out(Y_ctx, nullptr, nullptr, n);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  TcBuilder b(otiles, nott, 1, 0, TO, n, 0, EPI_STORE);
+  b.seg(mat(X_out, TO, k, k), mat(L.W, k, n, n), B_MN, k)
+      .seg(mat(XAbO, TO, r, lr), mat(Bp, n, r, lr), B_K, r)
+      .out(Y_ctx, nullptr, nullptr, n);
+  return gemm_tc(b.g, st);
+}
+
+slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+                           const void* X_out, const float* XA, const void* dY_ctx,
+                           const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
+                           Arena& ar, bool plan, cudaStream_t st) {
+  const TokenInfo& ti = L.ti;
+  const int r = L.r;
+  const int64_t k = L.k, n = L.n, ni = L.n_idx, T = ti.T, TC = ti.T_C, TO = ti.T_O;
+  const float s = L.s;
+  const int64_t lr = round8(r), ldi = round8(std::max<int64_t>(ni, 1));
+  const bool none = L.side == SLORA_SLICE_NONE, outr = L.side == SLORA_SLICE_OUT_ROWS;
+  const int64_t nct = count_tiles(tok, true), nott = count_tiles(tok, false);
+  auto bf = [&](int64_t rows, int64_t cols) {
+    return static_cast<void*>(ar.take<__nv_bfloat16>(size_t(std::max<int64_t>(rows * cols, 1))));
+  };
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TC, 1)));
+  int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(TO, 1)));
+  int4* ctiles = ar.take<int4>(size_t(std::max<int64_t>(nct, 1)));
+  int4* otiles = ar.take<int4>(size_t(std::max<int64_t>(nott, 1)));
+  int4* ptiles = ar.take<int4>(size_t((T + 127) / 128));
+  float* dYB = ar.take<float>(size_t(T) * r);
+  void* dYBb = bf(T, lr);     // s*dYB, full rows (NONE, IN_COLS)
+  void* dYBbC = bf(TC, lr);   // compact context rows (OUT_ROWS)
+  void* dYBbO = bf(TO, lr);   // compact output rows (OUT_ROWS)
+  void* WS = bf(ni, outr ? k : n);
+  void* AS = bf(ni, lr);      // A[:, idx]^T padded (IN_COLS)
+  void* At = bf(k, lr);       // A^T padded (IN_COLS)
+  void* dYpad = (outr && ni % 8) ? bf(TC, ldi) : nullptr;
+  void* Xpad = (!none && !outr && ni % 8) ? bf(TC, ldi) : nullptr;
+  float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
+  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  if (plan) return SLORA_OK;
+
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  if (none) {
+    SkRowOut o;
+    o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
+    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, part, rsp, st));
+    SLORA_TRY(make_plain_tiles(ptiles, T, st));
+    TcBuilder b(ptiles, (T + 127) / 128, 0, 0, T, k, 0, EPI_STORE);
+    b.seg(mat(dY_ctx, T, n, n), mat(L.W, n, k, k), B_MN, n)
+        .seg(mat(dYBb, T, r, lr), mat(L.A, r, k, k), B_MN, r)
+        .out(dX_ctx, nullptr, nullptr, k);
+    SLORA_TRY(gemm_tc(b.g, st));
+    SkColOut ca;
+    ca.out = dA; ca.ldo = k; ca.trans = 1; ca.scale = s;
+    SLORA_TRY(coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, part, rsp, st));
+    SkColOut cb;
+    cb.out = dB; cb.ldo = r; cb.scale = s;
+    return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, part, rsp, st);
+  }
+  if (outr) {
+    const void* dYc = dY_ctx;
+    int64_t lddc = ni;
+    if (dYpad) {
+      SLORA_TRY(gather_pad(dY_ctx, ni, nullptr, TC, ni, dYpad, ldi, st));
+      dYc = dYpad;
+      lddc = ldi;
+    }
+    {  // dYB = dY B on the rows' channels; dB = s dY^T XA (output rows first, then += S rows)
+      SkRowOut oc;
+      oc.out1 = dYB; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = dYBbC; oc.ld2 = lr; oc.s2 = s;
+      SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx), r, oc, part, rsp,
+                       st));
+      SkRowOut oo;
+      oo.out1 = dYB; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = dYBbO; oo.ld2 = lr; oo.s2 = s;
+      SLORA_TRY(rowdot(ykv(dY_out, n), TO, n, rkv(L.B, kBF16, r, 1), r, oo, part, rsp, st));
+      SkColOut bo;
+      bo.out = dB; bo.ldo = r; bo.scale = s;
+      SLORA_TRY(coldot(ykv(dY_out, n), TO, n, rkv(XA, kF32, r, 1, out_rows), r, bo, part, rsp,
+                       st));
+      SkColOut bc = bo;
+      bc.kmap = L.idx; bc.accumulate = 1;
+      SLORA_TRY(coldot(ykv(dYc, lddc), TC, ni, rkv(XA, kF32, r, 1, ctx_rows), r, bc, part, rsp,
+                       st));
+    }
+    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st));
+    {  // dX, context rows: dY_C W0[S] + s dYB_C A
+      TcBuilder b(ctiles, nct, 1, 0, TC, k, 0, EPI_STORE);
+      b.seg(mat(dYc, TC, ni, lddc), mat(WS, ni, k, k), B_MN, ni)
+          .seg(mat(dYBbC, TC, r, lr), mat(L.A, r, k, k), B_MN, r)
+          .out(dX_ctx, nullptr, nullptr, k);
+      SLORA_TRY(gemm_tc(b.g, st));
+    }
+    {
+      TcBuilder b(otiles, nott, 1, 0, TO, k, 0, EPI_STORE);
+      b.seg(mat(dY_out, TO, n, n), mat(L.W, n, k, k), B_MN, n)
+          .seg(mat(dYBbO, TO, r, lr), mat(L.A, r, k, k), B_MN, r)
+          .out(dX_ctx, nullptr, nullptr, k);
+      SLORA_TRY(gemm_tc(b.g, st));
+    }
+    SkColOut ca;  // dA = s dYB^T X over every row
+    ca.out = dA; ca.ldo = k; ca.trans = 1; ca.scale = s;
+    return coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, part, rsp, st);
+  }
+  // IN_COLS: W = W0^T [k x n]; dY is the full T x n gradient
+  const void* Xc = X_ctx;
+  int64_t ldxc = ni;
+  if (Xpad) {
+    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st));
+    Xc = Xpad;
+    ldxc = ldi;
+  }
+  {
+    SkRowOut o;
+    o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
+    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, part, rsp, st));
+  }
+  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st));
+  SLORA_TRY(transpose_rows(L.A, r, k, L.idx, ni, lr, AS, st));
+  SLORA_TRY(transpose_rows(L.A, r, k, nullptr, k, lr, At, st));
+  {  // dX_ctx = dY_C W0[:, S] + s dYB_C A[:, S]
+    TcBuilder b(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
+    b.seg(mat(dY_ctx, T, n, n), mat(WS, ni, n, n), B_K, n)
+        .seg(mat(dYBb, T, r, lr), mat(AS, ni, r, lr), B_K, r)
+        .out(dX_ctx, nullptr, nullptr, ni);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {
+    TcBuilder b(otiles, nott, 0, 1, TO, k, 0, EPI_STORE);
+    b.seg(mat(dY_ctx, T, n, n), mat(L.W, k, n, n), B_K, n)
+        .seg(mat(dYBb, T, r, lr), mat(At, k, r, lr), B_K, r)
+        .out(dX_out, nullptr, nullptr, k);
+    SLORA_TRY(gemm_tc(b.g, st));
+  }
+  {  // dA: output rows over every column, then += context rows on columns S
+    SkColOut ao;
+    ao.out = dA; ao.ldo = k; ao.trans = 1; ao.scale = s;
+    SLORA_TRY(coldot(ykv(X_out, k), TO, k, rkv(dYB, kF32, r, 1, out_rows), r, ao, part, rsp, st));
+    SkColOut ac = ao;
+    ac.kmap = L.idx; ac.accumulate = 1;
+    SLORA_TRY(coldot(ykv(Xc, ldxc), TC, ni, rkv(dYB, kF32, r, 1, ctx_rows), r, ac, part, rsp, st));
+  }
+  SkColOut cb;  // dB = s dY^T XA over every row
+  cb.out = dB; cb.ldo = r; cb.scale = s;
+  return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, part, rsp, st);
 }
 
 }  // namespace slora

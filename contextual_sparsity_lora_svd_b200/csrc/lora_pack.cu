@@ -79,6 +79,24 @@ __global__ void concat_cols_kernel(const float* __restrict__ a, const float* __r
   out[e] = c < ca ? a[rr * ca + c] : b[rr * cb + (c - ca)];
 }
 
+__global__ void gather_pad_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in,
+                                  const int32_t* __restrict__ idx, int64_t n, int64_t cols,
+                                  int64_t ldo, __nv_bfloat16* __restrict__ out) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n * ldo) return;
+  const int64_t j = e / ldo, c = e % ldo;
+  const int64_t src = idx ? int64_t(idx[j]) : j;
+  out[e] = c < cols ? in[src * ld_in + c] : __float2bfloat16_rn(0.0f);
+}
+
+__global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t nt) {
+  const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= nt) return;
+  const int64_t r0 = t * 128;
+  const int64_t nv = M - r0 < 128 ? M - r0 : 128;
+  tiles[t] = make_int4(int(r0), int(r0), int(nv), 0);
+}
+
 unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
 
 }  // namespace
@@ -135,6 +153,26 @@ slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64
                              int64_t cb, float* out, cudaStream_t st) {
   LaunchScope ls(kAux, 8.0 * double(rows) * (ca + cb), st);
   concat_cols_kernel<<<blocks(rows * (ca + cb)), 256, 0, st>>>(a, b, rows, ca, cb, out);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
+                        int64_t cols, void* out, int64_t ldo, cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(n) * (cols + ldo) * 2, st);
+  gather_pad_kernel<<<blocks(n * ldo), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), ld_in,
+                                                     idx, n, cols, ldo,
+                                                     static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st) {
+  const int64_t nt = (M + 127) / 128;
+  if (nt <= 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(nt) * 16, st);
+  plain_tiles_kernel<<<blocks(nt), 256, 0, st>>>(tiles, M, nt);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

@@ -23,4 +23,10 @@ slora_status copy_pad(const void* in, int64_t rows, int64_t cols, int64_t ldo, v
 // out [rows x (ca + cb)] fp32 = [a | b] (a: rows x ca, b: rows x cb, both row-major).
 slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64_t ca,
                              int64_t cb, float* out, cudaStream_t st);
+// out [n x ldo] bf16 = rows (idx ? idx[j] : j) of in [* x ld_in], first `cols`
+// columns, zero padded to ldo.
+slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
+                        int64_t cols, void* out, int64_t ldo, cudaStream_t st);
+// M-tile list {row0, row0, nvalid, 0} covering rows [0, M) in 128-row tiles.
+slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st);
 }  // namespace slora
