@@ -34,6 +34,26 @@ METRIC = "sparse LoRA fwd+bwd tokens/s; sliced-GEMM % bf16 peak; estimator HBM G
 UNIT = "tokens/s"
 
 
+def measured_traffic(kernel_file, summary):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        src = os.path.join(ROOT, "contextual_sparsity_lora_svd_b200", "csrc", kernel_file)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        vals = {}
+        for line in open(os.path.join(ROOT, "profiles", summary)):
+            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch",
+                                                      "kernel_source_sha256"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+        if vals.get("kernel_source_sha256") != sha:
+            return None
+        return float(vals["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -336,15 +356,19 @@ def run_ours(args, rank, world):
 
     # ---- roofline of the dominant kernel class (by device time)
     kernels = {}
+    ktot = sum(v[1] for v in prof.values())
     for c, (n, kms, work) in prof.items():
         if n:
             kernels[c] = {"launches_per_step": n / args.steps, "ms_per_step": kms / args.steps,
-                          "share": kms / ms if ms > 0 else None}
+                          "share": kms / ktot if ktot > 0 else None,
+                          "share_of_step": kms / ms if ms > 0 else None}
     gemm_cls = max(("gemm_tc", "gemm_simt"), key=lambda c: prof[c][1])
     n_g, ms_g, fl_g = prof[gemm_cls]
     achieved = fl_g / (ms_g / 1e3) / 1e12 if ms_g > 0 else 0.0
+    traffic = (measured_traffic("gemm_tc.cu", "tc_gemm_llama2_7b_ffn_bf16.md")
+               if gemm_cls == "gemm_tc" else None)
     roof = {"kernel": gemm_cls, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"],
-            "unit": "TFLOP/s", "frac": achieved / pk["bf16"], "traffic": None,
+            "unit": "TFLOP/s", "frac": achieved / pk["bf16"], "traffic": traffic,
             "peak_kind": f"bf16 burst, {pk['src']}",
             "frac_of_sustained": achieved / pk["bf16_sus"],
             "flops_per_launch": fl_g / max(n_g, 1), "ms_per_launch": ms_g / max(n_g, 1)}
