@@ -455,6 +455,321 @@ __global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__
   }
 }
 
+
+// ------------------------------------------------------------------------
+// 2-CTA variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16).  Each CTA loads only
+// its own operand halves: its 128 rows of A and its 128 rows (or two 64-wide
+// MN atoms) of B, so shared-memory traffic per SM per MMA is 8 KB instead of
+// 12 KB.  The leader CTA (rank 0) arms the stage barrier for both CTAs'
+// bytes; the peer's TMA loads complete on the leader's barrier
+// (.cta_group::2).  The leader's single MMA thread issues the MMAs and its
+// commits arrive on both CTAs' barriers (multicast commit).  Each CTA's
+// epilogue drains its own 128 TMEM lanes and signals the leader.  No TMA
+// multicast is used.
+namespace {
+constexpr int STAGES2 = 6;
+constexpr int A2_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int B2_BYTES = (BN / 2) * BK * 2;           // 16 KB (this CTA's half)
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;     // 32 KB
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2sm(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
+                                             int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4_2sm(void* dst, const CUtensorMap* m,
+                                                uint32_t bar_cluster, int x, int r0, int r1,
+                                                int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_2sm(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                             uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Commit the leader's MMAs; the arrival lands on the barrier at the same
+// offset in both CTAs of the pair.
+__device__ __forceinline__ void mma_commit_2sm(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(su32(bar)), "h"(uint16_t(3))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+}  // namespace
+
+__global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw2[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES2 * STAGE2_BYTES);
+  uint64_t* empty = full + STAGES2;
+  uint64_t* tfull = empty + STAGES2;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);  // four epilogue warps in each CTA of the pair
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     su32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote signal
+  fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const int n_mpairs = (p.n_mtiles + 1) / 2;
+  const int total = n_mpairs * p.n_ntiles;
+  const int cluster_id = blockIdx.x / 2, n_clusters = gridDim.x / 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int t = cluster_id; t < total && ok; t += n_clusters) {
+      const int mp = t % n_mpairs, nt = t / n_mpairs;
+      const int mt = 2 * mp + int(rank);
+      int a_row = 0;
+      if (mt < p.n_mtiles) {
+        const int4 tl = p.tiles[mt];
+        a_row = p.a_compact ? tl.y : tl.x;
+      }
+      const int n0 = nt * (p.paired ? BN / 2 : BN);
+      for (int s = 0; s < p.nseg && ok; ++s) {
+        const int mode = p.bmode[s];
+        const int32_t* idx = p.idx[s];
+        const int nidx = p.nidx[s];
+        const CUtensorMap* bm = &p.bmap[s][p.bpair[s] ? rank : 0];
+        // this CTA's 128 B rows start at
+        const int brow0 = p.bpair[s] ? n0 : nt * BN + 128 * int(rank);
+        int krow[4];
+        if (mode == B_K_GATHER) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            int n = brow0 + 4 * lane + q;
+            n = n < nidx ? n : nidx - 1;
+            krow[q] = __ldg(idx + n);
+          }
+        }
+        for (int kb = 0; kb < p.nkb[s]; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) { ok = false; break; }
+          const uint32_t fbar = map_to_rank(su32(&full[stage]), 0);
+          if (leader && lane == 0) mbar_expect_tx(&full[stage], 2 * STAGE2_BYTES);
+          __syncwarp();
+          uint8_t* sa = smem + stage * STAGE2_BYTES;
+          uint8_t* sb = sa + A2_BYTES;
+          if (lane == 0) tma_load_2sm(sa, &p.amap[s], fbar, kb * BK, a_row);
+          if (mode == B_K) {
+            if (lane == 1) tma_load_2sm(sb, bm, fbar, kb * BK, brow0);
+          } else if (mode == B_K_GATHER) {
+            tma_gather4_2sm(sb + lane * 512, bm, fbar, kb * BK, krow[0], krow[1], krow[2],
+                            krow[3]);
+          } else if (mode == B_MN) {
+            if (lane < 2)
+              tma_load_2sm(sb + lane * 8192, bm, fbar, n0 + 64 * (2 * int(rank) + lane), kb * BK);
+          } else {  // B_MN_GATHER
+            const int al = lane / 16, grp = lane % 16;
+            int r4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              int k = kb * BK + 4 * grp + q;
+              k = k < nidx ? k : nidx - 1;
+              r4[q] = __ldg(idx + k);
+            }
+            tma_gather4_2sm(sb + al * 8192 + grp * 512, bm, fbar,
+                            n0 + 64 * (2 * int(rank) + al), r4[0], r4[1], r4[2], r4[3]);
+          }
+          ++issued;
+          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+    if (!ok && leader && lane == 0) {
+      // let the copies already armed land before the CTA can exit
+      int st2 = stage;
+      uint32_t ph2 = phase;
+      for (int i = 0; i < STAGES2 && i < issued; ++i) {
+        if (--st2 < 0) { st2 = STAGES2 - 1; ph2 ^= 1u; }
+        const long long t0 = clock64();
+        while (!mbar_try(&full[st2], ph2) && clock64() - t0 < WAIT_BUDGET) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA (leader CTA only)
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < total && ok; t += n_clusters, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = uint32_t(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort)) break;
+        fence_after();
+        const uint32_t d = tbase + uint32_t(acc * BN);
+        bool first = true;
+        for (int s = 0; s < p.nseg && ok; ++s) {
+          const int bmn = p.bmode[s] >= B_MN;
+          const uint32_t idesc = idesc_bf16(2 * BM, BN, bmn);
+          for (int kb = 0; kb < p.nkb[s]; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
+            fence_after();
+            const uint32_t sa = su32(smem + stage * STAGE2_BYTES);
+            const uint32_t sb = sa + A2_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = sdesc(sa + k * 32, 16, 1024);
+              const uint64_t bd = bmn ? sdesc(sb + k * 2048, 8192, 1024) : sdesc(sb + k * 32, 16, 1024);
+              mma_bf16_2sm(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+            }
+            first = false;
+            mma_commit_2sm(&empty[stage]);
+            if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+          }
+        }
+        mma_commit_2sm(&tfull[acc]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - 4;
+    const int r = q * 32 + lane;  // row within this CTA's 128-row half == TMEM lane
+    const uint32_t tempty_leader0 = map_to_rank(su32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = map_to_rank(su32(&tempty[1]), 0);
+    int it = 0;
+    for (int t = cluster_id; t < total; t += n_clusters, ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = uint32_t(it >> 1) & 1u;
+      if (!mbar_wait(&tfull[acc], aph, abort)) break;
+      fence_after();
+      const int mp = t % n_mpairs, nt = t / n_mpairs;
+      const int mt = 2 * mp + int(rank);
+      int out_row = 0, nvalid = 0;
+      if (mt < p.n_mtiles) {
+        const int4 tl = p.tiles[mt];
+        out_row = p.out_compact ? tl.y : tl.x;
+        nvalid = tl.z;
+      }
+      const int n0 = nt * (p.paired ? BN / 2 : BN);
+      const bool valid = r < nvalid;
+      const int64_t orow = int64_t(out_row) + r;
+      const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+      float v[32], w[32];
+      if (p.epi == EPI_SWIGLU_FWD) {
+        __nv_bfloat16* g = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+        __nv_bfloat16* u = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out2) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tl + c * 32, v);
+          tmem_ld32(tl + 128 + c * 32, w);
+          if (valid) {
+            const int c0 = n0 + c * 32;
+            store_row32(g, c0, p.N, v);
+            store_row32(u, c0, p.N, w);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]) * w[j];
+            store_row32(h, c0, p.N, v);
+          }
+        }
+      } else if (p.epi == EPI_SWIGLU_BWD) {
+        const __nv_bfloat16* gi = static_cast<const __nv_bfloat16*>(p.in0) + orow * p.ldi;
+        const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
+        __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+        __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          tmem_ld32(tl + c * 32, v);  // dh
+          const int c0 = n0 + c * 32;
+          if (valid && c0 < p.N) {
+            float gv[32];
+            load_row32(gi, c0, p.N, gv);
+            load_row32(ui, c0, p.N, w);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float sg = sigmoid_f(gv[j]);
+              const float dh = v[j];
+              v[j] = dh * w[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
+              w[j] = dh * gv[j] * sg;                                 // dU
+            }
+            store_row32(dg, c0, p.N, v);
+            store_row32(du, c0, p.N, w);
+          }
+        }
+      } else {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          tmem_ld32(tl + c * 32, v);
+          const int c0 = n0 + c * 32;
+          if (valid && c0 < p.N) store_row32(o, c0, p.N, v, p.vec_out != 0);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the pair's MMAs, loads and remote arrivals are all finished
+  if (warp == 2) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;" ::"r"(tbase) : "memory");
+  }
+}
+
 // ----------------------------------------------------------- host helpers
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -492,6 +807,8 @@ slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y) {
 }
 
 bool g_attr_set = false;
+// 1: one-CTA 128x256 tiles; 2: two-CTA (cluster pair) 256x256 tiles.
+int g_tc_mode = 2;
 
 }  // namespace
 
@@ -565,7 +882,30 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   if (!g_attr_set) {
     SLORA_CUDA(cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     SMEM_BYTES));
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    SMEM2_BYTES));
     g_attr_set = true;
+  }
+  if (g_tc_mode == 2) {
+    const int64_t ctiles = int64_t((p.n_mtiles + 1) / 2) * p.n_ntiles;
+    const int64_t maxc = num_sms() / 2;
+    const int nclus = int(ctiles < maxc ? ctiles : maxc);
+    LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum),
+                   st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(2 * nclus), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel, p));
+    return SLORA_OK;
   }
   const int64_t tiles = int64_t(p.n_mtiles) * p.n_ntiles;
   const int grid = int(tiles < num_sms() ? tiles : num_sms());
@@ -575,6 +915,9 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
+
+void set_tc_mode(int mode) { g_tc_mode = mode == 1 ? 1 : 2; }
+int tc_mode() { return g_tc_mode; }
 
 slora_status tc_check_error(bool clear) {
   int v = 0;

@@ -66,6 +66,11 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st);
 // Device error flag of the tcgen05 kernels (a bounded wait that expired).
 slora_status tc_check_error(bool clear);
 
+// Tile variant of the tcgen05 GEMM: 1 = one-CTA 128x256 tiles, 2 = cluster
+// pairs with cta_group::2 256x256 tiles (default).
+void set_tc_mode(int mode);
+int tc_mode();
+
 // Number of SMs of the current device (cached).
 int num_sms();
 
