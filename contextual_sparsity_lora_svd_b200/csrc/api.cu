@@ -110,15 +110,12 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
                                   int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
                                   int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
                                   cudaStream_t st, bool has_pre, const float* P_pre,
-                                  int64_t ldp_pre) {
+                                  int64_t ldp_pre, unsigned* counters) {
   (void)tok;
   float* P = has_pre ? nullptr : ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
   float* ppart = (!has_pre && dt == kBF16)
                      ? ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)))
                      : nullptr;
-  void* prs = (!has_pre && dt == kBF16)
-                  ? static_cast<void*>(ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(d))))
-                  : nullptr;
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
   float* scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
   const int nsplit = ffn_score_splits(ti.T_C, n0);
@@ -142,7 +139,8 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
       rr.qsplit = rank; rr.ptr_b = L1; rr.dt_b = kF32; rr.si_b = rank; rr.sq_b = 1;
       SkRowOut o;
       o.out1 = P; o.ld1 = 2 * rank;
-      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, prs, st));
+      if (!counters) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "estimator: counter workspace missing");
+      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, counters, st));
     } else {  // fp32 activations: CUDA-core fp32 FMA
       for (int p = 0; p < 2; ++p) {
         GemmArgs g;
@@ -203,8 +201,10 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
       SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0/n1 must be heads*head_dim / kv_heads*head_dim", fn);
     kkeep = keep_count(head_dim, sparsity);
   }
+  const int64_t ncnt = skinny_counter_count(ti.T_C, d);
   Arena plan;
   plan.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  plan.take<unsigned>(size_t(ncnt));
   SLORA_TRY(estimate_select_body(crit, X, dt, tok, ti, nullptr, d, L0, U0, n0, L1, U1, rank,
                                  heads, kv_heads, head_dim, kkeep, idx_out, scores_out, plan,
                                  true, nullptr));
@@ -217,9 +217,11 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
   Arena ar;
   ar.base = static_cast<char*>(ws);
   int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st));
+  unsigned* cnt = ar.take<unsigned>(size_t(ncnt));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st, nullptr, nullptr, cnt, ncnt));
   return estimate_select_body(crit, X, dt, tok, ti, ctx_rows, d, L0, U0, n0, L1, U1, rank, heads,
-                              kv_heads, head_dim, kkeep, idx_out, scores_out, ar, false, st);
+                              kv_heads, head_dim, kkeep, idx_out, scores_out, ar, false, st,
+                              false, nullptr, 0, cnt);
 }
 
 // ------------------------------------------------------------ linear calls

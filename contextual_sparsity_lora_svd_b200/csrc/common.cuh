@@ -83,7 +83,8 @@ slora_status parse_tokens(const slora_tokens* tok, TokenInfo* info);
 // tile never crossing a sequence.
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles = nullptr,
-                            int4* out_tiles = nullptr);
+                            int4* out_tiles = nullptr, unsigned* zero = nullptr,
+                            int64_t nzero = 0);
 // Number of 128-row tiles of the context rows / output rows.
 int64_t count_tiles(const slora_tokens* tok, bool ctx);
 inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }

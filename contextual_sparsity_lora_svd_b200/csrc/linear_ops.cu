@@ -280,13 +280,14 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       npart = std::max(npart, coldot_part_floats(M, K, 2 * r));
     }
   float* part = ar.take<float>(size_t(npart));
-  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, d, Fd}))));
+  const int64_t ncnt = skinny_counter_count(std::max({T, d, Fd}), std::max({T, d, Fd}));
+  unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   if (!idx_force)
     SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
                                    L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
-                                   true, nullptr, fused, Pfull, 2 * rs));
+                                   true, nullptr, fused, Pfull, 2 * rs, rsp));
   if (plan) return SLORA_OK;
 
   auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
@@ -296,7 +297,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
   };
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
   SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
   {  // one stream over X: XA = X [Ag; Au]^T (fp32 and s*XA bf16) and, for the
      // estimator, P = X [Lg | Lu] (fp32-accurate, read for the context rows)
@@ -319,7 +320,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   } else {
     SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
                                    L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
-                                   false, st, fused, Pfull, 2 * rs));
+                                   false, st, fused, Pfull, 2 * rs, rsp));
   }
   // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
   SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st));
@@ -650,10 +651,11 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   void* WS = bf(ni, outr ? k : n);  // rows idx of W (W0 or W0^T)
   void* Xpad = (!none && !outr && ni % 8) ? bf(TC, ldi) : nullptr;  // X_ctx with 16-byte rows
   float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
-  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
+  unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   if (plan) return SLORA_OK;
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
   SLORA_TRY(gather_pad(L.B, r, nullptr, n, r, Bp, lr, st));
   if (none || outr) {
     SkRowOut o;
@@ -744,10 +746,11 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   void* dYpad = (outr && ni % 8) ? bf(TC, ldi) : nullptr;
   void* Xpad = (!none && !outr && ni % 8) ? bf(TC, ldi) : nullptr;
   float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
-  void* rsp = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
+  unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   if (plan) return SLORA_OK;
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
   if (none) {
     SkRowOut o;
     o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;

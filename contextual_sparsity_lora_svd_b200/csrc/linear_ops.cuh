@@ -48,6 +48,7 @@ slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
                                   int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
                                   int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
                                   cudaStream_t st, bool has_pre = false,
-                                  const float* P_pre = nullptr, int64_t ldp_pre = 0);
+                                  const float* P_pre = nullptr, int64_t ldp_pre = 0,
+                                  unsigned* counters = nullptr);
 
 }  // namespace slora

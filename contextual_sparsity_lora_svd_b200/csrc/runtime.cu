@@ -21,7 +21,10 @@ __global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
                                                       int32_t* __restrict__ ctx_rows,
                                                       int32_t* __restrict__ out_rows,
                                                       int4* __restrict__ ctx_tiles,
-                                                      int4* __restrict__ out_tiles) {
+                                                      int4* __restrict__ out_tiles,
+                                                      unsigned* __restrict__ zero,
+                                                      int64_t nzero) {
+  for (int64_t i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
   __shared__ int ctx_off[kMaxBatch], ct_off[kMaxBatch], ot_off[kMaxBatch];
   if (threadIdx.x == 0) {
     int acc = 0, ct = 0, ot = 0;
@@ -120,13 +123,14 @@ int64_t count_tiles(const slora_tokens* tok, bool ctx) {
 
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles,
-                            int4* out_tiles) {
+                            int4* out_tiles, unsigned* zero, int64_t nzero) {
   RowmapParams p;
   p.batch = ti.batch;
   p.seq = ti.seq;
   for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
   LaunchScope ls(kAux, double(ti.T) * 4, st);
-  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles);
+  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles, zero,
+                                    zero ? nzero : 0);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

@@ -68,14 +68,14 @@ struct SkColOut {
 };
 
 // c = number of R columns (1..64).  part: fp32 workspace of *_part_floats();
-// rsplit: bf16 workspace of skinny_rsplit_elems(I) elements, I = K (rowdot) or
-// M (coldot), holding the pre-split rank-sized operand.
+// counters: skinny_counter_count(M, K) unsigned ints that are zero on entry
+// (the kernels leave them zero again).
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c);
 int64_t coldot_part_floats(int64_t M, int64_t K, int c);
-int64_t skinny_rsplit_elems(int64_t I);
+int64_t skinny_counter_count(int64_t M, int64_t K);
 slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
-                    const SkRowOut& o, float* part, void* rsplit, cudaStream_t st);
+                    const SkRowOut& o, float* part, unsigned* counters, cudaStream_t st);
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
-                    const SkColOut& o, float* part, void* rsplit, cudaStream_t st);
+                    const SkColOut& o, float* part, unsigned* counters, cudaStream_t st);
 
 }  // namespace slora
