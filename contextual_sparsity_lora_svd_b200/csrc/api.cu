@@ -94,38 +94,43 @@ extern "C" slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, s
   SLORA_TRY(check_device());
   Arena ar;
   ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
   return svd_prepare_impl(W, n, k, dt, rank, n_iter, seed, L, U, W_t, ar, false,
                           static_cast<cudaStream_t>(stream));
 }
 
 // --------------------------------------------------------- estimate+select
 namespace slora {
-// Estimator body shared with the FFN call.  Writes idx (see slora.h layout).
-// With P_pre the low-rank projection of the context rows is already
-// available (full row layout, row t of the context set at P_pre[ctx_rows[t]]).
-slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
-                                  const slora_tokens* tok, const TokenInfo& ti,
-                                  const int32_t* ctx_rows, int64_t d, const float* L0,
-                                  const float* U0, int64_t n0, const float* L1, const float* U1,
-                                  int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
-                                  int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
-                                  cudaStream_t st, bool has_pre, const float* P_pre,
-                                  int64_t ldp_pre, unsigned* counters) {
-  (void)tok;
-  float* P = has_pre ? nullptr : ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
-  float* ppart = (!has_pre && dt == kBF16)
-                     ? ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)))
-                     : nullptr;
+EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int64_t d, int64_t n0,
+                         int rank, int kv_heads, int head_dim, bool has_pre, float* scores_out,
+                         Arena& ar) {
+  EstBufs eb;
+  if (!has_pre) eb.P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
+  if (!has_pre && dt == kBF16)
+    eb.ppart = ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)));
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
-  float* scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
-  const int nsplit = ffn_score_splits(ti.T_C, n0);
-  float* partial = nullptr;
-  double* gram = nullptr;
+  eb.scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
+  eb.nsplit = ffn_score_splits(ti.T_C, n0);
   if (crit == SLORA_CRIT_FFN_SWIGLU_L2)
-    partial = ar.take<float>(size_t(nsplit) * n0);
+    eb.partial = ar.take<float>(size_t(eb.nsplit) * n0);
   else
-    gram = ar.take<double>(size_t(2) * rank * rank * 33);
-  if (plan) return SLORA_OK;
+    eb.gram = ar.take<double>(size_t(2) * rank * rank * 33);
+  return eb;
+}
+
+slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
+                                    const TokenInfo& ti, const int32_t* ctx_rows, int64_t d,
+                                    const float* L0, const float* U0, int64_t n0, const float* L1,
+                                    const float* U1, int rank, int heads, int kv_heads,
+                                    int head_dim, int64_t kkeep, int32_t* idx_out,
+                                    const EstBufs& eb, cudaStream_t st, bool has_pre,
+                                    const float* P_pre, int64_t ldp_pre, unsigned* counters) {
+  float* P = eb.P;
+  float* ppart = eb.ppart;
+  float* scores = eb.scores;
+  float* partial = eb.partial;
+  double* gram = eb.gram;
+  const int nsplit = eb.nsplit;
   const float* Puse = P_pre;
   int64_t ldp = ldp_pre;
   const int32_t* pmap = has_pre ? ctx_rows : nullptr;
@@ -202,26 +207,22 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
     kkeep = keep_count(head_dim, sparsity);
   }
   const int64_t ncnt = skinny_counter_count(ti.T_C, d);
-  Arena plan;
-  plan.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
-  plan.take<unsigned>(size_t(ncnt));
-  SLORA_TRY(estimate_select_body(crit, X, dt, tok, ti, nullptr, d, L0, U0, n0, L1, U1, rank,
-                                 heads, kv_heads, head_dim, kkeep, idx_out, scores_out, plan,
-                                 true, nullptr));
+  Arena ar;  // one pass: sizes the query and places the buffers (finish_ws checks the size)
+  ar.base = static_cast<char*>(ws);
+  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
+  unsigned* cnt = ar.take<unsigned>(size_t(ncnt));
+  const EstBufs eb = estimate_reserve(crit, dt, ti, d, n0, rank, kv_heads, head_dim, false,
+                                      scores_out, ar);
   const bool query = ws == nullptr;
-  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  SLORA_TRY(finish_ws(fn, ar, ws, ws_bytes));
   *k_out = int32_t(kkeep);
   if (query) return SLORA_OK;
   SLORA_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Arena ar;
-  ar.base = static_cast<char*>(ws);
-  int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
-  unsigned* cnt = ar.take<unsigned>(size_t(ncnt));
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st, nullptr, nullptr, cnt, ncnt));
-  return estimate_select_body(crit, X, dt, tok, ti, ctx_rows, d, L0, U0, n0, L1, U1, rank, heads,
-                              kv_heads, head_dim, kkeep, idx_out, scores_out, ar, false, st,
-                              false, nullptr, 0, cnt);
+  return estimate_select_launch(crit, X, dt, ti, ctx_rows, d, L0, U0, n0, L1, U1, rank, heads,
+                                kv_heads, head_dim, kkeep, idx_out, eb, st, false, nullptr, 0,
+                                cnt);
 }
 
 // ------------------------------------------------------------ linear calls
@@ -271,6 +272,7 @@ extern "C" slora_status slora_linear_fwd(slora_dtype dt, const slora_tokens* tok
   SLORA_TRY(check_device());
   Arena ar;
   ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
   return linear_fwd_run(L, tok, X_ctx, X_out, Y_ctx, Y_out, XA_save, ar, false,
                         static_cast<cudaStream_t>(stream));
 }
@@ -301,6 +303,7 @@ extern "C" slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok
   SLORA_TRY(check_device());
   Arena ar;
   ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
   return linear_bwd_run(L, tok, X_ctx, X_out, XA_save, dY_ctx, dY_out, dX_ctx, dX_out, dA, dB, ar,
                         false, static_cast<cudaStream_t>(stream));
 }
@@ -353,6 +356,7 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   SLORA_TRY(check_device());
   Arena ar;
   ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
   return ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, ar, false,
                  static_cast<cudaStream_t>(stream));
 }

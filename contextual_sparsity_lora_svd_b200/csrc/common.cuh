@@ -52,10 +52,14 @@ void clear_error();
 
 // ------------------------------------------------------------- workspace
 // Bump allocator over the caller's workspace.  With base == nullptr it only
-// counts bytes (the workspace-size query).
+// counts bytes (the workspace-size query).  A run path takes every buffer it
+// needs before its first launch and then calls fits(): the planning pass and
+// the run pass must take the same sequence, and fits() turns any mismatch
+// into an error before a kernel could touch memory past the workspace.
 struct Arena {
   char* base = nullptr;
   size_t used = 0;
+  size_t cap = ~size_t(0);  // bytes of the caller's workspace (run pass)
   template <class T>
   T* take(size_t count) {
     size_t off = (used + 255) & ~size_t(255);
@@ -63,6 +67,7 @@ struct Arena {
     return base ? reinterpret_cast<T*>(base + off) : nullptr;
   }
 };
+slora_status arena_fits(const Arena& ar, const char* where);
 
 // ------------------------------------------------------------- devices
 slora_status check_device();  // sm_100 present and current

@@ -54,6 +54,7 @@ slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const 
   int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_O, 1)));
   float* XA = XA_save ? XA_save : ar.take<float>(size_t(ti.T) * r);
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "workspace"));
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
 
   if (L.side == SLORA_SLICE_NONE) {
@@ -115,6 +116,7 @@ slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const 
   int32_t* out_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_O, 1)));
   float* dYB = ar.take<float>(size_t(ti.T) * r);  // dY B per row, full row layout
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "workspace"));
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
 
   if (L.side == SLORA_SLICE_NONE) {
@@ -284,11 +286,11 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
+  EstBufs eb;
   if (!idx_force)
-    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
-                                   true, nullptr, fused, Pfull, 2 * rs, rsp));
+    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, rs, 0, 0, fused, nullptr, ar);
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
   auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
     SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
@@ -318,17 +320,17 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
                                  cudaMemcpyDeviceToDevice, st));
   } else {
-    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, nullptr, ar,
-                                   false, st, fused, Pfull, 2 * rs, rsp));
+    SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
+                                     L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, eb, st, fused,
+                                     Pfull, 2 * rs, rsp));
   }
   // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
-  SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st));
-  SLORA_TRY(gather_rows(L.Wu, d, idx, kk, d, WuS, d, st));
-  SLORA_TRY(gather_rows(L.Wd_t, d, idx, kk, d, WdS, d, st));
+  SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st, Fd));
+  SLORA_TRY(gather_rows(L.Wu, d, idx, kk, d, WuS, d, st, Fd));
+  SLORA_TRY(gather_rows(L.Wd_t, d, idx, kk, d, WdS, d, st, Fd));
   // LoRA operand packing (bf16, tiny)
-  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, st));
-  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, st));
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, st, Fd));
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, st, Fd));
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, st));
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, st));
   SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
@@ -478,11 +480,12 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
   void* hO = buf(TO, Fd);
   void* dGO = buf(TO, Fd);
   void* dUO = buf(TO, Fd);
+  EstBufs eb;
   if (!idx_force)
-    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
-                                   true, nullptr));
+    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, L.r_svd, 0, 0, false, nullptr,
+                          ar);
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
   if (idx_force) {
@@ -490,10 +493,8 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
       SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
                                  cudaMemcpyDeviceToDevice, st));
   } else {
-    // same arena offsets as the plan: the estimator's scratch follows the buffers above
-    SLORA_TRY(estimate_select_body(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, tok, ti, ctx_rows, d, L.Lg,
-                                   L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, nullptr, ar,
-                                   false, st));
+    SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
+                                     L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, eb, st));
   }
 
   // ---- forward
@@ -654,9 +655,10 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "workspace"));
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
-  SLORA_TRY(gather_pad(L.B, r, nullptr, n, r, Bp, lr, st));
+  SLORA_TRY(gather_pad(L.B, r, nullptr, n, r, Bp, lr, st, n));
   if (none || outr) {
     SkRowOut o;
     o.out1 = XA; o.ld1 = r; o.out2 = XAb; o.ld2 = lr; o.s2 = s;
@@ -671,8 +673,8 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     return gemm_tc(b.g, st);
   }
   if (outr) {
-    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st));
-    SLORA_TRY(gather_pad(L.B, r, L.idx, ni, r, BS, lr, st));
+    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
+    SLORA_TRY(gather_pad(L.B, r, L.idx, ni, r, BS, lr, st, n));
     {  // context rows, output channels S
       TcBuilder b(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
       b.seg(mat(X_ctx, T, k, k), mat(WS, ni, k, k), B_K, k)
@@ -690,7 +692,7 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   const void* Xc = X_ctx;
   int64_t ldxc = ni;
   if (Xpad) {
-    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st));
+    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st, TC));
     Xc = Xpad;
     ldxc = ldi;
   }
@@ -702,7 +704,7 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     oo.out1 = XA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = XAbO; oo.ld2 = lr; oo.s2 = s;
     SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, part, rsp, st));
   }
-  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st));
+  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
   {
     TcBuilder b(ctiles, nct, 1, 0, TC, n, 0, EPI_STORE);
     b.seg(mat(Xc, TC, ni, ldxc), mat(WS, ni, n, n), B_MN, ni)
@@ -749,6 +751,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "workspace"));
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
   if (none) {
@@ -772,7 +775,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     const void* dYc = dY_ctx;
     int64_t lddc = ni;
     if (dYpad) {
-      SLORA_TRY(gather_pad(dY_ctx, ni, nullptr, TC, ni, dYpad, ldi, st));
+      SLORA_TRY(gather_pad(dY_ctx, ni, nullptr, TC, ni, dYpad, ldi, st, TC));
       dYc = dYpad;
       lddc = ldi;
     }
@@ -793,7 +796,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
       SLORA_TRY(coldot(ykv(dYc, lddc), TC, ni, rkv(XA, kF32, r, 1, ctx_rows), r, bc, part, rsp,
                        st));
     }
-    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st));
+    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
     {  // dX, context rows: dY_C W0[S] + s dYB_C A
       TcBuilder b(ctiles, nct, 1, 0, TC, k, 0, EPI_STORE);
       b.seg(mat(dYc, TC, ni, lddc), mat(WS, ni, k, k), B_MN, ni)
@@ -816,7 +819,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   const void* Xc = X_ctx;
   int64_t ldxc = ni;
   if (Xpad) {
-    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st));
+    SLORA_TRY(gather_pad(X_ctx, ni, nullptr, TC, ni, Xpad, ldi, st, TC));
     Xc = Xpad;
     ldxc = ldi;
   }
@@ -825,7 +828,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
     SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, part, rsp, st));
   }
-  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st));
+  SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
   SLORA_TRY(transpose_rows(L.A, r, k, L.idx, ni, lr, AS, st));
   SLORA_TRY(transpose_rows(L.A, r, k, nullptr, k, lr, At, st));
   {  // dX_ctx = dY_C W0[:, S] + s dYB_C A[:, S]

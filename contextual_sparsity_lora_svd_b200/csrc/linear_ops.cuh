@@ -40,15 +40,30 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
                      void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
                      bool plan, cudaStream_t st);
 
-// Estimator body (estimate + select) shared by slora_estimate_select and the FFN call.
-slora_status estimate_select_body(slora_criterion crit, const void* X, int dt,
-                                  const slora_tokens* tok, const TokenInfo& ti,
-                                  const int32_t* ctx_rows, int64_t d, const float* L0,
-                                  const float* U0, int64_t n0, const float* L1, const float* U1,
-                                  int rank, int heads, int kv_heads, int head_dim, int64_t kkeep,
-                                  int32_t* idx_out, float* scores_out, Arena& ar, bool plan,
-                                  cudaStream_t st, bool has_pre = false,
-                                  const float* P_pre = nullptr, int64_t ldp_pre = 0,
-                                  unsigned* counters = nullptr);
+// Estimator (estimate + select) shared by slora_estimate_select and the FFN
+// call, in two steps so that a run path can take all of its workspace before
+// its first launch: estimate_reserve takes the scratch buffers from the arena
+// (nothing is launched), estimate_select_launch runs the kernels on them.
+struct EstBufs {
+  float* P = nullptr;        // X_C [L0 | L1] (when not supplied precomputed)
+  float* ppart = nullptr;    // split partials of that projection (bf16 path)
+  float* scores = nullptr;   // per-channel scores (the caller's scores_out when given)
+  float* partial = nullptr;  // FFN score partials over token chunks
+  double* gram = nullptr;    // q/k Gram matrices and their partials
+  int nsplit = 1;
+};
+EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int64_t d, int64_t n0,
+                         int rank, int kv_heads, int head_dim, bool has_pre, float* scores_out,
+                         Arena& ar);
+// With has_pre the low-rank projection of the context rows is already
+// available (full row layout, row t of the context set at P_pre[ctx_rows[t]]).
+slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
+                                    const TokenInfo& ti, const int32_t* ctx_rows, int64_t d,
+                                    const float* L0, const float* U0, int64_t n0, const float* L1,
+                                    const float* U1, int rank, int heads, int kv_heads,
+                                    int head_dim, int64_t kkeep, int32_t* idx_out,
+                                    const EstBufs& eb, cudaStream_t st, bool has_pre = false,
+                                    const float* P_pre = nullptr, int64_t ldp_pre = 0,
+                                    unsigned* counters = nullptr);
 
 }  // namespace slora

@@ -11,10 +11,20 @@
 namespace slora {
 namespace {
 
+// Raised by a gather that met an index outside its source (the row is read as
+// zeros instead); read and cleared by pack_check_error.
+__device__ int g_pack_bad_index = 0;
+__device__ __forceinline__ bool index_ok(int64_t v, int64_t n) {
+  if (v >= 0 && v < n) return true;
+  atomicExch(&g_pack_bad_index, 1);
+  return false;
+}
+
 __global__ void pack_gate_up_b_kernel(const __nv_bfloat16* __restrict__ Bg,
                                       const __nv_bfloat16* __restrict__ Bu,
                                       const int32_t* __restrict__ idx, int64_t N, int r,
-                                      int64_t rows, int64_t ldo, __nv_bfloat16* __restrict__ out) {
+                                      int64_t rows, int64_t ldo, int64_t rows_src,
+                                      __nv_bfloat16* __restrict__ out) {
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= rows * ldo) return;
   const int64_t R = e / ldo;
@@ -25,7 +35,7 @@ __global__ void pack_gate_up_b_kernel(const __nv_bfloat16* __restrict__ Bg,
   float v = 0.0f;
   if (c < N && col >= h * r && col < (h + 1) * r) {
     const int64_t src = idx ? idx[c] : c;
-    v = __bfloat162float((h ? Bu : Bg)[src * r + (col - h * r)]);
+    if (index_ok(src, rows_src)) v = __bfloat162float((h ? Bu : Bg)[src * r + (col - h * r)]);
   }
   out[e] = __float2bfloat16_rn(v);
 }
@@ -37,18 +47,19 @@ __global__ void transpose_rows_kernel(const __nv_bfloat16* __restrict__ in, int6
   if (e >= n * ldo) return;
   const int64_t c = e / ldo, q = e % ldo;
   const int64_t src = idx ? int64_t(idx[c]) : c;
-  out[e] = q < rows ? in[q * cols + src] : __float2bfloat16_rn(0.0f);
+  out[e] = (q < rows && index_ok(src, cols)) ? in[q * cols + src] : __float2bfloat16_rn(0.0f);
 }
 
 // One block per selected row and 2048-element column chunk; 16-byte copies.
 __global__ void gather_rows_kernel(const uint4* __restrict__ in, int64_t ld_in16,
-                                   const int32_t* __restrict__ idx, int64_t cols16,
-                                   uint4* __restrict__ out, int64_t ld_out16) {
+                                   const int32_t* __restrict__ idx, int64_t rows_in,
+                                   int64_t cols16, uint4* __restrict__ out, int64_t ld_out16) {
   const int64_t j = blockIdx.x;
   const int64_t src = idx[j];
+  const bool ok = index_ok(src, rows_in);
   for (int64_t c = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; c < cols16;
        c += int64_t(gridDim.y) * blockDim.x)
-    out[j * ld_out16 + c] = __ldg(in + src * ld_in16 + c);
+    out[j * ld_out16 + c] = ok ? __ldg(in + src * ld_in16 + c) : make_uint4(0, 0, 0, 0);
 }
 
 __global__ void stack_rows_kernel(const __nv_bfloat16* __restrict__ top,
@@ -81,12 +92,12 @@ __global__ void concat_cols_kernel(const float* __restrict__ a, const float* __r
 
 __global__ void gather_pad_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in,
                                   const int32_t* __restrict__ idx, int64_t n, int64_t cols,
-                                  int64_t ldo, __nv_bfloat16* __restrict__ out) {
+                                  int64_t ldo, int64_t rows_in, __nv_bfloat16* __restrict__ out) {
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= n * ldo) return;
   const int64_t j = e / ldo, c = e % ldo;
   const int64_t src = idx ? int64_t(idx[j]) : j;
-  out[e] = c < cols ? in[src * ld_in + c] : __float2bfloat16_rn(0.0f);
+  out[e] = (c < cols && index_ok(src, rows_in)) ? in[src * ld_in + c] : __float2bfloat16_rn(0.0f);
 }
 
 __global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t nt) {
@@ -102,13 +113,14 @@ unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
 }  // namespace
 
 slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, int64_t N, int r,
-                            int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st) {
+                            int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st,
+                            int64_t rows_src) {
   const int64_t rows = n_ntiles * 256;
   if (rows <= 0) return SLORA_OK;
   LaunchScope ls(kAux, double(rows) * ldo * 2 + double(N) * 2 * r * 2, st);
   pack_gate_up_b_kernel<<<blocks(rows * ldo), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(Bg), static_cast<const __nv_bfloat16*>(Bu), idx, N, r,
-      rows, ldo, static_cast<__nv_bfloat16*>(out));
+      rows, ldo, rows_src, static_cast<__nv_bfloat16*>(out));
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
@@ -125,7 +137,8 @@ slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const in
 }
 
 slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
-                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st) {
+                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st,
+                         int64_t rows_in) {
   if (n <= 0) return SLORA_OK;
   if (cols % 8 || ld_in % 8 || ld_out % 8)
     SLORA_FAIL(SLORA_ERR_ALIGN, "gather_rows: rows must be whole 16-byte units");
@@ -134,7 +147,8 @@ slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int6
   if (n > 2147483647) SLORA_FAIL(SLORA_ERR_SHAPE, "gather_rows: too many rows");
   LaunchScope ls(kCompact, 2.0 * double(n) * cols * 2, st);
   gather_rows_kernel<<<dim3(unsigned(n), gy), 256, 0, st>>>(
-      static_cast<const uint4*>(in), ld_in / 8, idx, c16, static_cast<uint4*>(out), ld_out / 8);
+      static_cast<const uint4*>(in), ld_in / 8, idx, rows_in, c16, static_cast<uint4*>(out),
+      ld_out / 8);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
@@ -158,11 +172,11 @@ slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64
 }
 
 slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
-                        int64_t cols, void* out, int64_t ldo, cudaStream_t st) {
+                        int64_t cols, void* out, int64_t ldo, cudaStream_t st, int64_t rows_in) {
   if (n <= 0) return SLORA_OK;
   LaunchScope ls(kAux, double(n) * (cols + ldo) * 2, st);
   gather_pad_kernel<<<blocks(n * ldo), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), ld_in,
-                                                     idx, n, cols, ldo,
+                                                     idx, n, cols, ldo, rows_in,
                                                      static_cast<__nv_bfloat16*>(out));
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
@@ -183,6 +197,17 @@ slora_status copy_pad(const void* in, int64_t rows, int64_t cols, int64_t ldo, v
   copy_pad_kernel<<<blocks(rows * ldo), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(in), rows,
                                                       cols, ldo, static_cast<__nv_bfloat16*>(out));
   SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status pack_check_error(bool clear) {
+  int v = 0;
+  SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_pack_bad_index, sizeof(int)));
+  if (clear && v) {
+    const int z = 0;
+    SLORA_CUDA(cudaMemcpyToSymbol(g_pack_bad_index, &z, sizeof(int)));
+  }
+  if (v) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "a gather met a channel index outside its weight");
   return SLORA_OK;
 }
 

@@ -4,16 +4,21 @@
 namespace slora {
 // out [n_ntiles*256 x ldo]: tile nt rows 0..127 = [Bg[c] | 0], rows 128..255 =
 // [0 | Bu[c]] for channels c = nt*128 + j (idx[c] if idx), zero past N.
+// rows_src: rows of Bg/Bu (valid channel indices are [0, rows_src)).
 slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, int64_t N, int r,
-                            int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st);
+                            int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st,
+                            int64_t rows_src);
 // out [n x ldo] with out[c][q] = in[q][idx ? idx[c] : c] (in is rows x cols,
 // n = number of output rows), zero columns past `rows`.
 slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const int32_t* idx,
                             int64_t n, int64_t ldo, void* out, cudaStream_t st);
 // Compaction of selected rows: out[j][:] = in[idx[j]][:] for j < n (bf16,
 // rows of `cols` elements, cols a multiple of 8, leading dimensions ld_in/ld_out).
+// rows_in: rows of `in`; an index outside [0, rows_in) yields a zero row and
+// raises the flag that pack_check_error reads.
 slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
-                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st);
+                         int64_t cols, void* out, int64_t ld_out, cudaStream_t st,
+                         int64_t rows_in);
 // out [(rows_top + rows_bottom) x cols] = [top; bottom].
 slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
                         int64_t rows_bottom, int64_t cols, void* out, cudaStream_t st);
@@ -26,7 +31,11 @@ slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64
 // out [n x ldo] bf16 = rows (idx ? idx[j] : j) of in [* x ld_in], first `cols`
 // columns, zero padded to ldo.
 slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
-                        int64_t cols, void* out, int64_t ldo, cudaStream_t st);
+                        int64_t cols, void* out, int64_t ldo, cudaStream_t st, int64_t rows_in);
+// Reads (and with `clear` resets) the flag the gathers above raise when an
+// index lies outside their source; SLORA_ERR_INVALID_ARG if it was raised.
+// Synchronous: waits for the device.
+slora_status pack_check_error(bool clear);
 // M-tile list {row0, row0, nvalid, 0} covering rows [0, M) in 128-row tiles.
 slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st);
 }  // namespace slora

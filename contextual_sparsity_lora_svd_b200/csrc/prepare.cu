@@ -242,6 +242,7 @@ slora_status svd_prepare_impl(const void* W, int64_t n, int64_t k, int dt, int r
   pb.E = ar.take<float>(size_t(b) * b);
   pb.lam = ar.take<float>(size_t(b));
   if (plan_only) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "slora_svd_prepare"));
 
   static bool attr_done = false;
   if (!attr_done) {

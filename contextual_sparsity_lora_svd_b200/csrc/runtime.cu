@@ -3,6 +3,8 @@
 #include <vector>
 
 #include "common.cuh"
+#include "gemm_tc.cuh"
+#include "lora_pack.cuh"
 
 namespace slora {
 
@@ -77,6 +79,13 @@ void set_error(const char* fmt, ...) {
 
 void clear_error() { g_error.clear(); }
 
+slora_status arena_fits(const Arena& ar, const char* where) {
+  if (ar.used > ar.cap)
+    SLORA_FAIL(SLORA_ERR_WORKSPACE, "%s: internal error: the run takes %zu workspace bytes, the "
+               "plan gave %zu", where, ar.used, ar.cap);
+  return SLORA_OK;
+}
+
 slora_status check_device() {
   int dev = -1;
   SLORA_CUDA(cudaGetDevice(&dev));
@@ -140,6 +149,16 @@ slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_
 extern "C" const char* slora_last_error_string(void) { return slora::g_error.c_str(); }
 
 extern "C" int slora_version(void) { return 100; }
+
+extern "C" slora_status slora_device_error(int clear) {
+  using namespace slora;
+  clear_error();
+  const slora_status a = pack_check_error(clear != 0);
+  const std::string first = a != SLORA_OK ? g_error : std::string();
+  const slora_status b = tc_check_error(clear != 0);
+  if (a != SLORA_OK) g_error = first;
+  return a != SLORA_OK ? a : b;
+}
 
 // ------------------------------------------------------------ launch record
 namespace slora {

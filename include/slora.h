@@ -88,6 +88,18 @@ const char* slora_last_error_string(void);
 int slora_version(void);
 
 /*
+ * Errors that kernels record on the device instead of faulting (not part of
+ * the method): a gather of selected weight rows that met a channel index
+ * outside the weight (the row is read as zeros), or a tensor-core pipeline
+ * wait that gave up.  Waits for the current device to finish its work, then
+ * returns SLORA_ERR_INVALID_ARG (bad index), SLORA_ERR_TIMEOUT (wait expired) or
+ * SLORA_OK; clear != 0 resets the recorded state.  Index lists that callers
+ * pass (idx, idx_force) must hold in-range channels: only the gathers check,
+ * the other kernels that read through an index list trust it.
+ */
+slora_status slora_device_error(int clear);
+
+/*
  * Launch accounting and optional per-kernel timing (not part of the method;
  * used to measure it).
  *   slora_launch_count()   kernels this library has launched in this process.
