@@ -106,8 +106,10 @@ EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int6
                          Arena& ar) {
   EstBufs eb;
   if (!has_pre) eb.P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
-  if (!has_pre && dt == kBF16)
+  if (!has_pre && dt == kBF16) {
     eb.ppart = ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)));
+    eb.prs = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(d)));
+  }
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
   eb.scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
   eb.nsplit = ffn_score_splits(ti.T_C, n0);
@@ -145,7 +147,11 @@ slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
       SkRowOut o;
       o.out1 = P; o.ld1 = 2 * rank;
       if (!counters) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "estimator: counter workspace missing");
-      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, ppart, counters, st));
+      SkWork w;
+      w.part = ppart;
+      w.rsplit = eb.prs;
+      w.counters = counters;
+      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, w, st));
     } else {  // fp32 activations: CUDA-core fp32 FMA
       for (int p = 0; p < 2; ++p) {
         GemmArgs g;

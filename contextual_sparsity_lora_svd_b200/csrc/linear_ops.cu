@@ -277,13 +277,18 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   const bool fused = !idx_force && 2 * r + 2 * rs <= 64;  // one pass over X for XA and P
   int64_t npart = 1;
   for (int64_t M : {T, TC, TO})
-    for (int64_t K : {d, kk, Fd}) {
-      npart = std::max(npart, rowdot_part_floats(M, K, fused ? 2 * r + 2 * rs : 2 * r));
-      npart = std::max(npart, coldot_part_floats(M, K, 2 * r));
-    }
+    for (int64_t K : {d, kk, Fd})
+      for (int c : {r, 2 * r, fused ? 2 * r + 2 * rs : 2 * r}) {
+        npart = std::max(npart, rowdot_part_floats(M, K, c));
+        npart = std::max(npart, coldot_part_floats(M, K, c));
+      }
   float* part = ar.take<float>(size_t(npart));
   const int64_t ncnt = skinny_counter_count(std::max({T, d, Fd}), std::max({T, d, Fd}));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
+  SkWork sw;
+  sw.part = part;
+  sw.rsplit = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, d, Fd}))));
+  sw.counters = rsp;
   float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   EstBufs eb;
@@ -313,7 +318,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       o.qsplit = 2 * r; o.out1b = Pfull; o.ld1b = 2 * rs;
       c = 2 * r + 2 * rs;
     }
-    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, sw, st));
   }
   if (idx_force) {
     if (kk > 0)
@@ -353,10 +358,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
     SkRowOut oc;
     oc.out1 = hA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = hAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, sw, st));
     SkRowOut oo;
     oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, sw, st));
   }
   {  // down projection, context rows: reads channels S only (rows S of Wd^T)
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -377,10 +382,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dOB = dOut Bd: fp32 and s*dOB bf16; dBd = s dOut^T hA (same stream of dOut)
     SkRowOut o;
     o.out1 = dOB; o.ld1 = r; o.out2 = dOBb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, sw, st));
     SkColOut c;
     c.out = G.dBd; c.ldo = r; c.scale = s;
-    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, part, rsp, st));
+    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, sw, st));
   }
   {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
@@ -401,10 +406,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
     SkColOut co;
     co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
-    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, part, rsp, st));
+    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, sw, st));
     SkColOut cc = co;
     cc.kmap = idx; cc.accumulate = 1;
-    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, part, rsp, st));
+    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, sw, st));
   }
   for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]; dB = s dG^T XA on the same stream
     const void* Bm = p ? L.Bu : L.Bg;
@@ -412,18 +417,18 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkRowOut oo;
     oo.out1 = dGB; oo.ld1 = 2 * r; oo.off1 = p * r; oo.map1 = out_rows;
     oo.out2 = dGBbO; oo.ld2 = lr2; oo.off2 = p * r; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, sw, st));
     SkColOut bo;
     bo.out = dBm; bo.ldo = r; bo.scale = s;
     SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
-                     bo, part, rsp, st));
+                     bo, sw, st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
-    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, part, rsp, st));
+    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, sw, st));
     SkColOut bc = bo;
     bc.kmap = idx; bc.accumulate = 1;
     SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
-                     bc, part, rsp, st));
+                     bc, sw, st));
   }
   {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -444,7 +449,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAg | dAu = s dGB^T X over every row, one stream of X
     SkColOut c;
     c.out = G.dAg; c.out_b = G.dAu; c.qsplit = r; c.ldo = d; c.trans = 1; c.scale = s;
-    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, part, rsp, st));
+    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, sw, st));
   }
   return SLORA_OK;
 }
@@ -654,6 +659,10 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
   const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
+  SkWork sw;
+  sw.part = part;
+  sw.rsplit = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  sw.counters = rsp;
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "workspace"));
 
@@ -662,7 +671,7 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   if (none || outr) {
     SkRowOut o;
     o.out1 = XA; o.ld1 = r; o.out2 = XAb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(ykv(X_ctx, k), T, k, rkv(L.A, kBF16, 1, k), r, o, part, rsp, st));
+    SLORA_TRY(rowdot(ykv(X_ctx, k), T, k, rkv(L.A, kBF16, 1, k), r, o, sw, st));
   }
   if (none) {
     SLORA_TRY(make_plain_tiles(ptiles, T, st));
@@ -699,10 +708,10 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   {
     SkRowOut oc;
     oc.out1 = XA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = XAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(ykv(Xc, ldxc), TC, ni, rkv(L.A, kBF16, 1, k, L.idx), r, oc, part, rsp, st));
+    SLORA_TRY(rowdot(ykv(Xc, ldxc), TC, ni, rkv(L.A, kBF16, 1, k, L.idx), r, oc, sw, st));
     SkRowOut oo;
     oo.out1 = XA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = XAbO; oo.ld2 = lr; oo.s2 = s;
-    SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, part, rsp, st));
+    SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, sw, st));
   }
   SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
   {
@@ -750,6 +759,10 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   float* part = ar.take<float>(size_t(skinny_part_bound(ti, k, n, ni, r)));
   const int64_t ncnt = skinny_counter_count(std::max({T, k, n}), std::max({T, k, n}));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
+  SkWork sw;
+  sw.part = part;
+  sw.rsplit = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
+  sw.counters = rsp;
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "workspace"));
 
@@ -757,7 +770,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   if (none) {
     SkRowOut o;
     o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, part, rsp, st));
+    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, sw, st));
     SLORA_TRY(make_plain_tiles(ptiles, T, st));
     TcBuilder b(ptiles, (T + 127) / 128, 0, 0, T, k, 0, EPI_STORE);
     b.seg(mat(dY_ctx, T, n, n), mat(L.W, n, k, k), B_MN, n)
@@ -766,10 +779,10 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     SLORA_TRY(gemm_tc(b.g, st));
     SkColOut ca;
     ca.out = dA; ca.ldo = k; ca.trans = 1; ca.scale = s;
-    SLORA_TRY(coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, part, rsp, st));
+    SLORA_TRY(coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, sw, st));
     SkColOut cb;
     cb.out = dB; cb.ldo = r; cb.scale = s;
-    return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, part, rsp, st);
+    return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, sw, st);
   }
   if (outr) {
     const void* dYc = dY_ctx;
@@ -782,18 +795,18 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     {  // dYB = dY B on the rows' channels; dB = s dY^T XA (output rows first, then += S rows)
       SkRowOut oc;
       oc.out1 = dYB; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = dYBbC; oc.ld2 = lr; oc.s2 = s;
-      SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx), r, oc, part, rsp,
+      SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx), r, oc, sw,
                        st));
       SkRowOut oo;
       oo.out1 = dYB; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = dYBbO; oo.ld2 = lr; oo.s2 = s;
-      SLORA_TRY(rowdot(ykv(dY_out, n), TO, n, rkv(L.B, kBF16, r, 1), r, oo, part, rsp, st));
+      SLORA_TRY(rowdot(ykv(dY_out, n), TO, n, rkv(L.B, kBF16, r, 1), r, oo, sw, st));
       SkColOut bo;
       bo.out = dB; bo.ldo = r; bo.scale = s;
-      SLORA_TRY(coldot(ykv(dY_out, n), TO, n, rkv(XA, kF32, r, 1, out_rows), r, bo, part, rsp,
+      SLORA_TRY(coldot(ykv(dY_out, n), TO, n, rkv(XA, kF32, r, 1, out_rows), r, bo, sw,
                        st));
       SkColOut bc = bo;
       bc.kmap = L.idx; bc.accumulate = 1;
-      SLORA_TRY(coldot(ykv(dYc, lddc), TC, ni, rkv(XA, kF32, r, 1, ctx_rows), r, bc, part, rsp,
+      SLORA_TRY(coldot(ykv(dYc, lddc), TC, ni, rkv(XA, kF32, r, 1, ctx_rows), r, bc, sw,
                        st));
     }
     SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
@@ -813,7 +826,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     }
     SkColOut ca;  // dA = s dYB^T X over every row
     ca.out = dA; ca.ldo = k; ca.trans = 1; ca.scale = s;
-    return coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, part, rsp, st);
+    return coldot(ykv(X_ctx, k), T, k, rkv(dYB, kF32, r, 1), r, ca, sw, st);
   }
   // IN_COLS: W = W0^T [k x n]; dY is the full T x n gradient
   const void* Xc = X_ctx;
@@ -826,7 +839,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   {
     SkRowOut o;
     o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, part, rsp, st));
+    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, sw, st));
   }
   SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
   SLORA_TRY(transpose_rows(L.A, r, k, L.idx, ni, lr, AS, st));
@@ -848,14 +861,14 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   {  // dA: output rows over every column, then += context rows on columns S
     SkColOut ao;
     ao.out = dA; ao.ldo = k; ao.trans = 1; ao.scale = s;
-    SLORA_TRY(coldot(ykv(X_out, k), TO, k, rkv(dYB, kF32, r, 1, out_rows), r, ao, part, rsp, st));
+    SLORA_TRY(coldot(ykv(X_out, k), TO, k, rkv(dYB, kF32, r, 1, out_rows), r, ao, sw, st));
     SkColOut ac = ao;
     ac.kmap = L.idx; ac.accumulate = 1;
-    SLORA_TRY(coldot(ykv(Xc, ldxc), TC, ni, rkv(dYB, kF32, r, 1, ctx_rows), r, ac, part, rsp, st));
+    SLORA_TRY(coldot(ykv(Xc, ldxc), TC, ni, rkv(dYB, kF32, r, 1, ctx_rows), r, ac, sw, st));
   }
   SkColOut cb;  // dB = s dY^T XA over every row
   cb.out = dB; cb.ldo = r; cb.scale = s;
-  return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, part, rsp, st);
+  return coldot(ykv(dY_ctx, n), T, n, rkv(XA, kF32, r, 1), r, cb, sw, st);
 }
 
 }  // namespace slora

@@ -47,6 +47,7 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
 struct EstBufs {
   float* P = nullptr;        // X_C [L0 | L1] (when not supplied precomputed)
   float* ppart = nullptr;    // split partials of that projection (bf16 path)
+  void* prs = nullptr;       // bf16 terms of [L0 | L1] for that projection (bf16 path)
   float* scores = nullptr;   // per-channel scores (the caller's scores_out when given)
   float* partial = nullptr;  // FFN score partials over token chunks
   double* gram = nullptr;    // q/k Gram matrices and their partials

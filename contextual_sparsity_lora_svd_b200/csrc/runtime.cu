@@ -5,6 +5,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "lora_pack.cuh"
+#include "skinny.cuh"
 
 namespace slora {
 
@@ -156,8 +157,11 @@ extern "C" slora_status slora_device_error(int clear) {
   const slora_status a = pack_check_error(clear != 0);
   const std::string first = a != SLORA_OK ? g_error : std::string();
   const slora_status b = tc_check_error(clear != 0);
+  const std::string second = b != SLORA_OK ? g_error : std::string();
+  const slora_status c = skinny_check_error(clear != 0);
   if (a != SLORA_OK) g_error = first;
-  return a != SLORA_OK ? a : b;
+  else if (b != SLORA_OK) g_error = second;
+  return a != SLORA_OK ? a : (b != SLORA_OK ? b : c);
 }
 
 // ------------------------------------------------------------ launch record

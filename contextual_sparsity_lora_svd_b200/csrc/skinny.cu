@@ -1,15 +1,30 @@
 // Skinny (rank-sized) contractions, see skinny.cuh.
 //
-// 128-thread blocks over 64 x 64 tiles of Y staged in shared memory with
-// cp.async (zero-filled past the edges, optional row gather); the rank-sized
-// operand is staged transposed as 1 or 3 bf16 terms.  Each warp owns 16 rows
-// (rowdot) or 16 columns (coldot) of the tile and issues mma.sync m16n8k16
-// (bf16 in, fp32 accumulate).  The rank-sized operand is loaded one chunk
-// ahead into registers and split on the fly.  Many small blocks per SM keep
-// the HBM stream of Y busy; partial sums over the split dimension go to a
-// workspace and the last block of each output block (atomic ticket) reduces
-// them in a fixed order and writes the outputs: one launch per contraction,
-// bit-reproducible results.
+// 128-thread blocks over 64 x 64 tiles of Y staged in shared memory by a 3-
+// or 4-stage cp.async pipeline (zero-filled past the edges, optional row
+// gather).  The rank-sized operand is split into NT bf16 terms once per call
+// (prep_r_kernel, laid out [term][column][index] so each stage copies it with
+// 16-byte cp.async) and staged beside Y.  Each warp owns 16 rows (rowdot) or
+// 16 columns (coldot) of the tile and issues mma.sync m16n8k16 (bf16 in, fp32
+// accumulate).  With a split over the reduced dimension, each block writes its
+// partial tile to a workspace and the last block of the output block to arrive
+// (atomic ticket) sums the partials in split order and writes the outputs:
+// bit-reproducible, no second launch.
+//
+// When Y is a plain strided matrix (no row gather) a second kernel takes the
+// contraction: a persistent, stream-K style grid of exactly one wave.  The
+// flattened (output block x reduction chunk) space is cut into one contiguous,
+// equal slice per CTA; each CTA streams its slice through a TMA ring of
+// 128-byte-swizzled 64 x 64 tiles of Y (plus the matching tile of the split
+// operand) completed on mbarriers, with fragments read by ldmatrix.  A block
+// covered by one CTA alone is written directly from its accumulators; a block
+// shared by several CTAs gets their partial tiles summed in CTA order by the
+// last one to finish.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "skinny.cuh"
 
 namespace slora {
@@ -22,8 +37,12 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, int bytes
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -72,6 +91,49 @@ __device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
   return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[off]);
 }
 
+// Pre-split of the rank-sized operand, once per call: RS[s][q][i] = term s of
+// R(i, q) (zero for q >= c or i >= I), rows of I64 = roundup(I, 64) elements.
+// Threads walk the source's contiguous index so the reads coalesce.
+template <int NT>
+__global__ void prep_r_kernel(const SkR R, int c, int CP, int64_t I, int64_t I64,
+                              __nv_bfloat16* __restrict__ RS) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= int64_t(CP) * I64) return;
+  const bool q_fast = R.sq == 1 && (R.ptr_b == nullptr || R.sq_b == 1);
+  int q;
+  int64_t i;
+  if (q_fast) {
+    q = int(e % CP);
+    i = e / CP;
+  } else {
+    q = int(e / I64);
+    i = e % I64;
+  }
+  const float v = (q < c && i < I) ? load_r(R, i, q) : 0.0f;
+  __nv_bfloat16 tv[3];
+  split_terms<NT>(v, tv);
+#pragma unroll
+  for (int s = 0; s < NT; ++s) RS[(int64_t(s) * CP + q) * I64 + i] = tv[s];
+}
+
+// Pipeline depth from the shared memory of one stage (Y tile + split R tile).
+constexpr int stage_bytes(int CP, int NT) { return TILE * PAD * 2 + NT * CP * PAD * 2; }
+constexpr int stages_for(int CP, int NT) { return stage_bytes(CP, NT) <= 16896 ? 4 : 3; }
+constexpr int smem_for(int CP, int NT) { return stages_for(CP, NT) * stage_bytes(CP, NT); }
+
+// Stage RS[:, :, i0 .. i0+64) into Rs[s][q][0..64) with 16-byte async copies.
+template <int CP, int NT>
+__device__ __forceinline__ void stage_r(__nv_bfloat16 (*Rs)[CP][PAD],
+                                        const __nv_bfloat16* __restrict__ RS, int64_t I64,
+                                        int64_t i0, int tid) {
+#pragma unroll
+  for (int e = tid; e < NT * CP * 8; e += NTH) {
+    const int seg = e & 7, row = e >> 3;  // row = s * CP + q
+    const int sidx = row / CP, q = row % CP;
+    cp_async16(&Rs[sidx][q][seg * 8], RS + int64_t(row) * I64 + i0 + seg * 8, 16);
+  }
+}
+
 // Stage the 64 x 64 tile of Y at (m0, k0) into Ys (rows m, columns k).
 __device__ __forceinline__ void stage_y(__nv_bfloat16 (*Ys)[PAD], const SkY& Y, int64_t M,
                                         int64_t K, int64_t m0, int64_t k0, int tid) {
@@ -89,50 +151,6 @@ __device__ __forceinline__ void stage_y(__nv_bfloat16 (*Ys)[PAD], const SkY& Y, 
       src = base + (Y.map ? int64_t(Y.map[m]) : m) * Y.ld + k;
     }
     cp_async16(&Ys[row][c8], src, bytes);
-  }
-}
-
-// The rank-sized operand for chunk rows [i0, i0 + 64): each thread holds
-// CP * 64 / NTH values in registers (loaded one chunk ahead) and stores their
-// NT-term split transposed into Rs[s][q][i].  Lanes walk q when q is the
-// contiguous index of the source, otherwise i.
-template <int CP>
-struct RRegs {
-  float v[CP * TILE / NTH];
-};
-template <int CP>
-__device__ __forceinline__ void rmap(const SkR& R, int e, int& q, int& ii) {
-  const bool q_fast = R.sq == 1 && (R.ptr_b == nullptr || R.sq_b == 1);
-  if (q_fast) {
-    q = e % CP;
-    ii = e / CP;
-  } else {
-    q = e / TILE;
-    ii = e % TILE;
-  }
-}
-template <int CP>
-__device__ __forceinline__ void load_r_regs(RRegs<CP>& rg, const SkR& R, int c, int64_t i0,
-                                            int64_t I, int tid) {
-#pragma unroll
-  for (int j = 0; j < CP * TILE / NTH; ++j) {
-    int q, ii;
-    rmap<CP>(R, tid + NTH * j, q, ii);
-    const int64_t i = i0 + ii;
-    rg.v[j] = (q < c && i < I) ? load_r(R, i, q) : 0.0f;
-  }
-}
-template <int CP, int NT>
-__device__ __forceinline__ void store_r_regs(__nv_bfloat16 (*Rs)[CP][PAD], const RRegs<CP>& rg,
-                                             const SkR& R, int tid) {
-#pragma unroll
-  for (int j = 0; j < CP * TILE / NTH; ++j) {
-    int q, ii;
-    rmap<CP>(R, tid + NTH * j, q, ii);
-    __nv_bfloat16 tv[3];
-    split_terms<NT>(rg.v[j], tv);
-#pragma unroll
-    for (int s = 0; s < NT; ++s) Rs[s][q][ii] = tv[s];
   }
 }
 
@@ -157,10 +175,25 @@ __device__ __forceinline__ void col_emit(const SkColOut& o, int64_t k, int q, fl
   *dst = o.accumulate ? *dst + v : v;
 }
 
-// cp.async double buffering: chunk j+1 is in flight while chunk j is consumed.
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_one() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
+// Fixed-order sum over the splits of 4 consecutive partial columns:
+// src[s * stride4] for s = 0 .. nsplit-1, eight loads in flight at a time.
+__device__ __forceinline__ float4 sum_splits4(const float4* src, int64_t stride4, int nsplit) {
+  float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  int s = 0;
+  for (; s + 8 <= nsplit; s += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (s + u) * stride4);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      a.x += v[u].x; a.y += v[u].y; a.z += v[u].z; a.w += v[u].w;
+    }
+  }
+  for (; s < nsplit; ++s) {
+    const float4 v = __ldcg(src + s * stride4);
+    a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+  }
+  return a;
 }
 
 // Returns true in the one CTA (of the `n` sharing `counter`) that arrives last,
@@ -179,59 +212,77 @@ __device__ __forceinline__ bool last_arrival(unsigned* counter, unsigned n, int 
   return s_last != 0;
 }
 
+// Partial tile of a warp's 16 x CP accumulators (rows / columns `r0`, `r0+8`
+// of the output block) at part[(split * nout + r) * CP + col].
+template <int NF>
+__device__ __forceinline__ void store_partial(float* part, int split, int64_t nout, int64_t r0,
+                                              int t, const float (*acc)[4]) {
+  constexpr int CP = NF * 8;
+#pragma unroll
+  for (int f = 0; f < NF; ++f) {
+    const int col = f * 8 + 2 * t;
+    if (r0 < nout)
+      *reinterpret_cast<float2*>(part + (int64_t(split) * nout + r0) * CP + col) =
+          make_float2(acc[f][0], acc[f][1]);
+    if (r0 + 8 < nout)
+      *reinterpret_cast<float2*>(part + (int64_t(split) * nout + r0 + 8) * CP + col) =
+          make_float2(acc[f][2], acc[f][3]);
+  }
+}
+
 template <int NF, int NT>
 __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int64_t K,
-                                                     const SkR R, int c, int chunks_per_split,
+                                                     const __nv_bfloat16* __restrict__ RS,
+                                                     int64_t I64, int c, int chunks_per_split,
                                                      float* __restrict__ part,
                                                      unsigned* __restrict__ counters,
                                                      const SkRowOut o) {
-  constexpr int CP = NF * 8;
+  constexpr int CP = NF * 8, S = stages_for(CP, NT);
   extern __shared__ __align__(16) unsigned char sk_smem[];
-  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [2][TILE][PAD]
-  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + 2 * TILE * PAD * 2);
+  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [S][TILE][PAD]
+  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + S * TILE * PAD * 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t m0 = int64_t(blockIdx.x) * TILE;
   const int ks = blockIdx.y, nsplit = gridDim.y;
   const int64_t nchunks = (K + TILE - 1) / TILE;
   const int64_t kc0 = int64_t(ks) * chunks_per_split;
-  const int64_t kc1 = kc0 + chunks_per_split < nchunks ? kc0 + chunks_per_split : nchunks;
+  const int n = int((kc0 + chunks_per_split < nchunks ? kc0 + chunks_per_split : nchunks) - kc0);
   float acc[NF][4];
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
-  RRegs<CP> rg;
-  if (kc0 < kc1) {
-    stage_y(Ys[0], Y, M, K, m0, kc0 * TILE, tid);
-    load_r_regs<CP>(rg, R, c, kc0 * TILE, K, tid);
-    store_r_regs<CP, NT>(Rs[0], rg, R, tid);
-  }
-  cp_async_commit();
-  int buf = 0;
-  for (int64_t kc = kc0; kc < kc1; ++kc, buf ^= 1) {
-    const bool more = kc + 1 < kc1;
-    if (more) {
-      stage_y(Ys[buf ^ 1], Y, M, K, m0, (kc + 1) * TILE, tid);
-      load_r_regs<CP>(rg, R, c, (kc + 1) * TILE, K, tid);
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (j < n) {
+      stage_y(Ys[j], Y, M, K, m0, (kc0 + j) * TILE, tid);
+      stage_r<CP, NT>(Rs[j], RS, I64, (kc0 + j) * TILE, tid);
     }
     cp_async_commit();
-    cp_async_wait_one();
-    __syncthreads();
-    const int r0 = warp * 16 + g;
+  }
+  const int r0 = warp * 16 + g;
+  for (int j = 0; j < n; ++j) {
+    cp_async_wait<S - 2>();
+    __syncthreads();  // chunk j landed; every warp is done with chunk j-1's slot
+    const int jn = j + S - 1;
+    if (jn < n) {
+      stage_y(Ys[jn % S], Y, M, K, m0, (kc0 + jn) * TILE, tid);
+      stage_r<CP, NT>(Rs[jn % S], RS, I64, (kc0 + jn) * TILE, tid);
+    }
+    cp_async_commit();
+    const int b = j % S;
 #pragma unroll
     for (int k16 = 0; k16 < TILE / 16; ++k16) {
       const int kb = k16 * 16 + 2 * t;
-      const uint32_t a0 = lds32(&Ys[buf][r0][kb]), a1 = lds32(&Ys[buf][r0 + 8][kb]);
-      const uint32_t a2 = lds32(&Ys[buf][r0][kb + 8]), a3 = lds32(&Ys[buf][r0 + 8][kb + 8]);
+      const uint32_t a0 = lds32(&Ys[b][r0][kb]), a1 = lds32(&Ys[b][r0 + 8][kb]);
+      const uint32_t a2 = lds32(&Ys[b][r0][kb + 8]), a3 = lds32(&Ys[b][r0 + 8][kb + 8]);
 #pragma unroll
       for (int f = 0; f < NF; ++f)
 #pragma unroll
         for (int s = 0; s < NT; ++s)
-          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[buf][s][f * 8 + g][kb]),
-                   lds32(&Rs[buf][s][f * 8 + g][kb + 8]));
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[b][s][f * 8 + g][kb]),
+                   lds32(&Rs[b][s][f * 8 + g][kb + 8]));
     }
-    __syncthreads();
-    if (more) store_r_regs<CP, NT>(Rs[buf ^ 1], rg, R, tid);
   }
-  const int64_t row0 = m0 + warp * 16 + g;
+  const int64_t row0 = m0 + r0;
   if (nsplit == 1) {  // no split: emit straight from the accumulators
 #pragma unroll
     for (int f = 0; f < NF; ++f) {
@@ -247,85 +298,76 @@ __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int
     }
     return;
   }
-#pragma unroll
-  for (int f = 0; f < NF; ++f) {
-    const int col = f * 8 + 2 * t;
-    if (row0 < M) {
-      float* p = part + (int64_t(ks) * M + row0) * CP + col;
-      p[0] = acc[f][0];
-      p[1] = acc[f][1];
-    }
-    if (row0 + 8 < M) {
-      float* p = part + (int64_t(ks) * M + row0 + 8) * CP + col;
-      p[0] = acc[f][2];
-      p[1] = acc[f][3];
-    }
-  }
+  store_partial<NF>(part, ks, M, row0, t, acc);
   if (!last_arrival(counters + blockIdx.x, unsigned(nsplit), tid)) return;
-  for (int e = tid; e < TILE * c; e += NTH) {
-    const int64_t m = m0 + e / c;
-    const int q = e % c;
+  const int nq4 = (c + 3) / 4;
+  for (int e = tid; e < TILE * nq4; e += NTH) {
+    const int64_t m = m0 + e / nq4;
+    const int q0 = (e % nq4) * 4;
     if (m >= M) continue;
-    float v = 0.0f;
-    for (int s2 = 0; s2 < nsplit; ++s2) v += __ldcg(part + (int64_t(s2) * M + m) * CP + q);
-    row_emit(o, m, q, v);
+    const float4 v = sum_splits4(reinterpret_cast<const float4*>(part + m * CP + q0),
+                                 M * CP / 4, nsplit);
+    row_emit(o, m, q0, v.x);
+    if (q0 + 1 < c) row_emit(o, m, q0 + 1, v.y);
+    if (q0 + 2 < c) row_emit(o, m, q0 + 2, v.z);
+    if (q0 + 3 < c) row_emit(o, m, q0 + 3, v.w);
   }
 }
 
 template <int NF, int NT>
 __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int64_t K,
-                                                     const SkR R, int c, int chunks_per_split,
+                                                     const __nv_bfloat16* __restrict__ RS,
+                                                     int64_t I64, int c, int chunks_per_split,
                                                      float* __restrict__ part,
                                                      unsigned* __restrict__ counters,
                                                      const SkColOut o) {
-  constexpr int CP = NF * 8;
+  constexpr int CP = NF * 8, S = stages_for(CP, NT);
   extern __shared__ __align__(16) unsigned char sk_smem[];
-  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [2][TILE][PAD]
-  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + 2 * TILE * PAD * 2);
+  auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [S][TILE][PAD]
+  auto Rs = reinterpret_cast<__nv_bfloat16 (*)[NT][CP][PAD]>(sk_smem + S * TILE * PAD * 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t k0 = int64_t(blockIdx.x) * TILE;
   const int ms = blockIdx.y, nsplit = gridDim.y;
   const int64_t nchunks = (M + TILE - 1) / TILE;
   const int64_t mc0 = int64_t(ms) * chunks_per_split;
-  const int64_t mc1 = mc0 + chunks_per_split < nchunks ? mc0 + chunks_per_split : nchunks;
+  const int n = int((mc0 + chunks_per_split < nchunks ? mc0 + chunks_per_split : nchunks) - mc0);
   float acc[NF][4];
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
   const int mq = lane >> 3, rr = lane & 7;  // ldmatrix: matrix index, row within it
-  RRegs<CP> rg;
-  if (mc0 < mc1) {
-    stage_y(Ys[0], Y, M, K, mc0 * TILE, k0, tid);
-    load_r_regs<CP>(rg, R, c, mc0 * TILE, M, tid);
-    store_r_regs<CP, NT>(Rs[0], rg, R, tid);
-  }
-  cp_async_commit();
-  int buf = 0;
-  for (int64_t mc = mc0; mc < mc1; ++mc, buf ^= 1) {
-    const bool more = mc + 1 < mc1;
-    if (more) {
-      stage_y(Ys[buf ^ 1], Y, M, K, (mc + 1) * TILE, k0, tid);
-      load_r_regs<CP>(rg, R, c, (mc + 1) * TILE, M, tid);
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (j < n) {
+      stage_y(Ys[j], Y, M, K, (mc0 + j) * TILE, k0, tid);
+      stage_r<CP, NT>(Rs[j], RS, I64, (mc0 + j) * TILE, tid);
     }
     cp_async_commit();
-    cp_async_wait_one();
+  }
+  for (int j = 0; j < n; ++j) {
+    cp_async_wait<S - 2>();
     __syncthreads();
+    const int jn = j + S - 1;
+    if (jn < n) {
+      stage_y(Ys[jn % S], Y, M, K, (mc0 + jn) * TILE, k0, tid);
+      stage_r<CP, NT>(Rs[jn % S], RS, I64, (mc0 + jn) * TILE, tid);
+    }
+    cp_async_commit();
+    const int b = j % S;
 #pragma unroll
     for (int m16 = 0; m16 < TILE / 16; ++m16) {
       // A = Y^T fragment (16 k x 16 m) for columns warp*16.. of the tile
       const int mb = m16 * 16 + (mq >> 1) * 8;
       const int kb = warp * 16 + (mq & 1) * 8;
       uint32_t a0, a1, a2, a3;
-      ldsm_x4_trans(a0, a1, a2, a3, &Ys[buf][mb + rr][kb]);
+      ldsm_x4_trans(a0, a1, a2, a3, &Ys[b][mb + rr][kb]);
       const int mcol = m16 * 16 + 2 * t;
 #pragma unroll
       for (int f = 0; f < NF; ++f)
 #pragma unroll
         for (int s = 0; s < NT; ++s)
-          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[buf][s][f * 8 + g][mcol]),
-                   lds32(&Rs[buf][s][f * 8 + g][mcol + 8]));
+          mma16816(acc[f], a0, a1, a2, a3, lds32(&Rs[b][s][f * 8 + g][mcol]),
+                   lds32(&Rs[b][s][f * 8 + g][mcol + 8]));
     }
-    __syncthreads();
-    if (more) store_r_regs<CP, NT>(Rs[buf ^ 1], rg, R, tid);
   }
   const int64_t kr = k0 + warp * 16 + g;
   if (nsplit == 1) {
@@ -343,37 +385,38 @@ __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int
     }
     return;
   }
-#pragma unroll
-  for (int f = 0; f < NF; ++f) {
-    const int col = f * 8 + 2 * t;
-    if (kr < K) {
-      float* p = part + (int64_t(ms) * K + kr) * CP + col;
-      p[0] = acc[f][0];
-      p[1] = acc[f][1];
-    }
-    if (kr + 8 < K) {
-      float* p = part + (int64_t(ms) * K + kr + 8) * CP + col;
-      p[0] = acc[f][2];
-      p[1] = acc[f][3];
-    }
-  }
+  store_partial<NF>(part, ms, K, kr, t, acc);
   if (!last_arrival(counters + blockIdx.x, unsigned(nsplit), tid)) return;
-  for (int e = tid; e < TILE * c; e += NTH) {
-    const int64_t k = k0 + e / c;
-    const int q = e % c;
+  const int nq4 = (c + 3) / 4;
+  for (int e = tid; e < TILE * nq4; e += NTH) {
+    const int64_t k = k0 + e / nq4;
+    const int q0 = (e % nq4) * 4;
     if (k >= K) continue;
-    float v = 0.0f;
-    for (int s2 = 0; s2 < nsplit; ++s2) v += __ldcg(part + (int64_t(s2) * K + k) * CP + q);
-    col_emit(o, k, q, v);
+    const float4 v = sum_splits4(reinterpret_cast<const float4*>(part + k * CP + q0),
+                                 K * CP / 4, nsplit);
+    col_emit(o, k, q0, v.x);
+    if (q0 + 1 < c) col_emit(o, k, q0 + 1, v.y);
+    if (q0 + 2 < c) col_emit(o, k, q0 + 2, v.z);
+    if (q0 + 3 < c) col_emit(o, k, q0 + 3, v.w);
   }
 }
 
-constexpr int kTargetBlocks = 148 * 8;
+// One full wave of resident blocks: the shared memory of a block bounds how
+// many fit on an SM (each keeps S-1 chunks of Y in flight).  The SM count is
+// the B200's, a constant, so the workspace query needs no device.
+constexpr int kSMs = 148;
+int64_t target_blocks(int CP, int NT) {
+  int per_sm = (200 * 1024) / smem_for(CP, NT);
+  if (per_sm > 8) per_sm = 8;
+  if (per_sm < 1) per_sm = 1;
+  return int64_t(kSMs) * per_sm;
+}
 
-int64_t splits_for(int64_t nblocks, int64_t nchunks) {
+int64_t splits_for(int64_t nblocks, int64_t nchunks, int CP, int NT) {
   if (nblocks < 1) nblocks = 1;
   if (nchunks < 1) nchunks = 1;
-  int64_t s = (kTargetBlocks + nblocks - 1) / nblocks;
+  const int64_t target = target_blocks(CP, NT);
+  int64_t s = (target + nblocks - 1) / nblocks;
   if (s > nchunks) s = nchunks;
   if (s < 1) s = 1;
   if (s > 64) s = 64;
@@ -381,15 +424,28 @@ int64_t splits_for(int64_t nblocks, int64_t nchunks) {
 }
 
 int padded(int c) { return ((c + 15) / 16) * 16; }  // NF even keeps the templates few
+int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
 bool fp32_terms(const SkR& R) { return R.dt == kF32 || (R.ptr_b && R.dt_b == kF32); }
-int smem_bytes(int CP, int NT) { return 2 * TILE * PAD * 2 + 2 * NT * CP * PAD * 2; }
+
+slora_status prep_r(const SkR& R, int c, int CP, int64_t I, int nt, __nv_bfloat16* RS,
+                    cudaStream_t st) {
+  const int64_t I64 = round64(std::max<int64_t>(I, 1));
+  const int64_t n = int64_t(CP) * I64;
+  LaunchScope ls(kSkinny, double(I) * c * (R.dt == kF32 ? 4 : 2) + double(nt) * n * 2, st);
+  if (nt == 3)
+    prep_r_kernel<3><<<unsigned((n + 255) / 256), 256, 0, st>>>(R, c, CP, I, I64, RS);
+  else
+    prep_r_kernel<1><<<unsigned((n + 255) / 256), 256, 0, st>>>(R, c, CP, I, I64, RS);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
 
 #define SLORA_SKINNY_CASE(KERNEL, NF_, NT)                                              \
   case NF_ * 8: {                                                                       \
     auto kfn = KERNEL<NF_, NT>;                                                         \
-    const int sm = smem_bytes(NF_ * 8, NT);                                             \
+    const int sm = smem_for(NF_ * 8, NT);                                               \
     cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);         \
-    kfn<<<grid, NTH, sm, st>>>(Y, M, K, R, c, cps, part, counters, o);                  \
+    kfn<<<grid, NTH, sm, st>>>(Y, M, K, RS, I64, c, cps, w.part, w.counters, o);        \
   } break;
 #define SLORA_SKINNY_SWITCH(KERNEL, NT)   \
   switch (CP) {                           \
@@ -400,36 +456,408 @@ int smem_bytes(int CP, int NT) { return 2 * TILE * PAD * 2 + 2 * NT * CP * PAD *
     SLORA_SKINNY_CASE(KERNEL, 8, NT)      \
   }
 
+// Split geometry shared by the launch and the workspace query.
+struct Geo {
+  int CP, nt, cps, nsplit;
+  int64_t nblocks;
+};
+Geo geometry(int64_t nout, int64_t nred, int c, bool fp32) {
+  Geo g;
+  g.CP = padded(c);
+  g.nt = fp32 ? 3 : 1;
+  g.nblocks = (nout + TILE - 1) / TILE;
+  const int64_t nch = std::max<int64_t>((nred + TILE - 1) / TILE, 1);
+  const int64_t ns = splits_for(g.nblocks, nch, g.CP, g.nt);
+  g.cps = int((nch + ns - 1) / ns);
+  g.nsplit = int((nch + g.cps - 1) / g.cps);
+  return g;
+}
+
+
+// ======================================================= TMA stream kernel
+__device__ int g_sk_error = 0;
+constexpr long long kSkWaitBudget = 2000000000LL;  // ~1 s of SM clocks per wait
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arm(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false (and the device error flag raised) when it expires.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* b, uint32_t parity) {
+  if (mbar_try(b, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try(b, parity)) {
+    if (clock64() - t0 > kSkWaitBudget) {
+      atomicExch(&g_sk_error, 1);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma2d(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
+                                      int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t a) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t a) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+// Slice of CTA c: flattened chunks [lo(c), lo(c+1)), lo(c) = c * total / ncta.
+struct StreamPlan {
+  int64_t nblocks = 0, nchunks = 0, total = 0;
+  int ncta = 1;
+};
+__device__ __forceinline__ int64_t slice_lo(const StreamPlan& p, int64_t c) {
+  return c * p.total / p.ncta;
+}
+// The CTA whose slice holds flattened chunk x.
+__device__ __forceinline__ int slice_owner(const StreamPlan& p, int64_t x) {
+  int64_t c = x * p.ncta / p.total;
+  while (c > 0 && slice_lo(p, c) > x) --c;
+  while (c + 1 < p.ncta && slice_lo(p, c + 1) <= x) ++c;
+  return int(c);
+}
+
+// Shared memory of the TMA kernel: S stages of [Y tile 64x64 | split-R tile],
+// each 1024-byte aligned (128-byte swizzle), then the stage barriers.
+constexpr int kYTile = TILE * TILE * 2;
+constexpr int tma_stage_bytes(int CP, int NT) { return kYTile + NT * CP * 128; }
+constexpr int tma_stages(int CP, int NT) {
+  return (113 * 1024 - 1088) / tma_stage_bytes(CP, NT) > 8
+             ? 8
+             : ((113 * 1024 - 1088) / tma_stage_bytes(CP, NT) < 2
+                    ? 2
+                    : (113 * 1024 - 1088) / tma_stage_bytes(CP, NT));
+}
+constexpr int tma_smem(int CP, int NT) {
+  return tma_stages(CP, NT) * tma_stage_bytes(CP, NT) + 1024 + 8 * 8;
+}
+constexpr int kTmaCtasPerSm = 2;
+
+// Element (row, k) of a 128-byte-swizzled tile whose rows are 64 bf16: byte
+// row * 128 + ((k / 8) ^ (row % 8)) * 16 + (k % 8) * 2.
+__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk16) {
+  return base + uint32_t(row) * 128u + (uint32_t((chunk16 ^ (row & 7))) << 4);
+}
+
+// COL = false: rowdot (output block = 64 rows of Y, reduction over K);
+// COL = true: coldot (output block = 64 columns of Y, reduction over M).
+template <int NF, int NT, bool COL>
+__global__ void __launch_bounds__(NTH) skinny_tma_kernel(
+    const __grid_constant__ CUtensorMap ymap, const __grid_constant__ CUtensorMap rmap,
+    const StreamPlan p, int c, int64_t M, int64_t K, float* __restrict__ part,
+    unsigned* __restrict__ counters, const SkRowOut ro, const SkColOut co) {
+  constexpr int CP = NF * 8, S = tma_stages(CP, NT), SB = tma_stage_bytes(CP, NT);
+  extern __shared__ unsigned char sk_smem[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(sk_smem) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + S * SB);
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int cta = blockIdx.x;
+  const int64_t lo = slice_lo(p, cta);
+  const int n = int(slice_lo(p, cta + 1) - lo);
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // (block, chunk) of slice position j, walked incrementally (no 64-bit
+  // division in the loop): the producer runs S positions ahead.
+  const int nch = int(p.nchunks);
+  const int b_first = int(lo / p.nchunks), kc_first = int(lo - int64_t(b_first) * p.nchunks);
+  int pb = b_first, pkc = kc_first;  // producer position (thread 0)
+  auto issue = [&](int j) {  // thread 0: position (pb, pkc) = chunk j into stage j % S
+    const int st = j % S;
+    unsigned char* ys = sm + st * SB;
+    mbar_arm(&full[st], uint32_t(SB));
+    if (COL)
+      tma2d(ys, &ymap, &full[st], pb * TILE, pkc * TILE);
+    else
+      tma2d(ys, &ymap, &full[st], pkc * TILE, pb * TILE);
+    tma2d(ys + kYTile, &rmap, &full[st], pkc * TILE, 0);
+    if (++pkc == nch) { pkc = 0; ++pb; }
+  };
+  if (tid == 0)
+    for (int j = 0; j < S && j < n; ++j) issue(j);
+
+  // per-lane fragment addressing (row % 8 == lane % 8 for every ldmatrix row)
+  const int l7 = lane & 7, mi = lane >> 3;
+  // rowdot A (Y rows): matrices {rows 0-7 | 8-15} x {k 0-7 | 8-15}
+  const int a_row = warp * 16 + l7 + (mi & 1) * 8, a_half = mi >> 1;
+  // coldot A (Y^T): rows m = m16*16 + (mi>>1)*8 + l7, k chunk = warp*2 + (mi&1)
+  const int at_rowoff = (mi >> 1) * 8 + l7, at_chunk = warp * 2 + (mi & 1);
+  // B (split R, rows s*CP + q): matrices {n-block f | f+1} x {k 0-7 | 8-15}
+  const int b_rowoff = (mi >> 1) * 8 + l7, b_half = mi & 1;
+
+  float acc[NF][4];
+#pragma unroll
+  for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
+
+  int j = 0, cb = b_first, ckc = kc_first;  // consumer position
+  for (; j < n; ++j) {
+    const int b = cb, kc = ckc;
+    if (++ckc == nch) { ckc = 0; ++cb; }
+    const int st = j % S;
+    if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1))) s_abort = 1;
+    if (!s_abort) {
+      const uint32_t ybase = su32(sm + st * SB), rbase = ybase + kYTile;
+#pragma unroll
+      for (int k16 = 0; k16 < TILE / 16; ++k16) {
+        uint32_t a[4];
+        if (COL)
+          ldsm4t(a, swz(ybase, k16 * 16 + at_rowoff, at_chunk));
+        else
+          ldsm4(a, swz(ybase, a_row, k16 * 2 + a_half));
+#pragma unroll
+        for (int s = 0; s < NT; ++s)
+#pragma unroll
+          for (int fp = 0; fp < NF / 2; ++fp) {
+            uint32_t bf[4];
+            ldsm4(bf, swz(rbase, s * CP + fp * 16 + b_rowoff, k16 * 2 + b_half));
+            mma16816(acc[2 * fp], a[0], a[1], a[2], a[3], bf[0], bf[1]);
+            mma16816(acc[2 * fp + 1], a[0], a[1], a[2], a[3], bf[2], bf[3]);
+          }
+      }
+    }
+    __syncthreads();  // every warp is done with stage st
+    if (s_abort) break;
+    if (tid == 0 && j + S < n) issue(j + S);
+    if (j + 1 < n && kc + 1 < nch) continue;  // the block goes on in this slice
+
+    // ---- end of this slice's segment of output block b
+    const int64_t nout = COL ? K : M;
+    const int64_t bx = int64_t(b) * p.nchunks;
+    const int c0 = slice_owner(p, bx), c1 = slice_owner(p, bx + p.nchunks - 1);
+    const int64_t r0 = int64_t(b) * TILE + warp * 16 + g;  // output index of acc rows g / g + 8
+    if (c0 == c1) {  // sole contributor: emit from the accumulators
+#pragma unroll
+      for (int f = 0; f < NF; ++f) {
+        const int col = f * 8 + 2 * t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t r = r0 + 8 * h;
+          if (r >= nout) continue;
+          if (COL) {
+            if (col < c) col_emit(co, r, col, acc[f][2 * h]);
+            if (col + 1 < c) col_emit(co, r, col + 1, acc[f][2 * h + 1]);
+          } else {
+            if (col < c) row_emit(ro, r, col, acc[f][2 * h]);
+            if (col + 1 < c) row_emit(ro, r, col + 1, acc[f][2 * h + 1]);
+          }
+        }
+      }
+    } else {
+      const int slot = (b_first == b) ? 0 : 1;
+      float* mine = part + (int64_t(cta) * 2 + slot) * TILE * CP;
+#pragma unroll
+      for (int f = 0; f < NF; ++f) {
+        const int col = f * 8 + 2 * t;
+        const int lr = warp * 16 + g;
+        *reinterpret_cast<float2*>(mine + lr * CP + col) = make_float2(acc[f][0], acc[f][1]);
+        *reinterpret_cast<float2*>(mine + (lr + 8) * CP + col) = make_float2(acc[f][2], acc[f][3]);
+      }
+      if (last_arrival(counters + b, unsigned(c1 - c0 + 1), tid)) {
+        const int nq4 = (c + 3) / 4;
+        for (int e = tid; e < TILE * nq4; e += NTH) {
+          const int lr = e / nq4, q0 = (e % nq4) * 4;
+          const int64_t r = int64_t(b) * TILE + lr;
+          if (r >= nout) continue;
+          float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          for (int cc = c0; cc <= c1; ++cc) {
+            const int sl = (slice_lo(p, cc) / p.nchunks == int64_t(b)) ? 0 : 1;
+            const float4 w = __ldcg(reinterpret_cast<const float4*>(
+                part + ((int64_t(cc) * 2 + sl) * TILE + lr) * CP + q0));
+            v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+          }
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (q0 + u >= c) break;
+            if (COL)
+              col_emit(co, r, q0 + u, vv[u]);
+            else
+              row_emit(ro, r, q0 + u, vv[u]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
+  }
+  if (s_abort && tid == 0) {  // let the copies already issued land before exiting
+    for (int jj = j; jj < n && jj < j + S; ++jj) mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_sk_encode = nullptr;
+std::once_flag g_sk_encode_once;
+
+// 2-D bf16 tensor map, 128-byte swizzle, box {box_x, box_y}, zero fill outside.
+slora_status encode_bf16(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+                         int box_x, int box_y) {
+  std::call_once(g_sk_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_sk_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_sk_encode) SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+  cuuint32_t box[2] = {cuuint32_t(box_x), cuuint32_t(box_y)};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = g_sk_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+                                 dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for a skinny operand", int(r));
+  return SLORA_OK;
+}
+
+bool tma_ok(const SkY& Y, int64_t rows, int64_t cols) {
+  return !Y.map && Y.ptr && (reinterpret_cast<uintptr_t>(Y.ptr) & 15) == 0 && Y.ld % 8 == 0 &&
+         rows > 0 && cols > 0 && Y.ld >= cols;
+}
+
+StreamPlan stream_plan(int64_t nout, int64_t nred) {
+  StreamPlan p;
+  p.nblocks = (nout + TILE - 1) / TILE;
+  p.nchunks = std::max<int64_t>((nred + TILE - 1) / TILE, 1);
+  p.total = p.nblocks * p.nchunks;
+  const int64_t cap = int64_t(kSMs) * kTmaCtasPerSm;
+  p.ncta = int(p.total < cap ? p.total : cap);
+  if (p.ncta < 1) p.ncta = 1;
+  return p;
+}
+
+#define SLORA_TMA_CASE(NF_, NT_, COL_)                                                       \
+  case NF_ * 8: {                                                                            \
+    auto kfn = skinny_tma_kernel<NF_, NT_, COL_>;                                            \
+    const int sm = tma_smem(NF_ * 8, NT_);                                                   \
+    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);              \
+    kfn<<<p.ncta, NTH, sm, st>>>(ym, rm, p, c, M, K, w.part, w.counters, ro, co);            \
+  } break;
+#define SLORA_TMA_SWITCH(NT_, COL_) \
+  switch (CP) {                     \
+    SLORA_TMA_CASE(2, NT_, COL_)    \
+    SLORA_TMA_CASE(4, NT_, COL_)    \
+    SLORA_TMA_CASE(6, NT_, COL_)    \
+    default:                        \
+    SLORA_TMA_CASE(8, NT_, COL_)    \
+  }
+
+// The rsplit rows (NT * CP) are one TMA box high; the map's height is the
+// rows that term count uses.
+slora_status launch_tma(bool col, const SkY& Y, int64_t M, int64_t K, int c, int nt,
+                        const SkRowOut& ro, const SkColOut& co, const SkWork& w, int64_t I64,
+                        cudaStream_t st) {
+  const int CP = padded(c);
+  const StreamPlan p = col ? stream_plan(K, M) : stream_plan(M, K);
+  CUtensorMap ym, rm;
+  SLORA_TRY(encode_bf16(&ym, Y.ptr, M, K, Y.ld, TILE, TILE));
+  SLORA_TRY(encode_bf16(&rm, w.rsplit, int64_t(nt) * CP, I64, I64, TILE, nt * CP));
+  LaunchScope ls(kSkinny, double(M) * K * 2, st);
+  if (col) {
+    if (nt == 3) {
+      SLORA_TMA_SWITCH(3, true)
+    } else {
+      SLORA_TMA_SWITCH(1, true)
+    }
+  } else {
+    if (nt == 3) {
+      SLORA_TMA_SWITCH(3, false)
+    } else {
+      SLORA_TMA_SWITCH(1, false)
+    }
+  }
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+int64_t tma_part_floats(int64_t nout, int64_t nred, int c) {
+  const StreamPlan p = stream_plan(nout, nred);
+  return int64_t(p.ncta) * 2 * TILE * padded(c);
+}
 }  // namespace
 
+// Workspace bounds hold for both term counts (the split count never exceeds
+// the one of the smaller, 1-term footprint).
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c) {
-  const int64_t mb = (M + TILE - 1) / TILE, nch = (K + TILE - 1) / TILE;
-  return splits_for(mb, nch) * std::max<int64_t>(M, 1) * padded(c);
+  const Geo a = geometry(M, K, c, false), b = geometry(M, K, c, true);
+  return std::max(int64_t(std::max(a.nsplit, b.nsplit)) * std::max<int64_t>(M, 1) * padded(c),
+                  tma_part_floats(M, K, c));
 }
 
 int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
-  const int64_t kb = (K + TILE - 1) / TILE, nch = (M + TILE - 1) / TILE;
-  return splits_for(kb, nch) * std::max<int64_t>(K, 1) * padded(c);
+  const Geo a = geometry(K, M, c, false), b = geometry(K, M, c, true);
+  return std::max(int64_t(std::max(a.nsplit, b.nsplit)) * std::max<int64_t>(K, 1) * padded(c),
+                  tma_part_floats(K, M, c));
 }
+
+slora_status skinny_check_error(bool clear) {
+  int v = 0;
+  SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_sk_error, sizeof(int)));
+  if (clear && v) {
+    const int z = 0;
+    SLORA_CUDA(cudaMemcpyToSymbol(g_sk_error, &z, sizeof(int)));
+  }
+  if (v) SLORA_FAIL(SLORA_ERR_TIMEOUT, "a skinny-contraction kernel's bounded wait expired");
+  return SLORA_OK;
+}
+
+int64_t skinny_rsplit_elems(int64_t I) { return 3 * 64 * round64(std::max<int64_t>(I, 1)); }
 
 int64_t skinny_counter_count(int64_t M, int64_t K) {
   return std::max<int64_t>((M + TILE - 1) / TILE, (K + TILE - 1) / TILE) + 1;
 }
 
 slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkRowOut& o,
-                    float* part, unsigned* counters, cudaStream_t st) {
+                    const SkWork& w, cudaStream_t st) {
   if (M <= 0 || c <= 0) return SLORA_OK;
   if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "rowdot: %d columns (max 64)", c);
-  const int CP = padded(c);
-  const int nt = fp32_terms(R) ? 3 : 1;
-  const int64_t mb = (M + TILE - 1) / TILE, nch = std::max<int64_t>((K + TILE - 1) / TILE, 1);
-  const int64_t ns = splits_for(mb, nch);
-  const int cps = int((nch + ns - 1) / ns);
-  const int nsplit = int((nch + cps - 1) / cps);
-  const dim3 grid = dim3(unsigned(mb), unsigned(nsplit), 1u);
-  LaunchScope ls(kSkinny, double(M) * K * 2 + double(nsplit > 1 ? 2 * nsplit : 0) * M * CP * 4,
-                 st);
-  if (nt == 3) {
+  const Geo g = geometry(M, K, c, fp32_terms(R));
+  const int CP = g.CP, cps = g.cps;
+  const int64_t I64 = round64(std::max<int64_t>(K, 1));
+  const __nv_bfloat16* RS = static_cast<const __nv_bfloat16*>(w.rsplit);
+  SLORA_TRY(prep_r(R, c, CP, K, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
+  if (tma_ok(Y, M, K)) return launch_tma(false, Y, M, K, c, g.nt, o, SkColOut(), w, I64, st);
+  const dim3 grid = dim3(unsigned(g.nblocks), unsigned(g.nsplit), 1u);
+  LaunchScope ls(kSkinny,
+                 double(M) * K * 2 + double(g.nsplit > 1 ? 2 * g.nsplit : 0) * M * CP * 4, st);
+  if (g.nt == 3) {
     SLORA_SKINNY_SWITCH(rowdot_kernel, 3)
   } else {
     SLORA_SKINNY_SWITCH(rowdot_kernel, 1)
@@ -439,19 +867,19 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
 }
 
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkColOut& o,
-                    float* part, unsigned* counters, cudaStream_t st) {
+                    const SkWork& w, cudaStream_t st) {
   if (K <= 0 || c <= 0) return SLORA_OK;
   if (c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "coldot: %d columns (max 64)", c);
-  const int CP = padded(c);
-  const int nt = fp32_terms(R) ? 3 : 1;
-  const int64_t kb = (K + TILE - 1) / TILE, nch = std::max<int64_t>((M + TILE - 1) / TILE, 1);
-  const int64_t ns = splits_for(kb, nch);
-  const int cps = int((nch + ns - 1) / ns);
-  const int nsplit = int((nch + cps - 1) / cps);
-  const dim3 grid = dim3(unsigned(kb), unsigned(nsplit), 1u);
-  LaunchScope ls(kSkinny, double(M) * K * 2 + double(nsplit > 1 ? 2 * nsplit : 0) * K * CP * 4,
-                 st);
-  if (nt == 3) {
+  const Geo g = geometry(K, M, c, fp32_terms(R));
+  const int CP = g.CP, cps = g.cps;
+  const int64_t I64 = round64(std::max<int64_t>(M, 1));
+  const __nv_bfloat16* RS = static_cast<const __nv_bfloat16*>(w.rsplit);
+  SLORA_TRY(prep_r(R, c, CP, M, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
+  if (tma_ok(Y, M, K)) return launch_tma(true, Y, M, K, c, g.nt, SkRowOut(), o, w, I64, st);
+  const dim3 grid = dim3(unsigned(g.nblocks), unsigned(g.nsplit), 1u);
+  LaunchScope ls(kSkinny,
+                 double(M) * K * 2 + double(g.nsplit > 1 ? 2 * g.nsplit : 0) * K * CP * 4, st);
+  if (g.nt == 3) {
     SLORA_SKINNY_SWITCH(coldot_kernel, 3)
   } else {
     SLORA_SKINNY_SWITCH(coldot_kernel, 1)

@@ -9,8 +9,11 @@
 //   rowdot:  P1[m, q] = sum_k Y[m, k] R1(k, q)      (e.g. X A^T, h A_d^T, dOut B_d)
 //   coldot:  P2[k, q] = sum_m Y[m, k] R2(m, q)      (LoRA gradients, sums over tokens)
 //
-// Both write fixed-order partial sums (K or M split across blocks) that a
-// finalize pass reduces in order: results are bit-reproducible.
+// The rank-sized operand is split into bf16 terms once per call (a small
+// pre-pass into the rsplit workspace); the main kernel streams Y through a
+// multi-stage cp.async pipeline and writes fixed-order partial sums (K or M
+// split across blocks); the last block of each output block to finish (an
+// atomic ticket) reduces them in order, so results are bit-reproducible.
 #pragma once
 
 #include "common.cuh"
@@ -67,15 +70,27 @@ struct SkColOut {
   int accumulate = 0;
 };
 
-// c = number of R columns (1..64).  part: fp32 workspace of *_part_floats();
-// counters: skinny_counter_count(M, K) unsigned ints that are zero on entry
-// (the kernels leave them zero again).
+// Workspace of one contraction (reusable by the next one on the same stream):
+//   part     fp32, *_part_floats() elements
+//   rsplit   bf16, skinny_rsplit_elems(I) elements, I = K (rowdot) or M (coldot)
+//   counters skinny_counter_count(M, K) unsigned ints, zero on entry; the
+//            kernels leave them zero again
+struct SkWork {
+  float* part = nullptr;
+  void* rsplit = nullptr;
+  unsigned* counters = nullptr;
+};
+
+// c = number of R columns (1..64).
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c);
 int64_t coldot_part_floats(int64_t M, int64_t K, int c);
+int64_t skinny_rsplit_elems(int64_t I);
 int64_t skinny_counter_count(int64_t M, int64_t K);
 slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
-                    const SkRowOut& o, float* part, unsigned* counters, cudaStream_t st);
+                    const SkRowOut& o, const SkWork& w, cudaStream_t st);
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
-                    const SkColOut& o, float* part, unsigned* counters, cudaStream_t st);
+                    const SkColOut& o, const SkWork& w, cudaStream_t st);
+// Device error flag of the TMA kernel (a bounded wait that expired).
+slora_status skinny_check_error(bool clear);
 
 }  // namespace slora
