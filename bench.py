@@ -164,35 +164,43 @@ class GpuLayer:
         Ud = torch.empty(d, rs, device="cuda")
         L.slora_svd_prepare(self.t["Wd"], rs, Ld, Ud, W_t=self.t["Wd_t"], seed=7)
         del self.t["Wd"]
-        T = case.tokens.T
-        self.X = bf(case.X)
-        self.dOut = bf(case.dOut)
-        self.out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
-        self.dX = torch.empty_like(self.out)
-        shapes = [(r, d), (F, r), (r, d), (F, r), (r, F), (d, r)]
-        self.gflat = torch.zeros(sum(a * b for a, b in shapes), device="cuda")
-        self.grads, o = [], 0
-        for a, b in shapes:
-            self.grads.append(self.gflat[o:o + a * b].view(a, b))
-            o += a * b
-        self.idx = torch.empty(F, dtype=torch.int32, device="cuda")
         t = self.t
         self.layer = L.ffn_layer_struct(d, F, rs, r, case.lora_scale, t["Wg"], t["Wu"], t["Wd_t"],
                                         t["Ag"], t["Bg"], t["Au"], t["Bu"], t["Ad"], t["Bd"],
                                         t["Lg"], t["Ug"], t["Lu"], t["Uu"])
-        self.gstruct = L.ffn_grads_struct(*self.grads)
-        tok = case.tokens
-        self.args, self.keep = L.ffn_args(L.BF16, self.layer, tok.batch, tok.seq, tok.ctx_len,
-                                          case.sparsity, self.X, self.dOut, self.out, self.dX,
-                                          self.gstruct, self.idx)
-        need = L.workspace_size("slora_ffn_fwd_bwd", self.args)
+        self.io = [self.make_io(bf(case.X), bf(case.dOut))]
+        self.X, self.dOut, self.out, self.dX, self.gflat = (self.io[0][k] for k in
+                                                            ("X", "dOut", "out", "dX", "gflat"))
+        need = L.workspace_size("slora_ffn_fwd_bwd", self.io[0]["args"])
         self.ws = torch.empty(need, dtype=torch.uint8, device="cuda")
         self.ws_bytes = L.c_sz(need)
 
-    def step(self, stream):
+    def make_io(self, X, dOut):
+        """Per-step inputs, outputs and LoRA gradients (one flat fp32 buffer)."""
+        L, d, F, r = self.L, self.d, self.F, self.r
+        T = self.case.tokens.T
+        io = {"X": X, "dOut": dOut,
+              "out": torch.empty(T, d, dtype=torch.bfloat16, device="cuda"),
+              "dX": torch.empty(T, d, dtype=torch.bfloat16, device="cuda"),
+              "idx": torch.empty(F, dtype=torch.int32, device="cuda")}
+        shapes = [(r, d), (F, r), (r, d), (F, r), (r, F), (d, r)]
+        io["gflat"] = torch.zeros(sum(a * b for a, b in shapes), device="cuda")
+        grads, o = [], 0
+        for a, b in shapes:
+            grads.append(io["gflat"][o:o + a * b].view(a, b))
+            o += a * b
+        io["gstruct"] = L.ffn_grads_struct(*grads)
+        tok = self.case.tokens
+        io["args"], io["keep"] = L.ffn_args(L.BF16, self.layer, tok.batch, tok.seq, tok.ctx_len,
+                                            self.case.sparsity, io["X"], io["dOut"], io["out"],
+                                            io["dX"], io["gstruct"], io["idx"])
+        return io
+
+    def step(self, stream, io=None):
         import ctypes
         L = self.L
-        st = L.lib().slora_ffn_fwd_bwd(*self.args, L.ptr(self.ws), ctypes.byref(self.ws_bytes),
+        io = io or self.io[0]
+        st = L.lib().slora_ffn_fwd_bwd(*io["args"], L.ptr(self.ws), ctypes.byref(self.ws_bytes),
                                        stream.cuda_stream)
         if st != 0:
             raise L.SloraError("slora_ffn_fwd_bwd", st, L.lib().slora_last_error_string().decode())
@@ -287,10 +295,14 @@ def run_ours(args, rank, world):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     T = case.tokens.T
 
+    from contextual_sparsity_lora_svd_b200 import dp
+
     def one_step():
+        # each rank runs its own block of sequences (weak scaling: 8 x 512 tokens
+        # per GPU), selecting from its own context tokens; the LoRA gradients are
+        # then summed over ranks (one NCCL all-reduce of the flat fp32 buffer)
         G.step(stream)
-        if world > 1:
-            torch.distributed.all_reduce(G.gflat)
+        dp.allreduce_grads(G.gflat)
 
     for _ in range(args.warmup):
         one_step()
@@ -299,60 +311,96 @@ def run_ours(args, rank, world):
         torch.distributed.barrier()
     torch.cuda.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    L.profile_enable(True)
-    n0 = L.launch_count()
-    if args.profile_region:
-        torch.cuda.profiler.start()
-    with ClockSampler(dev) as clk:
+    def timed(profile):
+        """K steps bracketed by CUDA events on the launching stream, L2 flushed
+        (outside the events) before each; with `profile` every launch of the
+        library is also bracketed by events, per kernel class."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        if profile:
+            L.profile_enable(True)
+        n0 = L.launch_count()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
             one_step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        launches = L.launch_count() - n0
+        prof = None
+        if profile:
+            prof = {c: L.profile_read(c) for c in L.KERNEL_CLASSES}
+            L.profile_enable(False)
+        return float(sum(a.elapsed_time(b) for a, b in ev)), launches, prof
+
+    if args.profile_region:
+        torch.cuda.profiler.start()
+    with ClockSampler(dev) as clk:
+        ms, launches, _ = timed(False)
     if args.profile_region:
         torch.cuda.profiler.stop()
-    launches = L.launch_count() - n0
-    prof = {c: L.profile_read(c) for c in L.KERNEL_CLASSES}
-    L.profile_enable(False)
-    ms = float(sum(a.elapsed_time(b) for a, b in ev))
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    # per-kernel durations: a second timed pass with events around every launch
+    ms_prof, _, prof = timed(True)
+    ms = dp.max_over_ranks(ms, device="cuda")
     ms_step = ms / args.steps
     value = world * T / (ms_step / 1e3)
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step's
+    # inputs go host->device and its outputs device->host inside the timed
+    # region; copies run on their own streams, double-buffered, so step i+1's
+    # upload and step i-1's download overlap step i's compute.
     Xh = G.X.cpu().pin_memory()
     dOh = G.dOut.cpu().pin_memory()
-    outh = torch.empty_like(G.out, device="cpu").pin_memory()
-    dXh = torch.empty_like(G.dX, device="cpu").pin_memory()
-    gh = torch.empty_like(G.gflat, device="cpu").pin_memory()
-    e2e_steps = max(1, min(args.steps, 10))
+    if len(G.io) < 2:
+        G.io.append(G.make_io(torch.empty_like(G.X), torch.empty_like(G.dOut)))
+    outs = [{k: torch.empty_like(io[k], device="cpu").pin_memory() for k in ("out", "dX", "gflat")}
+            for io in G.io]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    e2e_steps = max(2, min(args.steps, 10))
+    up = [torch.cuda.Event() for _ in range(2)]      # inputs of set i landed
+    done = [torch.cuda.Event() for _ in range(2)]    # compute on set i finished
+    down = [torch.cuda.Event() for _ in range(2)]    # outputs of set i read back
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        G.X.copy_(Xh, non_blocking=True)
-        G.dOut.copy_(dOh, non_blocking=True)
-        one_step()
-        outh.copy_(G.out, non_blocking=True)
-        dXh.copy_(G.dX, non_blocking=True)
-        gh.copy_(G.gflat, non_blocking=True)
-    e1.record(stream)
+    e0.record(h2d_s)
+    stream.wait_event(e0)
+    d2h_s.wait_event(e0)
+
+    def upload(i):
+        io = G.io[i % 2]
+        with torch.cuda.stream(h2d_s):
+            if i >= 2:
+                h2d_s.wait_event(done[i % 2])  # step i-2 has finished reading this set
+            io["X"].copy_(Xh, non_blocking=True)
+            io["dOut"].copy_(dOh, non_blocking=True)
+            up[i % 2].record(h2d_s)
+
+    upload(0)
+    for i in range(e2e_steps):
+        if i + 1 < e2e_steps:
+            upload(i + 1)
+        io = G.io[i % 2]
+        stream.wait_event(up[i % 2])
+        if i >= 2:
+            stream.wait_event(down[i % 2])  # step i-2's outputs are read back
+        G.step(stream, io)
+        dp.allreduce_grads(io["gflat"])
+        done[i % 2].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(done[i % 2])
+            for k in ("out", "dX", "gflat"):
+                outs[i % 2][k].copy_(io[k], non_blocking=True)
+            down[i % 2].record(d2h_s)
+    e1.record(d2h_s)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, device="cuda")
     h2d = Xh.numel() * 2 + dOh.numel() * 2
-    d2h = outh.numel() * 2 + dXh.numel() * 2 + gh.numel() * 4
+    d2h = sum(outs[0][k].numel() * outs[0][k].element_size() for k in ("out", "dX", "gflat"))
 
     # ---- roofline of the dominant kernel class (by device time)
     kernels = {}
@@ -361,7 +409,7 @@ def run_ours(args, rank, world):
         if n:
             kernels[c] = {"launches_per_step": n / args.steps, "ms_per_step": kms / args.steps,
                           "share": kms / ktot if ktot > 0 else None,
-                          "share_of_step": kms / ms if ms > 0 else None}
+                          "share_of_step": kms / ms_prof if ms_prof > 0 else None}
     gemm_cls = max(("gemm_tc", "gemm_simt"), key=lambda c: prof[c][1])
     n_g, ms_g, fl_g = prof[gemm_cls]
     achieved = fl_g / (ms_g / 1e3) / 1e12 if ms_g > 0 else 0.0
@@ -388,7 +436,9 @@ def run_ours(args, rank, world):
             "kernels": kernels, "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "overlap": "double-buffered: H2D, compute and D2H on separate streams"},
+            "profiled_ms_per_step": ms_prof / args.steps,
             "impl": "ours"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         set_threads()
@@ -414,9 +464,9 @@ def main():
         run_reference(args, rank, world)
         return
     if world > 1:
-        import datetime
+        from contextual_sparsity_lora_svd_b200 import dp
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dp.init_from_env("nccl", timeout_s=120)
     try:
         run_ours(args, rank, world)
     finally:

@@ -71,6 +71,7 @@ def _sig(name, res, args):
 _lib_err = _sig("slora_last_error_string", ctypes.c_char_p, [])
 _sig("slora_version", c_int, [])
 _sig("slora_device_error", c_int, [c_int])
+_sig("slora_set_wait_budget", c_int, [c_i64])
 _sig("slora_svd_prepare", c_int,
      [c_vp, c_i64, c_i64, c_int, c_int, c_int, c_u64, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
 _sig("slora_estimate_select", c_int,
@@ -99,7 +100,8 @@ EXPORTS = sorted(["slora_last_error_string", "slora_version", "slora_svd_prepare
                   "slora_estimate_select", "slora_linear_fwd", "slora_linear_bwd",
                   "slora_ffn_fwd_bwd", "slora_launch_count", "slora_profile_enable",
                   "slora_profile_read", "slora_noalloc_scratch_bytes",
-                  "slora_estimate_select_noalloc", "slora_device_error"])
+                  "slora_estimate_select_noalloc", "slora_device_error",
+                  "slora_set_wait_budget"])
 
 
 def lib():

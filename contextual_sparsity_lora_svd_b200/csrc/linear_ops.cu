@@ -42,9 +42,27 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
                            Arena& ar, bool plan, cudaStream_t st);
 
 // ------------------------------------------------------------------ forward
-slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+namespace {
+// The caller's channel list, copied into the workspace with out-of-range
+// entries replaced (sanitize_indices), so no kernel reads through a bad index.
+slora_status safe_indices(const LinearDesc& L, Arena& ar, bool plan, cudaStream_t st,
+                          LinearDesc* out) {
+  *out = L;
+  if (L.side == SLORA_SLICE_NONE || !L.idx || L.n_idx <= 0) return SLORA_OK;
+  int32_t* safe = ar.take<int32_t>(size_t(L.n_idx));
+  out->idx = safe;
+  if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "workspace"));
+  const int64_t limit = L.side == SLORA_SLICE_OUT_ROWS ? L.n : L.k;
+  return sanitize_indices(L.idx, L.n_idx, limit, safe, st);
+}
+}  // namespace
+
+slora_status linear_fwd_run(const LinearDesc& L0, const slora_tokens* tok, const void* X_ctx,
                             const void* X_out, void* Y_ctx, void* Y_out, float* XA_save,
                             Arena& ar, bool plan, cudaStream_t st) {
+  LinearDesc L;
+  SLORA_TRY(safe_indices(L0, ar, plan, st, &L));
   if (L.dt == kBF16)
     return linear_fwd_tc(L, tok, X_ctx, X_out, Y_ctx, Y_out, XA_save, ar, plan, st);
   const TokenInfo& ti = L.ti;
@@ -101,10 +119,12 @@ slora_status linear_fwd_run(const LinearDesc& L, const slora_tokens* tok, const 
 }
 
 // ----------------------------------------------------------------- backward
-slora_status linear_bwd_run(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
+slora_status linear_bwd_run(const LinearDesc& L0, const slora_tokens* tok, const void* X_ctx,
                             const void* X_out, const float* XA, const void* dY_ctx,
                             const void* dY_out, void* dX_ctx, void* dX_out, float* dA, float* dB,
                             Arena& ar, bool plan, cudaStream_t st) {
+  LinearDesc L;
+  SLORA_TRY(safe_indices(L0, ar, plan, st, &L));
   if (L.dt == kBF16)
     return linear_bwd_tc(L, tok, X_ctx, X_out, XA, dY_ctx, dY_out, dX_ctx, dX_out, dA, dB, ar,
                          plan, st);
@@ -300,8 +320,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
     SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
   };
-  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
-    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
+  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
+               int64_t map_limit = INT64_MAX) {
+    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
+    rr.map_limit = map_limit; return rr;
   };
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
@@ -322,8 +344,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   }
   if (idx_force) {
     if (kk > 0)
-      SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
-                                 cudaMemcpyDeviceToDevice, st));
+      SLORA_TRY(sanitize_indices(idx_force, kk, Fd, idx, st));
   } else {
     SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
                                      L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, eb, st, fused,
@@ -358,7 +379,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
     SkRowOut oc;
     oc.out1 = hA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = hAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx), r, oc, sw, st));
+    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx, Fd), r, oc, sw, st));
     SkRowOut oo;
     oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
     SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, sw, st));
@@ -408,7 +429,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
     SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, sw, st));
     SkColOut cc = co;
-    cc.kmap = idx; cc.accumulate = 1;
+    cc.kmap = idx; cc.kmap_limit = Fd; cc.accumulate = 1;
     SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, sw, st));
   }
   for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]; dB = s dG^T XA on the same stream
@@ -424,9 +445,9 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
                      bo, sw, st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
-    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx), r, oc, sw, st));
+    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx, Fd), r, oc, sw, st));
     SkColOut bc = bo;
-    bc.kmap = idx; bc.accumulate = 1;
+    bc.kmap = idx; bc.kmap_limit = Fd; bc.accumulate = 1;
     SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
                      bc, sw, st));
   }
@@ -495,8 +516,7 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
   if (idx_force) {
     if (kk > 0)
-      SLORA_CUDA(cudaMemcpyAsync(idx, idx_force, size_t(kk) * sizeof(int32_t),
-                                 cudaMemcpyDeviceToDevice, st));
+      SLORA_TRY(sanitize_indices(idx_force, kk, Fd, idx, st));
   } else {
     SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
                                      L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, eb, st));
@@ -616,8 +636,10 @@ namespace {
 SkY ykv(const void* p, int64_t ld, const int32_t* map = nullptr) {
   SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
 }
-SkR rkv(const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr) {
-  SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map; return rr;
+SkR rkv(const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
+        int64_t map_limit = INT64_MAX) {
+  SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
+  rr.map_limit = map_limit; return rr;
 }
 int64_t skinny_part_bound(const TokenInfo& ti, int64_t a, int64_t b, int64_t c2, int r) {
   int64_t np = 1;
@@ -708,7 +730,7 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   {
     SkRowOut oc;
     oc.out1 = XA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = XAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(ykv(Xc, ldxc), TC, ni, rkv(L.A, kBF16, 1, k, L.idx), r, oc, sw, st));
+    SLORA_TRY(rowdot(ykv(Xc, ldxc), TC, ni, rkv(L.A, kBF16, 1, k, L.idx, k), r, oc, sw, st));
     SkRowOut oo;
     oo.out1 = XA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = XAbO; oo.ld2 = lr; oo.s2 = s;
     SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, sw, st));
@@ -795,7 +817,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     {  // dYB = dY B on the rows' channels; dB = s dY^T XA (output rows first, then += S rows)
       SkRowOut oc;
       oc.out1 = dYB; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = dYBbC; oc.ld2 = lr; oc.s2 = s;
-      SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx), r, oc, sw,
+      SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx, n), r, oc, sw,
                        st));
       SkRowOut oo;
       oo.out1 = dYB; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = dYBbO; oo.ld2 = lr; oo.s2 = s;
@@ -805,7 +827,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
       SLORA_TRY(coldot(ykv(dY_out, n), TO, n, rkv(XA, kF32, r, 1, out_rows), r, bo, sw,
                        st));
       SkColOut bc = bo;
-      bc.kmap = L.idx; bc.accumulate = 1;
+      bc.kmap = L.idx; bc.kmap_limit = n; bc.accumulate = 1;
       SLORA_TRY(coldot(ykv(dYc, lddc), TC, ni, rkv(XA, kF32, r, 1, ctx_rows), r, bc, sw,
                        st));
     }
@@ -863,7 +885,7 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     ao.out = dA; ao.ldo = k; ao.trans = 1; ao.scale = s;
     SLORA_TRY(coldot(ykv(X_out, k), TO, k, rkv(dYB, kF32, r, 1, out_rows), r, ao, sw, st));
     SkColOut ac = ao;
-    ac.kmap = L.idx; ac.accumulate = 1;
+    ac.kmap = L.idx; ac.kmap_limit = k; ac.accumulate = 1;
     SLORA_TRY(coldot(ykv(Xc, ldxc), TC, ni, rkv(dYB, kF32, r, 1, ctx_rows), r, ac, sw, st));
   }
   SkColOut cb;  // dB = s dY^T XA over every row

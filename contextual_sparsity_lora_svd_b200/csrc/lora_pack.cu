@@ -100,6 +100,14 @@ __global__ void gather_pad_kernel(const __nv_bfloat16* __restrict__ in, int64_t 
   out[e] = (c < cols && index_ok(src, rows_in)) ? in[src * ld_in + c] : __float2bfloat16_rn(0.0f);
 }
 
+__global__ void sanitize_kernel(const int32_t* __restrict__ in, int64_t n, int64_t limit,
+                                int32_t* __restrict__ out) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int32_t v = in[i];
+  out[i] = index_ok(v, limit) ? v : 0;
+}
+
 __global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t nt) {
   const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= nt) return;
@@ -182,6 +190,15 @@ slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64
   return SLORA_OK;
 }
 
+slora_status sanitize_indices(const int32_t* in, int64_t n, int64_t limit, int32_t* out,
+                              cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(n) * 8, st);
+  sanitize_kernel<<<blocks(n), 256, 0, st>>>(in, n, limit, out);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
 slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st) {
   const int64_t nt = (M + 127) / 128;
   if (nt <= 0) return SLORA_OK;
@@ -207,7 +224,7 @@ slora_status pack_check_error(bool clear) {
     const int z = 0;
     SLORA_CUDA(cudaMemcpyToSymbol(g_pack_bad_index, &z, sizeof(int)));
   }
-  if (v) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "a gather met a channel index outside its weight");
+  if (v) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "a channel index list held an entry outside its weight (replaced by channel 0)");
   return SLORA_OK;
 }
 

@@ -32,6 +32,12 @@ slora_status concat_cols_f32(const float* a, const float* b, int64_t rows, int64
 // columns, zero padded to ldo.
 slora_status gather_pad(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
                         int64_t cols, void* out, int64_t ldo, cudaStream_t st, int64_t rows_in);
+// out[i] = in[i] for i < n when 0 <= in[i] < limit; an entry outside that
+// range becomes 0 and raises the flag that pack_check_error reads.  Every
+// caller-supplied channel index list goes through this before any kernel
+// reads through it, so a bad list gives wrong results, never a wild access.
+slora_status sanitize_indices(const int32_t* in, int64_t n, int64_t limit, int32_t* out,
+                              cudaStream_t st);
 // Reads (and with `clear` resets) the flag the gathers above raise when an
 // index lies outside their source; SLORA_ERR_INVALID_ARG if it was raised.
 // Synchronous: waits for the device.

@@ -164,6 +164,11 @@ extern "C" slora_status slora_device_error(int clear) {
   return a != SLORA_OK ? a : (b != SLORA_OK ? b : c);
 }
 
+extern "C" slora_status slora_set_wait_budget(int64_t cycles) {
+  slora::clear_error();
+  return slora::skinny_set_wait_budget(static_cast<long long>(cycles));
+}
+
 // ------------------------------------------------------------ launch record
 namespace slora {
 namespace {

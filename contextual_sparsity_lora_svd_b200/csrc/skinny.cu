@@ -77,8 +77,16 @@ __device__ __forceinline__ void split_terms(float v, __nv_bfloat16* out) {
   }
 }
 
+// Raised when a channel-index map holds a value outside its weight (the
+// element is read as zero / not written); reported by skinny_check_error.
+__device__ int g_sk_bad_index = 0;
+
 __device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
   const int64_t ii = R.map ? R.map[i] : i;
+  if (ii < 0 || ii >= R.map_limit) {
+    atomicExch(&g_sk_bad_index, 1);
+    return 0.0f;
+  }
   const void* p = R.ptr;
   int dt = R.dt;
   int64_t off = ii * R.si + int64_t(q) * R.sq;
@@ -169,6 +177,10 @@ __device__ __forceinline__ void row_emit(const SkRowOut& o, int64_t m, int q, fl
 __device__ __forceinline__ void col_emit(const SkColOut& o, int64_t k, int q, float v) {
   v *= o.scale;
   const int64_t kk = o.kmap ? int64_t(o.kmap[k]) : k;
+  if (kk < 0 || kk >= o.kmap_limit) {
+    atomicExch(&g_sk_bad_index, 1);
+    return;
+  }
   float* base = q < o.qsplit ? o.out : o.out_b;
   const int qq = q < o.qsplit ? q : q - o.qsplit;
   float* dst = base + (o.trans ? int64_t(qq) * o.ldo + kk : kk * o.ldo + qq);
@@ -477,6 +489,10 @@ Geo geometry(int64_t nout, int64_t nred, int c, bool fp32) {
 // ======================================================= TMA stream kernel
 __device__ int g_sk_error = 0;
 constexpr long long kSkWaitBudget = 2000000000LL;  // ~1 s of SM clocks per wait
+// Budget of the pipeline waits (settable for tests of the error path); the
+// drain after an abort always uses the full budget so every issued copy lands
+// before the CTA exits.
+__device__ long long g_sk_budget = kSkWaitBudget;
 
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -499,12 +515,30 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait; false (and the device error flag raised) when it expires.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* b, uint32_t parity) {
-  if (mbar_try(b, parity)) return true;
+// Non-blocking poll (try_wait may park the thread until the phase completes).
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; false (and the device error flag raised) when it expires.  The
+// first poll does not block, so a budget of 0 gives up at once.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* b, uint32_t parity,
+                                                  long long budget) {
+  if (mbar_test(b, parity)) return true;
+  if (budget <= 0) {
+    atomicExch(&g_sk_error, 1);
+    return false;
+  }
   const long long t0 = clock64();
   while (!mbar_try(b, parity)) {
-    if (clock64() - t0 > kSkWaitBudget) {
+    if (clock64() - t0 > budget) {
       atomicExch(&g_sk_error, 1);
       return false;
     }
@@ -628,7 +662,7 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
     const int b = cb, kc = ckc;
     if (++ckc == nch) { ckc = 0; ++cb; }
     const int st = j % S;
-    if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1))) s_abort = 1;
+    if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1), g_sk_budget)) s_abort = 1;
     if (!s_abort) {
       const uint32_t ybase = su32(sm + st * SB), rbase = ybase + kYTile;
 #pragma unroll
@@ -715,7 +749,8 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
     for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
   }
   if (s_abort && tid == 0) {  // let the copies already issued land before exiting
-    for (int jj = j; jj < n && jj < j + S; ++jj) mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1));
+    for (int jj = j; jj < n && jj < j + S; ++jj)
+      mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1), kSkWaitBudget);
   }
 }
 
@@ -827,13 +862,23 @@ int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
                   tma_part_floats(K, M, c));
 }
 
+slora_status skinny_set_wait_budget(long long cycles) {
+  const long long v = cycles < 0 ? kSkWaitBudget : cycles;
+  SLORA_CUDA(cudaMemcpyToSymbol(g_sk_budget, &v, sizeof(v)));
+  return SLORA_OK;
+}
+
 slora_status skinny_check_error(bool clear) {
-  int v = 0;
+  int v = 0, bad = 0;
   SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_sk_error, sizeof(int)));
-  if (clear && v) {
+  SLORA_CUDA(cudaMemcpyFromSymbol(&bad, g_sk_bad_index, sizeof(int)));
+  if (clear && (v || bad)) {
     const int z = 0;
     SLORA_CUDA(cudaMemcpyToSymbol(g_sk_error, &z, sizeof(int)));
+    SLORA_CUDA(cudaMemcpyToSymbol(g_sk_bad_index, &z, sizeof(int)));
   }
+  if (bad)
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "a channel index lies outside its weight (read as zero)");
   if (v) SLORA_FAIL(SLORA_ERR_TIMEOUT, "a skinny-contraction kernel's bounded wait expired");
   return SLORA_OK;
 }

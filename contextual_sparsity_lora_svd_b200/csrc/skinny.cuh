@@ -31,6 +31,7 @@ struct SkR {  // R(i, q) = ptr[(map ? map[i] : i) * si + q * sq], fp32 or bf16
   int dt = kF32;
   int64_t si = 0, sq = 0;
   const int32_t* map = nullptr;
+  int64_t map_limit = INT64_MAX;  // map values outside [0, map_limit) read as zero
   // columns q >= qsplit come from a second source: ptr_b[i' * si_b + (q - qsplit) * sq_b]
   int qsplit = 1 << 30;
   const void* ptr_b = nullptr;
@@ -66,6 +67,7 @@ struct SkColOut {
   int64_t ldo = 0;
   int trans = 0;
   const int32_t* kmap = nullptr;
+  int64_t kmap_limit = INT64_MAX;  // kmap values outside [0, kmap_limit) are not written
   float scale = 1.0f;
   int accumulate = 0;
 };
@@ -92,5 +94,7 @@ slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkColOut& o, const SkWork& w, cudaStream_t st);
 // Device error flag of the TMA kernel (a bounded wait that expired).
 slora_status skinny_check_error(bool clear);
+// Budget of the TMA kernel's pipeline waits in SM clock cycles (< 0: default).
+slora_status skinny_set_wait_budget(long long cycles);
 
 }  // namespace slora

@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "rng", "gaussian", "round_bf16", "orthonormal", "decaying_weight",
-    "Tokens", "FFNCase", "ffn_case", "QKCase", "qk_case", "WORKLOADS",
+    "Tokens", "FFNCase", "ffn_case", "QKCase", "qk_case", "WORKLOADS", "stack_sparsity",
 ]
 
 
@@ -215,4 +215,30 @@ WORKLOADS = {
             r_svd=8, r_lora=16, sparsity=0.5, bf16=True),
     2: dict(name="llama2-7b-attn-qk-bf16", batch=4, seq=1024, out_frac=0.25, d=4096,
             heads=32, kv_heads=32, head_dim=128, r_svd=8, r_lora=16, sparsity=0.5, bf16=True),
+    # 32 Llama-2-7B-shaped layers: FFN + q/k/v/o LoRA linears, per-layer sparsity
+    # from stack_sparsity()
+    3: dict(name="llama2-7b-stack32-bf16", layers=32, batch=4, seq=1024, out_frac=0.25,
+            d=4096, d_ff=11008, heads=32, kv_heads=32, head_dim=128, r_svd=8, r_lora=16,
+            bf16=True),
+    # Llama-3-8B-shaped layer (GQA 32 q / 8 kv heads), 8192 tokens per batch,
+    # swept over sequence length, sparsity and SVD rank
+    4: dict(name="llama3-8b-layer-bf16", tokens=8192, seqs=(256, 512, 1024, 2048, 4096),
+            out_frac=0.25, d=4096, d_ff=14336, heads=32, kv_heads=8, head_dim=128,
+            sparsities=(0.0, 0.3, 0.5, 0.7, 0.9), r_svds=(4, 8, 16), r_lora=16, bf16=True),
 }
+
+
+def stack_sparsity(layer: int, layers: int = 32, dense_layers: int = 4,
+                   ffn: tuple[float, float] = (0.5, 0.9),
+                   qk: tuple[float, float] = (0.3, 0.6)) -> tuple[float, float]:
+    """(FFN sparsity, QK sparsity) of one layer of the 32-layer stack: the first
+    `dense_layers` layers run dense, then both ramp linearly from their first
+    to their last value over the remaining layers (the plain reading of a
+    per-layer ramp; SparseLoRA article, section 1, keeps early layers dense and
+    sparsifies deeper ones more)."""
+    if not 0 <= layer < layers:
+        raise ValueError(f"layer {layer} outside [0, {layers})")
+    if layer < dense_layers:
+        return 0.0, 0.0
+    f = (layer - dense_layers) / max(layers - 1 - dense_layers, 1)
+    return ffn[0] + (ffn[1] - ffn[0]) * f, qk[0] + (qk[1] - qk[0]) * f

@@ -89,15 +89,31 @@ int slora_version(void);
 
 /*
  * Errors that kernels record on the device instead of faulting (not part of
- * the method): a gather of selected weight rows that met a channel index
- * outside the weight (the row is read as zeros), or a tensor-core pipeline
- * wait that gave up.  Waits for the current device to finish its work, then
- * returns SLORA_ERR_INVALID_ARG (bad index), SLORA_ERR_TIMEOUT (wait expired) or
- * SLORA_OK; clear != 0 resets the recorded state.  Index lists that callers
- * pass (idx, idx_force) must hold in-range channels: only the gathers check,
- * the other kernels that read through an index list trust it.
+ * the method).  Waits for the current device to finish its work, then returns
+ *   SLORA_ERR_INVALID_ARG  a caller-supplied channel list (idx of the linear
+ *                          calls, idx_force of the FFN call) held an entry
+ *                          outside its weight: the library replaced it by
+ *                          channel 0 before any kernel read through it, so
+ *                          that call's results are wrong but no memory
+ *                          outside the caller's buffers was touched;
+ *   SLORA_ERR_TIMEOUT      a pipeline wait inside a kernel gave up (its
+ *                          call's outputs are undefined);
+ *   SLORA_OK               neither happened since the last clear.
+ * clear != 0 resets the recorded state.
  */
 slora_status slora_device_error(int clear);
+
+/*
+ * Test hook for the error path above (not part of the method): the budget, in
+ * SM clock cycles, of the pipeline waits of the skinny-contraction stream
+ * kernel (the LoRA projections and gradients on strided inputs).  0 makes
+ * every wait that does not succeed at its first poll give up, so the next
+ * call raises the device flag that slora_device_error reports as
+ * SLORA_ERR_TIMEOUT and leaves its outputs undefined; the device stays usable.
+ * A negative value restores the default (about one second).  Synchronous;
+ * affects every later call on the current device.
+ */
+slora_status slora_set_wait_budget(int64_t cycles);
 
 /*
  * Launch accounting and optional per-kernel timing (not part of the method;
