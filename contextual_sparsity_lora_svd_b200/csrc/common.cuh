@@ -123,7 +123,7 @@ __device__ __forceinline__ void st_elem(void* p, int64_t i, int dt, float v) {
 // silu(x) = x * sigmoid(x) in fp32.  __expf is the fast exp2-based intrinsic
 // (relative error a few ulp); for x << 0 exp(-x) overflows to +inf and the
 // reciprocal gives 0, so silu -> 0 as it should.
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 }  // namespace slora

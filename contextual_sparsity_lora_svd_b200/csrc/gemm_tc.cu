@@ -182,9 +182,20 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* row, int c0, int N, c
       for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1]);
       dst[q] = *reinterpret_cast<uint4*>(h);
     }
-  } else {
-    for (int j = 0; j < 32 && c0 + j < N; ++j) row[c0 + j] = __float2bfloat16_rn(v[j]);
+  } else {  // right edge: unrolled with predicates so v stays in registers
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (c0 + j < N) row[c0 + j] = __float2bfloat16_rn(v[j]);
   }
+}
+// Bulk prefetch into L2 of columns [c0, min(c0 + 256, N)) of one bf16 row
+// (whole 16-byte units; rows start 16-byte aligned and c0 is a multiple of 256).
+__device__ __forceinline__ void prefetch_row256(const __nv_bfloat16* row, int c0, int N) {
+  const int cols = N - c0 < 256 ? N - c0 : 256;
+  const uint32_t bytes = uint32_t(cols > 0 ? cols : 0) * 2u & ~15u;
+  if (bytes)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(row + c0), "r"(bytes)
+                 : "memory");
 }
 __device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int c0, int N, float* v) {
   if (c0 + 32 <= N) {
@@ -201,6 +212,7 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int c0, int
       }
     }
   } else {
+#pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = (c0 + j < N) ? __bfloat162float(row[c0 + j]) : 0.0f;
   }
 }
@@ -414,23 +426,43 @@ __global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__
         const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
         __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
         __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+        if (valid) {  // the whole row segment of g and u on its way to L2 at once
+          prefetch_row256(gi, ti.n0, p.N);
+          prefetch_row256(ui, ti.n0, p.N);
+        }
+// g and u of chunk c + 1 are loaded while chunk c is computed, so each
+        // chunk's global-load latency hides behind the previous chunk's math
+        float gv[32], uv[32], gn[32], un[32];
+        if (valid && ti.n0 < p.N) {
+          load_row32(gi, ti.n0, p.N, gv);
+          load_row32(ui, ti.n0, p.N, uv);
+        }
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           tmem_ld32(tl + c * 32, v);  // dh
           const int c0 = ti.n0 + c * 32;
+          const bool next = valid && c + 1 < 8 && c0 + 32 < p.N;
+          if (next) {
+            load_row32(gi, c0 + 32, p.N, gn);
+            load_row32(ui, c0 + 32, p.N, un);
+          }
           if (valid && c0 < p.N) {
-            float gv[32];
-            load_row32(gi, c0, p.N, gv);
-            load_row32(ui, c0, p.N, w);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float sg = sigmoid_f(gv[j]);
               const float dh = v[j];
-              v[j] = dh * w[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
-              w[j] = dh * gv[j] * sg;                                 // dU
+              v[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
+              w[j] = dh * gv[j] * sg;                                  // dU
             }
             store_row32(dg, c0, p.N, v);
             store_row32(du, c0, p.N, w);
+          }
+          if (next) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              gv[j] = gn[j];
+              uv[j] = un[j];
+            }
           }
         }
       } else {
@@ -728,23 +760,43 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
         const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
         __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
         __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+        if (valid) {  // the whole row segment of g and u on its way to L2 at once
+          prefetch_row256(gi, n0, p.N);
+          prefetch_row256(ui, n0, p.N);
+        }
+// g and u of chunk c + 1 are loaded while chunk c is computed, so each
+        // chunk's global-load latency hides behind the previous chunk's math
+        float gv[32], uv[32], gn[32], un[32];
+        if (valid && n0 < p.N) {
+          load_row32(gi, n0, p.N, gv);
+          load_row32(ui, n0, p.N, uv);
+        }
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           tmem_ld32(tl + c * 32, v);  // dh
           const int c0 = n0 + c * 32;
+          const bool next = valid && c + 1 < 8 && c0 + 32 < p.N;
+          if (next) {
+            load_row32(gi, c0 + 32, p.N, gn);
+            load_row32(ui, c0 + 32, p.N, un);
+          }
           if (valid && c0 < p.N) {
-            float gv[32];
-            load_row32(gi, c0, p.N, gv);
-            load_row32(ui, c0, p.N, w);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float sg = sigmoid_f(gv[j]);
               const float dh = v[j];
-              v[j] = dh * w[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
-              w[j] = dh * gv[j] * sg;                                 // dU
+              v[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
+              w[j] = dh * gv[j] * sg;                                  // dU
             }
             store_row32(dg, c0, p.N, v);
             store_row32(du, c0, p.N, w);
+          }
+          if (next) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              gv[j] = gn[j];
+              uv[j] = un[j];
+            }
           }
         }
       } else {
