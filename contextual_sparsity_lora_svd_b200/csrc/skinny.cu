@@ -564,35 +564,33 @@ __device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t a) {
                : "r"(a));
 }
 
-// Slice of CTA c: flattened chunks [lo(c), lo(c+1)), lo(c) = c * total / ncta.
+// Work of one contraction: output blocks of 64 (rows for rowdot, columns for
+// coldot), each with nchunks reduction chunks of 64 cut into ngroups fixed
+// groups of up to G chunks.  A unit is one (block, group); units are handed
+// out by an atomic ticket in group-major order (ticket u -> block u % nblocks,
+// group u / nblocks), so SMs that stream faster take more units.  Each unit's
+// partial lands in its own slot and the last unit of a block to finish sums
+// the block's slots in group order: the result does not depend on which CTA
+// ran which unit.
 struct StreamPlan {
-  int64_t nblocks = 0, nchunks = 0, total = 0;
+  int nblocks = 0, nchunks = 0, G = 1, ngroups = 1, nunits = 0;
   int ncta = 1;
 };
-__device__ __forceinline__ int64_t slice_lo(const StreamPlan& p, int64_t c) {
-  return c * p.total / p.ncta;
-}
-// The CTA whose slice holds flattened chunk x.
-__device__ __forceinline__ int slice_owner(const StreamPlan& p, int64_t x) {
-  int64_t c = x * p.ncta / p.total;
-  while (c > 0 && slice_lo(p, c) > x) --c;
-  while (c + 1 < p.ncta && slice_lo(p, c + 1) <= x) ++c;
-  return int(c);
-}
 
 // Shared memory of the TMA kernel: S stages of [Y tile 64x64 | split-R tile],
-// each 1024-byte aligned (128-byte swizzle), then the stage barriers.
+// each 1024-byte aligned (128-byte swizzle), then the stage barriers and the
+// stages' work descriptors.
 constexpr int kYTile = TILE * TILE * 2;
 constexpr int tma_stage_bytes(int CP, int NT) { return kYTile + NT * CP * 128; }
 constexpr int tma_stages(int CP, int NT) {
-  return (113 * 1024 - 1088) / tma_stage_bytes(CP, NT) > 8
+  return (113 * 1024 - 1216) / tma_stage_bytes(CP, NT) > 8
              ? 8
-             : ((113 * 1024 - 1088) / tma_stage_bytes(CP, NT) < 2
+             : ((113 * 1024 - 1216) / tma_stage_bytes(CP, NT) < 2
                     ? 2
-                    : (113 * 1024 - 1088) / tma_stage_bytes(CP, NT));
+                    : (113 * 1024 - 1216) / tma_stage_bytes(CP, NT));
 }
 constexpr int tma_smem(int CP, int NT) {
-  return tma_stages(CP, NT) * tma_stage_bytes(CP, NT) + 1024 + 8 * 8;
+  return tma_stages(CP, NT) * tma_stage_bytes(CP, NT) + 1024 + 8 * 8 + 8 * 16;
 }
 constexpr int kTmaCtasPerSm = 2;
 
@@ -604,66 +602,86 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk16) {
 
 // COL = false: rowdot (output block = 64 rows of Y, reduction over K);
 // COL = true: coldot (output block = 64 columns of Y, reduction over M).
+// counters[0 .. nblocks) are the per-block arrival tickets, counters[nblocks]
+// the unit ticket; all are zero on entry and left zero.
 template <int NF, int NT, bool COL>
 __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
     const __grid_constant__ CUtensorMap ymap, const __grid_constant__ CUtensorMap rmap,
     const StreamPlan p, int c, int64_t M, int64_t K, float* __restrict__ part,
     unsigned* __restrict__ counters, const SkRowOut ro, const SkColOut co) {
   constexpr int CP = NF * 8, S = tma_stages(CP, NT), SB = tma_stage_bytes(CP, NT);
+  constexpr int kFirst = 1, kLast = 2, kEnd = 4;
   extern __shared__ unsigned char sk_smem[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(sk_smem) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + S * SB);
+  int4* info = reinterpret_cast<int4*>(sm + S * SB + 8 * 8);  // {block, chunk, flags, group}
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int cta = blockIdx.x;
-  const int64_t lo = slice_lo(p, cta);
-  const int n = int(slice_lo(p, cta + 1) - lo);
+  unsigned* work = counters + p.nblocks;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // (block, chunk) of slice position j, walked incrementally (no 64-bit
-  // division in the loop): the producer runs S positions ahead.
-  const int nch = int(p.nchunks);
-  const int b_first = int(lo / p.nchunks), kc_first = int(lo - int64_t(b_first) * p.nchunks);
-  int pb = b_first, pkc = kc_first;  // producer position (thread 0)
-  auto issue = [&](int j) {  // thread 0: position (pb, pkc) = chunk j into stage j % S
-    const int st = j % S;
+  // ---- producer state (thread 0): current unit and the next chunk of it
+  int pb = 0, pg = 0, pk = 0, pk1 = 0, issued = 0;
+  bool pdone = false;
+  auto next_unit = [&]() {  // false once the tickets are exhausted
+    const unsigned u = atomicAdd(work, 1u);
+    if (u >= unsigned(p.nunits)) {
+      if (u == unsigned(p.nunits + p.ncta - 1)) *work = 0u;  // the last ticket resets
+      return false;
+    }
+    pb = int(u % unsigned(p.nblocks));
+    pg = int(u / unsigned(p.nblocks));
+    pk = pg * p.G;
+    pk1 = pk + p.G < p.nchunks ? pk + p.G : p.nchunks;
+    return true;
+  };
+  auto issue = [&]() {  // thread 0: the next position of the stream into stage issued % S
+    const int st = issued % S;
+    if (!pdone && pk == pk1 && !next_unit()) pdone = true;
+    if (pdone) {  // end marker: completes the stage's phase without data
+      info[st] = make_int4(0, 0, kEnd, 0);
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&full[st])) : "memory");
+      ++issued;
+      return false;
+    }
+    const int flags = (pk == pg * p.G ? kFirst : 0) | (pk + 1 == pk1 ? kLast : 0);
+    info[st] = make_int4(pb, pk, flags, pg);
     unsigned char* ys = sm + st * SB;
     mbar_arm(&full[st], uint32_t(SB));
     if (COL)
-      tma2d(ys, &ymap, &full[st], pb * TILE, pkc * TILE);
+      tma2d(ys, &ymap, &full[st], pb * TILE, pk * TILE);
     else
-      tma2d(ys, &ymap, &full[st], pkc * TILE, pb * TILE);
-    tma2d(ys + kYTile, &rmap, &full[st], pkc * TILE, 0);
-    if (++pkc == nch) { pkc = 0; ++pb; }
+      tma2d(ys, &ymap, &full[st], pk * TILE, pb * TILE);
+    tma2d(ys + kYTile, &rmap, &full[st], pk * TILE, 0);
+    ++pk;
+    ++issued;
+    return true;
   };
-  if (tid == 0)
-    for (int j = 0; j < S && j < n; ++j) issue(j);
-
+  if (tid == 0) {
+    for (int j = 0; j < S; ++j)
+      if (!issue()) break;
+  }
   // per-lane fragment addressing (row % 8 == lane % 8 for every ldmatrix row)
   const int l7 = lane & 7, mi = lane >> 3;
-  // rowdot A (Y rows): matrices {rows 0-7 | 8-15} x {k 0-7 | 8-15}
-  const int a_row = warp * 16 + l7 + (mi & 1) * 8, a_half = mi >> 1;
-  // coldot A (Y^T): rows m = m16*16 + (mi>>1)*8 + l7, k chunk = warp*2 + (mi&1)
-  const int at_rowoff = (mi >> 1) * 8 + l7, at_chunk = warp * 2 + (mi & 1);
-  // B (split R, rows s*CP + q): matrices {n-block f | f+1} x {k 0-7 | 8-15}
-  const int b_rowoff = (mi >> 1) * 8 + l7, b_half = mi & 1;
+  const int a_row = warp * 16 + l7 + (mi & 1) * 8, a_half = mi >> 1;     // rowdot A (Y rows)
+  const int at_rowoff = (mi >> 1) * 8 + l7, at_chunk = warp * 2 + (mi & 1);  // coldot A (Y^T)
+  const int b_rowoff = (mi >> 1) * 8 + l7, b_half = mi & 1;              // split R
 
   float acc[NF][4];
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
 
-  int j = 0, cb = b_first, ckc = kc_first;  // consumer position
-  for (; j < n; ++j) {
-    const int b = cb, kc = ckc;
-    if (++ckc == nch) { ckc = 0; ++cb; }
+  int j = 0;
+  for (;; ++j) {
     const int st = j % S;
     if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1), g_sk_budget)) s_abort = 1;
-    if (!s_abort) {
+    const int4 inf = info[st];  // published before the stage's barrier arrival
+    if (!s_abort && !(inf.z & kEnd)) {
       const uint32_t ybase = su32(sm + st * SB), rbase = ybase + kYTile;
 #pragma unroll
       for (int k16 = 0; k16 < TILE / 16; ++k16) {
@@ -683,17 +701,16 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
           }
       }
     }
-    __syncthreads();  // every warp is done with stage st
-    if (s_abort) break;
-    if (tid == 0 && j + S < n) issue(j + S);
-    if (j + 1 < n && kc + 1 < nch) continue;  // the block goes on in this slice
+    __syncthreads();  // every warp is done with stage st (and has read its info)
+    if (s_abort || (inf.z & kEnd)) break;
+    if (tid == 0 && !pdone) issue();
+    if (!(inf.z & kLast)) continue;  // the unit goes on
 
-    // ---- end of this slice's segment of output block b
+    // ---- end of unit (block inf.x, group inf.w)
+    const int b = inf.x;
     const int64_t nout = COL ? K : M;
-    const int64_t bx = int64_t(b) * p.nchunks;
-    const int c0 = slice_owner(p, bx), c1 = slice_owner(p, bx + p.nchunks - 1);
     const int64_t r0 = int64_t(b) * TILE + warp * 16 + g;  // output index of acc rows g / g + 8
-    if (c0 == c1) {  // sole contributor: emit from the accumulators
+    if (p.ngroups == 1) {  // the unit is the whole block: emit from the accumulators
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
         const int col = f * 8 + 2 * t;
@@ -711,8 +728,7 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
         }
       }
     } else {
-      const int slot = (b_first == b) ? 0 : 1;
-      float* mine = part + (int64_t(cta) * 2 + slot) * TILE * CP;
+      float* mine = part + (int64_t(b) * p.ngroups + inf.w) * TILE * CP;
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
         const int col = f * 8 + 2 * t;
@@ -720,19 +736,15 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
         *reinterpret_cast<float2*>(mine + lr * CP + col) = make_float2(acc[f][0], acc[f][1]);
         *reinterpret_cast<float2*>(mine + (lr + 8) * CP + col) = make_float2(acc[f][2], acc[f][3]);
       }
-      if (last_arrival(counters + b, unsigned(c1 - c0 + 1), tid)) {
+      if (last_arrival(counters + b, unsigned(p.ngroups), tid)) {
         const int nq4 = (c + 3) / 4;
+        const float* blk = part + int64_t(b) * p.ngroups * TILE * CP;
         for (int e = tid; e < TILE * nq4; e += NTH) {
           const int lr = e / nq4, q0 = (e % nq4) * 4;
           const int64_t r = int64_t(b) * TILE + lr;
           if (r >= nout) continue;
-          float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          for (int cc = c0; cc <= c1; ++cc) {
-            const int sl = (slice_lo(p, cc) / p.nchunks == int64_t(b)) ? 0 : 1;
-            const float4 w = __ldcg(reinterpret_cast<const float4*>(
-                part + ((int64_t(cc) * 2 + sl) * TILE + lr) * CP + q0));
-            v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-          }
+          const float4 v = sum_splits4(reinterpret_cast<const float4*>(blk + lr * CP + q0),
+                                       int64_t(TILE) * CP / 4, p.ngroups);
           const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -749,7 +761,7 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
     for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
   }
   if (s_abort && tid == 0) {  // let the copies already issued land before exiting
-    for (int jj = j; jj < n && jj < j + S; ++jj)
+    for (int jj = j; jj < issued; ++jj)
       mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1), kSkWaitBudget);
   }
 }
@@ -787,13 +799,21 @@ bool tma_ok(const SkY& Y, int64_t rows, int64_t cols) {
          rows > 0 && cols > 0 && Y.ld >= cols;
 }
 
+// Units of G chunks: about two units per resident CTA (dynamic balance), at
+// most 32 groups per block (the last unit of a block sums that many tiles).
 StreamPlan stream_plan(int64_t nout, int64_t nred) {
   StreamPlan p;
-  p.nblocks = (nout + TILE - 1) / TILE;
-  p.nchunks = std::max<int64_t>((nred + TILE - 1) / TILE, 1);
-  p.total = p.nblocks * p.nchunks;
+  p.nblocks = int((nout + TILE - 1) / TILE);
+  p.nchunks = int(std::max<int64_t>((nred + TILE - 1) / TILE, 1));
   const int64_t cap = int64_t(kSMs) * kTmaCtasPerSm;
-  p.ncta = int(p.total < cap ? p.total : cap);
+  int64_t want = (2 * cap + p.nblocks - 1) / std::max(p.nblocks, 1);
+  if (want < 1) want = 1;
+  if (want > 32) want = 32;
+  if (want > p.nchunks) want = p.nchunks;
+  p.G = int((p.nchunks + want - 1) / want);
+  p.ngroups = (p.nchunks + p.G - 1) / p.G;
+  p.nunits = p.nblocks * p.ngroups;
+  p.ncta = int(std::min<int64_t>(p.nunits, cap));
   if (p.ncta < 1) p.ncta = 1;
   return p;
 }
@@ -844,7 +864,7 @@ slora_status launch_tma(bool col, const SkY& Y, int64_t M, int64_t K, int c, int
 
 int64_t tma_part_floats(int64_t nout, int64_t nred, int c) {
   const StreamPlan p = stream_plan(nout, nred);
-  return int64_t(p.ncta) * 2 * TILE * padded(c);
+  return int64_t(p.nunits) * TILE * padded(c);
 }
 }  // namespace
 
