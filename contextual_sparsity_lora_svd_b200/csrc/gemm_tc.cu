@@ -58,6 +58,13 @@ struct alignas(64) TcParams {
   const void* in0;
   const void* in1;
   long long ldi;
+  // rank-r projection of the epilogue's values (see TcGemm::proj_*)
+  const __nv_bfloat16* proj0;
+  const __nv_bfloat16* proj1;
+  long long ldproj;
+  int proj_r;
+  float* proj_part;
+  long long proj_rows;
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -215,6 +222,110 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16* row, int c0, int
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] = (c0 + j < N) ? __bfloat162float(row[c0 + j]) : 0.0f;
   }
+}
+
+// 32 consecutive bf16 of a row kept packed (4 x 16 bytes; zeros past N).
+__device__ __forceinline__ void load_row32_raw(const __nv_bfloat16* row, int c0, int N,
+                                               uint4 (&r)[4]) {
+  if (c0 + 32 <= N) {
+    const uint4* src = reinterpret_cast<const uint4*>(row + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = src[q];
+  } else {
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(r);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) h[j] = (c0 + j < N) ? row[c0 + j] : __float2bfloat16_rn(0.0f);
+  }
+}
+__device__ __forceinline__ float2 unpack2(const uint4 (&r)[4], int j2) {  // elements 2 j2, 2 j2 + 1
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(r);
+  return __bfloat1622float2(h[j2]);
+}
+
+// ---- rank-r projection of epilogue rows on the tensor cores (mma.sync)
+// Each epilogue warp stages its 32 rows x 32 values of a chunk as bf16 in a
+// padded shared buffer (80-byte rows: the 8 row addresses of an ldmatrix fall
+// in distinct bank groups), reads them back as m16n8k16 A fragments and
+// multiplies by the chunk's 32 x R slice of the projection matrix P.
+constexpr int PROJ_ROW = 40;                    // bf16 per staged row (32 + 8 padding)
+constexpr int PROJ_BUF = 32 * PROJ_ROW;         // bf16 per warp buffer
+constexpr int PROJ_SMEM = 4 * 2 * PROJ_BUF * 2;  // 4 epilogue warps x 2 buffers, bytes
+
+__device__ __forceinline__ void mma16816_tc(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Row `lane` of the warp's buffer = this lane's 32 values in bf16 (zeros if !valid).
+__device__ __forceinline__ void proj_stage(__nv_bfloat16* buf, int lane, const float* v,
+                                           bool valid) {
+  uint4* dst = reinterpret_cast<uint4*>(buf + lane * PROJ_ROW);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      h[e] = valid ? __floats2bfloat162_rn(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1])
+                   : __floats2bfloat162_rn(0.0f, 0.0f);
+    dst[q] = *reinterpret_cast<const uint4*>(h);
+  }
+}
+// acc[mb][nb] += rows mb*16.. of the staged 32 x 32 chunk times B[k][n] =
+// P[(c0 + k) * ld + n] (zero for channels c0 + k >= N), n < R.
+template <int R>
+__device__ __forceinline__ void proj_mma(float (&acc)[2][2][4], const __nv_bfloat16* buf,
+                                         const __nv_bfloat16* __restrict__ P, long long ld,
+                                         int c0, int N, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const unsigned short* Pu = reinterpret_cast<const unsigned short*>(P);
+  auto el = [&](int k, int n) -> uint32_t {
+    return (c0 + k < N) ? uint32_t(__ldg(Pu + (long long)(c0 + k) * ld + n)) : 0u;
+  };
+  uint32_t b[2][R / 8][2];
+#pragma unroll
+  for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+    for (int nb = 0; nb < R / 8; ++nb) {
+      const int k0 = kb * 16 + 2 * t, n = nb * 8 + g;
+      b[kb][nb][0] = el(k0, n) | (el(k0 + 1, n) << 16);
+      b[kb][nb][1] = el(k0 + 8, n) | (el(k0 + 9, n) << 16);
+    }
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, acol = (lane >> 4) * 8;
+#pragma unroll
+  for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      uint32_t a[4];
+      const uint32_t addr = su32(buf + (mb * 16 + arow) * PROJ_ROW + kb * 16 + acol);
+      asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                   : "r"(addr));
+#pragma unroll
+      for (int nb = 0; nb < R / 8; ++nb) mma16816_tc(acc[mb][nb], a, b[kb][nb][0], b[kb][nb][1]);
+    }
+}
+// The warp's partial of one N tile: rows rbase + mb*16 + g (+8) of the tile
+// (valid ones only), columns off + nb*8 + 2t (+1), at
+// part[((out_row + row) * n_ntiles + nt) * pc + col].
+template <int R>
+__device__ __forceinline__ void proj_store(float* part, long long out_row, int nvalid, int rbase,
+                                           int nt, int n_ntiles, int pc, int off,
+                                           const float (&acc)[2][2][4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = rbase + mb * 16 + g + 8 * h;
+      if (row >= nvalid) continue;
+      float* dst = part + ((out_row + row) * n_ntiles + nt) * pc + off;
+#pragma unroll
+      for (int nb = 0; nb < R / 8; ++nb)
+        *reinterpret_cast<float2*>(dst + nb * 8 + 2 * t) =
+            make_float2(acc[mb][nb][2 * h], acc[mb][nb][2 * h + 1]);
+    }
 }
 
 struct TileInfo {
@@ -430,7 +541,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__
           prefetch_row256(gi, ti.n0, p.N);
           prefetch_row256(ui, ti.n0, p.N);
         }
-// g and u of chunk c + 1 are loaded while chunk c is computed, so each
+        // g and u of chunk c + 1 are loaded while chunk c is computed, so each
         // chunk's global-load latency hides behind the previous chunk's math
         float gv[32], uv[32], gn[32], un[32];
         if (valid && ti.n0 < p.N) {
@@ -504,7 +615,7 @@ constexpr int STAGES2 = 6;
 constexpr int A2_BYTES = BM * BK * 2;                 // 16 KB
 constexpr int B2_BYTES = (BN / 2) * BK * 2;           // 16 KB (this CTA's half)
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;     // 32 KB
-constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512;
+constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512 + PROJ_SMEM;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -717,6 +828,9 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
     // ------------------------------------------------------------ epilogue
     const int q = warp - 4;
     const int r = q * 32 + lane;  // row within this CTA's 128-row half == TMEM lane
+    __nv_bfloat16* pbuf0 = reinterpret_cast<__nv_bfloat16*>(
+                               smem + STAGES2 * STAGE2_BYTES + 512) + q * 2 * PROJ_BUF;
+    __nv_bfloat16* pbuf1 = pbuf0 + PROJ_BUF;
     const uint32_t tempty_leader0 = map_to_rank(su32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = map_to_rank(su32(&tempty[1]), 0);
     int it = 0;
@@ -742,19 +856,33 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
         __nv_bfloat16* g = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
         __nv_bfloat16* u = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
         __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out2) + orow * p.ldo;
+        float pa[2][2][4] = {};  // rank projection of h over this tile's channels
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           tmem_ld32(tl + c * 32, v);
           tmem_ld32(tl + 128 + c * 32, w);
+          const int c0 = n0 + c * 32;
           if (valid) {
-            const int c0 = n0 + c * 32;
             store_row32(g, c0, p.N, v);
             store_row32(u, c0, p.N, w);
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]) * w[j];
             store_row32(h, c0, p.N, v);
           }
+          if (p.proj_r && c0 < p.N) {  // warp-uniform
+            proj_stage(pbuf0, lane, v, valid);
+            __syncwarp();
+            if (p.proj_r == 16)
+              proj_mma<16>(pa, pbuf0, p.proj0, p.ldproj, c0, p.N, lane);
+            else
+              proj_mma<8>(pa, pbuf0, p.proj0, p.ldproj, c0, p.N, lane);
+            __syncwarp();
+          }
         }
+        if (p.proj_r == 16)
+          proj_store<16>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 16, 0, pa, lane);
+        else if (p.proj_r == 8)
+          proj_store<8>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 8, 0, pa, lane);
       } else if (p.epi == EPI_SWIGLU_BWD) {
         const __nv_bfloat16* gi = static_cast<const __nv_bfloat16*>(p.in0) + orow * p.ldi;
         const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
@@ -764,12 +892,13 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
           prefetch_row256(gi, n0, p.N);
           prefetch_row256(ui, n0, p.N);
         }
-// g and u of chunk c + 1 are loaded while chunk c is computed, so each
+        // g and u of chunk c + 1 are loaded while chunk c is computed, so each
         // chunk's global-load latency hides behind the previous chunk's math
-        float gv[32], uv[32], gn[32], un[32];
+        uint4 gv[4], uv[4], gn[4], un[4];  // packed bf16 g and u of chunks c and c + 1
+        float pg[2][2][4] = {}, pu[2][2][4] = {};  // rank projections of dG and dU
         if (valid && n0 < p.N) {
-          load_row32(gi, n0, p.N, gv);
-          load_row32(ui, n0, p.N, uv);
+          load_row32_raw(gi, n0, p.N, gv);
+          load_row32_raw(ui, n0, p.N, uv);
         }
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -777,27 +906,54 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
           const int c0 = n0 + c * 32;
           const bool next = valid && c + 1 < 8 && c0 + 32 < p.N;
           if (next) {
-            load_row32(gi, c0 + 32, p.N, gn);
-            load_row32(ui, c0 + 32, p.N, un);
+            load_row32_raw(gi, c0 + 32, p.N, gn);
+            load_row32_raw(ui, c0 + 32, p.N, un);
           }
           if (valid && c0 < p.N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float sg = sigmoid_f(gv[j]);
-              const float dh = v[j];
-              v[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
-              w[j] = dh * gv[j] * sg;                                  // dU
+            for (int j2 = 0; j2 < 16; ++j2) {
+              const float2 g2 = unpack2(gv, j2), u2 = unpack2(uv, j2);
+              const float ga[2] = {g2.x, g2.y}, ua[2] = {u2.x, u2.y};
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int j = 2 * j2 + e;
+                const float sg = sigmoid_f(ga[e]);
+                const float dh = v[j];
+                v[j] = dh * ua[e] * sg * (1.0f + ga[e] * (1.0f - sg));  // dG
+                w[j] = dh * ga[e] * sg;                                  // dU
+              }
             }
             store_row32(dg, c0, p.N, v);
             store_row32(du, c0, p.N, w);
           }
+          if (p.proj_r && c0 < p.N) {  // warp-uniform
+            const bool ok = valid;
+            proj_stage(pbuf0, lane, v, ok);
+            proj_stage(pbuf1, lane, w, ok);
+            __syncwarp();
+            if (p.proj_r == 16) {
+              proj_mma<16>(pg, pbuf0, p.proj0, p.ldproj, c0, p.N, lane);
+              proj_mma<16>(pu, pbuf1, p.proj1, p.ldproj, c0, p.N, lane);
+            } else {
+              proj_mma<8>(pg, pbuf0, p.proj0, p.ldproj, c0, p.N, lane);
+              proj_mma<8>(pu, pbuf1, p.proj1, p.ldproj, c0, p.N, lane);
+            }
+            __syncwarp();
+          }
           if (next) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              gv[j] = gn[j];
-              uv[j] = un[j];
+            for (int q4 = 0; q4 < 4; ++q4) {
+              gv[q4] = gn[q4];
+              uv[q4] = un[q4];
             }
           }
+        }
+        if (p.proj_r == 16) {
+          proj_store<16>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 32, 0, pg, lane);
+          proj_store<16>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 32, 16, pu, lane);
+        } else if (p.proj_r == 8) {
+          proj_store<8>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 16, 0, pg, lane);
+          proj_store<8>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 16, 8, pu, lane);
         }
       } else {
         __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
@@ -875,7 +1031,18 @@ int num_sms() {
   return n;
 }
 
+int64_t tc_ntiles(const TcGemm& g) {
+  const int64_t ncols = g.paired ? BN / 2 : BN;
+  return (g.N + ncols - 1) / ncols;
+}
+
 slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
+  if (g.proj0 && (g_tc_mode != 2 || (g.proj_r != 8 && g.proj_r != 16) || g.ldproj % 8 ||
+                  !g.proj_part || (g.epi == EPI_SWIGLU_BWD && !g.proj1) || g.epi == EPI_STORE ||
+                  (reinterpret_cast<uintptr_t>(g.proj0) & 15) ||
+                  (reinterpret_cast<uintptr_t>(g.proj1) & 15) ||
+                  (reinterpret_cast<uintptr_t>(g.proj_part) & 15)))
+    SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "tcgen05 GEMM: epilogue projection not available here");
   if (g.N <= 0) return SLORA_OK;
   if (g.tiles == nullptr) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: tile list missing");
   if (g.n_mtiles <= 0) return SLORA_OK;
@@ -929,6 +1096,12 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   p.out2 = g.out2;
   p.ldo = g.ldo;
   p.in0 = g.in0;
+  p.proj0 = static_cast<const __nv_bfloat16*>(g.proj0);
+  p.proj1 = static_cast<const __nv_bfloat16*>(g.proj1);
+  p.ldproj = g.ldproj;
+  p.proj_r = g.proj0 ? g.proj_r : 0;
+  p.proj_part = g.proj_part;
+  p.proj_rows = g.proj_rows;
   p.in1 = g.in1;
   p.ldi = g.ldi;
   if (!g_attr_set) {

@@ -59,7 +59,23 @@ struct TcGemm {
   const void* in0 = nullptr;  // SWIGLU_BWD: g
   const void* in1 = nullptr;  // SWIGLU_BWD: u
   int64_t ldi = 0;
+  // Optional rank-r projection of the epilogue's values, r = proj_r in {8, 16}
+  // (one-of-two-CTA tile mode only): SWIGLU_FWD projects h with proj0,
+  // SWIGLU_BWD projects dG with proj0 and dU with proj1.  proj0/proj1 are bf16
+  // [N x ldproj] (row = output channel, ldproj a multiple of 8); each N tile
+  // writes, per output row (output layout), the fp32 partial sums over its
+  // channels to proj_part[(row * n_ntiles + nt) * pc + q], pc = r (FWD) or 2r
+  // (BWD, dU's after dG's), proj_rows rows.  reduce_row_partials() sums them.
+  const void* proj0 = nullptr;
+  const void* proj1 = nullptr;
+  int64_t ldproj = 0;
+  int proj_r = 0;
+  float* proj_part = nullptr;
+  int64_t proj_rows = 0;
 };
+
+// N tiles of a GEMM (the count the projection partials are laid out over).
+int64_t tc_ntiles(const TcGemm& g);
 
 slora_status gemm_tc(const TcGemm& g, cudaStream_t st);
 

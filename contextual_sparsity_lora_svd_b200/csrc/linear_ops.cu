@@ -240,6 +240,13 @@ struct TcBuilder {
     g.in0 = i0; g.in1 = i1; g.ldi = ldi;
     return *this;
   }
+  // rank projection of the epilogue values (h, or dG and dU), see TcGemm
+  TcBuilder& proj(const void* p0, const void* p1, int64_t ld, int pr, float* part,
+                  int64_t rows) {
+    g.proj0 = p0; g.proj1 = p1; g.ldproj = ld; g.proj_r = pr; g.proj_part = part;
+    g.proj_rows = rows;
+    return *this;
+  }
 };
 }  // namespace
 
@@ -278,6 +285,23 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   void* AdtS = bf(kk, lr);
   void* Adt = bf(Fd, lr);
   void* Bdp = bf(d, lr);
+  // rank-r projections done in the GEMM epilogues (h Ad^T in the gate|up GEMMs,
+  // [dG Bg | dU Bu] in the dh GEMMs) instead of separate passes over h, dG, dU;
+  // per-N-tile partials, summed in order by reduce_row_partials
+  const bool proj = tc_mode() == 2 && (lr == 8 || lr == 16);
+  const int64_t ntFc = (kk + 127) / 128, ntFo = (Fd + 127) / 128;  // paired gate|up tiles
+  const int64_t ntBc = (kk + 255) / 256, ntBo = (Fd + 255) / 256;  // dh tiles
+  const bool bpad = proj && (r != lr || !aligned16(L.Bg) || !aligned16(L.Bu));
+  void* BgS = proj ? bf(kk, lr) : nullptr;  // rows S of B_g, B_u (padded to lr columns)
+  void* BuS = proj ? bf(kk, lr) : nullptr;
+  void* BgP = bpad ? bf(Fd, lr) : nullptr;  // B_g, B_u padded / realigned copies
+  void* BuP = bpad ? bf(Fd, lr) : nullptr;
+  float* projC = proj ? ar.take<float>(size_t(std::max({ntFc * TC * lr, ntBc * TC * 2 * lr,
+                                                         int64_t(1)})))
+                      : nullptr;
+  float* projO = proj ? ar.take<float>(size_t(std::max({ntFo * TO * lr, ntBo * TO * 2 * lr,
+                                                         int64_t(1)})))
+                      : nullptr;
   void* AgAu = bf(2 * r, d);
   void* WgS = bf(kk, d);  // selected rows of the frozen weights, compacted once per step
   void* WuS = bf(kk, d);
@@ -360,6 +384,14 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, st));
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, st));
   SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
+  if (proj) {
+    SLORA_TRY(gather_pad(L.Bg, r, idx, kk, r, BgS, lr, st, Fd));
+    SLORA_TRY(gather_pad(L.Bu, r, idx, kk, r, BuS, lr, st, Fd));
+    if (bpad) {
+      SLORA_TRY(gather_pad(L.Bg, r, nullptr, Fd, r, BgP, lr, st, Fd));
+      SLORA_TRY(gather_pad(L.Bu, r, nullptr, Fd, r, BuP, lr, st, Fd));
+    }
+  }
 
   // ---- forward
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
@@ -367,6 +399,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, nullptr, 0, 1, mat(WuS, kk, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpC, nntC * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gC, uC, hC, ldk);
+    if (proj) b.proj(AdtS, nullptr, lr, int(lr), projC, TC);
     SLORA_TRY(gemm_tc(b.g, st));
   }
   {  // gate|up, output rows, every channel
@@ -374,15 +407,21 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K, d, nullptr, 0, 1, mat(L.Wu, Fd, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpO, nntO * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gO, uO, hO, Fd);
+    if (proj) b.proj(Adt, nullptr, lr, int(lr), projO, TO);
     SLORA_TRY(gemm_tc(b.g, st));
   }
   {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
     SkRowOut oc;
     oc.out1 = hA; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = hAbC; oc.ld2 = lr; oc.s2 = s;
-    SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx, Fd), r, oc, sw, st));
     SkRowOut oo;
     oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, sw, st));
+    if (proj) {
+      SLORA_TRY(reduce_row_partials(projC, int(ntFc), TC, int(lr), int(lr), r, oc, st));
+      SLORA_TRY(reduce_row_partials(projO, int(ntFo), TO, int(lr), int(lr), r, oo, st));
+    } else {
+      SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx, Fd), r, oc, sw, st));
+      SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, sw, st));
+    }
   }
   {  // down projection, context rows: reads channels S only (rows S of Wd^T)
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -414,6 +453,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .seg(mat(dOBb, T, r, lr), mat(AdtS, kk, r, lr), B_K, r)
         .out(dGC, dUC, nullptr, ldk)
         .in(gC, uC, ldk);
+    if (proj) b.proj(BgS, BuS, lr, int(lr), projC, TC);
     SLORA_TRY(gemm_tc(b.g, st));
   }
   {
@@ -422,6 +462,8 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .seg(mat(dOBb, T, r, lr), mat(Adt, Fd, r, lr), B_K, r)
         .out(dGO, dUO, nullptr, Fd)
         .in(gO, uO, Fd);
+    if (proj)
+      b.proj(bpad ? BgP : L.Bg, bpad ? BuP : L.Bu, bpad ? lr : r, int(lr), projO, TO);
     SLORA_TRY(gemm_tc(b.g, st));
   }
   {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
@@ -432,20 +474,31 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     cc.kmap = idx; cc.kmap_limit = Fd; cc.accumulate = 1;
     SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, sw, st));
   }
-  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu]; dB = s dG^T XA on the same stream
+  if (proj) {  // dGB = [dG Bg | dU Bu] from the dh GEMMs' epilogue partials
+    SkRowOut oc;
+    oc.out1 = dGB; oc.ld1 = 2 * r; oc.map1 = ctx_rows; oc.out2 = dGBbC; oc.ld2 = lr2; oc.s2 = s;
+    SLORA_TRY(reduce_row_partials(projC, int(ntBc), TC, int(2 * lr), int(lr), r, oc, st));
+    SkRowOut oo = oc;
+    oo.map1 = out_rows; oo.out2 = dGBbO;
+    SLORA_TRY(reduce_row_partials(projO, int(ntBo), TO, int(2 * lr), int(lr), r, oo, st));
+  }
+  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu] (when not fused); dB = s dG^T XA
     const void* Bm = p ? L.Bu : L.Bg;
     float* dBm = p ? G.dBu : G.dBg;
     SkRowOut oo;
     oo.out1 = dGB; oo.ld1 = 2 * r; oo.off1 = p * r; oo.map1 = out_rows;
     oo.out2 = dGBbO; oo.ld2 = lr2; oo.off2 = p * r; oo.s2 = s;
-    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, sw, st));
+    if (!proj)
+      SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, sw, st));
     SkColOut bo;
     bo.out = dBm; bo.ldo = r; bo.scale = s;
     SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
                      bo, sw, st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
-    SLORA_TRY(rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx, Fd), r, oc, sw, st));
+    if (!proj)
+      SLORA_TRY(
+          rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx, Fd), r, oc, sw, st));
     SkColOut bc = bo;
     bc.kmap = idx; bc.kmap_limit = Fd; bc.accumulate = 1;
     SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,

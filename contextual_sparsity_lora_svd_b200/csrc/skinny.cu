@@ -766,6 +766,32 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
   }
 }
 
+// Sum of per-N-tile projection partials written by a GEMM epilogue: thread
+// (row m, column q) adds part[(m * nparts + t) * pc + q] over t = 0 .. nparts-1
+// in order (eight loads in flight), then emits column (q / lr) * r + q % lr
+// for q % lr < r (groups of lr padded columns, r used) through the rowdot
+// output descriptor.
+__global__ void reduce_rows_kernel(const float* __restrict__ part, int nparts, int64_t M,
+                                   int pc, int lr, int r, const SkRowOut o) {
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= M * pc) return;
+  const int64_t m = e / pc;
+  const int q = int(e % pc);
+  const float* src = part + m * int64_t(nparts) * pc + q;
+  float v = 0.0f;
+  int t = 0;
+  for (; t + 8 <= nparts; t += 8) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + int64_t(t + u) * pc);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v += x[u];
+  }
+  for (; t < nparts; ++t) v += __ldcg(src + int64_t(t) * pc);
+  const int gi = q / lr, qq = q % lr;
+  if (qq < r) row_emit(o, m, gi * r + qq, v);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_sk_encode = nullptr;
 std::once_flag g_sk_encode_once;
 
@@ -880,6 +906,16 @@ int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
   const Geo a = geometry(K, M, c, false), b = geometry(K, M, c, true);
   return std::max(int64_t(std::max(a.nsplit, b.nsplit)) * std::max<int64_t>(K, 1) * padded(c),
                   tma_part_floats(K, M, c));
+}
+
+slora_status reduce_row_partials(const float* part, int nparts, int64_t M, int pc, int lr, int r,
+                                 const SkRowOut& o, cudaStream_t st) {
+  if (M <= 0 || pc <= 0) return SLORA_OK;
+  const int64_t n = M * pc;
+  LaunchScope ls(kSkinny, double(n) * nparts * 4 + double(M) * r * (pc / lr) * 6, st);
+  reduce_rows_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(part, nparts, M, pc, lr, r, o);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
 }
 
 slora_status skinny_set_wait_budget(long long cycles) {

@@ -92,6 +92,12 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkRowOut& o, const SkWork& w, cudaStream_t st);
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkColOut& o, const SkWork& w, cudaStream_t st);
+// Rows of a rank projection computed in a GEMM epilogue (TcGemm::proj_*):
+// out(m, g * r + q) = sum over t < nparts of part[(m * nparts + t) * pc + g * lr + q]
+// for q < r, g < pc / lr, emitted through `o` exactly as rowdot emits column
+// g * r + q.  Fixed summation order (bit-reproducible).
+slora_status reduce_row_partials(const float* part, int nparts, int64_t M, int pc, int lr, int r,
+                                 const SkRowOut& o, cudaStream_t st);
 // Device error flag of the TMA kernel (a bounded wait that expired).
 slora_status skinny_check_error(bool clear);
 // Budget of the TMA kernel's pipeline waits in SM clock cycles (< 0: default).
