@@ -112,7 +112,7 @@ EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int6
   }
   const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
   eb.scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
-  eb.nsplit = ffn_score_splits(ti.T_C, n0);
+  eb.nsplit = ffn_score_splits(ti.T_C, n0, rank);
   if (crit == SLORA_CRIT_FFN_SWIGLU_L2)
     eb.partial = ar.take<float>(size_t(eb.nsplit) * n0);
   else

@@ -11,32 +11,42 @@ namespace slora {
 namespace {
 
 // ---------------------------------------------------------------- FFN score
-// One thread per intermediate channel j, one block column per token chunk.
-// The thread keeps U_g[j,:], U_u[j,:] in registers and streams the chunk's
-// P rows through shared memory (broadcast reads).
+// Each thread scores CPT channels (c = first + 128 * i) over one token chunk:
+// it keeps their U_g, U_u rows in registers and reads each token's projected
+// row P_g | P_u from shared memory as 16-byte broadcasts, reused for its CPT
+// channels (the shared-memory reads, not the math, bounded the one-channel
+// version).  Partial sums of squares per (chunk, channel), fixed token order.
+constexpr int kScoreTT = 32;  // tokens staged per round
+template <int RP>
+constexpr int score_cpt() { return RP <= 8 ? 4 : (RP <= 16 ? 2 : 1); }
+
 template <int RP>
 __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
     const float* __restrict__ P, int64_t ldp, const int32_t* __restrict__ pmap, int64_t T_C,
     const float* __restrict__ Ug, const float* __restrict__ Uu, int64_t n, int r, int64_t chunk,
     float* __restrict__ partial) {
-  constexpr int TT = 32;
-  __shared__ float sp[TT][2 * RP];
-  const int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  constexpr int CPT = score_cpt<RP>();
+  __shared__ __align__(16) float sp[kScoreTT][2 * RP];
+  const int64_t j0 = int64_t(blockIdx.x) * 128 * CPT + threadIdx.x;
   const int64_t t0 = int64_t(blockIdx.y) * chunk;
   const int64_t t1 = min(T_C, t0 + chunk);
-  float ug[RP], uu[RP];
+  float ug[CPT][RP], uu[CPT][RP], acc[CPT];
 #pragma unroll
-  for (int q = 0; q < RP; ++q) {
-    ug[q] = (j < n && q < r) ? Ug[j * r + q] : 0.0f;
-    uu[q] = (j < n && q < r) ? Uu[j * r + q] : 0.0f;
+  for (int i = 0; i < CPT; ++i) {
+    const int64_t j = j0 + 128 * i;
+    acc[i] = 0.0f;
+#pragma unroll
+    for (int q = 0; q < RP; ++q) {
+      ug[i][q] = (j < n && q < r) ? Ug[j * r + q] : 0.0f;
+      uu[i][q] = (j < n && q < r) ? Uu[j * r + q] : 0.0f;
+    }
   }
-  float acc = 0.0f;
-  for (int64_t tb = t0; tb < t1; tb += TT) {
-    const int nt = int((t1 - tb) < TT ? (t1 - tb) : TT);
+  for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
+    const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
     __syncthreads();
-    for (int e = threadIdx.x; e < TT * 2 * RP; e += blockDim.x) {
-      int tt = e / (2 * RP), q = e % (2 * RP);
-      int half = q / RP, qq = q % RP;
+    for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x) {
+      const int tt = e / (2 * RP), q = e % (2 * RP);
+      const int half = q / RP, qq = q % RP;
       float v = 0.0f;
       if (tt < nt && qq < r) {
         const int64_t row = pmap ? int64_t(pmap[tb + tt]) : tb + tt;
@@ -46,17 +56,32 @@ __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
     }
     __syncthreads();
     for (int tt = 0; tt < nt; ++tt) {
-      float g = 0.0f, u = 0.0f;
+      float pg[RP], pu[RP];
 #pragma unroll
-      for (int q = 0; q < RP; ++q) {
-        g = fmaf(sp[tt][q], ug[q], g);
-        u = fmaf(sp[tt][RP + q], uu[q], u);
+      for (int q4 = 0; q4 < RP / 4; ++q4) {
+        const float4 a = *reinterpret_cast<const float4*>(&sp[tt][4 * q4]);
+        const float4 b = *reinterpret_cast<const float4*>(&sp[tt][RP + 4 * q4]);
+        pg[4 * q4] = a.x; pg[4 * q4 + 1] = a.y; pg[4 * q4 + 2] = a.z; pg[4 * q4 + 3] = a.w;
+        pu[4 * q4] = b.x; pu[4 * q4 + 1] = b.y; pu[4 * q4 + 2] = b.z; pu[4 * q4 + 3] = b.w;
       }
-      float a = silu_f(g) * u;
-      acc = fmaf(a, a, acc);
+#pragma unroll
+      for (int i = 0; i < CPT; ++i) {
+        float g = 0.0f, u = 0.0f;
+#pragma unroll
+        for (int q = 0; q < RP; ++q) {
+          g = fmaf(pg[q], ug[i][q], g);
+          u = fmaf(pu[q], uu[i][q], u);
+        }
+        const float a = silu_f(g) * u;
+        acc[i] = fmaf(a, a, acc[i]);
+      }
     }
   }
-  if (j < n) partial[int64_t(blockIdx.y) * n + j] = acc;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int64_t j = j0 + 128 * i;
+    if (j < n) partial[int64_t(blockIdx.y) * n + j] = acc[i];
+  }
 }
 
 __global__ void sumsq_finalize_kernel(const float* __restrict__ partial, int nsplit, int64_t n,
@@ -160,16 +185,32 @@ __global__ void __launch_bounds__(1024) topk_select_kernel(const float* __restri
       if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t cum = 0, want = s_want;
-      for (int dg = 255; dg >= 0; --dg) {
-        uint32_t h = hist[dg];
-        if (cum + h >= want) {
-          s_prefix = prefix | (uint32_t(dg) << shift);
-          s_want = want - cum;
-          break;
+    if (wid == 0) {  // the digit holding the want-th largest key: a warp-parallel scan
+      // lane l owns digits 255 - 8l down to 248 - 8l (descending key order)
+      const uint32_t want = s_want;
+      uint32_t own = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) own += hist[255 - 8 * lane - i];
+      uint32_t incl = own;  // inclusive prefix over lanes 0..l
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= want);
+      const int l = __ffs(hit) - 1;  // want <= count of keys with this prefix, so l exists
+      if (lane == l) {
+        uint32_t cum = incl - own;
+        for (int i = 0; i < 8; ++i) {
+          const int dg = 255 - 8 * lane - i;
+          const uint32_t h = hist[dg];
+          if (cum + h >= want) {
+            s_prefix = prefix | (uint32_t(dg) << shift);
+            s_want = want - cum;
+            break;
+          }
+          cum += h;
         }
-        cum += h;
       }
     }
     __syncthreads();
@@ -216,10 +257,12 @@ __global__ void __launch_bounds__(1024) topk_select_kernel(const float* __restri
 
 }  // namespace
 
-int ffn_score_splits(int64_t T_C, int64_t n) {
-  int64_t nb = (n + 127) / 128;
-  int64_t want = (4 * 148 + nb - 1) / nb;
-  int64_t maxs = (T_C + 31) / 32;
+int score_cpt_for(int r) { return r <= 8 ? 4 : (r <= 16 ? 2 : 1); }
+
+int ffn_score_splits(int64_t T_C, int64_t n, int r) {
+  const int64_t nb = (n + 128 * score_cpt_for(r) - 1) / (128 * score_cpt_for(r));
+  int64_t want = (6 * 148 + nb - 1) / nb;  // about six 128-thread blocks per SM
+  int64_t maxs = (T_C + kScoreTT - 1) / kScoreTT;
   int64_t s = want < maxs ? want : maxs;
   if (s < 1) s = 1;
   if (s > 64) s = 64;
@@ -231,7 +274,8 @@ slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_
                         int nsplit, float* scores, cudaStream_t st) {
   if (n <= 0) return SLORA_OK;
   const int64_t chunk = T_C > 0 ? (T_C + nsplit - 1) / nsplit : 1;
-  dim3 grid(unsigned((n + 127) / 128), unsigned(nsplit));
+  dim3 grid(unsigned((n + 128 * score_cpt_for(r) - 1) / (128 * score_cpt_for(r))),
+            unsigned(nsplit));
   {
   LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 + double(nsplit) * n * 4, st);
   if (r <= 8)

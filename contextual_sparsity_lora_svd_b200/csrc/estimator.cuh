@@ -12,7 +12,7 @@ namespace slora {
 slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
                         const float* Ug, const float* Uu, int64_t n, int r, float* partial,
                         int nsplit, float* scores, cudaStream_t st);
-int ffn_score_splits(int64_t T_C, int64_t n);
+int ffn_score_splits(int64_t T_C, int64_t n, int r);
 
 // QK: Gram matrices of P_q (cols [0,r)) and P_k (cols [r,2r)) in fp64, then
 // score[g, c] = ||K_hat[:, g, c]|| * sum_{h in g} ||Q_hat[:, h, c]||.
