@@ -333,6 +333,33 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   sw.part = part;
   sw.rsplit = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, d, Fd}))));
   sw.counters = rsp;
+  // split rank-r operands of the skinny contractions, prepared in three
+  // batched launches (prep_r_batch) instead of one launch per contraction
+  auto rsbuf = [&](int64_t I) {
+    return static_cast<void*>(ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(I))));
+  };
+  void* rsX = rsbuf(d);
+  void* rsBd = rsbuf(d);
+  void* rsHA = rsbuf(T);
+  void* rsDobO = rsbuf(TO);
+  void* rsDobC = rsbuf(TC);
+  void* rsXA[2][2];
+  for (int p = 0; p < 2; ++p) {
+    rsXA[p][0] = rsbuf(TO);
+    rsXA[p][1] = rsbuf(TC);
+  }
+  void* rsDgb = rsbuf(T);
+  auto prepared = [&](void* rs) {
+    SkWork w = sw;
+    w.rsplit = rs;
+    w.prepared = true;
+    return w;
+  };
+  auto job = [](const SkR& Rr, int c, int64_t I, void* rs) {
+    SkPrep j;
+    j.R = Rr; j.c = c; j.I = I; j.rs = rs;
+    return j;
+  };
   float* LgLu = fused ? ar.take<float>(size_t(d) * 2 * rs) : nullptr;
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   EstBufs eb;
@@ -364,7 +391,9 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       o.qsplit = 2 * r; o.out1b = Pfull; o.ld1b = 2 * rs;
       c = 2 * r + 2 * rs;
     }
-    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, sw, st));
+    const SkPrep jobs[2] = {job(rr, c, d, rsX), job(Rv(L.Bd, kBF16, r, 1), r, d, rsBd)};
+    SLORA_TRY(prep_r_batch(jobs, 2, st));
+    SLORA_TRY(rowdot(Yv(X, d), T, d, rr, c, o, prepared(rsX), st));
   }
   if (idx_force) {
     if (kk > 0)
@@ -416,8 +445,8 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkRowOut oo;
     oo.out1 = hA; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = hAbO; oo.ld2 = lr; oo.s2 = s;
     if (proj) {
-      SLORA_TRY(reduce_row_partials(projC, int(ntFc), TC, int(lr), int(lr), r, oc, st));
-      SLORA_TRY(reduce_row_partials(projO, int(ntFo), TO, int(lr), int(lr), r, oo, st));
+      SLORA_TRY(reduce_row_partials(projC, int(ntFc), TC, oc, projO, int(ntFo), TO, oo, int(lr),
+                                    int(lr), r, st));
     } else {
       SLORA_TRY(rowdot(Yv(hC, ldk), TC, kk, Rv(L.Ad, kBF16, 1, Fd, idx, Fd), r, oc, sw, st));
       SLORA_TRY(rowdot(Yv(hO, Fd), TO, Fd, Rv(L.Ad, kBF16, 1, Fd), r, oo, sw, st));
@@ -442,10 +471,20 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dOB = dOut Bd: fp32 and s*dOB bf16; dBd = s dOut^T hA (same stream of dOut)
     SkRowOut o;
     o.out1 = dOB; o.ld1 = r; o.out2 = dOBb; o.ld2 = lr; o.s2 = s;
-    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, sw, st));
+    SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, prepared(rsBd), st));
+    // every operand that hA, dOB and XA feed, split in one launch
+    const SkPrep jobs[7] = {
+        job(Rv(hA, kF32, r, 1), r, T, rsHA),
+        job(Rv(dOB, kF32, r, 1, out_rows), r, TO, rsDobO),
+        job(Rv(dOB, kF32, r, 1, ctx_rows), r, TC, rsDobC),
+        job(Rv(XA, kF32, 2 * r, 1, out_rows), r, TO, rsXA[0][0]),
+        job(Rv(XA, kF32, 2 * r, 1, ctx_rows), r, TC, rsXA[0][1]),
+        job(Rv(XA + r, kF32, 2 * r, 1, out_rows), r, TO, rsXA[1][0]),
+        job(Rv(XA + r, kF32, 2 * r, 1, ctx_rows), r, TC, rsXA[1][1])};
+    SLORA_TRY(prep_r_batch(jobs, 7, st));
     SkColOut c;
     c.out = G.dBd; c.ldo = r; c.scale = s;
-    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, sw, st));
+    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, prepared(rsHA), st));
   }
   {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
@@ -469,18 +508,20 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
     SkColOut co;
     co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
-    SLORA_TRY(coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, sw, st));
+    SLORA_TRY(
+        coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, prepared(rsDobO), st));
     SkColOut cc = co;
     cc.kmap = idx; cc.kmap_limit = Fd; cc.accumulate = 1;
-    SLORA_TRY(coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, sw, st));
+    SLORA_TRY(
+        coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, prepared(rsDobC), st));
   }
   if (proj) {  // dGB = [dG Bg | dU Bu] from the dh GEMMs' epilogue partials
     SkRowOut oc;
     oc.out1 = dGB; oc.ld1 = 2 * r; oc.map1 = ctx_rows; oc.out2 = dGBbC; oc.ld2 = lr2; oc.s2 = s;
-    SLORA_TRY(reduce_row_partials(projC, int(ntBc), TC, int(2 * lr), int(lr), r, oc, st));
     SkRowOut oo = oc;
     oo.map1 = out_rows; oo.out2 = dGBbO;
-    SLORA_TRY(reduce_row_partials(projO, int(ntBo), TO, int(2 * lr), int(lr), r, oo, st));
+    SLORA_TRY(reduce_row_partials(projC, int(ntBc), TC, oc, projO, int(ntBo), TO, oo,
+                                  int(2 * lr), int(lr), r, st));
   }
   for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu] (when not fused); dB = s dG^T XA
     const void* Bm = p ? L.Bu : L.Bg;
@@ -493,7 +534,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkColOut bo;
     bo.out = dBm; bo.ldo = r; bo.scale = s;
     SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
-                     bo, sw, st));
+                     bo, prepared(rsXA[p][0]), st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
     if (!proj)
@@ -502,7 +543,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SkColOut bc = bo;
     bc.kmap = idx; bc.kmap_limit = Fd; bc.accumulate = 1;
     SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
-                     bc, sw, st));
+                     bc, prepared(rsXA[p][1]), st));
   }
   {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);
@@ -523,7 +564,9 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   {  // dAg | dAu = s dGB^T X over every row, one stream of X
     SkColOut c;
     c.out = G.dAg; c.out_b = G.dAu; c.qsplit = r; c.ldo = d; c.trans = 1; c.scale = s;
-    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, sw, st));
+    const SkPrep jg = job(Rv(dGB, kF32, 2 * r, 1), 2 * r, T, rsDgb);
+    SLORA_TRY(prep_r_batch(&jg, 1, st));
+    SLORA_TRY(coldot(Yv(X, d), T, d, Rv(dGB, kF32, 2 * r, 1), 2 * r, c, prepared(rsDgb), st));
   }
   return SLORA_OK;
 }

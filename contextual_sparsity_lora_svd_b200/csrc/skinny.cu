@@ -124,6 +124,36 @@ __global__ void prep_r_kernel(const SkR R, int c, int CP, int64_t I, int64_t I64
   for (int s = 0; s < NT; ++s) RS[(int64_t(s) * CP + q) * I64 + i] = tv[s];
 }
 
+// Several operands at once: blockIdx.y picks the job.
+struct PrepBatch {
+  SkR R[8];
+  int c[8], CP[8], nt[8];
+  int64_t I[8], I64[8];
+  __nv_bfloat16* RS[8];
+};
+__global__ void prep_r_batch_kernel(const PrepBatch b) {
+  const int k = blockIdx.y;
+  const int CP = b.CP[k];
+  const int64_t I64 = b.I64[k];
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= int64_t(CP) * I64) return;
+  const SkR& R = b.R[k];
+  const bool q_fast = R.sq == 1 && (R.ptr_b == nullptr || R.sq_b == 1);
+  int q;
+  int64_t i;
+  if (q_fast) {
+    q = int(e % CP);
+    i = e / CP;
+  } else {
+    q = int(e / I64);
+    i = e % I64;
+  }
+  const float v = (q < b.c[k] && i < b.I[k]) ? load_r(R, i, q) : 0.0f;
+  __nv_bfloat16 tv[3];
+  if (b.nt[k] == 3) split_terms<3>(v, tv); else split_terms<1>(v, tv);
+  for (int s = 0; s < b.nt[k]; ++s) b.RS[k][(int64_t(s) * CP + q) * I64 + i] = tv[s];
+}
+
 // Pipeline depth from the shared memory of one stage (Y tile + split R tile).
 constexpr int stage_bytes(int CP, int NT) { return TILE * PAD * 2 + NT * CP * PAD * 2; }
 constexpr int stages_for(int CP, int NT) { return stage_bytes(CP, NT) <= 16896 ? 4 : 3; }
@@ -766,30 +796,62 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
   }
 }
 
-// Sum of per-N-tile projection partials written by a GEMM epilogue: thread
-// (row m, column q) adds part[(m * nparts + t) * pc + q] over t = 0 .. nparts-1
-// in order (eight loads in flight), then emits column (q / lr) * r + q % lr
-// for q % lr < r (groups of lr padded columns, r used) through the rowdot
-// output descriptor.
-__global__ void reduce_rows_kernel(const float* __restrict__ part, int nparts, int64_t M,
-                                   int pc, int lr, int r, const SkRowOut o) {
+// Sum of per-N-tile projection partials written by a GEMM epilogue.  Four
+// consecutive lanes share one (row m, 4 columns q0..q0+3): lane s adds the
+// float4s of tiles t = s, s + 4, ... in order (eight in flight), then the four
+// sums combine as (l0 + l1) + (l2 + l3) through xor shuffles, which every lane
+// of the four computes with the same operands (fixed order, bit-reproducible).
+// Column q of row m is emitted as (q / lr) * r + q % lr when q % lr < r.  Up to
+// two independent jobs per launch (blockIdx.y).
+struct RowReduceJob {
+  const float* part = nullptr;
+  int nparts = 0;
+  int64_t M = 0;
+  SkRowOut o;
+};
+__global__ void reduce_rows_kernel(const RowReduceJob j0, const RowReduceJob j1, int pc, int lr,
+                                   int r) {
+  const RowReduceJob& J = blockIdx.y ? j1 : j0;
+  const int nq4 = pc / 4;
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= M * pc) return;
-  const int64_t m = e / pc;
-  const int q = int(e % pc);
-  const float* src = part + m * int64_t(nparts) * pc + q;
-  float v = 0.0f;
-  int t = 0;
-  for (; t + 8 <= nparts; t += 8) {
-    float x[8];
+  const int64_t item = e >> 2;
+  const int sub = int(e & 3);
+  const bool live = item < J.M * nq4;  // whole groups of four lanes share `live`
+  const int64_t m = live ? item / nq4 : 0;
+  const int q0 = live ? int(item % nq4) * 4 : 0;
+  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (live) {
+    const float4* src = reinterpret_cast<const float4*>(J.part + m * int64_t(J.nparts) * pc + q0);
+    const int64_t stride4 = pc / 4;
+    int t = sub;
+    for (; t + 28 < J.nparts; t += 32) {
+      float4 x[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + int64_t(t + u) * pc);
+      for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + int64_t(t + 4 * u) * stride4);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v += x[u];
+      for (int u = 0; u < 8; ++u) {
+        v.x += x[u].x; v.y += x[u].y; v.z += x[u].z; v.w += x[u].w;
+      }
+    }
+    for (; t < J.nparts; t += 4) {
+      const float4 x = __ldcg(src + int64_t(t) * stride4);
+      v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+    }
   }
-  for (; t < nparts; ++t) v += __ldcg(src + int64_t(t) * pc);
-  const int gi = q / lr, qq = q % lr;
-  if (qq < r) row_emit(o, m, gi * r + qq, v);
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, off);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, off);
+    v.z += __shfl_xor_sync(0xffffffffu, v.z, off);
+    v.w += __shfl_xor_sync(0xffffffffu, v.w, off);
+  }
+  if (!live || sub != 0) return;
+  const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int q = q0 + u, gi = q / lr, qq = q % lr;
+    if (qq < r) row_emit(J.o, m, gi * r + qq, vv[u]);
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_sk_encode = nullptr;
@@ -908,12 +970,19 @@ int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
                   tma_part_floats(K, M, c));
 }
 
-slora_status reduce_row_partials(const float* part, int nparts, int64_t M, int pc, int lr, int r,
-                                 const SkRowOut& o, cudaStream_t st) {
-  if (M <= 0 || pc <= 0) return SLORA_OK;
-  const int64_t n = M * pc;
-  LaunchScope ls(kSkinny, double(n) * nparts * 4 + double(M) * r * (pc / lr) * 6, st);
-  reduce_rows_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(part, nparts, M, pc, lr, r, o);
+slora_status reduce_row_partials(const float* part0, int nparts0, int64_t M0, const SkRowOut& o0,
+                                 const float* part1, int nparts1, int64_t M1, const SkRowOut& o1,
+                                 int pc, int lr, int r, cudaStream_t st) {
+  if ((M0 <= 0 && M1 <= 0) || pc <= 0) return SLORA_OK;
+  if (pc % 4 || lr % 4) SLORA_FAIL(SLORA_ERR_SHAPE, "reduce_row_partials: pc, lr not multiples of 4");
+  RowReduceJob j0, j1;
+  j0.part = part0; j0.nparts = nparts0; j0.M = M0 > 0 ? M0 : 0; j0.o = o0;
+  j1.part = part1; j1.nparts = nparts1; j1.M = M1 > 0 ? M1 : 0; j1.o = o1;
+  const int64_t threads = std::max(j0.M, j1.M) * (pc / 4) * 4;
+  LaunchScope ls(kSkinny,
+                 (double(j0.M) * nparts0 + double(j1.M) * nparts1) * pc * 4 +
+                     double(j0.M + j1.M) * r * (pc / lr) * 6, st);
+  reduce_rows_kernel<<<dim3(unsigned((threads + 255) / 256), 2u), 256, 0, st>>>(j0, j1, pc, lr, r);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
@@ -945,6 +1014,31 @@ int64_t skinny_counter_count(int64_t M, int64_t K) {
   return std::max<int64_t>((M + TILE - 1) / TILE, (K + TILE - 1) / TILE) + 1;
 }
 
+slora_status prep_r_batch(const SkPrep* jobs, int n, cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  if (n > 8) SLORA_FAIL(SLORA_ERR_SHAPE, "prep_r_batch: %d jobs (max 8)", n);
+  PrepBatch b{};
+  int64_t most = 1;
+  double bytes = 0;
+  for (int k = 0; k < n; ++k) {
+    const SkPrep& j = jobs[k];
+    if (j.c <= 0 || j.c > 64) SLORA_FAIL(SLORA_ERR_SHAPE, "prep_r_batch: %d columns", j.c);
+    b.R[k] = j.R;
+    b.c[k] = j.c;
+    b.CP[k] = padded(j.c);
+    b.nt[k] = fp32_terms(j.R) ? 3 : 1;
+    b.I[k] = j.I;
+    b.I64[k] = round64(std::max<int64_t>(j.I, 1));
+    b.RS[k] = static_cast<__nv_bfloat16*>(j.rs);
+    most = std::max(most, int64_t(b.CP[k]) * b.I64[k]);
+    bytes += double(j.I) * j.c * (j.R.dt == kF32 ? 4 : 2) + double(b.nt[k]) * b.CP[k] * b.I64[k] * 2;
+  }
+  LaunchScope ls(kSkinny, bytes, st);
+  prep_r_batch_kernel<<<dim3(unsigned((most + 255) / 256), unsigned(n)), 256, 0, st>>>(b);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
 slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, const SkRowOut& o,
                     const SkWork& w, cudaStream_t st) {
   if (M <= 0 || c <= 0) return SLORA_OK;
@@ -953,7 +1047,7 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
   const int CP = g.CP, cps = g.cps;
   const int64_t I64 = round64(std::max<int64_t>(K, 1));
   const __nv_bfloat16* RS = static_cast<const __nv_bfloat16*>(w.rsplit);
-  SLORA_TRY(prep_r(R, c, CP, K, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
+  if (!w.prepared) SLORA_TRY(prep_r(R, c, CP, K, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
   if (tma_ok(Y, M, K)) return launch_tma(false, Y, M, K, c, g.nt, o, SkColOut(), w, I64, st);
   const dim3 grid = dim3(unsigned(g.nblocks), unsigned(g.nsplit), 1u);
   LaunchScope ls(kSkinny,
@@ -975,7 +1069,7 @@ slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
   const int CP = g.CP, cps = g.cps;
   const int64_t I64 = round64(std::max<int64_t>(M, 1));
   const __nv_bfloat16* RS = static_cast<const __nv_bfloat16*>(w.rsplit);
-  SLORA_TRY(prep_r(R, c, CP, M, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
+  if (!w.prepared) SLORA_TRY(prep_r(R, c, CP, M, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
   if (tma_ok(Y, M, K)) return launch_tma(true, Y, M, K, c, g.nt, SkRowOut(), o, w, I64, st);
   const dim3 grid = dim3(unsigned(g.nblocks), unsigned(g.nsplit), 1u);
   LaunchScope ls(kSkinny,

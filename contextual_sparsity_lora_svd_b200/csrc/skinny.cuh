@@ -81,7 +81,21 @@ struct SkWork {
   float* part = nullptr;
   void* rsplit = nullptr;
   unsigned* counters = nullptr;
+  bool prepared = false;  // rsplit already holds this call's split operand (prep_r_batch)
 };
+
+// One rank-sized operand to split ahead of its contraction: R with c columns
+// over I indices (I = K for a rowdot, M for a coldot) into rs (bf16,
+// skinny_rsplit_elems(I) elements), exactly as the contraction would.
+struct SkPrep {
+  SkR R;
+  int c = 0;
+  int64_t I = 0;
+  void* rs = nullptr;
+};
+// Splits up to 8 operands in one launch; the contractions then run with
+// SkWork{.rsplit = rs, .prepared = true}.
+slora_status prep_r_batch(const SkPrep* jobs, int n, cudaStream_t st);
 
 // c = number of R columns (1..64).
 int64_t rowdot_part_floats(int64_t M, int64_t K, int c);
@@ -92,12 +106,14 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkRowOut& o, const SkWork& w, cudaStream_t st);
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkColOut& o, const SkWork& w, cudaStream_t st);
-// Rows of a rank projection computed in a GEMM epilogue (TcGemm::proj_*):
-// out(m, g * r + q) = sum over t < nparts of part[(m * nparts + t) * pc + g * lr + q]
-// for q < r, g < pc / lr, emitted through `o` exactly as rowdot emits column
-// g * r + q.  Fixed summation order (bit-reproducible).
-slora_status reduce_row_partials(const float* part, int nparts, int64_t M, int pc, int lr, int r,
-                                 const SkRowOut& o, cudaStream_t st);
+// Rows of a rank projection computed in GEMM epilogues (TcGemm::proj_*), two
+// jobs per launch (typically the context-row and the output-row GEMM):
+// out_k(m, g * r + q) = sum over t < nparts_k of part_k[(m * nparts_k + t) * pc + g * lr + q]
+// for q < r, g < pc / lr, emitted through o_k exactly as rowdot emits column
+// g * r + q.  Fixed summation order (bit-reproducible).  pc, lr multiples of 4.
+slora_status reduce_row_partials(const float* part0, int nparts0, int64_t M0, const SkRowOut& o0,
+                                 const float* part1, int nparts1, int64_t M1, const SkRowOut& o1,
+                                 int pc, int lr, int r, cudaStream_t st);
 // Device error flag of the TMA kernel (a bounded wait that expired).
 slora_status skinny_check_error(bool clear);
 // Budget of the TMA kernel's pipeline waits in SM clock cycles (< 0: default).
