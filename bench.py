@@ -260,7 +260,9 @@ def config_dict(world):
             "d_ff": w["d_ff"], "ctx_frac": 1 - w["out_frac"], "sparsity": w["sparsity"],
             "r_svd": w["r_svd"], "r_lora": w["r_lora"],
             "parallelism": f"dp{world}" if world > 1 else "single",
-            "l2": "flushed between timed steps (256 MiB write, outside the timed events)"}
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+            "launch": "one slora_ffn_fwd_bwd call captured as a CUDA graph, replayed per step "
+                      "(per-kernel times from a separate eager pass)"}
 
 
 def run_reference(args, rank, world):
@@ -307,11 +309,33 @@ def run_ours(args, rank, world):
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
+    # one step captured as a CUDA graph per buffer set (the library call is
+    # capture-safe: fixed buffers and tensor maps per workspace); the headline
+    # and end-to-end passes replay it, the per-kernel profiled pass runs eagerly
+    if len(G.io) < 2:
+        G.io.append(G.make_io(torch.empty_like(G.X), torch.empty_like(G.dOut)))
+
+    def capture(io):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            G.step(torch.cuda.current_stream(), io)
+        return g
+
+    graphs = [capture(io) for io in G.io]
+    torch.cuda.synchronize()
+
+    def graph_step():
+        graphs[0].replay()
+        dp.allreduce_grads(G.gflat)
+
+    for _ in range(args.warmup):
+        graph_step()
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
 
-    def timed(profile):
+    def timed(profile, step_fn):
         """K steps bracketed by CUDA events on the launching stream, L2 flushed
         (outside the events) before each; with `profile` every launch of the
         library is also bracketed by events, per kernel class."""
@@ -326,7 +350,7 @@ def run_ours(args, rank, world):
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            one_step()
+            step_fn()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         launches = L.launch_count() - n0
@@ -339,11 +363,12 @@ def run_ours(args, rank, world):
     if args.profile_region:
         torch.cuda.profiler.start()
     with ClockSampler(dev) as clk:
-        ms, launches, _ = timed(False)
+        ms, _, _ = timed(False, graph_step)
     if args.profile_region:
         torch.cuda.profiler.stop()
     # per-kernel durations: a second timed pass with events around every launch
-    ms_prof, _, prof = timed(True)
+    ms_prof, launches_prof, prof = timed(True, one_step)
+    launches = launches_prof  # the graph replays the same launches as the eager step
     ms = dp.max_over_ranks(ms, device="cuda")
     ms_step = ms / args.steps
     value = world * T / (ms_step / 1e3)
@@ -354,8 +379,6 @@ def run_ours(args, rank, world):
     # upload and step i-1's download overlap step i's compute.
     Xh = G.X.cpu().pin_memory()
     dOh = G.dOut.cpu().pin_memory()
-    if len(G.io) < 2:
-        G.io.append(G.make_io(torch.empty_like(G.X), torch.empty_like(G.dOut)))
     outs = [{k: torch.empty_like(io[k], device="cpu").pin_memory() for k in ("out", "dX", "gflat")}
             for io in G.io]
     h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
@@ -388,7 +411,7 @@ def run_ours(args, rank, world):
         stream.wait_event(up[i % 2])
         if i >= 2:
             stream.wait_event(down[i % 2])  # step i-2's outputs are read back
-        G.step(stream, io)
+        graphs[i % 2].replay()
         dp.allreduce_grads(io["gflat"])
         done[i % 2].record(stream)
         with torch.cuda.stream(d2h_s):
