@@ -65,6 +65,10 @@ struct alignas(64) TcParams {
   int proj_r;
   float* proj_part;
   long long proj_rows;
+  // SwiGLU-backward epilogue through shared memory (two-CTA tiles): maps of
+  // g, u (loads), dG, dU (stores), 32 x 32 boxes with 64-byte swizzle, and of
+  // the projection matrices (32-channel x r boxes, unswizzled)
+  CUtensorMap emap[6];
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -617,6 +621,119 @@ constexpr int B2_BYTES = (BN / 2) * BK * 2;           // 16 KB (this CTA's half)
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;     // 32 KB
 constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + 1024 + 512 + PROJ_SMEM;
 
+// ---- TMA-staged SwiGLU-backward epilogue (two-CTA tiles)
+// Each epilogue warp owns 16 KB: two load buffers of 6 KB (g and u chunks of
+// 32 rows x 32 channels, 2 KB each, then the chunk's 32 x r slices of the two
+// projection matrices, 1 KB each) and one 4 KB store buffer (dG and dU).
+// Six main-loop stages leave too little shared memory for it, so this kernel
+// variant runs five.
+constexpr int STAGES2B = 5;
+constexpr int EPI_WARP_BYTES = 16384;
+constexpr int EPI_LOAD_BYTES = 6144;
+constexpr int EPI_STORE_OFF = 2 * EPI_LOAD_BYTES;
+constexpr int SMEM2B_BYTES = STAGES2B * STAGE2_BYTES + 1024 + 1024 + 4 * EPI_WARP_BYTES;
+static_assert(SMEM2B_BYTES <= 232448, "shared memory of the TMA-epilogue GEMM");
+
+// Byte offset of 16-byte unit j of row `row` in a buffer of 64-byte rows laid
+// out by the TMA 64-byte swizzle (unit index XOR bits 1-2 of the row); the
+// buffer starts on a 1024-byte boundary.
+__device__ __forceinline__ uint32_t sw64(int row, int j) {
+  return uint32_t(row * 64 + ((j ^ ((row >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t a, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+// generic-proxy shared-memory writes made visible to the TMA (async proxy)
+__device__ __forceinline__ void fence_proxy_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store(const CUtensorMap* m, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory reads of every committed bulk store are done
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed bulk store is complete
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Pack 32 fp32 values as bf16 into row `row` of a 64-byte-swizzled buffer.
+__device__ __forceinline__ void stage_row_sw64(uint32_t buf, int row, const float* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+    sts128(buf + sw64(row, j), *reinterpret_cast<const uint4*>(h));
+  }
+}
+// B fragments of a chunk's 32 x R projection slice staged densely (row k =
+// channel c0 + k, R bf16 per row): b[kb][nb][h] holds rows kb*16 + h*8 + 2t,
+// +1 of column nb*8 + g, the m16n8k16 B layout (ldmatrix .trans).
+template <int R>
+__device__ __forceinline__ void proj_bfrag(uint32_t (&b)[2][R / 8][2], uint32_t pbuf, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  if constexpr (R == 16) {
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      uint32_t r[4];
+      ldsm_x4_t(pbuf + uint32_t((kb * 16 + (mi & 1) * 8 + rr) * 32 + (mi >> 1) * 16), r);
+      b[kb][0][0] = r[0];
+      b[kb][0][1] = r[1];
+      b[kb][1][0] = r[2];
+      b[kb][1][1] = r[3];
+    }
+  } else {
+    uint32_t r[4];
+    ldsm_x4_t(pbuf + uint32_t(((mi >> 1) * 16 + (mi & 1) * 8 + rr) * 16), r);
+    b[0][0][0] = r[0];
+    b[0][0][1] = r[1];
+    b[1][0][0] = r[2];
+    b[1][0][1] = r[3];
+  }
+}
+// acc[mb][nb] += rows mb*16.. of the swizzle-staged 32 x 32 bf16 chunk times
+// the B fragments.
+template <int R>
+__device__ __forceinline__ void proj_mma_sw(float (&acc)[2][2][4], uint32_t buf,
+                                            const uint32_t (&b)[2][R / 8][2], int lane) {
+  const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, aj = lane >> 4;
+#pragma unroll
+  for (int mb = 0; mb < 2; ++mb)
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb) {
+      uint32_t a[4];
+      ldsm_x4(buf + sw64(mb * 16 + arow, kb * 2 + aj), a);
+#pragma unroll
+      for (int nb = 0; nb < R / 8; ++nb) mma16816_tc(acc[mb][nb], a, b[kb][nb][0], b[kb][nb][1]);
+    }
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -672,25 +789,184 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
 }
 }  // namespace
 
+__device__ __forceinline__ void tma_load_s(uint32_t dst, const CUtensorMap* m, uint64_t* bar,
+                                           int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// SwiGLU-backward epilogue of one epilogue warp (rows q*32 .. q*32 + 31 of
+// this CTA's 128-row half), staged through shared memory:
+//   * the g and u chunks (32 rows x 32 channels) and the chunk's slices of the
+//     two projection matrices arrive by TMA into one of two load buffers;
+//     chunks 0 and 1 of a tile are requested before the tile's accumulator is
+//     ready, chunk c + 2 once chunk c has been read;
+//   * dG and dU are packed to bf16 into the store buffer (64-byte swizzle,
+//     conflict-free per row), written out by two TMA stores when all 32 rows
+//     are valid (per-row stores otherwise), and read back by ldmatrix as the
+//     A operand of the rank-R projections (mma.sync, fp32 partials).
+template <int R>
+__device__ __forceinline__ void tc2_bwd_epilogue(const TcParams& p, uint8_t* wbuf, uint64_t* eb,
+                                                 uint64_t* tfull, uint64_t* tempty,
+                                                 volatile int* abort, uint32_t tbase,
+                                                 uint32_t rank, int q, int lane, int cluster_id,
+                                                 int n_clusters, int n_mpairs, int total) {
+  constexpr int RB = R > 0 ? R / 8 : 1;
+  const int r = q * 32 + lane;
+  const uint32_t sbuf = su32(wbuf);
+  const uint32_t obuf = sbuf + EPI_STORE_OFF;
+  const uint32_t tempty_leader0 = map_to_rank(su32(&tempty[0]), 0);
+  const uint32_t tempty_leader1 = map_to_rank(su32(&tempty[1]), 0);
+  const uint32_t ebytes = 2u * 2048u + 2u * 32u * uint32_t(R) * 2u;
+  uint32_t issued = 0, used = 0;
+  bool ok = true;
+  int it = 0;
+  for (int t = cluster_id; t < total && ok; t += n_clusters, ++it) {
+    const int acc = it & 1;
+    const uint32_t aph = uint32_t(it >> 1) & 1u;
+    const int mp = t % n_mpairs, nt = t / n_mpairs;
+    const int mt = 2 * mp + int(rank);
+    int out_row = 0, nvalid = 0;
+    if (mt < p.n_mtiles) {
+      const int4 tl = p.tiles[mt];
+      out_row = p.out_compact ? tl.y : tl.x;
+      nvalid = tl.z;
+    }
+    const int n0 = nt * BN;
+    const int nch = min(8, (p.N - n0 + 31) / 32);  // n0 < N for every N tile
+    const int row0 = out_row + q * 32;
+    const bool valid = r < nvalid;
+    const bool full_warp = q * 32 + 32 <= nvalid;
+    const int64_t orow = int64_t(out_row) + r;
+    auto issue = [&](int c) {  // warp-uniform; lane 0 requests chunk c
+      if (lane == 0) {
+        const uint32_t b = sbuf + (issued & 1u) * EPI_LOAD_BYTES;
+        uint64_t* bar = eb + (issued & 1u);
+        const int c0 = n0 + 32 * c;
+        mbar_expect_tx(bar, ebytes);
+        tma_load_s(b, &p.emap[0], bar, c0, row0);
+        tma_load_s(b + 2048, &p.emap[1], bar, c0, row0);
+        if (R > 0) {
+          tma_load_s(b + 4096, &p.emap[4], bar, 0, c0);
+          tma_load_s(b + 5120, &p.emap[5], bar, 0, c0);
+        }
+      }
+      ++issued;
+    };
+    issue(0);
+    if (nch > 1) issue(1);
+    if (valid) {  // the rest of the tile's g and u rows on their way to L2
+      prefetch_row256(static_cast<const __nv_bfloat16*>(p.in0) + orow * p.ldi, n0, p.N);
+      prefetch_row256(static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi, n0, p.N);
+    }
+    if (!mbar_wait(&tfull[acc], aph, abort)) { ok = false; break; }
+    fence_after();
+    const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
+    __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
+    __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
+    float pg[2][2][4] = {}, pu[2][2][4] = {};  // rank projections of dG and dU
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      float v[32], w[32];
+      tmem_ld32(tl + c * 32, v);  // dh
+      const uint32_t b = sbuf + (used & 1u) * EPI_LOAD_BYTES;
+      if (!mbar_wait(eb + (used & 1u), (used >> 1) & 1u, abort)) { ok = false; break; }
+      ++used;
+      uint4 gv[4], uv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        gv[j] = lds128(b + sw64(lane, j));
+        uv[j] = lds128(b + 2048 + sw64(lane, j));
+      }
+      uint32_t bg[2][RB][2], bu[2][RB][2];
+      if constexpr (R > 0) {
+        proj_bfrag<R>(bg, b + 4096, lane);
+        proj_bfrag<R>(bu, b + 5120, lane);
+      }
+#pragma unroll
+      for (int j2 = 0; j2 < 16; ++j2) {
+        const float2 g2 = unpack2(gv, j2), u2 = unpack2(uv, j2);
+        const float ga[2] = {g2.x, g2.y}, ua[2] = {u2.x, u2.y};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = 2 * j2 + e;
+          const float sg = sigmoid_f(ga[e]);
+          const float dh = v[j];
+          v[j] = dh * ua[e] * sg * (1.0f + ga[e] * (1.0f - sg));  // dG
+          w[j] = dh * ga[e] * sg;                                  // dU
+        }
+      }
+      __syncwarp();  // every lane has read the load buffer: it may be refilled
+      if (c + 2 < nch) issue(c + 2);
+      if (lane == 0) bulk_wait_read();  // the previous chunk's stores have read the store buffer
+      __syncwarp();
+      stage_row_sw64(obuf, lane, v);
+      stage_row_sw64(obuf + 2048, lane, w);
+      fence_proxy_smem();
+      __syncwarp();
+      const int c0 = n0 + c * 32;
+      if (full_warp) {
+        if (lane == 0) {
+          tma_store(&p.emap[2], obuf, c0, row0);
+          tma_store(&p.emap[3], obuf + 2048, c0, row0);
+          bulk_commit();
+        }
+      } else if (valid) {
+        store_row32(dg, c0, p.N, v);
+        store_row32(du, c0, p.N, w);
+      }
+      if constexpr (R > 0) {
+        proj_mma_sw<R>(pg, obuf, bg, lane);
+        proj_mma_sw<R>(pu, obuf + 2048, bu, lane);
+      }
+    }
+    if (!ok) break;
+    if constexpr (R > 0) {
+      proj_store<R>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 2 * R, 0, pg, lane);
+      proj_store<R>(p.proj_part, out_row, nvalid, q * 32, nt, p.n_ntiles, 2 * R, R, pu, lane);
+    }
+    fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+  }
+  // before the CTA may exit: chunk loads still in flight land (bounded), and
+  // the bulk stores complete
+  for (uint32_t k = used; k < issued; ++k) {
+    const long long t0 = clock64();
+    while (!mbar_try(eb + (k & 1u), (k >> 1) & 1u) && clock64() - t0 < WAIT_BUDGET) {
+    }
+  }
+  if (lane == 0) bulk_wait_all();
+  __syncwarp();
+}
+
+template <int kStages, bool kBwdTma>
 __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw2[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES2 * STAGE2_BYTES);
-  uint64_t* empty = full + STAGES2;
-  uint64_t* tfull = empty + STAGES2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * STAGE2_BYTES);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // epilogue chunk-load barriers, two per epilogue warp (TMA-epilogue variant)
+  uint64_t* ebar = reinterpret_cast<uint64_t*>(smem + kStages * STAGE2_BYTES + 256);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    if (kBwdTma)
+      for (int e = 0; e < 8; ++e) mbar_init(&ebar[e], 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 8);  // four epilogue warps in each CTA of the pair
@@ -772,7 +1048,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
                             n0 + 64 * (2 * int(rank) + al), r4[0], r4[1], r4[2], r4[3]);
           }
           ++issued;
-          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
     }
@@ -780,8 +1056,8 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
       // let the copies already armed land before the CTA can exit
       int st2 = stage;
       uint32_t ph2 = phase;
-      for (int i = 0; i < STAGES2 && i < issued; ++i) {
-        if (--st2 < 0) { st2 = STAGES2 - 1; ph2 ^= 1u; }
+      for (int i = 0; i < kStages && i < issued; ++i) {
+        if (--st2 < 0) { st2 = kStages - 1; ph2 ^= 1u; }
         const long long t0 = clock64();
         while (!mbar_try(&full[st2], ph2) && clock64() - t0 < WAIT_BUDGET) {
         }
@@ -817,19 +1093,31 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
             }
             first = false;
             mma_commit_2sm(&empty[stage]);
-            if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+            if (++stage == kStages) { stage = 0; phase ^= 1u; }
           }
         }
         mma_commit_2sm(&tfull[acc]);
       }
     }
     __syncwarp();
+  } else if (kBwdTma && warp >= 4) {
+    uint8_t* wb = smem + kStages * STAGE2_BYTES + 1024 + (warp - 4) * EPI_WARP_BYTES;
+    uint64_t* eb = ebar + 2 * (warp - 4);
+    if (p.proj_r == 16)
+      tc2_bwd_epilogue<16>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                           cluster_id, n_clusters, n_mpairs, total);
+    else if (p.proj_r == 8)
+      tc2_bwd_epilogue<8>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                          cluster_id, n_clusters, n_mpairs, total);
+    else
+      tc2_bwd_epilogue<0>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                          cluster_id, n_clusters, n_mpairs, total);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp - 4;
     const int r = q * 32 + lane;  // row within this CTA's 128-row half == TMEM lane
     __nv_bfloat16* pbuf0 = reinterpret_cast<__nv_bfloat16*>(
-                               smem + STAGES2 * STAGE2_BYTES + 512) + q * 2 * PROJ_BUF;
+                               smem + kStages * STAGE2_BYTES + 512) + q * 2 * PROJ_BUF;
     __nv_bfloat16* pbuf1 = pbuf0 + PROJ_BUF;
     const uint32_t tempty_leader0 = map_to_rank(su32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = map_to_rank(su32(&tempty[1]), 0);
@@ -995,7 +1283,8 @@ slora_status get_encode() {
   return SLORA_OK;
 }
 
-slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y) {
+slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y,
+                    CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (!t.ptr) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: null operand");
   if ((reinterpret_cast<uintptr_t>(t.ptr) & 15) || (t.ld % 8) || t.rows <= 0 || t.cols <= 0)
     SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: operand not 16-byte aligned (ld=%lld)",
@@ -1005,8 +1294,8 @@ slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y) {
   cuuint32_t box[2] = {cuuint32_t(box_x), cuuint32_t(box_y)};
   cuuint32_t es[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(t.ptr), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%lld cols=%lld ld=%lld",
@@ -1107,9 +1396,39 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   if (!g_attr_set) {
     SLORA_CUDA(cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     SMEM_BYTES));
-    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    SMEM2_BYTES));
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES));
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2B, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2B_BYTES));
     g_attr_set = true;
+  }
+  // SwiGLU backward through shared memory: operands addressable by TMA
+  auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
+  const bool bwd_tma = g_tc_mode == 2 && g.epi == EPI_SWIGLU_BWD && !g.paired && g.io_rows > 0 &&
+                       al16(g.in0) && al16(g.in1) && al16(g.out0) && al16(g.out1);
+  if (bwd_tma) {
+    TcMat e;
+    e.rows = g.io_rows;
+    e.cols = g.N;
+    e.ld = g.ldi;
+    e.ptr = g.in0;
+    SLORA_TRY(encode(&p.emap[0], e, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+    e.ptr = g.in1;
+    SLORA_TRY(encode(&p.emap[1], e, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+    e.ld = g.ldo;
+    e.ptr = g.out0;
+    SLORA_TRY(encode(&p.emap[2], e, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+    e.ptr = g.out1;
+    SLORA_TRY(encode(&p.emap[3], e, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
+    if (p.proj_r) {
+      e.rows = g.N;
+      e.cols = p.proj_r;
+      e.ld = g.ldproj;
+      e.ptr = g.proj0;
+      SLORA_TRY(encode(&p.emap[4], e, p.proj_r, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+      e.ptr = g.proj1;
+      SLORA_TRY(encode(&p.emap[5], e, p.proj_r, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
   }
   if (g_tc_mode == 2) {
     const int64_t ctiles = int64_t((p.n_mtiles + 1) / 2) * p.n_ntiles;
@@ -1120,7 +1439,7 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(2 * nclus), 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
-    cfg.dynamicSmemBytes = SMEM2_BYTES;
+    cfg.dynamicSmemBytes = bwd_tma ? SMEM2B_BYTES : SMEM2_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1129,7 +1448,10 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel, p));
+    if (bwd_tma)
+      SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2B, true>, p));
+    else
+      SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2, false>, p));
     return SLORA_OK;
   }
   const int64_t tiles = int64_t(p.n_mtiles) * p.n_ntiles;

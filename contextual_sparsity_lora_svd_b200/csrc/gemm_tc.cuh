@@ -72,6 +72,11 @@ struct TcGemm {
   int proj_r = 0;
   float* proj_part = nullptr;
   int64_t proj_rows = 0;
+  // SWIGLU_BWD: rows of in0, in1, out0 and out1 (all [io_rows x N], leading
+  // dimensions ldi / ldo).  When set (two-CTA tile mode, 16-byte aligned
+  // pointers) g and u are loaded and dG and dU stored by TMA through shared
+  // memory, and the projection slices too; 0 keeps per-row loads and stores.
+  int64_t io_rows = 0;
 };
 
 // N tiles of a GEMM (the count the projection partials are laid out over).

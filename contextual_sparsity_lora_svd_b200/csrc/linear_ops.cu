@@ -236,8 +236,9 @@ struct TcBuilder {
     g.out0 = o0; g.out1 = o1; g.out2 = o2; g.ldo = ldo;
     return *this;
   }
-  TcBuilder& in(const void* i0, const void* i1, int64_t ldi) {
-    g.in0 = i0; g.in1 = i1; g.ldi = ldi;
+  // SwiGLU-backward inputs g, u and the row count of g, u, dG and dU
+  TcBuilder& in(const void* i0, const void* i1, int64_t ldi, int64_t io_rows) {
+    g.in0 = i0; g.in1 = i1; g.ldi = ldi; g.io_rows = io_rows;
     return *this;
   }
   // rank projection of the epilogue values (h, or dG and dU), see TcGemm
@@ -491,7 +492,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     b.seg(mat(dOut, T, d, d), mat(WdS, kk, d, d), B_K, d)
         .seg(mat(dOBb, T, r, lr), mat(AdtS, kk, r, lr), B_K, r)
         .out(dGC, dUC, nullptr, ldk)
-        .in(gC, uC, ldk);
+        .in(gC, uC, ldk, TC);
     if (proj) b.proj(BgS, BuS, lr, int(lr), projC, TC);
     SLORA_TRY(gemm_tc(b.g, st));
   }
@@ -500,7 +501,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     b.seg(mat(dOut, T, d, d), mat(L.Wd_t, Fd, d, d), B_K, d)
         .seg(mat(dOBb, T, r, lr), mat(Adt, Fd, r, lr), B_K, r)
         .out(dGO, dUO, nullptr, Fd)
-        .in(gO, uO, Fd);
+        .in(gO, uO, Fd, TO);
     if (proj)
       b.proj(bpad ? BgP : L.Bg, bpad ? BuP : L.Bu, bpad ? lr : r, int(lr), projO, TO);
     SLORA_TRY(gemm_tc(b.g, st));
