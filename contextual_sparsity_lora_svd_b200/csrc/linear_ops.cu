@@ -317,6 +317,44 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   void* hO = bf(TO, Fd);
   void* dGO = bf(TO, Fd);
   void* dUO = bf(TO, Fd);
+  // context-row parts of dAd, dBg, dBu on the channel subset (added into the
+  // full-channel results after the batched contraction)
+  const bool ctxg = TC > 0 && kk > 0;
+  float* SAd = ar.take<float>(size_t(std::max<int64_t>(kk * r, 1)));
+  float* SBg = ar.take<float>(size_t(std::max<int64_t>(kk * r, 1)));
+  float* SBu = ar.take<float>(size_t(std::max<int64_t>(kk * r, 1)));
+  auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
+    SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
+  };
+  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
+               int64_t map_limit = INT64_MAX) {
+    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
+    rr.map_limit = map_limit; return rr;
+  };
+  // The rank-r gradients that sum over tokens, as one batched coldot:
+  // dBd = s dOut^T hA, dAd = s dOB^T h, dBg = s dG^T XA_g, dBu = s dU^T XA_u,
+  // each output-row part over every channel and each context-row part on S.
+  auto grad_jobs = [&](SkColJob* cj, void* rHA, void* rDO, void* rDC, void* rXgO, void* rXgC,
+                       void* rXuO, void* rXuC) {
+    auto cjob = [&](const void* Y, int64_t ld, int64_t M, int64_t K, const SkR& Rr, void* rsp_,
+                    float* o, int64_t ldo, int trans) {
+      SkColJob j;
+      j.Y = Yv(Y, ld); j.M = M; j.K = K; j.R = Rr; j.c = r; j.rs = rsp_;
+      j.o.out = o; j.o.ldo = ldo; j.o.trans = trans; j.o.scale = s;
+      return j;
+    };
+    int n = 0;
+    cj[n++] = cjob(dOut, d, T, d, Rv(hA, kF32, r, 1), rHA, G.dBd, r, 0);
+    cj[n++] = cjob(hO, Fd, TO, Fd, Rv(dOB, kF32, r, 1, out_rows), rDO, G.dAd, Fd, 1);
+    cj[n++] = cjob(dGO, Fd, TO, Fd, Rv(XA, kF32, 2 * r, 1, out_rows), rXgO, G.dBg, r, 0);
+    cj[n++] = cjob(dUO, Fd, TO, Fd, Rv(XA + r, kF32, 2 * r, 1, out_rows), rXuO, G.dBu, r, 0);
+    if (ctxg) {
+      cj[n++] = cjob(hC, ldk, TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), rDC, SAd, kk, 1);
+      cj[n++] = cjob(dGC, ldk, TC, kk, Rv(XA, kF32, 2 * r, 1, ctx_rows), rXgC, SBg, r, 0);
+      cj[n++] = cjob(dUC, ldk, TC, kk, Rv(XA + r, kF32, 2 * r, 1, ctx_rows), rXuC, SBu, r, 0);
+    }
+    return n;
+  };
   // partial sums of the skinny contractions (reused sequentially)
   const int rs = L.r_svd;
   const bool fused = !idx_force && 2 * r + 2 * rs <= 64;  // one pass over X for XA and P
@@ -327,8 +365,12 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         npart = std::max(npart, rowdot_part_floats(M, K, c));
         npart = std::max(npart, coldot_part_floats(M, K, c));
       }
+  SkColJob gj[7];
+  const int ngj = grad_jobs(gj, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  npart = std::max(npart, coldot_batch_part_floats(gj, ngj));
   float* part = ar.take<float>(size_t(npart));
-  const int64_t ncnt = skinny_counter_count(std::max({T, d, Fd}), std::max({T, d, Fd}));
+  const int64_t ncnt = std::max(skinny_counter_count(std::max({T, d, Fd}), std::max({T, d, Fd})),
+                                coldot_batch_counter_count(gj, ngj));
   unsigned* rsp = ar.take<unsigned>(size_t(ncnt));
   SkWork sw;
   sw.part = part;
@@ -369,14 +411,6 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
-  auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
-    SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
-  };
-  auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
-               int64_t map_limit = INT64_MAX) {
-    SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
-    rr.map_limit = map_limit; return rr;
-  };
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
   SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
@@ -469,7 +503,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   }
 
   // ---- backward
-  {  // dOB = dOut Bd: fp32 and s*dOB bf16; dBd = s dOut^T hA (same stream of dOut)
+  {  // dOB = dOut Bd: fp32 and s*dOB bf16
     SkRowOut o;
     o.out1 = dOB; o.ld1 = r; o.out2 = dOBb; o.ld2 = lr; o.s2 = s;
     SLORA_TRY(rowdot(Yv(dOut, d), T, d, Rv(L.Bd, kBF16, r, 1), r, o, prepared(rsBd), st));
@@ -483,9 +517,6 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         job(Rv(XA + r, kF32, 2 * r, 1, out_rows), r, TO, rsXA[1][0]),
         job(Rv(XA + r, kF32, 2 * r, 1, ctx_rows), r, TC, rsXA[1][1])};
     SLORA_TRY(prep_r_batch(jobs, 7, st));
-    SkColOut c;
-    c.out = G.dBd; c.ldo = r; c.scale = s;
-    SLORA_TRY(coldot(Yv(dOut, d), T, d, Rv(hA, kF32, r, 1), r, c, prepared(rsHA), st));
   }
   {  // dh_S = dOut_C Wd[:,S] + s dOB_C Ad[:,S]^T, SwiGLU backward in the epilogue
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 0, EPI_SWIGLU_BWD);
@@ -506,16 +537,6 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       b.proj(bpad ? BgP : L.Bg, bpad ? BuP : L.Bu, bpad ? lr : r, int(lr), projO, TO);
     SLORA_TRY(gemm_tc(b.g, st));
   }
-  {  // dAd = s dOB^T h: output rows over every channel, then += context rows on S
-    SkColOut co;
-    co.out = G.dAd; co.ldo = Fd; co.trans = 1; co.scale = s;
-    SLORA_TRY(
-        coldot(Yv(hO, Fd), TO, Fd, Rv(dOB, kF32, r, 1, out_rows), r, co, prepared(rsDobO), st));
-    SkColOut cc = co;
-    cc.kmap = idx; cc.kmap_limit = Fd; cc.accumulate = 1;
-    SLORA_TRY(
-        coldot(Yv(hC, ldk), TC, kk, Rv(dOB, kF32, r, 1, ctx_rows), r, cc, prepared(rsDobC), st));
-  }
   if (proj) {  // dGB = [dG Bg | dU Bu] from the dh GEMMs' epilogue partials
     SkRowOut oc;
     oc.out1 = dGB; oc.ld1 = 2 * r; oc.map1 = ctx_rows; oc.out2 = dGBbC; oc.ld2 = lr2; oc.s2 = s;
@@ -524,27 +545,29 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     SLORA_TRY(reduce_row_partials(projC, int(ntBc), TC, oc, projO, int(ntBo), TO, oo,
                                   int(2 * lr), int(lr), r, st));
   }
-  for (int p = 0; p < 2; ++p) {  // dGB = [dG Bg | dU Bu] (when not fused); dB = s dG^T XA
+  for (int p = 0; p < 2 && !proj; ++p) {  // dGB = [dG Bg | dU Bu] (when not fused)
     const void* Bm = p ? L.Bu : L.Bg;
-    float* dBm = p ? G.dBu : G.dBg;
     SkRowOut oo;
     oo.out1 = dGB; oo.ld1 = 2 * r; oo.off1 = p * r; oo.map1 = out_rows;
     oo.out2 = dGBbO; oo.ld2 = lr2; oo.off2 = p * r; oo.s2 = s;
-    if (!proj)
-      SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, sw, st));
-    SkColOut bo;
-    bo.out = dBm; bo.ldo = r; bo.scale = s;
-    SLORA_TRY(coldot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(XA + p * r, kF32, 2 * r, 1, out_rows), r,
-                     bo, prepared(rsXA[p][0]), st));
+    SLORA_TRY(rowdot(Yv(p ? dUO : dGO, Fd), TO, Fd, Rv(Bm, kBF16, r, 1), r, oo, sw, st));
     SkRowOut oc = oo;
     oc.map1 = ctx_rows; oc.out2 = dGBbC;
-    if (!proj)
-      SLORA_TRY(
-          rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx, Fd), r, oc, sw, st));
-    SkColOut bc = bo;
-    bc.kmap = idx; bc.kmap_limit = Fd; bc.accumulate = 1;
-    SLORA_TRY(coldot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(XA + p * r, kF32, 2 * r, 1, ctx_rows), r,
-                     bc, prepared(rsXA[p][1]), st));
+    SLORA_TRY(
+        rowdot(Yv(p ? dUC : dGC, ldk), TC, kk, Rv(Bm, kBF16, r, 1, idx, Fd), r, oc, sw, st));
+  }
+  {  // dBd, dAd, dBg, dBu in one launch; then the context rows' parts on S
+    SkColJob cj[7];
+    const int ncj = grad_jobs(cj, rsHA, rsDobO, rsDobC, rsXA[0][0], rsXA[0][1], rsXA[1][0],
+                              rsXA[1][1]);
+    SLORA_TRY(coldot_batch(cj, ncj, part, rsp, st));
+    if (ctxg) {
+      ScatterAddJob sj[3];
+      sj[0].dst = G.dAd; sj[0].ld_dst = Fd; sj[0].src = SAd; sj[0].ld_src = kk; sj[0].trans = 1;
+      sj[1].dst = G.dBg; sj[1].ld_dst = r; sj[1].src = SBg; sj[1].ld_src = r;
+      sj[2].dst = G.dBu; sj[2].ld_dst = r; sj[2].src = SBu; sj[2].ld_src = r;
+      SLORA_TRY(scatter_add_cols(sj, 3, idx, kk, r, Fd, st));
+    }
   }
   {  // dX, context rows: dG_S Wg[S] + dU_S Wu[S] + s [dG_S Bg[S] | dU_S Bu[S]] [Ag; Au]
     TcBuilder b(ctiles, nct, 1, 0, TC, d, 0, EPI_STORE);

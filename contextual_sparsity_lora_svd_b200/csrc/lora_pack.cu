@@ -108,6 +108,25 @@ __global__ void sanitize_kernel(const int32_t* __restrict__ in, int64_t n, int64
   out[i] = index_ok(v, limit) ? v : 0;
 }
 
+// One scatter-add job per blockIdx.y: element (j, q), j < n, q < r, of src
+// (row j: src[j * ld_src + q]; trans: src[q * ld_src + j]) is added to column
+// idx[j] of dst in the same orientation.  With trans, consecutive threads take
+// consecutive j (coalesced source rows); without, consecutive q.
+__global__ void scatter_add_kernel(const ScatterAddJobs J, const int32_t* __restrict__ idx,
+                                   int64_t n, int r, int64_t limit) {
+  const ScatterAddJob& jb = J.job[blockIdx.y];
+  const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= n * r) return;
+  const int64_t j = jb.trans ? e % n : e / r;
+  const int q = int(jb.trans ? e / n : e % r);
+  const int64_t c = idx[j];
+  if (!index_ok(c, limit)) return;
+  if (jb.trans)
+    jb.dst[int64_t(q) * jb.ld_dst + c] += jb.src[int64_t(q) * jb.ld_src + j];
+  else
+    jb.dst[c * jb.ld_dst + q] += jb.src[j * jb.ld_src + q];
+}
+
 __global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t nt) {
   const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= nt) return;
@@ -119,6 +138,19 @@ __global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t 
 unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
 
 }  // namespace
+
+slora_status scatter_add_cols(const ScatterAddJob* jobs, int njobs, const int32_t* idx,
+                              int64_t n, int r, int64_t limit, cudaStream_t st) {
+  if (njobs <= 0 || n <= 0 || r <= 0) return SLORA_OK;
+  if (njobs > ScatterAddJobs::kMax)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "scatter_add_cols: %d jobs (max %d)", njobs, ScatterAddJobs::kMax);
+  ScatterAddJobs J{};
+  for (int k = 0; k < njobs; ++k) J.job[k] = jobs[k];
+  LaunchScope ls(kAux, double(njobs) * double(n) * r * 12.0, st);
+  scatter_add_kernel<<<dim3(blocks(n * r), unsigned(njobs)), 256, 0, st>>>(J, idx, n, r, limit);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
 
 slora_status pack_gate_up_b(const void* Bg, const void* Bu, const int32_t* idx, int64_t N, int r,
                             int64_t n_ntiles, int64_t ldo, void* out, cudaStream_t st,

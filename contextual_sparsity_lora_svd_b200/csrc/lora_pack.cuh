@@ -42,6 +42,22 @@ slora_status sanitize_indices(const int32_t* in, int64_t n, int64_t limit, int32
 // index lies outside their source; SLORA_ERR_INVALID_ARG if it was raised.
 // Synchronous: waits for the device.
 slora_status pack_check_error(bool clear);
+// Adds fp32 results computed on a channel subset into the full-channel ones:
+// dst[idx[j]][q] += src[j][q] (trans: dst[q][idx[j]] += src[q][j]) for j < n,
+// q < r, up to four jobs sharing idx in one launch.  An index outside
+// [0, limit) is skipped and raises the flag that pack_check_error reads.
+struct ScatterAddJob {
+  float* dst = nullptr;
+  const float* src = nullptr;
+  int64_t ld_dst = 0, ld_src = 0;
+  int trans = 0;
+};
+struct ScatterAddJobs {
+  static constexpr int kMax = 4;
+  ScatterAddJob job[kMax];
+};
+slora_status scatter_add_cols(const ScatterAddJob* jobs, int njobs, const int32_t* idx,
+                              int64_t n, int r, int64_t limit, cudaStream_t st);
 // M-tile list {row0, row0, nvalid, 0} covering rows [0, M) in 128-row tiles.
 slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st);
 }  // namespace slora

@@ -594,18 +594,34 @@ __device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t a) {
                : "r"(a));
 }
 
-// Work of one contraction: output blocks of 64 (rows for rowdot, columns for
-// coldot), each with nchunks reduction chunks of 64 cut into ngroups fixed
-// groups of up to G chunks.  A unit is one (block, group); units are handed
-// out by an atomic ticket in group-major order (ticket u -> block u % nblocks,
-// group u / nblocks), so SMs that stream faster take more units.  Each unit's
-// partial lands in its own slot and the last unit of a block to finish sums
-// the block's slots in group order: the result does not depend on which CTA
-// ran which unit.
 struct StreamPlan {
   int nblocks = 0, nchunks = 0, G = 1, ngroups = 1, nunits = 0;
   int ncta = 1;
 };
+
+// One contraction of a TMA launch; a launch takes up to J of them (same
+// column padding and term count) and hands out their units from one ticket,
+// job after job.
+struct TmaJob {
+  CUtensorMap ymap;  // Y [M x K], 64 x 64 boxes
+  CUtensorMap rmap;  // split rank operand, 64 x (NT * CP) boxes
+  StreamPlan p;
+  int c = 0;
+  int unit0 = 0;                 // first ticket of the job
+  int64_t M = 0, K = 0;
+  float* part = nullptr;         // p.nunits partial tiles of 64 x CP floats
+  unsigned* counters = nullptr;  // p.nblocks block tickets, zero on entry, left zero
+  SkRowOut ro;
+  SkColOut co;
+};
+constexpr int kMaxTmaJobs = 7;  // keeps the launch parameters within 4 KB
+template <int J>
+struct TmaJobs {
+  TmaJob job[J];
+  int njobs = 0, nunits = 0, ncta = 1;
+  unsigned* ticket = nullptr;  // unit ticket, zero on entry, left zero
+};
+static_assert(sizeof(TmaJobs<kMaxTmaJobs>) <= 4096, "TMA job table beyond 4 KB of parameters");
 
 // Shared memory of the TMA kernel: S stages of [Y tile 64x64 | split-R tile],
 // each 1024-byte aligned (128-byte swizzle), then the stage barriers and the
@@ -632,15 +648,18 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk16) {
 
 // COL = false: rowdot (output block = 64 rows of Y, reduction over K);
 // COL = true: coldot (output block = 64 columns of Y, reduction over M).
-// counters[0 .. nblocks) are the per-block arrival tickets, counters[nblocks]
-// the unit ticket; all are zero on entry and left zero.
-template <int NF, int NT, bool COL>
-__global__ void __launch_bounds__(NTH) skinny_tma_kernel(
-    const __grid_constant__ CUtensorMap ymap, const __grid_constant__ CUtensorMap rmap,
-    const StreamPlan p, int c, int64_t M, int64_t K, float* __restrict__ part,
-    unsigned* __restrict__ counters, const SkRowOut ro, const SkColOut co) {
+// Work of one job: output blocks of 64 (rows for rowdot, columns for
+// coldot), each with nchunks reduction chunks of 64 cut into ngroups fixed
+// groups of up to G chunks.  A unit is one (block, group); units are handed
+// out by an atomic ticket in job order and, within a job, group-major order
+// (ticket u -> block u % nblocks, group u / nblocks), so SMs that stream
+// faster take more units.  Each unit's partial lands in its own slot and the
+// last unit of a block to finish sums the block's slots in group order: the
+// result does not depend on which CTA ran which unit.
+template <int NF, int NT, bool COL, int J>
+__global__ void __launch_bounds__(NTH) skinny_tma_kernel(const __grid_constant__ TmaJobs<J> jobs) {
   constexpr int CP = NF * 8, S = tma_stages(CP, NT), SB = tma_stage_bytes(CP, NT);
-  constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+  constexpr int kLast = 2, kEnd = 4, kJobShift = 4;
   extern __shared__ unsigned char sk_smem[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(sk_smem) + 1023) & ~uintptr_t(1023));
@@ -648,26 +667,33 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
   int4* info = reinterpret_cast<int4*>(sm + S * SB + 8 * 8);  // {block, chunk, flags, group}
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  unsigned* work = counters + p.nblocks;
+  unsigned* work = jobs.ticket;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // ---- producer state (thread 0): current unit and the next chunk of it
-  int pb = 0, pg = 0, pk = 0, pk1 = 0, issued = 0;
+  // ---- producer state (thread 0): current job and unit, and its next chunk
+  int pj = 0, pb = 0, pg = 0, pk = 0, pk1 = 0, issued = 0;
   bool pdone = false;
   auto next_unit = [&]() {  // false once the tickets are exhausted
     const unsigned u = atomicAdd(work, 1u);
-    if (u >= unsigned(p.nunits)) {
-      if (u == unsigned(p.nunits + p.ncta - 1)) *work = 0u;  // the last ticket resets
+    if (u >= unsigned(jobs.nunits)) {
+      if (u == unsigned(jobs.nunits + jobs.ncta - 1)) *work = 0u;  // the last ticket resets
       return false;
     }
-    pb = int(u % unsigned(p.nblocks));
-    pg = int(u / unsigned(p.nblocks));
-    pk = pg * p.G;
-    pk1 = pk + p.G < p.nchunks ? pk + p.G : p.nchunks;
+    int jb = 0;
+#pragma unroll
+    for (int x = 1; x < J; ++x)
+      if (x < jobs.njobs && u >= unsigned(jobs.job[x].unit0)) jb = x;
+    const StreamPlan& P = jobs.job[jb].p;
+    const unsigned lu = u - unsigned(jobs.job[jb].unit0);
+    pj = jb;
+    pb = int(lu % unsigned(P.nblocks));
+    pg = int(lu / unsigned(P.nblocks));
+    pk = pg * P.G;
+    pk1 = pk + P.G < P.nchunks ? pk + P.G : P.nchunks;
     return true;
   };
   auto issue = [&]() {  // thread 0: the next position of the stream into stage issued % S
@@ -679,15 +705,15 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
       ++issued;
       return false;
     }
-    const int flags = (pk == pg * p.G ? kFirst : 0) | (pk + 1 == pk1 ? kLast : 0);
-    info[st] = make_int4(pb, pk, flags, pg);
+    info[st] = make_int4(pb, pk, (pk + 1 == pk1 ? kLast : 0) | (pj << kJobShift), pg);
     unsigned char* ys = sm + st * SB;
+    const TmaJob& jb = jobs.job[pj];
     mbar_arm(&full[st], uint32_t(SB));
     if (COL)
-      tma2d(ys, &ymap, &full[st], pb * TILE, pk * TILE);
+      tma2d(ys, &jb.ymap, &full[st], pb * TILE, pk * TILE);
     else
-      tma2d(ys, &ymap, &full[st], pk * TILE, pb * TILE);
-    tma2d(ys + kYTile, &rmap, &full[st], pk * TILE, 0);
+      tma2d(ys, &jb.ymap, &full[st], pk * TILE, pb * TILE);
+    tma2d(ys + kYTile, &jb.rmap, &full[st], pk * TILE, 0);
     ++pk;
     ++issued;
     return true;
@@ -736,11 +762,12 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
     if (tid == 0 && !pdone) issue();
     if (!(inf.z & kLast)) continue;  // the unit goes on
 
-    // ---- end of unit (block inf.x, group inf.w)
-    const int b = inf.x;
-    const int64_t nout = COL ? K : M;
+    // ---- end of unit (job inf.z >> kJobShift, block inf.x, group inf.w)
+    const TmaJob& jb = jobs.job[inf.z >> kJobShift];
+    const int b = inf.x, c = jb.c, ngroups = jb.p.ngroups;
+    const int64_t nout = COL ? jb.K : jb.M;
     const int64_t r0 = int64_t(b) * TILE + warp * 16 + g;  // output index of acc rows g / g + 8
-    if (p.ngroups == 1) {  // the unit is the whole block: emit from the accumulators
+    if (ngroups == 1) {  // the unit is the whole block: emit from the accumulators
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
         const int col = f * 8 + 2 * t;
@@ -749,16 +776,16 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
           const int64_t r = r0 + 8 * h;
           if (r >= nout) continue;
           if (COL) {
-            if (col < c) col_emit(co, r, col, acc[f][2 * h]);
-            if (col + 1 < c) col_emit(co, r, col + 1, acc[f][2 * h + 1]);
+            if (col < c) col_emit(jb.co, r, col, acc[f][2 * h]);
+            if (col + 1 < c) col_emit(jb.co, r, col + 1, acc[f][2 * h + 1]);
           } else {
-            if (col < c) row_emit(ro, r, col, acc[f][2 * h]);
-            if (col + 1 < c) row_emit(ro, r, col + 1, acc[f][2 * h + 1]);
+            if (col < c) row_emit(jb.ro, r, col, acc[f][2 * h]);
+            if (col + 1 < c) row_emit(jb.ro, r, col + 1, acc[f][2 * h + 1]);
           }
         }
       }
     } else {
-      float* mine = part + (int64_t(b) * p.ngroups + inf.w) * TILE * CP;
+      float* mine = jb.part + (int64_t(b) * ngroups + inf.w) * TILE * CP;
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
         const int col = f * 8 + 2 * t;
@@ -766,23 +793,23 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(
         *reinterpret_cast<float2*>(mine + lr * CP + col) = make_float2(acc[f][0], acc[f][1]);
         *reinterpret_cast<float2*>(mine + (lr + 8) * CP + col) = make_float2(acc[f][2], acc[f][3]);
       }
-      if (last_arrival(counters + b, unsigned(p.ngroups), tid)) {
+      if (last_arrival(jb.counters + b, unsigned(ngroups), tid)) {
         const int nq4 = (c + 3) / 4;
-        const float* blk = part + int64_t(b) * p.ngroups * TILE * CP;
+        const float* blk = jb.part + int64_t(b) * ngroups * TILE * CP;
         for (int e = tid; e < TILE * nq4; e += NTH) {
           const int lr = e / nq4, q0 = (e % nq4) * 4;
           const int64_t r = int64_t(b) * TILE + lr;
           if (r >= nout) continue;
           const float4 v = sum_splits4(reinterpret_cast<const float4*>(blk + lr * CP + q0),
-                                       int64_t(TILE) * CP / 4, p.ngroups);
+                                       int64_t(TILE) * CP / 4, ngroups);
           const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             if (q0 + u >= c) break;
             if (COL)
-              col_emit(co, r, q0 + u, vv[u]);
+              col_emit(jb.co, r, q0 + u, vv[u]);
             else
-              row_emit(ro, r, q0 + u, vv[u]);
+              row_emit(jb.ro, r, q0 + u, vv[u]);
           }
         }
       }
@@ -887,14 +914,16 @@ bool tma_ok(const SkY& Y, int64_t rows, int64_t cols) {
          rows > 0 && cols > 0 && Y.ld >= cols;
 }
 
-// Units of G chunks: about two units per resident CTA (dynamic balance), at
-// most 32 groups per block (the last unit of a block sums that many tiles).
-StreamPlan stream_plan(int64_t nout, int64_t nred) {
+// Units of G chunks: about `target` units over the job's blocks (two per
+// resident CTA for a job alone: dynamic balance), at most 32 groups per block
+// (the last unit of a block sums that many tiles).
+StreamPlan stream_plan(int64_t nout, int64_t nred,
+                       int64_t target = 2 * int64_t(kSMs) * kTmaCtasPerSm) {
   StreamPlan p;
   p.nblocks = int((nout + TILE - 1) / TILE);
   p.nchunks = int(std::max<int64_t>((nred + TILE - 1) / TILE, 1));
   const int64_t cap = int64_t(kSMs) * kTmaCtasPerSm;
-  int64_t want = (2 * cap + p.nblocks - 1) / std::max(p.nblocks, 1);
+  int64_t want = (std::max<int64_t>(target, 1) + p.nblocks - 1) / std::max(p.nblocks, 1);
   if (want < 1) want = 1;
   if (want > 32) want = 32;
   if (want > p.nchunks) want = p.nchunks;
@@ -906,48 +935,69 @@ StreamPlan stream_plan(int64_t nout, int64_t nred) {
   return p;
 }
 
-#define SLORA_TMA_CASE(NF_, NT_, COL_)                                                       \
-  case NF_ * 8: {                                                                            \
-    auto kfn = skinny_tma_kernel<NF_, NT_, COL_>;                                            \
-    const int sm = tma_smem(NF_ * 8, NT_);                                                   \
-    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);              \
-    kfn<<<p.ncta, NTH, sm, st>>>(ym, rm, p, c, M, K, w.part, w.counters, ro, co);            \
-  } break;
-#define SLORA_TMA_SWITCH(NT_, COL_) \
-  switch (CP) {                     \
-    SLORA_TMA_CASE(2, NT_, COL_)    \
-    SLORA_TMA_CASE(4, NT_, COL_)    \
-    SLORA_TMA_CASE(6, NT_, COL_)    \
-    default:                        \
-    SLORA_TMA_CASE(8, NT_, COL_)    \
+template <int NF, int NT, bool COL, int J>
+slora_status launch_tma_kernel(const TmaJobs<J>& jb, cudaStream_t st) {
+  auto kfn = skinny_tma_kernel<NF, NT, COL, J>;
+  const int sm = tma_smem(NF * 8, NT);
+  SLORA_CUDA(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm));
+  kfn<<<jb.ncta, NTH, sm, st>>>(jb);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+template <bool COL, int J>
+slora_status launch_tma_jobs(const TmaJobs<J>& jb, int CP, int nt, cudaStream_t st) {
+  if (nt == 3) {
+    switch (CP) {
+      case 16: return launch_tma_kernel<2, 3, COL, J>(jb, st);
+      case 32: return launch_tma_kernel<4, 3, COL, J>(jb, st);
+      case 48: return launch_tma_kernel<6, 3, COL, J>(jb, st);
+      default: return launch_tma_kernel<8, 3, COL, J>(jb, st);
+    }
   }
+  switch (CP) {
+    case 16: return launch_tma_kernel<2, 1, COL, J>(jb, st);
+    case 32: return launch_tma_kernel<4, 1, COL, J>(jb, st);
+    case 48: return launch_tma_kernel<6, 1, COL, J>(jb, st);
+    default: return launch_tma_kernel<8, 1, COL, J>(jb, st);
+  }
+}
 
-// The rsplit rows (NT * CP) are one TMA box high; the map's height is the
-// rows that term count uses.
+// Fills job `x` of a launch (its maps, plan, workspace slices).  The rsplit
+// rows (NT * CP) are one TMA box high; the map's height is the rows that term
+// count uses.
+slora_status fill_tma_job(TmaJob& J, bool col, const SkY& Y, int64_t M, int64_t K, int c, int nt,
+                          const void* rsplit, const StreamPlan& p, float* part,
+                          unsigned* counters) {
+  const int CP = padded(c);
+  const int64_t I64 = round64(std::max<int64_t>(col ? M : K, 1));
+  SLORA_TRY(encode_bf16(&J.ymap, Y.ptr, M, K, Y.ld, TILE, TILE));
+  SLORA_TRY(encode_bf16(&J.rmap, rsplit, int64_t(nt) * CP, I64, I64, TILE, nt * CP));
+  J.p = p;
+  J.c = c;
+  J.M = M;
+  J.K = K;
+  J.part = part;
+  J.counters = counters;
+  return SLORA_OK;
+}
+
 slora_status launch_tma(bool col, const SkY& Y, int64_t M, int64_t K, int c, int nt,
                         const SkRowOut& ro, const SkColOut& co, const SkWork& w, int64_t I64,
                         cudaStream_t st) {
-  const int CP = padded(c);
+  (void)I64;
   const StreamPlan p = col ? stream_plan(K, M) : stream_plan(M, K);
-  CUtensorMap ym, rm;
-  SLORA_TRY(encode_bf16(&ym, Y.ptr, M, K, Y.ld, TILE, TILE));
-  SLORA_TRY(encode_bf16(&rm, w.rsplit, int64_t(nt) * CP, I64, I64, TILE, nt * CP));
+  TmaJobs<1> jb;
+  SLORA_TRY(fill_tma_job(jb.job[0], col, Y, M, K, c, nt, w.rsplit, p, w.part, w.counters));
+  jb.job[0].ro = ro;
+  jb.job[0].co = co;
+  jb.job[0].unit0 = 0;
+  jb.njobs = 1;
+  jb.nunits = p.nunits;
+  jb.ncta = p.ncta;
+  jb.ticket = w.counters + p.nblocks;
   LaunchScope ls(kSkinny, double(M) * K * 2, st);
-  if (col) {
-    if (nt == 3) {
-      SLORA_TMA_SWITCH(3, true)
-    } else {
-      SLORA_TMA_SWITCH(1, true)
-    }
-  } else {
-    if (nt == 3) {
-      SLORA_TMA_SWITCH(3, false)
-    } else {
-      SLORA_TMA_SWITCH(1, false)
-    }
-  }
-  SLORA_CHECK_LAUNCH();
-  return SLORA_OK;
+  return col ? launch_tma_jobs<true, 1>(jb, padded(c), nt, st)
+             : launch_tma_jobs<false, 1>(jb, padded(c), nt, st);
 }
 
 int64_t tma_part_floats(int64_t nout, int64_t nred, int c) {
@@ -968,6 +1018,105 @@ int64_t coldot_part_floats(int64_t M, int64_t K, int c) {
   const Geo a = geometry(K, M, c, false), b = geometry(K, M, c, true);
   return std::max(int64_t(std::max(a.nsplit, b.nsplit)) * std::max<int64_t>(K, 1) * padded(c),
                   tma_part_floats(K, M, c));
+}
+
+namespace {
+int job_terms(const SkColJob& j) { return fp32_terms(j.R) ? 3 : 1; }
+// The shapes allow one launch (the workspace is sized on this alone).
+bool batch_shape_ok(const SkColJob* jobs, int n) {
+  if (n < 1 || n > kMaxTmaJobs) return false;
+  const int CP = padded(jobs[0].c), nt = job_terms(jobs[0]);
+  for (int k = 0; k < n; ++k) {
+    const SkColJob& j = jobs[k];
+    if (j.c <= 0 || j.c > 64 || padded(j.c) != CP || job_terms(j) != nt || j.M <= 0 ||
+        j.K <= 0)
+      return false;
+  }
+  return true;
+}
+// ... and the operands too.
+bool batch_tma_ok(const SkColJob* jobs, int n) {
+  if (!batch_shape_ok(jobs, n)) return false;
+  for (int k = 0; k < n; ++k)
+    if (!jobs[k].rs || !tma_ok(jobs[k].Y, jobs[k].M, jobs[k].K)) return false;
+  return true;
+}
+// Each job's share of the two units per resident CTA, by its size.
+void batch_plans(const SkColJob* jobs, int n, StreamPlan* plans) {
+  double total = 0.0;
+  for (int k = 0; k < n; ++k) total += double(jobs[k].M) * double(jobs[k].K);
+  const double units = 2.0 * kSMs * kTmaCtasPerSm;
+  for (int k = 0; k < n; ++k) {
+    const double share = total > 0 ? double(jobs[k].M) * double(jobs[k].K) / total : 1.0;
+    plans[k] = stream_plan(jobs[k].K, jobs[k].M, std::max<int64_t>(1, llround(units * share)));
+  }
+}
+}  // namespace
+
+int64_t coldot_batch_part_floats(const SkColJob* jobs, int n) {
+  int64_t most = 1;
+  for (int k = 0; k < n; ++k)
+    most = std::max(most, coldot_part_floats(jobs[k].M, jobs[k].K, jobs[k].c));
+  if (!batch_shape_ok(jobs, n)) return most;
+  StreamPlan plans[kMaxTmaJobs];
+  batch_plans(jobs, n, plans);
+  int64_t sum = 0;
+  for (int k = 0; k < n; ++k) sum += int64_t(plans[k].nunits) * TILE * padded(jobs[k].c);
+  return std::max(most, sum);
+}
+
+int64_t coldot_batch_counter_count(const SkColJob* jobs, int n) {
+  int64_t most = 1;
+  for (int k = 0; k < n; ++k)
+    most = std::max(most, skinny_counter_count(jobs[k].M, jobs[k].K));
+  if (!batch_shape_ok(jobs, n)) return most;
+  StreamPlan plans[kMaxTmaJobs];
+  batch_plans(jobs, n, plans);
+  int64_t sum = 1;
+  for (int k = 0; k < n; ++k) sum += plans[k].nblocks;
+  return std::max(most, sum);
+}
+
+slora_status coldot_batch(const SkColJob* jobs, int n, float* part, unsigned* counters,
+                          cudaStream_t st) {
+  if (n <= 0) return SLORA_OK;
+  if (!batch_tma_ok(jobs, n)) {
+    for (int k = 0; k < n; ++k) {
+      SkWork w;
+      w.part = part;
+      w.counters = counters;
+      w.rsplit = jobs[k].rs;
+      w.prepared = jobs[k].rs != nullptr;
+      if (!w.prepared)
+        SLORA_FAIL(SLORA_ERR_INVALID_ARG, "coldot_batch: job %d has no split operand", k);
+      SLORA_TRY(coldot(jobs[k].Y, jobs[k].M, jobs[k].K, jobs[k].R, jobs[k].c, jobs[k].o, w, st));
+    }
+    return SLORA_OK;
+  }
+  StreamPlan plans[kMaxTmaJobs];
+  batch_plans(jobs, n, plans);
+  TmaJobs<kMaxTmaJobs> jb;
+  const int CP = padded(jobs[0].c), nt = job_terms(jobs[0]);
+  int unit = 0;
+  float* pp = part;
+  unsigned* cc = counters;
+  double bytes = 0.0;
+  for (int k = 0; k < n; ++k) {
+    const SkColJob& j = jobs[k];
+    SLORA_TRY(fill_tma_job(jb.job[k], true, j.Y, j.M, j.K, j.c, nt, j.rs, plans[k], pp, cc));
+    jb.job[k].co = j.o;
+    jb.job[k].unit0 = unit;
+    unit += plans[k].nunits;
+    pp += int64_t(plans[k].nunits) * TILE * CP;
+    cc += plans[k].nblocks;
+    bytes += double(j.M) * double(j.K) * 2.0;
+  }
+  jb.njobs = n;
+  jb.nunits = unit;
+  jb.ncta = int(std::min<int64_t>(unit, int64_t(kSMs) * kTmaCtasPerSm));
+  jb.ticket = cc;
+  LaunchScope ls(kSkinny, bytes, st);
+  return launch_tma_jobs<true, kMaxTmaJobs>(jb, CP, nt, st);
 }
 
 slora_status reduce_row_partials(const float* part0, int nparts0, int64_t M0, const SkRowOut& o0,

@@ -106,6 +106,24 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkRowOut& o, const SkWork& w, cudaStream_t st);
 slora_status coldot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c,
                     const SkColOut& o, const SkWork& w, cudaStream_t st);
+// One of several independent coldots (distinct outputs) run by coldot_batch.
+struct SkColJob {
+  SkY Y;              // no row map
+  int64_t M = 0, K = 0;
+  SkR R;              // its dtype fixes the term count; read only by the fallback
+  int c = 0;
+  void* rs = nullptr;  // R split by prep_r_batch
+  SkColOut o;
+};
+// Workspace of coldot_batch: part floats and counters (zero on entry, left zero).
+int64_t coldot_batch_part_floats(const SkColJob* jobs, int n);
+int64_t coldot_batch_counter_count(const SkColJob* jobs, int n);
+// Up to 7 coldots in one TMA launch whose units come from one ticket (each job
+// cut into units in proportion to its size), when every Y is a plain matrix
+// with 16-byte aligned rows, every job is non-empty and all share the column
+// padding and term count; otherwise one coldot per job, in order.
+slora_status coldot_batch(const SkColJob* jobs, int n, float* part, unsigned* counters,
+                          cudaStream_t st);
 // Rows of a rank projection computed in GEMM epilogues (TcGemm::proj_*), two
 // jobs per launch (typically the context-row and the output-row GEMM):
 // out_k(m, g * r + q) = sum over t < nparts_k of part_k[(m * nparts_k + t) * pc + g * lr + q]
