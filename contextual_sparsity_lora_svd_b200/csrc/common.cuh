@@ -90,6 +90,15 @@ slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles = nullptr,
                             int4* out_tiles = nullptr, unsigned* zero = nullptr,
                             int64_t nzero = 0);
+// A library-owned side stream of the current device (non-blocking, created on
+// first use, kept until exit) with a fork and a join event, for running small
+// independent launches of one call beside its main stream: fork_side() makes
+// `side` wait for the work issued so far on `st`; join_side() makes `st` wait
+// for what was issued on `side` since.  Both are stream-ordered (they work
+// inside a CUDA-graph capture of `st`).
+slora_status side_stream(cudaStream_t* side);
+slora_status fork_side(cudaStream_t st, cudaStream_t side);
+slora_status join_side(cudaStream_t st, cudaStream_t side);
 // Number of 128-row tiles of the context rows / output rows.
 int64_t count_tiles(const slora_tokens* tok, bool ctx);
 inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }

@@ -413,6 +413,20 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
 
 
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
+  // The small LoRA operand layouts run on the library's side stream, beside
+  // the pass over X and the estimator (first those independent of the
+  // selection, then, once it is known, the ones on the kept channels); the
+  // main stream joins them before the first GEMM.
+  cudaStream_t side = nullptr;
+  SLORA_TRY(side_stream(&side));
+  SLORA_TRY(fork_side(st, side));
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, side, Fd));
+  SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, side));
+  SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, side));
+  if (bpad) {
+    SLORA_TRY(gather_pad(L.Bg, r, nullptr, Fd, r, BgP, lr, side, Fd));
+    SLORA_TRY(gather_pad(L.Bu, r, nullptr, Fd, r, BuP, lr, side, Fd));
+  }
   SLORA_TRY(stack_rows(L.Ag, L.Au, r, r, d, AgAu, st));
   {  // one stream over X: XA = X [Ag; Au]^T (fp32 and s*XA bf16) and, for the
      // estimator, P = X [Lg | Lu] (fp32-accurate, read for the context rows)
@@ -438,24 +452,25 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
                                      L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, eb, st, fused,
                                      Pfull, 2 * rs, rsp));
   }
-  // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
-  SLORA_TRY(gather_rows(L.Wg, d, idx, kk, d, WgS, d, st, Fd));
-  SLORA_TRY(gather_rows(L.Wu, d, idx, kk, d, WuS, d, st, Fd));
-  SLORA_TRY(gather_rows(L.Wd_t, d, idx, kk, d, WdS, d, st, Fd));
-  // LoRA operand packing (bf16, tiny)
-  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, st, Fd));
-  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, st, Fd));
-  SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, st));
-  SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, st));
-  SLORA_TRY(copy_pad(L.Bd, d, r, lr, Bdp, st));
+  SLORA_TRY(fork_side(st, side));  // the selection is known
+  SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, side, Fd));
+  SLORA_TRY(transpose_rows(L.Ad, r, Fd, idx, kk, lr, AdtS, side));
   if (proj) {
-    SLORA_TRY(gather_pad(L.Bg, r, idx, kk, r, BgS, lr, st, Fd));
-    SLORA_TRY(gather_pad(L.Bu, r, idx, kk, r, BuS, lr, st, Fd));
-    if (bpad) {
-      SLORA_TRY(gather_pad(L.Bg, r, nullptr, Fd, r, BgP, lr, st, Fd));
-      SLORA_TRY(gather_pad(L.Bu, r, nullptr, Fd, r, BuP, lr, st, Fd));
-    }
+    SLORA_TRY(gather_pad(L.Bg, r, idx, kk, r, BgS, lr, side, Fd));
+    SLORA_TRY(gather_pad(L.Bu, r, idx, kk, r, BuS, lr, side, Fd));
   }
+  // selected slices of the frozen weights as contiguous rows (HBM-speed gather)
+  {
+    GatherJob gw[3];
+    const void* src[3] = {L.Wg, L.Wu, L.Wd_t};
+    void* dst[3] = {WgS, WuS, WdS};
+    for (int k = 0; k < 3; ++k) {
+      gw[k].in = src[k]; gw[k].out = dst[k];
+      gw[k].ld_in16 = d / 8; gw[k].ld_out16 = d / 8; gw[k].rows_in = Fd;
+    }
+    SLORA_TRY(gather_rows_multi(gw, 3, idx, kk, d, st));
+  }
+  SLORA_TRY(join_side(st, side));
 
   // ---- forward
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u

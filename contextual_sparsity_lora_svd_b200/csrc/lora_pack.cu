@@ -8,6 +8,8 @@
 //   stack_rows     : out = [top; bottom]      ([A_g; A_u], MN-major operand)
 #include "lora_pack.cuh"
 
+#include "gemm_tc.cuh"
+
 namespace slora {
 namespace {
 
@@ -60,6 +62,40 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ in, int64_t ld_in16
   for (int64_t c = int64_t(blockIdx.y) * blockDim.x + threadIdx.x; c < cols16;
        c += int64_t(gridDim.y) * blockDim.x)
     out[j * ld_out16 + c] = ok ? __ldg(in + src * ld_in16 + c) : make_uint4(0, 0, 0, 0);
+}
+
+// Several row compactions sharing one index list: warp w takes (job, row)
+// items w, w + nwarps, ...; each lane moves 8 16-byte units per round (all
+// loads of a round issued before its stores).
+__global__ void __launch_bounds__(256) gather_rows_multi_kernel(const GatherJobs J,
+                                                                const int32_t* __restrict__ idx,
+                                                                int64_t n, int64_t cols16) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = int64_t(gridDim.x) * (blockDim.x >> 5);
+  const int64_t items = n * J.njobs;
+  for (int64_t it = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+       it += nw) {
+    const int jb = int(it / n);
+    const int64_t j = it % n;
+    const GatherJob& g = J.job[jb];
+    const int64_t src = idx[j];
+    const bool ok = index_ok(src, g.rows_in);
+    const uint4* in = static_cast<const uint4*>(g.in) + (ok ? src : 0) * g.ld_in16;
+    uint4* out = static_cast<uint4*>(g.out) + j * g.ld_out16;
+    for (int64_t c0 = lane; c0 < cols16; c0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + 32 * u;
+        v[u] = (ok && c < cols16) ? __ldg(in + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t c = c0 + 32 * u;
+        if (c < cols16) out[c] = v[u];
+      }
+    }
+  }
 }
 
 __global__ void stack_rows_kernel(const __nv_bfloat16* __restrict__ top,
@@ -172,6 +208,30 @@ slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const in
   transpose_rows_kernel<<<blocks(n * ldo), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(in), rows, cols, idx, n, ldo,
       static_cast<__nv_bfloat16*>(out));
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status gather_rows_multi(const GatherJob* jobs, int njobs, const int32_t* idx, int64_t n,
+                               int64_t cols, cudaStream_t st) {
+  if (n <= 0 || njobs <= 0) return SLORA_OK;
+  if (njobs > GatherJobs::kMax)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "gather_rows_multi: %d jobs (max %d)", njobs, GatherJobs::kMax);
+  GatherJobs J{};
+  J.njobs = njobs;
+  for (int k = 0; k < njobs; ++k) {
+    const GatherJob& g = jobs[k];
+    if (cols % 8 || g.ld_in16 < 0 || g.ld_out16 < 0 ||
+        (reinterpret_cast<uintptr_t>(g.in) & 15) || (reinterpret_cast<uintptr_t>(g.out) & 15))
+      SLORA_FAIL(SLORA_ERR_ALIGN, "gather_rows_multi: rows must be whole 16-byte units");
+    J.job[k] = g;
+  }
+  const int64_t items = n * njobs;
+  const int64_t want = (items + 7) / 8;  // 8 warps per block
+  const int64_t cap = int64_t(num_sms()) * 4;  // 32 warps per SM, 16 KB of loads in flight each
+  LaunchScope ls(kCompact, 2.0 * double(njobs) * double(n) * cols * 2, st);
+  gather_rows_multi_kernel<<<unsigned(std::max<int64_t>(1, std::min(want, cap))), 256, 0, st>>>(
+      J, idx, n, cols / 8);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

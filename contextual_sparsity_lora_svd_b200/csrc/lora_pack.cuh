@@ -19,6 +19,22 @@ slora_status transpose_rows(const void* in, int64_t rows, int64_t cols, const in
 slora_status gather_rows(const void* in, int64_t ld_in, const int32_t* idx, int64_t n,
                          int64_t cols, void* out, int64_t ld_out, cudaStream_t st,
                          int64_t rows_in);
+// Up to three compactions sharing one index list in one launch: job k copies
+// rows idx[j] of in_k (rows_in_k rows, leading dimension ld_in16 x 16 bytes)
+// to row j of out_k (leading dimension ld_out16 x 16 bytes), `cols` bf16
+// (a multiple of 8) per row; same index rule as gather_rows.
+struct GatherJob {
+  const void* in = nullptr;
+  void* out = nullptr;
+  int64_t ld_in16 = 0, ld_out16 = 0, rows_in = 0;
+};
+struct GatherJobs {
+  static constexpr int kMax = 3;
+  GatherJob job[kMax];
+  int njobs = 0;
+};
+slora_status gather_rows_multi(const GatherJob* jobs, int njobs, const int32_t* idx, int64_t n,
+                               int64_t cols, cudaStream_t st);
 // out [(rows_top + rows_bottom) x cols] = [top; bottom].
 slora_status stack_rows(const void* top, const void* bottom, int64_t rows_top,
                         int64_t rows_bottom, int64_t cols, void* out, cudaStream_t st);

@@ -131,6 +131,58 @@ int64_t count_tiles(const slora_tokens* tok, bool ctx) {
   return n;
 }
 
+namespace {
+constexpr int kSideDevices = 64;
+struct Side {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+Side g_side[kSideDevices];
+slora_status side_for(Side** out) {
+  int dev = -1;
+  SLORA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kSideDevices)
+    SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kSideDevices);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  Side& sd = g_side[dev];
+  if (!sd.s) {
+    SLORA_CUDA(cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking));
+    SLORA_CUDA(cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming));
+    SLORA_CUDA(cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming));
+  }
+  *out = &sd;
+  return SLORA_OK;
+}
+}  // namespace
+
+slora_status side_stream(cudaStream_t* side) {
+  Side* sd = nullptr;
+  SLORA_TRY(side_for(&sd));
+  *side = sd->s;
+  return SLORA_OK;
+}
+
+// The record and the wait happen under the lock, so calls from several host
+// threads cannot interleave on the shared events.
+slora_status fork_side(cudaStream_t st, cudaStream_t side) {
+  Side* sd = nullptr;
+  SLORA_TRY(side_for(&sd));
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SLORA_CUDA(cudaEventRecord(sd->fork, st));
+  SLORA_CUDA(cudaStreamWaitEvent(side, sd->fork, 0));
+  return SLORA_OK;
+}
+
+slora_status join_side(cudaStream_t st, cudaStream_t side) {
+  Side* sd = nullptr;
+  SLORA_TRY(side_for(&sd));
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SLORA_CUDA(cudaEventRecord(sd->join, side));
+  SLORA_CUDA(cudaStreamWaitEvent(st, sd->join, 0));
+  return SLORA_OK;
+}
+
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles,
                             int4* out_tiles, unsigned* zero, int64_t nzero) {

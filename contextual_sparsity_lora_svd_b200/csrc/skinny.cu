@@ -12,14 +12,15 @@
 // bit-reproducible, no second launch.
 //
 // When Y is a plain strided matrix (no row gather) a second kernel takes the
-// contraction: a persistent, stream-K style grid of exactly one wave.  The
-// flattened (output block x reduction chunk) space is cut into one contiguous,
-// equal slice per CTA; each CTA streams its slice through a TMA ring of
-// 128-byte-swizzled 64 x 64 tiles of Y (plus the matching tile of the split
-// operand) completed on mbarriers, with fragments read by ldmatrix.  A block
-// covered by one CTA alone is written directly from its accumulators; a block
-// shared by several CTAs gets their partial tiles summed in CTA order by the
-// last one to finish.
+// contraction: a persistent grid of one wave (two CTAs per SM) that takes
+// fixed (output block, reduction group) units from an atomic ticket.  A
+// producer warp streams each unit through a TMA ring of 128-byte-swizzled
+// 64 x 64 tiles of Y (plus the matching tile of the split operand) completed
+// on mbarriers; four consumer warps read fragments by ldmatrix.  A block
+// covered by one unit is written directly from its accumulators; otherwise
+// every unit writes its partial tile to its own slot and the last unit of the
+// block to finish sums them in group order.  One launch may carry several
+// independent contractions (a job table sharing the ticket).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -624,20 +625,10 @@ struct TmaJobs {
 static_assert(sizeof(TmaJobs<kMaxTmaJobs>) <= 4096, "TMA job table beyond 4 KB of parameters");
 
 // Shared memory of the TMA kernel: S stages of [Y tile 64x64 | split-R tile],
-// each 1024-byte aligned (128-byte swizzle), then the stage barriers and the
-// stages' work descriptors.
+// each 1024-byte aligned (128-byte swizzle), then the stages' full and empty
+// barriers (8 slots each) and work descriptors.
 constexpr int kYTile = TILE * TILE * 2;
 constexpr int tma_stage_bytes(int CP, int NT) { return kYTile + NT * CP * 128; }
-constexpr int tma_stages(int CP, int NT) {
-  return (113 * 1024 - 1216) / tma_stage_bytes(CP, NT) > 8
-             ? 8
-             : ((113 * 1024 - 1216) / tma_stage_bytes(CP, NT) < 2
-                    ? 2
-                    : (113 * 1024 - 1216) / tma_stage_bytes(CP, NT));
-}
-constexpr int tma_smem(int CP, int NT) {
-  return tma_stages(CP, NT) * tma_stage_bytes(CP, NT) + 1024 + 8 * 8 + 8 * 16;
-}
 constexpr int kTmaCtasPerSm = 2;
 
 // Element (row, k) of a 128-byte-swizzled tile whose rows are 64 bf16: byte
@@ -646,6 +637,34 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk16) {
   return base + uint32_t(row) * 128u + (uint32_t((chunk16 ^ (row & 7))) << 4);
 }
 
+// Stages that fit two CTAs per SM (113 KB each with the barrier block), 2..8.
+constexpr int tma_stages(int CP, int NT) {
+  return (113 * 1024 - 1280) / tma_stage_bytes(CP, NT) > 8
+             ? 8
+             : ((113 * 1024 - 1280) / tma_stage_bytes(CP, NT) < 2
+                    ? 2
+                    : (113 * 1024 - 1280) / tma_stage_bytes(CP, NT));
+}
+constexpr int tma_smem(int CP, int NT) {
+  return tma_stages(CP, NT) * tma_stage_bytes(CP, NT) + 1024 + 64 + 64 + 128;
+}
+// Barrier of the four consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// last_arrival() among the consumer warps: true in every consumer thread of
+// the CTA that brings `counter` to n (and resets it).
+__device__ __forceinline__ bool last_arrival_c(unsigned* counter, unsigned n, int tid) {
+  __shared__ unsigned s_last_c;
+  __threadfence();
+  bar_consumers();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(counter, 1u);
+    s_last_c = (prev + 1 == n) ? 1u : 0u;
+    if (s_last_c) *counter = 0u;
+  }
+  bar_consumers();
+  if (s_last_c) __threadfence();
+  return s_last_c != 0;
+}
 // COL = false: rowdot (output block = 64 rows of Y, reduction over K);
 // COL = true: coldot (output block = 64 columns of Y, reduction over M).
 // Work of one job: output blocks of 64 (rows for rowdot, columns for
@@ -656,87 +675,103 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int chunk16) {
 // faster take more units.  Each unit's partial lands in its own slot and the
 // last unit of a block to finish sums the block's slots in group order: the
 // result does not depend on which CTA ran which unit.
+//
+// Warp 4 (one lane) produces: it takes the unit tickets and keeps every stage
+// of the TMA ring filled, refilling a stage as soon as the four consumer
+// warps have each released it on the stage's `empty` barrier.  Warps 0-3
+// consume: each owns 16 rows (rowdot) or 16 columns (coldot) of the 64 x 64
+// tile and issues the mma.sync fragments; they synchronise among themselves
+// (named barrier 1) only at the end of a unit whose block is shared.
 template <int NF, int NT, bool COL, int J>
-__global__ void __launch_bounds__(NTH) skinny_tma_kernel(const __grid_constant__ TmaJobs<J> jobs) {
+__global__ void __launch_bounds__(NTH + 32) skinny_tma_kernel(const __grid_constant__ TmaJobs<J> jobs) {
   constexpr int CP = NF * 8, S = tma_stages(CP, NT), SB = tma_stage_bytes(CP, NT);
   constexpr int kLast = 2, kEnd = 4, kJobShift = 4;
   extern __shared__ unsigned char sk_smem[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(sk_smem) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + S * SB);
-  int4* info = reinterpret_cast<int4*>(sm + S * SB + 8 * 8);  // {block, chunk, flags, group}
+  uint64_t* empty = full + 8;
+  int4* info = reinterpret_cast<int4*>(sm + S * SB + 128);  // {block, chunk, flags, group}
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   unsigned* work = jobs.ticket;
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // ---- producer state (thread 0): current job and unit, and its next chunk
-  int pj = 0, pb = 0, pg = 0, pk = 0, pk1 = 0, issued = 0;
-  bool pdone = false;
-  auto next_unit = [&]() {  // false once the tickets are exhausted
-    const unsigned u = atomicAdd(work, 1u);
-    if (u >= unsigned(jobs.nunits)) {
-      if (u == unsigned(jobs.nunits + jobs.ncta - 1)) *work = 0u;  // the last ticket resets
-      return false;
-    }
-    int jb = 0;
+  if (warp == 4) {
+    if (lane != 0) return;
+    int pj = 0, pb = 0, pg = 0, pk = 0, pk1 = 0, issued = 0;
+    bool pdone = false;
+    auto next_unit = [&]() {
+      const unsigned u = atomicAdd(work, 1u);
+      if (u >= unsigned(jobs.nunits)) {
+        if (u == unsigned(jobs.nunits + jobs.ncta - 1)) *work = 0u;
+        return false;
+      }
+      int jb = 0;
 #pragma unroll
-    for (int x = 1; x < J; ++x)
-      if (x < jobs.njobs && u >= unsigned(jobs.job[x].unit0)) jb = x;
-    const StreamPlan& P = jobs.job[jb].p;
-    const unsigned lu = u - unsigned(jobs.job[jb].unit0);
-    pj = jb;
-    pb = int(lu % unsigned(P.nblocks));
-    pg = int(lu / unsigned(P.nblocks));
-    pk = pg * P.G;
-    pk1 = pk + P.G < P.nchunks ? pk + P.G : P.nchunks;
-    return true;
-  };
-  auto issue = [&]() {  // thread 0: the next position of the stream into stage issued % S
-    const int st = issued % S;
-    if (!pdone && pk == pk1 && !next_unit()) pdone = true;
-    if (pdone) {  // end marker: completes the stage's phase without data
-      info[st] = make_int4(0, 0, kEnd, 0);
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&full[st])) : "memory");
+      for (int x = 1; x < J; ++x)
+        if (x < jobs.njobs && u >= unsigned(jobs.job[x].unit0)) jb = x;
+      const StreamPlan& P = jobs.job[jb].p;
+      const unsigned lu = u - unsigned(jobs.job[jb].unit0);
+      pj = jb;
+      pb = int(lu % unsigned(P.nblocks));
+      pg = int(lu / unsigned(P.nblocks));
+      pk = pg * P.G;
+      pk1 = pk + P.G < P.nchunks ? pk + P.G : P.nchunks;
+      return true;
+    };
+    bool ok = true;
+    while (true) {
+      const int st = issued % S;
+      if (issued >= S && !mbar_wait_bounded(&empty[st], uint32_t(((issued / S) - 1) & 1), g_sk_budget)) {
+        s_abort = 1;
+        ok = false;
+        break;
+      }
+      if (s_abort) { ok = false; break; }
+      if (!pdone && pk == pk1 && !next_unit()) pdone = true;
+      if (pdone) {
+        info[st] = make_int4(0, 0, kEnd, 0);
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&full[st])) : "memory");
+        ++issued;
+        break;
+      }
+      info[st] = make_int4(pb, pk, (pk + 1 == pk1 ? kLast : 0) | (pj << kJobShift), pg);
+      unsigned char* ys = sm + st * SB;
+      const TmaJob& jb = jobs.job[pj];
+      mbar_arm(&full[st], uint32_t(SB));
+      if (COL)
+        tma2d(ys, &jb.ymap, &full[st], pb * TILE, pk * TILE);
+      else
+        tma2d(ys, &jb.ymap, &full[st], pk * TILE, pb * TILE);
+      tma2d(ys + kYTile, &jb.rmap, &full[st], pk * TILE, 0);
+      ++pk;
       ++issued;
-      return false;
     }
-    info[st] = make_int4(pb, pk, (pk + 1 == pk1 ? kLast : 0) | (pj << kJobShift), pg);
-    unsigned char* ys = sm + st * SB;
-    const TmaJob& jb = jobs.job[pj];
-    mbar_arm(&full[st], uint32_t(SB));
-    if (COL)
-      tma2d(ys, &jb.ymap, &full[st], pb * TILE, pk * TILE);
-    else
-      tma2d(ys, &jb.ymap, &full[st], pk * TILE, pb * TILE);
-    tma2d(ys + kYTile, &jb.rmap, &full[st], pk * TILE, 0);
-    ++pk;
-    ++issued;
-    return true;
-  };
-  if (tid == 0) {
-    for (int j = 0; j < S; ++j)
-      if (!issue()) break;
+    if (!ok) {  // let the copies already issued land before exiting
+      for (int jj = issued > S ? issued - S : 0; jj < issued; ++jj)
+        mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1), kSkWaitBudget);
+    }
+    return;
   }
-  // per-lane fragment addressing (row % 8 == lane % 8 for every ldmatrix row)
   const int l7 = lane & 7, mi = lane >> 3;
-  const int a_row = warp * 16 + l7 + (mi & 1) * 8, a_half = mi >> 1;     // rowdot A (Y rows)
-  const int at_rowoff = (mi >> 1) * 8 + l7, at_chunk = warp * 2 + (mi & 1);  // coldot A (Y^T)
-  const int b_rowoff = (mi >> 1) * 8 + l7, b_half = mi & 1;              // split R
-
+  const int a_row = warp * 16 + l7 + (mi & 1) * 8, a_half = mi >> 1;
+  const int at_rowoff = (mi >> 1) * 8 + l7, at_chunk = warp * 2 + (mi & 1);
+  const int b_rowoff = (mi >> 1) * 8 + l7, b_half = mi & 1;
   float acc[NF][4];
 #pragma unroll
   for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
-
-  int j = 0;
-  for (;; ++j) {
+  for (int j = 0;; ++j) {
     const int st = j % S;
     if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1), g_sk_budget)) s_abort = 1;
-    const int4 inf = info[st];  // published before the stage's barrier arrival
+    const int4 inf = info[st];
     if (!s_abort && !(inf.z & kEnd)) {
       const uint32_t ybase = su32(sm + st * SB), rbase = ybase + kYTile;
 #pragma unroll
@@ -757,17 +792,15 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(const __grid_constant__
           }
       }
     }
-    __syncthreads();  // every warp is done with stage st (and has read its info)
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&empty[st])) : "memory");
     if (s_abort || (inf.z & kEnd)) break;
-    if (tid == 0 && !pdone) issue();
-    if (!(inf.z & kLast)) continue;  // the unit goes on
-
-    // ---- end of unit (job inf.z >> kJobShift, block inf.x, group inf.w)
+    if (!(inf.z & kLast)) continue;
     const TmaJob& jb = jobs.job[inf.z >> kJobShift];
     const int b = inf.x, c = jb.c, ngroups = jb.p.ngroups;
     const int64_t nout = COL ? jb.K : jb.M;
-    const int64_t r0 = int64_t(b) * TILE + warp * 16 + g;  // output index of acc rows g / g + 8
-    if (ngroups == 1) {  // the unit is the whole block: emit from the accumulators
+    const int64_t r0 = int64_t(b) * TILE + warp * 16 + g;
+    if (ngroups == 1) {
 #pragma unroll
       for (int f = 0; f < NF; ++f) {
         const int col = f * 8 + 2 * t;
@@ -793,7 +826,7 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(const __grid_constant__
         *reinterpret_cast<float2*>(mine + lr * CP + col) = make_float2(acc[f][0], acc[f][1]);
         *reinterpret_cast<float2*>(mine + (lr + 8) * CP + col) = make_float2(acc[f][2], acc[f][3]);
       }
-      if (last_arrival(jb.counters + b, unsigned(ngroups), tid)) {
+      if (last_arrival_c(jb.counters + b, unsigned(ngroups), tid)) {
         const int nq4 = (c + 3) / 4;
         const float* blk = jb.part + int64_t(b) * ngroups * TILE * CP;
         for (int e = tid; e < TILE * nq4; e += NTH) {
@@ -816,10 +849,6 @@ __global__ void __launch_bounds__(NTH) skinny_tma_kernel(const __grid_constant__
     }
 #pragma unroll
     for (int f = 0; f < NF; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.0f;
-  }
-  if (s_abort && tid == 0) {  // let the copies already issued land before exiting
-    for (int jj = j; jj < issued; ++jj)
-      mbar_wait_bounded(&full[jj % S], uint32_t((jj / S) & 1), kSkWaitBudget);
   }
 }
 
@@ -940,7 +969,7 @@ slora_status launch_tma_kernel(const TmaJobs<J>& jb, cudaStream_t st) {
   auto kfn = skinny_tma_kernel<NF, NT, COL, J>;
   const int sm = tma_smem(NF * 8, NT);
   SLORA_CUDA(cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, sm));
-  kfn<<<jb.ncta, NTH, sm, st>>>(jb);
+  kfn<<<jb.ncta, NTH + 32, sm, st>>>(jb);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
