@@ -15,10 +15,33 @@ namespace {
 // it keeps their U_g, U_u rows in registers and reads each token's projected
 // row P_g | P_u from shared memory as 16-byte broadcasts, reused for its CPT
 // channels (the shared-memory reads, not the math, bounded the one-channel
-// version).  Partial sums of squares per (chunk, channel), fixed token order.
+// version).  With an even CPT the rank-r dot products of two channels run as
+// one packed fma.rn.f32x2 per rank index (the token's projection is staged
+// duplicated, {v, v}); each lane's chain is the same fused multiply-adds in
+// the same order as the scalar form, so the scores are unchanged.  Partial
+// sums of squares per (chunk, channel), fixed token order.
 constexpr int kScoreTT = 32;  // tokens staged per round
+constexpr int kSMs148 = 148;  // B200 SM count (grid sizing only)
 template <int RP>
 constexpr int score_cpt() { return RP <= 8 ? 4 : (RP <= 16 ? 2 : 1); }
+
+__device__ __forceinline__ unsigned long long pack_f2(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_f2(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi), each rounded once (fused)
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 
 template <int RP>
 __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
@@ -26,54 +49,102 @@ __global__ void __launch_bounds__(128) ffn_score_partial_kernel(
     const float* __restrict__ Ug, const float* __restrict__ Uu, int64_t n, int r, int64_t chunk,
     float* __restrict__ partial) {
   constexpr int CPT = score_cpt<RP>();
-  __shared__ __align__(16) float sp[kScoreTT][2 * RP];
   const int64_t j0 = int64_t(blockIdx.x) * 128 * CPT + threadIdx.x;
   const int64_t t0 = int64_t(blockIdx.y) * chunk;
   const int64_t t1 = min(T_C, t0 + chunk);
-  float ug[CPT][RP], uu[CPT][RP], acc[CPT];
+  float acc[CPT];
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
+  for (int i = 0; i < CPT; ++i) acc[i] = 0.0f;
+  auto uval = [&](const float* U, int i, int q) {
     const int64_t j = j0 + 128 * i;
-    acc[i] = 0.0f;
+    return (j < n && q < r) ? U[j * r + q] : 0.0f;
+  };
+  auto pval = [&](int64_t tb, int tt, int nt, int q) {
+    const int half = q / RP, qq = q % RP;
+    if (tt >= nt || qq >= r) return 0.0f;
+    const int64_t row = pmap ? int64_t(pmap[tb + tt]) : tb + tt;
+    return P[row * ldp + half * r + qq];
+  };
+  if constexpr (CPT % 2 == 0) {
+    constexpr int NPR = CPT / 2;  // channel pairs per thread
+    __shared__ __align__(16) unsigned long long sp2[kScoreTT][2 * RP];
+    unsigned long long ug2[NPR][RP], uu2[NPR][RP];
 #pragma unroll
-    for (int q = 0; q < RP; ++q) {
-      ug[i][q] = (j < n && q < r) ? Ug[j * r + q] : 0.0f;
-      uu[i][q] = (j < n && q < r) ? Uu[j * r + q] : 0.0f;
-    }
-  }
-  for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
-    const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
-    __syncthreads();
-    for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x) {
-      const int tt = e / (2 * RP), q = e % (2 * RP);
-      const int half = q / RP, qq = q % RP;
-      float v = 0.0f;
-      if (tt < nt && qq < r) {
-        const int64_t row = pmap ? int64_t(pmap[tb + tt]) : tb + tt;
-        v = P[row * ldp + half * r + qq];
+    for (int pr = 0; pr < NPR; ++pr)
+#pragma unroll
+      for (int q = 0; q < RP; ++q) {
+        ug2[pr][q] = pack_f2(uval(Ug, 2 * pr, q), uval(Ug, 2 * pr + 1, q));
+        uu2[pr][q] = pack_f2(uval(Uu, 2 * pr, q), uval(Uu, 2 * pr + 1, q));
       }
-      sp[tt][q] = v;
-    }
-    __syncthreads();
-    for (int tt = 0; tt < nt; ++tt) {
-      float pg[RP], pu[RP];
-#pragma unroll
-      for (int q4 = 0; q4 < RP / 4; ++q4) {
-        const float4 a = *reinterpret_cast<const float4*>(&sp[tt][4 * q4]);
-        const float4 b = *reinterpret_cast<const float4*>(&sp[tt][RP + 4 * q4]);
-        pg[4 * q4] = a.x; pg[4 * q4 + 1] = a.y; pg[4 * q4 + 2] = a.z; pg[4 * q4 + 3] = a.w;
-        pu[4 * q4] = b.x; pu[4 * q4 + 1] = b.y; pu[4 * q4 + 2] = b.z; pu[4 * q4 + 3] = b.w;
+    for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
+      const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
+      __syncthreads();
+      for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x) {
+        const int tt = e / (2 * RP), q = e % (2 * RP);
+        const float v = pval(tb, tt, nt, q);
+        sp2[tt][q] = pack_f2(v, v);
       }
+      __syncthreads();
+      for (int tt = 0; tt < nt; ++tt) {
+        unsigned long long pg[RP], pu[RP];
 #pragma unroll
-      for (int i = 0; i < CPT; ++i) {
-        float g = 0.0f, u = 0.0f;
-#pragma unroll
-        for (int q = 0; q < RP; ++q) {
-          g = fmaf(pg[q], ug[i][q], g);
-          u = fmaf(pu[q], uu[i][q], u);
+        for (int q2 = 0; q2 < RP / 2; ++q2) {
+          const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(&sp2[tt][2 * q2]);
+          const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(&sp2[tt][RP + 2 * q2]);
+          pg[2 * q2] = a.x; pg[2 * q2 + 1] = a.y;
+          pu[2 * q2] = b.x; pu[2 * q2 + 1] = b.y;
         }
-        const float a = silu_f(g) * u;
-        acc[i] = fmaf(a, a, acc[i]);
+#pragma unroll
+        for (int pr = 0; pr < NPR; ++pr) {
+          unsigned long long g2 = 0ull, u2 = 0ull;
+#pragma unroll
+          for (int q = 0; q < RP; ++q) {
+            g2 = ffma2(pg[q], ug2[pr][q], g2);
+            u2 = ffma2(pu[q], uu2[pr][q], u2);
+          }
+          const float2 g = unpack_f2(g2), u = unpack_f2(u2);
+          const float a0 = silu_f(g.x) * u.x, a1 = silu_f(g.y) * u.y;
+          acc[2 * pr] = fmaf(a0, a0, acc[2 * pr]);
+          acc[2 * pr + 1] = fmaf(a1, a1, acc[2 * pr + 1]);
+        }
+      }
+    }
+  } else {
+    __shared__ __align__(16) float sp[kScoreTT][2 * RP];
+    float ug[CPT][RP], uu[CPT][RP];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i)
+#pragma unroll
+      for (int q = 0; q < RP; ++q) {
+        ug[i][q] = uval(Ug, i, q);
+        uu[i][q] = uval(Uu, i, q);
+      }
+    for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
+      const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
+      __syncthreads();
+      for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x)
+        sp[e / (2 * RP)][e % (2 * RP)] = pval(tb, e / (2 * RP), nt, e % (2 * RP));
+      __syncthreads();
+      for (int tt = 0; tt < nt; ++tt) {
+        float pg[RP], pu[RP];
+#pragma unroll
+        for (int q4 = 0; q4 < RP / 4; ++q4) {
+          const float4 a = *reinterpret_cast<const float4*>(&sp[tt][4 * q4]);
+          const float4 b = *reinterpret_cast<const float4*>(&sp[tt][RP + 4 * q4]);
+          pg[4 * q4] = a.x; pg[4 * q4 + 1] = a.y; pg[4 * q4 + 2] = a.z; pg[4 * q4 + 3] = a.w;
+          pu[4 * q4] = b.x; pu[4 * q4 + 1] = b.y; pu[4 * q4 + 2] = b.z; pu[4 * q4 + 3] = b.w;
+        }
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+          float g = 0.0f, u = 0.0f;
+#pragma unroll
+          for (int q = 0; q < RP; ++q) {
+            g = fmaf(pg[q], ug[i][q], g);
+            u = fmaf(pu[q], uu[i][q], u);
+          }
+          const float a = silu_f(g) * u;
+          acc[i] = fmaf(a, a, acc[i]);
+        }
       }
     }
   }
@@ -259,9 +330,35 @@ __global__ void __launch_bounds__(1024) topk_select_kernel(const float* __restri
 
 int score_cpt_for(int r) { return r <= 8 ? 4 : (r <= 16 ? 2 : 1); }
 
+// Resident 128-thread score blocks per SM for the kernel serving rank r
+// (register-limited; 4 if the query fails).
+int score_blocks_per_sm(int r) {
+  static int cached[4] = {0, 0, 0, 0};
+  const int slot = r <= 8 ? 0 : (r <= 16 ? 1 : (r <= 32 ? 2 : 3));
+  if (!cached[slot]) {
+    int b = 0;
+    cudaError_t e;
+    switch (slot) {
+      case 0: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<8>, 128, 0); break;
+      case 1: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<16>, 128, 0); break;
+      case 2: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<32>, 128, 0); break;
+      default: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<48>, 128, 0); break;
+    }
+    if (e != cudaSuccess || b < 1) {
+      cudaGetLastError();
+      b = 4;
+    }
+    cached[slot] = b;
+  }
+  return cached[slot];
+}
+
+// Token splits: as many as keep the grid within one wave of resident blocks
+// (a second, partial wave cost more than the split's extra partial sums).
 int ffn_score_splits(int64_t T_C, int64_t n, int r) {
   const int64_t nb = (n + 128 * score_cpt_for(r) - 1) / (128 * score_cpt_for(r));
-  int64_t want = (6 * 148 + nb - 1) / nb;  // about six 128-thread blocks per SM
+  const int64_t slots = int64_t(kSMs148) * score_blocks_per_sm(r);
+  int64_t want = slots / std::max<int64_t>(nb, 1);
   int64_t maxs = (T_C + kScoreTT - 1) / kScoreTT;
   int64_t s = want < maxs ? want : maxs;
   if (s < 1) s = 1;
