@@ -37,6 +37,12 @@
  *     call launches nothing (argument errors) or reports the first CUDA error
  *     (SLORA_ERR_CUDA).  slora_last_error_string() gives a thread-local text.
  *     Calls are re-entrant when given distinct workspaces and outputs.
+ *   - slora_ffn_fwd_bwd runs some small launches on a library-owned side
+ *     stream of the current device (created on first use, never destroyed),
+ *     forked from `stream` by an event and joined back to it before the call
+ *     returns, so everything stays ordered on `stream` and the call can be
+ *     captured into a CUDA graph.  While one host thread captures such a
+ *     call, no other thread may run an FFN call on the same device.
  *   - Requires an sm_100 device (SLORA_ERR_UNSUPPORTED otherwise).
  */
 #ifndef SLORA_H_

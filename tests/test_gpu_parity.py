@@ -254,14 +254,20 @@ def test_ffn_ragged_and_edges(L, bf16, ctx):
         assert np.all(res["dAd"][:, skip] == 0)
 
 
+@pytest.mark.parametrize("bf16", [False, True])
 @pytest.mark.parametrize("s", [0.0, 0.99])
-def test_ffn_sparsity_extremes(L, s):
+def test_ffn_sparsity_extremes(L, s, bf16):
+    """Every channel kept, and one or two kept: in bf16 the context-row GEMMs then
+    have N below one 32-channel epilogue chunk (clipped TMA boxes and stores)."""
     tok = _tok(2, 64, [48, 48])
-    case = synth.ffn_case(tok, 64, 136, 8, 4, s, bf16=False, workload=0, layer=4)
+    case = synth.ffn_case(tok, 64, 136, 8, 4, s, bf16=bf16, workload=0, layer=4)
     lay = _ffn_lay(case, 8)
     ref = O.ffn_fwd_bwd(case.X, case.dOut, tok.batch, tok.seq, tok.ctx_len, lay, s)
+    tol = TOL["bf16" if bf16 else "f32"]
     res = run_ffn_gpu(L, case, lay)
     assert res["k"] == ref["k"]
     nd = check_selection(res["idx"], ref["idx"], ref["scores"], ref["k"], "select")
     if nd == 0:
-        _compare_ffn(res, ref, TOL["f32"])
+        _compare_ffn(res, ref, tol)
+    res2 = run_ffn_gpu(L, case, lay, idx_force=ref["idx"])
+    _compare_ffn(res2, ref, tol)
