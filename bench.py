@@ -449,6 +449,20 @@ def run_ours(args, rank, world):
            "GB/s": (by_e + by_s) / ((ms_e + ms_s) / 1e3) / 1e9 if ms_e + ms_s > 0 else None}
     if est["GB/s"]:
         est["frac_hbm"] = est["GB/s"] / pk["hbm"]
+    # The FFN score is bound by arithmetic, not HBM: per (context token, channel)
+    # pair it needs 2 r_svd FMAs and two MUFU ops (exp, reciprocal) for the silu.
+    # Per SM and clock: 128 fp32 FMA lanes, 16 MUFU lanes; 148 SMs at the sampled
+    # SM clock (the maximum when NVML gave none).
+    w = WORKLOAD
+    pairs = w["batch"] * (w["seq"] - int(round(w["out_frac"] * w["seq"]))) * w["d_ff"]
+    mhz = clk.summary().get("sm_mhz") or clk.summary().get("sm_max_mhz") or 1965.0
+    hz = float(mhz) * 1e6
+    t_fma = pairs * 2 * w["r_svd"] / (128 * 148 * hz)
+    t_mufu = pairs * 2 / (16 * 148 * hz)
+    if ms_e > 0:
+        est["score_alu"] = {"bound": "alu", "pairs": pairs, "bound_us": 1e6 * max(t_fma, t_mufu),
+                            "achieved_us": 1e3 * ms_e / args.steps,
+                            "frac": 1e6 * max(t_fma, t_mufu) / (1e3 * ms_e / args.steps)}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
