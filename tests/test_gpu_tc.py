@@ -1,6 +1,7 @@
 """Parity of the bf16 tcgen05 path at sizes spanning several 128x256 tiles,
 ragged sequence lengths (tiles shorter than 128 rows), channel counts that are
-not multiples of the tile width, and both LoRA ranks used by the workloads."""
+not multiples of the tile width, both LoRA ranks used by the workloads and one
+above the ranks the GEMM epilogues project."""
 import numpy as np
 import pytest
 import torch
@@ -23,6 +24,9 @@ def L():
     ([300, 170, 320], 512, 1200, 0.5, 16),
     ([256, 256], 768, 2048, 0.3, 8),
     ([129, 1, 200], 264, 1000, 0.7, 16),
+    # rank above 16: no rank projections in the GEMM epilogues (hA and
+    # [dG Bg | dU Bu] by separate contractions), TMA epilogue without slices
+    ([300, 170, 320], 512, 1200, 0.5, 24),
 ])
 def test_ffn_tc_multi_tile(L, ctx, d, d_ff, s, r):
     tok = synth.Tokens(len(ctx), 320 if len(ctx) != 2 else 384, np.asarray(ctx, np.int32))
