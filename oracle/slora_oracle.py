@@ -27,7 +27,7 @@ import numpy as np
 
 __all__ = [
     "context_rows", "silu", "silu_grad", "svd_prepare", "project",
-    "ffn_scores", "qk_scores", "keep_count", "topk_select", "select_per_group",
+    "ffn_scores", "ffn_gram_scores", "qk_scores", "keep_count", "topk_select", "select_per_group",
     "estimate_select_ffn", "estimate_select_qk",
     "linear_fwd", "linear_bwd", "ffn_fwd", "ffn_bwd", "ffn_fwd_bwd",
 ]
@@ -89,6 +89,21 @@ def ffn_scores(P_g, P_u, U_g, U_u) -> np.ndarray:
     Uh = P_u @ U_u.T
     act = silu(G) * Uh
     return np.sqrt(np.sum(act * act, axis=0))
+
+
+def ffn_gram_scores(P_g, P_u, U_g, U_u) -> np.ndarray:
+    """Gram-computable FFN channel score, an estimator variant (reading of the
+    article's sections 1-2: a cheaper stand-in for the activation norm).
+
+    Score of channel j: ||g_hat[:, j]|| * ||u_hat[:, j]|| over the context
+    tokens, g_hat = P_g U_g^T, u_hat = P_u U_u^T.  Each factor is a quadratic
+    form of an r x r Gram matrix (||g_hat[:, j]||^2 = U_g[j] (P_g^T P_g) U_g[j]^T),
+    so no per-(token, channel) silu is needed; it bounds the activation-norm
+    score from above, since |silu(x)| <= |x| and ||a * b|| <= ||a|| ||b||.
+    """
+    G = P_g @ U_g.T
+    Uh = P_u @ U_u.T
+    return np.sqrt(np.sum(G * G, axis=0)) * np.sqrt(np.sum(Uh * Uh, axis=0))
 
 
 def qk_scores(P_q, P_k, U_q, U_k, heads: int, kv_heads: int, head_dim: int) -> np.ndarray:

@@ -120,6 +120,41 @@ def test_qk_score_gram_identity():
     np.testing.assert_allclose(got.ravel(), nq * nk, rtol=1e-12)
 
 
+def test_ffn_gram_score_full_rank_exact_and_gram_form():
+    """The Gram-computable FFN variant: at full rank it is the product of the
+    exact column norms of X W_g^T and X W_u^T; each norm equals its r x r Gram
+    quadratic form; and it is the one-head QK-norm of the gate/up factors (the
+    GPU path runs this variant through the QK criterion with one head)."""
+    tok = synth.Tokens(batch=2, seq=9, ctx_len=np.array([6, 8], np.int32))
+    d, d_ff = 10, 14
+    X = synth.gaussian((tok.T, d), 1.0, 41)
+    Wg = synth.decaying_weight(d_ff, d, 42).W * 10
+    Wu = synth.decaying_weight(d_ff, d, 43).W * 10
+    Lg, Ug = _full_rank_factors(Wg)
+    Lu, Uu = _full_rank_factors(Wu)
+    C, _ = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    Pg, Pu = O.project(X[C], Lg), O.project(X[C], Lu)
+    got = O.ffn_gram_scores(Pg, Pu, Ug, Uu)
+    exact = colnorm(X[C] @ Wg.T) * colnorm(X[C] @ Wu.T)
+    np.testing.assert_allclose(got, exact, rtol=1e-11)
+    ng = np.sqrt(np.einsum("cr,rs,cs->c", Ug, Pg.T @ Pg, Ug))
+    nu = np.sqrt(np.einsum("cr,rs,cs->c", Uu, Pu.T @ Pu, Uu))
+    np.testing.assert_allclose(got, ng * nu, rtol=1e-11)
+    np.testing.assert_allclose(got, O.qk_scores(Pg, Pu, Ug, Uu, 1, 1, d_ff)[0], rtol=1e-12)
+
+
+def test_ffn_gram_score_bounds_activation_norm():
+    """|silu(x)| <= |x| and ||a * b|| <= ||a|| ||b||: the Gram variant is an
+    upper bound of the activation-norm score, channel by channel."""
+    rg = synth.rng(44)
+    for t, r, n in ((5, 3, 7), (40, 8, 33)):
+        Pg, Pu = rg.standard_normal((t, r)), rg.standard_normal((t, r))
+        Ug, Uu = rg.standard_normal((n, r)), rg.standard_normal((n, r))
+        act = O.ffn_scores(Pg, Pu, Ug, Uu)
+        gram = O.ffn_gram_scores(Pg, Pu, Ug, Uu)
+        assert np.all(act <= gram * (1 + 1e-12))
+
+
 def test_qk_gqa_equals_mha_on_replicated_keys():
     """A GQA group score equals the sum of MHA scores of its query heads when
     the shared key head is replicated once per query head."""
