@@ -1,5 +1,5 @@
 """The reference arm of bench.py (the fp64 oracle on the host cores) keeps the
-JSON-line contract the driver reads: one line with the same metric, unit,
+bench's JSON-line contract: one line with the same metric, unit,
 direction and workload config as the GPU arm, impl "reference", a
 cpu_baseline describing the run and an e2e object with zero copy bytes."""
 import json
