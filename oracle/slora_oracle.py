@@ -27,8 +27,10 @@ import numpy as np
 
 __all__ = [
     "context_rows", "silu", "silu_grad", "svd_prepare", "project",
-    "ffn_scores", "ffn_gram_scores", "qk_scores", "keep_count", "topk_select", "select_per_group",
-    "estimate_select_ffn", "estimate_select_qk",
+    "ffn_scores", "ffn_gram_scores", "qk_scores", "qk_pair_scores", "l2_scores",
+    "keep_count", "topk_select", "select_per_group",
+    "estimate_select_ffn", "estimate_select_qk", "estimate_select_ffn_gram",
+    "estimate_select_qk_pairs", "estimate_select_l2",
     "linear_fwd", "linear_bwd", "ffn_fwd", "ffn_bwd", "ffn_fwd_bwd",
 ]
 
@@ -129,6 +131,43 @@ def qk_scores(P_q, P_k, U_q, U_k, heads: int, kv_heads: int, head_dim: int) -> n
     return out
 
 
+def qk_pair_scores(P_q, P_k, U_q, U_k, heads: int, kv_heads: int, head_dim: int) -> np.ndarray:
+    """QK-norm over rotate-half channel pairs, an estimator variant (reading of
+    the article's section 1 criterion for models with rotary embeddings).
+
+    Rotary position embedding turns channels c and c + head_dim/2 of a head
+    together by a token-dependent angle, so a pair is kept or dropped as one
+    unit.  The pair's norm over the context tokens is taken over both of its
+    channels, sqrt(||Y_hat[:, c]||^2 + ||Y_hat[:, c + half]||^2), which the
+    rotation leaves unchanged; pair p of group g scores ||K_hat_{g,p}|| times
+    the sum over the group's query heads of ||Q_hat_{h,p}||.  Returns a
+    (kv_heads, head_dim // 2) array.
+    """
+    half = head_dim // 2
+    Qh = P_q @ U_q.T
+    Kh = P_k @ U_k.T
+    sq = np.sum(Qh * Qh, axis=0).reshape(heads, head_dim)
+    sk = np.sum(Kh * Kh, axis=0).reshape(kv_heads, head_dim)
+    nq = np.sqrt(sq[:, :half] + sq[:, half:])
+    nk = np.sqrt(sk[:, :half] + sk[:, half:])
+    group = heads // kv_heads
+    out = np.zeros((kv_heads, half))
+    for g in range(kv_heads):
+        qsum = np.zeros(half)
+        for h in range(g * group, (g + 1) * group):
+            qsum = qsum + nq[h]
+        out[g] = nk[g] * qsum
+    return out
+
+
+def l2_scores(P, U, heads: int, head_dim: int) -> np.ndarray:
+    """Per-channel L2 norm of one estimated projection over the context tokens,
+    per head: a (heads, head_dim) array (reading for the value projection,
+    whose output channels are the input channels of the output projection)."""
+    Yh = P @ U.T
+    return np.sqrt(np.sum(Yh * Yh, axis=0)).reshape(heads, head_dim)
+
+
 # ---------------------------------------------------------------------------
 # selection (article section 1: per-input choice of active channels)
 # ---------------------------------------------------------------------------
@@ -178,6 +217,51 @@ def estimate_select_qk(X, batch, seq, ctx_len, L_q, U_q, L_k, U_k,
     idx_q = np.concatenate([h * head_dim + sel[h // group] for h in range(heads)])
     idx_k = np.concatenate([g * head_dim + sel[g] for g in range(kv_heads)])
     return idx_q, idx_k, k, scores
+
+
+def estimate_select_ffn_gram(X, batch, seq, ctx_len, L_g, U_g, L_u, U_u, sparsity):
+    """Estimator + selection for a SwiGLU FFN with the Gram-computable score
+    ``ffn_gram_scores`` in place of the activation norm: (idx, k_keep, scores)."""
+    C, _ = context_rows(batch, seq, ctx_len)
+    Xc = X[C]
+    scores = ffn_gram_scores(project(Xc, L_g), project(Xc, L_u), U_g, U_u)
+    k = keep_count(scores.size, sparsity)
+    return topk_select(scores, k), k, scores
+
+
+def estimate_select_qk_pairs(X, batch, seq, ctx_len, L_q, U_q, L_k, U_k,
+                             heads, kv_heads, head_dim, sparsity):
+    """Estimator + per-group selection of rotate-half pairs for q/k.
+
+    k_p = keep_count(head_dim / 2, s) pairs are kept per group; each head keeps
+    the 2 k_p channels of those pairs, listed as the pairs' first channels
+    (ascending) followed by their partners c + head_dim/2.  Returns
+    (idx_q, idx_k, 2 k_p, pair scores)."""
+    C, _ = context_rows(batch, seq, ctx_len)
+    Xc = X[C]
+    half = head_dim // 2
+    scores = qk_pair_scores(project(Xc, L_q), project(Xc, L_k), U_q, U_k, heads, kv_heads,
+                            head_dim)
+    kp = keep_count(half, sparsity)
+    sel = select_per_group(scores, kp)
+    chans = np.concatenate([sel, sel + half], axis=1)
+    group = heads // kv_heads
+    idx_q = np.concatenate([h * head_dim + chans[h // group] for h in range(heads)])
+    idx_k = np.concatenate([g * head_dim + chans[g] for g in range(kv_heads)])
+    return idx_q, idx_k, 2 * kp, scores
+
+
+def estimate_select_l2(X, batch, seq, ctx_len, L, U, heads, head_dim, sparsity):
+    """Estimator + per-head selection by the L2 norm of one projection's
+    estimated output: (idx, k_h, scores) with idx listing, for every head h,
+    its kept channels as h*head_dim + c (ascending)."""
+    C, _ = context_rows(batch, seq, ctx_len)
+    Xc = X[C]
+    scores = l2_scores(project(Xc, L), U, heads, head_dim)
+    k = keep_count(head_dim, sparsity)
+    sel = select_per_group(scores, k)
+    idx = np.concatenate([h * head_dim + sel[h] for h in range(heads)])
+    return idx, k, scores
 
 
 # ---------------------------------------------------------------------------

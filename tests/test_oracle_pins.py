@@ -238,6 +238,225 @@ def test_select_sparsity_zero_keeps_all():
     assert O.topk_select(score, O.keep_count(33, 0.0)).tolist() == list(range(33))
 
 
+# ------------------------------------------------------ QK per-group selection
+# A hand-built grouped-query case (4 query heads, 2 key heads, head_dim 4, one
+# context token, d = rank = 1).  With X_C = [[1]] and L = [[1]] the estimate is
+# Q_hat[0, c] = U_q[c, 0], so every channel norm is |U_q[c, 0]| and the scores
+# below follow by hand:
+#   group 0 (query heads 0, 1):  |K| = [1, 1, 1, 2],  sum|Q| = [4, 4, 3, 1.5]
+#                                score = [4, 4, 3, 3]
+#   group 1 (query heads 2, 3):  |K| = [2, 1, .5, 1], sum|Q| = [1, 3, 6, 2]
+#                                score = [2, 3, 3, 2]
+_QK_UQ = [[1, 4, 2, 0.5], [3, 0, 1, 1], [1, 1, 1, 1], [0, 2, 5, 1]]
+_QK_UK = [[1, 1, 1, 2], [2, 1, 0.5, 1]]
+# The second row is an output token with a huge value: it must not count.
+_QK_X = np.array([[1.0], [1000.0]])
+# (sparsity, expected idx_q, expected idx_k) written out literally:
+#   s = 0.5 keeps 2 per group: group 0 {0, 1}; group 1 {1, 2}.
+#   s = 0.25 keeps 3: group 0 {0, 1, 2} (the 3-3 tie goes to channel 2);
+#   group 1 {0, 1, 2} (the 2-2 tie goes to channel 0).
+#   s = 0 keeps all four channels of every head.
+_QK_EXPECT = [
+    (0.5, [0, 1, 4, 5, 9, 10, 13, 14], [0, 1, 5, 6]),
+    (0.25, [0, 1, 2, 4, 5, 6, 8, 9, 10, 12, 13, 14], [0, 1, 2, 4, 5, 6]),
+    (0.0, list(range(16)), list(range(8))),
+]
+
+
+def _qk_hand_case(estimator, s):
+    U_q = np.array(_QK_UQ, dtype=float).reshape(16, 1)
+    U_k = np.array(_QK_UK, dtype=float).reshape(8, 1)
+    one = np.ones((1, 1))
+    return estimator(_QK_X, 1, 2, [1], one, U_q, one, U_k, 4, 2, 4, s)
+
+
+def _check_qk_hand_case(estimator):
+    for s, want_q, want_k in _QK_EXPECT:
+        idx_q, idx_k, k, scores = _qk_hand_case(estimator, s)
+        assert k == len(want_k) // 2, (s, k)
+        assert np.asarray(idx_q).tolist() == want_q, (s, np.asarray(idx_q).tolist())
+        assert np.asarray(idx_k).tolist() == want_k, (s, np.asarray(idx_k).tolist())
+    np.testing.assert_allclose(scores, [[4, 4, 3, 3], [2, 3, 3, 2]], rtol=1e-15)
+
+
+def test_estimate_select_qk_hand_built_gqa_layout():
+    """Literal idx_q / idx_k of the hand-built 4-query / 2-key-head case: each
+    query head h takes its group's set (group h // 2) as h*4 + c, each key head
+    g its own set as g*4 + c; ties go to the lower channel; the output token is
+    ignored."""
+    _check_qk_hand_case(O.estimate_select_qk)
+
+
+def _brute_force_group_topk(row, k):
+    return _brute_force_topk(list(row), k)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_select_per_group_brute_force_with_ties(seed):
+    """Every row of select_per_group is the brute-force best k-subset of that
+    row (largest sum, then lowest indices), ascending."""
+    rg = synth.rng(300 + seed)
+    groups, N = int(rg.integers(1, 5)), int(rg.integers(1, 9))
+    k = int(rg.integers(0, N + 1))
+    scores = rg.integers(0, 3, size=(groups, N)).astype(float)
+    got = O.select_per_group(scores, k)
+    assert got.shape == (groups, k)
+    for g in range(groups):
+        assert got[g].tolist() == _brute_force_group_topk(scores[g], k)
+
+
+def test_estimate_select_qk_matches_exact_norms_and_brute_force():
+    """Full-rank factors on a random GQA case (3 groups of 2 query heads,
+    head_dim 6): the scores equal the exact norm products of X_C W^T (torch
+    column norms), and each group's set is the brute-force top-k of them."""
+    rg = synth.rng(77)
+    H, KV, hd, d = 6, 3, 6, 5
+    tok = synth.Tokens(batch=2, seq=4, ctx_len=np.array([3, 2], np.int32))
+    X = rg.standard_normal((tok.T, d))
+    Wq, Wk = rg.standard_normal((H * hd, d)), rg.standard_normal((KV * hd, d))
+    Lq, Uq = _full_rank_factors(Wq)
+    Lk, Uk = _full_rank_factors(Wk)
+    idx_q, idx_k, k, scores = O.estimate_select_qk(X, tok.batch, tok.seq, tok.ctx_len, Lq, Uq,
+                                                   Lk, Uk, H, KV, hd, 0.5)
+    Xc = X[[0, 1, 2, 4, 5]]
+    nq = colnorm(Xc @ Wq.T).reshape(H, hd)
+    nk = colnorm(Xc @ Wk.T).reshape(KV, hd)
+    want = np.stack([nk[g] * (nq[2 * g] + nq[2 * g + 1]) for g in range(KV)])
+    np.testing.assert_allclose(scores, want, rtol=1e-10)
+    assert k == 3
+    for g in range(KV):
+        sel = _brute_force_group_topk(want[g], k)
+        assert np.asarray(idx_k[g * k:(g + 1) * k]).tolist() == [g * hd + c for c in sel]
+        for h in (2 * g, 2 * g + 1):
+            assert np.asarray(idx_q[h * k:(h + 1) * k]).tolist() == [h * hd + c for c in sel]
+
+
+# ------------------------------------------------- estimator variants (pins)
+def _rope_rotate(Y, head_dim, seed):
+    """Rotate every (c, c + head_dim/2) pair of every head of Y (tokens x
+    heads*head_dim) by a token- and pair-dependent angle (rotary embedding's
+    rotate-half form), with torch: an implementation independent of the oracle."""
+    T, n = Y.shape
+    half = head_dim // 2
+    ang = torch.from_numpy(synth.rng(seed).uniform(-np.pi, np.pi, size=(T, half)))
+    t = torch.from_numpy(Y).reshape(T, n // head_dim, head_dim)
+    x1, x2 = t[..., :half], t[..., half:]
+    c, s = torch.cos(ang)[:, None, :], torch.sin(ang)[:, None, :]
+    out = torch.cat([x1 * c - x2 * s, x1 * s + x2 * c], dim=-1)
+    return out.reshape(T, n).numpy()
+
+
+def _pair_norms_torch(Y, heads, head_dim):
+    half = head_dim // 2
+    t = torch.from_numpy(Y).reshape(Y.shape[0], heads, 2, half)
+    return torch.sqrt((t * t).sum(dim=(0, 2))).numpy()  # (heads, half)
+
+
+@pytest.mark.parametrize("H,KV", [(3, 3), (4, 2)])
+def test_qk_pair_scores_equal_post_rotary_pair_norms(H, KV):
+    """Pair scores computed from the estimate before rotary embedding equal the
+    norm products of the rotated estimates, pair by pair: the rotate-half
+    partner of channel c is c + head_dim/2 (an adjacent pairing fails this)."""
+    rg = synth.rng(501)
+    hd, r, t = 6, 4, 9
+    P_q, P_k = rg.standard_normal((t, r)), rg.standard_normal((t, r))
+    U_q, U_k = rg.standard_normal((H * hd, r)), rg.standard_normal((KV * hd, r))
+    got = O.qk_pair_scores(P_q, P_k, U_q, U_k, H, KV, hd)
+    Qr = _rope_rotate(P_q @ U_q.T, hd, 502)
+    Kr = _rope_rotate(P_k @ U_k.T, hd, 503)
+    nq, nk = _pair_norms_torch(Qr, H, hd), _pair_norms_torch(Kr, KV, hd)
+    grp = H // KV
+    want = np.stack([nk[g] * nq[g * grp:(g + 1) * grp].sum(axis=0) for g in range(KV)])
+    np.testing.assert_allclose(got, want, rtol=1e-12)
+
+
+def test_qk_pair_scores_reduce_to_qk_when_partners_vanish():
+    """With the second half of every head zeroed, a pair's score is the plain
+    QK-norm score of its first channel."""
+    rg = synth.rng(504)
+    H, KV, hd, r, t = 4, 2, 8, 3, 7
+    P_q, P_k = rg.standard_normal((t, r)), rg.standard_normal((t, r))
+    U_q, U_k = rg.standard_normal((H * hd, r)), rg.standard_normal((KV * hd, r))
+    for U in (U_q, U_k):
+        U.reshape(-1, hd, r)[:, hd // 2:, :] = 0.0
+    pair = O.qk_pair_scores(P_q, P_k, U_q, U_k, H, KV, hd)
+    plain = O.qk_scores(P_q, P_k, U_q, U_k, H, KV, hd)
+    np.testing.assert_allclose(pair, plain[:, :hd // 2], rtol=1e-12)
+
+
+def test_qk_pair_score_bounds_rotated_products():
+    """Cauchy-Schwarz: whatever the rotation angles, a pair's summed share of
+    the query-key products |sum_t <q_t,p, k_t,p>| stays within its score (MHA)."""
+    rg = synth.rng(505)
+    H, hd, r, t = 2, 4, 3, 11
+    P_q, P_k = rg.standard_normal((t, r)), rg.standard_normal((t, r))
+    U_q, U_k = rg.standard_normal((H * hd, r)), rg.standard_normal((H * hd, r))
+    sc = O.qk_pair_scores(P_q, P_k, U_q, U_k, H, H, hd)
+    for seed in range(5):
+        Qr = _rope_rotate(P_q @ U_q.T, hd, 600 + seed).reshape(t, H, 2, hd // 2)
+        Kr = _rope_rotate(P_k @ U_k.T, hd, 700 + seed).reshape(t, H, 2, hd // 2)
+        share = np.abs(np.einsum("thap,thap->hp", Qr, Kr))
+        assert np.all(share <= sc * (1 + 1e-12))
+
+
+def test_estimate_select_qk_pairs_hand_built_layout():
+    """Two query heads sharing one key head, head_dim 4 (pairs (0, 2), (1, 3)),
+    one context token, d = rank = 1, so the norms are the factor entries:
+      query head 0 [1, 2, 3, 0] -> pair norms [sqrt(10), 2]
+      query head 1 [0, 1, 0, 1] -> pair norms [0, sqrt(2)]
+      key head     [1, 1, 1, 1] -> pair norms [sqrt(2), sqrt(2)]
+    scores: pair 0 = sqrt(2) sqrt(10) = 4.47, pair 1 = sqrt(2) (2 + sqrt(2)) = 4.83.
+    At s = 0.5 one pair (pair 1) is kept: channels 1 and 3 of every head."""
+    U_q = np.array([1, 2, 3, 0, 0, 1, 0, 1], dtype=float).reshape(8, 1)
+    U_k = np.ones((4, 1))
+    one = np.ones((1, 1))
+    X = np.array([[1.0], [50.0]])
+    iq, ik, k, sc = O.estimate_select_qk_pairs(X, 1, 2, [1], one, U_q, one, U_k, 2, 1, 4, 0.5)
+    np.testing.assert_allclose(sc, [[math.sqrt(20), 2 * math.sqrt(2) + 2]], rtol=1e-14)
+    assert k == 2
+    assert iq.tolist() == [1, 3, 5, 7] and ik.tolist() == [1, 3]
+    iq, ik, k, _ = O.estimate_select_qk_pairs(X, 1, 2, [1], one, U_q, one, U_k, 2, 1, 4, 0.0)
+    assert k == 4 and iq.tolist() == list(range(8)) and ik.tolist() == [0, 1, 2, 3]
+
+
+def test_l2_scores_full_rank_exact_and_per_head_selection():
+    """Full-rank factors: the scores are the exact column norms of X_C W^T per
+    head (torch), and each head keeps the brute-force top-k of its own norms,
+    listed as h*head_dim + c."""
+    rg = synth.rng(510)
+    H, hd, d = 3, 5, 4
+    tok = synth.Tokens(batch=2, seq=3, ctx_len=np.array([2, 3], np.int32))
+    X = rg.standard_normal((tok.T, d))
+    W = rg.standard_normal((H * hd, d))
+    Lw, Uw = _full_rank_factors(W)
+    idx, k, sc = O.estimate_select_l2(X, tok.batch, tok.seq, tok.ctx_len, Lw, Uw, H, hd, 0.4)
+    want = colnorm(X[[0, 1, 3, 4, 5]] @ W.T).reshape(H, hd)
+    np.testing.assert_allclose(sc, want, rtol=1e-10)
+    assert k == 3
+    for h in range(H):
+        sel = _brute_force_topk(list(want[h]), k)
+        assert idx[h * k:(h + 1) * k].tolist() == [h * hd + c for c in sel]
+
+
+def test_estimate_select_ffn_gram_full_rank_brute_force():
+    """Full-rank gate/up factors: the Gram score is the product of the exact
+    column norms of X_C Wg^T and X_C Wu^T, and the kept set is the brute-force
+    best subset."""
+    rg = synth.rng(511)
+    d, d_ff = 4, 9
+    tok = synth.Tokens(batch=1, seq=6, ctx_len=np.array([5], np.int32))
+    X = rg.standard_normal((tok.T, d))
+    Wg, Wu = rg.standard_normal((d_ff, d)), rg.standard_normal((d_ff, d))
+    Lg, Ug = _full_rank_factors(Wg)
+    Lu, Uu = _full_rank_factors(Wu)
+    idx, k, sc = O.estimate_select_ffn_gram(X, tok.batch, tok.seq, tok.ctx_len, Lg, Ug, Lu, Uu,
+                                            0.5)
+    Xc = X[:5]
+    want = colnorm(Xc @ Wg.T) * colnorm(Xc @ Wu.T)
+    np.testing.assert_allclose(sc, want, rtol=1e-10)
+    assert k == 5 and idx.tolist() == _brute_force_topk(list(want), k)
+
+
 # ---------------------------------------------------------------- LoRA linear
 def _lin_case(seed, n=9, k=7, r=3, tok=None):
     tok = tok or synth.Tokens(batch=2, seq=5, ctx_len=np.array([3, 4], np.int32))
@@ -479,6 +698,69 @@ def test_planted_tie_break_is_caught(monkeypatch):
     with pytest.raises(AssertionError):
         for seed in range(12):
             test_topk_brute_force_with_ties(seed)
+
+
+def _qk_variant(query_group, key_offset):
+    """estimate_select_qk with its index layout rebuilt from the oracle's own
+    pieces, so a planted layout mistake can be checked against the pins."""
+    def est(X, batch, seq, ctx_len, L_q, U_q, L_k, U_k, heads, kv_heads, head_dim, s):
+        C, _ = O.context_rows(batch, seq, ctx_len)
+        Xc = X[C]
+        scores = O.qk_scores(Xc @ L_q, Xc @ L_k, U_q, U_k, heads, kv_heads, head_dim)
+        k = O.keep_count(head_dim, s)
+        sel = O.select_per_group(scores, k)
+        group = heads // kv_heads
+        idx_q = np.concatenate([h * head_dim + sel[query_group(h, group, kv_heads)]
+                                for h in range(heads)])
+        idx_k = np.concatenate([key_offset(g, group, head_dim) + sel[g] for g in range(kv_heads)])
+        return idx_q, idx_k, k, scores
+    return est
+
+
+def test_planted_qk_layout_mistakes_are_caught():
+    """The correct layout passes the hand-built pin; a query head mapped to the
+    wrong group (h % kv_heads instead of h // group) or key heads offset by the
+    query-head stride (g * group * head_dim) fail it."""
+    _check_qk_hand_case(_qk_variant(lambda h, gr, kv: h // gr, lambda g, gr, hd: g * hd))
+    with pytest.raises(AssertionError):
+        _check_qk_hand_case(_qk_variant(lambda h, gr, kv: h % kv, lambda g, gr, hd: g * hd))
+    with pytest.raises(AssertionError):
+        _check_qk_hand_case(_qk_variant(lambda h, gr, kv: h // gr, lambda g, gr, hd: g * gr * hd))
+
+
+def test_planted_group_select_mistake_is_caught(monkeypatch):
+    """select_per_group that takes the k smallest instead of the k largest."""
+    monkeypatch.setattr(O, "select_per_group",
+                        lambda sc, k: np.stack([np.sort(np.argsort(r, kind="stable")[:k])
+                                                for r in sc]))
+    with pytest.raises(AssertionError):
+        test_estimate_select_qk_hand_built_gqa_layout()
+
+
+def test_planted_adjacent_pairing_is_caught(monkeypatch):
+    """Pairs (2i, 2i + 1) instead of rotate-half (c, c + head_dim/2)."""
+    def adjacent(P_q, P_k, U_q, U_k, heads, kv_heads, head_dim):
+        Qh, Kh = P_q @ U_q.T, P_k @ U_k.T
+        sq = np.sum(Qh * Qh, axis=0).reshape(heads, head_dim // 2, 2).sum(axis=2)
+        sk = np.sum(Kh * Kh, axis=0).reshape(kv_heads, head_dim // 2, 2).sum(axis=2)
+        grp = heads // kv_heads
+        return np.stack([np.sqrt(sk[g]) * np.sqrt(sq[g * grp:(g + 1) * grp]).sum(axis=0)
+                         for g in range(kv_heads)])
+    monkeypatch.setattr(O, "qk_pair_scores", adjacent)
+    with pytest.raises(AssertionError):
+        test_qk_pair_scores_equal_post_rotary_pair_norms(3, 3)
+
+
+def test_planted_l2_head_offset_is_caught(monkeypatch):
+    """estimate_select_l2 listing every head's channels without the h*head_dim offset."""
+    real = O.estimate_select_l2
+
+    def broken(X, batch, seq, ctx_len, L, U, heads, head_dim, s):
+        idx, k, sc = real(X, batch, seq, ctx_len, L, U, heads, head_dim, s)
+        return idx % head_dim, k, sc
+    monkeypatch.setattr(O, "estimate_select_l2", broken)
+    with pytest.raises(AssertionError):
+        test_l2_scores_full_rank_exact_and_per_head_selection()
 
 
 def test_oracle_package_exports():
