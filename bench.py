@@ -292,6 +292,15 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     pk = peaks()
     case = make_case()
+    if world > 1:
+        # weak scaling: every rank runs its own 8 x 512-token batch, drawn from
+        # its own seeds (same layer weights on every rank)
+        import dataclasses
+        T, d = case.X.shape
+        seed = 1000 * 1 + 1_000_003 * (rank + 1)
+        case = dataclasses.replace(
+            case, X=synth.round_bf16(synth.gaussian((T, d), 1.0, seed)),
+            dOut=synth.round_bf16(synth.gaussian((T, d), 1.0, seed + 1)))
     G = GpuLayer(case, L)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -484,6 +493,29 @@ def run_ours(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def torchrun_argv(argv, n, script=None, port=None):
+    """Command that runs `script` (this file by default) with `argv` as N
+    ranks on this node, one process per GPU, rendezvous on 127.0.0.1."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+            "--master-port", str(port or free_port()),
+            os.path.abspath(script or __file__), *argv]
+
+
+def launch(argv, n, script=None, timeout_s=None) -> int:
+    """Starts N ranks of `script` under torch.distributed.run and returns the
+    launcher's exit status."""
+    import subprocess
+    return subprocess.run(torchrun_argv(argv, n, script), timeout=timeout_s).returncode
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -495,8 +527,15 @@ def main():
                     help="bracket the timed steps with cudaProfilerStart/Stop (for ncu "
                          "--profile-from-start off)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: start the N ranks ourselves
+        raise SystemExit(launch(sys.argv[1:], args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

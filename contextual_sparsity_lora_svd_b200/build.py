@@ -1,6 +1,6 @@
 """Builds libslora.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m contextual_sparsity_lora_svd_b200.build [--debug]
+    python -m contextual_sparsity_lora_svd_b200.build [-v] [--ptxas-info]
 
 Each .cu file under csrc/ is compiled with nvcc (-gencode
 arch=compute_100a,code=sm_100a -lineinfo -O3) in parallel, then linked into
