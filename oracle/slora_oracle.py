@@ -251,17 +251,27 @@ def estimate_select_qk_pairs(X, batch, seq, ctx_len, L_q, U_q, L_k, U_k,
     return idx_q, idx_k, 2 * kp, scores
 
 
-def estimate_select_l2(X, batch, seq, ctx_len, L, U, heads, head_dim, sparsity):
+def estimate_select_l2(X, batch, seq, ctx_len, L, U, heads, kv_heads, head_dim, sparsity):
     """Estimator + per-head selection by the L2 norm of one projection's
-    estimated output: (idx, k_h, scores) with idx listing, for every head h,
-    its kept channels as h*head_dim + c (ascending)."""
+    estimated output, for slicing the value projection on its output channels
+    and the output projection on the matching input channels.
+
+    The scored projection has kv_heads heads (U is kv_heads*head_dim x r);
+    with grouped queries, value channel (g, c) feeds output-projection input
+    channel (h, c) of every query head h of group g (reading: attention mixes
+    tokens, not channels, so a dropped value channel empties the same channel
+    of the attention output).  Returns (idx_o, idx_v, k_h, scores): idx_o lists
+    for every query head h its group's kept channels as h*head_dim + c, idx_v
+    the same sets for the kv heads as g*head_dim + c."""
     C, _ = context_rows(batch, seq, ctx_len)
     Xc = X[C]
-    scores = l2_scores(project(Xc, L), U, heads, head_dim)
+    scores = l2_scores(project(Xc, L), U, kv_heads, head_dim)
     k = keep_count(head_dim, sparsity)
     sel = select_per_group(scores, k)
-    idx = np.concatenate([h * head_dim + sel[h] for h in range(heads)])
-    return idx, k, scores
+    group = heads // kv_heads
+    idx_o = np.concatenate([h * head_dim + sel[h // group] for h in range(heads)])
+    idx_v = np.concatenate([g * head_dim + sel[g] for g in range(kv_heads)])
+    return idx_o, idx_v, k, scores
 
 
 # ---------------------------------------------------------------------------

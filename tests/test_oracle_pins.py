@@ -419,23 +419,28 @@ def test_estimate_select_qk_pairs_hand_built_layout():
     assert k == 4 and iq.tolist() == list(range(8)) and ik.tolist() == [0, 1, 2, 3]
 
 
-def test_l2_scores_full_rank_exact_and_per_head_selection():
+@pytest.mark.parametrize("H,KV", [(3, 3), (4, 2)])
+def test_l2_scores_full_rank_exact_and_per_head_selection(H, KV):
     """Full-rank factors: the scores are the exact column norms of X_C W^T per
-    head (torch), and each head keeps the brute-force top-k of its own norms,
-    listed as h*head_dim + c."""
+    value head (torch); each value head keeps the brute-force top-k of its own
+    norms, listed as g*head_dim + c, and every query head h repeats the set of
+    its group h // (H / KV) as h*head_dim + c."""
     rg = synth.rng(510)
-    H, hd, d = 3, 5, 4
+    hd, d = 5, 4
     tok = synth.Tokens(batch=2, seq=3, ctx_len=np.array([2, 3], np.int32))
     X = rg.standard_normal((tok.T, d))
-    W = rg.standard_normal((H * hd, d))
+    W = rg.standard_normal((KV * hd, d))
     Lw, Uw = _full_rank_factors(W)
-    idx, k, sc = O.estimate_select_l2(X, tok.batch, tok.seq, tok.ctx_len, Lw, Uw, H, hd, 0.4)
-    want = colnorm(X[[0, 1, 3, 4, 5]] @ W.T).reshape(H, hd)
+    io, iv, k, sc = O.estimate_select_l2(X, tok.batch, tok.seq, tok.ctx_len, Lw, Uw, H, KV, hd,
+                                         0.4)
+    want = colnorm(X[[0, 1, 3, 4, 5]] @ W.T).reshape(KV, hd)
     np.testing.assert_allclose(sc, want, rtol=1e-10)
     assert k == 3
-    for h in range(H):
-        sel = _brute_force_topk(list(want[h]), k)
-        assert idx[h * k:(h + 1) * k].tolist() == [h * hd + c for c in sel]
+    for g in range(KV):
+        sel = _brute_force_topk(list(want[g]), k)
+        assert iv[g * k:(g + 1) * k].tolist() == [g * hd + c for c in sel]
+        for h in range(g * (H // KV), (g + 1) * (H // KV)):
+            assert io[h * k:(h + 1) * k].tolist() == [h * hd + c for c in sel]
 
 
 def test_estimate_select_ffn_gram_full_rank_brute_force():
@@ -752,16 +757,22 @@ def test_planted_adjacent_pairing_is_caught(monkeypatch):
 
 
 def test_planted_l2_head_offset_is_caught(monkeypatch):
-    """estimate_select_l2 listing every head's channels without the h*head_dim offset."""
+    """estimate_select_l2 listing the query heads' channels without the
+    h*head_dim offset, or the value heads' with the query-head stride."""
     real = O.estimate_select_l2
 
-    def broken(X, batch, seq, ctx_len, L, U, heads, head_dim, s):
-        idx, k, sc = real(X, batch, seq, ctx_len, L, U, heads, head_dim, s)
-        return idx % head_dim, k, sc
-    monkeypatch.setattr(O, "estimate_select_l2", broken)
-    with pytest.raises(AssertionError):
-        test_l2_scores_full_rank_exact_and_per_head_selection()
+    def no_offset(X, batch, seq, ctx_len, L, U, heads, kv_heads, head_dim, s):
+        io, iv, k, sc = real(X, batch, seq, ctx_len, L, U, heads, kv_heads, head_dim, s)
+        return io % head_dim, iv, k, sc
 
+    def query_stride(X, batch, seq, ctx_len, L, U, heads, kv_heads, head_dim, s):
+        io, iv, k, sc = real(X, batch, seq, ctx_len, L, U, heads, kv_heads, head_dim, s)
+        grp = heads // kv_heads
+        return io, (iv // head_dim) * grp * head_dim + iv % head_dim, k, sc
+    for bad in (no_offset, query_stride):
+        monkeypatch.setattr(O, "estimate_select_l2", bad)
+        with pytest.raises(AssertionError):
+            test_l2_scores_full_rank_exact_and_per_head_selection(4, 2)
 
 def test_oracle_package_exports():
     for name in O.__all__:
