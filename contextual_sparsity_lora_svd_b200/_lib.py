@@ -31,7 +31,7 @@ P_SZ = ctypes.POINTER(c_sz)
 P_I32 = ctypes.POINTER(c_i32)
 
 F32, BF16 = 0, 1
-CRIT_FFN, CRIT_QK = 0, 1
+CRIT_FFN, CRIT_QK, CRIT_FFN_GRAM, CRIT_QK_ROPE_PAIR, CRIT_L2 = 0, 1, 2, 3, 4
 SLICE_NONE, SLICE_OUT_ROWS, SLICE_IN_COLS = 0, 1, 2
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGN", 4: "WORKSPACE", 5: "UNSUPPORTED",

@@ -101,22 +101,62 @@ extern "C" slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, s
 
 // --------------------------------------------------------- estimate+select
 namespace slora {
+CritPlan crit_plan(slora_criterion crit, int64_t n0, int heads, int kv_heads, int head_dim,
+                   double sparsity) {
+  CritPlan cp;
+  switch (crit) {
+    case SLORA_CRIT_FFN_SWIGLU_L2:
+      cp.activation = true;
+      cp.N = cp.nkeys = int(n0);
+      break;
+    case SLORA_CRIT_FFN_GRAM:  // ||g_hat_j|| * ||u_hat_j||: one group over d_ff
+      cp.mode = kCritModeQK;
+      cp.N = cp.nkeys = int(n0);
+      break;
+    case SLORA_CRIT_QK_NORM:
+    case SLORA_CRIT_QK_ROPE_PAIR:
+      cp.mode = kCritModeQK;
+      cp.groups = kv_heads;
+      cp.rep = heads / kv_heads;
+      cp.N = head_dim;
+      cp.pairs = crit == SLORA_CRIT_QK_ROPE_PAIR;
+      cp.nkeys = cp.pairs ? head_dim / 2 : head_dim;
+      break;
+    case SLORA_CRIT_L2_NORM:
+      cp.mode = kCritModeL2;
+      cp.nmat = 1;
+      cp.groups = kv_heads;
+      cp.rep = heads / kv_heads;
+      cp.N = cp.nkeys = head_dim;
+      break;
+  }
+  cp.kkeep = keep_count(cp.nkeys, sparsity);
+  cp.per_head = cp.pairs ? 2 * cp.kkeep : cp.kkeep;
+  return cp;
+}
+
 EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int64_t d, int64_t n0,
-                         int rank, int kv_heads, int head_dim, bool has_pre, float* scores_out,
-                         Arena& ar) {
+                         int rank, int heads, int kv_heads, int head_dim, bool has_pre,
+                         float* scores_out, Arena& ar) {
+  const CritPlan cp = crit_plan(crit, n0, heads, kv_heads, head_dim, 0.0);
   EstBufs eb;
-  if (!has_pre) eb.P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * 2 * rank);
+  if (!has_pre) eb.P = ar.take<float>(size_t(std::max<int64_t>(ti.T_C, 1)) * cp.nmat * rank);
   if (!has_pre && dt == kBF16) {
-    eb.ppart = ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, 2 * rank)));
+    const int nc = cp.nmat * rank <= 64 ? cp.nmat * rank : rank;  // columns of one pass
+    eb.ppart = ar.take<float>(size_t(rowdot_part_floats(ti.T_C, d, nc)));
     eb.prs = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(d)));
   }
-  const int64_t nsc = crit == SLORA_CRIT_FFN_SWIGLU_L2 ? n0 : int64_t(kv_heads) * head_dim;
+  const int64_t nsc = int64_t(cp.groups) * cp.nkeys;
   eb.scores = scores_out ? scores_out : ar.take<float>(size_t(nsc));
-  eb.nsplit = ffn_score_splits(ti.T_C, n0, rank);
-  if (crit == SLORA_CRIT_FFN_SWIGLU_L2)
+  if (cp.activation) {
+    eb.nsplit = ffn_score_splits(ti.T_C, n0, rank);
     eb.partial = ar.take<float>(size_t(eb.nsplit) * n0);
-  else
-    eb.gram = ar.take<double>(size_t(2) * rank * rank * 33);
+  } else {
+    eb.gram_part = ar.take<double>(size_t(gram_blocks(ti.T_C)) * cp.nmat * rank * rank);
+    eb.gram = ar.take<double>(size_t(cp.nmat) * rank * rank);
+  }
+  eb.ncnt = estimator_counter_count(cp.nkeys, rank, cp.groups);
+  eb.cnt = ar.take<unsigned>(size_t(eb.ncnt));
   return eb;
 }
 
@@ -124,58 +164,61 @@ slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
                                     const TokenInfo& ti, const int32_t* ctx_rows, int64_t d,
                                     const float* L0, const float* U0, int64_t n0, const float* L1,
                                     const float* U1, int rank, int heads, int kv_heads,
-                                    int head_dim, int64_t kkeep, int32_t* idx_out,
+                                    int head_dim, double sparsity, int32_t* idx_out,
                                     const EstBufs& eb, cudaStream_t st, bool has_pre,
-                                    const float* P_pre, int64_t ldp_pre, unsigned* counters) {
-  float* P = eb.P;
-  float* ppart = eb.ppart;
-  float* scores = eb.scores;
-  float* partial = eb.partial;
-  double* gram = eb.gram;
-  const int nsplit = eb.nsplit;
+                                    const float* P_pre, int64_t ldp_pre, unsigned* sk_counters) {
+  const CritPlan cp = crit_plan(crit, n0, heads, kv_heads, head_dim, sparsity);
   const float* Puse = P_pre;
   int64_t ldp = ldp_pre;
   const int32_t* pmap = has_pre ? ctx_rows : nullptr;
+  const int nc = cp.nmat * rank;
   if (!has_pre) {
-    // P = X_C [L0 | L1]
+    // P = X_C [L0 | L1] (or X_C L0 alone)
     if (dt == kBF16) {  // tensor-core stream over X_C, fp32 factors split in 3 bf16 terms
       SkY y;
       y.ptr = X; y.ld = d; y.map = ctx_rows;
-      SkR rr;
-      rr.ptr = L0; rr.dt = kF32; rr.si = rank; rr.sq = 1;
-      rr.qsplit = rank; rr.ptr_b = L1; rr.dt_b = kF32; rr.si_b = rank; rr.sq_b = 1;
-      SkRowOut o;
-      o.out1 = P; o.ld1 = 2 * rank;
-      if (!counters) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "estimator: counter workspace missing");
+      if (!sk_counters) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "estimator: counter workspace missing");
       SkWork w;
-      w.part = ppart;
+      w.part = eb.ppart;
       w.rsplit = eb.prs;
-      w.counters = counters;
-      SLORA_TRY(rowdot(y, ti.T_C, d, rr, 2 * rank, o, w, st));
+      w.counters = sk_counters;
+      // one pass for both factors when their columns fit the stream kernel's 64,
+      // else one pass per factor
+      const bool one_pass = nc <= 64;
+      for (int p = 0; p < (one_pass ? 1 : cp.nmat); ++p) {
+        SkR rr;
+        rr.ptr = p == 0 ? L0 : L1; rr.dt = kF32; rr.si = rank; rr.sq = 1;
+        if (one_pass && cp.nmat == 2) {
+          rr.qsplit = rank; rr.ptr_b = L1; rr.dt_b = kF32; rr.si_b = rank; rr.sq_b = 1;
+        }
+        SkRowOut o;
+        o.out1 = eb.P; o.ld1 = nc; o.off1 = int64_t(p) * rank;
+        SLORA_TRY(rowdot(y, ti.T_C, d, rr, one_pass ? nc : rank, o, w, st));
+      }
     } else {  // fp32 activations: CUDA-core fp32 FMA
-      for (int p = 0; p < 2; ++p) {
+      for (int p = 0; p < cp.nmat; ++p) {
         GemmArgs g;
         g.M = ti.T_C; g.N = rank; g.nseg = 1;
         g.seg[0].a = rowmajor(X, dt, d, ctx_rows);
         g.seg[0].b = colmajor(p == 0 ? L0 : L1, kF32, rank);
         g.seg[0].K = d;
-        g.c = out_rowmajor(P + p * rank, kF32, 2 * rank);
+        g.c = out_rowmajor(eb.P + p * rank, kF32, nc);
         SLORA_TRY(gemm_simt(g, st));
       }
     }
-    Puse = P;
-    ldp = 2 * rank;
+    Puse = eb.P;
+    ldp = nc;
   }
-  if (crit == SLORA_CRIT_FFN_SWIGLU_L2) {
-    SLORA_TRY(ffn_scores(Puse, ldp, pmap, ti.T_C, U0, U1, n0, rank, partial, nsplit, scores, st));
-    SLORA_TRY(topk_select(scores, 1, int(n0), int(kkeep), 1, idx_out, nullptr, st));
-  } else {
-    SLORA_TRY(qk_scores(Puse, ldp, pmap, ti.T_C, U0, U1, rank, heads, kv_heads, head_dim, gram,
-                        scores, st));
-    SLORA_TRY(topk_select(scores, kv_heads, head_dim, int(kkeep), heads / kv_heads, idx_out,
-                          idx_out + int64_t(heads) * kkeep, st));
-  }
-  return SLORA_OK;
+  if (cp.activation)
+    return ffn_score_select(Puse, ldp, pmap, ti.T_C, U0, U1, n0, rank, eb.partial, eb.nsplit,
+                            eb.scores, eb.cnt, int(cp.kkeep), idx_out, st);
+  int32_t* out_b = nullptr;
+  if (crit == SLORA_CRIT_QK_NORM || crit == SLORA_CRIT_QK_ROPE_PAIR ||
+      crit == SLORA_CRIT_L2_NORM)
+    out_b = idx_out + int64_t(heads) * cp.per_head;
+  return gram_scores_select(cp.mode, Puse, ldp, pmap, ti.T_C, U0, U1, rank, cp.groups, cp.rep,
+                            cp.N, cp.pairs, int(cp.kkeep), eb.gram_part, eb.gram, eb.scores,
+                            eb.cnt, idx_out, out_b, st);
 }
 }  // namespace slora
 
@@ -189,9 +232,13 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
   const char* fn = "slora_estimate_select";
   clear_error();
   SLORA_TRY(check_dtype(fn, dt));
-  if (crit != SLORA_CRIT_FFN_SWIGLU_L2 && crit != SLORA_CRIT_QK_NORM)
+  if (crit != SLORA_CRIT_FFN_SWIGLU_L2 && crit != SLORA_CRIT_QK_NORM &&
+      crit != SLORA_CRIT_FFN_GRAM && crit != SLORA_CRIT_QK_ROPE_PAIR &&
+      crit != SLORA_CRIT_L2_NORM)
     SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: unknown criterion %d", fn, int(crit));
-  REQ_PTR(X); REQ_PTR(L0); REQ_PTR(U0); REQ_PTR(L1); REQ_PTR(U1); REQ_PTR(idx_out);
+  const bool one_matrix = crit == SLORA_CRIT_L2_NORM;
+  REQ_PTR(X); REQ_PTR(L0); REQ_PTR(U0); REQ_PTR(idx_out);
+  if (!one_matrix) { REQ_PTR(L1); REQ_PTR(U1); }
   OPT_PTR(scores_out); OPT_PTR(ws);
   if (!k_out) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: k_out is NULL", fn);
   SLORA_TRY(check_sparsity(fn, sparsity));
@@ -199,35 +246,49 @@ extern "C" slora_status slora_estimate_select(slora_criterion crit, const void* 
   if (rank < 1 || rank > 48) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: rank %d outside [1, 48]", fn, rank);
   TokenInfo ti;
   SLORA_TRY(parse_tokens(tok, &ti));
-  int64_t kkeep;
-  if (crit == SLORA_CRIT_FFN_SWIGLU_L2) {
+  if (crit == SLORA_CRIT_FFN_SWIGLU_L2 || crit == SLORA_CRIT_FFN_GRAM) {
     if (n0 <= 0 || n0 != n1) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: FFN needs n0 == n1 > 0", fn);
-    if (n0 > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0 too large", fn);
-    kkeep = keep_count(n0, sparsity);
+    if (n0 > topk_max_keys())
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0=%lld beyond the %lld channels one selection supports",
+                 fn, (long long)n0, (long long)topk_max_keys());
+  } else if (crit == SLORA_CRIT_L2_NORM) {
+    if (heads <= 0 || kv_heads <= 0 || head_dim <= 0 || heads % kv_heads ||
+        n0 != int64_t(kv_heads) * head_dim)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: L2 criterion needs n0 == kv_heads*head_dim and heads a "
+                 "multiple of kv_heads (heads=%d, kv_heads=%d, head_dim=%d)", fn, heads,
+                 kv_heads, head_dim);
+    if (head_dim > topk_max_keys())
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: head_dim %d too large", fn, head_dim);
   } else {
     if (heads <= 0 || kv_heads <= 0 || head_dim <= 0 || heads % kv_heads)
       SLORA_FAIL(SLORA_ERR_SHAPE, "%s: heads=%d kv_heads=%d head_dim=%d", fn, heads, kv_heads,
                  head_dim);
     if (n0 != int64_t(heads) * head_dim || n1 != int64_t(kv_heads) * head_dim)
       SLORA_FAIL(SLORA_ERR_SHAPE, "%s: n0/n1 must be heads*head_dim / kv_heads*head_dim", fn);
-    kkeep = keep_count(head_dim, sparsity);
+    if (crit == SLORA_CRIT_QK_ROPE_PAIR && head_dim % 2)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: rotate-half pairs need an even head_dim (%d)", fn,
+                 head_dim);
+    if (head_dim > topk_max_keys())
+      SLORA_FAIL(SLORA_ERR_SHAPE, "%s: head_dim %d too large", fn, head_dim);
   }
+  const CritPlan cp = crit_plan(crit, n0, heads, kv_heads, head_dim, sparsity);
   const int64_t ncnt = skinny_counter_count(ti.T_C, d);
   Arena ar;  // one pass: sizes the query and places the buffers (finish_ws checks the size)
   ar.base = static_cast<char*>(ws);
   int32_t* ctx_rows = ar.take<int32_t>(size_t(std::max<int64_t>(ti.T_C, 1)));
   unsigned* cnt = ar.take<unsigned>(size_t(ncnt));
-  const EstBufs eb = estimate_reserve(crit, dt, ti, d, n0, rank, kv_heads, head_dim, false,
+  const EstBufs eb = estimate_reserve(crit, dt, ti, d, n0, rank, heads, kv_heads, head_dim, false,
                                       scores_out, ar);
   const bool query = ws == nullptr;
   SLORA_TRY(finish_ws(fn, ar, ws, ws_bytes));
-  *k_out = int32_t(kkeep);
+  *k_out = int32_t(cp.per_head);
   if (query) return SLORA_OK;
   SLORA_TRY(check_device());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st, nullptr, nullptr, cnt, ncnt));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, nullptr, st, nullptr, nullptr, cnt, ncnt, eb.cnt,
+                           eb.ncnt));
   return estimate_select_launch(crit, X, dt, ti, ctx_rows, d, L0, U0, n0, L1, U1, rank, heads,
-                                kv_heads, head_dim, kkeep, idx_out, eb, st, false, nullptr, 0,
+                                kv_heads, head_dim, sparsity, idx_out, eb, st, false, nullptr, 0,
                                 cnt);
 }
 
@@ -352,7 +413,7 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   }
   TokenInfo ti;
   SLORA_TRY(parse_tokens(tok, &ti));
-  FfnDesc F{int(dt), ti, Ly, Gr, kkeep};
+  FfnDesc F{int(dt), ti, Ly, Gr, kkeep, sparsity};
   Arena plan;
   SLORA_TRY(ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr));
   const bool query = ws == nullptr;

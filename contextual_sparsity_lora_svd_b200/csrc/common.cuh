@@ -71,6 +71,9 @@ slora_status arena_fits(const Arena& ar, const char* where);
 
 // ------------------------------------------------------------- devices
 slora_status check_device();  // sm_100 present and current
+// SMs of the current device (queried once and cached; 148 when no device
+// answers, e.g. during a host-only workspace query).
+int num_sms();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -85,11 +88,12 @@ slora_status parse_tokens(const slora_tokens* tok, TokenInfo* info);
 // Writes ctx_rows[T_C] and out_rows[T_O] (int32 row indices into the full
 // layout) and, when given, the 128-row M-tile lists of the context and output
 // rows: int4 {full_row0, compact_row0, nvalid, 0}, one list per row kind, a
-// tile never crossing a sequence.
+// tile never crossing a sequence.  It also zeroes the counter ranges `zero`
+// [nzero] and `zero2` [nzero2] that later kernels of the call count on.
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles = nullptr,
                             int4* out_tiles = nullptr, unsigned* zero = nullptr,
-                            int64_t nzero = 0);
+                            int64_t nzero = 0, unsigned* zero2 = nullptr, int64_t nzero2 = 0);
 // A library-owned side stream of the current device (non-blocking, created on
 // first use, kept until exit) with a fork and a join event, for running small
 // independent launches of one call beside its main stream: fork_side() makes

@@ -5,429 +5,757 @@
 // layer's output on the current context tokens; section 1 names the channel
 // criteria (FFN: L2 norm of a neuron's activity; q/k: QK-norm built from the
 // query-key product) and the per-input choice of active channels.
+//
+// Kernels
+//   ffn_score_select_kernel  activation-norm score of the SwiGLU channels:
+//       the rank-r dot products g_hat = P_g U_g^T, u_hat = P_u U_u^T run on the
+//       tensor cores (mma.sync, both fp32 operands split into three bf16 terms,
+//       the six significant cross products packed along K), the silu and the
+//       square-sum on the CUDA cores / MUFU.  Partial sums per (token split,
+//       channel); the last split of a channel block to arrive sums them in a
+//       fixed order (fp64), the last channel block to finish runs the top-k.
+//   gram_partial_kernel      r x r Gram matrices of P over token chunks, fp64;
+//       the last chunk to arrive sums them in a fixed order.
+//   norm_score_select_kernel per-channel norms as Gram quadratic forms
+//       ||Y_hat[:, c]||^2 = u_c^T (P^T P) u_c, combined per criterion (QK-norm
+//       product with grouped query heads, plain L2 norm, rotate-half pairs);
+//       the last channel block of a group runs that group's top-k.
+//   topk_kernel              top-k per group for score vectors too long for
+//       the fused select.
+// Top-k: bisection on the fp32 bit pattern of the scores (non-negative, so
+// unsigned order is numeric order), keys held in registers, block-wide counts
+// per step; then ties at the threshold go to the lower index and the indices
+// are written in ascending order (each thread owns a contiguous index range).
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
 #include "estimator.cuh"
 
 namespace slora {
 namespace {
 
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ uint32_t score_key(float v) {
+  uint32_t b = __float_as_uint(v);
+  if (b & 0x80000000u) b = 0;  // -0 (or a negative) ranks as zero
+  if (b > 0x7f800000u) b = 0;  // NaN ranks lowest
+  return b;
+}
+
+__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// v = h + m + l with h, m, l bf16 (nearest each); the residuals are exact in
+// fp32, so the three terms carry v to ~2^-24 relative.
+struct Split3 {
+  __nv_bfloat16 t[3];
+};
+__device__ __forceinline__ Split3 split3(float v) {
+  Split3 s;
+  s.t[0] = __float2bfloat16_rn(v);
+  float r = v - __bfloat162float(s.t[0]);
+  s.t[1] = __float2bfloat16_rn(r);
+  r -= __bfloat162float(s.t[1]);
+  s.t[2] = __float2bfloat16_rn(r);
+  return s;
+}
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return uint32_t(__bfloat16_as_ushort(lo)) | (uint32_t(__bfloat16_as_ushort(hi)) << 16);
+}
+
+// ------------------------------------------------------------ block reductions
+// Scratch: kRedWords words of shared memory, double-buffered by `parity` so a
+// reduction needs one barrier.
+template <int B>
+struct BlockRed {
+  static constexpr int NW = B / 32;
+  uint32_t* s;  // [2][NW]
+  int parity = 0;
+  __device__ uint32_t sum(uint32_t v) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) s[parity * NW + w] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) t += s[parity * NW + i];
+    parity ^= 1;
+    return t;
+  }
+  __device__ uint32_t min(uint32_t v) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    v = __reduce_min_sync(0xffffffffu, v);
+    if (lane == 0) s[parity * NW + w] = v;
+    __syncthreads();
+    uint32_t t = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) t = ::min(t, s[parity * NW + i]);
+    parity ^= 1;
+    return t;
+  }
+  __device__ uint32_t max(uint32_t v) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (lane == 0) s[parity * NW + w] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) t = ::max(t, s[parity * NW + i]);
+    parity ^= 1;
+    return t;
+  }
+  // exclusive prefix sum in thread order
+  __device__ uint32_t excl_scan(uint32_t v) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += o;
+    }
+    if (lane == 31) s[parity * NW + w] = inc;
+    __syncthreads();
+    uint32_t base = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i)
+      if (i < w) base += s[parity * NW + i];
+    parity ^= 1;
+    return base + inc - v;
+  }
+};
+
+// Where a group's selection goes.  The group's kept local channels S (an
+// ascending list of k entries; with pairs, kp pairs p giving channels p and
+// p + half, listed as all p then all p + half) are written as
+//   a[(g*rep + j) * k + i] = (g*rep + j) * N + S[i]   for j < rep,
+//   b[g * k + i]           = g * N + S[i]              (if b != null).
+struct TopkOut {
+  int32_t* a = nullptr;
+  int32_t* b = nullptr;
+  int rep = 1;
+  int N = 0;         // channels of one head (stride of the head offsets)
+  int pair_half = 0; // > 0: keys are rotate-half pairs (p, p + pair_half)
+};
+
+__device__ __forceinline__ void topk_emit(const TopkOut& o, int g, int ktot, int kp, int pos,
+                                          int c) {
+  for (int j = 0; j < o.rep; ++j) {
+    const int h = g * o.rep + j;
+    int32_t* row = o.a + int64_t(h) * ktot;
+    row[pos] = h * o.N + c;
+    if (o.pair_half) row[kp + pos] = h * o.N + c + o.pair_half;
+  }
+  if (o.b) {
+    int32_t* row = o.b + int64_t(g) * ktot;
+    row[pos] = g * o.N + c;
+    if (o.pair_half) row[kp + pos] = g * o.N + c + o.pair_half;
+  }
+}
+
+// The k largest of n scores (ties to the lower index), written through `o`
+// for group g.  All B threads of the block call it; n <= B * MAXM.  Scores
+// are read through L2 (they may come from other blocks of the same launch).
+template <int B, int MAXM>
+__device__ void block_topk(const float* __restrict__ sc, int n, int k, const TopkOut& o, int g,
+                           uint32_t* red_smem) {
+  BlockRed<B> red{red_smem};
+  const int tid = threadIdx.x;
+  const int kp = k;
+  const int ktot = o.pair_half ? 2 * k : k;
+  if (k <= 0 || n <= 0) return;
+  const int m = (n + B - 1) / B;
+  const int i0 = tid * m;
+  const int mt = ::max(0, ::min(m, n - i0));
+  if (k >= n) {  // everything is kept: own range in order
+    for (int i = 0; i < mt; ++i) topk_emit(o, g, ktot, kp, i0 + i, i0 + i);
+    return;
+  }
+  uint32_t key[MAXM];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < MAXM; ++i) {
+    key[i] = 0u;
+    if (i < mt) {
+      key[i] = score_key(__ldcg(sc + i0 + i));
+      kmin = ::min(kmin, key[i]);
+      kmax = ::max(kmax, key[i]);
+    }
+  }
+  kmin = red.min(kmin);
+  kmax = red.max(kmax);
+  // largest v with count(key >= v) >= k: count(>= lo) >= k > count(>= hi)
+  uint32_t lo = kmin, hi = kmax + 1u;
+  bool exact = false;
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + (hi - lo) / 2u;
+    uint32_t c = 0;
+#pragma unroll
+    for (int i = 0; i < MAXM; ++i) c += (i < mt && key[i] >= mid) ? 1u : 0u;
+    c = red.sum(c);
+    if (c == uint32_t(k)) {  // exactly the keys >= mid: no ties to break
+      lo = mid;
+      exact = true;
+      break;
+    }
+    if (c > uint32_t(k)) lo = mid; else hi = mid;
+  }
+  // keep every key above lo; of the keys equal to lo keep the first `want`
+  uint32_t cgt = 0, ceq = 0;
+#pragma unroll
+  for (int i = 0; i < MAXM; ++i) {
+    if (i < mt) {
+      if (exact ? key[i] >= lo : key[i] > lo) ++cgt;
+      else if (!exact && key[i] == lo) ++ceq;
+    }
+  }
+  const uint32_t want = exact ? 0u : uint32_t(k) - red.sum(cgt);
+  const uint32_t tie_before = red.excl_scan(ceq);
+  const uint32_t take_eq =
+      want > tie_before ? ::min(ceq, want - tie_before) : 0u;
+  int pos = int(red.excl_scan(cgt + take_eq));
+  uint32_t taken = 0;
+#pragma unroll
+  for (int i = 0; i < MAXM; ++i) {
+    if (i < mt) {
+      const uint32_t kv = key[i];
+      bool s;
+      if (exact) {
+        s = kv >= lo;
+      } else if (kv > lo) {
+        s = true;
+      } else if (kv == lo) {
+        s = taken < take_eq;
+        ++taken;
+      } else {
+        s = false;
+      }
+      if (s) topk_emit(o, g, ktot, kp, pos++, i0 + i);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- FFN score
-// Each thread scores CPT channels (c = first + 128 * i) over one token chunk:
-// it keeps their U_g, U_u rows in registers and reads each token's projected
-// row P_g | P_u from shared memory as 16-byte broadcasts, reused for its CPT
-// channels (the shared-memory reads, not the math, bounded the one-channel
-// version).  With an even CPT the rank-r dot products of two channels run as
-// one packed fma.rn.f32x2 per rank index (the token's projection is staged
-// duplicated, {v, v}); each lane's chain is the same fused multiply-adds in
-// the same order as the scalar form, so the scores are unchanged.  Partial
-// sums of squares per (chunk, channel), fixed token order.
-constexpr int kScoreTT = 32;  // tokens staged per round
-constexpr int kSMs148 = 148;  // B200 SM count (grid sizing only)
-template <int RP>
-constexpr int score_cpt() { return RP <= 8 ? 4 : (RP <= 16 ? 2 : 1); }
+// Six cross products of the three-term splits P = Ph + Pm + Pl and
+// U = Uh + Um + Ul carry the dot product to ~2^-23 relative: (h,h), (h,m),
+// (m,h), (h,l), (l,h), (m,m).  For rank chunk ch (8 rank indices) the product
+// list gives 6 "units" of K = 8; unit u = product u / C at chunk u % C, and
+// K16 block kb of the mma packs units 2 kb (k 0..7) and 2 kb + 1 (k 8..15).
+constexpr int pterm(int p) { return p == 2 ? 1 : (p == 4 ? 2 : (p == 5 ? 1 : 0)); }
+constexpr int uterm(int p) { return p == 1 ? 1 : (p == 3 ? 2 : (p == 5 ? 1 : 0)); }
 
-__device__ __forceinline__ unsigned long long pack_f2(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack_f2(unsigned long long v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
-// (a.lo * b.lo + c.lo, a.hi * b.hi + c.hi), each rounded once (fused)
-__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kStageTokens = 128;  // tokens staged per round (multiple of 16)
+// n8 tiles per warp for rank chunks C
+constexpr int score_nt(int C) { return C == 1 ? 2 : 1; }
+// 32-bit words per staged token: 2 matrices x 3 terms x 4C words, padded to
+// a stride = 4 (mod 8) words so the fragment loads of a warp are
+// bank-conflict free
+constexpr int score_tw(int C) { return 24 * C + 4; }
+constexpr int score_stage_bytes(int C) { return kStageTokens * score_tw(C) * 4; }
+constexpr int kFusedSelMaxM = 64;  // fused select: n <= 256 * 64 keys
 
-template <int RP>
-__global__ void __launch_bounds__(128) ffn_score_partial_kernel(
-    const float* __restrict__ P, int64_t ldp, const int32_t* __restrict__ pmap, int64_t T_C,
-    const float* __restrict__ Ug, const float* __restrict__ Uu, int64_t n, int r, int64_t chunk,
-    float* __restrict__ partial) {
-  constexpr int CPT = score_cpt<RP>();
-  const int64_t j0 = int64_t(blockIdx.x) * 128 * CPT + threadIdx.x;
-  const int64_t t0 = int64_t(blockIdx.y) * chunk;
-  const int64_t t1 = min(T_C, t0 + chunk);
-  float acc[CPT];
+struct ScoreArgs {
+  const float* P;        // [rows x ldp] fp32: P_g in columns [0, r), P_u in [r, 2r)
+  int64_t ldp;
+  const int32_t* pmap;   // context token t -> row of P (null: identity)
+  int64_t T_C;
+  const float* Ug;       // [n x r]
+  const float* Uu;
+  int64_t n;
+  int r;
+  int nsplit;
+  int64_t chunk;         // tokens per split (multiple of 16)
+  float* partial;        // [nsplit x n]
+  float* scores;         // [n]
+  unsigned* counters;    // [nblocks + 1], zero on entry
+  int select;            // run the top-k in the last block
+  int k;
+  int32_t* idx_out;
+};
+
+template <int C>
+__global__ void __launch_bounds__(kScoreThreads) ffn_score_select_kernel(const ScoreArgs a) {
+  constexpr int NT = score_nt(C), TW = score_tw(C), KB = 3 * C;
+  constexpr int CH = kScoreWarps * NT * 8;  // channels per block
+  extern __shared__ __align__(16) uint32_t s_stage[];
+  __shared__ uint32_t s_red[2 * kScoreWarps];
+  __shared__ unsigned s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int64_t cb = blockIdx.x;
+  const int sp = blockIdx.y;
+  const int r = a.r;
+
+  // B fragments: channel (tile base + g), rank indices 8 ch + 2t, +1
+  uint32_t bfr[NT][2][KB][2];
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) acc[i] = 0.0f;
-  auto uval = [&](const float* U, int i, int q) {
-    const int64_t j = j0 + 128 * i;
-    return (j < n && q < r) ? U[j * r + q] : 0.0f;
-  };
-  auto pval = [&](int64_t tb, int tt, int nt, int q) {
-    const int half = q / RP, qq = q % RP;
-    if (tt >= nt || qq >= r) return 0.0f;
-    const int64_t row = pmap ? int64_t(pmap[tb + tt]) : tb + tt;
-    return P[row * ldp + half * r + qq];
-  };
-  if constexpr (CPT % 2 == 0) {
-    constexpr int NPR = CPT / 2;  // channel pairs per thread
-    __shared__ __align__(16) unsigned long long sp2[kScoreTT][2 * RP];
-    unsigned long long ug2[NPR][RP], uu2[NPR][RP];
+  for (int nt = 0; nt < NT; ++nt) {
+    const int64_t j = cb * CH + (warp * NT + nt) * 8 + g;
 #pragma unroll
-    for (int pr = 0; pr < NPR; ++pr)
+    for (int mat = 0; mat < 2; ++mat) {
+      const float* U = mat == 0 ? a.Ug : a.Uu;
+      Split3 s0[C], s1[C];
 #pragma unroll
-      for (int q = 0; q < RP; ++q) {
-        ug2[pr][q] = pack_f2(uval(Ug, 2 * pr, q), uval(Ug, 2 * pr + 1, q));
-        uu2[pr][q] = pack_f2(uval(Uu, 2 * pr, q), uval(Uu, 2 * pr + 1, q));
+      for (int ch = 0; ch < C; ++ch) {
+        const int q = 8 * ch + 2 * t;
+        const float v0 = (j < a.n && q < r) ? U[j * r + q] : 0.0f;
+        const float v1 = (j < a.n && q + 1 < r) ? U[j * r + q + 1] : 0.0f;
+        s0[ch] = split3(v0);
+        s1[ch] = split3(v1);
       }
-    for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
-      const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
-      __syncthreads();
-      for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x) {
-        const int tt = e / (2 * RP), q = e % (2 * RP);
-        const float v = pval(tb, tt, nt, q);
-        sp2[tt][q] = pack_f2(v, v);
-      }
-      __syncthreads();
-      for (int tt = 0; tt < nt; ++tt) {
-        unsigned long long pg[RP], pu[RP];
 #pragma unroll
-        for (int q2 = 0; q2 < RP / 2; ++q2) {
-          const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(&sp2[tt][2 * q2]);
-          const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(&sp2[tt][RP + 2 * q2]);
-          pg[2 * q2] = a.x; pg[2 * q2 + 1] = a.y;
-          pu[2 * q2] = b.x; pu[2 * q2 + 1] = b.y;
+      for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int u = 2 * kb + half, term = uterm(u / C), ch = u % C;
+          bfr[nt][mat][kb][half] = pack2(s0[ch].t[term], s1[ch].t[term]);
         }
+      }
+    }
+  }
+
+  float acc[NT][2];
 #pragma unroll
-        for (int pr = 0; pr < NPR; ++pr) {
-          unsigned long long g2 = 0ull, u2 = 0ull;
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = 0.0f;
+
+  const int64_t t0 = int64_t(sp) * a.chunk;
+  const int64_t t1 = ::min(a.T_C, t0 + a.chunk);
+  for (int64_t tb = t0; tb < t1; tb += kStageTokens) {
+    const int ntok = int(::min(int64_t(kStageTokens), t1 - tb));
+    const int ntile = (ntok + 15) / 16;
+    __syncthreads();
+    // stage the split terms of the round's P rows: item = (token, matrix, word)
+    for (int e = tid; e < ntile * 16 * 8 * C; e += kScoreThreads) {
+      const int tt = e / (8 * C), rem = e % (8 * C), mat = rem / (4 * C), w = rem % (4 * C);
+      float v0 = 0.0f, v1 = 0.0f;
+      if (tt < ntok) {
+        const int64_t row = a.pmap ? int64_t(a.pmap[tb + tt]) : tb + tt;
+        const float* p = a.P + row * a.ldp + mat * r;
+        if (2 * w < r) v0 = p[2 * w];
+        if (2 * w + 1 < r) v1 = p[2 * w + 1];
+      }
+      const Split3 s0 = split3(v0), s1 = split3(v1);
+      uint32_t* dst = s_stage + tt * TW + mat * 12 * C + w;
 #pragma unroll
-          for (int q = 0; q < RP; ++q) {
-            g2 = ffma2(pg[q], ug2[pr][q], g2);
-            u2 = ffma2(pu[q], uu2[pr][q], u2);
+      for (int term = 0; term < 3; ++term) dst[term * 4 * C] = pack2(s0.t[term], s1.t[term]);
+    }
+    __syncthreads();
+    for (int tile = 0; tile < ntile; ++tile) {
+      const uint32_t* r0 = s_stage + (tile * 16 + g) * TW;
+      const uint32_t* r1 = r0 + 8 * TW;
+      // A fragment of K16 block kb of matrix mat: tokens g, g + 8; rank
+      // indices 8 ch + 2t, +1 of the two units the block packs
+      auto load_a = [&](int mat, int kb, uint32_t* f) {
+        const int u0 = 2 * kb, u1 = 2 * kb + 1;
+        const int o0 = mat * 12 * C + pterm(u0 / C) * 4 * C + 4 * (u0 % C) + t;
+        const int o1 = mat * 12 * C + pterm(u1 / C) * 4 * C + 4 * (u1 % C) + t;
+        f[0] = r0[o0];
+        f[1] = r1[o0];
+        f[2] = r0[o1];
+        f[3] = r1[o1];
+      };
+      auto epilogue = [&](const float* cg, const float* cu, float* ac) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = silu_f(cg[e]) * cu[e];
+          ac[e & 1] = fmaf(v, v, ac[e & 1]);
+        }
+      };
+      if constexpr (C <= 2) {  // fragments loaded once per tile, reused by the NT tiles
+        uint32_t afr[2][KB][4];
+#pragma unroll
+        for (int mat = 0; mat < 2; ++mat)
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb) load_a(mat, kb, afr[mat][kb]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float cg[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cu[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb) {
+            mma_bf16(cg, afr[0][kb], bfr[nt][0][kb][0], bfr[nt][0][kb][1]);
+            mma_bf16(cu, afr[1][kb], bfr[nt][1][kb][0], bfr[nt][1][kb][1]);
           }
-          const float2 g = unpack_f2(g2), u = unpack_f2(u2);
-          const float a0 = silu_f(g.x) * u.x, a1 = silu_f(g.y) * u.y;
-          acc[2 * pr] = fmaf(a0, a0, acc[2 * pr]);
-          acc[2 * pr + 1] = fmaf(a1, a1, acc[2 * pr + 1]);
+          epilogue(cg, cu, acc[nt]);
         }
-      }
-    }
-  } else {
-    __shared__ __align__(16) float sp[kScoreTT][2 * RP];
-    float ug[CPT][RP], uu[CPT][RP];
+      } else {  // large rank, one tile per warp: fragments loaded per K16 block
 #pragma unroll
-    for (int i = 0; i < CPT; ++i)
+        for (int nt = 0; nt < NT; ++nt) {
+          float cg[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cu[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int q = 0; q < RP; ++q) {
-        ug[i][q] = uval(Ug, i, q);
-        uu[i][q] = uval(Uu, i, q);
-      }
-    for (int64_t tb = t0; tb < t1; tb += kScoreTT) {
-      const int nt = int((t1 - tb) < kScoreTT ? (t1 - tb) : kScoreTT);
-      __syncthreads();
-      for (int e = threadIdx.x; e < kScoreTT * 2 * RP; e += blockDim.x)
-        sp[e / (2 * RP)][e % (2 * RP)] = pval(tb, e / (2 * RP), nt, e % (2 * RP));
-      __syncthreads();
-      for (int tt = 0; tt < nt; ++tt) {
-        float pg[RP], pu[RP];
-#pragma unroll
-        for (int q4 = 0; q4 < RP / 4; ++q4) {
-          const float4 a = *reinterpret_cast<const float4*>(&sp[tt][4 * q4]);
-          const float4 b = *reinterpret_cast<const float4*>(&sp[tt][RP + 4 * q4]);
-          pg[4 * q4] = a.x; pg[4 * q4 + 1] = a.y; pg[4 * q4 + 2] = a.z; pg[4 * q4 + 3] = a.w;
-          pu[4 * q4] = b.x; pu[4 * q4 + 1] = b.y; pu[4 * q4 + 2] = b.z; pu[4 * q4 + 3] = b.w;
-        }
-#pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-          float g = 0.0f, u = 0.0f;
-#pragma unroll
-          for (int q = 0; q < RP; ++q) {
-            g = fmaf(pg[q], ug[i][q], g);
-            u = fmaf(pu[q], uu[i][q], u);
+          for (int kb = 0; kb < KB; ++kb) {
+            uint32_t fa[4], fb[4];
+            load_a(0, kb, fa);
+            load_a(1, kb, fb);
+            mma_bf16(cg, fa, bfr[nt][0][kb][0], bfr[nt][0][kb][1]);
+            mma_bf16(cu, fb, bfr[nt][1][kb][0], bfr[nt][1][kb][1]);
           }
-          const float a = silu_f(g) * u;
-          acc[i] = fmaf(a, a, acc[i]);
+          epilogue(cg, cu, acc[nt]);
         }
       }
     }
   }
+  // sum over the 8 token rows (lanes with equal t), fixed order
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const int64_t j = j0 + 128 * i;
-    if (j < n) partial[int64_t(blockIdx.y) * n + j] = acc[i];
-  }
-}
-
-__global__ void sumsq_finalize_kernel(const float* __restrict__ partial, int nsplit, int64_t n,
-                                      float* __restrict__ scores) {
-  int64_t j = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= n) return;
-  double s = 0.0;
-  for (int p = 0; p < nsplit; ++p) s += double(partial[int64_t(p) * n + j]);
-  scores[j] = float(sqrt(s));
-}
-
-// ----------------------------------------------------------------- QK score
-// Gram partials: block (p, split) sums P_p[t,a] P_p[t,b] over its token chunk.
-__global__ void qk_gram_partial_kernel(const float* __restrict__ P, int64_t ldp,
-                                       const int32_t* __restrict__ pmap, int64_t T_C, int r,
-                                       int64_t chunk, double* __restrict__ part) {
-  const int p = blockIdx.x, sp = blockIdx.y, nsp = gridDim.y;
-  const int64_t t0 = int64_t(sp) * chunk, t1 = min(T_C, t0 + chunk);
-  for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
-    int a = e / r, b = e % r;
-    double s = 0.0;
-    for (int64_t t = t0; t < t1; ++t) {
-      const int64_t row = pmap ? int64_t(pmap[t]) : t;
-      s += double(P[row * ldp + p * r + a]) * double(P[row * ldp + p * r + b]);
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      float v = acc[nt][c];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[nt][c] = v;
     }
-    part[(int64_t(p) * nsp + sp) * r * r + e] = s;
+  if (g == 0) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int64_t j = cb * CH + (warp * NT + nt) * 8 + 2 * t;
+      float* dst = a.partial + int64_t(sp) * a.n + j;
+      if (j < a.n) dst[0] = acc[nt][0];
+      if (j + 1 < a.n) dst[1] = acc[nt][1];
+    }
   }
-}
-
-__global__ void qk_gram_finalize_kernel(const double* __restrict__ part, int nsp, int r,
-                                        double* __restrict__ gram) {
-  const int p = blockIdx.x;
-  for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
+  // the last split of this channel block sums the partials in split order
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[cb], 1u) + 1u == unsigned(a.nsplit)) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int c = tid; c < CH; c += kScoreThreads) {
+    const int64_t j = cb * CH + c;
+    if (j >= a.n) break;
     double s = 0.0;
-    for (int sp = 0; sp < nsp; ++sp) s += part[(int64_t(p) * nsp + sp) * r * r + e];
-    gram[int64_t(p) * r * r + e] = s;
+    for (int p = 0; p < a.nsplit; ++p) s += double(__ldcg(a.partial + int64_t(p) * a.n + j));
+    a.scores[j] = float(sqrt(s));
+  }
+  if (!a.select) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[gridDim.x], 1u) + 1u == gridDim.x) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  TopkOut o;
+  o.a = a.idx_out;
+  o.N = int(a.n);
+  block_topk<kScoreThreads, kFusedSelMaxM>(a.scores, int(a.n), a.k, o, 0, s_red);
+}
+
+// ------------------------------------------------------------ Gram criterion
+constexpr int kGramThreads = 256;
+constexpr int kGramTokens = 64;  // P rows staged per round
+
+struct GramArgs {
+  const float* P;
+  int64_t ldp;
+  const int32_t* pmap;
+  int64_t T_C;
+  int r;
+  int nmat;        // 1 or 2 matrices: columns [m r, (m + 1) r)
+  int64_t chunk;   // tokens per block
+  double* part;    // [gridDim.x x nmat x r x r]
+  double* gram;    // [nmat x r x r]
+  unsigned* counter;
+};
+
+__global__ void __launch_bounds__(kGramThreads) gram_partial_kernel(const GramArgs a) {
+  __shared__ float sp[kGramTokens][2 * 48 + 1];
+  __shared__ unsigned s_last;
+  const int tid = threadIdx.x, r = a.r, ne = a.nmat * r * r;
+  const int64_t t0 = int64_t(blockIdx.x) * a.chunk, t1 = ::min(a.T_C, t0 + a.chunk);
+  double acc[(2 * 48 * 48 + kGramThreads - 1) / kGramThreads];
+  constexpr int NE = (2 * 48 * 48 + kGramThreads - 1) / kGramThreads;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) acc[i] = 0.0;
+  const int w = a.nmat * r;
+  for (int64_t tb = t0; tb < t1; tb += kGramTokens) {
+    const int nt = int(::min(int64_t(kGramTokens), t1 - tb));
+    __syncthreads();
+    for (int e = tid; e < nt * w; e += kGramThreads) {
+      const int tt = e / w, q = e % w;
+      const int64_t row = a.pmap ? int64_t(a.pmap[tb + tt]) : tb + tt;
+      sp[tt][q] = a.P[row * a.ldp + q];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+      const int e = tid + i * kGramThreads;
+      if (e < ne) {
+        const int m = e / (r * r), x = (e / r) % r, y = e % r;
+        double s = acc[i];
+        for (int tt = 0; tt < nt; ++tt)
+          s = fma(double(sp[tt][m * r + x]), double(sp[tt][m * r + y]), s);
+        acc[i] = s;
+      }
+    }
+  }
+  double* mine = a.part + int64_t(blockIdx.x) * ne;
+#pragma unroll
+  for (int i = 0; i < NE; ++i) {
+    const int e = tid + i * kGramThreads;
+    if (e < ne) mine[e] = acc[i];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(a.counter, 1u) + 1u == gridDim.x) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = tid; e < ne; e += kGramThreads) {
+    double s = 0.0;
+    for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(a.part + int64_t(b) * ne + e);
+    a.gram[e] = s;
   }
 }
 
-__device__ double quad_form(const double* G, const float* u, int r) {
+constexpr int kNormThreads = 256;
+
+struct NormArgs {
+  const double* gram;   // [nmat x r x r]
+  const float* U0;      // QK: U_q [heads*N x r]; L2: U [groups*N x r]
+  const float* U1;      // QK: U_k [kv*N x r]
+  int r;
+  int mode;             // kCritModeQK, kCritModeL2
+  int pair_half;        // > 0: score rotate-half pairs (c, c + half), half = N / 2
+  int N;                // channels per head
+  int rep;              // query heads per group (QK)
+  int nkeys;            // keys per group: N, or N / 2 with pairs
+  int blocks_per_group;
+  float* scores;        // [groups x nkeys]
+  unsigned* counters;   // [groups], zero on entry
+  int k;                // keys kept per group
+  TopkOut out;
+};
+
+__device__ __forceinline__ double quad_form(const double* G, const float* u, int r) {
   double s = 0.0;
-  for (int a = 0; a < r; ++a) {
-    double ga = 0.0;
-    for (int b = 0; b < r; ++b) ga += G[a * r + b] * double(u[b]);
-    s += double(u[a]) * ga;
+  for (int x = 0; x < r; ++x) {
+    double gx = 0.0;
+    for (int y = 0; y < r; ++y) gx = fma(G[x * r + y], double(u[y]), gx);
+    s = fma(double(u[x]), gx, s);
   }
   return s > 0.0 ? s : 0.0;
 }
 
-__global__ void qk_score_kernel(const double* __restrict__ gram, const float* __restrict__ Uq,
-                                const float* __restrict__ Uk, int r, int heads, int kv_heads,
-                                int head_dim, float* __restrict__ scores) {
-  int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (e >= int64_t(kv_heads) * head_dim) return;
-  const int g = int(e / head_dim), c = int(e % head_dim);
-  const int rep = heads / kv_heads;
-  const double* Gq = gram;
-  const double* Gk = gram + r * r;
-  double qs = 0.0;
-  for (int j = 0; j < rep; ++j) {
-    int h = g * rep + j;
-    qs += sqrt(quad_form(Gq, Uq + (int64_t(h) * head_dim + c) * r, r));
-  }
-  double nk = sqrt(quad_form(Gk, Uk + (int64_t(g) * head_dim + c) * r, r));
-  scores[e] = float(nk * qs);
-}
-
-// ----------------------------------------------------------------- select
-// Radix select on the fp32 bit pattern (scores are >= 0, so unsigned order of
-// the bits is numeric order), 4 passes of 8 bits, then an index-ordered
-// compaction with ballot scans so the output is ascending and equal scores
-// go to the lower index.
-__device__ __forceinline__ uint32_t score_key(float v) {
-  uint32_t b = __float_as_uint(v);
-  if (b & 0x80000000u) b = 0;   // -0 (or a negative) ranks as zero
-  if (b > 0x7f800000u) b = 0;   // NaN ranks lowest
-  return b;
-}
-
-__global__ void __launch_bounds__(1024) topk_select_kernel(const float* __restrict__ scores,
-                                                           int N, int k, int rep,
-                                                           int32_t* __restrict__ out_a,
-                                                           int32_t* __restrict__ out_b) {
-  const int g = blockIdx.x;
-  const float* sc = scores + int64_t(g) * N;
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_prefix, s_want;
-  __shared__ uint32_t warp_sel[32], warp_eq[32];
-  __shared__ uint32_t s_base, s_tie;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
-  if (k <= 0) return;
-  if (tid == 0) { s_prefix = 0; s_want = uint32_t(k); }
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (32 - 8 * pass));
-    for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix;
-    for (int j = tid; j < N; j += blockDim.x) {
-      uint32_t key = score_key(sc[j]);
-      if ((key & hi_mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (wid == 0) {  // the digit holding the want-th largest key: a warp-parallel scan
-      // lane l owns digits 255 - 8l down to 248 - 8l (descending key order)
-      const uint32_t want = s_want;
-      uint32_t own = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) own += hist[255 - 8 * lane - i];
-      uint32_t incl = own;  // inclusive prefix over lanes 0..l
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= want);
-      const int l = __ffs(hit) - 1;  // want <= count of keys with this prefix, so l exists
-      if (lane == l) {
-        uint32_t cum = incl - own;
-        for (int i = 0; i < 8; ++i) {
-          const int dg = 255 - 8 * lane - i;
-          const uint32_t h = hist[dg];
-          if (cum + h >= want) {
-            s_prefix = prefix | (uint32_t(dg) << shift);
-            s_want = want - cum;
-            break;
-          }
-          cum += h;
-        }
-      }
-    }
-    __syncthreads();
-  }
-  const uint32_t tau = s_prefix, want = s_want;  // take `want` of the keys equal to tau
-  if (tid == 0) { s_base = 0; s_tie = 0; }
+template <int MAXM>
+__global__ void __launch_bounds__(kNormThreads) norm_score_select_kernel(const NormArgs a) {
+  __shared__ double sg[2 * 48 * 48];
+  __shared__ uint32_t s_red[2 * (kNormThreads / 32)];
+  __shared__ unsigned s_last;
+  const int tid = threadIdx.x, r = a.r;
+  const int nmat = a.mode == kCritModeQK ? 2 : 1;
+  for (int e = tid; e < nmat * r * r; e += kNormThreads) sg[e] = a.gram[e];
   __syncthreads();
-  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
-    const int j = c0 + tid;
-    uint32_t key = j < N ? score_key(sc[j]) : 0u;
-    const bool gt = j < N && key > tau;
-    const bool eq = j < N && key == tau;
-    // exclusive rank of this lane among the block's ties
-    uint32_t beq = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) warp_eq[wid] = __popc(beq);
-    __syncthreads();
-    uint32_t tie_before = s_tie;
-    for (int w = 0; w < wid; ++w) tie_before += warp_eq[w];
-    tie_before += __popc(beq & ((1u << lane) - 1u));
-    const bool sel = gt || (eq && tie_before < want);
-    uint32_t bsel = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) warp_sel[wid] = __popc(bsel);
-    __syncthreads();
-    uint32_t pos = s_base;
-    for (int w = 0; w < wid; ++w) pos += warp_sel[w];
-    pos += __popc(bsel & ((1u << lane) - 1u));
-    if (sel) {
-      for (int q = 0; q < rep; ++q) {
-        const int h = g * rep + q;
-        out_a[int64_t(h) * k + pos] = h * N + j;
-      }
-      if (out_b) out_b[int64_t(g) * k + pos] = g * N + j;
+  const int grp = blockIdx.y;
+  const int key = blockIdx.x * kNormThreads + tid;
+  if (key < a.nkeys) {
+    // norm^2 of channel c of head h of matrix m
+    auto nsq = [&](int m, int h, int c) {
+      const float* U = m == 0 ? a.U0 : a.U1;
+      return quad_form(sg + m * r * r, U + (int64_t(h) * a.N + c) * r, r);
+    };
+    auto nrm = [&](int m, int h) {
+      double s = nsq(m, h, key);
+      if (a.pair_half) s += nsq(m, h, key + a.pair_half);
+      return sqrt(s);
+    };
+    double score;
+    if (a.mode == kCritModeQK) {
+      double qs = 0.0;
+      for (int j = 0; j < a.rep; ++j) qs += nrm(0, grp * a.rep + j);
+      score = nrm(1, grp) * qs;
+    } else {
+      score = nrm(0, grp);
     }
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t ts = 0, te = 0;
-      for (int w = 0; w < nw; ++w) { ts += warp_sel[w]; te += warp_eq[w]; }
-      s_base += ts;
-      s_tie += te;
-    }
-    __syncthreads();
+    a.scores[int64_t(grp) * a.nkeys + key] = float(score);
   }
+  if (a.k <= 0) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0)
+    s_last = (atomicAdd(&a.counters[grp], 1u) + 1u == unsigned(a.blocks_per_group)) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  block_topk<kNormThreads, MAXM>(a.scores + int64_t(grp) * a.nkeys, a.nkeys, a.k, a.out, grp,
+                                 s_red);
+}
+
+// ------------------------------------------------------ standalone top-k
+constexpr int kTopkThreads = 512;
+constexpr int kTopkMaxM = 64;
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores,
+                                                            int N, int k, TopkOut o) {
+  __shared__ uint32_t s_red[2 * (kTopkThreads / 32)];
+  block_topk<kTopkThreads, kTopkMaxM>(scores + int64_t(blockIdx.x) * N, N, k, o, blockIdx.x,
+                                      s_red);
+}
+
+int rank_chunks(int r) { return r <= 8 ? 1 : (r <= 16 ? 2 : (r <= 24 ? 3 : (r <= 32 ? 4 : 6))); }
+int channels_per_block(int r) { return kScoreWarps * score_nt(rank_chunks(r)) * 8; }
+
+template <int C>
+int score_blocks_per_sm_t() {
+  static int cached = 0;
+  if (!cached) {
+    int b = 0;
+    const int smem = score_stage_bytes(C);
+    if (cudaFuncSetAttribute(ffn_score_select_kernel<C>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_select_kernel<C>,
+                                                      kScoreThreads, smem) != cudaSuccess ||
+        b < 1) {
+      cudaGetLastError();
+      b = 1;
+    }
+    cached = b;
+  }
+  return cached;
+}
+int score_blocks_per_sm(int r) {
+  switch (rank_chunks(r)) {
+    case 1: return score_blocks_per_sm_t<1>();
+    case 2: return score_blocks_per_sm_t<2>();
+    case 3: return score_blocks_per_sm_t<3>();
+    case 4: return score_blocks_per_sm_t<4>();
+    default: return score_blocks_per_sm_t<6>();
+  }
+}
+
+template <int C>
+void launch_score(dim3 grid, const ScoreArgs& a, cudaStream_t st) {
+  score_blocks_per_sm_t<C>();  // sets the kernel's dynamic shared-memory limit once
+  const int smem = score_stage_bytes(C);
+  ffn_score_select_kernel<C><<<grid, kScoreThreads, smem, st>>>(a);
 }
 
 }  // namespace
 
-int score_cpt_for(int r) { return r <= 8 ? 4 : (r <= 16 ? 2 : 1); }
-
-// Resident 128-thread score blocks per SM for the kernel serving rank r
-// (register-limited; 4 if the query fails).
-int score_blocks_per_sm(int r) {
-  static int cached[4] = {0, 0, 0, 0};
-  const int slot = r <= 8 ? 0 : (r <= 16 ? 1 : (r <= 32 ? 2 : 3));
-  if (!cached[slot]) {
-    int b = 0;
-    cudaError_t e;
-    switch (slot) {
-      case 0: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<8>, 128, 0); break;
-      case 1: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<16>, 128, 0); break;
-      case 2: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<32>, 128, 0); break;
-      default: e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_partial_kernel<48>, 128, 0); break;
-    }
-    if (e != cudaSuccess || b < 1) {
-      cudaGetLastError();
-      b = 4;
-    }
-    cached[slot] = b;
-  }
-  return cached[slot];
+int64_t ffn_score_blocks(int64_t n, int r) {
+  const int ch = channels_per_block(r);
+  return (n + ch - 1) / ch;
 }
 
-// Token splits: as many as keep the grid within one wave of resident blocks
-// (a second, partial wave cost more than the split's extra partial sums).
+// Token splits: as many as keep the grid within one wave of resident blocks.
 int ffn_score_splits(int64_t T_C, int64_t n, int r) {
-  const int64_t nb = (n + 128 * score_cpt_for(r) - 1) / (128 * score_cpt_for(r));
-  const int64_t slots = int64_t(kSMs148) * score_blocks_per_sm(r);
+  const int64_t nb = ffn_score_blocks(n, r);
+  const int64_t slots = int64_t(num_sms()) * score_blocks_per_sm(r);
   int64_t want = slots / std::max<int64_t>(nb, 1);
-  int64_t maxs = (T_C + kScoreTT - 1) / kScoreTT;
-  int64_t s = want < maxs ? want : maxs;
+  const int64_t maxs = std::max<int64_t>((T_C + 15) / 16, 1);
+  int64_t s = std::min(want, maxs);
   if (s < 1) s = 1;
-  if (s > 64) s = 64;
+  if (s > 256) s = 256;
   return int(s);
 }
 
-slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
-                        const float* Ug, const float* Uu, int64_t n, int r, float* partial,
-                        int nsplit, float* scores, cudaStream_t st) {
+int64_t estimator_counter_count(int64_t n, int r, int groups) {
+  return ffn_score_blocks(n, r) + 1 + std::max(groups, 1) + 1;
+}
+
+int64_t gram_blocks(int64_t T_C) {
+  const int64_t want = (T_C + kGramTokens - 1) / kGramTokens;
+  return std::max<int64_t>(1, std::min<int64_t>(want, 64));
+}
+
+slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                              const float* Ug, const float* Uu, int64_t n, int r, float* partial,
+                              int nsplit, float* scores, unsigned* counters, int k,
+                              int32_t* idx_out, cudaStream_t st) {
   if (n <= 0) return SLORA_OK;
-  const int64_t chunk = T_C > 0 ? (T_C + nsplit - 1) / nsplit : 1;
-  dim3 grid(unsigned((n + 128 * score_cpt_for(r) - 1) / (128 * score_cpt_for(r))),
-            unsigned(nsplit));
+  const bool fused_select = n <= int64_t(kScoreThreads) * kFusedSelMaxM && idx_out;
+  ScoreArgs a;
+  a.P = P; a.ldp = ldp; a.pmap = pmap; a.T_C = T_C; a.Ug = Ug; a.Uu = Uu; a.n = n; a.r = r;
+  a.nsplit = nsplit;
+  a.chunk = T_C > 0 ? ((T_C + nsplit - 1) / nsplit + 15) / 16 * 16 : 16;
+  a.partial = partial; a.scores = scores; a.counters = counters;
+  a.select = fused_select ? 1 : 0;
+  a.k = k; a.idx_out = idx_out;
+  const dim3 grid(unsigned(ffn_score_blocks(n, r)), unsigned(nsplit));
   {
-  LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 + double(nsplit) * n * 4, st);
-  if (r <= 8)
-    ffn_score_partial_kernel<8><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
-                                                         partial);
-  else if (r <= 16)
-    ffn_score_partial_kernel<16><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
-                                                         partial);
-  else if (r <= 32)
-    ffn_score_partial_kernel<32><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
-                                                         partial);
-  else
-    ffn_score_partial_kernel<48><<<grid, 128, 0, st>>>(P, ldp, pmap, T_C, Ug, Uu, n, r, chunk,
-                                                         partial);
+    // bytes: P rows of the context tokens, both factors, partials and scores
+    LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 +
+                                  double(nsplit) * n * 8 + double(n) * 4, st);
+    switch (rank_chunks(r)) {
+      case 1: launch_score<1>(grid, a, st); break;
+      case 2: launch_score<2>(grid, a, st); break;
+      case 3: launch_score<3>(grid, a, st); break;
+      case 4: launch_score<4>(grid, a, st); break;
+      default: launch_score<6>(grid, a, st); break;
+    }
   }
   SLORA_CHECK_LAUNCH();
-  LaunchScope ls2(kEstimate, double(nsplit) * n * 4 + double(n) * 4, st);
-  sumsq_finalize_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(partial, nsplit, n, scores);
-  SLORA_CHECK_LAUNCH();
+  if (!fused_select && idx_out) SLORA_TRY(topk_select(scores, 1, int(n), k, 1, idx_out, nullptr, st));
   return SLORA_OK;
 }
 
-slora_status qk_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
-                       const float* Uq,
-                       const float* Uk, int r, int heads, int kv_heads, int head_dim,
-                       double* gram, float* scores, cudaStream_t st) {
-  constexpr int kSplits = 32;
-  double* part = gram + 2 * r * r;  // caller reserves 2*r*r*(1 + kSplits) doubles
-  const int64_t chunk = T_C > 0 ? (T_C + kSplits - 1) / kSplits : 1;
+slora_status gram_scores_select(int mode, const float* P, int64_t ldp, const int32_t* pmap,
+                                int64_t T_C, const float* U0, const float* U1, int r, int groups,
+                                int rep, int N, bool pairs, int k, double* gram_part,
+                                double* gram, float* scores, unsigned* counters, int32_t* out_a,
+                                int32_t* out_b, cudaStream_t st) {
+  const int nmat = mode == kCritModeQK ? 2 : 1;
+  GramArgs ga;
+  ga.P = P; ga.ldp = ldp; ga.pmap = pmap; ga.T_C = T_C; ga.r = r; ga.nmat = nmat;
+  const int64_t nb = gram_blocks(T_C);
+  ga.chunk = T_C > 0 ? (T_C + nb - 1) / nb : 1;
+  ga.part = gram_part; ga.gram = gram; ga.counter = counters;
   {
-  LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4, st);
-  qk_gram_partial_kernel<<<dim3(2, kSplits), 256, 0, st>>>(P, ldp, pmap, T_C, r, chunk, part);
-  SLORA_CHECK_LAUNCH();
+    LaunchScope ls(kEstimate, double(T_C) * nmat * r * 4 + double(nb) * nmat * r * r * 8, st);
+    gram_partial_kernel<<<unsigned(nb), kGramThreads, 0, st>>>(ga);
   }
   SLORA_CHECK_LAUNCH();
+  NormArgs na;
+  na.gram = gram; na.U0 = U0; na.U1 = U1; na.r = r; na.mode = mode;
+  na.pair_half = pairs ? N / 2 : 0;
+  na.N = N; na.rep = rep;
+  na.nkeys = pairs ? N / 2 : N;
+  na.blocks_per_group = (na.nkeys + kNormThreads - 1) / kNormThreads;
+  na.scores = scores; na.counters = counters + 1;
+  na.out.a = out_a; na.out.b = out_b; na.out.rep = rep; na.out.N = N;
+  na.out.pair_half = na.pair_half;
+  const bool fused_select = na.nkeys <= kNormThreads * kFusedSelMaxM && out_a;
+  na.k = fused_select ? k : 0;
+  const dim3 grid(unsigned(na.blocks_per_group), unsigned(groups));
   {
-  LaunchScope ls(kEstimate, double(kSplits) * 2 * r * r * 8, st);
-  qk_gram_finalize_kernel<<<2, 256, 0, st>>>(part, kSplits, r, gram);
+    const int nu = mode == kCritModeQK ? (rep + 1) : 1;
+    LaunchScope ls(kSelect, double(groups) * N * nu * r * 4 + double(groups) * na.nkeys * 4 +
+                                double(groups) * k * 4 * (rep + 1) * (pairs ? 2 : 1), st);
+    if (na.nkeys <= kNormThreads)
+      norm_score_select_kernel<1><<<grid, kNormThreads, 0, st>>>(na);
+    else
+      norm_score_select_kernel<kFusedSelMaxM><<<grid, kNormThreads, 0, st>>>(na);
   }
   SLORA_CHECK_LAUNCH();
-  const int64_t nsc = int64_t(kv_heads) * head_dim;
-  LaunchScope ls(kEstimate, double(heads + kv_heads) * head_dim * r * 4 + double(nsc) * 4, st);
-  qk_score_kernel<<<unsigned((nsc + 127) / 128), 128, 0, st>>>(gram, Uq, Uk, r, heads, kv_heads,
-                                                                head_dim, scores);
-  SLORA_CHECK_LAUNCH();
+  if (!fused_select && out_a) {
+    TopkOut o = na.out;
+    LaunchScope ls(kSelect, double(groups) * na.nkeys * 4, st);
+    topk_kernel<<<unsigned(groups), kTopkThreads, 0, st>>>(scores, na.nkeys, k, o);
+    SLORA_CHECK_LAUNCH();
+  }
   return SLORA_OK;
 }
 
 slora_status topk_select(const float* scores, int groups, int N, int k, int rep,
                          int32_t* out_a, int32_t* out_b, cudaStream_t st) {
   if (k <= 0 || groups <= 0) return SLORA_OK;
-  LaunchScope ls(kSelect, double(groups) * N * 4 * 5 + double(groups) * k * 4 * (rep + 1), st);
-  topk_select_kernel<<<groups, 1024, 0, st>>>(scores, N, k, rep, out_a, out_b);
+  if (int64_t(N) > int64_t(kTopkThreads) * kTopkMaxM)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "top-k over %d keys per group exceeds the supported %d", N,
+               kTopkThreads * kTopkMaxM);
+  TopkOut o;
+  o.a = out_a; o.b = out_b; o.rep = rep; o.N = N;
+  LaunchScope ls(kSelect, double(groups) * N * 4 + double(groups) * k * 4 * (rep + 1), st);
+  topk_kernel<<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
+
+int64_t topk_max_keys() { return int64_t(kTopkThreads) * kTopkMaxM; }
 
 }  // namespace slora

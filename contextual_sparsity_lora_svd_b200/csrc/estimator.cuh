@@ -5,28 +5,53 @@
 
 namespace slora {
 
-// FFN: sumsq partials over token chunks of (silu(P_g U_g^T) * (P_u U_u^T))^2,
-// then a fixed-order reduction and sqrt into scores[n].
-//   P [T_C x ldp] fp32 with P_g in columns [0, r) and P_u in [r, 2r).
-// P rows are read through pmap when given (row t of the context set is P[pmap[t]]).
-slora_status ffn_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
-                        const float* Ug, const float* Uu, int64_t n, int r, float* partial,
-                        int nsplit, float* scores, cudaStream_t st);
-int ffn_score_splits(int64_t T_C, int64_t n, int r);
-
-// QK: Gram matrices of P_q (cols [0,r)) and P_k (cols [r,2r)) in fp64, then
-// score[g, c] = ||K_hat[:, g, c]|| * sum_{h in g} ||Q_hat[:, h, c]||.
-slora_status qk_scores(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
-                       const float* Uq,
-                       const float* Uk, int r, int heads, int kv_heads, int head_dim,
-                       double* gram /* [2 r r] */, float* scores, cudaStream_t st);
-
-// Top-k per group: scores [groups x N] -> for each group its k best channels
-// (ties to the lower index) in ascending order.  The selected local channel
-// set S_g of group g is written as
+// Top-k outputs of a group (one key head and its `rep` query heads, or one
+// whole score vector): the kept local channels S_g, ascending, are written as
 //   out_a[(g*rep + j) * k + i] = (g*rep + j) * N + S_g[i]   for j < rep,
 //   out_b[g * k + i]           = g * N + S_g[i]              (if out_b != null).
+// Equal scores go to the lower index.
+
+// FFN activation-norm score and selection in one launch:
+//   scores[j] = sqrt(sum_t (silu(P_g[t] . U_g[j]) * (P_u[t] . U_u[j]))^2),
+//   P [rows x ldp] fp32 with P_g in columns [0, r), P_u in [r, 2r), context
+//   token t at row pmap[t] (identity when pmap is null);
+//   idx_out[0..k) = the k best channels (when idx_out != null).
+// partial: [nsplit x n] floats; counters: estimator_counter_count(n, r, 1)
+// unsigned ints, zero on entry.
+slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
+                              const float* Ug, const float* Uu, int64_t n, int r, float* partial,
+                              int nsplit, float* scores, unsigned* counters, int k,
+                              int32_t* idx_out, cudaStream_t st);
+int ffn_score_splits(int64_t T_C, int64_t n, int r);
+
+// Gram-form criteria.  G_m = P_m^T P_m (fp64) for the P matrices in columns
+// [m r, (m+1) r) of P; a channel's estimated norm is sqrt(u^T G_m u) for its
+// factor row u.
+//   mode 0 (QK-norm): group g scores channel c as
+//        ||K_hat[:, g, c]|| * sum_{j < rep} ||Q_hat[:, g*rep + j, c]||
+//        with Q from (P_0, U0) and K from (P_1, U1);
+//   mode 1 (L2 norm): group g scores channel c as ||Y_hat[:, g, c]|| from (P_0, U0)
+//        (its set still goes to the group's `rep` heads of out_a).
+// With `pairs`, the keys are the N/2 rotate-half pairs (c, c + N/2), each
+// norm taken over both channels of the pair; k is then the number of pairs
+// kept and each head keeps 2k channels (all pair firsts, then all seconds).
+// gram_part: gram_blocks(T_C) * nmat * r * r doubles; gram: nmat * r * r;
+// scores: groups * nkeys floats; counters: 1 + groups, zero on entry.
+constexpr int kCritModeQK = 0, kCritModeL2 = 1;
+slora_status gram_scores_select(int mode, const float* P, int64_t ldp, const int32_t* pmap,
+                                int64_t T_C, const float* U0, const float* U1, int r, int groups,
+                                int rep, int N, bool pairs, int k, double* gram_part,
+                                double* gram, float* scores, unsigned* counters, int32_t* out_a,
+                                int32_t* out_b, cudaStream_t st);
+int64_t gram_blocks(int64_t T_C);
+
+// Counters (zero on entry) the estimator kernels of one call need.
+int64_t estimator_counter_count(int64_t n, int r, int groups);
+
+// Top-k per group over scores [groups x N] (see the layout above).  N at most
+// topk_max_keys().
 slora_status topk_select(const float* scores, int groups, int N, int k, int rep,
                          int32_t* out_a, int32_t* out_b, cudaStream_t st);
+int64_t topk_max_keys();
 
 }  // namespace slora

@@ -34,6 +34,7 @@ struct FfnDesc {
   slora_ffn_layer L;
   slora_ffn_grads G;
   int64_t kkeep;
+  double sparsity;  // ratio the estimator selects at (unused with idx_force)
 };
 
 slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
@@ -50,21 +51,38 @@ struct EstBufs {
   void* prs = nullptr;       // bf16 terms of [L0 | L1] for that projection (bf16 path)
   float* scores = nullptr;   // per-channel scores (the caller's scores_out when given)
   float* partial = nullptr;  // FFN score partials over token chunks
-  double* gram = nullptr;    // q/k Gram matrices and their partials
+  double* gram = nullptr;    // Gram matrices of the projection
+  double* gram_part = nullptr;  // their partials over token chunks
+  unsigned* cnt = nullptr;   // arrival counters of the estimator kernels, zero on entry
+  int64_t ncnt = 0;
   int nsplit = 1;
 };
+// Layout of one criterion's scores and selection.
+struct CritPlan {
+  bool activation = false;  // SwiGLU activation norm (tensor-core score kernel)
+  int mode = 0;             // Gram-form criteria: kCritModeQK or kCritModeL2
+  int nmat = 2;             // projected matrices (columns of P: nmat * rank)
+  int groups = 1, rep = 1, N = 0, nkeys = 0;
+  bool pairs = false;
+  int64_t kkeep = 0;        // keys kept per group (pairs with `pairs`)
+  int64_t per_head = 0;     // channels kept per head (2 kkeep with pairs)
+};
+CritPlan crit_plan(slora_criterion crit, int64_t n0, int heads, int kv_heads, int head_dim,
+                   double sparsity);
 EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int64_t d, int64_t n0,
-                         int rank, int kv_heads, int head_dim, bool has_pre, float* scores_out,
-                         Arena& ar);
+                         int rank, int heads, int kv_heads, int head_dim, bool has_pre,
+                         float* scores_out, Arena& ar);
 // With has_pre the low-rank projection of the context rows is already
 // available (full row layout, row t of the context set at P_pre[ctx_rows[t]]).
+// sk_counters: zeroed counters of the projection stream (bf16 path without
+// has_pre); eb.cnt must have been zeroed too (launch_rowmaps).
 slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
                                     const TokenInfo& ti, const int32_t* ctx_rows, int64_t d,
                                     const float* L0, const float* U0, int64_t n0, const float* L1,
                                     const float* U1, int rank, int heads, int kv_heads,
-                                    int head_dim, int64_t kkeep, int32_t* idx_out,
+                                    int head_dim, double sparsity, int32_t* idx_out,
                                     const EstBufs& eb, cudaStream_t st, bool has_pre = false,
                                     const float* P_pre = nullptr, int64_t ldp_pre = 0,
-                                    unsigned* counters = nullptr);
+                                    unsigned* sk_counters = nullptr);
 
 }  // namespace slora

@@ -26,8 +26,11 @@ __global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
                                                       int4* __restrict__ ctx_tiles,
                                                       int4* __restrict__ out_tiles,
                                                       unsigned* __restrict__ zero,
-                                                      int64_t nzero) {
+                                                      int64_t nzero,
+                                                      unsigned* __restrict__ zero2,
+                                                      int64_t nzero2) {
   for (int64_t i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
+  for (int64_t i = threadIdx.x; i < nzero2; i += blockDim.x) zero2[i] = 0u;
   __shared__ int ctx_off[kMaxBatch], ct_off[kMaxBatch], ot_off[kMaxBatch];
   if (threadIdx.x == 0) {
     int acc = 0, ct = 0, ot = 0;
@@ -97,6 +100,20 @@ slora_status check_device() {
     SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
                dev, major, minor);
   return SLORA_OK;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      v = 148;
+    }
+    n = v;
+  }
+  return n;
 }
 
 slora_status parse_tokens(const slora_tokens* tok, TokenInfo* ti) {
@@ -185,14 +202,15 @@ slora_status join_side(cudaStream_t st, cudaStream_t side) {
 
 slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_t* ctx_rows,
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles,
-                            int4* out_tiles, unsigned* zero, int64_t nzero) {
+                            int4* out_tiles, unsigned* zero, int64_t nzero, unsigned* zero2,
+                            int64_t nzero2) {
   RowmapParams p;
   p.batch = ti.batch;
   p.seq = ti.seq;
   for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
   LaunchScope ls(kAux, double(ti.T) * 4, st);
   rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles, zero,
-                                    zero ? nzero : 0);
+                                    zero ? nzero : 0, zero2, zero2 ? nzero2 : 0);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }

@@ -71,8 +71,11 @@ typedef enum {
 typedef enum { SLORA_F32 = 0, SLORA_BF16 = 1 } slora_dtype;
 
 typedef enum {
-  SLORA_CRIT_FFN_SWIGLU_L2 = 0, /* SwiGLU FFN: L2 norm of the estimated activation */
-  SLORA_CRIT_QK_NORM = 1        /* attention q/k: QK-norm, top-k per head group     */
+  SLORA_CRIT_FFN_SWIGLU_L2 = 0, /* SwiGLU FFN: L2 norm of the estimated activation        */
+  SLORA_CRIT_QK_NORM = 1,       /* attention q/k: QK-norm, top-k per head group            */
+  SLORA_CRIT_FFN_GRAM = 2,      /* SwiGLU FFN variant: ||g_hat_j|| * ||u_hat_j||             */
+  SLORA_CRIT_QK_ROPE_PAIR = 3,  /* q/k QK-norm over rotate-half pairs (c, c + head_dim/2) */
+  SLORA_CRIT_L2_NORM = 4        /* one projection (v): L2 norm per channel, top-k per head */
 } slora_criterion;
 
 typedef enum {
@@ -185,10 +188,31 @@ slora_status slora_svd_prepare(const void* W, int64_t n, int64_t k, slora_dtype 
  *        channels are kept per group.  idx_out [(heads + kv_heads) * k_h] int32:
  *        first, for every query head h, its group's kept channels as
  *        h*head_dim + c (ascending); then for every key head g, g*head_dim + c.
- *   Ties: equal scores go to the lower index.
+ *   FFN_GRAM (estimator variant; [ART §1-§2], a cheaper stand-in for the
+ *        activation norm): as FFN, but score_j = ||g_hat_j|| * ||u_hat_j||, each
+ *        norm a quadratic form of the r x r Gram matrix of X_C L (no per-token
+ *        nonlinearity; an upper bound of the activation-norm score).
+ *   QK_ROPE_PAIR (estimator variant): as QK, but the keys of a head are the
+ *        head_dim/2 rotate-half pairs (c, c + head_dim/2) that rotary position
+ *        embedding turns together; a pair's norms are taken over both channels
+ *        (invariant under the rotation), k_p = head_dim/2 - floor(s*head_dim/2)
+ *        pairs are kept, so k_h = 2 k_p channels per head, listed as the kept
+ *        first channels c ascending, then the matching c + head_dim/2.
+ *   L2_NORM (projection-set variant: v sliced on its output channels and o
+ *        on the matching input channels; [ART §6]): one matrix (L0, U0 of
+ *        v; L1 and U1 may be NULL), n0 = kv_heads*head_dim (v's width).
+ *        Channel c of value head g scores ||V_hat[:, g, c]||; k_h = head_dim -
+ *        floor(s*head_dim) kept per value head.  idx_out [(heads + kv_heads)
+ *        * k_h] as for QK: first, for every query head h (o's input channels),
+ *        its group's set as h*head_dim + c; then for every value head g,
+ *        g*head_dim + c.
+ *   Ties: equal scores go to the lower index.  A selection spans at most
+ *        32768 channels (d_ff for the FFN criteria, head_dim otherwise).
  *   sparsity  s in [0, 1).
- *   k_out     HOST int32*, receives k_keep (FFN) or k_h (QK).
- *   scores_out optional [d_ff] (FFN) or [kv_heads*head_dim] (QK) fp32 scores.
+ *   k_out     HOST int32*, receives k_keep (FFN criteria) or k_h (per head).
+ *   scores_out optional fp32 scores: [d_ff] (FFN criteria), [kv_heads*head_dim]
+ *             (QK), [kv_heads*head_dim/2] (QK_ROPE_PAIR, one per pair),
+ *             [heads*head_dim] (L2_NORM).
  */
 slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dtype dt,
                                    const slora_tokens* tok, int64_t d, const float* L0,
@@ -219,7 +243,10 @@ slora_status slora_estimate_select(slora_criterion crit, const void* X, slora_dt
  *     slora_estimate_select with a workspace for those.
  *   - The first call on a device resolves the buffer's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached per device with the
+ *     context it was resolved in and resolved again when a call comes from
+ *     another context (a non-primary context, or the primary context
+ *     recreated after cudaDeviceReset).
  *   - All calls on a device share the one buffer and it keeps the last
  *     call's contents (nothing in it needs to start at zero).  Calls that
  *     overlap on the GPU (different streams, or different host threads

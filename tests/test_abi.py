@@ -140,3 +140,40 @@ def test_library_has_no_unresolved_internal_symbols(L):
     out = subprocess.run(["nm", "-D", "--undefined-only", L.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     assert "slora" not in out, out
+
+
+def _est_query(L, crit, n0, n1, heads, kv, hd, s=0.5, L1=FAKE, U1=FAKE, d=64):
+    tok, keep = L.make_tokens(4, 16, [12] * 4)
+    k_out = ctypes.c_int32(0)
+    args = [crit, FAKE, L.BF16, ctypes.byref(tok), d, FAKE, FAKE, n0, L1, U1, n1, 8, heads, kv,
+            hd, s, FAKE, ctypes.byref(k_out), None]
+    return L.workspace_size("slora_estimate_select", args), k_out.value
+
+
+def test_estimate_select_query_variant_criteria(L):
+    # rotate-half pairs: k_h = 2 * (16 - floor(0.5 * 16)) channels per head
+    need, k = _est_query(L, L.CRIT_QK_ROPE_PAIR, 8 * 32, 2 * 32, 8, 2, 32)
+    assert need > 0 and k == 16
+    need, k = _est_query(L, L.CRIT_QK_ROPE_PAIR, 8 * 32, 2 * 32, 8, 2, 32, s=0.3)
+    assert k == 2 * (16 - 4)
+    with pytest.raises(L.SloraError) as e:  # odd head_dim has no rotate-half pairs
+        _est_query(L, L.CRIT_QK_ROPE_PAIR, 8 * 33, 2 * 33, 8, 2, 33)
+    assert e.value.status == 2
+    # per-head L2 norm of one projection: the second factor pair may be NULL
+    need, k = _est_query(L, L.CRIT_L2, 2 * 64, 0, 6, 2, 64, s=0.25, L1=None, U1=None)
+    assert need > 0 and k == 48
+    with pytest.raises(L.SloraError):  # n0 must be kv_heads * head_dim
+        _est_query(L, L.CRIT_L2, 6 * 64, 0, 6, 2, 64, L1=None, U1=None)
+    with pytest.raises(L.SloraError):  # heads a multiple of kv_heads
+        _est_query(L, L.CRIT_L2, 4 * 64, 0, 6, 4, 64, L1=None, U1=None)
+    # Gram FFN score: gate and up widths must agree; one selection spans <= 32768
+    need, k = _est_query(L, L.CRIT_FFN_GRAM, 688, 688, 0, 0, 0)
+    assert need > 0 and k == 344
+    with pytest.raises(L.SloraError):
+        _est_query(L, L.CRIT_FFN_GRAM, 688, 680, 0, 0, 0)
+    with pytest.raises(L.SloraError) as e:
+        _est_query(L, L.CRIT_FFN, 40000, 40000, 0, 0, 0)
+    assert e.value.status == 2
+    with pytest.raises(L.SloraError) as e:
+        _est_query(L, 9, 688, 688, 0, 0, 0)
+    assert e.value.status == 1
