@@ -1,16 +1,16 @@
 // tcgen05 sliced GEMM for sm_100a (see gemm_tc.cuh for the operand forms).
 //
-// Persistent kernel, one 256-thread CTA per SM:
-//   warp 0      TMA producer: A tile (128 x 64) and B tile (256 x 64) per
-//               stage; gathered B rows arrive through cp.async.bulk.tensor
-//               tile::gather4 (4 rows per instruction, spread over the lanes)
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
-//               K=16, bf16 x bf16 -> fp32) into a TMEM accumulator
-//   warp 2      TMEM allocator (512 columns = two 128x256 fp32 accumulators)
+// Persistent grid of cluster pairs (two 256-thread CTAs on two SMs) computing
+// 256 x 256 tiles with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16,
+// bf16 x bf16 -> fp32 in TMEM):
+//   warp 0      TMA producer: this CTA's halves of the A tile (128 x 64) and
+//               of the B tile per stage
+//   warp 1      MMA issuer (leader CTA): one thread issues tcgen05.mma
+//   warp 2      TMEM allocator (512 columns = two 256-wide accumulators)
 //   warps 4..7  epilogue: tcgen05.ld rows of the finished accumulator, apply
 //               the epilogue, store bf16; the other accumulator is being
 //               filled meanwhile
-// Shared memory: 4 stages x (16 KB A + 32 KB B), 128-byte swizzle (the TMA
+// Shared memory: stages of (16 KB A + 16 KB B), 128-byte swizzle (the TMA
 // swizzle and the UMMA descriptor layout agree: 8-row / 1024-byte atoms).
 // Every mbarrier wait is bounded (clock64 budget); on expiry the CTA raises
 // an abort flag, waits (bounded) for its copies in flight, frees TMEM and
@@ -28,18 +28,12 @@ __device__ int g_tc_error = 0;
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;               // 16 KB
-constexpr int B_BYTES = BN * BK * 2;               // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 48 KB
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr long long WAIT_BUDGET = 4000000000LL;    // ~2 s of SM clocks per wait
 
 struct alignas(64) TcParams {
   CUtensorMap amap[4];
   CUtensorMap bmap[4][2];
-  const int32_t* idx[4];
-  int nidx[4];
   int nkb[4];
   int bmode[4];
   int bpair[4];
@@ -110,23 +104,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
     }
   }
 }
-__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
-                                         int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
-                                            int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(su32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3)
-      : "memory");
-}
 __device__ __forceinline__ void fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -147,21 +124,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) |
          (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
-}
-__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          su32(bar))
-      : "memory");
 }
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
@@ -332,277 +294,6 @@ __device__ __forceinline__ void proj_store(float* part, long long out_row, int n
     }
 }
 
-struct TileInfo {
-  int a_row, out_row, nvalid, n0;
-};
-__device__ __forceinline__ TileInfo tile_info(const TcParams& p, int t) {
-  const int mt = t % p.n_mtiles, nt = t / p.n_mtiles;
-  const int4 tl = p.tiles[mt];
-  TileInfo ti;
-  ti.a_row = p.a_compact ? tl.y : tl.x;
-  ti.out_row = p.out_compact ? tl.y : tl.x;
-  ti.nvalid = tl.z;
-  ti.n0 = nt * (p.paired ? BN / 2 : BN);
-  return ti;
-}
-
-__global__ void __launch_bounds__(256, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
-    }
-    *abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 2) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
-                     su32(tmem_slot))
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tbase = *tmem_slot;
-  const int total = p.n_mtiles * p.n_ntiles;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    int issued = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const TileInfo ti = tile_info(p, t);
-      const int nt = t / p.n_mtiles;
-      for (int s = 0; s < p.nseg && ok; ++s) {
-        const int mode = p.bmode[s];
-        const int32_t* idx = p.idx[s];
-        const int nidx = p.nidx[s];
-        // K-major gather: this lane's rows are fixed for the whole tile
-        int krow[2][4];
-        if (mode == B_K_GATHER) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int g = lane + 32 * j;  // 64 groups of 4 rows
-            const int h = g / 32, gi = g % 32;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              int n = p.bpair[s] ? (ti.n0 + 4 * gi + q) : (nt * BN + 128 * h + 4 * gi + q);
-              n = n < nidx ? n : nidx - 1;
-              krow[j][q] = __ldg(idx + n);
-            }
-          }
-        }
-        for (int kb = 0; kb < p.nkb[s]; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-          if (lane == 0) mbar_expect_tx(&full[stage], STAGE_BYTES);
-          __syncwarp();
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          if (lane == 0) tma_load(sa, &p.amap[s], &full[stage], kb * BK, ti.a_row);
-          if (mode == B_K) {
-            if (lane < 2) {
-              const int h = lane;
-              const int row = p.bpair[s] ? ti.n0 : nt * BN + 128 * h;
-              tma_load(sb + h * (B_BYTES / 2), &p.bmap[s][p.bpair[s] ? h : 0], &full[stage],
-                       kb * BK, row);
-            }
-          } else if (mode == B_K_GATHER) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int g = lane + 32 * j;
-              const int h = g / 32;
-              tma_gather4(sb + g * 512, &p.bmap[s][p.bpair[s] ? h : 0], &full[stage], kb * BK,
-                          krow[j][0], krow[j][1], krow[j][2], krow[j][3]);
-            }
-          } else if (mode == B_MN) {
-            if (lane < 4)
-              tma_load(sb + lane * 8192, &p.bmap[s][0], &full[stage], ti.n0 + 64 * lane, kb * BK);
-          } else {  // B_MN_GATHER
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int g = lane + 32 * j;
-              const int a = g / 16, grp = g % 16;
-              int r[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                int k = kb * BK + 4 * grp + q;
-                k = k < nidx ? k : nidx - 1;
-                r[q] = __ldg(idx + k);
-              }
-              tma_gather4(sb + a * 8192 + grp * 512, &p.bmap[s][0], &full[stage],
-                          ti.n0 + 64 * a, r[0], r[1], r[2], r[3]);
-            }
-          }
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-      }
-    }
-    if (!ok && lane == 0) {
-      // let the copies already issued land before the CTA can exit
-      int st2 = stage;
-      uint32_t ph2 = phase;
-      for (int i = 0; i < STAGES && i < issued; ++i) {
-        if (--st2 < 0) { st2 = STAGES - 1; ph2 ^= 1u; }
-        const long long t0 = clock64();
-        while (!mbar_try(&full[st2], ph2) && clock64() - t0 < WAIT_BUDGET) {
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t aph = uint32_t(it >> 1) & 1u;
-        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort)) break;
-        fence_after();
-        const uint32_t d = tbase + uint32_t(acc * BN);
-        bool first = true;
-        for (int s = 0; s < p.nseg && ok; ++s) {
-          const int bmn = p.bmode[s] >= B_MN;
-          const uint32_t idesc = idesc_bf16(BM, BN, bmn);
-          for (int kb = 0; kb < p.nkb[s]; ++kb) {
-            if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
-            fence_after();
-            const uint32_t sa = su32(smem + stage * STAGE_BYTES);
-            const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
-              const uint64_t ad = sdesc(sa + k * 32, 16, 1024);
-              const uint64_t bd = bmn ? sdesc(sb + k * 2048, 8192, 1024) : sdesc(sb + k * 32, 16, 1024);
-              mma_bf16(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
-            }
-            first = false;
-            mma_commit(&empty[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-        }
-        mma_commit(&tfull[acc]);
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp - 4;
-    const int r = q * 32 + lane;  // row within the tile == TMEM lane
-    int it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t aph = uint32_t(it >> 1) & 1u;
-      if (!mbar_wait(&tfull[acc], aph, abort)) break;
-      fence_after();
-      const TileInfo ti = tile_info(p, t);
-      const bool valid = r < ti.nvalid;
-      const int64_t orow = int64_t(ti.out_row) + r;
-      const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-      float v[32], w[32];
-      if (p.epi == EPI_SWIGLU_FWD) {
-        __nv_bfloat16* g = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
-        __nv_bfloat16* u = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
-        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out2) + orow * p.ldo;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tl + c * 32, v);
-          tmem_ld32(tl + 128 + c * 32, w);
-          if (valid) {
-            const int c0 = ti.n0 + c * 32;
-            store_row32(g, c0, p.N, v);
-            store_row32(u, c0, p.N, w);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = silu_f(v[j]) * w[j];
-            store_row32(h, c0, p.N, v);
-          }
-        }
-      } else if (p.epi == EPI_SWIGLU_BWD) {
-        const __nv_bfloat16* gi = static_cast<const __nv_bfloat16*>(p.in0) + orow * p.ldi;
-        const __nv_bfloat16* ui = static_cast<const __nv_bfloat16*>(p.in1) + orow * p.ldi;
-        __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
-        __nv_bfloat16* du = static_cast<__nv_bfloat16*>(p.out1) + orow * p.ldo;
-        if (valid) {  // the whole row segment of g and u on its way to L2 at once
-          prefetch_row256(gi, ti.n0, p.N);
-          prefetch_row256(ui, ti.n0, p.N);
-        }
-        // g and u of chunk c + 1 are loaded while chunk c is computed, so each
-        // chunk's global-load latency hides behind the previous chunk's math
-        float gv[32], uv[32], gn[32], un[32];
-        if (valid && ti.n0 < p.N) {
-          load_row32(gi, ti.n0, p.N, gv);
-          load_row32(ui, ti.n0, p.N, uv);
-        }
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          tmem_ld32(tl + c * 32, v);  // dh
-          const int c0 = ti.n0 + c * 32;
-          const bool next = valid && c + 1 < 8 && c0 + 32 < p.N;
-          if (next) {
-            load_row32(gi, c0 + 32, p.N, gn);
-            load_row32(ui, c0 + 32, p.N, un);
-          }
-          if (valid && c0 < p.N) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float sg = sigmoid_f(gv[j]);
-              const float dh = v[j];
-              v[j] = dh * uv[j] * sg * (1.0f + gv[j] * (1.0f - sg));  // dG
-              w[j] = dh * gv[j] * sg;                                  // dU
-            }
-            store_row32(dg, c0, p.N, v);
-            store_row32(du, c0, p.N, w);
-          }
-          if (next) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              gv[j] = gn[j];
-              uv[j] = un[j];
-            }
-          }
-        }
-      } else {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out0) + orow * p.ldo;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          tmem_ld32(tl + c * 32, v);
-          const int c0 = ti.n0 + c * 32;
-          if (valid && c0 < p.N) store_row32(o, c0, p.N, v, p.vec_out != 0);
-        }
-      }
-      fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-    }
-  }
-  fence_before();
-  __syncthreads();
-  if (warp == 2) {
-    fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tbase) : "memory");
-  }
-}
-
-
 // ------------------------------------------------------------------------
 // 2-CTA variant: a cluster of two CTAs computes a 256 x 256 tile with
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16).  Each CTA loads only
@@ -754,16 +445,6 @@ __device__ __forceinline__ void tma_load_2sm(void* dst, const CUtensorMap* m, ui
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(su32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4_2sm(void* dst, const CUtensorMap* m,
-                                                uint32_t bar_cluster, int x, int r0, int r1,
-                                                int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
-      "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3)
       : "memory");
 }
 __device__ __forceinline__ void mma_bf16_2sm(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -1005,20 +686,9 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
       const int n0 = nt * (p.paired ? BN / 2 : BN);
       for (int s = 0; s < p.nseg && ok; ++s) {
         const int mode = p.bmode[s];
-        const int32_t* idx = p.idx[s];
-        const int nidx = p.nidx[s];
         const CUtensorMap* bm = &p.bmap[s][p.bpair[s] ? rank : 0];
         // this CTA's 128 B rows start at
         const int brow0 = p.bpair[s] ? n0 : nt * BN + 128 * int(rank);
-        int krow[4];
-        if (mode == B_K_GATHER) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            int n = brow0 + 4 * lane + q;
-            n = n < nidx ? n : nidx - 1;
-            krow[q] = __ldg(idx + n);
-          }
-        }
         for (int kb = 0; kb < p.nkb[s]; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort)) { ok = false; break; }
           const uint32_t fbar = map_to_rank(su32(&full[stage]), 0);
@@ -1029,23 +699,9 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
           if (lane == 0) tma_load_2sm(sa, &p.amap[s], fbar, kb * BK, a_row);
           if (mode == B_K) {
             if (lane == 1) tma_load_2sm(sb, bm, fbar, kb * BK, brow0);
-          } else if (mode == B_K_GATHER) {
-            tma_gather4_2sm(sb + lane * 512, bm, fbar, kb * BK, krow[0], krow[1], krow[2],
-                            krow[3]);
-          } else if (mode == B_MN) {
+          } else {  // B_MN: two 64-wide MN atoms of this CTA's half
             if (lane < 2)
               tma_load_2sm(sb + lane * 8192, bm, fbar, n0 + 64 * (2 * int(rank) + lane), kb * BK);
-          } else {  // B_MN_GATHER
-            const int al = lane / 16, grp = lane % 16;
-            int r4[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              int k = kb * BK + 4 * grp + q;
-              k = k < nidx ? k : nidx - 1;
-              r4[q] = __ldg(idx + k);
-            }
-            tma_gather4_2sm(sb + al * 8192 + grp * 512, bm, fbar,
-                            n0 + 64 * (2 * int(rank) + al), r4[0], r4[1], r4[2], r4[3]);
           }
           ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -1078,7 +734,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
         const uint32_t d = tbase + uint32_t(acc * BN);
         bool first = true;
         for (int s = 0; s < p.nseg && ok; ++s) {
-          const int bmn = p.bmode[s] >= B_MN;
+          const int bmn = p.bmode[s] == B_MN;
           const uint32_t idesc = idesc_bf16(2 * BM, BN, bmn);
           for (int kb = 0; kb < p.nkb[s]; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
@@ -1304,21 +960,8 @@ slora_status encode(CUtensorMap* m, const TcMat& t, int box_x, int box_y,
 }
 
 bool g_attr_set = false;
-// 1: one-CTA 128x256 tiles; 2: two-CTA (cluster pair) 256x256 tiles.
-int g_tc_mode = 2;
 
 }  // namespace
-
-int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 int64_t tc_ntiles(const TcGemm& g) {
   const int64_t ncols = g.paired ? BN / 2 : BN;
@@ -1326,7 +969,7 @@ int64_t tc_ntiles(const TcGemm& g) {
 }
 
 slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
-  if (g.proj0 && (g_tc_mode != 2 || (g.proj_r != 8 && g.proj_r != 16) || g.ldproj % 8 ||
+  if (g.proj0 && ((g.proj_r != 8 && g.proj_r != 16) || g.ldproj % 8 ||
                   !g.proj_part || (g.epi == EPI_SWIGLU_BWD && !g.proj1) || g.epi == EPI_STORE ||
                   (reinterpret_cast<uintptr_t>(g.proj0) & 15) ||
                   (reinterpret_cast<uintptr_t>(g.proj1) & 15) ||
@@ -1347,23 +990,15 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
     const TcSeg& sg = g.seg[s];
     if (sg.K <= 0) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: segment %d has K=%lld", s, (long long)sg.K);
     SLORA_TRY(encode(&p.amap[s], sg.a, BK, BM));
-    const bool gather = sg.bmode == B_K_GATHER || sg.bmode == B_MN_GATHER;
-    if (gather && (!sg.idx || sg.nidx <= 0))
-      SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: gather without indices");
-    int by = 0;
-    switch (sg.bmode) {
-      case B_K: by = 128; break;
-      case B_MN: by = 64; break;
-      default: by = 1; break;
-    }
+    if (sg.bmode != B_K && sg.bmode != B_MN)
+      SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: unknown B operand form %d", sg.bmode);
+    const int by = sg.bmode == B_K ? 128 : 64;
     SLORA_TRY(encode(&p.bmap[s][0], sg.b0, BK, by));
     if (sg.bpair) {
-      if (sg.bmode != B_K && sg.bmode != B_K_GATHER)
+      if (sg.bmode != B_K)
         SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: paired halves need a K-major B");
       SLORA_TRY(encode(&p.bmap[s][1], sg.b1, BK, by));
     }
-    p.idx[s] = sg.idx;
-    p.nidx[s] = int(sg.nidx);
     p.nkb[s] = int((sg.K + BK - 1) / BK);
     p.bmode[s] = sg.bmode;
     p.bpair[s] = sg.bpair;
@@ -1394,8 +1029,6 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   p.in1 = g.in1;
   p.ldi = g.ldi;
   if (!g_attr_set) {
-    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    SMEM_BYTES));
     SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2, false>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES));
     SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2B, true>,
@@ -1404,7 +1037,7 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   }
   // SwiGLU backward through shared memory: operands addressable by TMA
   auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
-  const bool bwd_tma = g_tc_mode == 2 && g.epi == EPI_SWIGLU_BWD && !g.paired && g.io_rows > 0 &&
+  const bool bwd_tma = g.epi == EPI_SWIGLU_BWD && !g.paired && g.io_rows > 0 &&
                        al16(g.in0) && al16(g.in1) && al16(g.out0) && al16(g.out1);
   if (bwd_tma) {
     TcMat e;
@@ -1430,41 +1063,29 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
       SLORA_TRY(encode(&p.emap[5], e, p.proj_r, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
   }
-  if (g_tc_mode == 2) {
-    const int64_t ctiles = int64_t((p.n_mtiles + 1) / 2) * p.n_ntiles;
-    const int64_t maxc = num_sms() / 2;
-    const int nclus = int(ctiles < maxc ? ctiles : maxc);
-    LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum),
-                   st);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(2 * nclus), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.dynamicSmemBytes = bwd_tma ? SMEM2B_BYTES : SMEM2_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (bwd_tma)
-      SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2B, true>, p));
-    else
-      SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2, false>, p));
-    return SLORA_OK;
-  }
-  const int64_t tiles = int64_t(p.n_mtiles) * p.n_ntiles;
-  const int grid = int(tiles < num_sms() ? tiles : num_sms());
-  // algorithmic FLOPs: 2 * valid rows (g.M) * computed columns * sum of K
-  LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum), st);
-  tc_gemm_kernel<<<grid, 256, SMEM_BYTES, st>>>(p);
-  SLORA_CHECK_LAUNCH();
+  const int64_t ctiles = int64_t((p.n_mtiles + 1) / 2) * p.n_ntiles;
+  const int64_t maxc = num_sms() / 2;
+  const int nclus = int(ctiles < maxc ? ctiles : maxc);
+  LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum),
+                 st);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(2 * nclus), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = bwd_tma ? SMEM2B_BYTES : SMEM2_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (bwd_tma)
+    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2B, true>, p));
+  else
+    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2, false>, p));
   return SLORA_OK;
 }
-
-void set_tc_mode(int mode) { g_tc_mode = mode == 1 ? 1 : 2; }
-int tc_mode() { return g_tc_mode; }
 
 slora_status tc_check_error(bool clear) {
   int v = 0;

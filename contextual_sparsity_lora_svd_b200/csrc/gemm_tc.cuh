@@ -3,16 +3,14 @@
 //   C[M x N] = sum_seg A_seg[M x K_seg] . B_seg[N x K_seg]^T     (fp32 in TMEM)
 //
 // A operands are bf16 row-major (K-major) and loaded by TMA in 128 x 64
-// boxes.  B operands are bf16 and come in four forms:
-//   B_K          K-major, rows = output channels, contiguous rows
-//   B_K_GATHER   K-major, output channels = rows idx[n] (TMA tile::gather4)
-//   B_MN         MN-major, rows = reduction index k, contiguous
-//   B_MN_GATHER  MN-major, reduction index k -> row idx[k] (tile::gather4)
-// so a selected channel slice of a frozen weight is consumed in place, as
-// rows of W0 (output-side slice) or rows of W0^T (input-side slice), with no
-// compaction copy.  Up to four segments accumulate into one tile (the LoRA
-// branch is one more segment with K = rank).  Epilogues: plain bf16 store,
-// SwiGLU forward on paired gate/up halves (stores g, u and h = silu(g) u), and
+// boxes.  B operands are bf16, contiguous, in two forms:
+//   B_K   K-major, rows = output channels
+//   B_MN  MN-major, rows = reduction index k
+// so a selected channel slice, once compacted into contiguous rows, is
+// consumed as rows of W0 (output-side slice) or rows of W0^T (input-side
+// slice).  Up to four segments accumulate into one tile (the LoRA branch is
+// one more segment with K = rank).  Epilogues: plain bf16 store, SwiGLU
+// forward on paired gate/up halves (stores g, u and h = silu(g) u), and
 // SwiGLU backward (reads g, u; stores dG, dU).
 //
 // Rows: a list of 128-row M tiles {full_row0, compact_row0, nvalid}; a tile
@@ -24,7 +22,7 @@
 
 namespace slora {
 
-enum TcBMode : int { B_K = 0, B_K_GATHER = 1, B_MN = 2, B_MN_GATHER = 3 };
+enum TcBMode : int { B_K = 0, B_MN = 1 };
 enum TcEpi : int { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2 };
 
 struct TcMat {  // bf16 row-major matrix in global memory
@@ -37,8 +35,6 @@ struct TcSeg {
   TcMat b0, b1;     // b1 only with bpair (second half of the N tile)
   int bmode = B_K;
   int bpair = 0;    // K-major only: half h of the 256-row tile reads b_h rows n0p + r
-  const int32_t* idx = nullptr;  // gather list (N index for B_K_GATHER, K index for B_MN_GATHER)
-  int64_t nidx = 0;              // valid entries of idx
   int64_t K = 0;
 };
 
@@ -60,7 +56,7 @@ struct TcGemm {
   const void* in1 = nullptr;  // SWIGLU_BWD: u
   int64_t ldi = 0;
   // Optional rank-r projection of the epilogue's values, r = proj_r in {8, 16}
-  // (one-of-two-CTA tile mode only): SWIGLU_FWD projects h with proj0,
+  // SWIGLU_FWD projects h with proj0,
   // SWIGLU_BWD projects dG with proj0 and dU with proj1.  proj0/proj1 are bf16
   // [N x ldproj] (row = output channel, ldproj a multiple of 8); each N tile
   // writes, per output row (output layout), the fp32 partial sums over its
@@ -73,8 +69,8 @@ struct TcGemm {
   float* proj_part = nullptr;
   int64_t proj_rows = 0;
   // SWIGLU_BWD: rows of in0, in1, out0 and out1 (all [io_rows x N], leading
-  // dimensions ldi / ldo).  When set (two-CTA tile mode, 16-byte aligned
-  // pointers) g and u are loaded and dG and dU stored by TMA through shared
+  // dimensions ldi / ldo).  When set (16-byte aligned pointers) g and u are
+  // loaded and dG and dU stored by TMA through shared
   // memory, and the projection slices too; 0 keeps per-row loads and stores.
   int64_t io_rows = 0;
 };
@@ -86,13 +82,5 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st);
 
 // Device error flag of the tcgen05 kernels (a bounded wait that expired).
 slora_status tc_check_error(bool clear);
-
-// Tile variant of the tcgen05 GEMM: 1 = one-CTA 128x256 tiles, 2 = cluster
-// pairs with cta_group::2 256x256 tiles (default).
-void set_tc_mode(int mode);
-int tc_mode();
-
-// Number of SMs of the current device (cached).
-int num_sms();
 
 }  // namespace slora

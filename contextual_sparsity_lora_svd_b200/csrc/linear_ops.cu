@@ -208,9 +208,10 @@ slora_status linear_bwd_run(const LinearDesc& L0, const slora_tokens* tok, const
 // ------------------------------------------------------- FFN, bf16, tcgen05
 // The eight large contractions (gate|up forward, down forward, dh backward,
 // dX backward; each once for the context rows on the selected channels and
-// once for the dense output rows) run on the tcgen05 kernel with the selected
-// slices gathered in place; the rank-r LoRA projections and the LoRA
-// gradients (HBM-bound, N or M = r) run on the CUDA-core GEMM.
+// once for the dense output rows) run on the tcgen05 kernel over the selected
+// slices compacted into contiguous rows; the rank-r LoRA projections and the
+// LoRA gradients (HBM-bound, N or M = r) run on the skinny tensor-core
+// stream kernels.
 namespace {
 TcMat mat(const void* p, int64_t rows, int64_t cols, int64_t ld) {
   TcMat m;
@@ -224,12 +225,10 @@ struct TcBuilder {
     g.tiles = tiles; g.n_mtiles = int(ntiles); g.a_compact = a_compact;
     g.out_compact = out_compact; g.M = M; g.N = N; g.paired = paired; g.epi = epi;
   }
-  TcBuilder& seg(TcMat a, TcMat b0, int bmode, int64_t K, const int32_t* idx = nullptr,
-                 int64_t nidx = 0, int bpair = 0, TcMat b1 = TcMat()) {
+  TcBuilder& seg(TcMat a, TcMat b0, int bmode, int64_t K, int bpair = 0, TcMat b1 = TcMat()) {
     if (K <= 0) return *this;  // an empty slice contributes nothing
     TcSeg& s = g.seg[g.nseg++];
-    s.a = a; s.b0 = b0; s.b1 = b1; s.bmode = bmode; s.bpair = bpair; s.idx = idx;
-    s.nidx = nidx; s.K = K;
+    s.a = a; s.b0 = b0; s.b1 = b1; s.bmode = bmode; s.bpair = bpair; s.K = K;
     return *this;
   }
   TcBuilder& out(void* o0, void* o1, void* o2, int64_t ldo) {
@@ -289,7 +288,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   // rank-r projections done in the GEMM epilogues (h Ad^T in the gate|up GEMMs,
   // [dG Bg | dU Bu] in the dh GEMMs) instead of separate passes over h, dG, dU;
   // per-N-tile partials, summed in order by reduce_row_partials
-  const bool proj = tc_mode() == 2 && (lr == 8 || lr == 16);
+  const bool proj = lr == 8 || lr == 16;
   const int64_t ntFc = (kk + 127) / 128, ntFo = (Fd + 127) / 128;  // paired gate|up tiles
   const int64_t ntBc = (kk + 255) / 256, ntBo = (Fd + 255) / 256;  // dh tiles
   const bool bpad = proj && (r != lr || !aligned16(L.Bg) || !aligned16(L.Bu));
@@ -407,12 +406,14 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   float* Pfull = fused ? ar.take<float>(size_t(T) * 2 * rs) : nullptr;
   EstBufs eb;
   if (!idx_force)
-    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, rs, 0, 0, fused, nullptr, ar);
+    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, rs, 0, 0, 0, fused, nullptr,
+                          ar);
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt, eb.cnt,
+                           eb.ncnt));
   // The small LoRA operand layouts run on the library's side stream, beside
   // the pass over X and the estimator (first those independent of the
   // selection, then, once it is known, the ones on the kept channels); the
@@ -449,8 +450,8 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
       SLORA_TRY(sanitize_indices(idx_force, kk, Fd, idx, st));
   } else {
     SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
-                                     L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, kk, idx, eb, st, fused,
-                                     Pfull, 2 * rs, rsp));
+                                     L.Ug, Fd, L.Lu, L.Uu, rs, 0, 0, 0, F.sparsity, idx, eb, st,
+                                     fused, Pfull, 2 * rs, rsp));
   }
   SLORA_TRY(fork_side(st, side));  // the selection is known
   SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, idx, kk, r, nntC, lr2, BpC, side, Fd));
@@ -475,7 +476,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   // ---- forward
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
-    b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, nullptr, 0, 1, mat(WuS, kk, d, d))
+    b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, 1, mat(WuS, kk, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpC, nntC * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gC, uC, hC, ldk);
     if (proj) b.proj(AdtS, nullptr, lr, int(lr), projC, TC);
@@ -483,7 +484,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   }
   {  // gate|up, output rows, every channel
     TcBuilder b(otiles, nott, 0, 1, TO, Fd, 1, EPI_SWIGLU_FWD);
-    b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K, d, nullptr, 0, 1, mat(L.Wu, Fd, d, d))
+    b.seg(mat(X, T, d, d), mat(L.Wg, Fd, d, d), B_K, d, 1, mat(L.Wu, Fd, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpO, nntO * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gO, uO, hO, Fd);
     if (proj) b.proj(Adt, nullptr, lr, int(lr), projO, TO);
@@ -643,18 +644,20 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
   void* dUO = buf(TO, Fd);
   EstBufs eb;
   if (!idx_force)
-    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, L.r_svd, 0, 0, false, nullptr,
-                          ar);
+    eb = estimate_reserve(SLORA_CRIT_FFN_SWIGLU_L2, dt, ti, d, Fd, L.r_svd, 0, 0, 0, false,
+                          nullptr, ar);
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, nullptr, nullptr, nullptr, 0, eb.cnt,
+                           eb.ncnt));
   if (idx_force) {
     if (kk > 0)
       SLORA_TRY(sanitize_indices(idx_force, kk, Fd, idx, st));
   } else {
     SLORA_TRY(estimate_select_launch(SLORA_CRIT_FFN_SWIGLU_L2, X, dt, ti, ctx_rows, d, L.Lg,
-                                     L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, kk, idx, eb, st));
+                                     L.Ug, Fd, L.Lu, L.Uu, L.r_svd, 0, 0, 0, F.sparsity, idx, eb,
+                                     st));
   }
 
   // ---- forward
