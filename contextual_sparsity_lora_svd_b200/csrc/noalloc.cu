@@ -2,6 +2,8 @@
 // cannot hand the library a workspace (see include/slora.h).  Its scratch is a
 // file-scope device buffer of fixed size that every GPU loading this library
 // keeps until the process exits.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -13,27 +15,63 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// The resolved address is valid for the context it was resolved in: it is
+// cached per device together with that context's handle and resolved again
+// when the calling thread's current context differs (a non-primary context,
+// or the primary context recreated after cudaDeviceReset).
+struct Resolved {
+  CUcontext ctx = nullptr;
+  void* ptr = nullptr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+Resolved g_noalloc[kMaxDevices];
 
-// Device address of the scratch buffer on the current device.  In host code
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point lookup (no link
+// against the driver library).  *ctx is NULL when the thread has no current
+// context yet.
+slora_status current_context(CUcontext* ctx) {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    const cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f)
+      SLORA_FAIL(SLORA_ERR_CUDA, "driver entry point cuCtxGetCurrent unavailable: %s",
+                 cudaGetErrorString(e));
+    fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  }
+  *ctx = nullptr;
+  if (fn(ctx) != CUDA_SUCCESS) *ctx = nullptr;
+  return SLORA_OK;
+}
+
+// Device address of the scratch buffer in the current context.  In host code
 // the symbol itself only names a host-side stand-in, so the address comes
-// from cudaGetSymbolAddress, once per device, with that device current.
+// from cudaGetSymbolAddress, with the device current, once per context.
 slora_status noalloc_scratch(void** out) {
   int dev = -1;
   SLORA_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices)
     SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices);
+  CUcontext ctx = nullptr;
+  SLORA_TRY(current_context(&ctx));
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  Resolved& r = g_noalloc[dev];
+  if (!r.ptr || !ctx || r.ctx != ctx) {
+    // cudaGetSymbolAddress also makes the device's primary context current
+    // when the thread has none yet; the context is read again afterwards.
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       SLORA_FAIL(SLORA_ERR_CUDA, "cudaGetSymbolAddress of the scratch buffer failed: %s",
                  cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
+    SLORA_TRY(current_context(&ctx));
+    r.ctx = ctx;
+    r.ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = r.ptr;
   return SLORA_OK;
 }
 

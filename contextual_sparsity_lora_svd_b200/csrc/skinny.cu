@@ -446,13 +446,13 @@ __global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int
 
 // One full wave of resident blocks: the shared memory of a block bounds how
 // many fit on an SM (each keeps S-1 chunks of Y in flight).  The SM count is
-// the B200's, a constant, so the workspace query needs no device.
-constexpr int kSMs = 148;
+// the device's, queried once (num_sms), so a workspace query and the run it
+// sizes see the same value.
 int64_t target_blocks(int CP, int NT) {
   int per_sm = (200 * 1024) / smem_for(CP, NT);
   if (per_sm > 8) per_sm = 8;
   if (per_sm < 1) per_sm = 1;
-  return int64_t(kSMs) * per_sm;
+  return int64_t(num_sms()) * per_sm;
 }
 
 int64_t splits_for(int64_t nblocks, int64_t nchunks, int CP, int NT) {
@@ -608,6 +608,9 @@ struct TmaJob {
   CUtensorMap rmap;  // split rank operand, 64 x (NT * CP) boxes
   StreamPlan p;
   int c = 0;
+  // leading 16-column pairs whose second and third bf16 terms are zero (the
+  // columns come from a bf16 operand): their MMAs for those terms are skipped
+  int f1 = 0;
   int unit0 = 0;                 // first ticket of the job
   int64_t M = 0, K = 0;
   float* part = nullptr;         // p.nunits partial tiles of 64 x CP floats
@@ -620,7 +623,11 @@ template <int J>
 struct TmaJobs {
   TmaJob job[J];
   int njobs = 0, nunits = 0, ncta = 1;
-  unsigned* ticket = nullptr;  // unit ticket, zero on entry, left zero
+  // unit ticket: zero on entry (every call zeroes it with its row maps) and
+  // left zero by a launch that completes; after an expired wait
+  // (SLORA_ERR_TIMEOUT) it and the block counters are undefined until the
+  // next call zeroes them
+  unsigned* ticket = nullptr;
 };
 static_assert(sizeof(TmaJobs<kMaxTmaJobs>) <= 4096, "TMA job table beyond 4 KB of parameters");
 
@@ -773,6 +780,7 @@ __global__ void __launch_bounds__(NTH + 32) skinny_tma_kernel(const __grid_const
     if (!mbar_wait_bounded(&full[st], uint32_t((j / S) & 1), g_sk_budget)) s_abort = 1;
     const int4 inf = info[st];
     if (!s_abort && !(inf.z & kEnd)) {
+      const int f1 = jobs.job[inf.z >> kJobShift].f1;  // uniform over the CTA
       const uint32_t ybase = su32(sm + st * SB), rbase = ybase + kYTile;
 #pragma unroll
       for (int k16 = 0; k16 < TILE / 16; ++k16) {
@@ -785,6 +793,7 @@ __global__ void __launch_bounds__(NTH + 32) skinny_tma_kernel(const __grid_const
         for (int s = 0; s < NT; ++s)
 #pragma unroll
           for (int fp = 0; fp < NF / 2; ++fp) {
+            if (s > 0 && fp < f1) continue;  // zero terms of bf16 columns
             uint32_t bf[4];
             ldsm4(bf, swz(rbase, s * CP + fp * 16 + b_rowoff, k16 * 2 + b_half));
             mma16816(acc[2 * fp], a[0], a[1], a[2], a[3], bf[0], bf[1]);
@@ -947,11 +956,11 @@ bool tma_ok(const SkY& Y, int64_t rows, int64_t cols) {
 // resident CTA for a job alone: dynamic balance), at most 32 groups per block
 // (the last unit of a block sums that many tiles).
 StreamPlan stream_plan(int64_t nout, int64_t nred,
-                       int64_t target = 2 * int64_t(kSMs) * kTmaCtasPerSm) {
+                       int64_t target = 2 * int64_t(num_sms()) * kTmaCtasPerSm) {
   StreamPlan p;
   p.nblocks = int((nout + TILE - 1) / TILE);
   p.nchunks = int(std::max<int64_t>((nred + TILE - 1) / TILE, 1));
-  const int64_t cap = int64_t(kSMs) * kTmaCtasPerSm;
+  const int64_t cap = int64_t(num_sms()) * kTmaCtasPerSm;
   int64_t want = (std::max<int64_t>(target, 1) + p.nblocks - 1) / std::max(p.nblocks, 1);
   if (want < 1) want = 1;
   if (want > 32) want = 32;
@@ -1012,11 +1021,12 @@ slora_status fill_tma_job(TmaJob& J, bool col, const SkY& Y, int64_t M, int64_t 
 
 slora_status launch_tma(bool col, const SkY& Y, int64_t M, int64_t K, int c, int nt,
                         const SkRowOut& ro, const SkColOut& co, const SkWork& w, int64_t I64,
-                        cudaStream_t st) {
+                        cudaStream_t st, int f1 = 0) {
   (void)I64;
   const StreamPlan p = col ? stream_plan(K, M) : stream_plan(M, K);
   TmaJobs<1> jb;
   SLORA_TRY(fill_tma_job(jb.job[0], col, Y, M, K, c, nt, w.rsplit, p, w.part, w.counters));
+  jb.job[0].f1 = f1;
   jb.job[0].ro = ro;
   jb.job[0].co = co;
   jb.job[0].unit0 = 0;
@@ -1074,7 +1084,7 @@ bool batch_tma_ok(const SkColJob* jobs, int n) {
 void batch_plans(const SkColJob* jobs, int n, StreamPlan* plans) {
   double total = 0.0;
   for (int k = 0; k < n; ++k) total += double(jobs[k].M) * double(jobs[k].K);
-  const double units = 2.0 * kSMs * kTmaCtasPerSm;
+  const double units = 2.0 * num_sms() * kTmaCtasPerSm;
   for (int k = 0; k < n; ++k) {
     const double share = total > 0 ? double(jobs[k].M) * double(jobs[k].K) / total : 1.0;
     plans[k] = stream_plan(jobs[k].K, jobs[k].M, std::max<int64_t>(1, llround(units * share)));
@@ -1142,7 +1152,7 @@ slora_status coldot_batch(const SkColJob* jobs, int n, float* part, unsigned* co
   }
   jb.njobs = n;
   jb.nunits = unit;
-  jb.ncta = int(std::min<int64_t>(unit, int64_t(kSMs) * kTmaCtasPerSm));
+  jb.ncta = int(std::min<int64_t>(unit, int64_t(num_sms()) * kTmaCtasPerSm));
   jb.ticket = cc;
   LaunchScope ls(kSkinny, bytes, st);
   return launch_tma_jobs<true, kMaxTmaJobs>(jb, CP, nt, st);
@@ -1226,7 +1236,11 @@ slora_status rowdot(const SkY& Y, int64_t M, int64_t K, const SkR& R, int c, con
   const int64_t I64 = round64(std::max<int64_t>(K, 1));
   const __nv_bfloat16* RS = static_cast<const __nv_bfloat16*>(w.rsplit);
   if (!w.prepared) SLORA_TRY(prep_r(R, c, CP, K, g.nt, static_cast<__nv_bfloat16*>(w.rsplit), st));
-  if (tma_ok(Y, M, K)) return launch_tma(false, Y, M, K, c, g.nt, o, SkColOut(), w, I64, st);
+  if (tma_ok(Y, M, K)) {
+    // columns below qsplit taken from a bf16 operand carry one nonzero term
+    const int f1 = (g.nt == 3 && R.dt == kBF16 && R.ptr_b) ? std::min(R.qsplit, c) / 16 : 0;
+    return launch_tma(false, Y, M, K, c, g.nt, o, SkColOut(), w, I64, st, f1);
+  }
   const dim3 grid = dim3(unsigned(g.nblocks), unsigned(g.nsplit), 1u);
   LaunchScope ls(kSkinny,
                  double(M) * K * 2 + double(g.nsplit > 1 ? 2 * g.nsplit : 0) * M * CP * 4, st);
