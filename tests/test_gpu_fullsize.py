@@ -2,7 +2,8 @@
 times: the Llama-2-7B-shaped FFN layer (batch 8 x seq 512, d 4096, d_ff 11008,
 25% output tokens, SVD rank 8, LoRA rank 16, sparsity 50%) and the
 Llama-2-7B-shaped attention projections (batch 4 x seq 1024, 32 heads x 128,
-q/k sliced at 50% per head by QK-norm, v/o dense LoRA rank 16).
+q/k sliced at 50% per head by QK-norm; v/o dense LoRA rank 16, and the v/o
+variant sliced by the per-head L2 estimate).
 
 The estimator factors are the construction's exact top-r singular triplets
 (the weights are built from them), so both sides score with the same L, U.
@@ -104,3 +105,90 @@ def test_attention_projections_llama2_7b_full_size(L):
         for what, got, want in (("Y_ctx", Yc, Yc_o), ("Y_out", Yo, Yo_o), ("dX", dX, dX_o),
                                 ("dA", dA, dA_o), ("dB", dB, dB_o)):
             assert_close(host(got), want, TOL["bf16"], f"{name}:{what}")
+
+
+def _linear_pair(L, side, tok, X_ctx, X_out, W0, A, B, s, sel, dY_ctx, dY_out):
+    """One linear's forward and backward on the GPU (bf16) and in the oracle,
+    on the same channel set; returns the list of (name, got, want)."""
+    bf = torch.bfloat16
+    C, Orow = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    n, k = W0.shape
+    code = {"none": L.SLICE_NONE, "out_rows": L.SLICE_OUT_ROWS, "in_cols": L.SLICE_IN_COLS}[side]
+    Yc_o, Yo_o, XA_o = O.linear_fwd(side, X_ctx, X_out, tok.batch, tok.seq, tok.ctx_len, W0, A,
+                                    B, s, sel)
+    dXc_o, dXo_o, dA_o, dB_o = O.linear_bwd(side, X_ctx, X_out, XA_o, dY_ctx, dY_out, tok.batch,
+                                            tok.seq, tok.ctx_len, W0, A, B, s, sel)
+    Wdev = dev(W0.T.copy() if side == "in_cols" else W0, bf)
+    Ad_, Bd_ = dev(A, bf), dev(B, bf)
+    idx_d = dev(sel, torch.int32) if sel is not None else None
+    Xc = dev(X_ctx, bf)
+    Xo = dev(X_out, bf) if X_out is not None else None
+    Yc = torch.zeros(Yc_o.shape, dtype=bf, device="cuda")
+    Yo = torch.zeros(Yo_o.shape, dtype=bf, device="cuda") if Yo_o is not None else None
+    XA = torch.zeros(tok.T, A.shape[0], device="cuda")
+    L.slora_linear_fwd(code, tok.batch, tok.seq, tok.ctx_len, k, n, Wdev, Ad_, Bd_, s, idx_d, Xc,
+                       Yc, X_out=Xo, Y_out=Yo, XA_save=XA)
+    dXc = torch.zeros(dXc_o.shape, dtype=bf, device="cuda")
+    dXo = torch.zeros(dXo_o.shape, dtype=bf, device="cuda") if dXo_o is not None else None
+    dA = torch.zeros(A.shape, device="cuda")
+    dB = torch.zeros(B.shape, device="cuda")
+    L.slora_linear_bwd(code, tok.batch, tok.seq, tok.ctx_len, k, n, Wdev, Ad_, Bd_, s, idx_d, Xc,
+                       XA, dev(dY_ctx, bf), dXc, dA, dB, X_out=Xo,
+                       dY_out=dev(dY_out, bf) if dY_out is not None else None, dX_out=dXo)
+    torch.cuda.synchronize()
+    out = [("Y_ctx", Yc, Yc_o), ("XA", XA, XA_o), ("dX_ctx", dXc, dXc_o), ("dA", dA, dA_o),
+           ("dB", dB, dB_o)]
+    if Yo is not None:
+        out.append(("Y_out", Yo, Yo_o))
+    if dXo is not None:
+        out.append(("dX_out", dXo, dXo_o))
+    return out
+
+
+def test_value_and_output_projections_llama2_7b_full_size(L):
+    """The attention workload's v and o LoRA linears at full size (batch 4 x
+    seq 1024, d 4096, 32 heads x 128, LoRA rank 16): v dense (SLICE_NONE); then
+    the v/o projection-set variant, v sliced on its output channels
+    (SLICE_OUT_ROWS) and o on the matching input channels (SLICE_IN_COLS) by
+    the per-head L2 estimate at 50%, the GPU's selection checked against the
+    oracle's and both linears compared on the oracle's channel sets."""
+    w = synth.WORKLOADS[2]
+    tok = synth.Tokens.uniform(w["batch"], w["seq"], w["out_frac"])
+    H, hd, d, rs, r = w["heads"], w["head_dim"], w["d"], w["r_svd"], w["r_lora"]
+    rnd = synth.round_bf16
+    X = rnd(synth.gaussian((tok.T, d), 1.0, 2200))
+    Wv = synth.decaying_weight(H * hd, d, 2201, bf16=True, fast=True)
+    Wo = synth.decaying_weight(d, H * hd, 2202, bf16=True, fast=True)
+    Av, Bv = rnd(synth.gaussian((r, d), 0.02, 2203)), rnd(synth.gaussian((H * hd, r), 0.02, 2204))
+    Ao, Bo = rnd(synth.gaussian((r, H * hd), 0.02, 2205)), rnd(synth.gaussian((d, r), 0.02, 2206))
+    attn = rnd(synth.gaussian((tok.T, H * hd), 1.0, 2207))  # stand-in for the attention output
+    dYv = rnd(synth.gaussian((tok.T, H * hd), 1.0, 2208))
+    dYo = rnd(synth.gaussian((tok.T, d), 1.0, 2209))
+    C, Orow = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    # v dense
+    for what, got, want in _linear_pair(L, "none", tok, X, None, Wv.W, Av, Bv, 1.0, None, dYv,
+                                        None):
+        assert_close(host(got), want, TOL["bf16"], f"v dense:{what}")
+    # the v/o selection: GPU estimator against the oracle's
+    Lv, Uv = _factors(Wv, rs)
+    io, iv, kh, sc = O.estimate_select_l2(X, tok.batch, tok.seq, tok.ctx_len, Lv, Uv, H, H, hd,
+                                          0.5)
+    idx = torch.full((2 * H * hd,), -1, dtype=torch.int32, device="cuda")
+    f = lambda a: dev(a, torch.float32)
+    k = L.slora_estimate_select(L.CRIT_L2, dev(X, torch.bfloat16), tok.batch, tok.seq,
+                                tok.ctx_len, f(Lv), f(Uv), f(Lv), f(Uv), rs, 0.5, idx, heads=H,
+                                kv_heads=H, head_dim=hd)
+    torch.cuda.synchronize()
+    assert k == kh == 64
+    gi = host(idx).astype(np.int64)
+    for h in range(H):
+        check_selection(gi[H * kh + h * kh:H * kh + (h + 1) * kh] - h * hd,
+                        iv[h * kh:(h + 1) * kh] - h * hd, sc[h], kh, f"v head {h}")
+    # v sliced on output channels iv, o on input channels io (the same channels)
+    assert np.array_equal(io, iv)
+    for what, got, want in _linear_pair(L, "out_rows", tok, X, None, Wv.W, Av, Bv, 1.0, iv,
+                                        rnd(dYv[C][:, iv]), dYv[Orow]):
+        assert_close(host(got), want, TOL["bf16"], f"v sliced:{what}")
+    for what, got, want in _linear_pair(L, "in_cols", tok, attn[C][:, io], attn[Orow], Wo.W, Ao,
+                                        Bo, 1.0, io, dYo, None):
+        assert_close(host(got), want, TOL["bf16"], f"o sliced:{what}")
