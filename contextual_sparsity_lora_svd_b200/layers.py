@@ -74,6 +74,8 @@ class FfnLayer(_Runner):
     and the fp32 estimator factors Lg, Ug, Lu, Uu."""
 
     def __init__(self, w, d, d_ff, r_svd, r_lora, scale, batch, seq, ctx_len, sparsity, X, dOut):
+        # the argument lists hold raw device addresses of w, X and dOut, which
+        # the runner keeps alive
         self.w, self.d, self.d_ff, self.r = w, d, d_ff, r_lora
         self.sparsity = float(sparsity)
         T = batch * seq
@@ -117,6 +119,9 @@ class AttnLinears(_Runner):
     def __init__(self, w, d, heads, kv_heads, head_dim, r_svd, r_lora, scale, batch, seq, ctx_len,
                  qk_sparsity, X, attn_out, dY_o, dq, dk, dv, pairs=False, vo_sparsity=0.0):
         self.w = w
+        # the argument lists below hold raw device addresses: keep every
+        # caller tensor they point into alive as long as the runner
+        self._inputs = (X, attn_out, dY_o, dq, dk, dv)
         H, KV, hd = heads, kv_heads, head_dim
         nq, nkv = H * hd, KV * hd
         T = batch * seq

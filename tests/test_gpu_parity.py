@@ -173,6 +173,55 @@ def test_linear_fwd_bwd(L, bf16, side):
     assert_close(host(dB), dB_o, tol, "dB")
 
 
+def test_linear_fwd_bwd_single_tile(L):
+    """Every slice side with 128 rows in total (one M tile) and widths that are
+    whole multiples of the tile: k = n = 128."""
+    tok = _tok(2, 64, [48, 40])
+    k, n, r, s = 128, 128, 8, 1.0
+    X, W0, A, B = _lin(True, tok, k, n, r, 650)
+    C, Orow = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
+    idx_o = np.sort(synth.rng(651).choice(n, size=64, replace=False))
+    bf = torch.bfloat16
+    for side in ("none", "out_rows", "in_cols"):
+        code = {"none": L.SLICE_NONE, "out_rows": L.SLICE_OUT_ROWS,
+                "in_cols": L.SLICE_IN_COLS}[side]
+        sel = None if side == "none" else idx_o
+        if side == "in_cols":
+            Xin, Xout, Wdev = X[C][:, idx_o], X[Orow], dev(W0.T.copy(), bf)
+        else:
+            Xin, Xout, Wdev = X, None, dev(W0, bf)
+        Yc_o, Yo_o, XA_o = O.linear_fwd(side, Xin, Xout, tok.batch, tok.seq, tok.ctx_len, W0, A, B,
+                                        s, sel)
+        Yc = torch.zeros(Yc_o.shape, dtype=bf, device="cuda")
+        Yo = torch.zeros(Yo_o.shape, dtype=bf, device="cuda") if Yo_o is not None else None
+        XA = torch.zeros(tok.T, r, device="cuda")
+        idx = dev(sel, torch.int32) if sel is not None else None
+        Xin_d, Xout_d = dev(Xin, bf), (dev(Xout, bf) if Xout is not None else None)
+        L.slora_linear_fwd(code, tok.batch, tok.seq, tok.ctx_len, k, n, Wdev, dev(A, bf),
+                           dev(B, bf), s, idx, Xin_d, Yc, X_out=Xout_d, Y_out=Yo, XA_save=XA)
+        rg = synth.rng(652)
+        dY1 = synth.round_bf16(rg.standard_normal(Yc_o.shape))
+        dY2 = synth.round_bf16(rg.standard_normal(Yo_o.shape)) if Yo_o is not None else None
+        dXc_o, dXo_o, dA_o, dB_o = O.linear_bwd(side, Xin, Xout, XA_o, dY1, dY2, tok.batch,
+                                                tok.seq, tok.ctx_len, W0, A, B, s, sel)
+        dXc = torch.zeros(dXc_o.shape, dtype=bf, device="cuda")
+        dXo = torch.zeros(dXo_o.shape, dtype=bf, device="cuda") if dXo_o is not None else None
+        dA, dB = torch.zeros(r, k, device="cuda"), torch.zeros(n, r, device="cuda")
+        L.slora_linear_bwd(code, tok.batch, tok.seq, tok.ctx_len, k, n, Wdev, dev(A, bf),
+                           dev(B, bf), s, idx, Xin_d, XA, dev(dY1, bf), dXc, dA, dB, X_out=Xout_d,
+                           dY_out=dev(dY2, bf) if dY2 is not None else None, dX_out=dXo)
+        torch.cuda.synchronize()
+        tol = TOL["bf16"]
+        assert_close(host(Yc), Yc_o, tol, f"{side} Y_ctx")
+        if Yo is not None:
+            assert_close(host(Yo), Yo_o, tol, f"{side} Y_out")
+        assert_close(host(dXc), dXc_o, tol, f"{side} dX_ctx")
+        if dXo is not None:
+            assert_close(host(dXo), dXo_o, tol, f"{side} dX_out")
+        assert_close(host(dA), dA_o, tol, f"{side} dA")
+        assert_close(host(dB), dB_o, tol, f"{side} dB")
+
+
 # --------------------------------------------------------------------- FFN
 def _ffn_lay(case, r_svd):
     lay = dict(Wg=case.Wg.W, Wu=case.Wu.W, Wd=case.Wd.W, Ag=case.Ag, Bg=case.Bg, Au=case.Au,
