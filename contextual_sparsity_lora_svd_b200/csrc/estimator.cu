@@ -7,25 +7,25 @@
 // query-key product) and the per-input choice of active channels.
 //
 // Kernels
-//   ffn_score_select_kernel  activation-norm score of the SwiGLU channels:
-//       the rank-r dot products g_hat = P_g U_g^T, u_hat = P_u U_u^T run on the
-//       tensor cores (mma.sync, both fp32 operands split into three bf16 terms,
-//       the six significant cross products packed along K), the silu and the
-//       square-sum on the CUDA cores / MUFU.  Partial sums per (token split,
-//       channel); the last split of a channel block to arrive sums them in a
-//       fixed order (fp64), the last channel block to finish runs the top-k.
+//   ffn_score_fma_kernel / ffn_score_mma_kernel  activation-norm score of
+//       the SwiGLU channels: the rank-r dot products g_hat = P_g U_g^T,
+//       u_hat = P_u U_u^T on the FMA pipe as packed f32x2 pairs (r <= 16) or
+//       on the tensor cores (mma.sync, both fp32 operands split into three
+//       bf16 terms, the six significant cross products packed along K; larger
+//       r), the silu and the square-sum on the CUDA cores / MUFU.  Partial
+//       sums per (token split, channel); the last split of a channel block to
+//       arrive sums them in a fixed order (fp64).
 //   gram_partial_kernel      r x r Gram matrices of P over token chunks, fp64;
 //       the last chunk to arrive sums them in a fixed order.
-//   norm_score_select_kernel per-channel norms as Gram quadratic forms
+//   norm_score_kernel        per-channel norms as Gram quadratic forms
 //       ||Y_hat[:, c]||^2 = u_c^T (P^T P) u_c, combined per criterion (QK-norm
-//       product with grouped query heads, plain L2 norm, rotate-half pairs);
-//       the last channel block of a group runs that group's top-k.
-//   topk_kernel              top-k per group for score vectors too long for
-//       the fused select.
-// Top-k: bisection on the fp32 bit pattern of the scores (non-negative, so
-// unsigned order is numeric order), keys held in registers, block-wide counts
-// per step; then ties at the threshold go to the lower index and the indices
-// are written in ascending order (each thread owns a contiguous index range).
+//       product with grouped query heads, plain L2 norm, rotate-half pairs).
+//   topk_kernel              top-k per group, one block per group.
+// Top-k (block_topk): the scores' fp32 bit patterns are the keys (scores are
+// non-negative, so unsigned order is numeric order), held in registers; radix
+// passes over the bits below the keys' common prefix find the k-th largest
+// key; ties at it go to the lower index and the indices are written in
+// ascending order (each thread owns a contiguous index range).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -33,6 +33,11 @@
 #include "estimator.cuh"
 
 namespace slora {
+
+// Raised (instead of faulting) when a score kernel finds its shared staging
+// buffer off its 16-byte alignment; reported by est_check_error.
+__device__ int g_est_error = 0;
+
 namespace {
 
 // ------------------------------------------------------------------ helpers
@@ -70,43 +75,50 @@ __device__ __forceinline__ uint32_t pack2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
 }
 
 // ------------------------------------------------------------ block reductions
-// Scratch: kRedWords words of shared memory, double-buffered by `parity` so a
-// reduction needs one barrier.
+// The top-k's shared memory is touched only through these scalar 32-bit
+// accesses on shared-window addresses (explicit ld/st/red.shared.u32, so every
+// access keeps its own 4-byte width and order).
+__device__ __forceinline__ uint32_t sh_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void sh_st(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t sh_ld(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sh_add(uint32_t a, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+// Block-wide reductions and scan over B threads.  `s` is the shared address
+// of 2 x B/32 words, double-buffered by `parity` so each call needs one
+// barrier.
 template <int B>
 struct BlockRed {
   static constexpr int NW = B / 32;
-  uint32_t* s;  // [2][NW]
+  uint32_t s;
   int parity = 0;
-  __device__ uint32_t sum(uint32_t v) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    v = __reduce_add_sync(0xffffffffu, v);
-    if (lane == 0) s[parity * NW + w] = v;
-    __syncthreads();
-    uint32_t t = 0;
-#pragma unroll
-    for (int i = 0; i < NW; ++i) t += s[parity * NW + i];
-    parity ^= 1;
-    return t;
-  }
+  __device__ uint32_t slot(int i) const { return s + 4u * uint32_t(parity * NW + i); }
   __device__ uint32_t min(uint32_t v) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     v = __reduce_min_sync(0xffffffffu, v);
-    if (lane == 0) s[parity * NW + w] = v;
+    if (lane == 0) sh_st(slot(w), v);
     __syncthreads();
     uint32_t t = 0xffffffffu;
-#pragma unroll
-    for (int i = 0; i < NW; ++i) t = ::min(t, s[parity * NW + i]);
+    for (int i = 0; i < NW; ++i) t = ::min(t, sh_ld(slot(i)));
     parity ^= 1;
     return t;
   }
   __device__ uint32_t max(uint32_t v) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     v = __reduce_max_sync(0xffffffffu, v);
-    if (lane == 0) s[parity * NW + w] = v;
+    if (lane == 0) sh_st(slot(w), v);
     __syncthreads();
     uint32_t t = 0;
-#pragma unroll
-    for (int i = 0; i < NW; ++i) t = ::max(t, s[parity * NW + i]);
+    for (int i = 0; i < NW; ++i) t = ::max(t, sh_ld(slot(i)));
     parity ^= 1;
     return t;
   }
@@ -116,15 +128,13 @@ struct BlockRed {
     uint32_t inc = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, inc, off);
-      if (lane >= off) inc += o;
+      const uint32_t up = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += up;
     }
-    if (lane == 31) s[parity * NW + w] = inc;
+    if (lane == 31) sh_st(slot(w), inc);
     __syncthreads();
     uint32_t base = 0;
-#pragma unroll
-    for (int i = 0; i < NW; ++i)
-      if (i < w) base += s[parity * NW + i];
+    for (int i = 0; i < w; ++i) base += sh_ld(slot(i));
     parity ^= 1;
     return base + inc - v;
   }
@@ -143,7 +153,7 @@ struct TopkOut {
   int pair_half = 0; // > 0: keys are rotate-half pairs (p, p + pair_half)
 };
 
-__device__ __forceinline__ void topk_emit(const TopkOut& o, int g, int ktot, int kp, int pos,
+__device__ __forceinline__ void topk_emit(const TopkOut o, int g, int ktot, int kp, int pos,
                                           int c) {
   for (int j = 0; j < o.rep; ++j) {
     const int h = g * o.rep + j;
@@ -159,13 +169,27 @@ __device__ __forceinline__ void topk_emit(const TopkOut& o, int g, int ktot, int
 }
 
 // The k largest of n scores (ties to the lower index), written through `o`
-// for group g.  All B threads of the block call it; n <= B * MAXM.  Scores
-// are read through L2 (they may come from other blocks of the same launch).
+// for group g.  All B threads of the block call it; n <= B * MAXM.
+//   1. keys (score bits) in registers, each thread a contiguous index range;
+//   2. the keys share their bits above hb, the highest bit where the largest
+//      and the smallest key differ; below it, radix passes of up to 8 bits
+//      each (at most four) narrow the prefix of the k-th largest key: a pass
+//      counts the keys that match the prefix so far in per-warp 256-bin
+//      histograms (`hist`, [B/32][256] words), sums them, and warp 0 finds
+//      the digit holding the wanted rank; the keys in the digits above it
+//      are all kept (`above`) and the rank left is sought inside the digit;
+//   3. after the last pass the prefix is the k-th largest key tau itself:
+//      every key above tau is kept, and of the keys equal to tau the first
+//      ones in index order; block scans give each thread its output
+//      position, so the indices come out ascending.
+// Shared memory (32-bit shared-window addresses): `red` 2 x B/32 words,
+// `hist` B/32 x 256 words, `bc` 4 broadcast words.
 template <int B, int MAXM>
-__device__ void block_topk(const float* __restrict__ sc, int n, int k, const TopkOut& o, int g,
-                           uint32_t* red_smem) {
+__device__ void block_topk(const float* __restrict__ sc, int n, int k, const TopkOut o, int g,
+                           uint32_t red_smem, uint32_t hist, uint32_t bc) {
+  constexpr int NW = B / 32;
   BlockRed<B> red{red_smem};
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int kp = k;
   const int ktot = o.pair_half ? 2 * k : k;
   if (k <= 0 || n <= 0) return;
@@ -189,53 +213,87 @@ __device__ void block_topk(const float* __restrict__ sc, int n, int k, const Top
   }
   kmin = red.min(kmin);
   kmax = red.max(kmax);
-  // largest v with count(key >= v) >= k: count(>= lo) >= k > count(>= hi)
-  uint32_t lo = kmin, hi = kmax + 1u;
-  bool exact = false;
-  while (hi - lo > 1u) {
-    const uint32_t mid = lo + (hi - lo) / 2u;
-    uint32_t c = 0;
+  // tau: the k-th largest key; above: how many keys exceed it
+  uint32_t tau = kmin, above = 0;
+  if (kmin != kmax) {
+    int top = 31 - __clz(int(kmin ^ kmax));  // <= 30: keys are below 2^31
+    uint32_t prefix = kmin & ~((2u << top) - 1u);
+    uint32_t need = uint32_t(k);  // rank of tau among the keys matching prefix
+    while (true) {
+      const int shift = top > 7 ? top - 7 : 0;
+      const uint32_t dmask = (2u << (top - shift)) - 1u;  // digit = bits top .. shift
+      const uint32_t pmask = ~((2u << top) - 1u);         // bits above top
+      for (int i = tid; i < NW * 256; i += B) sh_st(hist + 4u * uint32_t(i), 0u);
+      __syncthreads();
 #pragma unroll
-    for (int i = 0; i < MAXM; ++i) c += (i < mt && key[i] >= mid) ? 1u : 0u;
-    c = red.sum(c);
-    if (c == uint32_t(k)) {  // exactly the keys >= mid: no ties to break
-      lo = mid;
-      exact = true;
-      break;
+      for (int i = 0; i < MAXM; ++i)
+        if (i < mt && (key[i] & pmask) == prefix)
+          sh_add(hist + 4u * (uint32_t(w) * 256u + ((key[i] >> shift) & dmask)), 1u);
+      __syncthreads();
+      for (int d = tid; d < 256; d += B) {
+        uint32_t t = 0;
+        for (int v = 0; v < NW; ++v) t += sh_ld(hist + 4u * uint32_t(v * 256 + d));
+        sh_st(hist + 4u * uint32_t(d), t);  // warp 0's row now holds the totals
+      }
+      __syncthreads();
+      if (w == 0) {  // lane l owns digits 255-8l .. 248-8l, scanned from the top
+        uint32_t own = 0;
+        for (int i = 0; i < 8; ++i) own += sh_ld(hist + 4u * uint32_t(255 - 8 * lane - i));
+        uint32_t incl = own;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t x = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += x;
+        }
+        const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need);
+        if (lane == __ffs(hit) - 1) {
+          uint32_t cum = incl - own;
+          for (int i = 0; i < 8; ++i) {
+            const int dg = 255 - 8 * lane - i;
+            const uint32_t h = sh_ld(hist + 4u * uint32_t(dg));
+            if (cum + h >= need) {
+              sh_st(bc, uint32_t(dg));
+              sh_st(bc + 4u, cum);  // keys of this prefix in higher digits
+              break;
+            }
+            cum += h;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t dstar = sh_ld(bc), higher = sh_ld(bc + 4u);
+      above += higher;
+      need -= higher;
+      prefix |= dstar << shift;
+      if (shift == 0) break;
+      top = shift - 1;
     }
-    if (c > uint32_t(k)) lo = mid; else hi = mid;
+    tau = prefix;
   }
-  // keep every key above lo; of the keys equal to lo keep the first `want`
+  // keep every key above tau; of the keys equal to tau the first ones
   uint32_t cgt = 0, ceq = 0;
 #pragma unroll
   for (int i = 0; i < MAXM; ++i) {
     if (i < mt) {
-      if (exact ? key[i] >= lo : key[i] > lo) ++cgt;
-      else if (!exact && key[i] == lo) ++ceq;
+      if (key[i] > tau) ++cgt;
+      else if (key[i] == tau) ++ceq;
     }
   }
-  const uint32_t want = exact ? 0u : uint32_t(k) - red.sum(cgt);
+  const uint32_t want = uint32_t(k) - above;
   const uint32_t tie_before = red.excl_scan(ceq);
-  const uint32_t take_eq =
-      want > tie_before ? ::min(ceq, want - tie_before) : 0u;
+  const uint32_t take_eq = want > tie_before ? ::min(ceq, want - tie_before) : 0u;
   int pos = int(red.excl_scan(cgt + take_eq));
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < MAXM; ++i) {
     if (i < mt) {
       const uint32_t kv = key[i];
-      bool s;
-      if (exact) {
-        s = kv >= lo;
-      } else if (kv > lo) {
-        s = true;
-      } else if (kv == lo) {
-        s = taken < take_eq;
+      bool sel = kv > tau;
+      if (kv == tau) {
+        sel = taken < take_eq;
         ++taken;
-      } else {
-        s = false;
       }
-      if (s) topk_emit(o, g, ktot, kp, pos++, i0 + i);
+      if (sel) topk_emit(o, g, ktot, kp, pos++, i0 + i);
     }
   }
 }
@@ -259,7 +317,6 @@ constexpr int score_nt(int C) { return C == 1 ? 2 : 1; }
 // bank-conflict free
 constexpr int score_tw(int C) { return 24 * C + 4; }
 constexpr int score_stage_bytes(int C) { return kStageTokens * score_tw(C) * 4; }
-constexpr int kFusedSelMaxM = 64;  // fused select: n <= 256 * 64 keys
 
 struct ScoreArgs {
   const float* P;        // [rows x ldp] fp32: P_g in columns [0, r), P_u in [r, 2r)
@@ -274,18 +331,180 @@ struct ScoreArgs {
   int64_t chunk;         // tokens per split (multiple of 16)
   float* partial;        // [nsplit x n]
   float* scores;         // [n]
-  unsigned* counters;    // [nblocks + 1], zero on entry
-  int select;            // run the top-k in the last block
-  int k;
-  int32_t* idx_out;
+  unsigned* counters;    // [nblocks], zero on entry
 };
 
+// Common end of the score kernels: the last split of a channel block to
+// arrive sums the block's partials in split order (fp64) and writes its
+// scores.  `s_last` is one word of the kernel's shared memory.
+template <int CH>
+__device__ void score_tail(const ScoreArgs& a, int64_t cb, unsigned* s_last) {
+  const int tid = threadIdx.x;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) *s_last = (atomicAdd(&a.counters[cb], 1u) + 1u == unsigned(a.nsplit)) ? 1u : 0u;
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  for (int c = tid; c < CH; c += kScoreThreads) {
+    const int64_t j = cb * CH + c;
+    if (j >= a.n) break;
+    double sum = 0.0;
+    for (int p = 0; p < a.nsplit; ++p) sum += double(__ldcg(a.partial + int64_t(p) * a.n + j));
+    a.scores[j] = float(sqrt(sum));
+  }
+}
+
+// ---- packed-FMA score kernel (rank <= 16)
+// Thread t owns NPAIR pairs of adjacent channels (j, j + 1) and keeps their
+// rows of U_g and U_u in registers as f32x2 pairs; each context token's
+// projected row (P_g | P_u) is staged once per block in shared memory with
+// every value duplicated ({v, v}), so one fma.rn.f32x2 advances the dot
+// products of both channels of a pair.  The silu tail runs on the pairs too
+// (exp and reciprocal stay scalar on the MUFU unit).  Legacy mma.sync issues
+// at a small fraction of the FMA pipe's rate on this GPU, so at rank <= 16
+// the dot products are cheaper on the FMA pipe.
+__device__ __forceinline__ unsigned long long pack_f2(float lo, float hi) {
+  unsigned long long v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
+}
+__device__ __forceinline__ float2 unpack_f2(unsigned long long v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fmul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr int kFmaTokens = 64;  // tokens staged per round
+template <int RP>
+constexpr int fma_npair() { return RP <= 8 ? 2 : 1; }
+template <int RP>
+constexpr int fma_channels() { return kScoreThreads * 2 * fma_npair<RP>(); }
+
+template <int RP>
+__global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const ScoreArgs a) {
+  constexpr int NP = fma_npair<RP>(), CH = fma_channels<RP>();
+  __shared__ __align__(16) unsigned long long sp[kFmaTokens][2 * RP];  // {v, v} pairs
+  __shared__ unsigned s_last;
+  const int tid = threadIdx.x;
+  const int64_t cb = blockIdx.x;
+  const int sp_id = blockIdx.y;
+  const int r = a.r;
+  if (reinterpret_cast<uintptr_t>(&sp[0][0]) & 15u) {  // the 16-byte loads below need it
+    if (tid == 0) atomicExch(&g_est_error, 1);
+    return;
+  }
+  // this thread's channel pairs: j = cb*CH + 2*(tid + kScoreThreads*p) + {0, 1}
+  unsigned long long ug[NP][RP], uu[NP][RP], acc[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int64_t j = cb * CH + 2 * (tid + kScoreThreads * p);
+#pragma unroll
+    for (int q = 0; q < RP; ++q) {
+      const bool ok = q < r;
+      const float g0 = (ok && j < a.n) ? a.Ug[j * r + q] : 0.0f;
+      const float g1 = (ok && j + 1 < a.n) ? a.Ug[(j + 1) * r + q] : 0.0f;
+      const float u0 = (ok && j < a.n) ? a.Uu[j * r + q] : 0.0f;
+      const float u1 = (ok && j + 1 < a.n) ? a.Uu[(j + 1) * r + q] : 0.0f;
+      ug[p][q] = pack_f2(g0, g1);
+      uu[p][q] = pack_f2(u0, u1);
+    }
+    acc[p] = 0ull;
+  }
+  const unsigned long long neg_log2e = pack_f2(-1.4426950408889634f, -1.4426950408889634f);
+  const unsigned long long one2 = pack_f2(1.0f, 1.0f);
+  const int64_t t0 = int64_t(sp_id) * a.chunk;
+  const int64_t t1 = ::min(a.T_C, t0 + a.chunk);
+  for (int64_t tb = t0; tb < t1; tb += kFmaTokens) {
+    const int nt = int(::min(int64_t(kFmaTokens), t1 - tb));
+    __syncthreads();
+    for (int e = tid; e < nt * 2 * RP; e += kScoreThreads) {
+      const int tt = e / (2 * RP), q = e % (2 * RP), mat = q / RP, qq = q % RP;
+      float v = 0.0f;
+      if (qq < r) {
+        const int64_t row = a.pmap ? int64_t(a.pmap[tb + tt]) : tb + tt;
+        v = a.P[row * a.ldp + mat * r + qq];
+      }
+      sp[tt][q] = pack_f2(v, v);
+    }
+    __syncthreads();
+    for (int tt = 0; tt < nt; ++tt) {
+      const ulonglong2* row = reinterpret_cast<const ulonglong2*>(sp[tt]);
+      unsigned long long g2[NP], u2[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) g2[p] = u2[p] = 0ull;
+#pragma unroll
+      for (int q2 = 0; q2 < RP / 2; ++q2) {
+        const ulonglong2 pg = row[q2];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          g2[p] = ffma2(pg.x, ug[p][2 * q2], g2[p]);
+          g2[p] = ffma2(pg.y, ug[p][2 * q2 + 1], g2[p]);
+        }
+      }
+#pragma unroll
+      for (int q2 = 0; q2 < RP / 2; ++q2) {
+        const ulonglong2 pu = row[RP / 2 + q2];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          u2[p] = ffma2(pu.x, uu[p][2 * q2], u2[p]);
+          u2[p] = ffma2(pu.y, uu[p][2 * q2 + 1], u2[p]);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        // silu(g) u = g u / (1 + 2^(-g log2 e)), on both channels of the pair
+        const float2 x = unpack_f2(fmul2(g2[p], neg_log2e));
+        const unsigned long long den = fadd2(pack_f2(ex2_approx(x.x), ex2_approx(x.y)), one2);
+        const float2 dn = unpack_f2(den);
+        const unsigned long long inv = pack_f2(rcp_approx(dn.x), rcp_approx(dn.y));
+        const unsigned long long v = fmul2(fmul2(g2[p], inv), u2[p]);
+        acc[p] = ffma2(v, v, acc[p]);
+      }
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < NP; ++p) {
+    const int64_t j = cb * CH + 2 * (tid + kScoreThreads * p);
+    const float2 f = unpack_f2(acc[p]);
+    float* dst = a.partial + int64_t(sp_id) * a.n + j;
+    if (j < a.n) dst[0] = f.x;
+    if (j + 1 < a.n) dst[1] = f.y;
+  }
+  score_tail<CH>(a, cb, &s_last);
+}
+
 template <int C>
-__global__ void __launch_bounds__(kScoreThreads) ffn_score_select_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads) ffn_score_mma_kernel(const ScoreArgs a) {
   constexpr int NT = score_nt(C), TW = score_tw(C), KB = 3 * C;
   constexpr int CH = kScoreWarps * NT * 8;  // channels per block
   extern __shared__ __align__(16) uint32_t s_stage[];
-  __shared__ uint32_t s_red[2 * kScoreWarps];
   __shared__ unsigned s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const int64_t cb = blockIdx.x;
@@ -420,31 +639,7 @@ __global__ void __launch_bounds__(kScoreThreads) ffn_score_select_kernel(const S
       if (j + 1 < a.n) dst[1] = acc[nt][1];
     }
   }
-  // the last split of this channel block sums the partials in split order
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.counters[cb], 1u) + 1u == unsigned(a.nsplit)) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int c = tid; c < CH; c += kScoreThreads) {
-    const int64_t j = cb * CH + c;
-    if (j >= a.n) break;
-    double s = 0.0;
-    for (int p = 0; p < a.nsplit; ++p) s += double(__ldcg(a.partial + int64_t(p) * a.n + j));
-    a.scores[j] = float(sqrt(s));
-  }
-  if (!a.select) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.counters[gridDim.x], 1u) + 1u == gridDim.x) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  TopkOut o;
-  o.a = a.idx_out;
-  o.N = int(a.n);
-  block_topk<kScoreThreads, kFusedSelMaxM>(a.scores, int(a.n), a.k, o, 0, s_red);
+  score_tail<CH>(a, cb, &s_last);
 }
 
 // ------------------------------------------------------------ Gram criterion
@@ -507,10 +702,15 @@ __global__ void __launch_bounds__(kGramThreads) gram_partial_kernel(const GramAr
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int e = tid; e < ne; e += kGramThreads) {
+  // one warp per entry: lanes load the chunks' partials (all loads in flight
+  // at once) and a fixed-order shuffle tree sums them
+  const int lane = tid & 31, wid = tid >> 5;
+  for (int e = wid; e < ne; e += kGramThreads / 32) {
     double s = 0.0;
-    for (unsigned b = 0; b < gridDim.x; ++b) s += __ldcg(a.part + int64_t(b) * ne + e);
-    a.gram[e] = s;
+    for (unsigned b = lane; b < gridDim.x; b += 32) s += __ldcg(a.part + int64_t(b) * ne + e);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_down_sync(0xffffffffu, s, off);
+    if (lane == 0) a.gram[e] = s;
   }
 }
 
@@ -526,11 +726,7 @@ struct NormArgs {
   int N;                // channels per head
   int rep;              // query heads per group (QK)
   int nkeys;            // keys per group: N, or N / 2 with pairs
-  int blocks_per_group;
   float* scores;        // [groups x nkeys]
-  unsigned* counters;   // [groups], zero on entry
-  int k;                // keys kept per group
-  TopkOut out;
 };
 
 __device__ __forceinline__ double quad_form(const double* G, const float* u, int r) {
@@ -543,97 +739,99 @@ __device__ __forceinline__ double quad_form(const double* G, const float* u, int
   return s > 0.0 ? s : 0.0;
 }
 
-template <int MAXM>
-__global__ void __launch_bounds__(kNormThreads) norm_score_select_kernel(const NormArgs a) {
+__global__ void __launch_bounds__(kNormThreads) norm_score_kernel(const NormArgs a) {
   __shared__ double sg[2 * 48 * 48];
-  __shared__ uint32_t s_red[2 * (kNormThreads / 32)];
-  __shared__ unsigned s_last;
   const int tid = threadIdx.x, r = a.r;
   const int nmat = a.mode == kCritModeQK ? 2 : 1;
   for (int e = tid; e < nmat * r * r; e += kNormThreads) sg[e] = a.gram[e];
   __syncthreads();
   const int grp = blockIdx.y;
   const int key = blockIdx.x * kNormThreads + tid;
-  if (key < a.nkeys) {
-    // norm^2 of channel c of head h of matrix m
-    auto nsq = [&](int m, int h, int c) {
-      const float* U = m == 0 ? a.U0 : a.U1;
-      return quad_form(sg + m * r * r, U + (int64_t(h) * a.N + c) * r, r);
-    };
-    auto nrm = [&](int m, int h) {
-      double s = nsq(m, h, key);
-      if (a.pair_half) s += nsq(m, h, key + a.pair_half);
-      return sqrt(s);
-    };
-    double score;
-    if (a.mode == kCritModeQK) {
-      double qs = 0.0;
-      for (int j = 0; j < a.rep; ++j) qs += nrm(0, grp * a.rep + j);
-      score = nrm(1, grp) * qs;
-    } else {
-      score = nrm(0, grp);
-    }
-    a.scores[int64_t(grp) * a.nkeys + key] = float(score);
+  if (key >= a.nkeys) return;
+  // norm^2 of channel c of head h of matrix m
+  auto nsq = [&](int m, int h, int c) {
+    const float* U = m == 0 ? a.U0 : a.U1;
+    return quad_form(sg + m * r * r, U + (int64_t(h) * a.N + c) * r, r);
+  };
+  auto nrm = [&](int m, int h) {
+    double s = nsq(m, h, key);
+    if (a.pair_half) s += nsq(m, h, key + a.pair_half);
+    return sqrt(s);
+  };
+  double score;
+  if (a.mode == kCritModeQK) {
+    double qs = 0.0;
+    for (int j = 0; j < a.rep; ++j) qs += nrm(0, grp * a.rep + j);
+    score = nrm(1, grp) * qs;
+  } else {
+    score = nrm(0, grp);
   }
-  if (a.k <= 0) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0)
-    s_last = (atomicAdd(&a.counters[grp], 1u) + 1u == unsigned(a.blocks_per_group)) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  block_topk<kNormThreads, MAXM>(a.scores + int64_t(grp) * a.nkeys, a.nkeys, a.k, a.out, grp,
-                                 s_red);
+  a.scores[int64_t(grp) * a.nkeys + key] = float(score);
 }
 
-// ------------------------------------------------------ standalone top-k
+// ------------------------------------------------------------------ top-k
+// One block per group; the scratch lives in the kernel's own shared arrays.
 constexpr int kTopkThreads = 512;
-constexpr int kTopkMaxM = 64;
+constexpr int kTopkMaxM = 64;  // keys per thread: n <= 512 * 64
 
+template <int MAXM>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores,
                                                             int N, int k, TopkOut o) {
-  __shared__ uint32_t s_red[2 * (kTopkThreads / 32)];
-  block_topk<kTopkThreads, kTopkMaxM>(scores + int64_t(blockIdx.x) * N, N, k, o, blockIdx.x,
-                                      s_red);
+  __shared__ __align__(16) uint32_t s_red[2 * (kTopkThreads / 32)];
+  __shared__ __align__(16) uint32_t s_hist[(kTopkThreads / 32) * 256];
+  __shared__ __align__(16) uint32_t s_bc[4];
+  block_topk<kTopkThreads, MAXM>(scores + int64_t(blockIdx.x) * N, N, k, o, blockIdx.x,
+                                 sh_addr(s_red), sh_addr(s_hist), sh_addr(s_bc));
 }
 
 int rank_chunks(int r) { return r <= 8 ? 1 : (r <= 16 ? 2 : (r <= 24 ? 3 : (r <= 32 ? 4 : 6))); }
-int channels_per_block(int r) { return kScoreWarps * score_nt(rank_chunks(r)) * 8; }
+// Score kernel by rank: packed FMA for r <= 16, tensor cores above (whose
+// factor rows no longer fit the registers of the FMA form).
+int channels_per_block(int r) {
+  if (r <= 8) return fma_channels<8>();
+  if (r <= 16) return fma_channels<16>();
+  return kScoreWarps * score_nt(rank_chunks(r)) * 8;
+}
 
-template <int C>
-int score_blocks_per_sm_t() {
-  static int cached = 0;
-  if (!cached) {
-    int b = 0;
-    const int smem = score_stage_bytes(C);
-    if (cudaFuncSetAttribute(ffn_score_select_kernel<C>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, ffn_score_select_kernel<C>,
-                                                      kScoreThreads, smem) != cudaSuccess ||
-        b < 1) {
-      cudaGetLastError();
-      b = 1;
-    }
-    cached = b;
+template <class K>
+int blocks_per_sm_of(K kernel, int smem) {
+  int b = 0;
+  // the dynamic limit is raised whenever there is dynamic memory: static and
+  // dynamic together may pass 48 KB even when the dynamic part alone does not
+  if ((smem > 0 &&
+       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+           cudaSuccess) ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, kScoreThreads, smem) !=
+          cudaSuccess ||
+      b < 1) {
+    cudaGetLastError();
+    b = 1;
   }
-  return cached;
+  return b;
 }
 int score_blocks_per_sm(int r) {
-  switch (rank_chunks(r)) {
-    case 1: return score_blocks_per_sm_t<1>();
-    case 2: return score_blocks_per_sm_t<2>();
-    case 3: return score_blocks_per_sm_t<3>();
-    case 4: return score_blocks_per_sm_t<4>();
-    default: return score_blocks_per_sm_t<6>();
+  static int cached[5] = {0, 0, 0, 0, 0};
+  const int v = r <= 8 ? 0 : (r <= 16 ? 1 : (r <= 24 ? 2 : (r <= 32 ? 3 : 4)));
+  if (!cached[v]) {
+    switch (v) {
+      case 0: cached[v] = blocks_per_sm_of(ffn_score_fma_kernel<8>, 0); break;
+      case 1: cached[v] = blocks_per_sm_of(ffn_score_fma_kernel<16>, 0); break;
+      case 2: cached[v] = blocks_per_sm_of(ffn_score_mma_kernel<3>, score_stage_bytes(3)); break;
+      case 3: cached[v] = blocks_per_sm_of(ffn_score_mma_kernel<4>, score_stage_bytes(4)); break;
+      default: cached[v] = blocks_per_sm_of(ffn_score_mma_kernel<6>, score_stage_bytes(6));
+    }
   }
+  return cached[v];
 }
 
 template <int C>
-void launch_score(dim3 grid, const ScoreArgs& a, cudaStream_t st) {
-  score_blocks_per_sm_t<C>();  // sets the kernel's dynamic shared-memory limit once
+slora_status launch_score_mma(dim3 grid, const ScoreArgs& a, cudaStream_t st) {
   const int smem = score_stage_bytes(C);
-  ffn_score_select_kernel<C><<<grid, kScoreThreads, smem, st>>>(a);
+  // static (the top-k scratch) plus dynamic staging passes 48 KB
+  SLORA_CUDA(cudaFuncSetAttribute(ffn_score_mma_kernel<C>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  ffn_score_mma_kernel<C><<<grid, kScoreThreads, smem, st>>>(a);
+  return SLORA_OK;
 }
 
 }  // namespace
@@ -656,7 +854,8 @@ int ffn_score_splits(int64_t T_C, int64_t n, int r) {
 }
 
 int64_t estimator_counter_count(int64_t n, int r, int groups) {
-  return ffn_score_blocks(n, r) + 1 + std::max(groups, 1) + 1;
+  (void)groups;  // the score kernels count per channel block, the Gram pass in one word
+  return std::max<int64_t>(ffn_score_blocks(n, r), 1) + 1;
 }
 
 int64_t gram_blocks(int64_t T_C) {
@@ -664,35 +863,61 @@ int64_t gram_blocks(int64_t T_C) {
   return std::max<int64_t>(1, std::min<int64_t>(want, 64));
 }
 
+namespace {
+// One top-k block per group, the register array sized to the keys per thread.
+slora_status launch_topk(const float* scores, int groups, int N, int k, const TopkOut& o,
+                         cudaStream_t st) {
+  if (k <= 0 || groups <= 0) return SLORA_OK;
+  if (int64_t(N) > int64_t(kTopkThreads) * kTopkMaxM)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "top-k over %d keys per group exceeds the supported %d", N,
+               kTopkThreads * kTopkMaxM);
+  const int per_head = o.pair_half ? 2 * k : k;
+  LaunchScope ls(kSelect, double(groups) * N * 4 + double(groups) * per_head * 4 * (o.rep + 1),
+                 st);
+  const int m = (N + kTopkThreads - 1) / kTopkThreads;
+  if (m <= 8)
+    topk_kernel<8><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
+  else if (m <= 32)
+    topk_kernel<32><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
+  else
+    topk_kernel<kTopkMaxM><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+}  // namespace
+
 slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
                               const float* Ug, const float* Uu, int64_t n, int r, float* partial,
                               int nsplit, float* scores, unsigned* counters, int k,
                               int32_t* idx_out, cudaStream_t st) {
   if (n <= 0) return SLORA_OK;
-  const bool fused_select = n <= int64_t(kScoreThreads) * kFusedSelMaxM && idx_out;
   ScoreArgs a;
   a.P = P; a.ldp = ldp; a.pmap = pmap; a.T_C = T_C; a.Ug = Ug; a.Uu = Uu; a.n = n; a.r = r;
   a.nsplit = nsplit;
   a.chunk = T_C > 0 ? ((T_C + nsplit - 1) / nsplit + 15) / 16 * 16 : 16;
   a.partial = partial; a.scores = scores; a.counters = counters;
-  a.select = fused_select ? 1 : 0;
-  a.k = k; a.idx_out = idx_out;
   const dim3 grid(unsigned(ffn_score_blocks(n, r)), unsigned(nsplit));
   {
     // bytes: P rows of the context tokens, both factors, partials and scores
     LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 +
                                   double(nsplit) * n * 8 + double(n) * 4, st);
-    switch (rank_chunks(r)) {
-      case 1: launch_score<1>(grid, a, st); break;
-      case 2: launch_score<2>(grid, a, st); break;
-      case 3: launch_score<3>(grid, a, st); break;
-      case 4: launch_score<4>(grid, a, st); break;
-      default: launch_score<6>(grid, a, st); break;
-    }
+    if (r <= 8)
+      ffn_score_fma_kernel<8><<<grid, kScoreThreads, 0, st>>>(a);
+    else if (r <= 16)
+      ffn_score_fma_kernel<16><<<grid, kScoreThreads, 0, st>>>(a);
+    else if (r <= 24)
+      SLORA_TRY(launch_score_mma<3>(grid, a, st));
+    else if (r <= 32)
+      SLORA_TRY(launch_score_mma<4>(grid, a, st));
+    else
+      SLORA_TRY(launch_score_mma<6>(grid, a, st));
   }
   SLORA_CHECK_LAUNCH();
-  if (!fused_select && idx_out) SLORA_TRY(topk_select(scores, 1, int(n), k, 1, idx_out, nullptr, st));
-  return SLORA_OK;
+  if (!idx_out) return SLORA_OK;
+  TopkOut o;
+  o.a = idx_out;
+  o.N = int(n);
+  return launch_topk(scores, 1, int(n), k, o, st);
 }
 
 slora_status gram_scores_select(int mode, const float* P, int64_t ldp, const int32_t* pmap,
@@ -716,46 +941,38 @@ slora_status gram_scores_select(int mode, const float* P, int64_t ldp, const int
   na.pair_half = pairs ? N / 2 : 0;
   na.N = N; na.rep = rep;
   na.nkeys = pairs ? N / 2 : N;
-  na.blocks_per_group = (na.nkeys + kNormThreads - 1) / kNormThreads;
-  na.scores = scores; na.counters = counters + 1;
-  na.out.a = out_a; na.out.b = out_b; na.out.rep = rep; na.out.N = N;
-  na.out.pair_half = na.pair_half;
-  const bool fused_select = na.nkeys <= kNormThreads * kFusedSelMaxM && out_a;
-  na.k = fused_select ? k : 0;
-  const dim3 grid(unsigned(na.blocks_per_group), unsigned(groups));
+  na.scores = scores;
+  const dim3 grid(unsigned((na.nkeys + kNormThreads - 1) / kNormThreads), unsigned(groups));
   {
     const int nu = mode == kCritModeQK ? (rep + 1) : 1;
-    LaunchScope ls(kSelect, double(groups) * N * nu * r * 4 + double(groups) * na.nkeys * 4 +
-                                double(groups) * k * 4 * (rep + 1) * (pairs ? 2 : 1), st);
-    if (na.nkeys <= kNormThreads)
-      norm_score_select_kernel<1><<<grid, kNormThreads, 0, st>>>(na);
-    else
-      norm_score_select_kernel<kFusedSelMaxM><<<grid, kNormThreads, 0, st>>>(na);
+    LaunchScope ls(kSelect, double(groups) * N * nu * r * 4 + double(groups) * na.nkeys * 4, st);
+    norm_score_kernel<<<grid, kNormThreads, 0, st>>>(na);
   }
   SLORA_CHECK_LAUNCH();
-  if (!fused_select && out_a) {
-    TopkOut o = na.out;
-    LaunchScope ls(kSelect, double(groups) * na.nkeys * 4, st);
-    topk_kernel<<<unsigned(groups), kTopkThreads, 0, st>>>(scores, na.nkeys, k, o);
-    SLORA_CHECK_LAUNCH();
-  }
-  return SLORA_OK;
+  if (!out_a) return SLORA_OK;
+  TopkOut o;
+  o.a = out_a; o.b = out_b; o.rep = rep; o.N = N; o.pair_half = na.pair_half;
+  return launch_topk(scores, groups, na.nkeys, k, o, st);
 }
 
 slora_status topk_select(const float* scores, int groups, int N, int k, int rep,
                          int32_t* out_a, int32_t* out_b, cudaStream_t st) {
-  if (k <= 0 || groups <= 0) return SLORA_OK;
-  if (int64_t(N) > int64_t(kTopkThreads) * kTopkMaxM)
-    SLORA_FAIL(SLORA_ERR_SHAPE, "top-k over %d keys per group exceeds the supported %d", N,
-               kTopkThreads * kTopkMaxM);
   TopkOut o;
   o.a = out_a; o.b = out_b; o.rep = rep; o.N = N;
-  LaunchScope ls(kSelect, double(groups) * N * 4 + double(groups) * k * 4 * (rep + 1), st);
-  topk_kernel<<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
-  SLORA_CHECK_LAUNCH();
-  return SLORA_OK;
+  return launch_topk(scores, groups, N, k, o, st);
 }
 
 int64_t topk_max_keys() { return int64_t(kTopkThreads) * kTopkMaxM; }
+
+slora_status est_check_error(bool clear) {
+  int v = 0;
+  SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_est_error, sizeof(int)));
+  if (clear && v) {
+    int z = 0;
+    SLORA_CUDA(cudaMemcpyToSymbol(g_est_error, &z, sizeof(int)));
+  }
+  if (v) SLORA_FAIL(SLORA_ERR_CUDA, "estimator: a score kernel's shared staging buffer is misaligned");
+  return SLORA_OK;
+}
 
 }  // namespace slora

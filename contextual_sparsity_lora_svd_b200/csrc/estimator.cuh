@@ -11,13 +11,13 @@ namespace slora {
 //   out_b[g * k + i]           = g * N + S_g[i]              (if out_b != null).
 // Equal scores go to the lower index.
 
-// FFN activation-norm score and selection in one launch:
+// FFN activation-norm score (one launch), then the selection (one launch):
 //   scores[j] = sqrt(sum_t (silu(P_g[t] . U_g[j]) * (P_u[t] . U_u[j]))^2),
 //   P [rows x ldp] fp32 with P_g in columns [0, r), P_u in [r, 2r), context
 //   token t at row pmap[t] (identity when pmap is null);
 //   idx_out[0..k) = the k best channels (when idx_out != null).
 // partial: [nsplit x n] floats; counters: estimator_counter_count(n, r, 1)
-// unsigned ints, zero on entry.
+// unsigned ints, zero on entry; n at most topk_max_keys() when selecting.
 slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
                               const float* Ug, const float* Uu, int64_t n, int r, float* partial,
                               int nsplit, float* scores, unsigned* counters, int k,
@@ -36,7 +36,7 @@ int ffn_score_splits(int64_t T_C, int64_t n, int r);
 // norm taken over both channels of the pair; k is then the number of pairs
 // kept and each head keeps 2k channels (all pair firsts, then all seconds).
 // gram_part: gram_blocks(T_C) * nmat * r * r doubles; gram: nmat * r * r;
-// scores: groups * nkeys floats; counters: 1 + groups, zero on entry.
+// scores: groups * nkeys floats; counters: 1, zero on entry.
 constexpr int kCritModeQK = 0, kCritModeL2 = 1;
 slora_status gram_scores_select(int mode, const float* P, int64_t ldp, const int32_t* pmap,
                                 int64_t T_C, const float* U0, const float* U1, int r, int groups,
@@ -53,5 +53,8 @@ int64_t estimator_counter_count(int64_t n, int r, int groups);
 slora_status topk_select(const float* scores, int groups, int N, int k, int rep,
                          int32_t* out_a, int32_t* out_b, cudaStream_t st);
 int64_t topk_max_keys();
+
+// Device flag of the estimator kernels (see slora_device_error).
+slora_status est_check_error(bool clear);
 
 }  // namespace slora

@@ -325,10 +325,12 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   auto Yv = [](const void* p, int64_t ld, const int32_t* map = nullptr) {
     SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
   };
+  // rank-r operands of the LoRA contractions: fp32 ones rounded to one bf16
+  // term (the estimator's factors keep three, set on the pass over X below)
   auto Rv = [](const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
                int64_t map_limit = INT64_MAX) {
     SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
-    rr.map_limit = map_limit; return rr;
+    rr.map_limit = map_limit; rr.terms = dtp == kF32 ? 1 : 0; return rr;
   };
   // The rank-r gradients that sum over tokens, as one batched coldot:
   // dBd = s dOut^T hA, dAd = s dOB^T h, dBg = s dG^T XA_g, dBu = s dU^T XA_u,
@@ -774,10 +776,11 @@ namespace {
 SkY ykv(const void* p, int64_t ld, const int32_t* map = nullptr) {
   SkY y; y.ptr = p; y.ld = ld; y.map = map; return y;
 }
+// rank-r operand of a LoRA contraction; fp32 ones are rounded to one bf16 term
 SkR rkv(const void* p, int dtp, int64_t si, int64_t sq, const int32_t* map = nullptr,
         int64_t map_limit = INT64_MAX) {
   SkR rr; rr.ptr = p; rr.dt = dtp; rr.si = si; rr.sq = sq; rr.map = map;
-  rr.map_limit = map_limit; return rr;
+  rr.map_limit = map_limit; rr.terms = dtp == kF32 ? 1 : 0; return rr;
 }
 int64_t skinny_part_bound(const TokenInfo& ti, int64_t a, int64_t b, int64_t c2, int r) {
   int64_t np = 1;

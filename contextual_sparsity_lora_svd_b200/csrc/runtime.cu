@@ -3,6 +3,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "estimator.cuh"
 #include "gemm_tc.cuh"
 #include "lora_pack.cuh"
 #include "skinny.cuh"
@@ -12,15 +13,21 @@ namespace slora {
 namespace {
 thread_local std::string g_error;
 
+// The host's ctx_len travels in the kernel parameters: a small block for the
+// usual batch sizes, the full kMaxBatch block otherwise (a parameter block
+// of 8 KB makes every launch slower).
+template <int CAP>
 struct RowmapParams {
   int batch, seq;
-  int ctx_len[kMaxBatch];
+  int ctx_len[CAP];
 };
+constexpr int kSmallBatch = 64;
 
 // One block: scan ctx_len into per-sequence offsets, then every row t of the
 // full layout lands in ctx_rows or out_rows at its compact position, and every
 // sequence emits its context and output M tiles.
-__global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
+template <int CAP>
+__global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams<CAP> p,
                                                       int32_t* __restrict__ ctx_rows,
                                                       int32_t* __restrict__ out_rows,
                                                       int4* __restrict__ ctx_tiles,
@@ -31,7 +38,7 @@ __global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams p,
                                                       int64_t nzero2) {
   for (int64_t i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0u;
   for (int64_t i = threadIdx.x; i < nzero2; i += blockDim.x) zero2[i] = 0u;
-  __shared__ int ctx_off[kMaxBatch], ct_off[kMaxBatch], ot_off[kMaxBatch];
+  __shared__ int ctx_off[CAP], ct_off[CAP], ot_off[CAP];
   if (threadIdx.x == 0) {
     int acc = 0, ct = 0, ot = 0;
     for (int b = 0; b < p.batch; ++b) {
@@ -204,13 +211,24 @@ slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_
                             int32_t* out_rows, cudaStream_t st, int4* ctx_tiles,
                             int4* out_tiles, unsigned* zero, int64_t nzero, unsigned* zero2,
                             int64_t nzero2) {
-  RowmapParams p;
-  p.batch = ti.batch;
-  p.seq = ti.seq;
-  for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
   LaunchScope ls(kAux, double(ti.T) * 4, st);
-  rowmap_kernel<<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles, zero,
-                                    zero ? nzero : 0, zero2, zero2 ? nzero2 : 0);
+  if (ti.batch <= kSmallBatch) {
+    RowmapParams<kSmallBatch> p;
+    p.batch = ti.batch;
+    p.seq = ti.seq;
+    for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
+    rowmap_kernel<kSmallBatch><<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles,
+                                                   zero, zero ? nzero : 0, zero2,
+                                                   zero2 ? nzero2 : 0);
+  } else {
+    RowmapParams<kMaxBatch> p;
+    p.batch = ti.batch;
+    p.seq = ti.seq;
+    for (int b = 0; b < ti.batch; ++b) p.ctx_len[b] = tok->ctx_len[b];
+    rowmap_kernel<kMaxBatch><<<1, 1024, 0, st>>>(p, ctx_rows, out_rows, ctx_tiles, out_tiles,
+                                                 zero, zero ? nzero : 0, zero2,
+                                                 zero2 ? nzero2 : 0);
+  }
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
@@ -229,9 +247,12 @@ extern "C" slora_status slora_device_error(int clear) {
   const slora_status b = tc_check_error(clear != 0);
   const std::string second = b != SLORA_OK ? g_error : std::string();
   const slora_status c = skinny_check_error(clear != 0);
+  const std::string third = c != SLORA_OK ? g_error : std::string();
+  const slora_status d = est_check_error(clear != 0);
   if (a != SLORA_OK) g_error = first;
   else if (b != SLORA_OK) g_error = second;
-  return a != SLORA_OK ? a : (b != SLORA_OK ? b : c);
+  else if (c != SLORA_OK) g_error = third;
+  return a != SLORA_OK ? a : (b != SLORA_OK ? b : (c != SLORA_OK ? c : d));
 }
 
 extern "C" slora_status slora_set_wait_budget(int64_t cycles) {

@@ -468,7 +468,9 @@ int64_t splits_for(int64_t nblocks, int64_t nchunks, int CP, int NT) {
 
 int padded(int c) { return ((c + 15) / 16) * 16; }  // NF even keeps the templates few
 int64_t round64(int64_t x) { return (x + 63) / 64 * 64; }
-bool fp32_terms(const SkR& R) { return R.dt == kF32 || (R.ptr_b && R.dt_b == kF32); }
+bool fp32_terms(const SkR& R) {
+  return R.terms != 1 && (R.dt == kF32 || (R.ptr_b && R.dt_b == kF32));
+}
 
 slora_status prep_r(const SkR& R, int c, int CP, int64_t I, int nt, __nv_bfloat16* RS,
                     cudaStream_t st) {

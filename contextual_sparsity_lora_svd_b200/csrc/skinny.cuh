@@ -4,7 +4,9 @@
 // Y, so they run on mma.sync bf16 tensor-core fragments inside CUDA-core
 // tiles (the tcgen05 tile shape would waste the machine on N = c), with fp32
 // operands split into three bf16 terms (hi + mid + lo, relative residual
-// 2^-24) so the result is fp32-accurate.
+// 2^-24) where the result must be fp32-accurate (the estimator's projection),
+// or rounded to one bf16 term (the LoRA gradients, whose forward GEMMs use the
+// same rank-r operands in bf16).
 //
 //   rowdot:  P1[m, q] = sum_k Y[m, k] R1(k, q)      (e.g. X A^T, h A_d^T, dOut B_d)
 //   coldot:  P2[k, q] = sum_m Y[m, k] R2(m, q)      (LoRA gradients, sums over tokens)
@@ -29,6 +31,10 @@ struct SkY {  // Y(m, k) = ptr[(map ? map[m] : m) * ld + k], bf16, valid k < K
 struct SkR {  // R(i, q) = ptr[(map ? map[i] : i) * si + q * sq], fp32 or bf16
   const void* ptr = nullptr;
   int dt = kF32;
+  // bf16 terms an fp32 operand is split into: 0 = three (fp32-accurate
+  // products, ~2^-24 relative), 1 = one (the operand rounded to bf16, as the
+  // GEMMs' LoRA segments use it); bf16 operands always take one
+  int terms = 0;
   int64_t si = 0, sq = 0;
   const int32_t* map = nullptr;
   int64_t map_limit = INT64_MAX;  // map values outside [0, map_limit) read as zero
