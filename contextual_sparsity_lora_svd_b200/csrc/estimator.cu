@@ -153,60 +153,101 @@ struct TopkOut {
   int pair_half = 0; // > 0: keys are rotate-half pairs (p, p + pair_half)
 };
 
-__device__ __forceinline__ void topk_emit(const TopkOut o, int g, int ktot, int kp, int pos,
-                                          int c) {
-  for (int j = 0; j < o.rep; ++j) {
-    const int h = g * o.rep + j;
-    int32_t* row = o.a + int64_t(h) * ktot;
-    row[pos] = h * o.N + c;
-    if (o.pair_half) row[kp + pos] = h * o.N + c + o.pair_half;
-  }
-  if (o.b) {
-    int32_t* row = o.b + int64_t(g) * ktot;
-    row[pos] = g * o.N + c;
-    if (o.pair_half) row[kp + pos] = g * o.N + c + o.pair_half;
+// The output fields travel as plain scalar arguments (registers): read
+// through a struct, every index stored paid a slow reload of the fields.
+// ONE: a single index list (rep 1, no b, no pairs), written directly.
+template <bool ONE>
+__device__ __forceinline__ void topk_emit(int32_t* __restrict__ oa, int32_t* __restrict__ ob,
+                                          int rep, int hN, int ph, int g, int ktot, int kp,
+                                          int pos, int c) {
+  if constexpr (ONE) {
+    oa[pos] = c;
+  } else {
+    for (int j = 0; j < rep; ++j) {
+      const int h = g * rep + j;
+      int32_t* row = oa + int64_t(h) * ktot;
+      row[pos] = h * hN + c;
+      if (ph) row[kp + pos] = h * hN + c + ph;
+    }
+    if (ob) {
+      int32_t* row = ob + int64_t(g) * ktot;
+      row[pos] = g * hN + c;
+      if (ph) row[kp + pos] = g * hN + c + ph;
+    }
   }
 }
 
-// The k largest of n scores (ties to the lower index), written through `o`
-// for group g.  All B threads of the block call it; n <= B * MAXM.
-//   1. keys (score bits) in registers, each thread a contiguous index range;
-//   2. the keys share their bits above hb, the highest bit where the largest
-//      and the smallest key differ; below it, radix passes of up to 8 bits
-//      each (at most four) narrow the prefix of the k-th largest key: a pass
-//      counts the keys that match the prefix so far in per-warp 256-bin
-//      histograms (`hist`, [B/32][256] words), sums them, and warp 0 finds
-//      the digit holding the wanted rank; the keys in the digits above it
-//      are all kept (`above`) and the rank left is sought inside the digit;
-//   3. after the last pass the prefix is the k-th largest key tau itself:
-//      every key above tau is kept, and of the keys equal to tau the first
-//      ones in index order; block scans give each thread its output
-//      position, so the indices come out ascending.
-// Shared memory (32-bit shared-window addresses): `red` 2 x B/32 words,
-// `hist` B/32 x 256 words, `bc` 4 broadcast words.
+__device__ __forceinline__ uint32_t sh_atom_add(uint32_t a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(a), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Radix digits of 11 bits: one shared 2048-bin histogram per pass.
+constexpr int kTopkBins = 2048;
+// Keys of the wanted key's bin that warp 0 finishes in registers (8 a lane).
+constexpr int kCandMax = 256;
+
+// Shared words of block_topk<B, MAXM> (see the kernel's arrays).
+constexpr int topk_hist_words() { return kTopkBins; }
 template <int B, int MAXM>
-__device__ void block_topk(const float* __restrict__ sc, int n, int k, const TopkOut o, int g,
-                           uint32_t red_smem, uint32_t hist, uint32_t bc) {
+constexpr int topk_tab_words() { return MAXM * (B / 32); }
+constexpr int topk_cand_words() { return kCandMax; }
+
+// The k largest of n scores (ties to the lower index), written through the
+// output fields for group g.  All B threads of the block call it;
+// n <= B * MAXM.  Key j (the score's fp32 bits) sits in row i = j / B of
+// thread j % B, so every global access of a row is one coalesced line.
+//   1. the keys share their bits above hb, the highest bit where the largest
+//      and the smallest key differ; a radix pass counts, in one shared
+//      2048-bin histogram, the 11 bits below the prefix fixed so far, and a
+//      descending block scan of the bins finds the digit holding the wanted
+//      rank; the keys in higher digits are all kept (`above`) and the search
+//      goes on inside the digit;
+//   2. once the digit holds at most kCandMax keys they are compacted into
+//      shared memory, and warp 0 takes them into registers and finds the
+//      wanted key by bisection over the remaining bits;
+//   3. tau is the k-th largest key: every key above it is kept, and of the
+//      keys equal to it the first ones in index order.  Each (row, warp)
+//      counts its keys above / equal to tau by ballot; one block scan over
+//      that table, in index order, gives every kept key its output position.
+// Shared memory (32-bit shared-window addresses): `red` 2 x B/32 words,
+// `hist` topk_hist_words, `cand` topk_cand_words, `tab` topk_tab_words,
+// `bc` 8 broadcast words.
+template <int B, int MAXM, bool ONE>
+__device__ void block_topk(const float* __restrict__ sc, int n, int k, int32_t* __restrict__ oa,
+                           int32_t* __restrict__ ob, int rep, int hN, int ph, int g,
+                           uint32_t red_smem, uint32_t hist, uint32_t cand, uint32_t tab,
+                           uint32_t bc) {
   constexpr int NW = B / 32;
+  constexpr int CPL = kCandMax / 32;  // candidates per lane of warp 0
+  constexpr int BPT = kTopkBins / B;  // histogram bins per thread in the scan
   BlockRed<B> red{red_smem};
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int kp = k;
-  const int ktot = o.pair_half ? 2 * k : k;
+  const int ktot = ph ? 2 * k : k;
   if (k <= 0 || n <= 0) return;
-  const int m = (n + B - 1) / B;
-  const int i0 = tid * m;
-  const int mt = ::max(0, ::min(m, n - i0));
-  if (k >= n) {  // everything is kept: own range in order
-    for (int i = 0; i < mt; ++i) topk_emit(o, g, ktot, kp, i0 + i, i0 + i);
+  const int rows = (n + B - 1) / B;
+  if (k >= n) {  // everything is kept
+    for (int i = 0; i < rows; ++i)
+      if (i * B + tid < n)
+        topk_emit<ONE>(oa, ob, rep, hN, ph, g, ktot, kp, i * B + tid, i * B + tid);
     return;
   }
+  if (tid == 0) sh_st(bc + 8u, 0u);  // candidate count (ordered by the barriers below)
   uint32_t key[MAXM];
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int i = 0; i < MAXM; ++i) {
+    const int j = i * B + tid;
     key[i] = 0u;
-    if (i < mt) {
-      key[i] = score_key(__ldcg(sc + i0 + i));
+    if (i < rows && j < n) {
+      key[i] = score_key(__ldcg(sc + j));
       kmin = ::min(kmin, key[i]);
       kmax = ::max(kmax, key[i]);
     }
@@ -220,81 +261,169 @@ __device__ void block_topk(const float* __restrict__ sc, int n, int k, const Top
     uint32_t prefix = kmin & ~((2u << top) - 1u);
     uint32_t need = uint32_t(k);  // rank of tau among the keys matching prefix
     while (true) {
-      const int shift = top > 7 ? top - 7 : 0;
+      const int shift = top > 10 ? top - 10 : 0;
       const uint32_t dmask = (2u << (top - shift)) - 1u;  // digit = bits top .. shift
       const uint32_t pmask = ~((2u << top) - 1u);         // bits above top
-      for (int i = tid; i < NW * 256; i += B) sh_st(hist + 4u * uint32_t(i), 0u);
+      for (int i = tid; i < kTopkBins; i += B) sh_st(hist + 4u * uint32_t(i), 0u);
       __syncthreads();
 #pragma unroll
       for (int i = 0; i < MAXM; ++i)
-        if (i < mt && (key[i] & pmask) == prefix)
-          sh_add(hist + 4u * (uint32_t(w) * 256u + ((key[i] >> shift) & dmask)), 1u);
+        if (i < rows && i * B + tid < n && (key[i] & pmask) == prefix)
+          sh_add(hist + 4u * ((key[i] >> shift) & dmask), 1u);
       __syncthreads();
-      for (int d = tid; d < 256; d += B) {
-        uint32_t t = 0;
-        for (int v = 0; v < NW; ++v) t += sh_ld(hist + 4u * uint32_t(v * 256 + d));
-        sh_st(hist + 4u * uint32_t(d), t);  // warp 0's row now holds the totals
+      // thread t owns bins [2048 - BPT (t + 1), 2048 - BPT t): thread order is
+      // descending digit order, so the exclusive scan counts the higher digits
+      const int b_top = kTopkBins - 1 - BPT * tid;
+      uint32_t own = 0;
+      for (int i = 0; i < BPT; ++i) own += sh_ld(hist + 4u * uint32_t(b_top - i));
+      const uint32_t higher_t = red.excl_scan(own);
+      if (higher_t < need && higher_t + own >= need) {
+        uint32_t cum = higher_t;
+        for (int i = 0; i < BPT; ++i) {
+          const uint32_t h = sh_ld(hist + 4u * uint32_t(b_top - i));
+          if (cum + h >= need) {
+            sh_st(bc, uint32_t(b_top - i));
+            sh_st(bc + 4u, cum);  // keys of this prefix in higher digits
+            sh_st(bc + 12u, h);   // keys in the digit
+            break;
+          }
+          cum += h;
+        }
       }
       __syncthreads();
-      if (w == 0) {  // lane l owns digits 255-8l .. 248-8l, scanned from the top
-        uint32_t own = 0;
-        for (int i = 0; i < 8; ++i) own += sh_ld(hist + 4u * uint32_t(255 - 8 * lane - i));
-        uint32_t incl = own;
+      const uint32_t dstar = sh_ld(bc), higher = sh_ld(bc + 4u), nbin = sh_ld(bc + 12u);
+      above += higher;
+      need -= higher;
+      prefix |= dstar << shift;
+      if (shift == 0) {
+        tau = prefix;
+        break;
+      }
+      top = shift - 1;
+      if (nbin <= uint32_t(kCandMax)) {
+        // compact the digit's keys (one shared atomic per warp for its base)
+        const uint32_t pm = ~((2u << top) - 1u);
+        uint32_t mine = 0;
+#pragma unroll
+        for (int i = 0; i < MAXM; ++i)
+          if (i < rows && i * B + tid < n && (key[i] & pm) == prefix) ++mine;
+        uint32_t incl = mine;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const uint32_t x = __shfl_up_sync(0xffffffffu, incl, off);
           if (lane >= off) incl += x;
         }
-        const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need);
-        if (lane == __ffs(hit) - 1) {
-          uint32_t cum = incl - own;
-          for (int i = 0; i < 8; ++i) {
-            const int dg = 255 - 8 * lane - i;
-            const uint32_t h = sh_ld(hist + 4u * uint32_t(dg));
-            if (cum + h >= need) {
-              sh_st(bc, uint32_t(dg));
-              sh_st(bc + 4u, cum);  // keys of this prefix in higher digits
+        uint32_t base = 0;
+        if (lane == 31) base = sh_atom_add(bc + 8u, incl);
+        uint32_t pos = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
+#pragma unroll
+        for (int i = 0; i < MAXM; ++i)
+          if (i < rows && i * B + tid < n && (key[i] & pm) == prefix)
+            sh_st(cand + 4u * pos++, key[i]);
+        __syncthreads();
+        if (w == 0) {
+          // bisection over the remaining bits top .. 0 with the candidates in
+          // registers; the padding (0) never reaches a threshold above the
+          // prefix
+          uint32_t ck[CPL];
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) {
+            const uint32_t idx = uint32_t(q * 32 + lane);
+            ck[q] = idx < nbin ? sh_ld(cand + 4u * idx) : 0u;
+          }
+          uint32_t lo = prefix, hi = prefix + (2u << top);
+          while (hi - lo > 1u) {
+            const uint32_t mid = lo + (hi - lo) / 2u;
+            uint32_t c0 = 0, c1 = 0;
+#pragma unroll
+            for (int q = 0; q < CPL; q += 2) {
+              c0 += ck[q] >= mid ? 1u : 0u;
+              c1 += ck[q + 1] >= mid ? 1u : 0u;
+            }
+            const uint32_t c = __reduce_add_sync(0xffffffffu, c0 + c1);
+            if (c == need) {  // the wanted keys are exactly those >= mid
+              uint32_t mn = 0xffffffffu;
+#pragma unroll
+              for (int q = 0; q < CPL; ++q)
+                if (ck[q] >= mid) mn = ::min(mn, ck[q]);
+              lo = __reduce_min_sync(0xffffffffu, mn);
               break;
             }
-            cum += h;
+            if (c > need) lo = mid; else hi = mid;
+          }
+          uint32_t gt = 0;
+#pragma unroll
+          for (int q = 0; q < CPL; ++q) gt += ck[q] > lo ? 1u : 0u;
+          gt = __reduce_add_sync(0xffffffffu, gt);
+          if (lane == 0) {
+            sh_st(bc + 16u, lo);
+            sh_st(bc + 20u, gt);
           }
         }
+        __syncthreads();
+        tau = sh_ld(bc + 16u);
+        above += sh_ld(bc + 20u);
+        break;
       }
-      __syncthreads();
-      const uint32_t dstar = sh_ld(bc), higher = sh_ld(bc + 4u);
-      above += higher;
-      need -= higher;
-      prefix |= dstar << shift;
-      if (shift == 0) break;
-      top = shift - 1;
-    }
-    tau = prefix;
-  }
-  // keep every key above tau; of the keys equal to tau the first ones
-  uint32_t cgt = 0, ceq = 0;
-#pragma unroll
-  for (int i = 0; i < MAXM; ++i) {
-    if (i < mt) {
-      if (key[i] > tau) ++cgt;
-      else if (key[i] == tau) ++ceq;
     }
   }
-  const uint32_t want = uint32_t(k) - above;
-  const uint32_t tie_before = red.excl_scan(ceq);
-  const uint32_t take_eq = want > tie_before ? ::min(ceq, want - tie_before) : 0u;
-  int pos = int(red.excl_scan(cgt + take_eq));
-  uint32_t taken = 0;
+  // output positions in index order: per (row, warp) the counts of keys above
+  // tau (high half) and equal to it (low half), kept by the lane whose index
+  // is the row; n <= 2^15 keeps both halves apart through the scan
+  static_assert(MAXM <= 64, "two table words per lane");
+  const uint32_t want = uint32_t(k) - above;  // keys equal to tau that are kept
+  unsigned long long fgt = 0ull, feq = 0ull;
+  uint32_t row_lo = 0, row_hi = 0;  // rows lane and lane + 32
 #pragma unroll
   for (int i = 0; i < MAXM; ++i) {
-    if (i < mt) {
-      const uint32_t kv = key[i];
-      bool sel = kv > tau;
-      if (kv == tau) {
-        sel = taken < take_eq;
-        ++taken;
-      }
-      if (sel) topk_emit(o, g, ktot, kp, pos++, i0 + i);
+    if (i < rows) {
+      const int j = i * B + tid;
+      const bool gt = j < n && key[i] > tau, eq = j < n && key[i] == tau;
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+      if (gt) fgt |= 1ull << i;
+      if (eq) feq |= 1ull << i;
+      const uint32_t cnt = (uint32_t(__popc(bg)) << 16) | uint32_t(__popc(be));
+      if (i < 32) row_lo = lane == i ? cnt : row_lo;
+      else row_hi = lane == i - 32 ? cnt : row_hi;
     }
+  }
+  if (lane < rows) sh_st(tab + 4u * uint32_t(lane * NW + w), row_lo);
+  if (MAXM > 32 && lane + 32 < rows) sh_st(tab + 4u * uint32_t((lane + 32) * NW + w), row_hi);
+  __syncthreads();
+  {
+    constexpr int EPT = (MAXM * NW + B - 1) / B;  // table entries per thread
+    const int ne = rows * NW;
+    uint32_t v[EPT], sum = 0;
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) {
+      const int e = tid * EPT + q;
+      v[q] = e < ne ? sh_ld(tab + 4u * uint32_t(e)) : 0u;
+      sum += v[q];
+    }
+    uint32_t run = red.excl_scan(sum);
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) {
+      const int e = tid * EPT + q;
+      if (e < ne) sh_st(tab + 4u * uint32_t(e), run);
+      run += v[q];
+    }
+  }
+  __syncthreads();
+  const uint32_t pre_lo = lane < rows ? sh_ld(tab + 4u * uint32_t(lane * NW + w)) : 0u;
+  const uint32_t pre_hi =
+      MAXM > 32 && lane + 32 < rows ? sh_ld(tab + 4u * uint32_t((lane + 32) * NW + w)) : 0u;
+  const uint32_t lt = lanemask_lt();
+  // a rolled loop: unrolled over every row, the general emission's code
+  // outgrew the instruction cache
+#pragma unroll 1
+  for (int i = 0; i < rows; ++i) {
+    const bool gt = (fgt >> i) & 1ull, eq = (feq >> i) & 1ull;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const uint32_t pre = __shfl_sync(0xffffffffu, i < 32 ? pre_lo : pre_hi, i & 31);
+    const uint32_t gtb = (pre >> 16) + uint32_t(__popc(bg & lt));
+    const uint32_t eqb = (pre & 0xffffu) + uint32_t(__popc(be & lt));
+    if (gt || (eq && eqb < want))
+      topk_emit<ONE>(oa, ob, rep, hN, ph, g, ktot, kp, int(gtb + ::min(eqb, want)), i * B + tid);
   }
 }
 
@@ -408,7 +537,7 @@ template <int RP>
 constexpr int fma_channels() { return kScoreThreads * 2 * fma_npair<RP>(); }
 
 template <int RP>
-__global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const __grid_constant__ ScoreArgs a) {
   constexpr int NP = fma_npair<RP>(), CH = fma_channels<RP>();
   __shared__ __align__(16) unsigned long long sp[kFmaTokens][2 * RP];  // {v, v} pairs
   __shared__ unsigned s_last;
@@ -501,7 +630,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const S
 }
 
 template <int C>
-__global__ void __launch_bounds__(kScoreThreads) ffn_score_mma_kernel(const ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads) ffn_score_mma_kernel(const __grid_constant__ ScoreArgs a) {
   constexpr int NT = score_nt(C), TW = score_tw(C), KB = 3 * C;
   constexpr int CH = kScoreWarps * NT * 8;  // channels per block
   extern __shared__ __align__(16) uint32_t s_stage[];
@@ -659,7 +788,7 @@ struct GramArgs {
   unsigned* counter;
 };
 
-__global__ void __launch_bounds__(kGramThreads) gram_partial_kernel(const GramArgs a) {
+__global__ void __launch_bounds__(kGramThreads) gram_partial_kernel(const __grid_constant__ GramArgs a) {
   __shared__ float sp[kGramTokens][2 * 48 + 1];
   __shared__ unsigned s_last;
   const int tid = threadIdx.x, r = a.r, ne = a.nmat * r * r;
@@ -739,7 +868,7 @@ __device__ __forceinline__ double quad_form(const double* G, const float* u, int
   return s > 0.0 ? s : 0.0;
 }
 
-__global__ void __launch_bounds__(kNormThreads) norm_score_kernel(const NormArgs a) {
+__global__ void __launch_bounds__(kNormThreads) norm_score_kernel(const __grid_constant__ NormArgs a) {
   __shared__ double sg[2 * 48 * 48];
   const int tid = threadIdx.x, r = a.r;
   const int nmat = a.mode == kCritModeQK ? 2 : 1;
@@ -771,17 +900,21 @@ __global__ void __launch_bounds__(kNormThreads) norm_score_kernel(const NormArgs
 
 // ------------------------------------------------------------------ top-k
 // One block per group; the scratch lives in the kernel's own shared arrays.
-constexpr int kTopkThreads = 512;
-constexpr int kTopkMaxM = 64;  // keys per thread: n <= 512 * 64
+// 512 threads for long score vectors, 128 for short per-head ones.
+constexpr int kTopkMaxM = 64;  // rows per thread: n <= 512 * 64
 
-template <int MAXM>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores,
-                                                            int N, int k, TopkOut o) {
-  __shared__ __align__(16) uint32_t s_red[2 * (kTopkThreads / 32)];
-  __shared__ __align__(16) uint32_t s_hist[(kTopkThreads / 32) * 256];
-  __shared__ __align__(16) uint32_t s_bc[4];
-  block_topk<kTopkThreads, MAXM>(scores + int64_t(blockIdx.x) * N, N, k, o, blockIdx.x,
-                                 sh_addr(s_red), sh_addr(s_hist), sh_addr(s_bc));
+template <int B, int MAXM, bool ONE>
+__global__ void __launch_bounds__(B) topk_kernel(const float* __restrict__ scores, int N, int k,
+                                                 int32_t* out_a, int32_t* out_b, int rep, int hN,
+                                                 int pair_half) {
+  __shared__ __align__(16) uint32_t s_red[2 * (B / 32)];
+  __shared__ __align__(16) uint32_t s_hist[topk_hist_words()];
+  __shared__ __align__(16) uint32_t s_cand[topk_cand_words()];
+  __shared__ __align__(16) uint32_t s_tab[topk_tab_words<B, MAXM>()];
+  __shared__ __align__(16) uint32_t s_bc[8];
+  block_topk<B, MAXM, ONE>(scores + int64_t(blockIdx.x) * N, N, k, out_a, out_b, rep, hN,
+                           pair_half, blockIdx.x, sh_addr(s_red), sh_addr(s_hist),
+                           sh_addr(s_cand), sh_addr(s_tab), sh_addr(s_bc));
 }
 
 int rank_chunks(int r) { return r <= 8 ? 1 : (r <= 16 ? 2 : (r <= 24 ? 3 : (r <= 32 ? 4 : 6))); }
@@ -864,23 +997,36 @@ int64_t gram_blocks(int64_t T_C) {
 }
 
 namespace {
+template <bool ONE>
+void launch_topk_kernel(const float* scores, int groups, int N, int k, const TopkOut& o,
+                        cudaStream_t st) {
+  const unsigned gr = unsigned(groups);
+  if (N <= 128 * 8)
+    topk_kernel<128, 8, ONE><<<gr, 128, 0, st>>>(scores, N, k, o.a, o.b, o.rep, o.N, o.pair_half);
+  else if (N <= 512 * 8)
+    topk_kernel<512, 8, ONE><<<gr, 512, 0, st>>>(scores, N, k, o.a, o.b, o.rep, o.N, o.pair_half);
+  else if (N <= 512 * 32)
+    topk_kernel<512, 32, ONE><<<gr, 512, 0, st>>>(scores, N, k, o.a, o.b, o.rep, o.N,
+                                                  o.pair_half);
+  else
+    topk_kernel<512, kTopkMaxM, ONE><<<gr, 512, 0, st>>>(scores, N, k, o.a, o.b, o.rep, o.N,
+                                                         o.pair_half);
+}
+
 // One top-k block per group, the register array sized to the keys per thread.
 slora_status launch_topk(const float* scores, int groups, int N, int k, const TopkOut& o,
                          cudaStream_t st) {
   if (k <= 0 || groups <= 0) return SLORA_OK;
-  if (int64_t(N) > int64_t(kTopkThreads) * kTopkMaxM)
+  if (int64_t(N) > int64_t(512) * kTopkMaxM)
     SLORA_FAIL(SLORA_ERR_SHAPE, "top-k over %d keys per group exceeds the supported %d", N,
-               kTopkThreads * kTopkMaxM);
+               512 * kTopkMaxM);
   const int per_head = o.pair_half ? 2 * k : k;
   LaunchScope ls(kSelect, double(groups) * N * 4 + double(groups) * per_head * 4 * (o.rep + 1),
                  st);
-  const int m = (N + kTopkThreads - 1) / kTopkThreads;
-  if (m <= 8)
-    topk_kernel<8><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
-  else if (m <= 32)
-    topk_kernel<32><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
+  if (o.rep == 1 && !o.b && !o.pair_half)
+    launch_topk_kernel<true>(scores, groups, N, k, o, st);
   else
-    topk_kernel<kTopkMaxM><<<unsigned(groups), kTopkThreads, 0, st>>>(scores, N, k, o);
+    launch_topk_kernel<false>(scores, groups, N, k, o, st);
   SLORA_CHECK_LAUNCH();
   return SLORA_OK;
 }
@@ -962,7 +1108,7 @@ slora_status topk_select(const float* scores, int groups, int N, int k, int rep,
   return launch_topk(scores, groups, N, k, o, st);
 }
 
-int64_t topk_max_keys() { return int64_t(kTopkThreads) * kTopkMaxM; }
+int64_t topk_max_keys() { return int64_t(512) * kTopkMaxM; }
 
 slora_status est_check_error(bool clear) {
   int v = 0;

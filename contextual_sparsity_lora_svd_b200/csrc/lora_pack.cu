@@ -67,7 +67,7 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ in, int64_t ld_in16
 // Several row compactions sharing one index list: warp w takes (job, row)
 // items w, w + nwarps, ...; each lane moves 8 16-byte units per round (all
 // loads of a round issued before its stores).
-__global__ void __launch_bounds__(256) gather_rows_multi_kernel(const GatherJobs J,
+__global__ void __launch_bounds__(256) gather_rows_multi_kernel(const __grid_constant__ GatherJobs J,
                                                                 const int32_t* __restrict__ idx,
                                                                 int64_t n, int64_t cols16) {
   const int lane = threadIdx.x & 31;
@@ -148,7 +148,7 @@ __global__ void sanitize_kernel(const int32_t* __restrict__ in, int64_t n, int64
 // (row j: src[j * ld_src + q]; trans: src[q * ld_src + j]) is added to column
 // idx[j] of dst in the same orientation.  With trans, consecutive threads take
 // consecutive j (coalesced source rows); without, consecutive q.
-__global__ void scatter_add_kernel(const ScatterAddJobs J, const int32_t* __restrict__ idx,
+__global__ void scatter_add_kernel(const __grid_constant__ ScatterAddJobs J, const int32_t* __restrict__ idx,
                                    int64_t n, int r, int64_t limit) {
   const ScatterAddJob& jb = J.job[blockIdx.y];
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;

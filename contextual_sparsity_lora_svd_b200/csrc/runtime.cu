@@ -27,7 +27,7 @@ constexpr int kSmallBatch = 64;
 // full layout lands in ctx_rows or out_rows at its compact position, and every
 // sequence emits its context and output M tiles.
 template <int CAP>
-__global__ void __launch_bounds__(1024) rowmap_kernel(const RowmapParams<CAP> p,
+__global__ void __launch_bounds__(1024) rowmap_kernel(const __grid_constant__ RowmapParams<CAP> p,
                                                       int32_t* __restrict__ ctx_rows,
                                                       int32_t* __restrict__ out_rows,
                                                       int4* __restrict__ ctx_tiles,

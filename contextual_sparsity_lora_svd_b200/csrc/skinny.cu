@@ -104,7 +104,7 @@ __device__ __forceinline__ float load_r(const SkR& R, int64_t i, int q) {
 // R(i, q) (zero for q >= c or i >= I), rows of I64 = roundup(I, 64) elements.
 // Threads walk the source's contiguous index so the reads coalesce.
 template <int NT>
-__global__ void prep_r_kernel(const SkR R, int c, int CP, int64_t I, int64_t I64,
+__global__ void prep_r_kernel(const __grid_constant__ SkR R, int c, int CP, int64_t I, int64_t I64,
                               __nv_bfloat16* __restrict__ RS) {
   const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= int64_t(CP) * I64) return;
@@ -132,7 +132,7 @@ struct PrepBatch {
   int64_t I[8], I64[8];
   __nv_bfloat16* RS[8];
 };
-__global__ void prep_r_batch_kernel(const PrepBatch b) {
+__global__ void prep_r_batch_kernel(const __grid_constant__ PrepBatch b) {
   const int k = blockIdx.y;
   const int CP = b.CP[k];
   const int64_t I64 = b.I64[k];
@@ -274,12 +274,12 @@ __device__ __forceinline__ void store_partial(float* part, int split, int64_t no
 }
 
 template <int NF, int NT>
-__global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int64_t K,
+__global__ void __launch_bounds__(NTH) rowdot_kernel(const __grid_constant__ SkY Y, int64_t M, int64_t K,
                                                      const __nv_bfloat16* __restrict__ RS,
                                                      int64_t I64, int c, int chunks_per_split,
                                                      float* __restrict__ part,
                                                      unsigned* __restrict__ counters,
-                                                     const SkRowOut o) {
+                                                     const __grid_constant__ SkRowOut o) {
   constexpr int CP = NF * 8, S = stages_for(CP, NT);
   extern __shared__ __align__(16) unsigned char sk_smem[];
   auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [S][TILE][PAD]
@@ -358,12 +358,12 @@ __global__ void __launch_bounds__(NTH) rowdot_kernel(const SkY Y, int64_t M, int
 }
 
 template <int NF, int NT>
-__global__ void __launch_bounds__(NTH) coldot_kernel(const SkY Y, int64_t M, int64_t K,
+__global__ void __launch_bounds__(NTH) coldot_kernel(const __grid_constant__ SkY Y, int64_t M, int64_t K,
                                                      const __nv_bfloat16* __restrict__ RS,
                                                      int64_t I64, int c, int chunks_per_split,
                                                      float* __restrict__ part,
                                                      unsigned* __restrict__ counters,
-                                                     const SkColOut o) {
+                                                     const __grid_constant__ SkColOut o) {
   constexpr int CP = NF * 8, S = stages_for(CP, NT);
   extern __shared__ __align__(16) unsigned char sk_smem[];
   auto Ys = reinterpret_cast<__nv_bfloat16 (*)[TILE][PAD]>(sk_smem);  // [S][TILE][PAD]
@@ -876,7 +876,8 @@ struct RowReduceJob {
   int64_t M = 0;
   SkRowOut o;
 };
-__global__ void reduce_rows_kernel(const RowReduceJob j0, const RowReduceJob j1, int pc, int lr,
+__global__ void reduce_rows_kernel(const __grid_constant__ RowReduceJob j0,
+                                   const __grid_constant__ RowReduceJob j1, int pc, int lr,
                                    int r) {
   const RowReduceJob& J = blockIdx.y ? j1 : j0;
   const int nq4 = pc / 4;
