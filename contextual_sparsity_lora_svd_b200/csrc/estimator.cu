@@ -531,13 +531,22 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 constexpr int kFmaTokens = 64;  // tokens staged per round
+// One channel pair per thread (its U rows in registers); resident blocks per
+// SM by rank (the rank-16 rows take twice the registers).
 template <int RP>
-constexpr int fma_npair() { return RP <= 8 ? 2 : 1; }
+constexpr int fma_npair() { return 1; }
 template <int RP>
 constexpr int fma_channels() { return kScoreThreads * 2 * fma_npair<RP>(); }
-
 template <int RP>
-__global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const __grid_constant__ ScoreArgs a) {
+constexpr int fma_min_blocks() { return RP <= 8 ? 3 : 2; }
+
+// silu(g) u = g u / (1 + e^-g).  With g' = -g log2(e) and u' = -u ln(2)
+// (the constants folded into the thread's U rows once), g u = g' u', and
+// e^-g = 2^g', so each (token, channel) takes one ex2, one add, one
+// reciprocal and two multiplies.
+template <int RP>
+__global__ void __launch_bounds__(kScoreThreads, fma_min_blocks<RP>())
+    ffn_score_fma_kernel(const __grid_constant__ ScoreArgs a) {
   constexpr int NP = fma_npair<RP>(), CH = fma_channels<RP>();
   __shared__ __align__(16) unsigned long long sp[kFmaTokens][2 * RP];  // {v, v} pairs
   __shared__ unsigned s_last;
@@ -550,6 +559,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const _
     return;
   }
   // this thread's channel pairs: j = cb*CH + 2*(tid + kScoreThreads*p) + {0, 1}
+  constexpr float kNegLog2e = -1.4426950408889634f, kNegLn2 = -0.6931471805599453f;
   unsigned long long ug[NP][RP], uu[NP][RP], acc[NP];
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
@@ -561,60 +571,104 @@ __global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const _
       const float g1 = (ok && j + 1 < a.n) ? a.Ug[(j + 1) * r + q] : 0.0f;
       const float u0 = (ok && j < a.n) ? a.Uu[j * r + q] : 0.0f;
       const float u1 = (ok && j + 1 < a.n) ? a.Uu[(j + 1) * r + q] : 0.0f;
-      ug[p][q] = pack_f2(g0, g1);
-      uu[p][q] = pack_f2(u0, u1);
+      ug[p][q] = pack_f2(g0 * kNegLog2e, g1 * kNegLog2e);
+      uu[p][q] = pack_f2(u0 * kNegLn2, u1 * kNegLn2);
     }
     acc[p] = 0ull;
   }
-  const unsigned long long neg_log2e = pack_f2(-1.4426950408889634f, -1.4426950408889634f);
   const unsigned long long one2 = pack_f2(1.0f, 1.0f);
   const int64_t t0 = int64_t(sp_id) * a.chunk;
   const int64_t t1 = ::min(a.T_C, t0 + a.chunk);
+  // the staging's parameters in registers, read once
+  const float* __restrict__ P = a.P;
+  const int32_t* __restrict__ pmap = a.pmap;
+  const int64_t ldp = a.ldp;
+  // staging: each thread carries EPT values of a stage's P rows; the next
+  // stage's values, and the row indices of the stage after it, are loaded
+  // into registers while the current one is computed (so no P load waits on
+  // its row index).  Rows past the last token are zero (g' = 0 gives v = 0).
+  constexpr int EPT = kFmaTokens * 2 * RP / kScoreThreads;
+  const uint32_t sp0 = sh_addr(&sp[0][0]);
+  float pf[EPT];
+  int32_t prow[EPT];  // rows of P for the stage loaded next (-1: past the end)
+  auto load_rows = [&](int64_t tb) {
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int tt = (tid + e * kScoreThreads) / (2 * RP);
+      prow[e] = tb + tt < t1 ? (pmap ? pmap[tb + tt] : int32_t(tb + tt)) : -1;
+    }
+  };
+  auto load_vals = [&]() {
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int q = (tid + e * kScoreThreads) % (2 * RP), mat = q / RP, qq = q % RP;
+      pf[e] = (qq < r && prow[e] >= 0) ? P[int64_t(prow[e]) * ldp + mat * r + qq] : 0.0f;
+    }
+  };
+  // g' and u' of one channel pair for the token row at shared address `row`
+  auto dots = [&](uint32_t row, int p, unsigned long long& g2, unsigned long long& u2) {
+    g2 = u2 = 0ull;
+#pragma unroll
+    for (int q2 = 0; q2 < RP / 2; ++q2) {
+      unsigned long long px, py;
+      asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(px), "=l"(py) : "r"(row + 16u * q2));
+      g2 = ffma2(px, ug[p][2 * q2], g2);
+      g2 = ffma2(py, ug[p][2 * q2 + 1], g2);
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < RP / 2; ++q2) {
+      unsigned long long px, py;
+      asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
+                   : "=l"(px), "=l"(py)
+                   : "r"(row + 16u * (RP / 2 + q2)));
+      u2 = ffma2(px, uu[p][2 * q2], u2);
+      u2 = ffma2(py, uu[p][2 * q2 + 1], u2);
+    }
+  };
+  auto tail = [&](unsigned long long g2, unsigned long long u2, unsigned long long& ac) {
+    const float2 x = unpack_f2(g2);
+    const unsigned long long den = fadd2(pack_f2(ex2_approx(x.x), ex2_approx(x.y)), one2);
+    const float2 dn = unpack_f2(den);
+    const unsigned long long inv = pack_f2(rcp_approx(dn.x), rcp_approx(dn.y));
+    const unsigned long long v = fmul2(fmul2(g2, u2), inv);
+    ac = ffma2(v, v, ac);
+  };
+  if (t0 < t1) {
+    load_rows(t0);
+    load_vals();
+    load_rows(t0 + kFmaTokens);
+  }
   for (int64_t tb = t0; tb < t1; tb += kFmaTokens) {
     const int nt = int(::min(int64_t(kFmaTokens), t1 - tb));
-    __syncthreads();
-    for (int e = tid; e < nt * 2 * RP; e += kScoreThreads) {
-      const int tt = e / (2 * RP), q = e % (2 * RP), mat = q / RP, qq = q % RP;
-      float v = 0.0f;
-      if (qq < r) {
-        const int64_t row = a.pmap ? int64_t(a.pmap[tb + tt]) : tb + tt;
-        v = a.P[row * a.ldp + mat * r + qq];
-      }
-      sp[tt][q] = pack_f2(v, v);
+    __syncthreads();  // the previous stage has been consumed
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const uint64_t v = pack_f2(pf[e], pf[e]);
+      asm volatile("st.shared.u64 [%0], %1;" ::"r"(sp0 + 8u * uint32_t(tid + e * kScoreThreads)),
+                   "l"(v));
     }
     __syncthreads();
-    for (int tt = 0; tt < nt; ++tt) {
-      const ulonglong2* row = reinterpret_cast<const ulonglong2*>(sp[tt]);
-      unsigned long long g2[NP], u2[NP];
-#pragma unroll
-      for (int p = 0; p < NP; ++p) g2[p] = u2[p] = 0ull;
-#pragma unroll
-      for (int q2 = 0; q2 < RP / 2; ++q2) {
-        const ulonglong2 pg = row[q2];
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          g2[p] = ffma2(pg.x, ug[p][2 * q2], g2[p]);
-          g2[p] = ffma2(pg.y, ug[p][2 * q2 + 1], g2[p]);
-        }
-      }
-#pragma unroll
-      for (int q2 = 0; q2 < RP / 2; ++q2) {
-        const ulonglong2 pu = row[RP / 2 + q2];
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          u2[p] = ffma2(pu.x, uu[p][2 * q2], u2[p]);
-          u2[p] = ffma2(pu.y, uu[p][2 * q2 + 1], u2[p]);
-        }
-      }
+    if (tb + kFmaTokens < t1) {
+      load_vals();                          // stage s + 1 (its rows are known)
+      load_rows(tb + 2 * kFmaTokens);       // rows of stage s + 2
+    }
+    // rank <= 8: two tokens per step (independent chains; a stage's rows past
+    // nt are zero); rank 16: one (its U rows fill the registers)
+    constexpr int TPS = RP <= 8 ? 2 : 1;
+    for (int tt = 0; tt < nt; tt += TPS) {
+      const uint32_t row = sp0 + uint32_t(tt) * (16u * RP);
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
-        // silu(g) u = g u / (1 + 2^(-g log2 e)), on both channels of the pair
-        const float2 x = unpack_f2(fmul2(g2[p], neg_log2e));
-        const unsigned long long den = fadd2(pack_f2(ex2_approx(x.x), ex2_approx(x.y)), one2);
-        const float2 dn = unpack_f2(den);
-        const unsigned long long inv = pack_f2(rcp_approx(dn.x), rcp_approx(dn.y));
-        const unsigned long long v = fmul2(fmul2(g2[p], inv), u2[p]);
-        acc[p] = ffma2(v, v, acc[p]);
+        unsigned long long ga, ua;
+        dots(row, p, ga, ua);
+        if constexpr (TPS == 2) {
+          unsigned long long gb, ub;
+          dots(row + 16u * RP, p, gb, ub);
+          tail(ga, ua, acc[p]);
+          tail(gb, ub, acc[p]);
+        } else {
+          tail(ga, ua, acc[p]);
+        }
       }
     }
   }
@@ -630,7 +684,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) ffn_score_fma_kernel(const _
 }
 
 template <int C>
-__global__ void __launch_bounds__(kScoreThreads) ffn_score_mma_kernel(const __grid_constant__ ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads)
+    ffn_score_mma_kernel(const __grid_constant__ ScoreArgs a) {
   constexpr int NT = score_nt(C), TW = score_tw(C), KB = 3 * C;
   constexpr int CH = kScoreWarps * NT * 8;  // channels per block
   extern __shared__ __align__(16) uint32_t s_stage[];
