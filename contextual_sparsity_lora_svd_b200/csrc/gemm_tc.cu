@@ -65,6 +65,31 @@ struct alignas(64) TcParams {
   CUtensorMap emap[6];
 };
 
+// One launch over the tiles of one or two GEMMs of the same epilogue kind
+// (a context-row GEMM and its output-row twin): tile t < tot0 is tile t of
+// p[0], the rest are p[1]'s, so the second GEMM's tiles fill the last round
+// of the first's.
+struct alignas(64) TcGroup {
+  TcParams p[2];
+  int ng;
+  int tot0, tot1;
+  int mpairs[2];
+};
+
+// The GEMM of combined tile t, its tile index and its M pair count.
+struct TcPick {
+  const TcParams* p;
+  int t, n_mpairs;
+};
+__device__ __forceinline__ TcPick tc_pick(const TcGroup& G, int t) {
+  TcPick k;
+  const bool second = t >= G.tot0;
+  k.p = &G.p[second ? 1 : 0];
+  k.t = second ? t - G.tot0 : t;
+  k.n_mpairs = G.mpairs[second ? 1 : 0];
+  return k;
+}
+
 // ------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -490,11 +515,11 @@ __device__ __forceinline__ void tma_load_s(uint32_t dst, const CUtensorMap* m, u
 //     are valid (per-row stores otherwise), and read back by ldmatrix as the
 //     A operand of the rank-R projections (mma.sync, fp32 partials).
 template <int R>
-__device__ __forceinline__ void tc2_bwd_epilogue(const TcParams& p, uint8_t* wbuf, uint64_t* eb,
+__device__ __forceinline__ void tc2_bwd_epilogue(const TcGroup& G, uint8_t* wbuf, uint64_t* eb,
                                                  uint64_t* tfull, uint64_t* tempty,
                                                  volatile int* abort, uint32_t tbase,
                                                  uint32_t rank, int q, int lane, int cluster_id,
-                                                 int n_clusters, int n_mpairs, int total) {
+                                                 int n_clusters, int total) {
   constexpr int RB = R > 0 ? R / 8 : 1;
   const int r = q * 32 + lane;
   const uint32_t sbuf = su32(wbuf);
@@ -508,7 +533,9 @@ __device__ __forceinline__ void tc2_bwd_epilogue(const TcParams& p, uint8_t* wbu
   for (int t = cluster_id; t < total && ok; t += n_clusters, ++it) {
     const int acc = it & 1;
     const uint32_t aph = uint32_t(it >> 1) & 1u;
-    const int mp = t % n_mpairs, nt = t / n_mpairs;
+    const TcPick pk = tc_pick(G, t);
+    const TcParams& p = *pk.p;
+    const int mp = pk.t % pk.n_mpairs, nt = pk.t / pk.n_mpairs;
     const int mt = 2 * mp + int(rank);
     int out_row = 0, nvalid = 0;
     if (mt < p.n_mtiles) {
@@ -625,7 +652,7 @@ __device__ __forceinline__ void tc2_bwd_epilogue(const TcParams& p, uint8_t* wbu
 }
 
 template <int kStages, bool kBwdTma>
-__global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant__ TcGroup G) {
   extern __shared__ uint8_t smem_raw2[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
@@ -665,8 +692,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
   cluster_sync_all();  // barriers of both CTAs initialised before any remote signal
   fence_after();
   const uint32_t tbase = *tmem_slot;
-  const int n_mpairs = (p.n_mtiles + 1) / 2;
-  const int total = n_mpairs * p.n_ntiles;
+  const int total = G.tot0 + G.tot1;
   const int cluster_id = blockIdx.x / 2, n_clusters = gridDim.x / 2;
 
   if (warp == 0) {
@@ -676,7 +702,9 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
     int issued = 0;
     bool ok = true;
     for (int t = cluster_id; t < total && ok; t += n_clusters) {
-      const int mp = t % n_mpairs, nt = t / n_mpairs;
+      const TcPick pk = tc_pick(G, t);
+      const TcParams& p = *pk.p;
+      const int mp = pk.t % pk.n_mpairs, nt = pk.t / pk.n_mpairs;
       const int mt = 2 * mp + int(rank);
       int a_row = 0;
       if (mt < p.n_mtiles) {
@@ -727,6 +755,7 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
       int it = 0;
       bool ok = true;
       for (int t = cluster_id; t < total && ok; t += n_clusters, ++it) {
+        const TcParams& p = *tc_pick(G, t).p;
         const int acc = it & 1;
         const uint32_t aph = uint32_t(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort)) break;
@@ -759,15 +788,16 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
   } else if (kBwdTma && warp >= 4) {
     uint8_t* wb = smem + kStages * STAGE2_BYTES + 1024 + (warp - 4) * EPI_WARP_BYTES;
     uint64_t* eb = ebar + 2 * (warp - 4);
-    if (p.proj_r == 16)
-      tc2_bwd_epilogue<16>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
-                           cluster_id, n_clusters, n_mpairs, total);
-    else if (p.proj_r == 8)
-      tc2_bwd_epilogue<8>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
-                          cluster_id, n_clusters, n_mpairs, total);
+    // the group's GEMMs share proj_r (checked on the host)
+    if (G.p[0].proj_r == 16)
+      tc2_bwd_epilogue<16>(G, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                           cluster_id, n_clusters, total);
+    else if (G.p[0].proj_r == 8)
+      tc2_bwd_epilogue<8>(G, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                          cluster_id, n_clusters, total);
     else
-      tc2_bwd_epilogue<0>(p, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
-                          cluster_id, n_clusters, n_mpairs, total);
+      tc2_bwd_epilogue<0>(G, wb, eb, tfull, tempty, abort, tbase, rank, warp - 4, lane,
+                          cluster_id, n_clusters, total);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int q = warp - 4;
@@ -783,7 +813,9 @@ __global__ void __launch_bounds__(256, 1) tc_gemm2_kernel(const __grid_constant_
       const uint32_t aph = uint32_t(it >> 1) & 1u;
       if (!mbar_wait(&tfull[acc], aph, abort)) break;
       fence_after();
-      const int mp = t % n_mpairs, nt = t / n_mpairs;
+      const TcPick pk = tc_pick(G, t);
+      const TcParams& p = *pk.p;
+      const int mp = pk.t % pk.n_mpairs, nt = pk.t / pk.n_mpairs;
       const int mt = 2 * mp + int(rank);
       int out_row = 0, nvalid = 0;
       if (mt < p.n_mtiles) {
@@ -968,7 +1000,11 @@ int64_t tc_ntiles(const TcGemm& g) {
   return (g.N + ncols - 1) / ncols;
 }
 
-slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
+namespace {
+// Kernel parameters of one GEMM; false in *run when it has no work.
+slora_status build_params(const TcGemm& g, TcParams* pp, bool* run, bool* bwd_tma,
+                          double* flops) {
+  *run = false;
   if (g.proj0 && ((g.proj_r != 8 && g.proj_r != 16) || g.ldproj % 8 ||
                   !g.proj_part || (g.epi == EPI_SWIGLU_BWD && !g.proj1) || g.epi == EPI_STORE ||
                   (reinterpret_cast<uintptr_t>(g.proj0) & 15) ||
@@ -983,12 +1019,13 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
     SLORA_FAIL(SLORA_ERR_ALIGN, "tcgen05 GEMM: SwiGLU operands need rows of whole 16 bytes");
   if (g.N > (int64_t(1) << 30)) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: N too large");
   SLORA_TRY(get_encode());
-  TcParams p;
+  TcParams& p = *pp;
   memset(&p, 0, sizeof(p));
   int64_t ksum = 0;
   for (int s = 0; s < g.nseg; ++s) {
     const TcSeg& sg = g.seg[s];
-    if (sg.K <= 0) SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: segment %d has K=%lld", s, (long long)sg.K);
+    if (sg.K <= 0)
+      SLORA_FAIL(SLORA_ERR_SHAPE, "tcgen05 GEMM: segment %d has K=%lld", s, (long long)sg.K);
     SLORA_TRY(encode(&p.amap[s], sg.a, BK, BM));
     if (sg.bmode != B_K && sg.bmode != B_MN)
       SLORA_FAIL(SLORA_ERR_INVALID_ARG, "tcgen05 GEMM: unknown B operand form %d", sg.bmode);
@@ -1028,18 +1065,11 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   p.proj_rows = g.proj_rows;
   p.in1 = g.in1;
   p.ldi = g.ldi;
-  if (!g_attr_set) {
-    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2, false>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES));
-    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2B, true>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2B_BYTES));
-    g_attr_set = true;
-  }
   // SwiGLU backward through shared memory: operands addressable by TMA
   auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15) == 0; };
-  const bool bwd_tma = g.epi == EPI_SWIGLU_BWD && !g.paired && g.io_rows > 0 &&
-                       al16(g.in0) && al16(g.in1) && al16(g.out0) && al16(g.out1);
-  if (bwd_tma) {
+  *bwd_tma = g.epi == EPI_SWIGLU_BWD && !g.paired && g.io_rows > 0 && al16(g.in0) &&
+             al16(g.in1) && al16(g.out0) && al16(g.out1);
+  if (*bwd_tma) {
     TcMat e;
     e.rows = g.io_rows;
     e.cols = g.N;
@@ -1063,15 +1093,54 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
       SLORA_TRY(encode(&p.emap[5], e, p.proj_r, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
   }
-  const int64_t ctiles = int64_t((p.n_mtiles + 1) / 2) * p.n_ntiles;
+  *flops = 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum);
+  *run = true;
+  return SLORA_OK;
+}
+
+// Up to two GEMMs in one launch (their tiles in one persistent schedule).
+slora_status launch_group(const TcGemm* const* gs, int n, cudaStream_t st) {
+  TcGroup G;  // copied into the launch's parameter buffer
+  memset(&G, 0, sizeof(G));
+  int ng = 0;
+  bool tma[2] = {false, false};
+  double flops = 0.0;
+  for (int i = 0; i < n; ++i) {
+    bool run = false;
+    double f = 0.0;
+    SLORA_TRY(build_params(*gs[i], &G.p[ng], &run, &tma[ng], &f));
+    if (!run) continue;
+    flops += f;
+    ++ng;
+  }
+  if (ng == 0) return SLORA_OK;
+  if (ng == 2 && (G.p[0].epi != G.p[1].epi || tma[0] != tma[1] ||
+                  G.p[0].proj_r != G.p[1].proj_r)) {
+    // different epilogue forms: one launch each
+    const TcGemm* a[1] = {gs[0]};
+    const TcGemm* b[1] = {gs[1]};
+    SLORA_TRY(launch_group(a, 1, st));
+    return launch_group(b, 1, st);
+  }
+  G.ng = ng;
+  for (int i = 0; i < ng; ++i) G.mpairs[i] = (G.p[i].n_mtiles + 1) / 2;
+  G.tot0 = G.mpairs[0] * G.p[0].n_ntiles;
+  G.tot1 = ng > 1 ? G.mpairs[1] * G.p[1].n_ntiles : 0;
+  if (!g_attr_set) {
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2_BYTES));
+    SLORA_CUDA(cudaFuncSetAttribute(tc_gemm2_kernel<STAGES2B, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM2B_BYTES));
+    g_attr_set = true;
+  }
+  const int64_t ctiles = int64_t(G.tot0) + G.tot1;
   const int64_t maxc = num_sms() / 2;
   const int nclus = int(ctiles < maxc ? ctiles : maxc);
-  LaunchScope ls(kGemmTC, 2.0 * double(g.M) * double(g.paired ? 2 * g.N : g.N) * double(ksum),
-                 st);
+  LaunchScope ls(kGemmTC, flops, st);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(2 * nclus), 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = bwd_tma ? SMEM2B_BYTES : SMEM2_BYTES;
+  cfg.dynamicSmemBytes = tma[0] ? SMEM2B_BYTES : SMEM2_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1080,11 +1149,22 @@ slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (bwd_tma)
-    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2B, true>, p));
+  if (tma[0])
+    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2B, true>, G));
   else
-    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2, false>, p));
+    SLORA_CUDA(cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<STAGES2, false>, G));
   return SLORA_OK;
+}
+}  // namespace
+
+slora_status gemm_tc(const TcGemm& g, cudaStream_t st) {
+  const TcGemm* gs[1] = {&g};
+  return launch_group(gs, 1, st);
+}
+
+slora_status gemm_tc_pair(const TcGemm& a, const TcGemm& b, cudaStream_t st) {
+  const TcGemm* gs[2] = {&a, &b};
+  return launch_group(gs, 2, st);
 }
 
 slora_status tc_check_error(bool clear) {

@@ -79,6 +79,10 @@ struct TcGemm {
 int64_t tc_ntiles(const TcGemm& g);
 
 slora_status gemm_tc(const TcGemm& g, cudaStream_t st);
+// Two GEMMs of the same epilogue kind (same projection rank and shared-memory
+// epilogue form) in one launch: the second's tiles fill the first's last
+// round.  Either may have no work.
+slora_status gemm_tc_pair(const TcGemm& a, const TcGemm& b, cudaStream_t st);
 
 // Device error flag of the tcgen05 kernels (a bounded wait that expired).
 slora_status tc_check_error(bool clear);

@@ -475,14 +475,15 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   }
   SLORA_TRY(join_side(st, side));
 
-  // ---- forward
+  // ---- forward (each context-row GEMM runs in one launch with its output-row twin)
+  TcGemm first;
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
     b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, 1, mat(WuS, kk, d, d))
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpC, nntC * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gC, uC, hC, ldk);
     if (proj) b.proj(AdtS, nullptr, lr, int(lr), projC, TC);
-    SLORA_TRY(gemm_tc(b.g, st));
+    first = b.g;
   }
   {  // gate|up, output rows, every channel
     TcBuilder b(otiles, nott, 0, 1, TO, Fd, 1, EPI_SWIGLU_FWD);
@@ -490,7 +491,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .seg(mat(XAb, T, 2 * r, lr2), mat(BpO, nntO * 256, 2 * r, lr2), B_K, 2 * r)
         .out(gO, uO, hO, Fd);
     if (proj) b.proj(Adt, nullptr, lr, int(lr), projO, TO);
-    SLORA_TRY(gemm_tc(b.g, st));
+    SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
   {  // hA = h Ad^T on the channels used: fp32 (full rows) and s*hA bf16 (compact)
     SkRowOut oc;
@@ -510,14 +511,14 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
     b.seg(mat(hC, TC, kk, ldk), mat(WdS, kk, d, d), B_MN, kk)
         .seg(mat(hAbC, TC, r, lr), mat(Bdp, d, r, lr), B_K, r)
         .out(out, nullptr, nullptr, d);
-    SLORA_TRY(gemm_tc(b.g, st));
+    first = b.g;
   }
   {  // down projection, output rows, dense
     TcBuilder b(otiles, nott, 1, 0, TO, d, 0, EPI_STORE);
     b.seg(mat(hO, TO, Fd, Fd), mat(L.Wd_t, Fd, d, d), B_MN, Fd)
         .seg(mat(hAbO, TO, r, lr), mat(Bdp, d, r, lr), B_K, r)
         .out(out, nullptr, nullptr, d);
-    SLORA_TRY(gemm_tc(b.g, st));
+    SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
 
   // ---- backward
@@ -543,7 +544,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .out(dGC, dUC, nullptr, ldk)
         .in(gC, uC, ldk, TC);
     if (proj) b.proj(BgS, BuS, lr, int(lr), projC, TC);
-    SLORA_TRY(gemm_tc(b.g, st));
+    first = b.g;
   }
   {
     TcBuilder b(otiles, nott, 0, 1, TO, Fd, 0, EPI_SWIGLU_BWD);
@@ -553,7 +554,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .in(gO, uO, Fd, TO);
     if (proj)
       b.proj(bpad ? BgP : L.Bg, bpad ? BuP : L.Bu, bpad ? lr : r, int(lr), projO, TO);
-    SLORA_TRY(gemm_tc(b.g, st));
+    SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
   if (proj) {  // dGB = [dG Bg | dU Bu] from the dh GEMMs' epilogue partials
     SkRowOut oc;
@@ -593,7 +594,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .seg(mat(dUC, TC, kk, ldk), mat(WuS, kk, d, d), B_MN, kk)
         .seg(mat(dGBbC, TC, 2 * r, lr2), mat(AgAu, 2 * r, d, d), B_MN, 2 * r)
         .out(dX, nullptr, nullptr, d);
-    SLORA_TRY(gemm_tc(b.g, st));
+    first = b.g;
   }
   {  // dX, output rows, dense
     TcBuilder b(otiles, nott, 1, 0, TO, d, 0, EPI_STORE);
@@ -601,7 +602,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .seg(mat(dUO, TO, Fd, Fd), mat(L.Wu, Fd, d, d), B_MN, Fd)
         .seg(mat(dGBbO, TO, 2 * r, lr2), mat(AgAu, 2 * r, d, d), B_MN, 2 * r)
         .out(dX, nullptr, nullptr, d);
-    SLORA_TRY(gemm_tc(b.g, st));
+    SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
   {  // dAg | dAu = s dGB^T X over every row, one stream of X
     SkColOut c;
@@ -847,18 +848,16 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   if (outr) {
     SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
     SLORA_TRY(gather_pad(L.B, r, L.idx, ni, r, BS, lr, st, n));
-    {  // context rows, output channels S
-      TcBuilder b(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
-      b.seg(mat(X_ctx, T, k, k), mat(WS, ni, k, k), B_K, k)
-          .seg(mat(XAb, T, r, lr), mat(BS, ni, r, lr), B_K, r)
-          .out(Y_ctx, nullptr, nullptr, ni);
-      SLORA_TRY(gemm_tc(b.g, st));
-    }
+    // context rows, output channels S, in one launch with the dense output rows
+    TcBuilder bc(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
+    bc.seg(mat(X_ctx, T, k, k), mat(WS, ni, k, k), B_K, k)
+        .seg(mat(XAb, T, r, lr), mat(BS, ni, r, lr), B_K, r)
+        .out(Y_ctx, nullptr, nullptr, ni);
     TcBuilder b(otiles, nott, 0, 1, TO, n, 0, EPI_STORE);  // output rows, dense
     b.seg(mat(X_ctx, T, k, k), mat(L.W, n, k, k), B_K, k)
         .seg(mat(XAb, T, r, lr), mat(Bp, n, r, lr), B_K, r)
         .out(Y_out, nullptr, nullptr, n);
-    return gemm_tc(b.g, st);
+    return gemm_tc_pair(bc.g, b.g, st);
   }
   // IN_COLS: W = W0^T [k x n]; context rows read input channels S only
   const void* Xc = X_ctx;
@@ -877,18 +876,15 @@ slora_status linear_fwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
     SLORA_TRY(rowdot(ykv(X_out, k), TO, k, rkv(L.A, kBF16, 1, k), r, oo, sw, st));
   }
   SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
-  {
-    TcBuilder b(ctiles, nct, 1, 0, TC, n, 0, EPI_STORE);
-    b.seg(mat(Xc, TC, ni, ldxc), mat(WS, ni, n, n), B_MN, ni)
-        .seg(mat(XAbC, TC, r, lr), mat(Bp, n, r, lr), B_K, r)
-        .out(Y_ctx, nullptr, nullptr, n);
-    SLORA_TRY(gemm_tc(b.g, st));
-  }
-  TcBuilder b(otiles, nott, 1, 0, TO, n, 0, EPI_STORE);
+  TcBuilder bc(ctiles, nct, 1, 0, TC, n, 0, EPI_STORE);  // context rows, input channels S
+  bc.seg(mat(Xc, TC, ni, ldxc), mat(WS, ni, n, n), B_MN, ni)
+      .seg(mat(XAbC, TC, r, lr), mat(Bp, n, r, lr), B_K, r)
+      .out(Y_ctx, nullptr, nullptr, n);
+  TcBuilder b(otiles, nott, 1, 0, TO, n, 0, EPI_STORE);  // output rows, dense
   b.seg(mat(X_out, TO, k, k), mat(L.W, k, n, n), B_MN, k)
       .seg(mat(XAbO, TO, r, lr), mat(Bp, n, r, lr), B_K, r)
       .out(Y_ctx, nullptr, nullptr, n);
-  return gemm_tc(b.g, st);
+  return gemm_tc_pair(bc.g, b.g, st);
 }
 
 slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const void* X_ctx,
@@ -973,19 +969,16 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
                        st));
     }
     SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
-    {  // dX, context rows: dY_C W0[S] + s dYB_C A
-      TcBuilder b(ctiles, nct, 1, 0, TC, k, 0, EPI_STORE);
-      b.seg(mat(dYc, TC, ni, lddc), mat(WS, ni, k, k), B_MN, ni)
+    {  // dX, context rows: dY_C W0[S] + s dYB_C A; output rows dense; one launch
+      TcBuilder bc(ctiles, nct, 1, 0, TC, k, 0, EPI_STORE);
+      bc.seg(mat(dYc, TC, ni, lddc), mat(WS, ni, k, k), B_MN, ni)
           .seg(mat(dYBbC, TC, r, lr), mat(L.A, r, k, k), B_MN, r)
           .out(dX_ctx, nullptr, nullptr, k);
-      SLORA_TRY(gemm_tc(b.g, st));
-    }
-    {
       TcBuilder b(otiles, nott, 1, 0, TO, k, 0, EPI_STORE);
       b.seg(mat(dY_out, TO, n, n), mat(L.W, n, k, k), B_MN, n)
           .seg(mat(dYBbO, TO, r, lr), mat(L.A, r, k, k), B_MN, r)
           .out(dX_ctx, nullptr, nullptr, k);
-      SLORA_TRY(gemm_tc(b.g, st));
+      SLORA_TRY(gemm_tc_pair(bc.g, b.g, st));
     }
     SkColOut ca;  // dA = s dYB^T X over every row
     ca.out = dA; ca.ldo = k; ca.trans = 1; ca.scale = s;
@@ -1007,19 +1000,16 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   SLORA_TRY(gather_rows(L.W, n, L.idx, ni, n, WS, n, st, k));
   SLORA_TRY(transpose_rows(L.A, r, k, L.idx, ni, lr, AS, st));
   SLORA_TRY(transpose_rows(L.A, r, k, nullptr, k, lr, At, st));
-  {  // dX_ctx = dY_C W0[:, S] + s dYB_C A[:, S]
-    TcBuilder b(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
-    b.seg(mat(dY_ctx, T, n, n), mat(WS, ni, n, n), B_K, n)
+  {  // dX_ctx = dY_C W0[:, S] + s dYB_C A[:, S]; dX_out dense; one launch
+    TcBuilder bc(ctiles, nct, 0, 1, TC, ni, 0, EPI_STORE);
+    bc.seg(mat(dY_ctx, T, n, n), mat(WS, ni, n, n), B_K, n)
         .seg(mat(dYBb, T, r, lr), mat(AS, ni, r, lr), B_K, r)
         .out(dX_ctx, nullptr, nullptr, ni);
-    SLORA_TRY(gemm_tc(b.g, st));
-  }
-  {
     TcBuilder b(otiles, nott, 0, 1, TO, k, 0, EPI_STORE);
     b.seg(mat(dY_ctx, T, n, n), mat(L.W, k, n, n), B_K, n)
         .seg(mat(dYBb, T, r, lr), mat(At, k, r, lr), B_K, r)
         .out(dX_out, nullptr, nullptr, k);
-    SLORA_TRY(gemm_tc(b.g, st));
+    SLORA_TRY(gemm_tc_pair(bc.g, b.g, st));
   }
   {  // dA: output rows over every column, then += context rows on columns S
     SkColOut ao;
