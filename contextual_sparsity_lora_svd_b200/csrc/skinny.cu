@@ -241,11 +241,13 @@ __device__ __forceinline__ float4 sum_splits4(const float4* src, int64_t stride4
 
 // Returns true in the one CTA (of the `n` sharing `counter`) that arrives last,
 // after every CTA's partial is visible; that CTA resets the counter.
+// The CTA's writes are ordered before thread 0's fence by the barrier, and
+// the fence (cumulative) publishes them all before the counter increment.
 __device__ __forceinline__ bool last_arrival(unsigned* counter, unsigned n, int tid) {
   __shared__ unsigned s_last;
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const unsigned prev = atomicAdd(counter, 1u);
     s_last = (prev + 1 == n) ? 1u : 0u;
     if (s_last) *counter = 0u;
@@ -663,9 +665,9 @@ __device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, 128;
 // the CTA that brings `counter` to n (and resets it).
 __device__ __forceinline__ bool last_arrival_c(unsigned* counter, unsigned n, int tid) {
   __shared__ unsigned s_last_c;
-  __threadfence();
   bar_consumers();
   if (tid == 0) {
+    __threadfence();  // publishes the consumer warps' partials (ordered by the barrier)
     const unsigned prev = atomicAdd(counter, 1u);
     s_last_c = (prev + 1 == n) ? 1u : 0u;
     if (s_last_c) *counter = 0u;
