@@ -742,7 +742,7 @@ def run_attn(args, H, pk, rank, world):
     w, fac = attn_weights_gpu(L, wf, d, Hh, KV, hd, (rs,), r, 2000, vo=True)
     base = build_attn(L, w, fac, d, Hh, KV, hd, rs, r, batch, seq, s, 2100 + 97 * rank)
     T = batch * seq
-    grads_flat = torch.cat([g.view(-1) for g in base.grads.values()])
+    grads_flat = base.gflat
     allreduce = (lambda: dp.allreduce_grads(grads_flat)) if world > 1 else None
     ws = torch.empty(base.workspace_bytes(), dtype=torch.uint8, device="cuda")
     g = H.capture(lambda: base.step(ws))
@@ -757,12 +757,17 @@ def run_attn(args, H, pk, rank, world):
     ms_step = ms / args.steps
     mhz = clk.summary().get("sm_mhz") or 1965.0
     # end to end: X, the attention-output stand-in and the upstream gradients
-    # go up, the four linears' outputs and the LoRA gradients come back
-    sets = [{"X": base.X, "attn_out": base.attn_out, "dY_o": base.dY_o,
-             "Yq": base.bufs["q"][0], "Yk": base.bufs["k"][0], "Yo": base.bufs["o"][0],
-             "dXq": base.dX["q"], "grads": grads_flat}] * 2
-    e2e_ms, h2d, d2h = e2e_measure(H, [g, g], sets, ("X", "attn_out", "dY_o"),
-                                   ("Yq", "Yk", "Yo", "dXq", "grads"), max(2, min(args.steps, 10)))
+    # go up, the four linears' outputs and the LoRA gradients come back; a
+    # second runner (same weights, its own buffers and inputs) double-buffers
+    base2 = build_attn(L, w, fac, d, Hh, KV, hd, rs, r, batch, seq, s, 2150 + 97 * rank)
+    g2 = H.capture(lambda: base2.step(ws))
+    sets = [{"X": b.X, "attn_out": b.attn_out, "dY_o": b.dY_o, "Yq": b.bufs["q"][0],
+             "Yk": b.bufs["k"][0], "Yo": b.bufs["o"][0], "dXq": b.dX["q"], "grads": b.gflat}
+            for b in (base, base2)]
+    e2e_ms, h2d, d2h = e2e_measure(H, [g, g2], sets, ("X", "attn_out", "dY_o"),
+                                   ("Yq", "Yk", "Yo", "dXq", "grads"), max(2, min(args.steps, 10)),
+                                   (lambda i: dp.allreduce_grads(sets[i]["grads"]))
+                                   if world > 1 else None)
     # the q/k estimator alone, by algorithmic bytes
     est = Estimator(L, L.CRIT_QK, base.X, batch, seq, [768] * batch, fac[rs]["Lq"],
                     fac[rs]["Uq"], fac[rs]["Lk"], fac[rs]["Uk"], rs, s, heads=Hh, kv=KV, hd=hd)

@@ -159,10 +159,17 @@ class AttnLinears(_Runner):
             return fwd, bwd
 
         r = r_lora
-        grads = {}
+        # the eight LoRA gradients are views of one flat fp32 buffer (one
+        # all-reduce, one read-back); every view starts on 16 bytes
+        shapes = []
         for nm, n, k in (("q", nq, d), ("k", nkv, d), ("v", nkv, d), ("o", d, nq)):
-            grads["dA" + nm] = torch.zeros(r, k, device="cuda")
-            grads["dB" + nm] = torch.zeros(n, r, device="cuda")
+            shapes += [("dA" + nm, (r, k)), ("dB" + nm, (n, r))]
+        sizes = [(a * b + 3) // 4 * 4 for _, (a, b) in shapes]
+        self.gflat = torch.zeros(sum(sizes), device="cuda")
+        grads, o = {}, 0
+        for (key, (a, b)), sz in zip(shapes, sizes):
+            grads[key] = self.gflat[o:o + a * b].view(a, b)
+            o += sz
         self.grads = grads
         self.dX = {nm: _bf16_empty(T, d) for nm in ("q", "k", "v")}
         fwds, bwds = [], []
