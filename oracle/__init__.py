@@ -13,3 +13,4 @@ to closed forms, invariants, brute force or finite differences; none of its
 results is "parity unpinned".
 """
 from .slora_oracle import *  # noqa: F401,F403
+from . import stack_oracle  # noqa: F401,E402
