@@ -87,6 +87,23 @@ _sig("slora_ffn_fwd_bwd", c_int,
       c_vp,
       ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 
+_sig("slora_rope_pack", c_int,
+     [c_int, ctypes.POINTER(Tokens), c_i64, c_int, ctypes.c_double, c_vp, c_i32, c_vp, c_vp, c_vp,
+      c_vp, c_vp, P_SZ, c_vp])
+_sig("slora_rope_unpack", c_int,
+     [c_int, ctypes.POINTER(Tokens), c_i64, c_int, ctypes.c_double, c_vp, c_i32, c_vp, c_vp, c_vp,
+      c_vp, c_vp, P_SZ, c_vp])
+_sig("slora_attention_fwd", c_int,
+     [c_int, ctypes.POINTER(Tokens), c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, P_SZ,
+      c_vp])
+_sig("slora_attention_bwd", c_int,
+     [c_int, ctypes.POINTER(Tokens), c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+      c_vp, c_vp, c_vp, P_SZ, c_vp])
+_sig("slora_rmsnorm_fwd", c_int,
+     [c_int, c_i64, c_i64, c_f32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
+_sig("slora_rmsnorm_bwd", c_int,
+     [c_int, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, P_SZ, c_vp])
+
 _sig("slora_noalloc_scratch_bytes", c_sz, [])
 _sig("slora_estimate_select_noalloc", c_int,
      [c_int, c_vp, c_int, ctypes.POINTER(Tokens), c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_i64,
@@ -101,7 +118,9 @@ EXPORTS = sorted(["slora_last_error_string", "slora_version", "slora_svd_prepare
                   "slora_ffn_fwd_bwd", "slora_launch_count", "slora_profile_enable",
                   "slora_profile_read", "slora_noalloc_scratch_bytes",
                   "slora_estimate_select_noalloc", "slora_device_error",
-                  "slora_set_wait_budget"])
+                  "slora_set_wait_budget", "slora_rope_pack", "slora_rope_unpack",
+                  "slora_attention_fwd", "slora_attention_bwd", "slora_rmsnorm_fwd",
+                  "slora_rmsnorm_bwd"])
 
 
 def lib():
@@ -129,7 +148,7 @@ def profile_read(kernel_class: str) -> tuple[int, float, float]:
 
 
 KERNEL_CLASSES = ["gemm_tc", "gemm_simt", "estimate", "select", "elementwise", "aux", "prepare",
-                  "skinny", "compact"]
+                  "skinny", "compact", "attention", "norm"]
 
 
 def ptr(x) -> int | None:
@@ -269,7 +288,8 @@ def ffn_args(dt, layer, batch, seq, ctx_len, sparsity, X, dOut, out, dX, grads, 
     k_out = c_i32(0)
     k_force = 0 if idx_force is None else idx_force.numel()
     args = [dt, ctypes.byref(layer), ctypes.byref(tok), float(sparsity), ptr(X), ptr(dOut),
-            ptr(out), ptr(dX), ctypes.byref(grads), ptr(idx_out), ctypes.byref(k_out),
+            ptr(out), ptr(dX), None if grads is None else ctypes.byref(grads), ptr(idx_out),
+            ctypes.byref(k_out),
             ptr(idx_force), k_force]
     return args, (tok, keep, k_out, layer, grads)
 
@@ -281,3 +301,54 @@ def slora_ffn_fwd_bwd(layer: FfnLayer, batch, seq, ctx_len, sparsity, X, dOut, o
                           grads, idx_out, idx_force)
     _run("slora_ffn_fwd_bwd", args, ws, stream)
     return int(keep[2].value)
+
+
+# ------------------------------------------- decoder-layer pieces
+ROPE_BASE = 10000.0
+RMS_EPS = 1e-5
+
+
+def slora_rope_pack(batch, seq, ctx_len, n, head_dim, Y_rot, Y=None, Y_ctx=None, Y_out=None,
+                    idx=None, rope_base=ROPE_BASE, ws=None, stream=None):
+    tok, keep = make_tokens(batch, seq, ctx_len)
+    n_idx = 0 if idx is None else idx.numel()
+    _run("slora_rope_pack", [BF16, ctypes.byref(tok), n, head_dim, float(rope_base), ptr(idx),
+                             n_idx, ptr(Y), ptr(Y_ctx), ptr(Y_out), ptr(Y_rot)], ws, stream)
+    del keep
+
+
+def slora_rope_unpack(batch, seq, ctx_len, n, head_dim, G, dY=None, dY_ctx=None, dY_out=None,
+                      idx=None, rope_base=ROPE_BASE, ws=None, stream=None):
+    tok, keep = make_tokens(batch, seq, ctx_len)
+    n_idx = 0 if idx is None else idx.numel()
+    _run("slora_rope_unpack", [BF16, ctypes.byref(tok), n, head_dim, float(rope_base), ptr(idx),
+                               n_idx, ptr(G), ptr(dY), ptr(dY_ctx), ptr(dY_out)], ws, stream)
+    del keep
+
+
+def slora_attention_fwd(batch, seq, heads, kv_heads, head_dim, Q, K, V, O, lse, stream=None):
+    tok, keep = make_tokens(batch, seq, [seq] * batch)
+    _run("slora_attention_fwd", [BF16, ctypes.byref(tok), heads, kv_heads, head_dim, ptr(Q),
+                                 ptr(K), ptr(V), ptr(O), ptr(lse)], None, stream)
+    del keep
+
+
+def slora_attention_bwd(batch, seq, heads, kv_heads, head_dim, Q, K, V, O, lse, dO, dQ, dK, dV,
+                        ws=None, stream=None):
+    tok, keep = make_tokens(batch, seq, [seq] * batch)
+    _run("slora_attention_bwd", [BF16, ctypes.byref(tok), heads, kv_heads, head_dim, ptr(Q),
+                                 ptr(K), ptr(V), ptr(O), ptr(lse), ptr(dO), ptr(dQ), ptr(dK),
+                                 ptr(dV)], ws, stream)
+    del keep
+
+
+def slora_rmsnorm_fwd(X, g, N=None, A=None, H=None, rstd=None, eps=RMS_EPS, stream=None):
+    T, d = X.shape
+    _run("slora_rmsnorm_fwd", [BF16, T, d, float(eps), ptr(X), ptr(A), ptr(g), ptr(H), ptr(N),
+                               ptr(rstd)], None, stream)
+
+
+def slora_rmsnorm_bwd(H, rstd, g, dN0, dX, dN1=None, dN2=None, dRes=None, stream=None):
+    T, d = H.shape
+    _run("slora_rmsnorm_bwd", [BF16, T, d, ptr(H), ptr(rstd), ptr(g), ptr(dN0), ptr(dN1),
+                               ptr(dN2), ptr(dRes), ptr(dX)], None, stream)

@@ -386,14 +386,21 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   const char* fn = "slora_ffn_fwd_bwd";
   clear_error();
   SLORA_TRY(check_dtype(fn, dt));
-  if (!layer || !grads) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: layer or grads is NULL", fn);
+  // dOut == NULL: forward only (dX and grads unused)
+  const bool fwd_only = dOut == nullptr;
+  if (!layer || (!grads && !fwd_only))
+    SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: layer or grads is NULL", fn);
   const slora_ffn_layer& Ly = *layer;
-  const slora_ffn_grads& Gr = *grads;
+  const slora_ffn_grads Gr = grads ? *grads : slora_ffn_grads{};
   REQ_PTR(Ly.Wg); REQ_PTR(Ly.Wu); REQ_PTR(Ly.Wd_t);
   REQ_PTR(Ly.Ag); REQ_PTR(Ly.Bg); REQ_PTR(Ly.Au); REQ_PTR(Ly.Bu); REQ_PTR(Ly.Ad); REQ_PTR(Ly.Bd);
-  REQ_PTR(X); REQ_PTR(dOut); REQ_PTR(out); REQ_PTR(dX); REQ_PTR(idx_out);
-  REQ_PTR(Gr.dAg); REQ_PTR(Gr.dBg); REQ_PTR(Gr.dAu); REQ_PTR(Gr.dBu); REQ_PTR(Gr.dAd);
-  REQ_PTR(Gr.dBd); OPT_PTR(ws); OPT_PTR(idx_force);
+  REQ_PTR(X); REQ_PTR(out); REQ_PTR(idx_out);
+  if (!fwd_only) {
+    REQ_PTR(dOut); REQ_PTR(dX);
+    REQ_PTR(Gr.dAg); REQ_PTR(Gr.dBg); REQ_PTR(Gr.dAu); REQ_PTR(Gr.dBu); REQ_PTR(Gr.dAd);
+    REQ_PTR(Gr.dBd);
+  }
+  OPT_PTR(ws); OPT_PTR(idx_force);
   if (!k_out) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: k_out is NULL", fn);
   SLORA_TRY(check_row(fn, "d", Ly.d, dt));
   SLORA_TRY(check_row(fn, "d_ff", Ly.d_ff, dt));

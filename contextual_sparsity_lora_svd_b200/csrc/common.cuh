@@ -110,7 +110,7 @@ inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 // ------------------------------------------------------------- launches
 // Kernel classes for launch accounting (names in slora_profile_read).
 enum KClass : int { kGemmTC = 0, kGemmSimt, kEstimate, kSelect, kElementwise, kAux, kPrepare,
-                    kSkinny, kCompact, kNumClasses };
+                    kSkinny, kCompact, kAttention, kNorm, kNumClasses };
 // Construct immediately before a kernel launch: counts it and, while
 // profiling is on, records CUDA events around it on `st`.
 struct LaunchScope {

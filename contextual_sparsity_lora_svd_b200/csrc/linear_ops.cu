@@ -520,6 +520,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .out(out, nullptr, nullptr, d);
     SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
+  if (!dOut) return SLORA_OK;  // forward only
 
   // ---- backward
   {  // dOB = dOut Bd: fp32 and s*dOB bf16
@@ -700,6 +701,7 @@ slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, c
     add(oo, rowmajor(hA, kF32, r, out_rows), rowmajor(L.Bd, dt, r), r, s);
     SLORA_TRY(gemm(oo, st));
   }
+  if (!dOut) return SLORA_OK;  // forward only
 
   // ---- backward
   {

@@ -264,7 +264,8 @@ extern "C" slora_status slora_set_wait_budget(int64_t cycles) {
 namespace slora {
 namespace {
 const char* kClassNames[kNumClasses] = {"gemm_tc", "gemm_simt", "estimate", "select",
-                                        "elementwise", "aux", "prepare", "skinny", "compact"};
+                                        "elementwise", "aux", "prepare", "skinny", "compact",
+                                        "attention", "norm"};
 struct Rec {
   int cls;
   double work;

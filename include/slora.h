@@ -136,10 +136,13 @@ slora_status slora_set_wait_budget(int64_t cycles);
  *                          "select" (top-k), "elementwise", "aux" (row maps,
  *                          operand packing), "prepare", "skinny" (rank-r
  *                          LoRA projections and gradients), "compact"
- *                          (selected-row gather).  It synchronizes the
+ *                          (selected-row gather), "attention" (the causal
+ *                          attention core and its rotary packing), "norm"
+ *                          (RMS normalisation).  It synchronizes the
  *                          recorded events.  work = algorithmic FLOPs for the
- *                          GEMM classes (2*M*N*K on the selected sizes), bytes
- *                          moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
+ *                          GEMM classes (2*M*N*K on the selected sizes) and
+ *                          the attention kernels (2 M N K per product over the
+ *                          causal tiles computed), bytes moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
  */
 int64_t slora_launch_count(void);
 void slora_profile_enable(int on);
@@ -346,6 +349,11 @@ typedef struct {
  *   idx_force optional device int32 [k_force] ascending channel set: skips the
  *             estimator and uses this set (same-index parity runs); then
  *             sparsity is ignored and k_keep = k_force.
+ *   dOut == NULL runs the forward only (estimate, select, out, idx_out); dX
+ *             and grads may then be NULL.  A layer stack runs its forwards
+ *             this way and, in the backward, calls again with dOut and the
+ *             forward's channel set as idx_force (the FFN forward recomputed
+ *             instead of stored).
  */
 slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
                                const slora_tokens* tok, double sparsity, const void* X,
@@ -353,6 +361,95 @@ slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
                                int32_t* idx_out, int32_t* k_out, const int32_t* idx_force,
                                int32_t k_force, void* ws, size_t* ws_bytes,
                                slora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The rest of a decoder layer around the sparse linears: rotary packing of
+ * the q/k rows, the causal attention core and RMS normalisation.  These make
+ * the whole-layer training step (sparse q/k feeding the attention core, v/o,
+ * the FFN, residuals and norms) run on this library's kernels.  The pages name
+ * Llama models without restating their layer; the plainest reading is taken:
+ * pre-normalised residual blocks, RMS norm with a frozen gain, rotate-half
+ * rotary embedding (pair i with i + head_dim/2, angle p * base^(-2i/head_dim)
+ * at position p counted from the start of the sequence), causal softmax
+ * attention within each sequence with scale 1/sqrt(head_dim), and query head
+ * h reading key/value head h / (heads / kv_heads).  A context row's skipped
+ * q/k channels are zero before the rotation [ART §1, §3].
+ *
+ * Every call takes (ws, ws_bytes, stream) like the calls above (ws == NULL
+ * queries the size; a call that needs none reports 0).  bf16 only
+ * (SLORA_F32: SLORA_ERR_UNSUPPORTED); head_dim 64 or 128; all pointers device,
+ * 16-byte aligned, rows contiguous.
+ * ---------------------------------------------------------------------- */
+
+/*
+ * slora_rope_pack — full-width rotated q or k rows for the attention core.
+ *   n          channels (heads * head_dim), a multiple of head_dim.
+ *   idx==NULL: Y [T x n] is the projection output; Y_ctx, Y_out unused.
+ *   idx!=NULL: Y_ctx [T_C x n_idx] holds the context rows' computed channels
+ *              idx (any order, each in [0, n)), Y_out [T_O x n] the dense
+ *              output rows; channels outside idx are zero on context rows.
+ *   Y_rot      [T x n] written: every head's pairs rotated by the row's angle.
+ */
+slora_status slora_rope_pack(slora_dtype dt, const slora_tokens* tok, int64_t n, int head_dim,
+                             double rope_base, const int32_t* idx, int32_t n_idx, const void* Y,
+                             const void* Y_ctx, const void* Y_out, void* Y_rot, void* ws,
+                             size_t* ws_bytes, slora_stream_t stream);
+
+/*
+ * slora_rope_unpack — transpose of slora_rope_pack for the gradient.
+ *   G [T x n] fp32 gradient of Y_rot.  idx==NULL: dY [T x n] written.
+ *   idx!=NULL: dY_ctx [T_C x n_idx] (kept channels) and dY_out [T_O x n]
+ *   written; the skipped channels of context rows had no computed output, so
+ *   their gradient is dropped.
+ */
+slora_status slora_rope_unpack(slora_dtype dt, const slora_tokens* tok, int64_t n, int head_dim,
+                               double rope_base, const int32_t* idx, int32_t n_idx,
+                               const float* G, void* dY, void* dY_ctx, void* dY_out, void* ws,
+                               size_t* ws_bytes, slora_stream_t stream);
+
+/*
+ * slora_attention_fwd — O = softmax(Q K^T / sqrt(head_dim) + causal mask) V
+ * per sequence and query head.
+ *   Q [T x heads*head_dim], K, V [T x kv_heads*head_dim] (rotated q/k).
+ *   O [T x heads*head_dim] written; lse [batch x heads x seq] fp32 written
+ *   (natural log-sum-exp of each row's scaled scores, for the backward).
+ */
+slora_status slora_attention_fwd(slora_dtype dt, const slora_tokens* tok, int heads,
+                                 int kv_heads, int head_dim, const void* Q, const void* K,
+                                 const void* V, void* O, float* lse, void* ws, size_t* ws_bytes,
+                                 slora_stream_t stream);
+
+/*
+ * slora_attention_bwd — gradients of slora_attention_fwd for the upstream dO.
+ *   dQ [T x heads*head_dim] and dK [T x kv_heads*head_dim] fp32, dV
+ *   [T x kv_heads*head_dim] in dt, all written (key/value gradients summed
+ *   over their query-head group).  dQ sums per-key-tile parts with atomic
+ *   adds: its rounding order is not fixed from run to run.
+ */
+slora_status slora_attention_bwd(slora_dtype dt, const slora_tokens* tok, int heads,
+                                 int kv_heads, int head_dim, const void* Q, const void* K,
+                                 const void* V, const void* O, const float* lse, const void* dO,
+                                 float* dQ, float* dK, void* dV, void* ws, size_t* ws_bytes,
+                                 slora_stream_t stream);
+
+/*
+ * slora_rmsnorm_fwd — H = X + A (A may be NULL: H = X and H is not written),
+ * N = H / sqrt(mean(H^2) + eps) * g per row; rstd [T] fp32 = 1/sqrt(mean(H^2)+eps).
+ *   X, A, H, N [T x d]; g [d]; d a multiple of 8.  N may be NULL (only the add).
+ */
+slora_status slora_rmsnorm_fwd(slora_dtype dt, int64_t T, int64_t d, float eps, const void* X,
+                               const void* A, const void* g, void* H, void* N, float* rstd,
+                               void* ws, size_t* ws_bytes, slora_stream_t stream);
+
+/*
+ * slora_rmsnorm_bwd — dX = dRes + J^T (dN0 + dN1 + dN2) for N = rmsnorm(H)
+ * with g frozen: J^T dN = rstd g dN - H rstd^3 mean(H g dN).  Any of dN1, dN2,
+ * dRes may be NULL (dN0 is required).  All [T x d] in dt; dX written.
+ */
+slora_status slora_rmsnorm_bwd(slora_dtype dt, int64_t T, int64_t d, const void* H,
+                               const float* rstd, const void* g, const void* dN0,
+                               const void* dN1, const void* dN2, const void* dRes, void* dX,
+                               void* ws, size_t* ws_bytes, slora_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -177,3 +177,63 @@ def test_estimate_select_query_variant_criteria(L):
     with pytest.raises(L.SloraError) as e:
         _est_query(L, 9, 688, 688, 0, 0, 0)
     assert e.value.status == 1
+
+
+# ------------------------------------------- decoder-layer pieces (host side)
+def _status(L, name, args):
+    need = ctypes.c_size_t(0)
+    return getattr(L.lib(), name)(*args, None, ctypes.byref(need), None), int(need.value)
+
+
+def test_attention_and_norm_validation(L):
+    tok, keep = L.make_tokens(2, 100, [75, 75])
+    a = lambda dt, H, KV, hd, q=FAKE: [dt, ctypes.byref(tok), H, KV, hd, q, FAKE, FAKE, FAKE, FAKE]
+    assert _status(L, "slora_attention_fwd", a(L.BF16, 4, 2, 128)) == (0, 0)
+    assert _status(L, "slora_attention_fwd", a(L.F32, 4, 2, 128))[0] == 5       # UNSUPPORTED
+    assert _status(L, "slora_attention_fwd", a(L.BF16, 4, 2, 96))[0] == 2       # SHAPE
+    assert _status(L, "slora_attention_fwd", a(L.BF16, 4, 3, 64))[0] == 2       # heads % kv
+    assert _status(L, "slora_attention_fwd", a(L.BF16, 4, 2, 64, FAKE + 8))[0] == 3  # ALIGN
+    bw = [L.BF16, ctypes.byref(tok), 4, 2, 64] + [FAKE] * 9
+    st, need = _status(L, "slora_attention_bwd", bw)
+    assert st == 0 and need >= 200 * 4 * 4       # D: one float per (row, query head)
+    nf = lambda T, d, A, N: [L.BF16, T, d, ctypes.c_float(1e-5), FAKE, A, FAKE, FAKE, N, FAKE]
+    assert _status(L, "slora_rmsnorm_fwd", nf(16, 64, None, FAKE))[0] == 0
+    assert _status(L, "slora_rmsnorm_fwd", nf(16, 60, None, FAKE))[0] == 2      # d % 8
+    assert _status(L, "slora_rmsnorm_fwd", nf(16, 64, None, None))[0] == 1      # nothing out
+    nb = [L.BF16, 16, 64, FAKE, FAKE, FAKE, None, None, None, None, FAKE]
+    assert _status(L, "slora_rmsnorm_bwd", nb)[0] == 1                          # dN0 required
+    del keep
+
+
+def test_rope_validation_and_workspace(L):
+    tok, keep = L.make_tokens(2, 100, [75, 70])
+    base = ctypes.c_double(10000.0)
+    dense = [L.BF16, ctypes.byref(tok), 512, 128, base, None, 0, FAKE, None, None, FAKE]
+    st, need_dense = _status(L, "slora_rope_pack", dense)
+    assert st == 0 and need_dense >= 100 * 64 * 8          # cos/sin table per (position, pair)
+    sliced = [L.BF16, ctypes.byref(tok), 512, 128, base, FAKE, 256, None, FAKE, FAKE, FAKE]
+    st, need = _status(L, "slora_rope_pack", sliced)
+    assert st == 0 and need >= need_dense + 200 * 4 + 512 * 4  # + row kinds and channel map
+    bad = list(sliced)
+    bad[3] = 96
+    assert _status(L, "slora_rope_pack", bad)[0] == 2
+    bad = list(sliced)
+    bad[6] = 513
+    assert _status(L, "slora_rope_pack", bad)[0] == 2                           # n_idx > n
+    bad = list(sliced)
+    bad[4] = ctypes.c_double(1.0)
+    assert _status(L, "slora_rope_pack", bad)[0] == 1                           # base <= 1
+    un = [L.BF16, ctypes.byref(tok), 512, 128, base, FAKE, 256, FAKE, None, FAKE, FAKE]
+    assert _status(L, "slora_rope_unpack", un)[0] == 0
+    un[9] = None                                                                # dY_out missing
+    assert _status(L, "slora_rope_unpack", un)[0] == 1
+    del keep
+
+
+def test_ffn_forward_only_needs_no_backward_buffers(L):
+    lay = L.ffn_layer_struct(256, 688, 8, 8, 1.0, *([FAKE] * 9), FAKE, FAKE, FAKE, FAKE)
+    args, keep = L.ffn_args(L.BF16, lay, 1, 256, [192], 0.5, FAKE, None, FAKE, None, None, FAKE)
+    assert L.workspace_size("slora_ffn_fwd_bwd", args) > 0
+    args, keep = L.ffn_args(L.BF16, lay, 1, 256, [192], 0.5, FAKE, FAKE, FAKE, None, None, FAKE)
+    with pytest.raises(L.SloraError):
+        L.workspace_size("slora_ffn_fwd_bwd", args)

@@ -1,0 +1,190 @@
+"""GPU parity of the decoder-layer pieces around the sparse linears, each
+called through the C ABI and compared with the float64 oracle on the same
+(bf16-rounded) inputs: rotary packing of sliced and dense q/k rows and its
+transpose, the causal attention core forward and backward (ragged tiles,
+grouped key/value heads, head widths 64 and 128, and sampled heads at the
+32-layer stack's full size), RMS normalisation forward and backward, and the
+forward-only mode of the FFN call."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import slora_oracle as SO
+from oracle import stack_oracle as S
+from contextual_sparsity_lora_svd_b200 import synth
+from tests.helpers import TOL, assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+TOLB = TOL["bf16"]
+
+
+@pytest.fixture(scope="module")
+def L():
+    from contextual_sparsity_lora_svd_b200 import _lib
+    return _lib
+
+
+def _bf(a):
+    return dev(a, torch.bfloat16)
+
+
+def _rb(a):
+    return synth.round_bf16(np.asarray(a, dtype=np.float64))
+
+
+# ------------------------------------------------------------------ rotary
+@pytest.mark.parametrize("hd,H,seq,ctx", [(128, 4, 100, [75, 60]), (64, 3, 37, [37, 0])])
+def test_rope_pack_unpack_sliced_and_dense(L, hd, H, seq, ctx):
+    b, n = 2, H * hd
+    rng = np.random.default_rng(hd + seq)
+    C, O = SO.context_rows(b, seq, ctx)
+    # per-head kept channels (ascending within each head), like the QK selection
+    idx = np.concatenate([h * hd + np.sort(rng.choice(hd, hd // 2, replace=False))
+                          for h in range(H)]).astype(np.int64)
+    Yc, Yo = _rb(rng.normal(size=(len(C), idx.size))), _rb(rng.normal(size=(len(O), n)))
+    out = torch.empty(b * seq, n, dtype=torch.bfloat16, device="cuda")
+    L.slora_rope_pack(b, seq, ctx, n, hd, out, Y_ctx=_bf(Yc), Y_out=_bf(Yo),
+                      idx=dev(idx, torch.int32))
+    want = S.rope_apply(S.assemble_qk(Yc, Yo, b, seq, ctx, n, idx), b, seq, hd)
+    got = host(out)
+    assert_close(got, want, TOLB, "rope pack (sliced)")
+    assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-6), "rope pack elementwise"
+    Y = _rb(rng.normal(size=(b * seq, n)))
+    L.slora_rope_pack(b, seq, ctx, n, hd, out, Y=_bf(Y))
+    assert_close(host(out), S.rope_apply(Y, b, seq, hd), TOLB, "rope pack (dense)")
+    # transpose on an fp32 gradient
+    G = rng.normal(size=(b * seq, n))
+    dYc = torch.zeros(len(C), idx.size, dtype=torch.bfloat16, device="cuda")
+    dYo = torch.zeros(len(O), n, dtype=torch.bfloat16, device="cuda")
+    L.slora_rope_unpack(b, seq, ctx, n, hd, dev(G, torch.float32), dY_ctx=dYc, dY_out=dYo,
+                        idx=dev(idx, torch.int32))
+    wc, wo = S.split_qk(S.rope_apply_t(G, b, seq, hd), b, seq, ctx, idx)
+    if len(C):
+        assert_close(host(dYc), wc, TOLB, "rope unpack ctx")
+    assert_close(host(dYo), wo, TOLB, "rope unpack out")
+    dY = torch.empty(b * seq, n, dtype=torch.bfloat16, device="cuda")
+    L.slora_rope_unpack(b, seq, ctx, n, hd, dev(G, torch.float32), dY=dY)
+    assert_close(host(dY), S.rope_apply_t(G, b, seq, hd), TOLB, "rope unpack dense")
+
+
+# ------------------------------------------------------------- attention
+def _attn_inputs(b, seq, H, KV, hd, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    Q = _rb(rng.normal(size=(b * seq, H * hd)) * scale)
+    K = _rb(rng.normal(size=(b * seq, KV * hd)) * scale)
+    V = _rb(rng.normal(size=(b * seq, KV * hd)))
+    dO = _rb(rng.normal(size=(b * seq, H * hd)))
+    return Q, K, V, dO
+
+
+def _attn_gpu(L, b, seq, H, KV, hd, Q, K, V, dO):
+    T = b * seq
+    q, k, v, do = _bf(Q), _bf(K), _bf(V), _bf(dO)
+    o = torch.empty(T, H * hd, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(b, H, seq, device="cuda")
+    L.slora_attention_fwd(b, seq, H, KV, hd, q, k, v, o, lse)
+    dq = torch.empty(T, H * hd, device="cuda")
+    dk = torch.empty(T, KV * hd, device="cuda")
+    dv = torch.empty(T, KV * hd, dtype=torch.bfloat16, device="cuda")
+    L.slora_attention_bwd(b, seq, H, KV, hd, q, k, v, o, lse, do, dq, dk, dv)
+    return host(o), host(lse), host(dq), host(dk), host(dv)
+
+
+@pytest.mark.parametrize("b,seq,H,KV,hd", [(2, 100, 4, 2, 128), (1, 64, 2, 2, 64),
+                                           (3, 130, 4, 1, 64), (1, 1, 2, 1, 128),
+                                           (2, 257, 2, 2, 128)])
+def test_attention_fwd_bwd_matches_oracle(L, b, seq, H, KV, hd):
+    # score scale ~ N(0, 1) per entry: softmax rows neither flat nor one-hot
+    Q, K, V, dO = _attn_inputs(b, seq, H, KV, hd, seed=seq + hd, scale=hd ** -0.25 * 1.5)
+    o, lse, dq, dk, dv = _attn_gpu(L, b, seq, H, KV, hd, Q, K, V, dO)
+    Ow, lw = S.attention_fwd(Q, K, V, b, seq, H, KV, hd)
+    assert_close(o, Ow, TOLB, "O")
+    assert np.max(np.abs(lse - lw)) < 2e-3, "lse"
+    # the backward of the oracle at the GPU's own (bf16) O, as the kernel uses it
+    dQw, dKw, dVw = S.attention_bwd(Q, K, V, _rb(Ow), lw, dO, b, seq, H, KV, hd)
+    assert_close(dq, dQw, TOLB, "dQ")
+    assert_close(dk, dKw, TOLB, "dK")
+    assert_close(dv, dVw, TOLB, "dV")
+
+
+def test_attention_full_size_sampled_heads(L):
+    """The 32-layer stack's attention shape (4 x 1024 tokens, 32 heads x 128);
+    heads are independent, so the oracle recomputes two sampled (sequence,
+    head) pairs from their own slices."""
+    b, seq, H, KV, hd = 4, 1024, 32, 32, 128
+    Q, K, V, dO = _attn_inputs(b, seq, H, KV, hd, seed=5, scale=hd ** -0.25 * 1.5)
+    o, lse, dq, dk, dv = _attn_gpu(L, b, seq, H, KV, hd, Q, K, V, dO)
+    for bb, h in ((0, 0), (3, 31), (2, 17)):
+        rows = slice(bb * seq, (bb + 1) * seq)
+        cols = slice(h * hd, (h + 1) * hd)
+        q, k, v, do = Q[rows, cols], K[rows, cols], V[rows, cols], dO[rows, cols]
+        Ow, lw = S.attention_fwd(q, k, v, 1, seq, 1, 1, hd)
+        assert_close(o[rows, cols], Ow, TOLB, f"O ({bb},{h})")
+        assert np.max(np.abs(lse[bb, h] - lw[0, 0])) < 2e-3
+        dQw, dKw, dVw = S.attention_bwd(q, k, v, _rb(Ow), lw, do, 1, seq, 1, 1, hd)
+        assert_close(dq[rows, cols], dQw, TOLB, f"dQ ({bb},{h})")
+        assert_close(dk[rows, cols], dKw, TOLB, f"dK ({bb},{h})")
+        assert_close(dv[rows, cols], dVw, TOLB, f"dV ({bb},{h})")
+
+
+# -------------------------------------------------------------- RMS norm
+@pytest.mark.parametrize("T,d", [(37, 256), (8, 4096)])
+def test_rmsnorm_fwd_bwd_matches_oracle(L, T, d):
+    rng = np.random.default_rng(T + d)
+    X, A = _rb(rng.normal(size=(T, d)) * 2), _rb(rng.normal(size=(T, d)))
+    g = _rb(1.0 + 0.1 * rng.normal(size=d))
+    Hh = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    N = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    rstd = torch.empty(T, device="cuda")
+    L.slora_rmsnorm_fwd(_bf(X), _bf(g), N=N, A=_bf(A), H=Hh, rstd=rstd)
+    Hw = _rb(X + A)
+    assert np.array_equal(host(Hh), Hw), "residual sum rounds once"
+    Nw, rw = S.rmsnorm_fwd(Hw, g)
+    assert_close(host(N), Nw, TOLB, "N")
+    np.testing.assert_allclose(host(rstd), rw, rtol=1e-5)
+    dN = [_rb(rng.normal(size=(T, d))) for _ in range(3)]
+    dR = _rb(rng.normal(size=(T, d)))
+    dX = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    L.slora_rmsnorm_bwd(Hh, rstd, _bf(g), _bf(dN[0]), dX, dN1=_bf(dN[1]), dN2=_bf(dN[2]),
+                        dRes=_bf(dR))
+    want = dR + S.rmsnorm_bwd(Hw, g, rw, dN[0] + dN[1] + dN[2])
+    assert_close(host(dX), want, TOLB, "dX")
+    L.slora_rmsnorm_bwd(Hh, rstd, _bf(g), _bf(dN[0]), dX)
+    assert_close(host(dX), S.rmsnorm_bwd(Hw, g, rw, dN[0]), TOLB, "dX (one branch)")
+
+
+# ----------------------------------------------------- FFN forward only
+def test_ffn_forward_only_equals_the_full_call(L):
+    """dOut = NULL runs the forward only: same output and channel set as the
+    forward half of the full call, on the estimator path and on a forced set."""
+    tok = synth.Tokens(2, 96, np.array([70, 50], np.int32))
+    case = synth.ffn_case(tok, d=128, d_ff=344, r_svd=8, r_lora=8, sparsity=0.5, bf16=True,
+                          workload=0, layer=7)
+    Ls, Us = {}, {}
+    for m, W in (("g", case.Wg.W), ("u", case.Wu.W)):
+        Ls[m], Us[m] = SO.svd_prepare(W, 8)
+    t = {k: _bf(getattr(case, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    t.update(Wg=_bf(case.Wg.W), Wu=_bf(case.Wu.W), Wd_t=_bf(case.Wd.W.T.copy()))
+    f = {k: dev(v, torch.float32) for k, v in
+         (("Lg", Ls["g"]), ("Ug", Us["g"]), ("Lu", Ls["u"]), ("Uu", Us["u"]))}
+    layer = L.ffn_layer_struct(128, 344, 8, 8, 1.0, t["Wg"], t["Wu"], t["Wd_t"], t["Ag"], t["Bg"],
+                               t["Au"], t["Bu"], t["Ad"], t["Bd"], f["Lg"], f["Ug"], f["Lu"],
+                               f["Uu"])
+    X, dOut = _bf(case.X), _bf(case.dOut)
+    T = tok.T
+    for force in (None, dev(np.arange(0, 344, 3), torch.int32)):
+        outs, idxs = [], []
+        for full in (True, False):
+            out = torch.empty(T, 128, dtype=torch.bfloat16, device="cuda")
+            idx = torch.empty(344, dtype=torch.int32, device="cuda")
+            g = [torch.empty(*sh, device="cuda") for sh in
+                 [(8, 128), (344, 8), (8, 128), (344, 8), (8, 344), (128, 8)]]
+            G = L.ffn_grads_struct(*g) if full else None
+            dX = torch.empty_like(out) if full else None
+            k = L.slora_ffn_fwd_bwd(layer, tok.batch, tok.seq, tok.ctx_len, 0.5, X,
+                                    dOut if full else None, out, dX, G, idx, idx_force=force)
+            torch.cuda.synchronize()
+            outs.append(host(out))
+            idxs.append(host(idx[:k]))
+        assert np.array_equal(outs[0], outs[1])
+        assert np.array_equal(idxs[0], idxs[1])
