@@ -19,6 +19,10 @@ weights; `--workload`, default the first):
   llama3-8b-layer-bf16    one Llama-3-8B-shaped layer (d_ff=14336, GQA 32 q /
                           8 kv heads), 8192 tokens: sparsity x SVD-rank sweep
                           at seq 1024 and a sequence sweep at 50% / rank 8.
+  llama2-7b-decoder32-bf16  the 32-layer stack's whole training step with the
+                          attention core, RMS norms and residuals (forward of
+                          every layer, then backward), beside the same stack
+                          run dense.
 
 Prints one JSON line (rank 0).
 
@@ -55,7 +59,7 @@ from contextual_sparsity_lora_svd_b200 import synth  # noqa: E402
 METRIC = "sparse LoRA fwd+bwd tokens/s; sliced-GEMM % bf16 peak; estimator HBM GB/s"
 UNIT = "tokens/s"
 WORKLOAD_NAMES = ["llama2-7b-ffn-bf16", "llama2-7b-attn-qk-bf16", "llama2-7b-stack32-bf16",
-                  "llama3-8b-layer-bf16"]
+                  "llama3-8b-layer-bf16", "llama2-7b-decoder32-bf16"]
 
 
 # ------------------------------------------------------------------ peaks
@@ -196,6 +200,22 @@ def workload_config(name, world):
                 "v_o": "dense LoRA",
                 "excluded": "attention core, norms, embeddings (their tensors are synthetic; "
                             "every layer reads the same X)", "parallelism": par, "l2": L2_NOTE}
+    if name == "llama2-7b-decoder32-bf16":
+        from contextual_sparsity_lora_svd_b200.schedule import llama2_7b_stack
+        w = synth.WORKLOADS[3]
+        t = llama2_7b_stack()
+        return {"workload": name, "model": "32 Llama-2-7B decoder layers: RMS norms, q/k/v/o "
+                                           "LoRA linears, rotary embedding, causal attention, "
+                                           "residuals, SwiGLU FFN",
+                "global_batch": w["batch"] * world, "seq_len": w["seq"], "layers": w["layers"],
+                "d": w["d"], "d_ff": w["d_ff"], "heads": w["heads"], "r_svd": w["r_svd"],
+                "r_lora": w["r_lora"], "ffn_sparsity": list(t.ffn), "qk_sparsity": list(t.qk),
+                "v_o": "dense LoRA", "ffn_backward": "forward recomputed from the saved FFN "
+                                                     "input with the forward's channel set",
+                "excluded": "embeddings, final norm and loss (a synthetic output gradient)",
+                "parallelism": par, "l2": L2_NOTE,
+                "launch": "the whole step (forward of 32 layers, then backward) captured as one "
+                          "CUDA graph"}
     w = synth.WORKLOADS[4]
     return {"workload": name, "model": "Llama-3-8B layer: q/k/v/o LoRA linears (GQA 32/8) + "
                                        "SwiGLU FFN",
@@ -920,6 +940,146 @@ def run_stack(args, H, pk, rank, world):
     return line
 
 
+# ============================================================ decoder stack
+def decoder_weights(L, wf, d, F, Hh, KV, hd, rs, r, seed):
+    """One decoder layer's device tensors: attention and FFN weights with their
+    LoRA pairs and estimator factors, and the two RMS gains."""
+    fw, ffac = ffn_weights_gpu(L, wf, d, F, (rs,), r, seed)
+    fw["Lg"], fw["Ug"], fw["Lu"], fw["Uu"] = ffac[rs]
+    aw, afac = attn_weights_gpu(L, wf, d, Hh, KV, hd, (rs,), r, seed)
+    w = dict(fw)
+    w.update(aw)
+    w.update(afac[rs])
+    g = torch.Generator(device="cuda").manual_seed(int(seed) + 40)
+    for k in ("g1", "g2"):
+        w[k] = (1.0 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(torch.bfloat16)
+    return w
+
+
+def oracle_decoder_layer(d, F, Hh, KV, hd, rs, r, _cache={}):
+    """Random-weight float64 layer of the given shapes for the oracle timing
+    (the timing does not depend on the spectrum)."""
+    key = (d, F, Hh, KV, hd, rs, r)
+    if key not in _cache:
+        rng = np.random.default_rng(11)
+        lay = {"scale": 1.0}
+        for nm, n, k in (("q", Hh * hd, d), ("k", KV * hd, d), ("v", KV * hd, d),
+                         ("o", d, Hh * hd), ("g", F, d), ("u", F, d), ("d", d, F)):
+            lay["W" + nm] = rng.standard_normal((n, k)) / np.sqrt(k)
+            lay["A" + nm] = rng.standard_normal((r, k)) * 0.02
+            lay["B" + nm] = rng.standard_normal((n, r)) * 0.02
+            if nm in ("q", "k", "g", "u"):
+                lay["L" + nm] = rng.standard_normal((k, rs)) / np.sqrt(k)
+                lay["U" + nm] = rng.standard_normal((n, rs)) / np.sqrt(rs)
+        lay["g1"] = 1.0 + 0.1 * rng.standard_normal(d)
+        lay["g2"] = 1.0 + 0.1 * rng.standard_normal(d)
+        _cache.clear()
+        _cache[key] = lay
+    return _cache[key]
+
+
+def oracle_decoder_time(seq, d, F, Hh, KV, hd, rs, r, s_qk, s_ffn):
+    """Seconds of the oracle's step (forward with its own selections, then
+    backward) for one decoder layer on 1 x seq tokens."""
+    from oracle import stack_oracle as S
+    lay = oracle_decoder_layer(d, F, Hh, KV, hd, rs, r)
+    rng = np.random.default_rng(12)
+    x, dy = rng.standard_normal((seq, d)), rng.standard_normal((seq, d))
+    ctx = [seq - int(round(0.25 * seq))]
+    t0 = time.perf_counter()
+    S.stack_fwd_bwd(x, dy, [lay], 1, seq, ctx, Hh, KV, hd, qk_sparsity=[s_qk],
+                    ffn_sparsity=[s_ffn])
+    return time.perf_counter() - t0
+
+
+def run_decoder(args, H, pk, rank, world):
+    """The 32-layer decoder stack's whole training step (layers.DecoderStack):
+    sparse q/k feeding the attention core, v/o, residuals, RMS norms and the
+    sparse FFN, forward through all layers then backward, with the per-layer
+    ratio table; and the same stack dense (every layer at ratio 0)."""
+    from contextual_sparsity_lora_svd_b200 import dp
+    from contextual_sparsity_lora_svd_b200.layers import DecoderStack
+    from contextual_sparsity_lora_svd_b200.schedule import ProgressiveSchedule, llama2_7b_stack
+    L = H.L
+    wl = synth.WORKLOADS[3]
+    d, F, Hh, KV, hd = wl["d"], wl["d_ff"], wl["heads"], wl["kv_heads"], wl["head_dim"]
+    rs, r, batch, seq, nl = wl["r_svd"], wl["r_lora"], wl["batch"], wl["seq"], wl["layers"]
+    T = batch * seq
+    ctx = [seq - int(round(0.25 * seq))] * batch
+    table = llama2_7b_stack()
+    wf = WeightFactory()
+    X = randn_bf16((T, d), 3000 + 97 * rank)
+    dY = randn_bf16((T, d), 3001 + 97 * rank)
+    t_setup = time.perf_counter()
+    layers = [decoder_weights(L, wf, d, F, Hh, KV, hd, rs, r, 3100 + 10 * l) for l in range(nl)]
+    torch.cuda.synchronize()
+    t_setup = time.perf_counter() - t_setup
+    sparse = DecoderStack(layers, d, Hh, KV, hd, F, rs, r, 1.0, batch, seq, ctx, list(table.qk),
+                          list(table.ffn), X, dY)
+    ws = torch.empty(sparse.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    allreduce = (lambda: dp.allreduce_grads(sparse.gflat)) if world > 1 else None
+    g = H.capture(lambda: sparse.step(ws))
+    for _ in range(args.warmup):
+        g.replay()
+        if allreduce:
+            allreduce()
+    with ClockSampler(H.dev) as clk:
+        ms = H.time_steps(g.replay, args.steps, allreduce)
+    ms_prof, launches, prof = H.profile(lambda: sparse.step(ws), args.steps, allreduce)
+    ms = dp.max_over_ranks(ms, device="cuda")
+    ms_sparse = ms / args.steps
+    e2e_steps = max(2, min(args.steps, 5))
+    sets = [{"X": X, "dY": dY, "grads": sparse.gflat}] * 2
+    e2e_ms, h2d, d2h = e2e_measure(H, [g, g], sets, ("X", "dY"), ("grads",), e2e_steps)
+    del g
+    del sparse
+    torch.cuda.empty_cache()
+    # the same stack with every layer dense (the first phase of the schedule)
+    dense = DecoderStack(layers, d, Hh, KV, hd, F, rs, r, 1.0, batch, seq, ctx, [0.0] * nl,
+                         [0.0] * nl, X, dY)
+    wsd = torch.empty(dense.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    gd = H.capture(lambda: dense.step(wsd))
+    gd.replay()
+    nd = max(2, args.steps // 2)
+    ms_dense = dp.max_over_ranks(H.time_steps(gd.replay, nd), device="cuda") / nd
+    del gd, dense, wsd
+    sch = ProgressiveSchedule(table, total_steps=1000)
+    run_ms = sum(n * (ms_dense if f == 0.0 else ms_sparse) for _, n, f in sch.phases())
+    n_a, ms_a, fl_a = prof["attention"]
+    att = fl_a / (ms_a / 1e3) / 1e12 if ms_a > 0 else 0.0
+    line = {"metric": METRIC, "value": world * T / (ms_sparse / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_sparse, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded inputs, random-init decaying-spectrum weights built on "
+                    "the GPU, distinct per layer)",
+            "config": workload_config("llama2-7b-decoder32-bf16", world),
+            "roofline": gemm_roofline(prof, pk),
+            "attention_core": {"kernels": "attn_fwd_kernel / attn_bwd_kernel (mma.sync "
+                                          "m16n8k16)", "achieved": att, "unit": "TFLOP/s",
+                               "peak": pk["bf16"], "frac": att / pk["bf16"],
+                               "ms_per_step": ms_a / args.steps,
+                               "flops_per_step": fl_a / args.steps},
+            "dense_vs_sparse": {"dense_ms_per_step": ms_dense, "sparse_ms_per_step": ms_sparse,
+                                "speedup": ms_dense / ms_sparse,
+                                "run_steps": 1000, "dense_steps": sch.dense_steps,
+                                "run_tokens_per_s": world * T * 1000 / (run_ms / 1e3)},
+            "kernels": kernel_table(prof, args.steps, ms_prof), "gpu_launches": int(launches),
+            "clocks": clk.summary(), "setup_s": t_setup,
+            "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "profiled_ms_per_step": ms_prof / args.steps, "impl": "ours"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        set_threads()
+        t = oracle_decoder_time(1024, d, F, Hh, KV, hd, rs, r, table.qk[17], table.ffn[17])
+        line["cpu_baseline"] = {"value": 1024 / (nl * t), "unit": UNIT, "cores": host_cores(),
+                                "kind": "oracle",
+                                "sample": "one decoder layer (layer 17 ratios) on 1 x 1024 "
+                                          "tokens, random weights of its shapes, fp64 NumPy "
+                                          "oracle, time x 32 layers"}
+    return line
+
+
 # ========================================================== llama3 sweep
 def run_llama3(args, H, pk, rank, world):
     from contextual_sparsity_lora_svd_b200.layers import FfnLayer
@@ -999,7 +1159,8 @@ def run_llama3(args, H, pk, rank, world):
 
 
 RUNNERS = {"llama2-7b-ffn-bf16": run_ffn, "llama2-7b-attn-qk-bf16": run_attn,
-           "llama2-7b-stack32-bf16": run_stack, "llama3-8b-layer-bf16": run_llama3}
+           "llama2-7b-stack32-bf16": run_stack, "llama3-8b-layer-bf16": run_llama3,
+           "llama2-7b-decoder32-bf16": run_decoder}
 
 
 # ------------------------------------------------------------- reference
@@ -1017,6 +1178,15 @@ def run_reference(args, rank, world):
     elif name == "llama2-7b-attn-qk-bf16":
         fn, T = (lambda: oracle_attn_time(1, 1024, 4096, 32, 32, 128, 8, 16, 0.5)), 1024
         sample = "1 x 1024 tokens (ctx 768 + out 256) of the layer's q/k/v/o linears"
+    elif name == "llama2-7b-decoder32-bf16":
+        from contextual_sparsity_lora_svd_b200.schedule import llama2_7b_stack
+        t = llama2_7b_stack()
+
+        def fn():
+            return 32 * oracle_decoder_time(1024, 4096, 11008, 32, 32, 128, 8, 16, t.qk[17],
+                                            t.ffn[17])
+        T = 1024
+        sample = "1 x 1024 tokens of one decoder layer (layer 17 ratios), x 32 layers"
     else:
         wl = synth.WORKLOADS[3 if name == "llama2-7b-stack32-bf16" else 4]
         F, KV = wl["d_ff"], wl["kv_heads"]
@@ -1035,7 +1205,8 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         t0 = time.perf_counter()
         r = fn()
-        ts.append(r if name in ("llama2-7b-stack32-bf16", "llama3-8b-layer-bf16")
+        ts.append(r if name in ("llama2-7b-stack32-bf16", "llama3-8b-layer-bf16",
+                                "llama2-7b-decoder32-bf16")
                   else time.perf_counter() - t0)
     v = T / float(np.mean(ts))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,

@@ -668,7 +668,7 @@ slora_status rope_run(bool backward, const void* Y, const void* Yc, const void* 
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "rope"));
   {
-    LaunchScope ls(kAttention, double(ti.seq) * half * 8, st);
+    LaunchScope ls(kAux, double(ti.seq) * half * 8, st);
     rope_table_kernel<<<blocks_for(int64_t(ti.seq) * half, 256), 256, 0, st>>>(tab, ti.seq, half,
                                                                                base);
     SLORA_CHECK_LAUNCH();
@@ -694,7 +694,7 @@ slora_status rope_run(bool backward, const void* Y, const void* Yc, const void* 
   }
   const int64_t threads = ti.T * int64_t(n / hd) * (hd / 4);
   const double bytes = backward ? double(ti.T) * n * 6 : double(ti.T) * n * 4;
-  LaunchScope ls(kAttention, bytes, st);
+  LaunchScope ls(kElementwise, bytes, st);
   if (!backward) {
     rope_pack_kernel<<<blocks_for(threads, 256), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(Y), static_cast<const __nv_bfloat16*>(Yc),
@@ -709,11 +709,12 @@ slora_status rope_run(bool backward, const void* Y, const void* Yc, const void* 
   return SLORA_OK;
 }
 
-// Algorithmic FLOPs of one causal product (2 M N K) over the 64 x 64 tiles a
-// kernel computes: per sequence and head, nq (nq + 1) / 2 tiles.
-static double causal_tile_flops(const TokenInfo& ti, int heads, int hd) {
-  const double nq = double((ti.seq + kBM - 1) / kBM);
-  return 2.0 * kBM * kBN * hd * nq * (nq + 1) / 2 * heads * ti.batch;
+// Algorithmic FLOPs of one causal product: 2 hd per (query, key <= query)
+// pair, seq (seq + 1) / 2 pairs per sequence and head (the masked halves of
+// the diagonal tiles the kernels also compute are not counted).
+static double causal_flops(const TokenInfo& ti, int heads, int hd) {
+  const double s = double(ti.seq);
+  return 2.0 * hd * s * (s + 1) / 2 * heads * ti.batch;
 }
 
 slora_status attention_fwd_run(const void* Q, const void* K, const void* V, const TokenInfo& ti,
@@ -728,7 +729,7 @@ slora_status attention_fwd_run(const void* Q, const void* K, const void* V, cons
   p.nqb = (ti.seq + kBM - 1) / kBM;
   p.sl2 = float(1.0 / std::sqrt(double(hd)) * 1.4426950408889634);
   const dim3 grid(p.nqb, H, ti.batch);
-  LaunchScope ls(kAttention, 2.0 * causal_tile_flops(ti, H, hd), st);
+  LaunchScope ls(kAttention, 2.0 * causal_flops(ti, H, hd), st);
   if (hd == 128) {
     SLORA_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<128>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem<128>()));
@@ -751,7 +752,7 @@ slora_status attention_bwd_run(const void* Q, const void* K, const void* V, cons
   SLORA_TRY(arena_fits(ar, "attention_bwd"));
   SLORA_CUDA(cudaMemsetAsync(dQ, 0, size_t(ti.T) * H * hd * sizeof(float), st));
   {
-    LaunchScope ls(kAttention, double(ti.T) * H * hd * 4, st);
+    LaunchScope ls(kElementwise, double(ti.T) * H * hd * 4, st);
     const int64_t thr = ti.T * H * 32;
     if (hd == 128)
       attn_rowdot_kernel<128><<<blocks_for(thr, 256), 256, 0, st>>>(
@@ -775,7 +776,7 @@ slora_status attention_bwd_run(const void* Q, const void* K, const void* V, cons
   p.scale = float(1.0 / std::sqrt(double(hd)));
   p.sl2 = float(double(p.scale) * 1.4426950408889634);
   const dim3 grid(p.nqb, KV, ti.batch);
-  LaunchScope ls(kAttention, 5.0 * causal_tile_flops(ti, H, hd), st);
+  LaunchScope ls(kAttention, 5.0 * causal_flops(ti, H, hd), st);
   if (hd == 128) {
     SLORA_CUDA(cudaFuncSetAttribute(attn_bwd_kernel<128>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, bwd_smem<128>()));

@@ -252,3 +252,236 @@ class AttnLinears(_Runner):
         # step: estimators, forwards (q, k, v, o), backwards in reverse order
         self.calls = calls + fwds + bwds[::-1]
         self.X, self.attn_out, self.dY_o = X, attn_out, dY_o
+
+
+class DecoderStack(_Runner):
+    """One training step of a stack of decoder layers, every number on
+    libslora's kernels:
+
+      forward, per layer:  n1 = rms(x); q/k channel selection on n1 (QK-norm,
+        per head) for sparse layers; q, k (sliced on context rows), v, o LoRA
+        linears; rotary packing of q, k; causal attention; h = x + o(attn);
+        n2 = rms(h); FFN forward only (its own estimate + select);
+        x' = h + ffn (fused into the next normalisation);
+      backward, last layer first: the FFN again with its forward channel set
+        (forward recomputed, then the sparse backward), the norm backward with
+        the residual, o backward, attention backward, rotary unpacking, q/k/v
+        backward, the norm backward summing the three branch gradients and the
+        residual.
+
+    `layers` holds one dict per layer of device tensors: g1, g2 (RMS gains,
+    bf16 [d]), Wq, Wk, Wv, Wo and their A*/B* LoRA factors, the FFN weights
+    Wg, Wu, Wd_t with Ag..Bd, and the fp32 estimator factors Lq, Uq, Lk, Uk,
+    Lg, Ug, Lu, Uu.  `qk_sparsity` / `ffn_sparsity` give each layer's ratio (0:
+    dense).  X [T x d] is the stack input, dY [T x d] the gradient of its
+    output.  After step(): `y` is the output, `dX` the input gradient,
+    `grads[l]` layer l's LoRA gradients (views of `gflat`), `idx_qk[l]` /
+    `idx_ffn[l]` (first `k_ffn[l]` entries) the channel sets used."""
+
+    GRAD_ORDER = ("q", "k", "v", "o")
+
+    def __init__(self, layers, d, heads, kv_heads, head_dim, d_ff, r_svd, r_lora, scale, batch,
+                 seq, ctx_len, qk_sparsity, ffn_sparsity, X, dY, rope_base=10000.0,
+                 eps=1e-5):
+        H, KV, hd = heads, kv_heads, head_dim
+        nq, nkv, T = H * hd, KV * hd, batch * seq
+        tok, tok_keep = L.make_tokens(batch, seq, ctx_len)
+        self._keep = [tok, tok_keep, X, dY, layers]
+        TC = int(sum(int(c) for c in ctx_len))
+        TO = T - TC
+        s = float(scale)
+        r = r_lora
+        bf = _bf16_empty
+        f32 = lambda *sh: torch.empty(*sh, device="cuda")
+        nl = len(layers)
+        self.nl = nl
+        # ---- saved activations, per layer
+        self.x = [X] + [bf(T, d) for _ in range(nl - 1)]
+        self.y = bf(T, d)
+        sv = []
+        for _ in range(nl):
+            sv.append(dict(n1=bf(T, d), r1=f32(T), Qr=bf(T, nq), Kr=bf(T, nkv), V=bf(T, nkv),
+                           O=bf(T, nq), lse=f32(batch, H, seq), XAq=f32(T, r), XAk=f32(T, r),
+                           XAv=f32(T, r), XAo=f32(T, r), h=bf(T, d), n2=bf(T, d), r2=f32(T)))
+        self.saved = sv
+        # ---- scratch shared by the layers
+        a_out, f_out, f_re = bf(T, d), bf(T, d), bf(T, d)
+        dn2, dh, dxq, dxk, dxv = bf(T, d), bf(T, d), bf(T, d), bf(T, d), bf(T, d)
+        dx_pp = [bf(T, d), bf(T, d)]
+        dO_att = bf(T, nq)
+        dQr, dKr, dV = f32(T, nq), f32(T, nkv), bf(T, nkv)
+        self._scratch = (a_out, f_out, f_re, dn2, dh, dxq, dxk, dxv, dx_pp, dO_att, dQr, dKr, dV)
+        # ---- gradients: one flat fp32 buffer, 16-byte aligned views
+        shapes = []
+        for nm, n, k in (("q", nq, d), ("k", nkv, d), ("v", nkv, d), ("o", d, nq)):
+            shapes += [("dA" + nm, (r, k)), ("dB" + nm, (n, r))]
+        shapes += list(zip(("dAg", "dBg", "dAu", "dBu", "dAd", "dBd"),
+                           lora_grad_shapes_ffn(d, d_ff, r)))
+        sizes = [(a * b + 3) // 4 * 4 for _, (a, b) in shapes]
+        per = sum(sizes)
+        self.gflat = torch.zeros(nl * per, device="cuda")
+        self.grads = []
+        for l in range(nl):
+            g, o = {}, l * per
+            for (key, (a, b)), sz in zip(shapes, sizes):
+                g[key] = self.gflat[o:o + a * b].view(a, b)
+                o += sz
+            self.grads.append(g)
+
+        calls, bwd = [], []
+        self.idx_qk, self.idx_ffn, self.k_ffn, self.kh = [], [], [], []
+        self._structs = []
+        for l, w in enumerate(layers):
+            S_ = sv[l]
+            G = self.grads[l]
+            # -- input normalisation (the first layer reads X; later ones add
+            # the previous FFN output to the previous residual)
+            if l == 0:
+                calls.append(_Call("slora_rmsnorm_fwd", [L.BF16, T, d, L.c_f32(eps), L.ptr(X),
+                                                         None, L.ptr(w["g1"]), None,
+                                                         L.ptr(S_["n1"]), L.ptr(S_["r1"])]))
+            else:
+                calls.append(_Call("slora_rmsnorm_fwd",
+                                   [L.BF16, T, d, L.c_f32(eps), L.ptr(sv[l - 1]["h"]),
+                                    L.ptr(f_out), L.ptr(w["g1"]), L.ptr(self.x[l]),
+                                    L.ptr(S_["n1"]), L.ptr(S_["r1"])]))
+            n1 = S_["n1"]
+            # -- q/k channel selection
+            sq = float(qk_sparsity[l])
+            if sq > 0.0:
+                idx = torch.empty(nq + nkv, dtype=torch.int32, device="cuda")
+                k_out = L.c_i32(0)
+                scores = f32(KV * hd)
+                c = _Call("slora_estimate_select",
+                          [L.CRIT_QK, L.ptr(n1), L.BF16, ctypes.byref(tok), d, L.ptr(w["Lq"]),
+                           L.ptr(w["Uq"]), nq, L.ptr(w["Lk"]), L.ptr(w["Uk"]), nkv, r_svd, H, KV,
+                           hd, sq, L.ptr(idx), ctypes.byref(k_out), L.ptr(scores)],
+                          (k_out, idx, scores))
+                c.need()
+                kh = int(k_out.value)
+                calls.append(c)
+                iq, ik = idx[:H * kh], idx[H * kh:H * kh + KV * kh]
+            else:
+                idx, kh, iq, ik = None, hd, None, None
+            self.idx_qk.append(idx)
+            self.kh.append(kh)
+            # -- q, k, v, o linears and the attention core
+            proj = {}
+            for nm, n, ii in (("q", nq, iq), ("k", nkv, ik)):
+                base = [L.BF16, ctypes.byref(tok), d, n, L.ptr(w["W" + nm]), L.ptr(w["A" + nm]),
+                        L.ptr(w["B" + nm]), r, s]
+                XA = S_["XA" + nm]
+                R = S_["Qr" if nm == "q" else "Kr"]
+                dR = dQr if nm == "q" else dKr
+                dXn = dxq if nm == "q" else dxk
+                if ii is not None:
+                    ni = ii.numel()
+                    Yc, Yo, dYc, dYo = bf(TC, ni), bf(TO, n), bf(TC, ni), bf(TO, n)
+                    self._keep += [Yc, Yo, dYc, dYo]
+                    fwd = _Call("slora_linear_fwd", base + [L.SLICE_OUT_ROWS, L.ptr(ii), ni,
+                                                            L.ptr(n1), None, L.ptr(Yc),
+                                                            L.ptr(Yo), L.ptr(XA)])
+                    rope = _Call("slora_rope_pack", [L.BF16, ctypes.byref(tok), n, hd,
+                                                     float(rope_base), L.ptr(ii), ni, None,
+                                                     L.ptr(Yc), L.ptr(Yo), L.ptr(R)])
+                    unrope = _Call("slora_rope_unpack", [L.BF16, ctypes.byref(tok), n, hd,
+                                                         float(rope_base), L.ptr(ii), ni,
+                                                         L.ptr(dR), None, L.ptr(dYc),
+                                                         L.ptr(dYo)])
+                    back = _Call("slora_linear_bwd", base + [L.SLICE_OUT_ROWS, L.ptr(ii), ni,
+                                                             L.ptr(n1), None, L.ptr(XA),
+                                                             L.ptr(dYc), L.ptr(dYo), L.ptr(dXn),
+                                                             None, L.ptr(G["dA" + nm]),
+                                                             L.ptr(G["dB" + nm])])
+                else:
+                    Y, dYd = bf(T, n), bf(T, n)
+                    self._keep += [Y, dYd]
+                    fwd = _Call("slora_linear_fwd", base + [L.SLICE_NONE, None, 0, L.ptr(n1),
+                                                            None, L.ptr(Y), None, L.ptr(XA)])
+                    rope = _Call("slora_rope_pack", [L.BF16, ctypes.byref(tok), n, hd,
+                                                     float(rope_base), None, 0, L.ptr(Y), None,
+                                                     None, L.ptr(R)])
+                    unrope = _Call("slora_rope_unpack", [L.BF16, ctypes.byref(tok), n, hd,
+                                                         float(rope_base), None, 0, L.ptr(dR),
+                                                         L.ptr(dYd), None, None])
+                    back = _Call("slora_linear_bwd", base + [L.SLICE_NONE, None, 0, L.ptr(n1),
+                                                             None, L.ptr(XA), L.ptr(dYd), None,
+                                                             L.ptr(dXn), None,
+                                                             L.ptr(G["dA" + nm]),
+                                                             L.ptr(G["dB" + nm])])
+                proj[nm] = (fwd, rope, unrope, back)
+            vbase = [L.BF16, ctypes.byref(tok), d, nkv, L.ptr(w["Wv"]), L.ptr(w["Av"]),
+                     L.ptr(w["Bv"]), r, s, L.SLICE_NONE, None, 0]
+            v_f = _Call("slora_linear_fwd", vbase + [L.ptr(n1), None, L.ptr(S_["V"]), None,
+                                                     L.ptr(S_["XAv"])])
+            v_b = _Call("slora_linear_bwd", vbase + [L.ptr(n1), None, L.ptr(S_["XAv"]),
+                                                     L.ptr(dV), None, L.ptr(dxv), None,
+                                                     L.ptr(G["dAv"]), L.ptr(G["dBv"])])
+            att_f = _Call("slora_attention_fwd", [L.BF16, ctypes.byref(tok), H, KV, hd,
+                                                  L.ptr(S_["Qr"]), L.ptr(S_["Kr"]),
+                                                  L.ptr(S_["V"]), L.ptr(S_["O"]),
+                                                  L.ptr(S_["lse"])])
+            att_b = _Call("slora_attention_bwd", [L.BF16, ctypes.byref(tok), H, KV, hd,
+                                                  L.ptr(S_["Qr"]), L.ptr(S_["Kr"]),
+                                                  L.ptr(S_["V"]), L.ptr(S_["O"]),
+                                                  L.ptr(S_["lse"]), L.ptr(dO_att), L.ptr(dQr),
+                                                  L.ptr(dKr), L.ptr(dV)])
+            obase = [L.BF16, ctypes.byref(tok), nq, d, L.ptr(w["Wo"]), L.ptr(w["Ao"]),
+                     L.ptr(w["Bo"]), r, s, L.SLICE_NONE, None, 0]
+            o_f = _Call("slora_linear_fwd", obase + [L.ptr(S_["O"]), None, L.ptr(a_out), None,
+                                                     L.ptr(S_["XAo"])])
+            o_b = _Call("slora_linear_bwd", obase + [L.ptr(S_["O"]), None, L.ptr(S_["XAo"]),
+                                                     L.ptr(dh), None, L.ptr(dO_att), None,
+                                                     L.ptr(G["dAo"]), L.ptr(G["dBo"])])
+            calls += [proj["q"][0], proj["k"][0], v_f, proj["q"][1], proj["k"][1], att_f, o_f]
+            # -- residual + second normalisation, FFN forward (its own selection)
+            calls.append(_Call("slora_rmsnorm_fwd", [L.BF16, T, d, L.c_f32(eps),
+                                                     L.ptr(self.x[l]), L.ptr(a_out),
+                                                     L.ptr(w["g2"]), L.ptr(S_["h"]),
+                                                     L.ptr(S_["n2"]), L.ptr(S_["r2"])]))
+            sf = float(ffn_sparsity[l])
+            fidx = torch.empty(d_ff, dtype=torch.int32, device="cuda")
+            fidx_re = torch.empty(d_ff, dtype=torch.int32, device="cuda")
+            force = torch.arange(d_ff, dtype=torch.int32, device="cuda") if sf == 0.0 else None
+            lay = L.ffn_layer_struct(d, d_ff, r_svd, r, s, w["Wg"], w["Wu"], w["Wd_t"], w["Ag"],
+                                     w["Bg"], w["Au"], w["Bu"], w["Ad"], w["Bd"], w["Lg"],
+                                     w["Ug"], w["Lu"], w["Uu"])
+            fgs = L.ffn_grads_struct(G["dAg"], G["dBg"], G["dAu"], G["dBu"], G["dAd"], G["dBd"])
+            fa, fk = L.ffn_args(L.BF16, lay, batch, seq, ctx_len, sf, S_["n2"], None, f_out, None,
+                                None, fidx, force)
+            ffn_f = _Call("slora_ffn_fwd_bwd", fa, fk + (lay, force))
+            ffn_f.need()
+            kf = int(fk[2].value)
+            self.idx_ffn.append(fidx)
+            self.k_ffn.append(kf)
+            calls.append(ffn_f)
+            # backward of this layer (issued in reverse layer order below)
+            self._structs += [lay, fgs]
+            bwd.append(dict(fgs=fgs, lay=lay, fidx=fidx, fidx_re=fidx_re, kf=kf, q=proj["q"],
+                            k=proj["k"], v_b=v_b, att_b=att_b, o_b=o_b, w=w, S=S_))
+        # -- the stack output: last residual + last FFN output
+        calls.append(_Call("slora_rmsnorm_fwd", [L.BF16, T, d, L.c_f32(eps),
+                                                 L.ptr(sv[-1]["h"]), L.ptr(f_out),
+                                                 L.ptr(layers[-1]["g2"]), L.ptr(self.y), None,
+                                                 None]))
+        # ---- backward, last layer first
+        dx_cur = dY
+        for l in range(nl - 1, -1, -1):
+            B = bwd[l]
+            S_, w = B["S"], B["w"]
+            dx_next = dx_pp[(nl - 1 - l) % 2]
+            fa, fk = L.ffn_args(L.BF16, B["lay"], batch, seq, ctx_len, 0.0, S_["n2"], dx_cur,
+                                f_re, dn2, B["fgs"], B["fidx_re"], B["fidx"][:B["kf"]])
+            calls.append(_Call("slora_ffn_fwd_bwd", fa, fk + (B["fidx"],)))
+            calls.append(_Call("slora_rmsnorm_bwd", [L.BF16, T, d, L.ptr(S_["h"]),
+                                                     L.ptr(S_["r2"]), L.ptr(w["g2"]), L.ptr(dn2),
+                                                     None, None, L.ptr(dx_cur), L.ptr(dh)]))
+            calls += [B["o_b"], B["att_b"], B["q"][2], B["k"][2], B["q"][3], B["k"][3],
+                      B["v_b"]]
+            calls.append(_Call("slora_rmsnorm_bwd", [L.BF16, T, d, L.ptr(self.x[l]),
+                                                     L.ptr(S_["r1"]), L.ptr(w["g1"]), L.ptr(dxq),
+                                                     L.ptr(dxk), L.ptr(dxv), L.ptr(dh),
+                                                     L.ptr(dx_next)]))
+            dx_cur = dx_next
+        self.dX = dx_cur
+        self.calls = calls

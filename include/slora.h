@@ -137,12 +137,13 @@ slora_status slora_set_wait_budget(int64_t cycles);
  *                          operand packing), "prepare", "skinny" (rank-r
  *                          LoRA projections and gradients), "compact"
  *                          (selected-row gather), "attention" (the causal
- *                          attention core and its rotary packing), "norm"
+ *                          attention core's forward and backward), "norm"
  *                          (RMS normalisation).  It synchronizes the
  *                          recorded events.  work = algorithmic FLOPs for the
  *                          GEMM classes (2*M*N*K on the selected sizes) and
- *                          the attention kernels (2 M N K per product over the
- *                          causal tiles computed), bytes moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
+ *                          the attention kernels (2 head_dim per causal
+ *                          query-key pair and product: two forward, five
+ *                          backward), bytes moved for the others.  Unknown class: SLORA_ERR_INVALID_ARG.
  */
 int64_t slora_launch_count(void);
 void slora_profile_enable(int on);
