@@ -625,6 +625,15 @@ def run_ffn(args, H, pk, rank, world):
     est_m = measure_estimator(H, est, args.steps, pk, mhz)
     n_e, ms_e, _ = prof["estimate"]
     n_s, ms_s, _ = prof["select"]
+    # the per-sequence variant: one channel set per sequence (same inputs)
+    ps = FfnLayer(w, d, F, rs, r, case.lora_scale, tok.batch, tok.seq, tok.ctx_len,
+                  wl["sparsity"], layers[0].X, layers[0].dOut, per_sequence=True)
+    ws_ps = torch.empty(ps.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    g_ps = H.capture(lambda: ps.step(ws_ps))
+    g_ps.replay()
+    n_ps = max(3, args.steps // 2)
+    ms_ps = dp.max_over_ranks(H.time_steps(g_ps.replay, n_ps), device="cuda") / n_ps
+    del g_ps, ps, ws_ps
     est_m["in_step_us"] = {"score_and_select": (ms_e + ms_s) * 1e3 / args.steps,
                            "note": "inside slora_ffn_fwd_bwd the projection X_C [Lg|Lu] rides "
                                    "the LoRA X A^T stream over X (class 'skinny')"}
@@ -636,6 +645,10 @@ def run_ffn(args, H, pk, rank, world):
             "config": workload_config(wl["name"], world),
             "roofline": gemm_roofline(prof, pk, workload=wl["name"]),
             "estimator": est_m,
+            "per_sequence_sets": {"ms_per_step": ms_ps, "tokens_per_s": world * T / (ms_ps / 1e3),
+                                  "vs_per_batch_set": ms_step / ms_ps,
+                                  "call": "slora_ffn_fwd_bwd_per_seq (one channel set per "
+                                          "sequence; same inputs)"},
             "kernels": kernel_table(prof, args.steps, ms_prof), "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

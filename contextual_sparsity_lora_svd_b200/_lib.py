@@ -87,6 +87,9 @@ _sig("slora_ffn_fwd_bwd", c_int,
       c_vp,
       ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 
+_sig("slora_ffn_fwd_bwd_per_seq", c_int,
+     [c_int, ctypes.POINTER(FfnLayer), ctypes.POINTER(Tokens), ctypes.c_double, c_vp, c_vp, c_vp,
+      c_vp, ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 _sig("slora_rope_pack", c_int,
      [c_int, ctypes.POINTER(Tokens), c_i64, c_int, ctypes.c_double, c_vp, c_i32, c_vp, c_vp, c_vp,
       c_vp, c_vp, P_SZ, c_vp])
@@ -118,7 +121,7 @@ EXPORTS = sorted(["slora_last_error_string", "slora_version", "slora_svd_prepare
                   "slora_ffn_fwd_bwd", "slora_launch_count", "slora_profile_enable",
                   "slora_profile_read", "slora_noalloc_scratch_bytes",
                   "slora_estimate_select_noalloc", "slora_device_error",
-                  "slora_set_wait_budget", "slora_rope_pack", "slora_rope_unpack",
+                  "slora_set_wait_budget", "slora_ffn_fwd_bwd_per_seq", "slora_rope_pack", "slora_rope_unpack",
                   "slora_attention_fwd", "slora_attention_bwd", "slora_rmsnorm_fwd",
                   "slora_rmsnorm_bwd"])
 
@@ -295,11 +298,16 @@ def ffn_args(dt, layer, batch, seq, ctx_len, sparsity, X, dOut, out, dX, grads, 
 
 
 def slora_ffn_fwd_bwd(layer: FfnLayer, batch, seq, ctx_len, sparsity, X, dOut, out, dX,
-                      grads: FfnGrads, idx_out, idx_force=None, ws=None, stream=None) -> int:
-    """Returns k_keep."""
+                      grads: FfnGrads, idx_out, idx_force=None, ws=None, stream=None,
+                      per_sequence=False) -> int:
+    """Returns k_keep.  per_sequence: one channel set per sequence
+    (slora_ffn_fwd_bwd_per_seq; idx_out is [batch x d_ff], idx_force
+    [batch x k_force])."""
     args, keep = ffn_args(dtype_code(X), layer, batch, seq, ctx_len, sparsity, X, dOut, out, dX,
                           grads, idx_out, idx_force)
-    _run("slora_ffn_fwd_bwd", args, ws, stream)
+    if per_sequence and idx_force is not None:
+        args[-1] = idx_force.numel() // batch
+    _run("slora_ffn_fwd_bwd_per_seq" if per_sequence else "slora_ffn_fwd_bwd", args, ws, stream)
     return int(keep[2].value)
 
 

@@ -7,6 +7,7 @@
 #include "estimator.cuh"
 #include "gemm_simt.cuh"
 #include "linear_ops.cuh"
+#include "lora_pack.cuh"
 #include "skinny.cuh"
 #include "swiglu.cuh"
 
@@ -376,15 +377,13 @@ extern "C" slora_status slora_linear_bwd(slora_dtype dt, const slora_tokens* tok
 }
 
 // ------------------------------------------------------------------- FFN
-extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
-                                          const slora_tokens* tok, double sparsity, const void* X,
-                                          const void* dOut, void* out, void* dX,
-                                          const slora_ffn_grads* grads, int32_t* idx_out,
-                                          int32_t* k_out, const int32_t* idx_force,
-                                          int32_t k_force, void* ws, size_t* ws_bytes,
-                                          slora_stream_t stream) {
-  const char* fn = "slora_ffn_fwd_bwd";
-  clear_error();
+namespace {
+// Checks shared by the per-batch and the per-sequence FFN calls; sets kkeep.
+slora_status ffn_validate(const char* fn, slora_dtype dt, const slora_ffn_layer* layer,
+                          const slora_ffn_grads* grads, double sparsity, const void* X,
+                          const void* dOut, void* out, void* dX, int32_t* idx_out,
+                          int32_t* k_out, const int32_t* idx_force, int32_t k_force, void* ws,
+                          int64_t* kkeep) {
   SLORA_TRY(check_dtype(fn, dt));
   // dOut == NULL: forward only (dX and grads unused)
   const bool fwd_only = dOut == nullptr;
@@ -406,21 +405,101 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   SLORA_TRY(check_row(fn, "d_ff", Ly.d_ff, dt));
   if (Ly.r_lora < 1 || Ly.r_lora > 32)
     SLORA_FAIL(SLORA_ERR_SHAPE, "%s: r_lora %d outside [1, 32]", fn, Ly.r_lora);
-  int64_t kkeep;
   if (idx_force) {
     if (k_force < 0 || k_force > Ly.d_ff)
       SLORA_FAIL(SLORA_ERR_SHAPE, "%s: k_force=%d outside [0, d_ff]", fn, k_force);
-    kkeep = k_force;
+    *kkeep = k_force;
   } else {
     SLORA_TRY(check_sparsity(fn, sparsity));
     REQ_PTR(Ly.Lg); REQ_PTR(Ly.Ug); REQ_PTR(Ly.Lu); REQ_PTR(Ly.Uu);
     if (Ly.r_svd < 1 || Ly.r_svd > 48)
       SLORA_FAIL(SLORA_ERR_SHAPE, "%s: r_svd %d outside [1, 48]", fn, Ly.r_svd);
-    kkeep = keep_count(Ly.d_ff, sparsity);
+    *kkeep = keep_count(Ly.d_ff, sparsity);
   }
+  return SLORA_OK;
+}
+
+// One channel set per sequence: the per-batch path run on each sequence's
+// rows in turn (each call estimates and selects from that sequence's context
+// rows), its LoRA gradients kept per sequence in the workspace and summed in
+// sequence order at the end.
+slora_status ffn_per_seq_run(const FfnDesc& F, const slora_tokens* tok, const void* X,
+                             const void* dOut, void* out, void* dX, int32_t* idx,
+                             const int32_t* idx_force, int64_t k_force, Arena& ar, bool plan,
+                             cudaStream_t st) {
+  const slora_ffn_layer& L = F.L;
+  const int B = tok->batch, seq = tok->seq, r = L.r_lora;
+  const int64_t d = L.d, Fd = L.d_ff;
+  const int64_t es = dt_size(F.dt);
+  const bool fwd_only = dOut == nullptr;
+  const int64_t glen[6] = {r * d, Fd * r, r * d, Fd * r, r * Fd, d * r};
+  int64_t goff[6], gtot = 0;
+  for (int q = 0; q < 6; ++q) {
+    goff[q] = gtot;
+    gtot += (glen[q] + 63) / 64 * 64;
+  }
+  float* gbuf = fwd_only ? nullptr : ar.take<float>(size_t(B) * gtot);
+  // one sub-workspace, reused by every sequence in stream order
+  size_t sub = 16;
+  for (int b = 0; b < B; ++b) {
+    slora_tokens tb{1, seq, &tok->ctx_len[b]};
+    FfnDesc Fb = F;
+    SLORA_TRY(parse_tokens(&tb, &Fb.ti));
+    Arena p;
+    SLORA_TRY(ffn_run(Fb, &tb, X, dOut, out, dX, idx, idx_force, p, true, nullptr));
+    sub = std::max(sub, p.used);
+  }
+  char* subws = ar.take<char>(sub);
+  if (plan) return SLORA_OK;
+  SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd_per_seq"));
+  for (int b = 0; b < B; ++b) {
+    slora_tokens tb{1, seq, &tok->ctx_len[b]};
+    FfnDesc Fb = F;
+    SLORA_TRY(parse_tokens(&tb, &Fb.ti));
+    if (!fwd_only) {
+      float* g = gbuf + size_t(b) * gtot;
+      Fb.G.dAg = g + goff[0]; Fb.G.dBg = g + goff[1]; Fb.G.dAu = g + goff[2];
+      Fb.G.dBu = g + goff[3]; Fb.G.dAd = g + goff[4]; Fb.G.dBd = g + goff[5];
+    }
+    const int64_t row0 = int64_t(b) * seq;
+    auto at = [&](const void* p) -> const char* {
+      return p ? static_cast<const char*>(p) + row0 * d * es : nullptr;
+    };
+    Arena a;
+    a.base = subws;
+    a.cap = sub;
+    SLORA_TRY(ffn_run(Fb, &tb, at(X), at(dOut), const_cast<char*>(at(out)),
+                      const_cast<char*>(at(dX)), idx + int64_t(b) * Fd,
+                      idx_force ? idx_force + int64_t(b) * k_force : nullptr, a, false, st));
+  }
+  if (fwd_only) return SLORA_OK;
+  float* dst[6] = {F.G.dAg, F.G.dBg, F.G.dAu, F.G.dBu, F.G.dAd, F.G.dBd};
+  SumSeg segs[6];
+  for (int q = 0; q < 6; ++q) {
+    segs[q].dst = dst[q];
+    segs[q].off = goff[q];
+    segs[q].len = glen[q];
+  }
+  return sum_groups(gbuf, B, gtot, segs, 6, st);
+}
+}  // namespace
+
+extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
+                                          const slora_tokens* tok, double sparsity, const void* X,
+                                          const void* dOut, void* out, void* dX,
+                                          const slora_ffn_grads* grads, int32_t* idx_out,
+                                          int32_t* k_out, const int32_t* idx_force,
+                                          int32_t k_force, void* ws, size_t* ws_bytes,
+                                          slora_stream_t stream) {
+  const char* fn = "slora_ffn_fwd_bwd";
+  clear_error();
+  int64_t kkeep = 0;
+  SLORA_TRY(ffn_validate(fn, dt, layer, grads, sparsity, X, dOut, out, dX, idx_out, k_out,
+                         idx_force, k_force, ws, &kkeep));
+  const slora_ffn_grads Gr = grads ? *grads : slora_ffn_grads{};
   TokenInfo ti;
   SLORA_TRY(parse_tokens(tok, &ti));
-  FfnDesc F{int(dt), ti, Ly, Gr, kkeep, sparsity};
+  FfnDesc F{int(dt), ti, *layer, Gr, kkeep, sparsity};
   Arena plan;
   SLORA_TRY(ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr));
   const bool query = ws == nullptr;
@@ -433,4 +512,33 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
   ar.cap = *ws_bytes;
   return ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, ar, false,
                  static_cast<cudaStream_t>(stream));
+}
+
+extern "C" slora_status slora_ffn_fwd_bwd_per_seq(
+    slora_dtype dt, const slora_ffn_layer* layer, const slora_tokens* tok, double sparsity,
+    const void* X, const void* dOut, void* out, void* dX, const slora_ffn_grads* grads,
+    int32_t* idx_out, int32_t* k_out, const int32_t* idx_force, int32_t k_force, void* ws,
+    size_t* ws_bytes, slora_stream_t stream) {
+  const char* fn = "slora_ffn_fwd_bwd_per_seq";
+  clear_error();
+  int64_t kkeep = 0;
+  SLORA_TRY(ffn_validate(fn, dt, layer, grads, sparsity, X, dOut, out, dX, idx_out, k_out,
+                         idx_force, k_force, ws, &kkeep));
+  const slora_ffn_grads Gr = grads ? *grads : slora_ffn_grads{};
+  TokenInfo ti;
+  SLORA_TRY(parse_tokens(tok, &ti));
+  FfnDesc F{int(dt), ti, *layer, Gr, kkeep, sparsity};
+  Arena plan;
+  SLORA_TRY(ffn_per_seq_run(F, tok, X, dOut, out, dX, idx_out, idx_force, k_force, plan, true,
+                            nullptr));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  *k_out = int32_t(kkeep);
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
+  return ffn_per_seq_run(F, tok, X, dOut, out, dX, idx_out, idx_force, k_force, ar, false,
+                         static_cast<cudaStream_t>(stream));
 }

@@ -6,6 +6,8 @@
 //                    LoRA up-projection of both halves is one K = 2r segment
 //   transpose_rows : out[c][q] = in[q][c]     (A_d^T, rows = channels)
 //   stack_rows     : out = [top; bottom]      ([A_g; A_u], MN-major operand)
+#include <algorithm>
+
 #include "lora_pack.cuh"
 
 #include "gemm_tc.cuh"
@@ -173,7 +175,35 @@ __global__ void plain_tiles_kernel(int4* __restrict__ tiles, int64_t M, int64_t 
 
 unsigned blocks(int64_t n) { return unsigned((n + 255) / 256); }
 
+__global__ void sum_groups_kernel(const float* __restrict__ src, int groups, int64_t stride,
+                                  const __grid_constant__ SumSegs S) {
+  const SumSeg& q = S.seg[blockIdx.y];
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= q.len) return;
+  float acc = 0.f;
+  for (int g = 0; g < groups; ++g) acc += src[g * stride + q.off + i];
+  q.dst[i] = acc;
+}
+
 }  // namespace
+
+slora_status sum_groups(const float* src, int groups, int64_t stride, const SumSeg* segs,
+                        int nseg, cudaStream_t st) {
+  if (nseg <= 0) return SLORA_OK;
+  if (nseg > SumSegs::kMax)
+    SLORA_FAIL(SLORA_ERR_SHAPE, "sum_groups: %d segments (max %d)", nseg, SumSegs::kMax);
+  SumSegs S{};
+  int64_t mx = 0;
+  for (int k = 0; k < nseg; ++k) {
+    S.seg[k] = segs[k];
+    mx = std::max(mx, segs[k].len);
+  }
+  if (mx == 0) return SLORA_OK;
+  LaunchScope ls(kAux, double(groups) * stride * 4, st);
+  sum_groups_kernel<<<dim3(blocks(mx), unsigned(nseg)), 256, 0, st>>>(src, groups, stride, S);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
 
 slora_status scatter_add_cols(const ScatterAddJob* jobs, int njobs, const int32_t* idx,
                               int64_t n, int r, int64_t limit, cudaStream_t st) {

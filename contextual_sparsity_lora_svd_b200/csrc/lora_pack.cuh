@@ -74,6 +74,19 @@ struct ScatterAddJobs {
 };
 slora_status scatter_add_cols(const ScatterAddJob* jobs, int njobs, const int32_t* idx,
                               int64_t n, int r, int64_t limit, cudaStream_t st);
+// Sums of per-group fp32 results in a fixed order: for each segment q,
+// dst_q[i] = sum over g = 0 .. groups-1 of src[g * stride + off_q + i], i < len_q
+// (up to six segments, one launch).
+struct SumSeg {
+  float* dst = nullptr;
+  int64_t off = 0, len = 0;
+};
+struct SumSegs {
+  static constexpr int kMax = 6;
+  SumSeg seg[kMax];
+};
+slora_status sum_groups(const float* src, int groups, int64_t stride, const SumSeg* segs,
+                        int nseg, cudaStream_t st);
 // M-tile list {row0, row0, nvalid, 0} covering rows [0, M) in 128-row tiles.
 slora_status make_plain_tiles(int4* tiles, int64_t M, cudaStream_t st);
 }  // namespace slora

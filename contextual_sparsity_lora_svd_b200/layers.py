@@ -9,7 +9,8 @@ part of the method: every number is produced by libslora's kernels.
 
   FfnLayer      one SwiGLU FFN: slora_ffn_fwd_bwd (estimate, select, sliced
                 forward and backward; a ratio of 0 runs every channel through
-                idx_force, the dense path).
+                idx_force, the dense path), or with per_sequence one channel set
+                per sequence (slora_ffn_fwd_bwd_per_seq).
   AttnLinears   the q/k/v/o LoRA linears of one attention layer around a
                 stand-in for the attention core (its output is an input
                 tensor: the core itself is not part of this library).  q/k are
@@ -73,7 +74,8 @@ class FfnLayer(_Runner):
     Wd_t [d_ff x d] (the transposed down weight), Ag, Bg, Au, Bu, Ad, Bd (bf16)
     and the fp32 estimator factors Lg, Ug, Lu, Uu."""
 
-    def __init__(self, w, d, d_ff, r_svd, r_lora, scale, batch, seq, ctx_len, sparsity, X, dOut):
+    def __init__(self, w, d, d_ff, r_svd, r_lora, scale, batch, seq, ctx_len, sparsity, X, dOut,
+                 per_sequence=False):
         # the argument lists hold raw device addresses of w, X and dOut, which
         # the runner keeps alive
         self.w, self.d, self.d_ff, self.r = w, d, d_ff, r_lora
@@ -87,7 +89,9 @@ class FfnLayer(_Runner):
         for a, b in shapes:
             self.grads.append(self.gflat[o:o + a * b].view(a, b))
             o += a * b
-        self.idx = torch.empty(d_ff, dtype=torch.int32, device="cuda")
+        # per_sequence: one channel set per sequence (idx holds batch sets of d_ff)
+        self.idx = torch.empty(d_ff * (batch if per_sequence else 1), dtype=torch.int32,
+                               device="cuda")
         # a ratio of 0 is the dense path: every channel, no estimator
         self.force = (torch.arange(d_ff, dtype=torch.int32, device="cuda")
                       if self.sparsity == 0.0 else None)
@@ -98,7 +102,8 @@ class FfnLayer(_Runner):
         self.gstruct = L.ffn_grads_struct(*self.grads)
         args, keep = L.ffn_args(L.BF16, self.layer, batch, seq, ctx_len, self.sparsity, X, dOut,
                                 self.out, self.dX, self.gstruct, self.idx, self.force)
-        self.calls = [_Call("slora_ffn_fwd_bwd", args, keep + (self.layer, self.gstruct))]
+        name = "slora_ffn_fwd_bwd_per_seq" if per_sequence else "slora_ffn_fwd_bwd"
+        self.calls = [_Call(name, args, keep + (self.layer, self.gstruct))]
         self._kout = keep[2]
 
     def kept(self) -> int:

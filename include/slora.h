@@ -363,6 +363,27 @@ slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
                                int32_t k_force, void* ws, size_t* ws_bytes,
                                slora_stream_t stream);
 
+/*
+ * slora_ffn_fwd_bwd_per_seq — slora_ffn_fwd_bwd with one channel set per
+ * sequence instead of one per batch [ART §1: the channels are chosen per
+ * input]: each sequence's context rows are scored and selected on their own
+ * and computed on their own set S_b; output rows stay dense; the LoRA
+ * gradients are the sum over sequences, added in sequence order.
+ *   Arguments as slora_ffn_fwd_bwd, except:
+ *   idx_out   device int32 [batch x d_ff]: sequence b's k_keep channels
+ *             (ascending) at idx_out + b*d_ff.
+ *   idx_force optional device int32 [batch x k_force]: sequence b's forced set
+ *             at idx_force + b*k_force.
+ *   The workspace holds one set of LoRA gradients per sequence.
+ */
+slora_status slora_ffn_fwd_bwd_per_seq(slora_dtype dt, const slora_ffn_layer* layer,
+                                       const slora_tokens* tok, double sparsity, const void* X,
+                                       const void* dOut, void* out, void* dX,
+                                       const slora_ffn_grads* grads, int32_t* idx_out,
+                                       int32_t* k_out, const int32_t* idx_force,
+                                       int32_t k_force, void* ws, size_t* ws_bytes,
+                                       slora_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * The rest of a decoder layer around the sparse linears: rotary packing of
  * the q/k rows, the causal attention core and RMS normalisation.  These make

@@ -32,6 +32,7 @@ __all__ = [
     "estimate_select_ffn", "estimate_select_qk", "estimate_select_ffn_gram",
     "estimate_select_qk_pairs", "estimate_select_l2",
     "linear_fwd", "linear_bwd", "ffn_fwd", "ffn_bwd", "ffn_fwd_bwd",
+    "ffn_fwd_bwd_per_seq", "ffn_fwd_down_only",
 ]
 
 
@@ -439,3 +440,44 @@ def ffn_fwd_bwd(X, dOut, batch, seq, ctx_len, lay: dict, sparsity: float, idx_fo
     out, saved = ffn_fwd(X, batch, seq, ctx_len, lay, idx)
     grads = ffn_bwd(X, dOut, lay, idx, saved)
     return dict(idx=idx, k=k, scores=scores, out=out, **grads)
+
+
+# ---------------------------------------------------------------------------
+# projection-set variants (article section 6: which projections run sparse;
+# section 1: the channels are chosen per input)
+# ---------------------------------------------------------------------------
+def ffn_fwd_bwd_per_seq(X, dOut, batch, seq, ctx_len, lay: dict, sparsity: float,
+                        idx_force=None):
+    """One channel set per sequence instead of one per batch (reading of
+    "per input"): each sequence is its own one-sequence batch for the estimate,
+    the selection and the sliced computation; the LoRA gradients of the layer
+    are the sums over sequences.  ``idx_force[b]`` fixes sequence b's set.
+    Returns dict(idx=[per-sequence sets], k, out, dX, dAg, ...)."""
+    T, d = X.shape
+    out, dX = np.zeros_like(X), np.zeros_like(X)
+    grads, sets, k = None, [], None
+    for b in range(batch):
+        rows = slice(b * seq, (b + 1) * seq)
+        force = None if idx_force is None else idx_force[b]
+        r = ffn_fwd_bwd(X[rows], dOut[rows], 1, seq, [ctx_len[b]], lay, sparsity, force)
+        out[rows], dX[rows] = r["out"], r["dX"]
+        sets.append(r["idx"])
+        k = r["k"]
+        g = {n: r[n] for n in ("dAg", "dBg", "dAu", "dBu", "dAd", "dBd")}
+        grads = g if grads is None else {n: grads[n] + g[n] for n in g}
+    return dict(idx=sets, k=k, out=out, dX=dX, **grads)
+
+
+def ffn_fwd_down_only(X, batch, seq, ctx_len, lay: dict, idx):
+    """The down-projection-only variant: gate and up computed on every channel
+    for every row, the down projection of context rows reading only the
+    channels idx (the others' activations dropped).  Returns out."""
+    s = lay["scale"]
+    C, _ = context_rows(batch, seq, ctx_len)
+    g = X @ lay["Wg"].T + s * ((X @ lay["Ag"].T) @ lay["Bg"].T)
+    u = X @ lay["Wu"].T + s * ((X @ lay["Au"].T) @ lay["Bu"].T)
+    h = silu(g) * u
+    keep = np.zeros(h.shape[1], dtype=bool)
+    keep[np.asarray(idx, dtype=np.int64)] = True
+    h[np.ix_(C, ~keep)] = 0.0
+    return h @ lay["Wd"].T + s * ((h @ lay["Ad"].T) @ lay["Bd"].T)

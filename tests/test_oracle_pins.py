@@ -777,3 +777,81 @@ def test_planted_l2_head_offset_is_caught(monkeypatch):
 def test_oracle_package_exports():
     for name in O.__all__:
         assert hasattr(oracle, name)
+
+
+# ------------------------------------------------- projection-set variants
+def _tiny_ffn(seed, d=12, d_ff=20, r=3, r_svd=4):
+    rng_ = np.random.default_rng(seed)
+    lay = {"scale": 0.7}
+    for nm, n, k in (("g", d_ff, d), ("u", d_ff, d), ("d", d, d_ff)):
+        lay["W" + nm] = rng_.normal(size=(n, k)) / np.sqrt(k)
+        lay["A" + nm] = rng_.normal(size=(r, k)) * 0.3
+        lay["B" + nm] = rng_.normal(size=(n, r)) * 0.3
+    lay["Lg"], lay["Ug"] = O.svd_prepare(lay["Wg"], r_svd)
+    lay["Lu"], lay["Uu"] = O.svd_prepare(lay["Wu"], r_svd)
+    return lay
+
+
+def test_per_sequence_sets_with_identical_sequences_equal_the_batch_set():
+    """Pooling over identical sequences multiplies every score by the same
+    factor: the per-batch set is each sequence's set, and the per-batch
+    gradients are the per-sequence sums."""
+    lay = _tiny_ffn(1)
+    seq, d = 7, 12
+    x1 = np.random.default_rng(2).normal(size=(seq, d))
+    dy1 = np.random.default_rng(3).normal(size=(seq, d))
+    X, dY = np.vstack([x1, x1, x1]), np.vstack([dy1, dy1, dy1])
+    per = O.ffn_fwd_bwd_per_seq(X, dY, 3, seq, [5, 5, 5], lay, 0.5)
+    bat = O.ffn_fwd_bwd(X, dY, 3, seq, [5, 5, 5], lay, 0.5)
+    for s_ in per["idx"]:
+        np.testing.assert_array_equal(s_, bat["idx"])
+    for key in ("out", "dX", "dAg", "dBg", "dAu", "dBu", "dAd", "dBd"):
+        np.testing.assert_allclose(per[key], bat[key], rtol=1e-12, atol=1e-13)
+
+
+def test_per_sequence_matches_row_masked_dense_autograd():
+    """Independent formulation: a dense SwiGLU FFN in PyTorch float64 whose
+    context rows multiply the intermediate activations by their own
+    sequence's 0/1 channel mask, gradients by autograd."""
+    lay = _tiny_ffn(4)
+    b, seq, d = 3, 6, 12
+    ctx = [4, 6, 2]
+    rng_ = np.random.default_rng(5)
+    X, dY = rng_.normal(size=(b * seq, d)), rng_.normal(size=(b * seq, d))
+    per = O.ffn_fwd_bwd_per_seq(X, dY, b, seq, ctx, lay, 0.6)
+    assert len({tuple(s_) for s_ in per["idx"]}) > 1   # the sets do differ
+    mask = np.ones((b * seq, 20))
+    for bb in range(b):
+        m = np.zeros(20)
+        m[per["idx"][bb]] = 1.0
+        mask[bb * seq: bb * seq + ctx[bb]] = m
+    t = {k: torch.from_numpy(np.asarray(v, dtype=np.float64).copy()).requires_grad_()
+         for k, v in lay.items() if k[0] in "AB"}
+    W = {k: torch.from_numpy(lay[k]) for k in ("Wg", "Wu", "Wd")}
+    tx = torch.from_numpy(X.copy()).requires_grad_()
+    s_ = lay["scale"]
+    g = tx @ W["Wg"].T + s_ * (tx @ t["Ag"].T) @ t["Bg"].T
+    u = tx @ W["Wu"].T + s_ * (tx @ t["Au"].T) @ t["Bu"].T
+    h = torch.nn.functional.silu(g) * u * torch.from_numpy(mask)
+    y = h @ W["Wd"].T + s_ * (h @ t["Ad"].T) @ t["Bd"].T
+    np.testing.assert_allclose(per["out"], y.detach().numpy(), rtol=1e-11, atol=1e-12)
+    (y * torch.from_numpy(dY)).sum().backward()
+    np.testing.assert_allclose(per["dX"], tx.grad.numpy(), rtol=1e-10, atol=1e-12)
+    for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd"):
+        np.testing.assert_allclose(per["d" + k], t[k].grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_down_projection_only_equals_the_sliced_ffn():
+    """Dropping a channel's activation before the down projection gives the
+    sliced FFN's output: the gate/up values of a skipped channel reach the
+    output only through its down-projection column."""
+    lay = _tiny_ffn(6)
+    b, seq = 2, 5
+    X = np.random.default_rng(7).normal(size=(b * seq, 12))
+    idx = np.array([0, 3, 4, 9, 15, 19])
+    out, _ = O.ffn_fwd(X, b, seq, [3, 5], lay, idx)
+    np.testing.assert_allclose(O.ffn_fwd_down_only(X, b, seq, [3, 5], lay, idx), out,
+                               rtol=1e-12, atol=1e-13)
+    full = O.ffn_fwd_down_only(X, b, seq, [0, 0], lay, idx)   # no context rows: dense
+    dense, _ = O.ffn_fwd(X, b, seq, [0, 0], lay, np.arange(20))
+    np.testing.assert_allclose(full, dense, rtol=1e-12, atol=1e-13)
