@@ -828,6 +828,262 @@ __global__ void __launch_bounds__(kScoreThreads)
   score_tail<CH>(a, cb, &s_last);
 }
 
+// ---- tensor-core score kernel (rank <= 8)
+// The dot products g_hat = P_g U_g^T and u_hat = P_u U_u^T of a 128-channel
+// x 64-token tile run on tcgen05 (M = 128 channels, N = 64 tokens, bf16 in,
+// fp32 accumulators in tensor memory).  fp32 accuracy comes from three-term
+// bf16 splits of both operands: the K dimension (64) holds six blocks of
+// `rank` values pairing (U_h, P_h), (U_m, P_h), (U_h, P_m), (U_l, P_h),
+// (U_h, P_l), (U_m, P_m), the rest zero.  The constants -log2(e) (gate) and
+// -ln(2) (up) are folded into U before the split, so each (token, channel)
+// costs one ex2, one reciprocal and three FMA-pipe operations in the
+// epilogue, where 8 warps read the accumulators with tcgen05.ld (warp w: the
+// 32 channels of lane quarter w % 4, the 32 tokens of half w / 4).  Operands
+// are staged by the threads themselves (the split is a transformation) in the
+// 128-byte-swizzled K-major layout the MMA descriptors describe.  Software
+// pipeline over the block's tiles: while the epilogue of tile i reads its
+// accumulators, the MMAs of tile i + 1 run into the other half of the block's
+// 256 tensor-memory columns (both operand and accumulator buffers are
+// doubled) and the P rows of tile i + 2 are in flight into registers.  Two
+// blocks share an SM.
+constexpr int kTcTok = 64;            // tokens per tile (MMA N)
+constexpr int kTcCh = 128;            // channels per block (MMA M)
+constexpr int kTcK = 64;              // padded K (six blocks of <= 8)
+constexpr int kTcABytes = kTcCh * kTcK * 2;   // A tile: 128 rows x 64 bf16
+constexpr int kTcBBytes = kTcTok * kTcK * 2;  // B tile: 64 rows x 64 bf16
+// A_g, A_u, 2 x (B_g, B_u) + alignment + barriers, padded so that at most two
+// blocks (2 x 256 tensor-memory columns) are resident per SM
+constexpr int kTcSmem = 80 * 1024;
+constexpr float kTcNegLog2e = -1.4426950408889634f, kTcNegLn2 = -0.6931471805599453f;
+constexpr long long kTcWaitBudget = 2000000000LL;  // clock cycles
+
+__device__ __forceinline__ uint32_t tc_swz(int row, int chunk) {
+  return uint32_t(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(16 >> 4) << 16;    // leading byte offset (unused with this swizzle)
+  d |= uint64_t(1024 >> 4) << 32;  // 8-row group stride
+  d |= uint64_t(1) << 46;          // descriptor version
+  d |= uint64_t(2) << 61;          // 128-byte swizzle
+  return d;
+}
+// kind::f16, bf16 A and B (K-major), fp32 D, M = 128, N = 64
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTcTok >> 3) << 17) |
+                              (uint32_t(kTcCh >> 4) << 24);
+
+// Three-term bf16 split of 8 fp32 values: hi, mid, lo as 16-byte chunks.
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& h, uint4& m, uint4& l) {
+  __nv_bfloat162* ph = reinterpret_cast<__nv_bfloat162*>(&h);
+  __nv_bfloat162* pm = reinterpret_cast<__nv_bfloat162*>(&m);
+  __nv_bfloat162* pl = reinterpret_cast<__nv_bfloat162*>(&l);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = x[2 * i], b = x[2 * i + 1];
+    const __nv_bfloat162 vh = __floats2bfloat162_rn(a, b);
+    const float ra = a - __low2float(vh), rb = b - __high2float(vh);
+    const __nv_bfloat162 vm = __floats2bfloat162_rn(ra, rb);
+    ph[i] = vh;
+    pm[i] = vm;
+    pl[i] = __floats2bfloat162_rn(ra - __low2float(vm), rb - __high2float(vm));
+  }
+}
+__device__ __forceinline__ void sts16(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+// Row `row` of an operand tile: the six K blocks in the order of `pat` (0 =
+// hi, 1 = mid, 2 = lo), then two zero chunks.
+__device__ __forceinline__ void stage_split_row(uint32_t tile, int row, const float (&x)[8],
+                                                const int (&pat)[6]) {
+  uint4 t[3];
+  split8(x, t[0], t[1], t[2]);
+#pragma unroll
+  for (int c = 0; c < 6; ++c) sts16(tile + tc_swz(row, c), t[pat[c]]);
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  sts16(tile + tc_swz(row, 6), z);
+  sts16(tile + tc_swz(row, 7), z);
+}
+__device__ __forceinline__ bool tc_mbar_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok = 0;
+  const long long t0 = clock64();
+  while (true) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > kTcWaitBudget) {
+      atomicExch(&g_est_error, 2);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kScoreThreads, 2)
+    ffn_score_tc_kernel(const __grid_constant__ ScoreArgs a) {
+  extern __shared__ __align__(1024) unsigned char tc_smem[];
+  __shared__ uint32_t s_tmem;
+  __shared__ unsigned s_last;
+  __shared__ float s_half[kTcCh];
+  // 1024-byte aligned operand tiles (the swizzle pattern repeats every 1024 bytes)
+  const uint32_t base = (sh_addr(tc_smem) + 1023u) & ~1023u;
+  const uint32_t sAg = base, sAu = base + kTcABytes;
+  const uint32_t sB = base + 2 * kTcABytes;  // [2 buffers][g, u] x kTcBBytes
+  const uint32_t bar0 = sB + 4 * kTcBBytes;   // two mbarriers, one per buffer
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t cb = blockIdx.x;
+  const int sp = blockIdx.y;
+  const int r = a.r;
+  constexpr int patA[6] = {0, 1, 0, 2, 0, 1};  // U terms per K block
+  constexpr int patB[6] = {0, 0, 1, 0, 2, 1};  // P terms per K block
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     sh_addr(&s_tmem))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // A: this block's 128 channels of U_g (x -log2 e) and U_u (x -ln 2)
+  {
+    const int row = tid & 127, mat = tid >> 7;
+    const int64_t j = cb * kTcCh + row;
+    const float* U = mat ? a.Uu : a.Ug;
+    const float c = mat ? kTcNegLn2 : kTcNegLog2e;
+    float x[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = (j < a.n && q < r) ? U[j * r + q] * c : 0.f;
+    stage_split_row(mat ? sAu : sAg, row, x, patA);
+  }
+  const int64_t t0 = int64_t(sp) * a.chunk;
+  const int64_t t1 = ::min(a.T_C, t0 + a.chunk);
+  const int ntile = t1 > t0 ? int((t1 - t0 + kTcTok - 1) / kTcTok) : 0;
+  // staging role: threads 0..63 the P_g row of token tid, 64..127 its P_u row
+  const bool stager = tid < 2 * kTcTok;
+  const int srow = tid & (kTcTok - 1), smat = tid / kTcTok;
+  auto load_p = [&](int it, float (&x)[8]) {
+    const int64_t t = t0 + int64_t(it) * kTcTok + srow;
+    if (stager && it < ntile && t < t1) {
+      const int64_t prow = a.pmap ? a.pmap[t] : t;
+      const float* src = a.P + prow * a.ldp + smat * r;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) x[q] = q < r ? src[q] : 0.f;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) x[q] = 0.f;
+    }
+  };
+  auto stage_b = [&](int it, const float (&x)[8]) {
+    if (stager) stage_split_row(sB + ((it & 1) * 2 + smat) * kTcBBytes, srow, x, patB);
+  };
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  auto issue = [&](int it) {  // MMAs of tile `it` into accumulator buffer it & 1
+    const int b = it & 1;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t sa = m ? sAu : sAg, sb = sB + (b * 2 + m) * kTcBBytes;
+      const uint32_t d = tmem + uint32_t(b * 2 * kTcTok + m * kTcTok);
+#pragma unroll
+      for (int k = 0; k < kTcK / 16; ++k) {
+        const uint64_t ad = tc_sdesc(sa + k * 32), bd = tc_sdesc(sb + k * 32);
+        const uint32_t en = k ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+            "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(en)
+            : "memory");
+      }
+    }
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            bar0 + 8 * b)
+        : "memory");
+  };
+  const int q4 = warp & 3, half = warp >> 2;
+  float acc = 0.f;
+  bool ok = true;
+  float xn[8];
+  if (ntile > 0) {  // prologue: tile 0 staged and issued, tile 1's P rows in flight
+    load_p(0, xn);
+    stage_b(0, xn);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) issue(0);
+    load_p(1, xn);
+  }
+  for (int it = 0; it < ntile; ++it) {
+    if (it + 1 < ntile) stage_b(it + 1, xn);  // its buffer's MMAs (tile it - 1) are done
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();  // staged rows written; tile it - 1's accumulator reads done
+    tc_fence_after();
+    if (tid == 0 && it + 1 < ntile) issue(it + 1);
+    load_p(it + 2, xn);
+    const bool w = tc_mbar_wait(bar0 + 8 * (it & 1), uint32_t((it >> 1) & 1));
+    ok = __syncthreads_and(w ? 1 : 0) != 0;
+    tc_fence_after();
+    if (!ok) break;
+    // epilogue: this warp's 32 channels x 32 tokens of tile it
+    uint32_t g[32], u[32];
+    const uint32_t ta = tmem + (uint32_t(q4 * 32) << 16) +
+                        uint32_t((it & 1) * 2 * kTcTok + half * 32);
+    tc_ld32(ta, g);
+    tc_ld32(ta + kTcTok, u);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float gp = __uint_as_float(g[i]), up = __uint_as_float(u[i]);
+      const float v = gp * up * rcp_approx(1.f + ex2_approx(gp));
+      acc = fmaf(v, v, acc);
+    }
+  }
+  // the two token halves of each channel, added in order
+  tc_fence_before();
+  if (half) s_half[q4 * 32 + lane] = acc;
+  __syncthreads();
+  if (!half) {
+    const int64_t j = cb * kTcCh + q4 * 32 + lane;
+    if (j < a.n) a.partial[int64_t(sp) * a.n + j] = acc + s_half[q4 * 32 + lane];
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem)
+                 : "memory");
+  }
+  score_tail<kTcCh>(a, cb, &s_last);
+}
+
 // ------------------------------------------------------------ Gram criterion
 constexpr int kGramThreads = 256;
 constexpr int kGramTokens = 64;  // P rows staged per round
@@ -980,7 +1236,7 @@ int rank_chunks(int r) { return r <= 8 ? 1 : (r <= 16 ? 2 : (r <= 24 ? 3 : (r <=
 // Score kernel by rank: packed FMA for r <= 16, tensor cores above (whose
 // factor rows no longer fit the registers of the FMA form).
 int channels_per_block(int r) {
-  if (r <= 8) return fma_channels<8>();
+  if (r <= 8) return kTcCh;
   if (r <= 16) return fma_channels<16>();
   return kScoreWarps * score_nt(rank_chunks(r)) * 8;
 }
@@ -1002,11 +1258,11 @@ int blocks_per_sm_of(K kernel, int smem) {
   return b;
 }
 int score_blocks_per_sm(int r) {
+  if (r <= 8) return 2;  // the tensor-core kernel: two blocks of 256 TMEM columns
   static int cached[5] = {0, 0, 0, 0, 0};
-  const int v = r <= 8 ? 0 : (r <= 16 ? 1 : (r <= 24 ? 2 : (r <= 32 ? 3 : 4)));
+  const int v = r <= 16 ? 1 : (r <= 24 ? 2 : (r <= 32 ? 3 : 4));
   if (!cached[v]) {
     switch (v) {
-      case 0: cached[v] = blocks_per_sm_of(ffn_score_fma_kernel<8>, 0); break;
       case 1: cached[v] = blocks_per_sm_of(ffn_score_fma_kernel<16>, 0); break;
       case 2: cached[v] = blocks_per_sm_of(ffn_score_mma_kernel<3>, score_stage_bytes(3)); break;
       case 3: cached[v] = blocks_per_sm_of(ffn_score_mma_kernel<4>, score_stage_bytes(4)); break;
@@ -1033,8 +1289,17 @@ int64_t ffn_score_blocks(int64_t n, int r) {
   return (n + ch - 1) / ch;
 }
 
-// Token splits: as many as keep the grid within one wave of resident blocks.
+// Token splits: for the tensor-core kernel (rank <= 8) enough blocks for
+// about one and a half per SM, two of them resident per SM (each block
+// pipelines its tiles); otherwise as many as keep the grid within one wave of
+// resident blocks.
 int ffn_score_splits(int64_t T_C, int64_t n, int r) {
+  if (r <= 8) {
+    const int64_t tiles = std::max<int64_t>((T_C + kTcTok - 1) / kTcTok, 1);
+    const int64_t nb = std::max<int64_t>(ffn_score_blocks(n, r), 1);
+    const int64_t want = (int64_t(num_sms()) * 3 / 2 + nb - 1) / nb;
+    return int(std::min<int64_t>(std::max<int64_t>(want, 1), std::min<int64_t>(tiles, 256)));
+  }
   const int64_t nb = ffn_score_blocks(n, r);
   const int64_t slots = int64_t(num_sms()) * score_blocks_per_sm(r);
   int64_t want = slots / std::max<int64_t>(nb, 1);
@@ -1102,16 +1367,23 @@ slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, 
   ScoreArgs a;
   a.P = P; a.ldp = ldp; a.pmap = pmap; a.T_C = T_C; a.Ug = Ug; a.Uu = Uu; a.n = n; a.r = r;
   a.nsplit = nsplit;
-  a.chunk = T_C > 0 ? ((T_C + nsplit - 1) / nsplit + 15) / 16 * 16 : 16;
+  // tokens per split: whole 128-token tiles for the tensor-core kernel, 16 otherwise
+  const int64_t q = r <= 8 ? kTcTok : 16;
+  a.chunk = T_C > 0 ? ((T_C + nsplit - 1) / nsplit + q - 1) / q * q : q;
   a.partial = partial; a.scores = scores; a.counters = counters;
   const dim3 grid(unsigned(ffn_score_blocks(n, r)), unsigned(nsplit));
   {
     // bytes: P rows of the context tokens, both factors, partials and scores
     LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 +
                                   double(nsplit) * n * 8 + double(n) * 4, st);
-    if (r <= 8)
-      ffn_score_fma_kernel<8><<<grid, kScoreThreads, 0, st>>>(a);
-    else if (r <= 16)
+    if (r <= 8) {
+      SLORA_CUDA(cudaFuncSetAttribute(ffn_score_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem));
+      // the largest shared-memory carveout, or only one block fits per SM
+      SLORA_CUDA(cudaFuncSetAttribute(ffn_score_tc_kernel,
+                                      cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+      ffn_score_tc_kernel<<<grid, kScoreThreads, kTcSmem, st>>>(a);
+    } else if (r <= 16)
       ffn_score_fma_kernel<16><<<grid, kScoreThreads, 0, st>>>(a);
     else if (r <= 24)
       SLORA_TRY(launch_score_mma<3>(grid, a, st));

@@ -128,7 +128,7 @@ def test_attention_full_size_sampled_heads(L):
 
 
 # -------------------------------------------------------------- RMS norm
-@pytest.mark.parametrize("T,d", [(37, 256), (8, 4096)])
+@pytest.mark.parametrize("T,d", [(37, 256), (8, 4096), (3, 17408)])
 def test_rmsnorm_fwd_bwd_matches_oracle(L, T, d):
     rng = np.random.default_rng(T + d)
     X, A = _rb(rng.normal(size=(T, d)) * 2), _rb(rng.normal(size=(T, d)))
