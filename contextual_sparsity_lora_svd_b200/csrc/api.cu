@@ -152,6 +152,7 @@ EstBufs estimate_reserve(slora_criterion crit, int dt, const TokenInfo& ti, int6
   if (cp.activation) {
     eb.nsplit = ffn_score_splits(ti.T_C, n0, rank);
     eb.partial = ar.take<float>(size_t(eb.nsplit) * n0);
+    if (rank <= 8) eb.psplit = ar.take<uint4>(size_t(score_split_tiles(ti.T_C)) * 1024);
   } else {
     eb.gram_part = ar.take<double>(size_t(gram_blocks(ti.T_C)) * cp.nmat * rank * rank);
     eb.gram = ar.take<double>(size_t(cp.nmat) * rank * rank);
@@ -212,7 +213,7 @@ slora_status estimate_select_launch(slora_criterion crit, const void* X, int dt,
   }
   if (cp.activation)
     return ffn_score_select(Puse, ldp, pmap, ti.T_C, U0, U1, n0, rank, eb.partial, eb.nsplit,
-                            eb.scores, eb.cnt, int(cp.kkeep), idx_out, st);
+                            eb.scores, eb.cnt, int(cp.kkeep), idx_out, eb.psplit, st);
   int32_t* out_b = nullptr;
   if (crit == SLORA_CRIT_QK_NORM || crit == SLORA_CRIT_QK_ROPE_PAIR ||
       crit == SLORA_CRIT_L2_NORM)

@@ -461,6 +461,7 @@ struct ScoreArgs {
   float* partial;        // [nsplit x n]
   float* scores;         // [n]
   unsigned* counters;    // [nblocks], zero on entry
+  const uint4* psplit;   // tensor-core kernel: split P rows per 64-token tile (16 KB each)
 };
 
 // Common end of the score kernels: the last split of a channel block to
@@ -836,9 +837,10 @@ __global__ void __launch_bounds__(kScoreThreads)
 // `rank` values pairing (U_h, P_h), (U_m, P_h), (U_h, P_m), (U_l, P_h),
 // (U_h, P_l), (U_m, P_m), the rest zero.  The constants -log2(e) (gate) and
 // -ln(2) (up) are folded into U before the split, so each (token, channel)
-// costs one ex2, one reciprocal and three FMA-pipe operations in the
-// epilogue, where 8 warps read the accumulators with tcgen05.ld (warp w: the
-// 32 channels of lane quarter w % 4, the 32 tokens of half w / 4).  Operands
+// costs one ex2, half a reciprocal (two tokens share one) and a few FMA-pipe
+// operations in the epilogue, where 8 warps read the accumulators with
+// tcgen05.ld (warp w: the 32 channels of lane quarter w % 4, the 32 tokens
+// of half w / 4).  Operands
 // are staged by the threads themselves (the split is a transformation) in the
 // 128-byte-swizzled K-major layout the MMA descriptors describe.  Software
 // pipeline over the block's tiles: while the epilogue of tile i reads its
@@ -943,7 +945,51 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(kScoreThreads, 2)
+// The split operand rows of every 64-token tile, once for all channel blocks:
+// psplit[tile][mat][row] is 128 bytes (the six K blocks of P_mat's row of
+// token tile * 64 + row, then zeros) with the 128-byte swizzle applied, so a
+// plain bulk copy into a 1024-byte aligned buffer gives the MMA layout.
+// Rows past T_C are zero.
+__global__ void score_split_p_kernel(const float* __restrict__ P, int64_t ldp,
+                                     const int32_t* __restrict__ pmap, int64_t T_C, int r,
+                                     int64_t ntiles, uint4* __restrict__ psplit) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // (tile, mat, row)
+  if (i >= ntiles * 2 * kTcTok) return;
+  const int row = int(i % kTcTok), mat = int((i / kTcTok) % 2);
+  const int64_t tile = i / (2 * kTcTok);
+  const int64_t t = tile * kTcTok + row;
+  float x[8];
+  if (t < T_C) {
+    const int64_t prow = pmap ? pmap[t] : t;
+    const float* src = P + prow * ldp + mat * r;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = q < r ? src[q] : 0.f;
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[q] = 0.f;
+  }
+  uint4 t3[3];
+  split8(x, t3[0], t3[1], t3[2]);
+  constexpr int patB[6] = {0, 0, 1, 0, 2, 1};  // P terms per K block
+  uint4* dst = psplit + ((tile * 2 + mat) * kTcTok + row) * 8;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) dst[c ^ (row & 7)] = c < 6 ? t3[patB[c]] : make_uint4(0, 0, 0, 0);
+}
+
+constexpr int kTcEpiWarps = 8;                       // epilogue warps
+constexpr int kTcThreads = (kTcEpiWarps + 1) * 32;    // + one producer / MMA warp
+
+__device__ __forceinline__ void tc_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Warp-specialized: warps 0-7 read the accumulators and run the silu
+// epilogue; lane 0 of warp 8 brings each tile's split P rows in by one bulk
+// copy and issues the MMAs.  Handoffs through mbarriers only: loaded[b] (the
+// rows of the tile in buffer b have landed), full[b] (its MMAs are done:
+// tensor memory readable, its operand rows free) and empty[b] (the 8
+// epilogue warps have read buffer b's accumulators).
+__global__ void __launch_bounds__(kTcThreads, 2)
     ffn_score_tc_kernel(const __grid_constant__ ScoreArgs a) {
   extern __shared__ __align__(1024) unsigned char tc_smem[];
   __shared__ uint32_t s_tmem;
@@ -952,8 +998,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
   // 1024-byte aligned operand tiles (the swizzle pattern repeats every 1024 bytes)
   const uint32_t base = (sh_addr(tc_smem) + 1023u) & ~1023u;
   const uint32_t sAg = base, sAu = base + kTcABytes;
-  const uint32_t sB = base + 2 * kTcABytes;  // [2 buffers][g, u] x kTcBBytes
-  const uint32_t bar0 = sB + 4 * kTcBBytes;   // two mbarriers, one per buffer
+  const uint32_t sB = base + 2 * kTcABytes;   // [2 buffers][g, u] x kTcBBytes
+  const uint32_t full0 = sB + 4 * kTcBBytes;  // full[2], empty[2], loaded[2]
+  const uint32_t empty0 = full0 + 16, loaded0 = full0 + 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t cb = blockIdx.x;
   const int sp = blockIdx.y;
@@ -967,12 +1014,17 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8) : "memory");
+    for (int b = 0; b < 2; ++b) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * b) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8 * b),
+                   "r"(kTcEpiWarps)
+                   : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(loaded0 + 8 * b) : "memory");
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // A: this block's 128 channels of U_g (x -log2 e) and U_u (x -ln 2)
-  {
+  if (tid < 2 * kTcCh) {
     const int row = tid & 127, mat = tid >> 7;
     const int64_t j = cb * kTcCh + row;
     const float* U = mat ? a.Uu : a.Ug;
@@ -985,94 +1037,106 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
   const int64_t t0 = int64_t(sp) * a.chunk;
   const int64_t t1 = ::min(a.T_C, t0 + a.chunk);
   const int ntile = t1 > t0 ? int((t1 - t0 + kTcTok - 1) / kTcTok) : 0;
-  // staging role: threads 0..63 the P_g row of token tid, 64..127 its P_u row
-  const bool stager = tid < 2 * kTcTok;
-  const int srow = tid & (kTcTok - 1), smat = tid / kTcTok;
-  auto load_p = [&](int it, float (&x)[8]) {
-    const int64_t t = t0 + int64_t(it) * kTcTok + srow;
-    if (stager && it < ntile && t < t1) {
-      const int64_t prow = a.pmap ? a.pmap[t] : t;
-      const float* src = a.P + prow * a.ldp + smat * r;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) x[q] = q < r ? src[q] : 0.f;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) x[q] = 0.f;
-    }
-  };
-  auto stage_b = [&](int it, const float (&x)[8]) {
-    if (stager) stage_split_row(sB + ((it & 1) * 2 + smat) * kTcBBytes, srow, x, patB);
-  };
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  auto issue = [&](int it) {  // MMAs of tile `it` into accumulator buffer it & 1
-    const int b = it & 1;
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const uint32_t sa = m ? sAu : sAg, sb = sB + (b * 2 + m) * kTcBBytes;
-      const uint32_t d = tmem + uint32_t(b * 2 * kTcTok + m * kTcTok);
-#pragma unroll
-      for (int k = 0; k < kTcK / 16; ++k) {
-        const uint64_t ad = tc_sdesc(sa + k * 32), bd = tc_sdesc(sb + k * 32);
-        const uint32_t en = k ? 1u : 0u;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-            "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(en)
-            : "memory");
-      }
-    }
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            bar0 + 8 * b)
-        : "memory");
-  };
-  const int q4 = warp & 3, half = warp >> 2;
   float acc = 0.f;
-  bool ok = true;
-  float xn[8];
-  if (ntile > 0) {  // prologue: tile 0 staged and issued, tile 1's P rows in flight
-    load_p(0, xn);
-    stage_b(0, xn);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0) issue(0);
-    load_p(1, xn);
-  }
-  for (int it = 0; it < ntile; ++it) {
-    if (it + 1 < ntile) stage_b(it + 1, xn);  // its buffer's MMAs (tile it - 1) are done
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();  // staged rows written; tile it - 1's accumulator reads done
-    tc_fence_after();
-    if (tid == 0 && it + 1 < ntile) issue(it + 1);
-    load_p(it + 2, xn);
-    const bool w = tc_mbar_wait(bar0 + 8 * (it & 1), uint32_t((it >> 1) & 1));
-    ok = __syncthreads_and(w ? 1 : 0) != 0;
-    tc_fence_after();
-    if (!ok) break;
-    // epilogue: this warp's 32 channels x 32 tokens of tile it
-    uint32_t g[32], u[32];
-    const uint32_t ta = tmem + (uint32_t(q4 * 32) << 16) +
-                        uint32_t((it & 1) * 2 * kTcTok + half * 32);
-    tc_ld32(ta, g);
-    tc_ld32(ta + kTcTok, u);
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  const int q4 = warp & 3, half = (warp >> 2) & 1;
+  if (warp == kTcEpiWarps) {
+    // ---- producer (lane 0): each tile's split P rows arrive by one bulk copy
+    // (prepared once for every channel block by score_split_p_kernel), two
+    // tiles ahead; the MMAs of a tile start once its rows have landed and the
+    // epilogue has read the accumulator buffer they overwrite
+    const int64_t tile0 = t0 / kTcTok;
+    bool ok = true;
+    auto copy = [&](int it) {
+      const int b = it & 1;
+      const uint32_t lb = loaded0 + 8 * b;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(lb),
+                   "r"(2 * kTcBBytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+          "[%3];" ::"r"(sB + b * 2 * kTcBBytes),
+          "l"(a.psplit + (tile0 + it) * (2 * kTcBBytes / 16)), "r"(2 * kTcBBytes), "r"(lb)
+          : "memory");
+    };
+    if (lane == 0) {
+      for (int it = 0; it < ::min(ntile, 2); ++it) copy(it);
+      for (int it = 0; it < ntile && ok; ++it) {
+        const int b = it & 1;
+        const uint32_t par = uint32_t((it >> 1) & 1);
+        ok = tc_mbar_wait(loaded0 + 8 * b, par);                            // rows landed
+        if (ok && it >= 2) ok = tc_mbar_wait(empty0 + 8 * b, par ^ 1u);    // tile it-2 read
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float gp = __uint_as_float(g[i]), up = __uint_as_float(u[i]);
-      const float v = gp * up * rcp_approx(1.f + ex2_approx(gp));
-      acc = fmaf(v, v, acc);
+        for (int m = 0; m < 2; ++m) {
+          const uint32_t sa = m ? sAu : sAg, sb = sB + (b * 2 + m) * kTcBBytes;
+          const uint32_t d = tmem + uint32_t(b * 2 * kTcTok + m * kTcTok);
+#pragma unroll
+          for (int k = 0; k < kTcK / 16; ++k) {
+            const uint64_t ad = tc_sdesc(sa + k * 32), bd = tc_sdesc(sb + k * 32);
+            const uint32_t en = k ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+                "l"(ad), "l"(bd), "r"(kTcIdesc), "r"(en)
+                : "memory");
+          }
+        }
+        asm volatile(
+            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                full0 + 8 * b)
+            : "memory");
+        if (it + 2 < ntile) {  // its operand rows are free once these MMAs are done
+          ok = tc_mbar_wait(full0 + 8 * b, par);
+          if (ok) copy(it + 2);
+        }
+      }
+      // the last MMAs complete before the block releases its tensor memory
+      if (ok && ntile > 0)
+        tc_mbar_wait(full0 + 8 * ((ntile - 1) & 1), uint32_t(((ntile - 1) >> 1) & 1));
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: this warp's 32 channels x 32 tokens of each tile
+    for (int it = 0; it < ntile; ++it) {
+      const int b = it & 1;
+      if (!tc_mbar_wait(full0 + 8 * b, uint32_t((it >> 1) & 1))) break;
+      tc_fence_after();
+      uint32_t g[32], u[32];
+      const uint32_t ta = tmem + (uint32_t(q4 * 32) << 16) + uint32_t(b * 2 * kTcTok + half * 32);
+      tc_ld32(ta, g);
+      tc_ld32(ta + kTcTok, u);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc_arrive(empty0 + 8 * b);
+      // silu(g) u = g' u' / (1 + 2^g') for two tokens at a time with one
+      // reciprocal (Montgomery's simultaneous inversion: 1/d1 = d2 / (d1 d2));
+      // 2^g' is capped at 2^60 so the product stays finite (a capped term is
+      // below 2^-60 g' u' either way)
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const float g1 = __uint_as_float(g[i]), u1 = __uint_as_float(u[i]);
+        const float g2 = __uint_as_float(g[i + 1]), u2 = __uint_as_float(u[i + 1]);
+        const float d1 = 1.f + fminf(ex2_approx(g1), 0x1p60f);
+        const float d2 = 1.f + fminf(ex2_approx(g2), 0x1p60f);
+        const float R = rcp_approx(d1 * d2);
+        const float v1 = g1 * u1 * (d2 * R), v2 = g2 * u2 * (d1 * R);
+        acc = fmaf(v1, v1, acc);
+        acc = fmaf(v2, v2, acc);
+      }
     }
   }
   // the two token halves of each channel, added in order
   tc_fence_before();
-  if (half) s_half[q4 * 32 + lane] = acc;
+  if (warp < kTcEpiWarps && half) s_half[q4 * 32 + lane] = acc;
   __syncthreads();
-  if (!half) {
+  if (warp < kTcEpiWarps && !half) {
     const int64_t j = cb * kTcCh + q4 * 32 + lane;
     if (j < a.n) a.partial[int64_t(sp) * a.n + j] = acc + s_half[q4 * 32 + lane];
   }
@@ -1289,10 +1353,10 @@ int64_t ffn_score_blocks(int64_t n, int r) {
   return (n + ch - 1) / ch;
 }
 
-// Token splits: for the tensor-core kernel (rank <= 8) enough blocks for
-// about one and a half per SM, two of them resident per SM (each block
-// pipelines its tiles); otherwise as many as keep the grid within one wave of
-// resident blocks.
+// Token splits: for the tensor-core kernel (rank <= 8) about one and a half
+// blocks per SM, two resident per SM, each pipelining its tiles (blocks of a
+// few tiles measured slower: their setup does not amortise); otherwise as
+// many as keep the grid within one wave of resident blocks.
 int ffn_score_splits(int64_t T_C, int64_t n, int r) {
   if (r <= 8) {
     const int64_t tiles = std::max<int64_t>((T_C + kTcTok - 1) / kTcTok, 1);
@@ -1309,6 +1373,8 @@ int ffn_score_splits(int64_t T_C, int64_t n, int r) {
   if (s > 256) s = 256;
   return int(s);
 }
+
+int64_t score_split_tiles(int64_t T_C) { return std::max<int64_t>((T_C + kTcTok - 1) / kTcTok, 1); }
 
 int64_t estimator_counter_count(int64_t n, int r, int groups) {
   (void)groups;  // the score kernels count per channel block, the Gram pass in one word
@@ -1362,11 +1428,12 @@ slora_status launch_topk(const float* scores, int groups, int N, int k, const To
 slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
                               const float* Ug, const float* Uu, int64_t n, int r, float* partial,
                               int nsplit, float* scores, unsigned* counters, int k,
-                              int32_t* idx_out, cudaStream_t st) {
+                              int32_t* idx_out, void* psplit, cudaStream_t st) {
   if (n <= 0) return SLORA_OK;
   ScoreArgs a;
   a.P = P; a.ldp = ldp; a.pmap = pmap; a.T_C = T_C; a.Ug = Ug; a.Uu = Uu; a.n = n; a.r = r;
   a.nsplit = nsplit;
+  a.psplit = static_cast<const uint4*>(psplit);
   // tokens per split: whole 128-token tiles for the tensor-core kernel, 16 otherwise
   const int64_t q = r <= 8 ? kTcTok : 16;
   a.chunk = T_C > 0 ? ((T_C + nsplit - 1) / nsplit + q - 1) / q * q : q;
@@ -1377,12 +1444,20 @@ slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, 
     LaunchScope ls(kEstimate, double(T_C) * 2 * r * 4 + double(n) * 2 * r * 4 +
                                   double(nsplit) * n * 8 + double(n) * 4, st);
     if (r <= 8) {
+      if (!psplit) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "score: split-operand workspace missing");
+      const int64_t ntiles = score_split_tiles(T_C);
+      {
+        LaunchScope lp(kEstimate, double(T_C) * 2 * r * 4 + double(ntiles) * 2 * kTcBBytes, st);
+        score_split_p_kernel<<<unsigned((ntiles * 2 * kTcTok + 255) / 256), 256, 0, st>>>(
+            P, ldp, pmap, T_C, r, ntiles, static_cast<uint4*>(psplit));
+        SLORA_CHECK_LAUNCH();
+      }
       SLORA_CUDA(cudaFuncSetAttribute(ffn_score_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem));
       // the largest shared-memory carveout, or only one block fits per SM
       SLORA_CUDA(cudaFuncSetAttribute(ffn_score_tc_kernel,
                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-      ffn_score_tc_kernel<<<grid, kScoreThreads, kTcSmem, st>>>(a);
+      ffn_score_tc_kernel<<<grid, kTcThreads, kTcSmem, st>>>(a);
     } else if (r <= 16)
       ffn_score_fma_kernel<16><<<grid, kScoreThreads, 0, st>>>(a);
     else if (r <= 24)

@@ -21,8 +21,11 @@ namespace slora {
 slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, int64_t T_C,
                               const float* Ug, const float* Uu, int64_t n, int r, float* partial,
                               int nsplit, float* scores, unsigned* counters, int k,
-                              int32_t* idx_out, cudaStream_t st);
+                              int32_t* idx_out, void* psplit, cudaStream_t st);
 int ffn_score_splits(int64_t T_C, int64_t n, int r);
+// 64-token tiles of the split operand rows the rank <= 8 score kernel reads
+// (16 KB each in the workspace argument psplit of ffn_score_select).
+int64_t score_split_tiles(int64_t T_C);
 
 // Gram-form criteria.  G_m = P_m^T P_m (fp64) for the P matrices in columns
 // [m r, (m+1) r) of P; a channel's estimated norm is sqrt(u^T G_m u) for its

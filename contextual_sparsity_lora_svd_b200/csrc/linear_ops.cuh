@@ -54,6 +54,7 @@ struct EstBufs {
   double* gram = nullptr;    // Gram matrices of the projection
   double* gram_part = nullptr;  // their partials over token chunks
   unsigned* cnt = nullptr;   // arrival counters of the estimator kernels, zero on entry
+  void* psplit = nullptr;    // split operand rows of the tensor-core score kernel
   int64_t ncnt = 0;
   int nsplit = 1;
 };
