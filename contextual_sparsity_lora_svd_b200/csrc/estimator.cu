@@ -1447,7 +1447,7 @@ slora_status ffn_score_select(const float* P, int64_t ldp, const int32_t* pmap, 
       if (!psplit) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "score: split-operand workspace missing");
       const int64_t ntiles = score_split_tiles(T_C);
       {
-        LaunchScope lp(kEstimate, double(T_C) * 2 * r * 4 + double(ntiles) * 2 * kTcBBytes, st);
+        LaunchScope lp(kAux, double(T_C) * 2 * r * 4 + double(ntiles) * 2 * kTcBBytes, st);
         score_split_p_kernel<<<unsigned((ntiles * 2 * kTcTok + 255) / 256), 256, 0, st>>>(
             P, ldp, pmap, T_C, r, ntiles, static_cast<uint4*>(psplit));
         SLORA_CHECK_LAUNCH();
