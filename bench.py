@@ -210,8 +210,8 @@ def workload_config(name, world):
                 "global_batch": w["batch"] * world, "seq_len": w["seq"], "layers": w["layers"],
                 "d": w["d"], "d_ff": w["d_ff"], "heads": w["heads"], "r_svd": w["r_svd"],
                 "r_lora": w["r_lora"], "ffn_sparsity": list(t.ffn), "qk_sparsity": list(t.qk),
-                "v_o": "dense LoRA", "ffn_backward": "forward recomputed from the saved FFN "
-                                                     "input with the forward's channel set",
+                "v_o": "dense LoRA", "ffn_backward": "from the forward state kept in each "
+                                                     "layer's FFN workspace (slora_ffn_bwd)",
                 "excluded": "embeddings, final norm and loss (a synthetic output gradient)",
                 "parallelism": par, "l2": L2_NOTE,
                 "launch": "the whole step (forward of 32 layers, then backward) captured as one "

@@ -87,6 +87,9 @@ _sig("slora_ffn_fwd_bwd", c_int,
       c_vp,
       ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 
+_sig("slora_ffn_bwd", c_int,
+     [c_int, ctypes.POINTER(FfnLayer), ctypes.POINTER(Tokens), ctypes.c_double, c_vp, c_vp, c_vp,
+      c_vp, ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
 _sig("slora_ffn_fwd_bwd_per_seq", c_int,
      [c_int, ctypes.POINTER(FfnLayer), ctypes.POINTER(Tokens), ctypes.c_double, c_vp, c_vp, c_vp,
       c_vp, ctypes.POINTER(FfnGrads), c_vp, P_I32, c_vp, c_i32, c_vp, P_SZ, c_vp])
@@ -121,7 +124,8 @@ EXPORTS = sorted(["slora_last_error_string", "slora_version", "slora_svd_prepare
                   "slora_ffn_fwd_bwd", "slora_launch_count", "slora_profile_enable",
                   "slora_profile_read", "slora_noalloc_scratch_bytes",
                   "slora_estimate_select_noalloc", "slora_device_error",
-                  "slora_set_wait_budget", "slora_ffn_fwd_bwd_per_seq", "slora_rope_pack", "slora_rope_unpack",
+                  "slora_set_wait_budget", "slora_ffn_bwd", "slora_ffn_fwd_bwd_per_seq",
+                  "slora_rope_pack", "slora_rope_unpack",
                   "slora_attention_fwd", "slora_attention_bwd", "slora_rmsnorm_fwd",
                   "slora_rmsnorm_bwd"])
 
@@ -309,6 +313,23 @@ def slora_ffn_fwd_bwd(layer: FfnLayer, batch, seq, ctx_len, sparsity, X, dOut, o
         args[-1] = idx_force.numel() // batch
     _run("slora_ffn_fwd_bwd_per_seq" if per_sequence else "slora_ffn_fwd_bwd", args, ws, stream)
     return int(keep[2].value)
+
+
+def slora_ffn_bwd(layer: FfnLayer, batch, seq, ctx_len, sparsity, X, dOut, out, dX,
+                  grads: FfnGrads, idx_out, ws, idx_force=None, stream=None) -> int:
+    """The backward half on the workspace `ws` of an earlier forward-only
+    slora_ffn_fwd_bwd call with the same arguments.  Returns k_keep."""
+    args, keep = ffn_args(dtype_code(X), layer, batch, seq, ctx_len, sparsity, X, dOut, out, dX,
+                          grads, idx_out, idx_force)
+    _run("slora_ffn_bwd", args, ws, stream)
+    return int(keep[2].value)
+
+
+def ffn_workspace_bytes(layer: FfnLayer, batch, seq, ctx_len, sparsity, X, out, idx_out,
+                        idx_force=None) -> int:
+    args, keep = ffn_args(dtype_code(X), layer, batch, seq, ctx_len, sparsity, X, None, out, None,
+                          None, idx_out, idx_force)
+    return workspace_size("slora_ffn_fwd_bwd", args)
 
 
 # ------------------------------------------- decoder-layer pieces

@@ -515,6 +515,35 @@ extern "C" slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer*
                  static_cast<cudaStream_t>(stream));
 }
 
+extern "C" slora_status slora_ffn_bwd(slora_dtype dt, const slora_ffn_layer* layer,
+                                      const slora_tokens* tok, double sparsity, const void* X,
+                                      const void* dOut, void* out, void* dX,
+                                      const slora_ffn_grads* grads, int32_t* idx_out,
+                                      int32_t* k_out, const int32_t* idx_force, int32_t k_force,
+                                      void* ws, size_t* ws_bytes, slora_stream_t stream) {
+  const char* fn = "slora_ffn_bwd";
+  clear_error();
+  if (!dOut) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "%s: dOut is NULL", fn);
+  int64_t kkeep = 0;
+  SLORA_TRY(ffn_validate(fn, dt, layer, grads, sparsity, X, dOut, out, dX, idx_out, k_out,
+                         idx_force, k_force, ws, &kkeep));
+  TokenInfo ti;
+  SLORA_TRY(parse_tokens(tok, &ti));
+  FfnDesc F{int(dt), ti, *layer, *grads, kkeep, sparsity};
+  Arena plan;
+  SLORA_TRY(ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, plan, true, nullptr, true));
+  const bool query = ws == nullptr;
+  SLORA_TRY(finish_ws(fn, plan, ws, ws_bytes));
+  *k_out = int32_t(kkeep);
+  if (query) return SLORA_OK;
+  SLORA_TRY(check_device());
+  Arena ar;
+  ar.base = static_cast<char*>(ws);
+  ar.cap = *ws_bytes;
+  return ffn_run(F, tok, X, dOut, out, dX, idx_out, idx_force, ar, false,
+                 static_cast<cudaStream_t>(stream), true);
+}
+
 extern "C" slora_status slora_ffn_fwd_bwd_per_seq(
     slora_dtype dt, const slora_ffn_layer* layer, const slora_tokens* tok, double sparsity,
     const void* X, const void* dOut, void* out, void* dX, const slora_ffn_grads* grads,

@@ -252,7 +252,8 @@ struct TcBuilder {
 
 slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X,
                         const void* dOut, void* out, void* dX, int32_t* idx,
-                        const int32_t* idx_force, Arena& ar, bool plan, cudaStream_t st) {
+                        const int32_t* idx_force, Arena& ar, bool plan, cudaStream_t st,
+                        bool bwd_only) {
   const TokenInfo& ti = F.ti;
   const slora_ffn_layer& L = F.L;
   const slora_ffn_grads& G = F.G;
@@ -413,7 +414,10 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd"));
 
-
+  TcGemm first;  // the context-row half of each paired launch
+  // bwd_only: the workspace still holds the forward state of a forward-only
+  // call with the same arguments (same carve-up): resume at the backward
+  if (!bwd_only) {
   SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt, eb.cnt,
                            eb.ncnt));
   // The small LoRA operand layouts run on the library's side stream, beside
@@ -476,7 +480,6 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   SLORA_TRY(join_side(st, side));
 
   // ---- forward (each context-row GEMM runs in one launch with its output-row twin)
-  TcGemm first;
   {  // gate|up, context rows, channels S: g, u, h = silu(g) u
     TcBuilder b(ctiles, nct, 0, 1, TC, kk, 1, EPI_SWIGLU_FWD);
     b.seg(mat(X, T, d, d), mat(WgS, kk, d, d), B_K, d, 1, mat(WuS, kk, d, d))
@@ -520,6 +523,7 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
         .out(out, nullptr, nullptr, d);
     SLORA_TRY(gemm_tc_pair(first, b.g, st));
   }
+  }  // forward
   if (!dOut) return SLORA_OK;  // forward only
 
   // ---- backward
@@ -618,8 +622,11 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
 // ---------------------------------------------------------------------- FFN
 slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
                      void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
-                     bool plan, cudaStream_t st) {
-  if (F.dt == kBF16) return ffn_run_tc(F, tok, X, dOut, out, dX, idx, idx_force, ar, plan, st);
+                     bool plan, cudaStream_t st, bool bwd_only) {
+  if (F.dt == kBF16)
+    return ffn_run_tc(F, tok, X, dOut, out, dX, idx, idx_force, ar, plan, st, bwd_only);
+  if (bwd_only)
+    SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "slora_ffn_bwd: the fp32 path has no separate backward");
   const TokenInfo& ti = F.ti;
   const slora_ffn_layer& L = F.L;
   const slora_ffn_grads& G = F.G;

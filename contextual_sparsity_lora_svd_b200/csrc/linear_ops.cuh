@@ -39,7 +39,7 @@ struct FfnDesc {
 
 slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,
                      void* out, void* dX, int32_t* idx, const int32_t* idx_force, Arena& ar,
-                     bool plan, cudaStream_t st);
+                     bool plan, cudaStream_t st, bool bwd_only = false);
 
 // Estimator (estimate + select) shared by slora_estimate_select and the FFN
 // call, in two steps so that a run path can take all of its workspace before

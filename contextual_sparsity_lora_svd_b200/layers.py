@@ -41,11 +41,13 @@ def lora_grad_shapes_ffn(d, d_ff, r):
 
 class _Call:
     """One library call with its argument list fixed (before ws, ws_bytes,
-    stream) and the objects that must stay alive while it is used."""
+    stream) and the objects that must stay alive while it is used.  A call
+    with `own_ws` (a device tensor) runs on that workspace instead of the
+    runner's shared one (state kept from one call to a later one)."""
 
-    def __init__(self, name, args, keep=()):
+    def __init__(self, name, args, keep=(), own_ws=None):
         self.fn = getattr(L.lib(), name)
-        self.name, self.args, self.keep = name, args, keep
+        self.name, self.args, self.keep, self.own_ws = name, args, keep, own_ws
 
     def need(self) -> int:
         need = L.c_sz(0)
@@ -53,6 +55,8 @@ class _Call:
         return int(need.value)
 
     def __call__(self, ws_ptr, ws_bytes, stream):
+        if self.own_ws is not None:
+            ws_ptr, ws_bytes = self.own_ws.data_ptr(), L.c_sz(self.own_ws.numel())
         L._check(self.name, self.fn(*self.args, ws_ptr, ctypes.byref(ws_bytes), stream))
 
 
@@ -60,7 +64,7 @@ class _Runner:
     calls: list
 
     def workspace_bytes(self) -> int:
-        return max([c.need() for c in self.calls] + [16])
+        return max([c.need() for c in self.calls if c.own_ws is None] + [16])
 
     def step(self, ws: torch.Tensor, stream=None):
         st = (stream or torch.cuda.current_stream()).cuda_stream
@@ -268,9 +272,9 @@ class DecoderStack(_Runner):
         linears; rotary packing of q, k; causal attention; h = x + o(attn);
         n2 = rms(h); FFN forward only (its own estimate + select);
         x' = h + ffn (fused into the next normalisation);
-      backward, last layer first: the FFN again with its forward channel set
-        (forward recomputed, then the sparse backward), the norm backward with
-        the residual, o backward, attention backward, rotary unpacking, q/k/v
+      backward, last layer first: the FFN's sparse backward from the state
+        its forward call left in the layer's own workspace, the norm backward
+        with the residual, o backward, attention backward, rotary unpacking, q/k/v
         backward, the norm backward summing the three branch gradients and the
         residual.
 
@@ -310,12 +314,12 @@ class DecoderStack(_Runner):
                            XAv=f32(T, r), XAo=f32(T, r), h=bf(T, d), n2=bf(T, d), r2=f32(T)))
         self.saved = sv
         # ---- scratch shared by the layers
-        a_out, f_out, f_re = bf(T, d), bf(T, d), bf(T, d)
+        a_out, f_out = bf(T, d), bf(T, d)
         dn2, dh, dxq, dxk, dxv = bf(T, d), bf(T, d), bf(T, d), bf(T, d), bf(T, d)
         dx_pp = [bf(T, d), bf(T, d)]
         dO_att = bf(T, nq)
         dQr, dKr, dV = f32(T, nq), f32(T, nkv), bf(T, nkv)
-        self._scratch = (a_out, f_out, f_re, dn2, dh, dxq, dxk, dxv, dx_pp, dO_att, dQr, dKr, dV)
+        self._scratch = (a_out, f_out, dn2, dh, dxq, dxk, dxv, dx_pp, dO_att, dQr, dKr, dV)
         # ---- gradients: one flat fp32 buffer, 16-byte aligned views
         shapes = []
         for nm, n, k in (("q", nq, d), ("k", nkv, d), ("v", nkv, d), ("o", d, nq)):
@@ -446,7 +450,6 @@ class DecoderStack(_Runner):
                                                      L.ptr(S_["n2"]), L.ptr(S_["r2"])]))
             sf = float(ffn_sparsity[l])
             fidx = torch.empty(d_ff, dtype=torch.int32, device="cuda")
-            fidx_re = torch.empty(d_ff, dtype=torch.int32, device="cuda")
             force = torch.arange(d_ff, dtype=torch.int32, device="cuda") if sf == 0.0 else None
             lay = L.ffn_layer_struct(d, d_ff, r_svd, r, s, w["Wg"], w["Wu"], w["Wd_t"], w["Ag"],
                                      w["Bg"], w["Au"], w["Bu"], w["Ad"], w["Bd"], w["Lg"],
@@ -455,15 +458,17 @@ class DecoderStack(_Runner):
             fa, fk = L.ffn_args(L.BF16, lay, batch, seq, ctx_len, sf, S_["n2"], None, f_out, None,
                                 None, fidx, force)
             ffn_f = _Call("slora_ffn_fwd_bwd", fa, fk + (lay, force))
-            ffn_f.need()
+            # the layer's FFN workspace keeps its forward state for the backward
+            ffn_ws = torch.empty(max(ffn_f.need(), 16), dtype=torch.uint8, device="cuda")
+            ffn_f.own_ws = ffn_ws
             kf = int(fk[2].value)
             self.idx_ffn.append(fidx)
             self.k_ffn.append(kf)
             calls.append(ffn_f)
             # backward of this layer (issued in reverse layer order below)
             self._structs += [lay, fgs]
-            bwd.append(dict(fgs=fgs, lay=lay, fidx=fidx, fidx_re=fidx_re, kf=kf, q=proj["q"],
-                            k=proj["k"], v_b=v_b, att_b=att_b, o_b=o_b, w=w, S=S_))
+            bwd.append(dict(fgs=fgs, lay=lay, fidx=fidx, kf=kf, sf=sf, force=force, ws=ffn_ws,
+                            q=proj["q"], k=proj["k"], v_b=v_b, att_b=att_b, o_b=o_b, w=w, S=S_))
         # -- the stack output: last residual + last FFN output
         calls.append(_Call("slora_rmsnorm_fwd", [L.BF16, T, d, L.c_f32(eps),
                                                  L.ptr(sv[-1]["h"]), L.ptr(f_out),
@@ -475,9 +480,11 @@ class DecoderStack(_Runner):
             B = bwd[l]
             S_, w = B["S"], B["w"]
             dx_next = dx_pp[(nl - 1 - l) % 2]
-            fa, fk = L.ffn_args(L.BF16, B["lay"], batch, seq, ctx_len, 0.0, S_["n2"], dx_cur,
-                                f_re, dn2, B["fgs"], B["fidx_re"], B["fidx"][:B["kf"]])
-            calls.append(_Call("slora_ffn_fwd_bwd", fa, fk + (B["fidx"],)))
+            # the FFN backward resumes from the state its forward left in the
+            # layer's workspace (same arguments as the forward call)
+            fa, fk = L.ffn_args(L.BF16, B["lay"], batch, seq, ctx_len, B["sf"], S_["n2"], dx_cur,
+                                f_out, dn2, B["fgs"], B["fidx"], B["force"])
+            calls.append(_Call("slora_ffn_bwd", fa, fk + (B["force"],), own_ws=B["ws"]))
             calls.append(_Call("slora_rmsnorm_bwd", [L.BF16, T, d, L.ptr(S_["h"]),
                                                      L.ptr(S_["r2"]), L.ptr(w["g2"]), L.ptr(dn2),
                                                      None, None, L.ptr(dx_cur), L.ptr(dh)]))

@@ -364,6 +364,23 @@ slora_status slora_ffn_fwd_bwd(slora_dtype dt, const slora_ffn_layer* layer,
                                slora_stream_t stream);
 
 /*
+ * slora_ffn_bwd — the backward half of slora_ffn_fwd_bwd, for callers that run
+ * a layer's forward earlier (a layer stack: every forward, then every
+ * backward) without recomputing it.  The previous call on this workspace must
+ * have been slora_ffn_fwd_bwd with dOut == NULL and the same dt, layer, tok,
+ * sparsity, X, out, idx_out, idx_force and k_force, and the workspace must be
+ * untouched since: it holds that forward's state (row maps, compacted weight
+ * slices, g, u, h and the LoRA projections).  dOut, dX and grads as in
+ * slora_ffn_fwd_bwd; out and idx_out are not written; the fp32 path returns
+ * SLORA_ERR_UNSUPPORTED.
+ */
+slora_status slora_ffn_bwd(slora_dtype dt, const slora_ffn_layer* layer, const slora_tokens* tok,
+                           double sparsity, const void* X, const void* dOut, void* out, void* dX,
+                           const slora_ffn_grads* grads, int32_t* idx_out, int32_t* k_out,
+                           const int32_t* idx_force, int32_t k_force, void* ws,
+                           size_t* ws_bytes, slora_stream_t stream);
+
+/*
  * slora_ffn_fwd_bwd_per_seq — slora_ffn_fwd_bwd with one channel set per
  * sequence instead of one per batch [ART §1: the channels are chosen per
  * input]: each sequence's context rows are scored and selected on their own

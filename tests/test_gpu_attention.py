@@ -188,3 +188,47 @@ def test_ffn_forward_only_equals_the_full_call(L):
             idxs.append(host(idx[:k]))
         assert np.array_equal(outs[0], outs[1])
         assert np.array_equal(idxs[0], idxs[1])
+
+
+def test_ffn_backward_half_equals_the_full_call(L):
+    """A forward-only call followed by slora_ffn_bwd on the same workspace
+    gives the full call's dX and LoRA gradients bit for bit."""
+    tok = synth.Tokens(2, 96, np.array([70, 50], np.int32))
+    case = synth.ffn_case(tok, d=128, d_ff=344, r_svd=8, r_lora=8, sparsity=0.5, bf16=True,
+                          workload=0, layer=8)
+    Ls, Us = {}, {}
+    for m, W in (("g", case.Wg.W), ("u", case.Wu.W)):
+        Ls[m], Us[m] = SO.svd_prepare(W, 8)
+    t = {k: _bf(getattr(case, k)) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    t.update(Wg=_bf(case.Wg.W), Wu=_bf(case.Wu.W), Wd_t=_bf(case.Wd.W.T.copy()))
+    f = {k: dev(v, torch.float32) for k, v in
+         (("Lg", Ls["g"]), ("Ug", Us["g"]), ("Lu", Ls["u"]), ("Uu", Us["u"]))}
+    layer = L.ffn_layer_struct(128, 344, 8, 8, 1.0, t["Wg"], t["Wu"], t["Wd_t"], t["Ag"], t["Bg"],
+                               t["Au"], t["Bu"], t["Ad"], t["Bd"], f["Lg"], f["Ug"], f["Lu"],
+                               f["Uu"])
+    X, dOut = _bf(case.X), _bf(case.dOut)
+    T = tok.T
+    shapes = [(8, 128), (344, 8), (8, 128), (344, 8), (8, 344), (128, 8)]
+    for force in (None, dev(np.arange(1, 344, 2), torch.int32)):
+        res = []
+        for split in (False, True):
+            out = torch.empty(T, 128, dtype=torch.bfloat16, device="cuda")
+            dX = torch.empty_like(out)
+            idx = torch.empty(344, dtype=torch.int32, device="cuda")
+            g = [torch.full(sh, float("nan"), device="cuda") for sh in shapes]
+            G = L.ffn_grads_struct(*g)
+            if split:
+                n = L.ffn_workspace_bytes(layer, tok.batch, tok.seq, tok.ctx_len, 0.5, X, out, idx,
+                                          idx_force=force)
+                ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+                L.slora_ffn_fwd_bwd(layer, tok.batch, tok.seq, tok.ctx_len, 0.5, X, None, out,
+                                    None, None, idx, idx_force=force, ws=ws)
+                L.slora_ffn_bwd(layer, tok.batch, tok.seq, tok.ctx_len, 0.5, X, dOut, out, dX, G,
+                                idx, ws, idx_force=force)
+            else:
+                L.slora_ffn_fwd_bwd(layer, tok.batch, tok.seq, tok.ctx_len, 0.5, X, dOut, out, dX,
+                                    G, idx, idx_force=force)
+            torch.cuda.synchronize()
+            res.append([host(out), host(dX)] + [host(x) for x in g])
+        for a, b in zip(*res):
+            assert np.array_equal(a, b)
