@@ -931,10 +931,121 @@ slora_status linear_bwd_tc(const LinearDesc& L, const slora_tokens* tok, const v
   sw.part = part;
   sw.rsplit = ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(std::max({T, k, n}))));
   sw.counters = rsp;
+  // The batched form (NONE, and OUT_ROWS with context and output rows): every
+  // rank operand known up front split in one launch, and the token-summed
+  // contractions (dA over X, dB over dY by row kind) in one launch; the
+  // context rows' dB part lands in SB and is added onto rows idx of dB.
+  const bool batched = (none && T > 0) || (outr && TC > 0 && TO > 0 && ni > 0);
+  auto rsbuf = [&](int64_t I) {
+    return static_cast<void*>(ar.take<__nv_bfloat16>(size_t(skinny_rsplit_elems(I))));
+  };
+  void* rsB0 = nullptr;  // B for the dYB rowdot(s): NONE: every row; OUT_ROWS: rows idx
+  void* rsB1 = nullptr;  // OUT_ROWS: B for the output rows
+  void* rsX0 = nullptr;  // XA: NONE every row; OUT_ROWS output rows
+  void* rsX1 = nullptr;  // OUT_ROWS: XA of the context rows
+  void* rsDY = nullptr;  // dYB (for dA)
+  float* SB = nullptr;
+  SkColJob bj[3];
+  int nbj = 0;
+  auto prepared = [&](void* rs) {
+    SkWork w = sw;
+    w.rsplit = rs;
+    w.prepared = true;
+    return w;
+  };
+  auto cjob = [&](const void* Y, int64_t ld, int64_t M, int64_t K, const SkR& Rr, void* rs_,
+                  float* o, int64_t ldo, int trans) {
+    SkColJob j;
+    j.Y = ykv(Y, ld); j.M = M; j.K = K; j.R = Rr; j.c = r; j.rs = rs_;
+    j.o.out = o; j.o.ldo = ldo; j.o.trans = trans; j.o.scale = s;
+    return j;
+  };
+  if (batched) {
+    rsB0 = rsbuf(none ? n : ni);
+    rsX0 = rsbuf(none ? T : TO);
+    rsDY = rsbuf(T);
+    if (outr) {
+      rsB1 = rsbuf(n);
+      rsX1 = rsbuf(TC);
+      SB = ar.take<float>(size_t(ni) * r);
+    }
+    const void* dYc0 = dYpad ? dYpad : dY_ctx;
+    const int64_t lddc0 = dYpad ? ldi : ni;
+    if (none) {
+      bj[nbj++] = cjob(X_ctx, k, T, k, rkv(dYB, kF32, r, 1), rsDY, dA, k, 1);
+      bj[nbj++] = cjob(dY_ctx, n, T, n, rkv(XA, kF32, r, 1), rsX0, dB, r, 0);
+    } else {
+      bj[nbj++] = cjob(X_ctx, k, T, k, rkv(dYB, kF32, r, 1), rsDY, dA, k, 1);
+      bj[nbj++] = cjob(dY_out, n, TO, n, rkv(XA, kF32, r, 1, out_rows), rsX0, dB, r, 0);
+      bj[nbj++] = cjob(dYc0, lddc0, TC, ni, rkv(XA, kF32, r, 1, ctx_rows), rsX1, SB, r, 0);
+    }
+  }
+  float* bpart = nullptr;
+  unsigned* bcnt = nullptr;
+  if (batched) {
+    bpart = ar.take<float>(size_t(coldot_batch_part_floats(bj, nbj)));
+    bcnt = ar.take<unsigned>(size_t(coldot_batch_counter_count(bj, nbj)));
+  }
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "workspace"));
 
-  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt));
+  SLORA_TRY(launch_rowmaps(tok, ti, ctx_rows, out_rows, st, ctiles, otiles, rsp, ncnt, bcnt,
+                           bcnt ? coldot_batch_counter_count(bj, nbj) : 0));
+  if (batched && none) {
+    const SkPrep jobs[2] = {{rkv(L.B, kBF16, r, 1), r, n, rsB0}, {rkv(XA, kF32, r, 1), r, T, rsX0}};
+    SLORA_TRY(prep_r_batch(jobs, 2, st));
+    SkRowOut o;
+    o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
+    SLORA_TRY(rowdot(ykv(dY_ctx, n), T, n, rkv(L.B, kBF16, r, 1), r, o, prepared(rsB0), st));
+    SLORA_TRY(make_plain_tiles(ptiles, T, st));
+    TcBuilder b(ptiles, (T + 127) / 128, 0, 0, T, k, 0, EPI_STORE);
+    b.seg(mat(dY_ctx, T, n, n), mat(L.W, n, k, k), B_MN, n)
+        .seg(mat(dYBb, T, r, lr), mat(L.A, r, k, k), B_MN, r)
+        .out(dX_ctx, nullptr, nullptr, k);
+    SLORA_TRY(gemm_tc(b.g, st));
+    const SkPrep jd = {rkv(dYB, kF32, r, 1), r, T, rsDY};
+    SLORA_TRY(prep_r_batch(&jd, 1, st));
+    return coldot_batch(bj, nbj, bpart, bcnt, st);
+  }
+  if (batched && outr) {
+    const void* dYc = dY_ctx;
+    int64_t lddc = ni;
+    if (dYpad) {
+      SLORA_TRY(gather_pad(dY_ctx, ni, nullptr, TC, ni, dYpad, ldi, st, TC));
+      dYc = dYpad;
+      lddc = ldi;
+    }
+    const SkPrep jobs[4] = {{rkv(L.B, kBF16, r, 1, L.idx, n), r, ni, rsB0},
+                            {rkv(L.B, kBF16, r, 1), r, n, rsB1},
+                            {rkv(XA, kF32, r, 1, out_rows), r, TO, rsX0},
+                            {rkv(XA, kF32, r, 1, ctx_rows), r, TC, rsX1}};
+    SLORA_TRY(prep_r_batch(jobs, 4, st));
+    SkRowOut oc;
+    oc.out1 = dYB; oc.ld1 = r; oc.map1 = ctx_rows; oc.out2 = dYBbC; oc.ld2 = lr; oc.s2 = s;
+    SLORA_TRY(rowdot(ykv(dYc, lddc), TC, ni, rkv(L.B, kBF16, r, 1, L.idx, n), r, oc,
+                     prepared(rsB0), st));
+    SkRowOut oo;
+    oo.out1 = dYB; oo.ld1 = r; oo.map1 = out_rows; oo.out2 = dYBbO; oo.ld2 = lr; oo.s2 = s;
+    SLORA_TRY(rowdot(ykv(dY_out, n), TO, n, rkv(L.B, kBF16, r, 1), r, oo, prepared(rsB1), st));
+    SLORA_TRY(gather_rows(L.W, k, L.idx, ni, k, WS, k, st, n));
+    {  // dX, context rows: dY_C W0[S] + s dYB_C A; output rows dense; one launch
+      TcBuilder bc(ctiles, nct, 1, 0, TC, k, 0, EPI_STORE);
+      bc.seg(mat(dYc, TC, ni, lddc), mat(WS, ni, k, k), B_MN, ni)
+          .seg(mat(dYBbC, TC, r, lr), mat(L.A, r, k, k), B_MN, r)
+          .out(dX_ctx, nullptr, nullptr, k);
+      TcBuilder b(otiles, nott, 1, 0, TO, k, 0, EPI_STORE);
+      b.seg(mat(dY_out, TO, n, n), mat(L.W, n, k, k), B_MN, n)
+          .seg(mat(dYBbO, TO, r, lr), mat(L.A, r, k, k), B_MN, r)
+          .out(dX_ctx, nullptr, nullptr, k);
+      SLORA_TRY(gemm_tc_pair(bc.g, b.g, st));
+    }
+    const SkPrep jd = {rkv(dYB, kF32, r, 1), r, T, rsDY};
+    SLORA_TRY(prep_r_batch(&jd, 1, st));
+    SLORA_TRY(coldot_batch(bj, nbj, bpart, bcnt, st));
+    ScatterAddJob sj;
+    sj.dst = dB; sj.ld_dst = r; sj.src = SB; sj.ld_src = r; sj.trans = 0;
+    return scatter_add_cols(&sj, 1, L.idx, ni, r, n, st);
+  }
   if (none) {
     SkRowOut o;
     o.out1 = dYB; o.ld1 = r; o.out2 = dYBb; o.ld2 = lr; o.s2 = s;
