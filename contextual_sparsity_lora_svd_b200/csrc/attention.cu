@@ -730,6 +730,7 @@ slora_status attention_fwd_run(const void* Q, const void* K, const void* V, cons
   p.sl2 = float(1.0 / std::sqrt(double(hd)) * 1.4426950408889634);
   const dim3 grid(p.nqb, H, ti.batch);
   LaunchScope ls(kAttention, 2.0 * causal_flops(ti, H, hd), st);
+  if (attention_fwd_tc_ok(Q, K, V, O, hd)) return attention_fwd_tc_run(Q, K, V, ti, H, KV, O, lse, st);
   if (hd == 128) {
     SLORA_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<128>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem<128>()));

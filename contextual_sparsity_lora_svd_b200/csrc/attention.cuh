@@ -20,6 +20,13 @@ slora_status rope_run(bool backward, const void* Y, const void* Yc, const void* 
 // bf16.  lse: [batch][H][seq] fp32 natural log-sum-exp of the scaled scores.
 slora_status attention_fwd_run(const void* Q, const void* K, const void* V, const TokenInfo& ti,
                                int H, int KV, int hd, void* O, float* lse, cudaStream_t st);
+// The tcgen05 forward (attention_tc.cu): head width 128, 16-byte aligned Q,
+// K, V, O; attention_fwd_run takes it whenever attention_fwd_tc_ok holds.
+bool attention_fwd_tc_ok(const void* Q, const void* K, const void* V, const void* O, int hd);
+slora_status attention_fwd_tc_run(const void* Q, const void* K, const void* V, const TokenInfo& ti,
+                                  int H, int KV, void* O, float* lse, cudaStream_t st);
+// Raised when a tcgen05 attention kernel's bounded wait ran out.
+slora_status attn_check_error(bool clear);
 // dQ [T x H hd] and dK [T x KV hd] fp32, dV [T x KV hd] bf16 (all written).
 slora_status attention_bwd_run(const void* Q, const void* K, const void* V, const void* O,
                                const float* lse, const void* dO, const TokenInfo& ti, int H,

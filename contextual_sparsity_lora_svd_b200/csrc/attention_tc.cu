@@ -1,0 +1,636 @@
+// Causal attention forward on the 5th-generation tensor cores (head width 128).
+//
+// Same result as attn_fwd_kernel (attention.cu): O = softmax(scale Q K^T,
+// causal within each sequence) V per query head, with grouped key/value heads,
+// and the natural-log log-sum-exp of every row's scaled scores; the P fed to
+// the P V product is the bf16 rounding of the fp32 probabilities, and the row
+// sums are taken before that rounding (SparseLoRA article, section 1: the
+// attention core between the sparse q/k projections and the o projection).
+//
+// One CTA per (128 query rows, query head, sequence), 320 threads:
+//   warps 0-7  softmax: query row r is tensor-memory lane r; warps w and
+//              w + 4 share rows 32 (w % 4) .. + 31, w taking key / output
+//              columns 0-63 and w + 4 columns 64-127.  Each reads its half row
+//              of S with tcgen05.ld, masks, swaps the half maxima with its
+//              partner through shared memory, exponentiates, and writes its
+//              half row of P (bf16 pairs) back into tensor memory with
+//              tcgen05.st; at the end it reads its half row of O, divides by
+//              the row sum and stores it;
+//   warp 8     TMA producer: the Q tile once, then the 128-key K and V tiles
+//              through two stages (a K stage is refilled once its S is
+//              computed, a V stage once its P V is done);
+//   warp 9     MMA issuer (one thread): S_j = Q K_j^T into one of two S
+//              buffers, and O += P_j V_j with P_j read from tensor memory as
+//              the A operand and V read MN-major from shared memory.
+// Tensor memory (512 columns): S at 0 and 128, O at 256, P at 384 and 448
+// (128 keys as 64 columns of bf16 pairs).  S_{j+1} is computed while the
+// softmax warps work on S_j; P is double-buffered, so softmax j writes P_j
+// while P_{j-1} V_{j-1} may still run, and waits only for P_{j-2} V_{j-2}
+// (or for P_{j-1} V_{j-1} when it has to rescale O).  Online softmax with a
+// lazily moved reference: a row keeps the maximum m it started scaling with
+// until a tile's maximum exceeds it by more than 8 (in log2 units); only then
+// are its O row and sum rescaled by 2^(m_old - m_new).  Between rescales
+// every probability is 2^(s - m) <= 2^8, so nothing overflows, and the final
+// O / l and lse = (m + log2 l) ln 2 are the same quantities as with a
+// reference that moves every tile.
+//
+// Every mbarrier wait is bounded; a wait that gives up raises g_attn_error
+// (read by attn_check_error) and the CTA winds down: the producer waits (again
+// bounded) for its copies in flight, the MMA thread for its MMAs, and the
+// tensor memory is released.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "attention.cuh"
+
+namespace slora {
+
+__device__ int g_attn_error = 0;
+
+namespace {
+
+constexpr int kRows = 128;                 // query rows per CTA, keys per tile
+constexpr int kHD = 128;                   // head width
+constexpr int kPanel = 128 * 128;          // bytes: 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr int kTile = 2 * kPanel;          // 128 x 128 bf16
+constexpr int kOffQ = 0;
+constexpr int kOffK = kTile;               // 2 stages
+constexpr int kOffV = 3 * kTile;           // 2 stages
+constexpr int kOffBar = 5 * kTile;         // 18 mbarriers, the tensor-memory address, a flag
+constexpr int kOffX = kOffBar + 256;       // row-block maxima: [tile parity][half][row] fp32
+constexpr int kOffL = kOffX + 2048;        // row-sum halves: [half][row] fp32
+constexpr int kSmem = kOffL + 1024 + 1024; // + 1024-byte alignment slack
+constexpr int kSoftWarps = 8;              // two per row block (one per 64-column half)
+constexpr int kThreadsTc = (kSoftWarps + 2) * 32;
+constexpr int kHalf = 64;                  // columns per softmax thread
+constexpr uint32_t kTmemCols = 512;        // S buffers at 0 and 128, O at 256, P at 384 and 448
+constexpr uint32_t kColP = 384;            // P: 128 keys as 64 columns of bf16 pairs, two buffers
+constexpr float kLn2f = 0.6931471805599453f;
+constexpr float kMasked = -1.0e30f;
+constexpr float kLazy = 8.0f;              // rescale when the maximum rises by more
+constexpr long long kWaitBudget = 2000000000LL;  // clock cycles
+
+// kind::f16 instruction descriptor: fp32 D, bf16 A and B, A K-major, B K-major
+// (b_mn = 0) or MN-major (1), M = 128, N = 128.
+constexpr uint32_t idesc(int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) | (uint32_t(128 >> 3) << 17) |
+         (uint32_t(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 version bits).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// Bounded wait on the phase of parity `par`; false (and the error flag) when
+// the budget runs out or another role of the CTA already gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t par, volatile int* abort) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(par)
+        : "memory");
+    if (ok) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudget) {
+      *abort = 1;
+      atomicExch(&g_attn_error, 1);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* m, uint32_t bar, int x,
+                                         int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(id), "r"(acc)
+      : "memory");
+}
+// A operand (M rows in lanes, two bf16 per 32-bit column) in tensor memory.
+__device__ __forceinline__ void mma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 32 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tst32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tst_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+struct TcFwdP {
+  CUtensorMap mq, mk, mv;   // Q [T x H 128], K and V [T x KV 128]; boxes 64 x 128, 128-byte swizzle
+  __nv_bfloat16* O;         // [T x H 128]
+  float* lse;               // [batch][H][seq]
+  int seq, H, KV, batch, nqb;
+  int items;                // nqb * H * batch work items (query tile, head, sequence)
+  float sl2;                // softmax scale * log2(e)
+};
+
+// Work item `it` (longest causal rows first): query tile qb, head h, sequence b.
+// CTA c takes, in round k, item k G + c (k even) or k G + G - 1 - c (k odd):
+// the alternating direction evens out the causal tile counts across CTAs.
+__device__ __forceinline__ int item_at(int k, int G) {
+  return k * G + ((k & 1) ? G - 1 - int(blockIdx.x) : int(blockIdx.x));
+}
+struct Item {
+  int qb, h, b;
+};
+__device__ __forceinline__ Item item_of(const TcFwdP& p, int it) {
+  const int hb = p.H * p.batch;
+  Item x;
+  x.qb = p.nqb - 1 - it / hb;
+  x.h = (it % hb) % p.H;
+  x.b = (it % hb) / p.H;
+  return x;
+}
+
+}  // namespace
+
+namespace {
+
+// Waits for the phase of parity `par` with its own budget, ignoring the
+// abort flag: used to let copies and MMAs already issued finish before the
+// CTA releases its memory.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t par) {
+  volatile int never = 0;
+  if (!mbar_wait(bar, par, &never)) atomicExch(&g_attn_error, 1);
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid_constant__ TcFwdP p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;  // the swizzle pattern repeats every 1024 bytes
+  unsigned char* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
+  const uint32_t bar = base + kOffBar;
+  // mbarriers; those with two copies are indexed by buffer / stage (tile t uses t % 2)
+  const uint32_t q_full = bar, q_empty = bar + 8, k_full = bar + 16, v_full = bar + 32,
+                 k_empty = bar + 48, v_empty = bar + 64, s_full = bar + 80, s_free = bar + 96,
+                 p_full = bar + 112, pv_done = bar + 128, o_empty = bar + 144,
+                 mma_done = bar + 152;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kOffBar + 192);
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + 200);
+  float* xmax = reinterpret_cast<float*>(gbase + kOffX);  // [tile parity][half][row]
+  float* lsum = reinterpret_cast<float*>(gbase + kOffL);  // [half][row]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = int(gridDim.x);
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 32) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
+      mbar_init(s_full + 8 * s, 1);
+      mbar_init(s_free + 8 * s, kSoftWarps);
+      mbar_init(p_full + 8 * s, kSoftWarps);
+      mbar_init(pv_done + 8 * s, 1);
+    }
+    mbar_init(o_empty, kSoftWarps);
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == kSoftWarps) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int t = 0, nq = 0, nk = 0, nv = 0;
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        const int it = item_at(n, G);
+        if (it >= p.items) break;
+        const Item x = item_of(p, it);
+        const int row0 = x.b * p.seq, g = x.h / (p.H / p.KV);
+        // Q_n once every S of item n - 1 is computed
+        if (n >= 1 && !mbar_wait(q_empty, uint32_t((n - 1) & 1), abort)) break;
+        mbar_expect_tx(q_full, kTile);
+        tma_load(sQ, &p.mq, q_full, x.h * kHD, row0 + x.qb * kRows);
+        tma_load(sQ + kPanel, &p.mq, q_full, x.h * kHD + 64, row0 + x.qb * kRows);
+        nq = n + 1;
+        for (int j = 0; j <= x.qb; ++j, ++t) {
+          const int s = t & 1;
+          const uint32_t par = uint32_t(((t - 2) >> 1) & 1);
+          const int y = row0 + j * kRows;
+          // K_t once S_{t-2} is computed, V_t once P_{t-2} V_{t-2} is done
+          if (t >= 2 && !mbar_wait(k_empty + 8 * s, par, abort)) { ok = false; break; }
+          const uint32_t kb = sK + uint32_t(s * kTile), vb = sV + uint32_t(s * kTile);
+          mbar_expect_tx(k_full + 8 * s, kTile);
+          tma_load(kb, &p.mk, k_full + 8 * s, g * kHD, y);
+          tma_load(kb + kPanel, &p.mk, k_full + 8 * s, g * kHD + 64, y);
+          nk = t + 1;
+          if (t >= 2 && !mbar_wait(v_empty + 8 * s, par, abort)) { ok = false; break; }
+          mbar_expect_tx(v_full + 8 * s, kTile);
+          tma_load(vb, &p.mv, v_full + 8 * s, g * kHD, y);
+          tma_load(vb + kPanel, &p.mv, v_full + 8 * s, g * kHD + 64, y);
+          nv = t + 1;
+        }
+      }
+      // the copies issued last into each buffer have landed before the CTA
+      // can release its shared memory (on the normal path they were consumed)
+      if (nq >= 1) mbar_drain(q_full, uint32_t((nq - 1) & 1));
+      for (int u = ::max(0, nk - 2); u < nk; ++u)
+        mbar_drain(k_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+      for (int u = ::max(0, nv - 2); u < nv; ++u)
+        mbar_drain(v_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+    }
+    __syncwarp();
+  } else if (warp == kSoftWarps + 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int t = 0;
+      // P V of the previous tile, issued after the next tile's S: its tile
+      // index, whether it opens an item, and the item's ordinal
+      int pv_t = -1, pv_n = 0;
+      bool pv_first = false;
+      auto issue_pv = [&]() -> bool {
+        const int sp = pv_t & 1;
+        if (!mbar_wait(p_full + 8 * sp, uint32_t((pv_t >> 1) & 1), abort)) return false;
+        if (!mbar_wait(v_full + 8 * sp, uint32_t((pv_t >> 1) & 1), abort)) return false;
+        // the first P V of an item overwrites O: the previous item's O is read
+        if (pv_first && pv_n >= 1 && !mbar_wait(o_empty, uint32_t((pv_n - 1) & 1), abort))
+          return false;
+        fence_after();
+        const uint32_t vt = sV + uint32_t(sp * kTile);
+        const uint32_t pa = tmem + kColP + uint32_t(sp * 64);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          mma_ta(tmem + 2u * kRows, pa + uint32_t(kk * 8),
+                 sdesc(vt + uint32_t(kk * 2048), kPanel, 1024), idesc(1),
+                 (!pv_first || kk > 0) ? 1u : 0u);
+        commit(pv_done + 8 * sp);
+        commit(v_empty + 8 * sp);
+        return true;
+      };
+      for (int n = 0; ok; ++n) {
+        const int it = item_at(n, G);
+        if (it >= p.items) break;
+        const Item x = item_of(p, it);
+        // the previous item's last P V goes first: its epilogue waits on it,
+        // while this item's S waits for its Q and K to land
+        if (pv_t >= 0) {
+          if (!issue_pv()) { ok = false; break; }
+          pv_t = -1;
+        }
+        if (!mbar_wait(q_full, uint32_t(n & 1), abort)) { ok = false; break; }
+        for (int j = 0; j <= x.qb; ++j, ++t) {
+          const int s = t & 1;
+          // S_t = Q K_t^T into S buffer t % 2
+          if (!mbar_wait(k_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
+              (t >= 2 && !mbar_wait(s_free + 8 * s, uint32_t(((t - 2) >> 1) & 1), abort))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t d = tmem + uint32_t(s * kRows);
+          const uint32_t kt = sK + uint32_t(s * kTile);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mma(d, sdesc(sQ + off, 16, 1024), sdesc(kt + off, 16, 1024), idesc(0),
+                kk > 0 ? 1u : 0u);
+          }
+          commit(s_full + 8 * s);
+          commit(k_empty + 8 * s);
+          if (j == x.qb) commit(q_empty);  // every S of this item issued
+          if (pv_t >= 0 && !issue_pv()) { ok = false; break; }
+          pv_t = t;
+          pv_n = n;
+          pv_first = j == 0;
+        }
+      }
+      if (ok && pv_t >= 0) issue_pv();
+      // every MMA issued has completed before the tensor memory is released
+      commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ softmax
+    // warp w: rows 32 (w % 4) .. + 31 (its tensor-memory lanes), key / output
+    // columns 64 (w / 4) .. + 63; the two warps of a row block share each
+    // tile's maximum through shared memory (named barrier 1 + w % 4).  A wait
+    // that gives up turns this warp's `ok` off (warp-uniform, since the
+    // tensor-memory accesses are warp-collective); the loops still run to
+    // their end so that both warps of a row block meet at every pair barrier,
+    // the waits after an abort returning at once.
+    const int lq = warp & 3, hf = warp >> 2;
+    const int r = lq * 32 + lane;
+    const uint32_t lbase = tmem + (uint32_t(lq * 32) << 16);
+    const uint32_t pair_bar = uint32_t(1 + lq);
+    bool ok = true;
+    int t = 0;
+    for (int n = 0;; ++n) {
+      const int it = item_at(n, G);
+      if (it >= p.items) break;
+      const Item x = item_of(p, it);
+      const int row0 = x.b * p.seq;
+      const int qi = x.qb * kRows + r;
+      float m = kMasked, l = 0.f;
+      for (int j = 0; j <= x.qb; ++j, ++t) {
+        const int s = t & 1;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(s_full + 8 * s, uint32_t((t >> 1) & 1), abort));
+        uint32_t sv[kHalf];
+        float mh = kMasked;
+        if (ok) {
+          fence_after();
+          tld32(lbase + uint32_t(s * kRows + hf * kHalf), sv);
+          tld32(lbase + uint32_t(s * kRows + hf * kHalf + 32), sv + 32);
+          tld_wait();
+          fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free + 8 * s);
+          // maximum over the raw scores (the scale is positive); the last
+          // tile holds the keys past this row (causal) and past the sequence,
+          // set to a huge negative raw score.  Eight partial maxima and sums
+          // keep the dependency chains short.
+          float mx[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx[e] = kMasked;
+          if (j == x.qb) {
+            const int lim = ::min(qi, p.seq - 1) - j * kRows - hf * kHalf;  // last live column
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) {
+              if (i > lim) sv[i] = __float_as_uint(kMasked);
+              mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < kHalf; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sv[i]));
+          }
+          mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        }
+        xmax[(s * 2 + hf) * kRows + r] = mh;
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        if (!ok) continue;
+        const float mt = fmaxf(mh, xmax[(s * 2 + (hf ^ 1)) * kRows + r]) * p.sl2;
+        float c = 1.f;
+        bool resc = false;
+        if (j == 0) {
+          m = mt;
+        } else if (mt > m + kLazy) {
+          c = ex2(m - mt);
+          m = mt;
+          resc = true;
+        }
+        const float nm = -m;
+        float sm[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sm[e] = 0.f;
+        uint32_t pk[kHalf / 2];
+#pragma unroll
+        for (int i = 0; i < kHalf / 2; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), p.sl2, nm));
+          const float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), p.sl2, nm));
+          sm[(2 * i) & 7] += p0;
+          sm[(2 * i + 1) & 7] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+        l = l * c + rs;  // this half's share of the row sum
+        // P_t goes to tensor-memory buffer t % 2, free once P_{t-2} V_{t-2}
+        // is done; O is rescaled only after P_{t-1} V_{t-1} is done (MMAs
+        // complete in order, so that covers P_{t-2} V_{t-2} too)
+        if (__any_sync(0xffffffffu, resc)) {
+          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + 8 * ((t - 1) & 1),
+                                                 uint32_t(((t - 1) >> 1) & 1), abort));
+          if (!ok) continue;
+          fence_after();
+#pragma unroll
+          for (int q = 0; q < kHalf / 32; ++q) {
+            uint32_t o[32];
+            const uint32_t ta = lbase + uint32_t(2 * kRows + hf * kHalf + 32 * q);
+            tld32(ta, o);
+            tld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * c);
+            tst32(ta, o);
+          }
+        } else if (t >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(pv_done + 8 * s, uint32_t(((t - 2) >> 1) & 1), abort));
+          if (!ok) continue;
+          fence_after();
+        }
+        // this half of row r of P: keys 64 hf .. + 63 as 32 columns of bf16 pairs
+        tst32(lbase + kColP + uint32_t(s * 64 + hf * 32), pk);
+        tst_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + 8 * s);
+      }
+      // both halves of the row sum, added in a fixed order
+      lsum[hf * kRows + r] = l;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      const float lt = lsum[r] + lsum[kRows + r];
+      const int tl = t - 1;  // the item's last tile
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(pv_done + 8 * (tl & 1),
+                                                   uint32_t((tl >> 1) & 1), abort));
+      if (ok) {
+        fence_after();
+        uint32_t o[kHalf];
+        tld32(lbase + uint32_t(2 * kRows + hf * kHalf), o);
+        tld32(lbase + uint32_t(2 * kRows + hf * kHalf + 32), o + 32);
+        tld_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_empty);  // the next item's P V may overwrite O
+        if (qi < p.seq) {
+          const float inv = 1.f / lt;
+          uint4* dst = reinterpret_cast<uint4*>(p.O + (int64_t(row0) + qi) * (int64_t(p.H) * kHD) +
+                                                x.h * kHD + hf * kHalf);
+#pragma unroll
+          for (int v = 0; v < kHalf / 8; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+            dst[v] = w;
+          }
+          if (hf == 0) p.lse[(int64_t(x.b) * p.H + x.h) * p.seq + qi] = (m + log2f(lt)) * kLn2f;
+        }
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ----------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
+std::once_flag g_enc_once;
+
+slora_status encode_rows(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+  std::call_once(g_enc_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_enc) SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  cuuint32_t box[2] = {64, cuuint32_t(kRows)};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = g_enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    SLORA_FAIL(SLORA_ERR_CUDA, "attention: cuTensorMapEncodeTiled failed (%d) rows=%lld cols=%lld",
+               int(r), (long long)rows, (long long)cols);
+  return SLORA_OK;
+}
+
+}  // namespace
+
+bool attention_fwd_tc_ok(const void* Q, const void* K, const void* V, const void* O, int hd) {
+  return hd == kHD && aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O);
+}
+
+slora_status attention_fwd_tc_run(const void* Q, const void* K, const void* V, const TokenInfo& ti,
+                                  int H, int KV, void* O, float* lse, cudaStream_t st) {
+  if (!attention_fwd_tc_ok(Q, K, V, O, kHD))
+    SLORA_FAIL(SLORA_ERR_ALIGN, "attention: Q, K, V and O must be 16-byte aligned");
+  TcFwdP p;
+  SLORA_TRY(encode_rows(&p.mq, Q, ti.T, int64_t(H) * kHD));
+  SLORA_TRY(encode_rows(&p.mk, K, ti.T, int64_t(KV) * kHD));
+  SLORA_TRY(encode_rows(&p.mv, V, ti.T, int64_t(KV) * kHD));
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.seq = ti.seq; p.H = H; p.KV = KV;
+  p.nqb = (ti.seq + kRows - 1) / kRows;
+  p.batch = ti.batch;
+  p.items = p.nqb * H * ti.batch;
+  p.sl2 = float(1.0 / std::sqrt(double(kHD)) * 1.4426950408889634);
+  SLORA_CUDA(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kSmem));
+  // persistent: one CTA per SM (the shared memory admits no second one)
+  const dim3 grid(unsigned(std::min(p.items, num_sms())));
+  attn_fwd_tc_kernel<<<grid, kThreadsTc, kSmem, st>>>(p);
+  SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+slora_status attn_check_error(bool clear) {
+  int v = 0;
+  SLORA_CUDA(cudaMemcpyFromSymbol(&v, g_attn_error, sizeof(int)));
+  if (clear && v) {
+    int z = 0;
+    SLORA_CUDA(cudaMemcpyToSymbol(g_attn_error, &z, sizeof(int)));
+  }
+  if (v) SLORA_FAIL(SLORA_ERR_TIMEOUT, "attention: a tensor-core wait ran out of its budget");
+  return SLORA_OK;
+}
+
+}  // namespace slora

@@ -2,6 +2,7 @@
 #include <mutex>
 #include <vector>
 
+#include "attention.cuh"
 #include "common.cuh"
 #include "estimator.cuh"
 #include "gemm_tc.cuh"
@@ -249,10 +250,13 @@ extern "C" slora_status slora_device_error(int clear) {
   const slora_status c = skinny_check_error(clear != 0);
   const std::string third = c != SLORA_OK ? g_error : std::string();
   const slora_status d = est_check_error(clear != 0);
+  const std::string fourth = d != SLORA_OK ? g_error : std::string();
+  const slora_status e = attn_check_error(clear != 0);
   if (a != SLORA_OK) g_error = first;
   else if (b != SLORA_OK) g_error = second;
   else if (c != SLORA_OK) g_error = third;
-  return a != SLORA_OK ? a : (b != SLORA_OK ? b : (c != SLORA_OK ? c : d));
+  else if (d != SLORA_OK) g_error = fourth;
+  return a != SLORA_OK ? a : (b != SLORA_OK ? b : (c != SLORA_OK ? c : (d != SLORA_OK ? d : e)));
 }
 
 extern "C" slora_status slora_set_wait_budget(int64_t cycles) {

@@ -1,6 +1,6 @@
 """GPU parity of the estimator and top-k kernels (through the C ABI) with the
 CPU oracle: every rank template of the activation-norm score kernel, ragged
-and empty context sets, score vectors beyond the fused select, the Gram-form
+and empty context sets, long score lists, the Gram-form
 criteria (QK-norm, rotate-half pairs, per-head L2, Gram FFN score), exact
 tie-breaking, bit-reproducibility, and the offline prepare at the benchmark's
 own weight shapes.  Scores are compared at relative Frobenius 1e-5 (fp32
@@ -69,8 +69,8 @@ def test_ffn_activation_score_all_rank_templates(L, r):
 
 @pytest.mark.parametrize("s", [0.0, 0.3, 0.7, 0.99])
 def test_ffn_activation_score_long_vector_standalone_select(L, s):
-    """d_ff = 20000 channels exceeds the fused in-kernel select (16384), so the
-    standalone top-k kernel runs; few context tokens keep the oracle quick."""
+    """d_ff = 20000 channels (the top-k block with 64 register rows per
+    thread); few context tokens keep the oracle quick."""
     tok = _tok(2, 40, [30, 25])
     d, d_ff, r = 32, 20000, 8
     rg = synth.rng(810)
@@ -186,6 +186,47 @@ def test_l2_norm_criterion(L, heads, kv, s):
         check_selection(vg, iv[g * k:(g + 1) * k] - g * hd, so[g], k, f"l2 value head {g}")
         for h in range(g * grp, (g + 1) * grp):
             assert np.array_equal(gi[h * k:(h + 1) * k] - h * hd, vg)
+
+
+@pytest.mark.parametrize("n", [1025, 3000, 11008, 16384, 16385, 32768])
+@pytest.mark.parametrize("distinct", [7, 0])
+def test_long_list_select_is_the_exact_top_k_of_its_scores(L, n, distinct):
+    """Selection from one long score list (every register-row template of the
+    top-k block): the kept set must be exactly the top-k of the GPU's own
+    scores with ties to the lower index.  With `distinct` > 0 every channel's
+    factor rows come from that many base rows, so the scores take only that
+    many values and tie bit for bit (same rows, same arithmetic), thousands
+    of keys equal to the threshold spread over all rows; 0 draws every row."""
+    tok = _tok(1, 48, [40])
+    d, r = 32, 4
+    rg = synth.rng(880 + n + distinct)
+    X = synth.round_bf16(rg.standard_normal((tok.T, d)))
+    Lg, Lu = rg.standard_normal((d, r)), rg.standard_normal((d, r))
+    if distinct:
+        pick = rg.integers(0, distinct, size=n)
+        Ug = rg.standard_normal((distinct, r))[pick]
+        Uu = rg.standard_normal((distinct, r))[pick]
+    else:
+        Ug, Uu = rg.standard_normal((n, r)), rg.standard_normal((n, r))
+    for s in (0.01, 0.5, 0.93):
+        k, gi, gs = _run(L, L.CRIT_FFN_GRAM, X, tok, Lg, Ug, Lu, Uu, r, s, n, n)
+        assert k == O.keep_count(n, s)
+        assert gi[:k].tolist() == O.topk_select(gs.astype(np.float64), k).tolist(), \
+            f"n={n} s={s}"
+
+
+def test_long_list_select_all_scores_equal(L):
+    """No context token: all 11008 scores are 0 and the lowest k indices are
+    kept (the top-k's all-keys-equal path)."""
+    tok = _tok(2, 16, [0, 0])
+    d, n, r = 32, 11008, 4
+    rg = synth.rng(890)
+    X = synth.round_bf16(rg.standard_normal((tok.T, d)))
+    Lg, Lu = rg.standard_normal((d, r)), rg.standard_normal((d, r))
+    Ug, Uu = rg.standard_normal((n, r)), rg.standard_normal((n, r))
+    k, gi, gs = _run(L, L.CRIT_FFN, X, tok, Lg, Ug, Lu, Uu, r, 0.3, n, n)
+    assert np.all(gs == 0.0)
+    assert gi[:k].tolist() == list(range(k))
 
 
 def test_exact_ties_go_to_the_lower_index(L):
