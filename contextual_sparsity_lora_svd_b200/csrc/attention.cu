@@ -751,7 +751,8 @@ slora_status attention_bwd_run(const void* Q, const void* K, const void* V, cons
   float* D = ar.take<float>(size_t(ti.T) * H);
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "attention_bwd"));
-  SLORA_CUDA(cudaMemsetAsync(dQ, 0, size_t(ti.T) * H * hd * sizeof(float), st));
+  const bool tc = attention_bwd_tc_ok(Q, K, V, dO, dQ, dK, dV, hd);
+  if (!tc) SLORA_CUDA(cudaMemsetAsync(dQ, 0, size_t(ti.T) * H * hd * sizeof(float), st));
   {
     LaunchScope ls(kElementwise, double(ti.T) * H * hd * 4, st);
     const int64_t thr = ti.T * H * 32;
@@ -765,6 +766,9 @@ slora_status attention_bwd_run(const void* Q, const void* K, const void* V, cons
           ti.seq, D);
     SLORA_CHECK_LAUNCH();
   }
+  if (tc)
+    return attention_bwd_tc_run(Q, K, V, dO, lse, D, ti, H, KV, dQ, dK, dV,
+                                causal_flops(ti, H, hd), st);
   AttnBwdP p;
   p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.K = static_cast<const __nv_bfloat16*>(K);

@@ -25,6 +25,16 @@ slora_status attention_fwd_run(const void* Q, const void* K, const void* V, cons
 bool attention_fwd_tc_ok(const void* Q, const void* K, const void* V, const void* O, int hd);
 slora_status attention_fwd_tc_run(const void* Q, const void* K, const void* V, const TokenInfo& ti,
                                   int H, int KV, void* O, float* lse, cudaStream_t st);
+// The tcgen05 backward (attention_tc.cu): a dK/dV kernel and a dQ kernel,
+// each output row written once (dQ needs no zeroing); D = rowsum(dO * O)
+// [batch][H][seq] computed beforehand.  attention_bwd_run takes it whenever
+// attention_bwd_tc_ok holds.
+bool attention_bwd_tc_ok(const void* Q, const void* K, const void* V, const void* dO,
+                         const void* dQ, const void* dK, const void* dV, int hd);
+slora_status attention_bwd_tc_run(const void* Q, const void* K, const void* V, const void* dO,
+                                  const float* lse, const float* D, const TokenInfo& ti, int H,
+                                  int KV, float* dQ, float* dK, void* dV, double flops_per_product,
+                                  cudaStream_t st);
 // Raised when a tcgen05 attention kernel's bounded wait ran out.
 slora_status attn_check_error(bool clear);
 // dQ [T x H hd] and dK [T x KV hd] fp32, dV [T x KV hd] bf16 (all written).

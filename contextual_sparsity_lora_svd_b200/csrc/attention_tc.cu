@@ -564,6 +564,583 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
   }
 }
 
+// ----------------------------------------------------------------- backward
+// The backward as two persistent kernels, no atomics (each output row is
+// written once):
+//   attn_bwd_dq_tc_kernel   per (query tile, head, sequence): for each key
+//       tile j <= the query tile, S = Q K_j^T and dP = dO V_j^T into tensor
+//       memory; the softmax warps form P = 2^(S scale log2e - lse log2e)
+//       (causal) and dS = P (dP - D) and write dS (bf16 pairs) back into
+//       tensor memory, double-buffered; dQ += dS K_j with dS as the
+//       tensor-memory A operand and K_j MN-major.  dQ = scale dQ, fp32.
+//   attn_bwd_dkv_tc_kernel  per (key block, key/value head, sequence): K
+//       and V stay in shared memory; for every query head of the group and
+//       query tile at or after the block, S^T = K Q^T and dP^T = V dO^T; the
+//       softmax warps (key rows) form P^T and dS^T and write them (bf16
+//       pairs) over the half rows of S^T and dP^T they have read; dV +=
+//       P^T dO and dK += dS^T Q (Q and dO MN-major).  dK = scale dK (fp32),
+//       dV bf16.
+struct TcBwdP {
+  CUtensorMap mq, mk, mv, mdo;  // Q, dO [T x H 128]; K, V [T x KV 128]; boxes 64 x 128
+  const float* lse;             // [batch][H][seq], natural log
+  const float* D;               // [batch][H][seq], rowsum(dO * O)
+  float* dQ;                    // [T x H 128]
+  float* dK;                    // [T x KV 128]
+  __nv_bfloat16* dV;            // [T x KV 128]
+  int seq, H, KV, batch, nqb;
+  int items_q, items_k;         // nqb H batch, nqb KV batch
+  float sl2, scale;
+};
+
+constexpr float kLog2ef = 1.4426950408889634f;
+
+// dQ kernel: Q and dO at 0 and 32 KB, K and V stages from 64 KB; tensor
+// memory S 0, dP 128, dQ 256, dS at 384 and 448.
+constexpr int kQOffQ = 0, kQOffO = kTile, kQOffK = 2 * kTile, kQOffV = 4 * kTile;
+constexpr int kQOffBar = 6 * kTile;
+constexpr int kQSmem = kQOffBar + 256 + 1024;
+constexpr uint32_t kColDP = 128, kColDQ = 256, kColDS = 384;
+
+__global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __grid_constant__ TcBwdP p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + kQOffQ, sO = base + kQOffO, sK = base + kQOffK, sV = base + kQOffV;
+  const uint32_t bar = base + kQOffBar;
+  const uint32_t qo_full = bar, qo_empty = bar + 8, k_full = bar + 16, v_full = bar + 32,
+                 k_empty = bar + 48, v_empty = bar + 64, s_full = bar + 80, s_free = bar + 88,
+                 p_full = bar + 96, dq_done = bar + 112, dq_empty = bar + 128,
+                 mma_done = bar + 136;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kQOffBar + 192);
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kQOffBar + 200);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = int(gridDim.x);
+  TcFwdP ip;  // item decoding only
+  ip.H = p.H; ip.batch = p.batch; ip.nqb = p.nqb;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 32) {
+    mbar_init(qo_full, 1);
+    mbar_init(qo_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(v_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
+      mbar_init(v_empty + 8 * s, 1);
+      mbar_init(p_full + 8 * s, kSoftWarps);
+      mbar_init(dq_done + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftWarps);
+    mbar_init(dq_empty, kSoftWarps);
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == kSoftWarps) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int t = 0, nq = 0, nk = 0, nv = 0;
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        const int it = item_at(n, G);
+        if (it >= p.items_q) break;
+        const Item x = item_of(ip, it);
+        const int row0 = x.b * p.seq, g = x.h / (p.H / p.KV);
+        const int yq = row0 + x.qb * kRows;
+        if (n >= 1 && !mbar_wait(qo_empty, uint32_t((n - 1) & 1), abort)) break;
+        mbar_expect_tx(qo_full, 2 * kTile);
+        tma_load(sQ, &p.mq, qo_full, x.h * kHD, yq);
+        tma_load(sQ + kPanel, &p.mq, qo_full, x.h * kHD + 64, yq);
+        tma_load(sO, &p.mdo, qo_full, x.h * kHD, yq);
+        tma_load(sO + kPanel, &p.mdo, qo_full, x.h * kHD + 64, yq);
+        nq = n + 1;
+        for (int j = 0; j <= x.qb; ++j, ++t) {
+          const int s = t & 1;
+          const uint32_t par = uint32_t(((t - 2) >> 1) & 1);
+          const int y = row0 + j * kRows;
+          // K_t once dQ += dS_{t-2} K_{t-2} is done, V_t once dP_{t-2} is
+          if (t >= 2 && !mbar_wait(v_empty + 8 * s, par, abort)) { ok = false; break; }
+          const uint32_t kb = sK + uint32_t(s * kTile), vb = sV + uint32_t(s * kTile);
+          mbar_expect_tx(v_full + 8 * s, kTile);
+          tma_load(vb, &p.mv, v_full + 8 * s, g * kHD, y);
+          tma_load(vb + kPanel, &p.mv, v_full + 8 * s, g * kHD + 64, y);
+          nv = t + 1;
+          if (t >= 2 && !mbar_wait(k_empty + 8 * s, par, abort)) { ok = false; break; }
+          mbar_expect_tx(k_full + 8 * s, kTile);
+          tma_load(kb, &p.mk, k_full + 8 * s, g * kHD, y);
+          tma_load(kb + kPanel, &p.mk, k_full + 8 * s, g * kHD + 64, y);
+          nk = t + 1;
+        }
+      }
+      if (nq >= 1) mbar_drain(qo_full, uint32_t((nq - 1) & 1));
+      for (int u = ::max(0, nk - 2); u < nk; ++u)
+        mbar_drain(k_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+      for (int u = ::max(0, nv - 2); u < nv; ++u)
+        mbar_drain(v_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+    }
+    __syncwarp();
+  } else if (warp == kSoftWarps + 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int t = 0;
+      int pd_t = -1, pd_n = 0;  // the pending dQ += dS K: tile, item ordinal
+      bool pd_first = false;
+      auto issue_dq = [&]() -> bool {
+        const int sp = pd_t & 1;
+        if (!mbar_wait(p_full + 8 * sp, uint32_t((pd_t >> 1) & 1), abort)) return false;
+        // the first dQ product of an item overwrites the accumulator: the
+        // previous item's dQ has been read
+        if (pd_first && pd_n >= 1 && !mbar_wait(dq_empty, uint32_t((pd_n - 1) & 1), abort))
+          return false;
+        fence_after();
+        const uint32_t kt = sK + uint32_t(sp * kTile);
+        const uint32_t da = tmem + kColDS + uint32_t(sp * 64);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          mma_ta(tmem + kColDQ, da + uint32_t(kk * 8), sdesc(kt + uint32_t(kk * 2048), kPanel, 1024),
+                 idesc(1), (!pd_first || kk > 0) ? 1u : 0u);
+        commit(dq_done + 8 * sp);
+        commit(k_empty + 8 * sp);
+        return true;
+      };
+      for (int n = 0; ok; ++n) {
+        const int it = item_at(n, G);
+        if (it >= p.items_q) break;
+        const Item x = item_of(ip, it);
+        if (pd_t >= 0) {
+          if (!issue_dq()) { ok = false; break; }
+          pd_t = -1;
+        }
+        if (!mbar_wait(qo_full, uint32_t(n & 1), abort)) { ok = false; break; }
+        for (int j = 0; j <= x.qb; ++j, ++t) {
+          const int s = t & 1;
+          if (!mbar_wait(k_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
+              !mbar_wait(v_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
+              (t >= 1 && !mbar_wait(s_free, uint32_t((t - 1) & 1), abort))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t kt = sK + uint32_t(s * kTile), vt = sV + uint32_t(s * kTile);
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mma(tmem, sdesc(sQ + off, 16, 1024), sdesc(kt + off, 16, 1024), idesc(0),
+                kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mma(tmem + kColDP, sdesc(sO + off, 16, 1024), sdesc(vt + off, 16, 1024), idesc(0),
+                kk > 0 ? 1u : 0u);
+          }
+          commit(s_full);
+          commit(v_empty + 8 * s);
+          if (j == x.qb) commit(qo_empty);
+          if (pd_t >= 0 && !issue_dq()) { ok = false; break; }
+          pd_t = t;
+          pd_n = n;
+          pd_first = j == 0;
+        }
+      }
+      if (ok && pd_t >= 0) issue_dq();
+      commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ dS (row r, key half hf)
+    const int lq = warp & 3, hf = warp >> 2;
+    const int r = lq * 32 + lane;
+    const uint32_t lbase = tmem + (uint32_t(lq * 32) << 16);
+    bool ok = true;
+    int t = 0;
+    for (int n = 0;; ++n) {
+      const int it = item_at(n, G);
+      if (it >= p.items_q) break;
+      const Item x = item_of(ip, it);
+      const int row0 = x.b * p.seq;
+      const int qi = x.qb * kRows + r;
+      const bool live = qi < p.seq;
+      const int64_t li = (int64_t(x.b) * p.H + x.h) * p.seq + (live ? qi : 0);
+      const float nl2 = live ? -p.lse[li] * kLog2ef : 0.f;
+      const float drow = live ? p.D[li] : 0.f;
+      for (int j = 0; j <= x.qb; ++j, ++t) {
+        const int s = t & 1;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(s_full, uint32_t(t & 1), abort));
+        if (!ok) continue;
+        fence_after();
+        uint32_t sv[kHalf], dp[kHalf];
+        tld32(lbase + uint32_t(hf * kHalf), sv);
+        tld32(lbase + uint32_t(hf * kHalf + 32), sv + 32);
+        tld32(lbase + kColDP + uint32_t(hf * kHalf), dp);
+        tld32(lbase + kColDP + uint32_t(hf * kHalf + 32), dp + 32);
+        tld_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // keys past this row (causal) carry P = 0; a row past the sequence is all 0
+        const int lim = live ? qi - j * kRows - hf * kHalf : -1;
+        uint32_t pk[kHalf / 2];
+#pragma unroll
+        for (int i = 0; i < kHalf / 2; ++i) {
+          float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), p.sl2, nl2));
+          float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), p.sl2, nl2));
+          if (2 * i > lim) p0 = 0.f;
+          if (2 * i + 1 > lim) p1 = 0.f;
+          pk[i] = pack_bf16x2(p0 * (__uint_as_float(dp[2 * i]) - drow),
+                              p1 * (__uint_as_float(dp[2 * i + 1]) - drow));
+        }
+        // dS buffer t % 2 is free once dQ += dS_{t-2} K_{t-2} is done
+        if (t >= 2) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(dq_done + 8 * s, uint32_t(((t - 2) >> 1) & 1), abort));
+          if (!ok) continue;
+          fence_after();
+        }
+        tst32(lbase + kColDS + uint32_t(s * 64 + hf * 32), pk);
+        tst_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + 8 * s);
+      }
+      const int tl = t - 1;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(dq_done + 8 * (tl & 1),
+                                                   uint32_t((tl >> 1) & 1), abort));
+      if (ok) {
+        fence_after();
+        uint32_t o[kHalf];
+        tld32(lbase + kColDQ + uint32_t(hf * kHalf), o);
+        tld32(lbase + kColDQ + uint32_t(hf * kHalf + 32), o + 32);
+        tld_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_empty);
+        if (live) {
+          float4* dst = reinterpret_cast<float4*>(p.dQ + (int64_t(row0) + qi) * (int64_t(p.H) * kHD) +
+                                                  x.h * kHD + hf * kHalf);
+#pragma unroll
+          for (int v = 0; v < kHalf / 4; ++v)
+            dst[v] = make_float4(__uint_as_float(o[4 * v]) * p.scale, __uint_as_float(o[4 * v + 1]) * p.scale,
+                                 __uint_as_float(o[4 * v + 2]) * p.scale,
+                                 __uint_as_float(o[4 * v + 3]) * p.scale);
+        }
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// dK/dV kernel: K and V at 0 and 32 KB, (Q, dO) stages from 64 KB; per stage
+// the query tile's -lse log2e and D in shared vectors; tensor memory S^T 0,
+// dP^T 128, dV 256, dK 384.  P^T / dS^T of the first 64 queries overwrite
+// columns 0-31 of S^T / dP^T, those of the last 64 columns 96-127 (each inside
+// the half row its warp has already read).
+constexpr int kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;  // stage s: Q at +2s, dO at +2s+1 tiles
+constexpr int kKOffBar = 6 * kTile;
+constexpr int kKOffVec = kKOffBar + 256;  // [stage][lse2 | D][128] fp32
+constexpr int kKSmem = kKOffVec + 2048 + 1024;
+constexpr uint32_t kColDV = 256, kColDK = 384;
+
+// Item `it` of the dK/dV kernel (longest first: key block kb ascending).
+struct KItem {
+  int kb, g, b;
+};
+__device__ __forceinline__ KItem kitem_of(const TcBwdP& p, int it) {
+  const int gb = p.KV * p.batch;
+  KItem x;
+  x.kb = it / gb;
+  x.g = (it % gb) % p.KV;
+  x.b = (it % gb) / p.KV;
+  return x;
+}
+// A-operand column of K block kk (16 rows) in the overwritten halves.
+__device__ __forceinline__ uint32_t half_col(int kk) {
+  return uint32_t(kk < 4 ? kk * 8 : 96 + (kk - 4) * 8);
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __grid_constant__ TcBwdP p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + kKOffK, sV = base + kKOffV, sQ0 = base + kKOffQ;
+  const uint32_t bar = base + kKOffBar;
+  const uint32_t kv_full = bar, kv_empty = bar + 8, qo_full = bar + 16, qo_empty = bar + 32,
+                 vec_full = bar + 48, st_full = bar + 64, p_full = bar + 72, pv_done = bar + 80,
+                 dkv_empty = bar + 88, mma_done = bar + 96;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kKOffBar + 192);
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kKOffBar + 200);
+  float* vec = reinterpret_cast<float*>(gbase + kKOffVec);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = int(gridDim.x);
+  const int rep = p.H / p.KV;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     su32(s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 32) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qo_full + 8 * s, 1);
+      mbar_init(qo_empty + 8 * s, 1);
+      mbar_init(vec_full + 8 * s, 32);
+    }
+    mbar_init(st_full, 1);
+    mbar_init(p_full, kSoftWarps);
+    mbar_init(pv_done, 1);
+    mbar_init(dkv_empty, kSoftWarps);
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == kSoftWarps) {
+    // ------------------------------------------------ producer warp: lane 0
+    // issues the copies, every lane stages the query vectors
+    int t = 0, nkv = 0, nqo = 0;
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      const int it = item_at(n, G);
+      if (it >= p.items_k) break;
+      const KItem x = kitem_of(p, it);
+      const int row0 = x.b * p.seq, nq = p.nqb - x.kb;
+      ok = __all_sync(0xffffffffu, n == 0 || mbar_wait(kv_empty, uint32_t((n - 1) & 1), abort));
+      if (!ok) break;
+      if (lane == 0) {
+        const int y = row0 + x.kb * kRows;
+        mbar_expect_tx(kv_full, 2 * kTile);
+        tma_load(sK, &p.mk, kv_full, x.g * kHD, y);
+        tma_load(sK + kPanel, &p.mk, kv_full, x.g * kHD + 64, y);
+        tma_load(sV, &p.mv, kv_full, x.g * kHD, y);
+        tma_load(sV + kPanel, &p.mv, kv_full, x.g * kHD + 64, y);
+      }
+      nkv = n + 1;
+      for (int jj = 0; jj < rep * nq; ++jj, ++t) {
+        const int s = t & 1;
+        const int hq = x.g * rep + jj / nq, qt = x.kb + jj % nq;
+        ok = __all_sync(0xffffffffu, t < 2 || mbar_wait(qo_empty + 8 * s,
+                                                        uint32_t(((t - 2) >> 1) & 1), abort));
+        if (!ok) break;
+        const uint32_t sq = sQ0 + uint32_t(2 * s * kTile), so = sq + kTile;
+        const int y = row0 + qt * kRows;
+        if (lane == 0) {
+          mbar_expect_tx(qo_full + 8 * s, 2 * kTile);
+          tma_load(sq, &p.mq, qo_full + 8 * s, hq * kHD, y);
+          tma_load(sq + kPanel, &p.mq, qo_full + 8 * s, hq * kHD + 64, y);
+          tma_load(so, &p.mdo, qo_full + 8 * s, hq * kHD, y);
+          tma_load(so + kPanel, &p.mdo, qo_full + 8 * s, hq * kHD + 64, y);
+        }
+        nqo = t + 1;
+        const int64_t l0 = (int64_t(x.b) * p.H + hq) * p.seq;
+        float* vl = vec + s * 2 * kRows;
+#pragma unroll
+        for (int c = lane; c < kRows; c += 32) {
+          const int q = qt * kRows + c;
+          vl[c] = q < p.seq ? -p.lse[l0 + q] * kLog2ef : 0.f;
+          vl[kRows + c] = q < p.seq ? p.D[l0 + q] : 0.f;
+        }
+        mbar_arrive(vec_full + 8 * s);
+      }
+    }
+    if (lane == 0) {
+      if (nkv >= 1) mbar_drain(kv_full, uint32_t((nkv - 1) & 1));
+      for (int u = ::max(0, nqo - 2); u < nqo; ++u)
+        mbar_drain(qo_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+    }
+    __syncwarp();
+  } else if (warp == kSoftWarps + 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int t = 0;
+      for (int n = 0; ok; ++n) {
+        const int it = item_at(n, G);
+        if (it >= p.items_k) break;
+        const KItem x = kitem_of(p, it);
+        const int ntile = rep * (p.nqb - x.kb);
+        if (!mbar_wait(kv_full, uint32_t(n & 1), abort)) { ok = false; break; }
+        for (int jj = 0; jj < ntile; ++jj, ++t) {
+          const int s = t & 1;
+          const uint32_t sq = sQ0 + uint32_t(2 * s * kTile), so = sq + kTile;
+          // S^T and dP^T overwrite the columns P^T_{t-1} and dS^T_{t-1} were read from
+          if (!mbar_wait(qo_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
+              (t >= 1 && !mbar_wait(pv_done, uint32_t((t - 1) & 1), abort))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mma(tmem, sdesc(sK + off, 16, 1024), sdesc(sq + off, 16, 1024), idesc(0),
+                kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mma(tmem + kColDP, sdesc(sV + off, 16, 1024), sdesc(so + off, 16, 1024), idesc(0),
+                kk > 0 ? 1u : 0u);
+          }
+          commit(st_full);
+          if (jj == ntile - 1) commit(kv_empty);  // K and V of this block are read
+          if (!mbar_wait(p_full, uint32_t(t & 1), abort) ||
+              (jj == 0 && n >= 1 && !mbar_wait(dkv_empty, uint32_t((n - 1) & 1), abort))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          // dV += P^T dO and dK += dS^T Q (dO and Q MN-major)
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ta(tmem + kColDV, tmem + half_col(kk),
+                   sdesc(so + uint32_t(kk * 2048), kPanel, 1024), idesc(1),
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ta(tmem + kColDK, tmem + kColDP + half_col(kk),
+                   sdesc(sq + uint32_t(kk * 2048), kPanel, 1024), idesc(1),
+                   (jj > 0 || kk > 0) ? 1u : 0u);
+          commit(pv_done);
+          commit(qo_empty + 8 * s);
+        }
+      }
+      commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ P^T, dS^T (key row r, query half hf)
+    const int lq = warp & 3, hf = warp >> 2;
+    const int r = lq * 32 + lane;
+    const uint32_t lbase = tmem + (uint32_t(lq * 32) << 16);
+    const uint32_t ocol = hf ? 96u : 0u;  // where this half's bf16 pairs go
+    bool ok = true;
+    int t = 0;
+    for (int n = 0;; ++n) {
+      const int it = item_at(n, G);
+      if (it >= p.items_k) break;
+      const KItem x = kitem_of(p, it);
+      const int nq = p.nqb - x.kb, ntile = rep * nq;
+      const int key = x.kb * kRows + r;
+      for (int jj = 0; jj < ntile; ++jj, ++t) {
+        const int s = t & 1;
+        const int qt = x.kb + jj % nq;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(vec_full + 8 * s, uint32_t((t >> 1) & 1), abort) &&
+                                         mbar_wait(st_full, uint32_t(t & 1), abort));
+        if (!ok) continue;
+        fence_after();
+        uint32_t sv[kHalf], dp[kHalf];
+        tld32(lbase + uint32_t(hf * kHalf), sv);
+        tld32(lbase + uint32_t(hf * kHalf + 32), sv + 32);
+        tld32(lbase + kColDP + uint32_t(hf * kHalf), dp);
+        tld32(lbase + kColDP + uint32_t(hf * kHalf + 32), dp + 32);
+        tld_wait();
+        // query columns c of this half with key <= query < seq
+        const int q0 = qt * kRows + hf * kHalf;
+        const int lo = key - q0, hi = p.seq - q0;  // keep lo <= c < hi
+        const float4* vl = reinterpret_cast<const float4*>(vec + s * 2 * kRows + hf * kHalf);
+        const float4* vd = reinterpret_cast<const float4*>(vec + s * 2 * kRows + kRows + hf * kHalf);
+        uint32_t pp[kHalf / 2], pd[kHalf / 2];
+#pragma unroll
+        for (int v = 0; v < kHalf / 4; ++v) {
+          const float4 l4 = vl[v], d4 = vd[v];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pe[4], de[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * v + e;
+            float pv = ex2(fmaf(__uint_as_float(sv[c]), p.sl2, lv[e]));
+            if (c < lo || c >= hi) pv = 0.f;
+            pe[e] = pv;
+            de[e] = pv * (__uint_as_float(dp[c]) - dv[e]);
+          }
+          pp[2 * v] = pack_bf16x2(pe[0], pe[1]);
+          pp[2 * v + 1] = pack_bf16x2(pe[2], pe[3]);
+          pd[2 * v] = pack_bf16x2(de[0], de[1]);
+          pd[2 * v + 1] = pack_bf16x2(de[2], de[3]);
+        }
+        tst32(lbase + ocol, pp);
+        tst32(lbase + kColDP + ocol, pd);
+        tst_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      const int tl = t - 1;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(pv_done, uint32_t(tl & 1), abort));
+      if (ok) {
+        fence_after();
+        uint32_t a[kHalf], c[kHalf];
+        tld32(lbase + kColDV + uint32_t(hf * kHalf), a);
+        tld32(lbase + kColDV + uint32_t(hf * kHalf + 32), a + 32);
+        tld32(lbase + kColDK + uint32_t(hf * kHalf), c);
+        tld32(lbase + kColDK + uint32_t(hf * kHalf + 32), c + 32);
+        tld_wait();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dkv_empty);
+        if (key < p.seq) {
+          const int64_t row = int64_t(x.b) * p.seq + key;
+          const int64_t col = int64_t(x.g) * kHD + hf * kHalf;
+          uint4* dv = reinterpret_cast<uint4*>(p.dV + row * (int64_t(p.KV) * kHD) + col);
+          float4* dk = reinterpret_cast<float4*>(p.dK + row * (int64_t(p.KV) * kHD) + col);
+#pragma unroll
+          for (int v = 0; v < kHalf / 8; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1]));
+            w.y = pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3]));
+            w.z = pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5]));
+            w.w = pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7]));
+            dv[v] = w;
+          }
+#pragma unroll
+          for (int v = 0; v < kHalf / 4; ++v)
+            dk[v] = make_float4(__uint_as_float(c[4 * v]) * p.scale, __uint_as_float(c[4 * v + 1]) * p.scale,
+                                __uint_as_float(c[4 * v + 2]) * p.scale,
+                                __uint_as_float(c[4 * v + 3]) * p.scale);
+        }
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 // ----------------------------------------------------------------- host
 PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
 std::once_flag g_enc_once;
@@ -619,6 +1196,50 @@ slora_status attention_fwd_tc_run(const void* Q, const void* K, const void* V, c
   const dim3 grid(unsigned(std::min(p.items, num_sms())));
   attn_fwd_tc_kernel<<<grid, kThreadsTc, kSmem, st>>>(p);
   SLORA_CHECK_LAUNCH();
+  return SLORA_OK;
+}
+
+bool attention_bwd_tc_ok(const void* Q, const void* K, const void* V, const void* dO,
+                         const void* dQ, const void* dK, const void* dV, int hd) {
+  return hd == kHD && aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(dO) &&
+         aligned16(dQ) && aligned16(dK) && aligned16(dV);
+}
+
+slora_status attention_bwd_tc_run(const void* Q, const void* K, const void* V, const void* dO,
+                                  const float* lse, const float* D, const TokenInfo& ti, int H,
+                                  int KV, float* dQ, float* dK, void* dV, double flops_per_product,
+                                  cudaStream_t st) {
+  if (!attention_bwd_tc_ok(Q, K, V, dO, dQ, dK, dV, kHD))
+    SLORA_FAIL(SLORA_ERR_ALIGN, "attention backward: operands must be 16-byte aligned");
+  TcBwdP p;
+  SLORA_TRY(encode_rows(&p.mq, Q, ti.T, int64_t(H) * kHD));
+  SLORA_TRY(encode_rows(&p.mdo, dO, ti.T, int64_t(H) * kHD));
+  SLORA_TRY(encode_rows(&p.mk, K, ti.T, int64_t(KV) * kHD));
+  SLORA_TRY(encode_rows(&p.mv, V, ti.T, int64_t(KV) * kHD));
+  p.lse = lse; p.D = D; p.dQ = dQ; p.dK = dK;
+  p.dV = static_cast<__nv_bfloat16*>(dV);
+  p.seq = ti.seq; p.H = H; p.KV = KV; p.batch = ti.batch;
+  p.nqb = (ti.seq + kRows - 1) / kRows;
+  p.items_q = p.nqb * H * ti.batch;
+  p.items_k = p.nqb * KV * ti.batch;
+  p.scale = float(1.0 / std::sqrt(double(kHD)));
+  p.sl2 = float(double(p.scale) * 1.4426950408889634);
+  {
+    // algorithmic work: S^T, dP^T, dV, dK (the dQ launch books dQ alone; its
+    // S and dP are recomputed)
+    LaunchScope ls(kAttention, 4.0 * flops_per_product, st);
+    SLORA_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_tc_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kKSmem));
+    attn_bwd_dkv_tc_kernel<<<unsigned(std::min(p.items_k, num_sms())), kThreadsTc, kKSmem, st>>>(p);
+    SLORA_CHECK_LAUNCH();
+  }
+  {
+    LaunchScope ls(kAttention, 1.0 * flops_per_product, st);
+    SLORA_CUDA(cudaFuncSetAttribute(attn_bwd_dq_tc_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem));
+    attn_bwd_dq_tc_kernel<<<unsigned(std::min(p.items_q, num_sms())), kThreadsTc, kQSmem, st>>>(p);
+    SLORA_CHECK_LAUNCH();
+  }
   return SLORA_OK;
 }
 
