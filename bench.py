@@ -1068,8 +1068,12 @@ def run_decoder(args, H, pk, rank, world):
                     "the GPU, distinct per layer)",
             "config": workload_config("llama2-7b-decoder32-bf16", world),
             "roofline": gemm_roofline(prof, pk),
-            "attention_core": {"kernels": "attn_fwd_kernel / attn_bwd_kernel (mma.sync "
-                                          "m16n8k16)", "achieved": att, "unit": "TFLOP/s",
+            "attention_core": {"kernels": "attn_fwd_tc_kernel / attn_bwd_dkv_tc_kernel + "
+                                          "attn_bwd_dq_tc_kernel (tcgen05, tensor-memory "
+                                          "accumulators)",
+                               "work": "algorithmic: 2 causal products forward, 5 backward "
+                                       "(the dQ kernel's recomputed S and dP not counted)",
+                               "achieved": att, "unit": "TFLOP/s",
                                "peak": pk["bf16"], "frac": att / pk["bf16"],
                                "ms_per_step": ms_a / args.steps,
                                "flops_per_step": fl_a / args.steps},
