@@ -57,13 +57,14 @@ constexpr int kRows = 128;                 // query rows per CTA, keys per tile
 constexpr int kHD = 128;                   // head width
 constexpr int kPanel = 128 * 128;          // bytes: 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr int kTile = 2 * kPanel;          // 128 x 128 bf16
-constexpr int kOffQ = 0;
-constexpr int kOffK = kTile;               // 2 stages
-constexpr int kOffV = 3 * kTile;           // 2 stages
-constexpr int kOffBar = 5 * kTile;         // 18 mbarriers, the tensor-memory address, a flag
+constexpr int kOffQ = 0;                   // 2 buffers (item parity)
+constexpr int kOffK = 2 * kTile;           // 2 stages
+constexpr int kOffV = 4 * kTile;           // 2 stages
+constexpr int kOffBar = 6 * kTile;         // 22 mbarriers, the tensor-memory address, a flag
 constexpr int kOffX = kOffBar + 256;       // row-block maxima: [tile parity][half][row] fp32
 constexpr int kOffL = kOffX + 2048;        // row-sum halves: [half][row] fp32
-constexpr int kSmem = kOffL + 1024 + 1024; // + 1024-byte alignment slack
+constexpr int kOffSt = kOffL + 1024;       // per-warp store staging (8 softmax warps)
+constexpr int kSmem = kOffSt + 8 * 32 * 5 * 16 + 1024; // + 1024-byte alignment slack
 constexpr int kSoftWarps = 8;              // two per row block (one per 64-column half)
 constexpr int kThreadsTc = (kSoftWarps + 2) * 32;
 constexpr int kHalf = 64;                  // columns per softmax thread
@@ -204,6 +205,41 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Warp-cooperative store of 32 rows (one per lane) through the warp's own
+// shared staging area (32 x 5 chunks of 16 bytes): each lane hands in 4
+// chunks (64 contiguous bytes) of its row; the warp writes them back 8 rows
+// per instruction, each row's 64 bytes by 4 adjacent lanes, so a store
+// instruction touches 8 row segments instead of 32.  `dst` is the lane's
+// row address, `live` whether its row is stored.
+constexpr int kStageWarp = 32 * 5 * 16;
+__device__ __forceinline__ void warp_store_rows(uint32_t stage, const uint4 (&v)[4], char* dst,
+                                                bool live) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage + uint32_t((lane * 5 + c) * 16)),
+                 "r"(v[c].x), "r"(v[c].y), "r"(v[c].z), "r"(v[c].w)
+                 : "memory");
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = k * 8 + (lane >> 2), c = lane & 3;
+    char* rp = reinterpret_cast<char*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), row));
+    const bool lv = __shfl_sync(0xffffffffu, live ? 1 : 0, row) != 0;
+    uint4 x;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                 : "r"(stage + uint32_t((row * 5 + c) * 16))
+                 : "memory");
+    if (lv) reinterpret_cast<uint4*>(rp)[c] = x;
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ uint4 f4bits(float a, float b, float c, float d) {
+  return make_uint4(__float_as_uint(a), __float_as_uint(b), __float_as_uint(c), __float_as_uint(d));
+}
+
 struct TcFwdP {
   CUtensorMap mq, mk, mv;   // Q [T x H 128], K and V [T x KV 128]; boxes 64 x 128, 128-byte swizzle
   __nv_bfloat16* O;         // [T x H 128]
@@ -251,10 +287,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
   const uint32_t sQ = base + kOffQ, sK = base + kOffK, sV = base + kOffV;
   const uint32_t bar = base + kOffBar;
   // mbarriers; those with two copies are indexed by buffer / stage (tile t uses t % 2)
-  const uint32_t q_full = bar, q_empty = bar + 8, k_full = bar + 16, v_full = bar + 32,
-                 k_empty = bar + 48, v_empty = bar + 64, s_full = bar + 80, s_free = bar + 96,
-                 p_full = bar + 112, pv_done = bar + 128, o_empty = bar + 144,
-                 mma_done = bar + 152;
+  const uint32_t k_full = bar + 16, v_full = bar + 32, k_empty = bar + 48, v_empty = bar + 64,
+                 s_full = bar + 80, s_free = bar + 96, p_full = bar + 112, pv_done = bar + 128,
+                 o_empty = bar + 144, mma_done = bar + 152, q_full = bar + 160,
+                 q_empty = bar + 176;  // Q buffer of item n: n % 2
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kOffBar + 192);
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + 200);
   float* xmax = reinterpret_cast<float*>(gbase + kOffX);  // [tile parity][half][row]
@@ -269,9 +305,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 32) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full + 8 * s, 1);
+      mbar_init(q_empty + 8 * s, 1);
       mbar_init(k_full + 8 * s, 1);
       mbar_init(v_full + 8 * s, 1);
       mbar_init(k_empty + 8 * s, 1);
@@ -301,11 +337,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
         if (it >= p.items) break;
         const Item x = item_of(p, it);
         const int row0 = x.b * p.seq, g = x.h / (p.H / p.KV);
-        // Q_n once every S of item n - 1 is computed
-        if (n >= 1 && !mbar_wait(q_empty, uint32_t((n - 1) & 1), abort)) break;
-        mbar_expect_tx(q_full, kTile);
-        tma_load(sQ, &p.mq, q_full, x.h * kHD, row0 + x.qb * kRows);
-        tma_load(sQ + kPanel, &p.mq, q_full, x.h * kHD + 64, row0 + x.qb * kRows);
+        // Q_n into buffer n % 2 once every S of item n - 2 is computed
+        const int qb2 = n & 1;
+        const uint32_t qf = q_full + 8 * qb2, sq = sQ + uint32_t(qb2 * kTile);
+        if (n >= 2 && !mbar_wait(q_empty + 8 * qb2, uint32_t(((n - 2) >> 1) & 1), abort)) break;
+        mbar_expect_tx(qf, kTile);
+        tma_load(sq, &p.mq, qf, x.h * kHD, row0 + x.qb * kRows);
+        tma_load(sq + kPanel, &p.mq, qf, x.h * kHD + 64, row0 + x.qb * kRows);
         nq = n + 1;
         for (int j = 0; j <= x.qb; ++j, ++t) {
           const int s = t & 1;
@@ -327,7 +365,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
       }
       // the copies issued last into each buffer have landed before the CTA
       // can release its shared memory (on the normal path they were consumed)
-      if (nq >= 1) mbar_drain(q_full, uint32_t((nq - 1) & 1));
+      for (int u = ::max(0, nq - 2); u < nq; ++u)
+        mbar_drain(q_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
       for (int u = ::max(0, nk - 2); u < nk; ++u)
         mbar_drain(k_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
       for (int u = ::max(0, nv - 2); u < nv; ++u)
@@ -372,7 +411,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
           if (!issue_pv()) { ok = false; break; }
           pv_t = -1;
         }
-        if (!mbar_wait(q_full, uint32_t(n & 1), abort)) { ok = false; break; }
+        const uint32_t sq = sQ + uint32_t((n & 1) * kTile);
+        if (!mbar_wait(q_full + 8 * (n & 1), uint32_t((n >> 1) & 1), abort)) { ok = false; break; }
         for (int j = 0; j <= x.qb; ++j, ++t) {
           const int s = t & 1;
           // S_t = Q K_t^T into S buffer t % 2
@@ -387,12 +427,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
             const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
-            mma(d, sdesc(sQ + off, 16, 1024), sdesc(kt + off, 16, 1024), idesc(0),
+            mma(d, sdesc(sq + off, 16, 1024), sdesc(kt + off, 16, 1024), idesc(0),
                 kk > 0 ? 1u : 0u);
           }
           commit(s_full + 8 * s);
           commit(k_empty + 8 * s);
-          if (j == x.qb) commit(q_empty);  // every S of this item issued
+          if (j == x.qb) commit(q_empty + 8 * (n & 1));  // every S of this item issued
           if (pv_t >= 0 && !issue_pv()) { ok = false; break; }
           pv_t = t;
           pv_n = n;
@@ -536,19 +576,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_empty);  // the next item's P V may overwrite O
-        if (qi < p.seq) {
+        {
           const float inv = 1.f / lt;
-          uint4* dst = reinterpret_cast<uint4*>(p.O + (int64_t(row0) + qi) * (int64_t(p.H) * kHD) +
-                                                x.h * kHD + hf * kHalf);
+          char* dst = reinterpret_cast<char*>(p.O + (int64_t(row0) + qi) * (int64_t(p.H) * kHD) +
+                                              x.h * kHD + hf * kHalf);
+          const uint32_t stage = base + uint32_t(kOffSt + warp * kStageWarp);
 #pragma unroll
-          for (int v = 0; v < kHalf / 8; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-            dst[v] = w;
+          for (int hh = 0; hh < 2; ++hh) {  // 32 columns (64 bytes) per pass
+            uint4 w[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint32_t* oo = o + 32 * hh + 8 * v;
+              w[v].x = pack_bf16x2(__uint_as_float(oo[0]) * inv, __uint_as_float(oo[1]) * inv);
+              w[v].y = pack_bf16x2(__uint_as_float(oo[2]) * inv, __uint_as_float(oo[3]) * inv);
+              w[v].z = pack_bf16x2(__uint_as_float(oo[4]) * inv, __uint_as_float(oo[5]) * inv);
+              w[v].w = pack_bf16x2(__uint_as_float(oo[6]) * inv, __uint_as_float(oo[7]) * inv);
+            }
+            warp_store_rows(stage, w, dst + 64 * hh, qi < p.seq);
           }
+        }
+        if (qi < p.seq) {
           if (hf == 0) p.lse[(int64_t(x.b) * p.H + x.h) * p.seq + qi] = (m + log2f(lt)) * kLn2f;
         }
       }
@@ -594,10 +641,13 @@ struct TcBwdP {
 
 constexpr float kLog2ef = 1.4426950408889634f;
 
-// dQ kernel: Q and dO at 0 and 32 KB, K and V stages from 64 KB; tensor
-// memory S 0, dP 128, dQ 256, dS at 384 and 448.
-constexpr int kQOffQ = 0, kQOffO = kTile, kQOffK = 2 * kTile, kQOffV = 4 * kTile;
-constexpr int kQOffBar = 6 * kTile;
+// dQ kernel: Q and dO at 0 and 32 KB, three K stages from 64 KB (a K tile
+// stays until its dQ product is done, so its refill needs two tiles of
+// lead), two V stages from 160 KB; tensor memory S 0, dP 128, dQ 256, dS at
+// 384 and 448.
+constexpr int kQKStages = 3;
+constexpr int kQOffQ = 0, kQOffO = kTile, kQOffK = 2 * kTile, kQOffV = 5 * kTile;
+constexpr int kQOffBar = 7 * kTile;
 constexpr int kQSmem = kQOffBar + 256 + 1024;
 constexpr uint32_t kColDP = 128, kColDQ = 256, kColDS = 384;
 
@@ -608,10 +658,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
   unsigned char* gbase = smem_raw + (base - raw);
   const uint32_t sQ = base + kQOffQ, sO = base + kQOffO, sK = base + kQOffK, sV = base + kQOffV;
   const uint32_t bar = base + kQOffBar;
-  const uint32_t qo_full = bar, qo_empty = bar + 8, k_full = bar + 16, v_full = bar + 32,
-                 k_empty = bar + 48, v_empty = bar + 64, s_full = bar + 80, s_free = bar + 88,
-                 p_full = bar + 96, dq_done = bar + 112, dq_empty = bar + 128,
-                 mma_done = bar + 136;
+  const uint32_t qo_full = bar, qo_empty = bar + 8, v_full = bar + 16, v_empty = bar + 32,
+                 s_full = bar + 48, s_free = bar + 56, p_full = bar + 64, dq_done = bar + 80,
+                 dq_empty = bar + 96, mma_done = bar + 104, k_full = bar + 112,
+                 k_empty = bar + 136;  // K stage of tile t: t % 3
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kQOffBar + 192);
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + kQOffBar + 200);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -629,12 +679,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
     mbar_init(qo_full, 1);
     mbar_init(qo_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(k_full + 8 * s, 1);
       mbar_init(v_full + 8 * s, 1);
-      mbar_init(k_empty + 8 * s, 1);
       mbar_init(v_empty + 8 * s, 1);
       mbar_init(p_full + 8 * s, kSoftWarps);
       mbar_init(dq_done + 8 * s, 1);
+    }
+    for (int s = 0; s < kQKStages; ++s) {
+      mbar_init(k_full + 8 * s, 1);
+      mbar_init(k_empty + 8 * s, 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftWarps);
@@ -667,26 +719,32 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
         tma_load(sO + kPanel, &p.mdo, qo_full, x.h * kHD + 64, yq);
         nq = n + 1;
         for (int j = 0; j <= x.qb; ++j, ++t) {
-          const int s = t & 1;
-          const uint32_t par = uint32_t(((t - 2) >> 1) & 1);
+          const int s = t & 1, s3 = t % kQKStages;
           const int y = row0 + j * kRows;
-          // K_t once dQ += dS_{t-2} K_{t-2} is done, V_t once dP_{t-2} is
-          if (t >= 2 && !mbar_wait(v_empty + 8 * s, par, abort)) { ok = false; break; }
-          const uint32_t kb = sK + uint32_t(s * kTile), vb = sV + uint32_t(s * kTile);
+          // V_t once dP_{t-2} is done, K_t once dQ += dS_{t-3} K_{t-3} is
+          if (t >= 2 && !mbar_wait(v_empty + 8 * s, uint32_t(((t - 2) >> 1) & 1), abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t kb = sK + uint32_t(s3 * kTile), vb = sV + uint32_t(s * kTile);
           mbar_expect_tx(v_full + 8 * s, kTile);
           tma_load(vb, &p.mv, v_full + 8 * s, g * kHD, y);
           tma_load(vb + kPanel, &p.mv, v_full + 8 * s, g * kHD + 64, y);
           nv = t + 1;
-          if (t >= 2 && !mbar_wait(k_empty + 8 * s, par, abort)) { ok = false; break; }
-          mbar_expect_tx(k_full + 8 * s, kTile);
-          tma_load(kb, &p.mk, k_full + 8 * s, g * kHD, y);
-          tma_load(kb + kPanel, &p.mk, k_full + 8 * s, g * kHD + 64, y);
+          if (t >= kQKStages &&
+              !mbar_wait(k_empty + 8 * s3, uint32_t(((t - kQKStages) / kQKStages) & 1), abort)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(k_full + 8 * s3, kTile);
+          tma_load(kb, &p.mk, k_full + 8 * s3, g * kHD, y);
+          tma_load(kb + kPanel, &p.mk, k_full + 8 * s3, g * kHD + 64, y);
           nk = t + 1;
         }
       }
       if (nq >= 1) mbar_drain(qo_full, uint32_t((nq - 1) & 1));
-      for (int u = ::max(0, nk - 2); u < nk; ++u)
-        mbar_drain(k_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+      for (int u = ::max(0, nk - kQKStages); u < nk; ++u)
+        mbar_drain(k_full + 8 * (u % kQKStages), uint32_t((u / kQKStages) & 1));
       for (int u = ::max(0, nv - 2); u < nv; ++u)
         mbar_drain(v_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
     }
@@ -706,14 +764,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
         if (pd_first && pd_n >= 1 && !mbar_wait(dq_empty, uint32_t((pd_n - 1) & 1), abort))
           return false;
         fence_after();
-        const uint32_t kt = sK + uint32_t(sp * kTile);
+        const uint32_t kt = sK + uint32_t((pd_t % kQKStages) * kTile);
         const uint32_t da = tmem + kColDS + uint32_t(sp * 64);
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk)
           mma_ta(tmem + kColDQ, da + uint32_t(kk * 8), sdesc(kt + uint32_t(kk * 2048), kPanel, 1024),
                  idesc(1), (!pd_first || kk > 0) ? 1u : 0u);
         commit(dq_done + 8 * sp);
-        commit(k_empty + 8 * sp);
+        commit(k_empty + 8 * (pd_t % kQKStages));
         return true;
       };
       for (int n = 0; ok; ++n) {
@@ -726,15 +784,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
         }
         if (!mbar_wait(qo_full, uint32_t(n & 1), abort)) { ok = false; break; }
         for (int j = 0; j <= x.qb; ++j, ++t) {
-          const int s = t & 1;
-          if (!mbar_wait(k_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
+          const int s = t & 1, s3 = t % kQKStages;
+          if (!mbar_wait(k_full + 8 * s3, uint32_t((t / kQKStages) & 1), abort) ||
               !mbar_wait(v_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
               (t >= 1 && !mbar_wait(s_free, uint32_t((t - 1) & 1), abort))) {
             ok = false;
             break;
           }
           fence_after();
-          const uint32_t kt = sK + uint32_t(s * kTile), vt = sV + uint32_t(s * kTile);
+          const uint32_t kt = sK + uint32_t(s3 * kTile), vt = sV + uint32_t(s * kTile);
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
             const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
@@ -859,7 +917,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
 constexpr int kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;  // stage s: Q at +2s, dO at +2s+1 tiles
 constexpr int kKOffBar = 6 * kTile;
 constexpr int kKOffVec = kKOffBar + 256;  // [stage][lse2 | D][128] fp32
-constexpr int kKSmem = kKOffVec + 2048 + 1024;
+constexpr int kKOffSt = kKOffVec + 2048;  // per-warp store staging
+constexpr int kKSmem = kKOffSt + 8 * kStageWarp + 1024;
 constexpr uint32_t kColDV = 256, kColDK = 384;
 
 // Item `it` of the dK/dV kernel (longest first: key block kb ascending).
@@ -1108,25 +1167,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dkv_empty);
-        if (key < p.seq) {
-          const int64_t row = int64_t(x.b) * p.seq + key;
-          const int64_t col = int64_t(x.g) * kHD + hf * kHalf;
-          uint4* dv = reinterpret_cast<uint4*>(p.dV + row * (int64_t(p.KV) * kHD) + col);
-          float4* dk = reinterpret_cast<float4*>(p.dK + row * (int64_t(p.KV) * kHD) + col);
+        const int64_t row = int64_t(x.b) * p.seq + key;
+        const int64_t col = int64_t(x.g) * kHD + hf * kHalf;
+        char* dvp = reinterpret_cast<char*>(p.dV + row * (int64_t(p.KV) * kHD) + col);
+        char* dkp = reinterpret_cast<char*>(p.dK + row * (int64_t(p.KV) * kHD) + col);
+        const uint32_t stage = base + uint32_t(kKOffSt + warp * kStageWarp);
+        const bool live = key < p.seq;
 #pragma unroll
-          for (int v = 0; v < kHalf / 8; ++v) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1]));
-            w.y = pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3]));
-            w.z = pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5]));
-            w.w = pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7]));
-            dv[v] = w;
+        for (int hh = 0; hh < 2; ++hh) {  // dV: 32 bf16 (64 bytes) per pass
+          uint4 w[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t* aa = a + 32 * hh + 8 * v;
+            w[v].x = pack_bf16x2(__uint_as_float(aa[0]), __uint_as_float(aa[1]));
+            w[v].y = pack_bf16x2(__uint_as_float(aa[2]), __uint_as_float(aa[3]));
+            w[v].z = pack_bf16x2(__uint_as_float(aa[4]), __uint_as_float(aa[5]));
+            w[v].w = pack_bf16x2(__uint_as_float(aa[6]), __uint_as_float(aa[7]));
           }
+          warp_store_rows(stage, w, dvp + 64 * hh, live);
+        }
 #pragma unroll
-          for (int v = 0; v < kHalf / 4; ++v)
-            dk[v] = make_float4(__uint_as_float(c[4 * v]) * p.scale, __uint_as_float(c[4 * v + 1]) * p.scale,
-                                __uint_as_float(c[4 * v + 2]) * p.scale,
-                                __uint_as_float(c[4 * v + 3]) * p.scale);
+        for (int qq = 0; qq < 4; ++qq) {  // dK: 16 fp32 (64 bytes) per pass
+          uint4 w[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t* cc = c + 16 * qq + 4 * v;
+            w[v] = f4bits(__uint_as_float(cc[0]) * p.scale, __uint_as_float(cc[1]) * p.scale,
+                          __uint_as_float(cc[2]) * p.scale, __uint_as_float(cc[3]) * p.scale);
+          }
+          warp_store_rows(stage, w, dkp + 64 * qq, live);
         }
       }
     }
