@@ -77,8 +77,8 @@ constexpr long long kWaitBudget = 2000000000LL;  // clock cycles
 
 // kind::f16 instruction descriptor: fp32 D, bf16 A and B, A K-major, B K-major
 // (b_mn = 0) or MN-major (1), M = 128, N = 128.
-constexpr uint32_t idesc(int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) | (uint32_t(128 >> 3) << 17) |
+constexpr uint32_t idesc(int b_mn, int n = 128) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) | (uint32_t(n >> 3) << 17) |
          (uint32_t(128 >> 4) << 24);
 }
 
@@ -187,6 +187,15 @@ __device__ __forceinline__ void tst32(uint32_t taddr, const uint32_t* r) {
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tst16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tld_wait() {
@@ -629,6 +638,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
 //       dV bf16.
 struct TcBwdP {
   CUtensorMap mq, mk, mv, mdo;  // Q, dO [T x H 128]; K, V [T x KV 128]; boxes 64 x 128
+  CUtensorMap mq64, mdo64;      // Q, dO with boxes of 64 columns x 64 rows
   const float* lse;             // [batch][H][seq], natural log
   const float* D;               // [batch][H][seq], rowsum(dO * O)
   float* dQ;                    // [T x H 128]
@@ -909,15 +919,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dq_tc_kernel(const __g
   }
 }
 
-// dK/dV kernel: K and V at 0 and 32 KB, (Q, dO) stages from 64 KB; per stage
-// the query tile's -lse log2e and D in shared vectors; tensor memory S^T 0,
-// dP^T 128, dV 256, dK 384.  P^T / dS^T of the first 64 queries overwrite
-// columns 0-31 of S^T / dP^T, those of the last 64 columns 96-127 (each inside
-// the half row its warp has already read).
-constexpr int kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;  // stage s: Q at +2s, dO at +2s+1 tiles
-constexpr int kKOffBar = 6 * kTile;
-constexpr int kKOffVec = kKOffBar + 256;  // [stage][lse2 | D][128] fp32
-constexpr int kKOffSt = kKOffVec + 2048;  // per-warp store staging
+// dK/dV kernel: K and V at 0 and 32 KB, four (Q, dO) stages of 64 queries
+// from 64 KB (Q 16 KB, dO 16 KB); per stage the tile's -lse log2e and D in
+// shared vectors.  Tensor memory: S^T buffers at 0 and 64 (64 queries each),
+// dP^T buffers at 128 and 192, dV 256, dK 384.  Within a buffer, P^T / dS^T
+// of queries 0-31 overwrite columns 0-15 and those of queries 32-63 columns
+// 48-63 (each inside the 32 columns its warp has read).  With two buffers the
+// next tile's S^T and dP^T run while the softmax warps work on this one.
+constexpr int kQT = 64;                    // queries per tile
+constexpr int kKStages = 4;
+constexpr int kPanel64 = 64 * 128;         // 64 rows x 64 bf16
+constexpr int kKStage = 2 * 2 * kPanel64;  // Q and dO of one tile
+constexpr int kKOffK = 0, kKOffV = kTile, kKOffQ = 2 * kTile;
+constexpr int kKOffBar = 2 * kTile + kKStages * kKStage;
+constexpr int kKOffVec = kKOffBar + 256;  // [stage][lse2 | D][64] fp32
+constexpr int kKOffSt = kKOffVec + kKStages * 2 * kQT * 4;  // per-warp store staging
 constexpr int kKSmem = kKOffSt + 8 * kStageWarp + 1024;
 constexpr uint32_t kColDV = 256, kColDK = 384;
 
@@ -933,9 +949,9 @@ __device__ __forceinline__ KItem kitem_of(const TcBwdP& p, int it) {
   x.b = (it % gb) / p.KV;
   return x;
 }
-// A-operand column of K block kk (16 rows) in the overwritten halves.
+// A-operand column of query block kk (16 queries) in the overwritten halves.
 __device__ __forceinline__ uint32_t half_col(int kk) {
-  return uint32_t(kk < 4 ? kk * 8 : 96 + (kk - 4) * 8);
+  return uint32_t(kk < 2 ? kk * 8 : 48 + (kk - 2) * 8);
 }
 
 __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __grid_constant__ TcBwdP p) {
@@ -945,9 +961,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
   unsigned char* gbase = smem_raw + (base - raw);
   const uint32_t sK = base + kKOffK, sV = base + kKOffV, sQ0 = base + kKOffQ;
   const uint32_t bar = base + kKOffBar;
-  const uint32_t kv_full = bar, kv_empty = bar + 8, qo_full = bar + 16, qo_empty = bar + 32,
-                 vec_full = bar + 48, st_full = bar + 64, p_full = bar + 72, pv_done = bar + 80,
-                 dkv_empty = bar + 88, mma_done = bar + 96;
+  const uint32_t kv_full = bar, kv_empty = bar + 8, qo_full = bar + 16, qo_empty = bar + 48,
+                 vec_full = bar + 80, st_full = bar + 112, p_full = bar + 128,
+                 pv_done = bar + 144, dkv_empty = bar + 160, mma_done = bar + 168;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gbase + kKOffBar + 192);
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + kKOffBar + 200);
   float* vec = reinterpret_cast<float*>(gbase + kKOffVec);
@@ -964,14 +980,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
   if (tid == 32) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(qo_full + 8 * s, 1);
       mbar_init(qo_empty + 8 * s, 1);
       mbar_init(vec_full + 8 * s, 32);
     }
-    mbar_init(st_full, 1);
-    mbar_init(p_full, kSoftWarps);
-    mbar_init(pv_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(st_full + 8 * s, 1);
+      mbar_init(p_full + 8 * s, kSoftWarps);
+      mbar_init(pv_done + 8 * s, 1);
+    }
     mbar_init(dkv_empty, kSoftWarps);
     mbar_init(mma_done, 1);
     *abort = 0;
@@ -991,7 +1009,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
       const int it = item_at(n, G);
       if (it >= p.items_k) break;
       const KItem x = kitem_of(p, it);
-      const int row0 = x.b * p.seq, nq = p.nqb - x.kb;
+      const int row0 = x.b * p.seq, nq2 = 2 * (p.nqb - x.kb);
       ok = __all_sync(0xffffffffu, n == 0 || mbar_wait(kv_empty, uint32_t((n - 1) & 1), abort));
       if (!ok) break;
       if (lane == 0) {
@@ -1003,37 +1021,38 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
         tma_load(sV + kPanel, &p.mv, kv_full, x.g * kHD + 64, y);
       }
       nkv = n + 1;
-      for (int jj = 0; jj < rep * nq; ++jj, ++t) {
-        const int s = t & 1;
-        const int hq = x.g * rep + jj / nq, qt = x.kb + jj % nq;
-        ok = __all_sync(0xffffffffu, t < 2 || mbar_wait(qo_empty + 8 * s,
-                                                        uint32_t(((t - 2) >> 1) & 1), abort));
+      for (int jj = 0; jj < rep * nq2; ++jj, ++t) {
+        const int s4 = t % kKStages;
+        const int hq = x.g * rep + jj / nq2, qt = 2 * x.kb + jj % nq2;  // 64-query tile
+        ok = __all_sync(0xffffffffu,
+                        t < kKStages || mbar_wait(qo_empty + 8 * s4,
+                                                  uint32_t(((t - kKStages) / kKStages) & 1), abort));
         if (!ok) break;
-        const uint32_t sq = sQ0 + uint32_t(2 * s * kTile), so = sq + kTile;
-        const int y = row0 + qt * kRows;
+        const uint32_t sq = sQ0 + uint32_t(s4 * kKStage), so = sq + 2 * kPanel64;
+        const int y = row0 + qt * kQT;
         if (lane == 0) {
-          mbar_expect_tx(qo_full + 8 * s, 2 * kTile);
-          tma_load(sq, &p.mq, qo_full + 8 * s, hq * kHD, y);
-          tma_load(sq + kPanel, &p.mq, qo_full + 8 * s, hq * kHD + 64, y);
-          tma_load(so, &p.mdo, qo_full + 8 * s, hq * kHD, y);
-          tma_load(so + kPanel, &p.mdo, qo_full + 8 * s, hq * kHD + 64, y);
+          mbar_expect_tx(qo_full + 8 * s4, kKStage);
+          tma_load(sq, &p.mq64, qo_full + 8 * s4, hq * kHD, y);
+          tma_load(sq + kPanel64, &p.mq64, qo_full + 8 * s4, hq * kHD + 64, y);
+          tma_load(so, &p.mdo64, qo_full + 8 * s4, hq * kHD, y);
+          tma_load(so + kPanel64, &p.mdo64, qo_full + 8 * s4, hq * kHD + 64, y);
         }
         nqo = t + 1;
         const int64_t l0 = (int64_t(x.b) * p.H + hq) * p.seq;
-        float* vl = vec + s * 2 * kRows;
+        float* vl = vec + s4 * 2 * kQT;
 #pragma unroll
-        for (int c = lane; c < kRows; c += 32) {
-          const int q = qt * kRows + c;
+        for (int c = lane; c < kQT; c += 32) {
+          const int q = qt * kQT + c;
           vl[c] = q < p.seq ? -p.lse[l0 + q] * kLog2ef : 0.f;
-          vl[kRows + c] = q < p.seq ? p.D[l0 + q] : 0.f;
+          vl[kQT + c] = q < p.seq ? p.D[l0 + q] : 0.f;
         }
-        mbar_arrive(vec_full + 8 * s);
+        mbar_arrive(vec_full + 8 * s4);
       }
     }
     if (lane == 0) {
       if (nkv >= 1) mbar_drain(kv_full, uint32_t((nkv - 1) & 1));
-      for (int u = ::max(0, nqo - 2); u < nqo; ++u)
-        mbar_drain(qo_full + 8 * (u & 1), uint32_t((u >> 1) & 1));
+      for (int u = ::max(0, nqo - kKStages); u < nqo; ++u)
+        mbar_drain(qo_full + 8 * (u % kKStages), uint32_t((u / kKStages) & 1));
     }
     __syncwarp();
   } else if (warp == kSoftWarps + 1) {
@@ -1041,57 +1060,74 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
     if (lane == 0) {
       bool ok = true;
       int t = 0;
+      int pv_t = -1, pv_n = 0;  // the pending dV / dK products: tile, item ordinal
+      bool pv_first = false;
+      auto issue_pv = [&]() -> bool {
+        const int bb = pv_t & 1, s4 = pv_t % kKStages;
+        if (!mbar_wait(p_full + 8 * bb, uint32_t((pv_t >> 1) & 1), abort)) return false;
+        // the first products of an item overwrite dV and dK: the previous item's are read
+        if (pv_first && pv_n >= 1 && !mbar_wait(dkv_empty, uint32_t((pv_n - 1) & 1), abort))
+          return false;
+        fence_after();
+        const uint32_t sq = sQ0 + uint32_t(s4 * kKStage), so = sq + 2 * kPanel64;
+        const uint32_t ps = tmem + uint32_t(bb * kQT), pd = tmem + 128u + uint32_t(bb * kQT);
+        // dV += P^T dO and dK += dS^T Q (dO and Q MN-major: two 64-column atoms)
+#pragma unroll
+        for (int kk = 0; kk < kQT / 16; ++kk)
+          mma_ta(tmem + kColDV, ps + half_col(kk), sdesc(so + uint32_t(kk * 2048), kPanel64, 1024),
+                 idesc(1), (!pv_first || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kQT / 16; ++kk)
+          mma_ta(tmem + kColDK, pd + half_col(kk), sdesc(sq + uint32_t(kk * 2048), kPanel64, 1024),
+                 idesc(1), (!pv_first || kk > 0) ? 1u : 0u);
+        commit(pv_done + 8 * bb);
+        commit(qo_empty + 8 * s4);
+        return true;
+      };
       for (int n = 0; ok; ++n) {
         const int it = item_at(n, G);
         if (it >= p.items_k) break;
         const KItem x = kitem_of(p, it);
-        const int ntile = rep * (p.nqb - x.kb);
+        const int ntile = rep * 2 * (p.nqb - x.kb);
+        // the previous item's last products first: its epilogue waits on them
+        if (pv_t >= 0) {
+          if (!issue_pv()) { ok = false; break; }
+          pv_t = -1;
+        }
         if (!mbar_wait(kv_full, uint32_t(n & 1), abort)) { ok = false; break; }
         for (int jj = 0; jj < ntile; ++jj, ++t) {
-          const int s = t & 1;
-          const uint32_t sq = sQ0 + uint32_t(2 * s * kTile), so = sq + kTile;
-          // S^T and dP^T overwrite the columns P^T_{t-1} and dS^T_{t-1} were read from
-          if (!mbar_wait(qo_full + 8 * s, uint32_t((t >> 1) & 1), abort) ||
-              (t >= 1 && !mbar_wait(pv_done, uint32_t((t - 1) & 1), abort))) {
+          const int bb = t & 1, s4 = t % kKStages;
+          const uint32_t sq = sQ0 + uint32_t(s4 * kKStage), so = sq + 2 * kPanel64;
+          // S^T / dP^T buffer t % 2 is free once the products of tile t - 2 are done
+          if (!mbar_wait(qo_full + 8 * s4, uint32_t((t / kKStages) & 1), abort) ||
+              (t >= 2 && !mbar_wait(pv_done + 8 * bb, uint32_t(((t - 2) >> 1) & 1), abort))) {
             ok = false;
             break;
           }
           fence_after();
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
-            mma(tmem, sdesc(sK + off, 16, 1024), sdesc(sq + off, 16, 1024), idesc(0),
-                kk > 0 ? 1u : 0u);
+            const uint32_t ok128 = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            const uint32_t ok64 = uint32_t((kk >> 2) * kPanel64 + (kk & 3) * 32);
+            mma(tmem + uint32_t(bb * kQT), sdesc(sK + ok128, 16, 1024), sdesc(sq + ok64, 16, 1024),
+                idesc(0, kQT), kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kHD / 16; ++kk) {
-            const uint32_t off = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
-            mma(tmem + kColDP, sdesc(sV + off, 16, 1024), sdesc(so + off, 16, 1024), idesc(0),
-                kk > 0 ? 1u : 0u);
+            const uint32_t ok128 = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            const uint32_t ok64 = uint32_t((kk >> 2) * kPanel64 + (kk & 3) * 32);
+            mma(tmem + 128u + uint32_t(bb * kQT), sdesc(sV + ok128, 16, 1024),
+                sdesc(so + ok64, 16, 1024), idesc(0, kQT), kk > 0 ? 1u : 0u);
           }
-          commit(st_full);
+          commit(st_full + 8 * bb);
           if (jj == ntile - 1) commit(kv_empty);  // K and V of this block are read
-          if (!mbar_wait(p_full, uint32_t(t & 1), abort) ||
-              (jj == 0 && n >= 1 && !mbar_wait(dkv_empty, uint32_t((n - 1) & 1), abort))) {
-            ok = false;
-            break;
-          }
-          fence_after();
-          // dV += P^T dO and dK += dS^T Q (dO and Q MN-major)
-#pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_ta(tmem + kColDV, tmem + half_col(kk),
-                   sdesc(so + uint32_t(kk * 2048), kPanel, 1024), idesc(1),
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_ta(tmem + kColDK, tmem + kColDP + half_col(kk),
-                   sdesc(sq + uint32_t(kk * 2048), kPanel, 1024), idesc(1),
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-          commit(pv_done);
-          commit(qo_empty + 8 * s);
+          if (pv_t >= 0 && !issue_pv()) { ok = false; break; }
+          pv_t = t;
+          pv_n = n;
+          pv_first = jj == 0;
         }
       }
+      if (ok && pv_t >= 0) issue_pv();
       commit(mma_done);
       mbar_drain(mma_done, 0);
     }
@@ -1101,36 +1137,36 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
     const int lq = warp & 3, hf = warp >> 2;
     const int r = lq * 32 + lane;
     const uint32_t lbase = tmem + (uint32_t(lq * 32) << 16);
-    const uint32_t ocol = hf ? 96u : 0u;  // where this half's bf16 pairs go
+    const uint32_t ocol = hf ? 48u : 0u;  // where this half's bf16 pairs go
     bool ok = true;
     int t = 0;
     for (int n = 0;; ++n) {
       const int it = item_at(n, G);
       if (it >= p.items_k) break;
       const KItem x = kitem_of(p, it);
-      const int nq = p.nqb - x.kb, ntile = rep * nq;
+      const int nq2 = 2 * (p.nqb - x.kb), ntile = rep * nq2;
       const int key = x.kb * kRows + r;
       for (int jj = 0; jj < ntile; ++jj, ++t) {
-        const int s = t & 1;
-        const int qt = x.kb + jj % nq;
-        ok = __all_sync(0xffffffffu, ok && mbar_wait(vec_full + 8 * s, uint32_t((t >> 1) & 1), abort) &&
-                                         mbar_wait(st_full, uint32_t(t & 1), abort));
+        const int bb = t & 1, s4 = t % kKStages;
+        const int qt = 2 * x.kb + jj % nq2;
+        ok = __all_sync(0xffffffffu,
+                        ok && mbar_wait(vec_full + 8 * s4, uint32_t((t / kKStages) & 1), abort) &&
+                            mbar_wait(st_full + 8 * bb, uint32_t((t >> 1) & 1), abort));
         if (!ok) continue;
         fence_after();
-        uint32_t sv[kHalf], dp[kHalf];
-        tld32(lbase + uint32_t(hf * kHalf), sv);
-        tld32(lbase + uint32_t(hf * kHalf + 32), sv + 32);
-        tld32(lbase + kColDP + uint32_t(hf * kHalf), dp);
-        tld32(lbase + kColDP + uint32_t(hf * kHalf + 32), dp + 32);
+        const uint32_t cs = lbase + uint32_t(bb * kQT), cd = cs + 128u;
+        uint32_t sv[32], dp[32];
+        tld32(cs + uint32_t(hf * 32), sv);
+        tld32(cd + uint32_t(hf * 32), dp);
         tld_wait();
         // query columns c of this half with key <= query < seq
-        const int q0 = qt * kRows + hf * kHalf;
+        const int q0 = qt * kQT + hf * 32;
         const int lo = key - q0, hi = p.seq - q0;  // keep lo <= c < hi
-        const float4* vl = reinterpret_cast<const float4*>(vec + s * 2 * kRows + hf * kHalf);
-        const float4* vd = reinterpret_cast<const float4*>(vec + s * 2 * kRows + kRows + hf * kHalf);
-        uint32_t pp[kHalf / 2], pd[kHalf / 2];
+        const float4* vl = reinterpret_cast<const float4*>(vec + s4 * 2 * kQT + hf * 32);
+        const float4* vd = reinterpret_cast<const float4*>(vec + s4 * 2 * kQT + kQT + hf * 32);
+        uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int v = 0; v < kHalf / 4; ++v) {
+        for (int v = 0; v < 8; ++v) {
           const float4 l4 = vl[v], d4 = vd[v];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
           float pe[4], de[4];
@@ -1147,15 +1183,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
           pd[2 * v] = pack_bf16x2(de[0], de[1]);
           pd[2 * v + 1] = pack_bf16x2(de[2], de[3]);
         }
-        tst32(lbase + ocol, pp);
-        tst32(lbase + kColDP + ocol, pd);
+        tst16(cs + ocol, pp);
+        tst16(cd + ocol, pd);
         tst_wait();
         fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(p_full + 8 * bb);
       }
       const int tl = t - 1;
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(pv_done, uint32_t(tl & 1), abort));
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(pv_done + 8 * (tl & 1),
+                                                   uint32_t((tl >> 1) & 1), abort));
       if (ok) {
         fence_after();
         uint32_t a[kHalf], c[kHalf];
@@ -1214,7 +1251,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_bwd_dkv_tc_kernel(const __
 PFN_cuTensorMapEncodeTiled_v12000 g_enc = nullptr;
 std::once_flag g_enc_once;
 
-slora_status encode_rows(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+slora_status encode_rows(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
+                         int box_rows = kRows) {
   std::call_once(g_enc_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -1226,7 +1264,7 @@ slora_status encode_rows(CUtensorMap* m, const void* ptr, int64_t rows, int64_t 
   if (!g_enc) SLORA_FAIL(SLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
   cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
-  cuuint32_t box[2] = {64, cuuint32_t(kRows)};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   cuuint32_t es[2] = {1, 1};
   const CUresult r = g_enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1285,6 +1323,8 @@ slora_status attention_bwd_tc_run(const void* Q, const void* K, const void* V, c
   SLORA_TRY(encode_rows(&p.mdo, dO, ti.T, int64_t(H) * kHD));
   SLORA_TRY(encode_rows(&p.mk, K, ti.T, int64_t(KV) * kHD));
   SLORA_TRY(encode_rows(&p.mv, V, ti.T, int64_t(KV) * kHD));
+  SLORA_TRY(encode_rows(&p.mq64, Q, ti.T, int64_t(H) * kHD, kQT));
+  SLORA_TRY(encode_rows(&p.mdo64, dO, ti.T, int64_t(H) * kHD, kQT));
   p.lse = lse; p.D = D; p.dQ = dQ; p.dK = dK;
   p.dV = static_cast<__nv_bfloat16*>(dV);
   p.seq = ti.seq; p.H = H; p.KV = KV; p.batch = ti.batch;
