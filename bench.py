@@ -629,6 +629,7 @@ def run_ffn(args, H, pk, rank, world):
     ps = FfnLayer(w, d, F, rs, r, case.lora_scale, tok.batch, tok.seq, tok.ctx_len,
                   wl["sparsity"], layers[0].X, layers[0].dOut, per_sequence=True)
     ws_ps = torch.empty(ps.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    ps.step(ws_ps)  # eager first: the library creates its lane streams outside the capture
     g_ps = H.capture(lambda: ps.step(ws_ps))
     g_ps.replay()
     n_ps = max(3, args.steps // 2)

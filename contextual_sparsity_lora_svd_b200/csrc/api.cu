@@ -440,7 +440,14 @@ slora_status ffn_per_seq_run(const FfnDesc& F, const slora_tokens* tok, const vo
     gtot += (glen[q] + 63) / 64 * 64;
   }
   float* gbuf = fwd_only ? nullptr : ar.take<float>(size_t(B) * gtot);
-  // one sub-workspace, reused by every sequence in stream order
+  // The sequences run in up to kSeqLanes lanes at once: lane 0 on the
+  // caller's stream, lane i on side stream i of the library's pool, each
+  // with its own sub-workspace (reused by its sequences in stream order) and
+  // its own side stream for the operand layouts.  Every sequence writes its
+  // own rows, index list and gradient slot; the gradients are summed in
+  // sequence order afterwards, so the result does not depend on the lanes.
+  constexpr int kSeqLanes = 4;
+  const int lanes = std::min(B, kSeqLanes);
   size_t sub = 16;
   for (int b = 0; b < B; ++b) {
     slora_tokens tb{1, seq, &tok->ctx_len[b]};
@@ -450,12 +457,27 @@ slora_status ffn_per_seq_run(const FfnDesc& F, const slora_tokens* tok, const vo
     SLORA_TRY(ffn_run(Fb, &tb, X, dOut, out, dX, idx, idx_force, p, true, nullptr));
     sub = std::max(sub, p.used);
   }
-  char* subws = ar.take<char>(sub);
+  char* subws[kSeqLanes] = {};
+  for (int i = 0; i < lanes; ++i) subws[i] = ar.take<char>(sub);
   if (plan) return SLORA_OK;
   SLORA_TRY(arena_fits(ar, "slora_ffn_fwd_bwd_per_seq"));
+  // one lane while a capture is under way and the stream pool does not exist
+  // yet (streams are not created inside a capture)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  SLORA_CUDA(cudaStreamIsCapturing(st, &cap));
+  const int nl =
+      (cap == cudaStreamCaptureStatusNone || side_pool_ready(2 * kSeqLanes)) ? lanes : 1;
+  cudaStream_t lane_st[kSeqLanes] = {st}, lane_side[kSeqLanes] = {};
+  for (int i = 0; i < nl; ++i) {
+    if (i > 0) SLORA_TRY(side_stream_at(i, &lane_st[i]));
+    SLORA_TRY(side_stream_at(kSeqLanes + i, &lane_side[i]));
+  }
+  for (int i = 1; i < nl; ++i) SLORA_TRY(fork_side(st, lane_st[i]));
   for (int b = 0; b < B; ++b) {
+    const int ln = b % nl;
     slora_tokens tb{1, seq, &tok->ctx_len[b]};
     FfnDesc Fb = F;
+    Fb.side = lane_side[ln];
     SLORA_TRY(parse_tokens(&tb, &Fb.ti));
     if (!fwd_only) {
       float* g = gbuf + size_t(b) * gtot;
@@ -467,12 +489,14 @@ slora_status ffn_per_seq_run(const FfnDesc& F, const slora_tokens* tok, const vo
       return p ? static_cast<const char*>(p) + row0 * d * es : nullptr;
     };
     Arena a;
-    a.base = subws;
+    a.base = subws[ln];
     a.cap = sub;
     SLORA_TRY(ffn_run(Fb, &tb, at(X), at(dOut), const_cast<char*>(at(out)),
                       const_cast<char*>(at(dX)), idx + int64_t(b) * Fd,
-                      idx_force ? idx_force + int64_t(b) * k_force : nullptr, a, false, st));
+                      idx_force ? idx_force + int64_t(b) * k_force : nullptr, a, false,
+                      lane_st[ln]));
   }
+  for (int i = 1; i < nl; ++i) SLORA_TRY(join_side(st, lane_st[i]));
   if (fwd_only) return SLORA_OK;
   float* dst[6] = {F.G.dAg, F.G.dBg, F.G.dAu, F.G.dBu, F.G.dAd, F.G.dBd};
   SumSeg segs[6];

@@ -101,6 +101,13 @@ slora_status launch_rowmaps(const slora_tokens* tok, const TokenInfo& ti, int32_
 // for what was issued on `side` since.  Both are stream-ordered (they work
 // inside a CUDA-graph capture of `st`).
 slora_status side_stream(cudaStream_t* side);
+// Entry i of a per-device pool of kSidePool such streams (entry 0 is the one
+// side_stream() gives), each with its own fork and join events; fork_side /
+// join_side take any pool stream.  side_pool_ready(n): entries 1 .. n - 1
+// exist (creating one is not done while a stream is being captured).
+constexpr int kSidePool = 8;
+slora_status side_stream_at(int i, cudaStream_t* side);
+bool side_pool_ready(int n);
 slora_status fork_side(cudaStream_t st, cudaStream_t side);
 slora_status join_side(cudaStream_t st, cudaStream_t side);
 // Number of 128-row tiles of the context rows / output rows.

@@ -424,8 +424,8 @@ slora_status ffn_run_tc(const FfnDesc& F, const slora_tokens* tok, const void* X
   // the pass over X and the estimator (first those independent of the
   // selection, then, once it is known, the ones on the kept channels); the
   // main stream joins them before the first GEMM.
-  cudaStream_t side = nullptr;
-  SLORA_TRY(side_stream(&side));
+  cudaStream_t side = F.side;
+  if (!side) SLORA_TRY(side_stream(&side));
   SLORA_TRY(fork_side(st, side));
   SLORA_TRY(pack_gate_up_b(L.Bg, L.Bu, nullptr, Fd, r, nntO, lr2, BpO, side, Fd));
   SLORA_TRY(transpose_rows(L.Ad, r, Fd, nullptr, Fd, lr, Adt, side));

@@ -35,6 +35,7 @@ struct FfnDesc {
   slora_ffn_grads G;
   int64_t kkeep;
   double sparsity;  // ratio the estimator selects at (unused with idx_force)
+  cudaStream_t side = nullptr;  // side stream for the small operand layouts (null: the default one)
 };
 
 slora_status ffn_run(const FfnDesc& F, const slora_tokens* tok, const void* X, const void* dOut,

@@ -163,14 +163,17 @@ struct Side {
   cudaEvent_t fork = nullptr, join = nullptr;
 };
 std::mutex g_side_mu;
-Side g_side[kSideDevices];
-slora_status side_for(Side** out) {
+// Per device: entry 0 is the side stream of a single call; the others serve
+// calls that run several lanes of work at once.
+Side g_side[kSideDevices][kSidePool];
+slora_status side_for(int i, Side** out) {
   int dev = -1;
   SLORA_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kSideDevices)
     SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kSideDevices);
+  if (i < 0 || i >= kSidePool) SLORA_FAIL(SLORA_ERR_INVALID_ARG, "side stream %d of %d", i, kSidePool);
   std::lock_guard<std::mutex> lock(g_side_mu);
-  Side& sd = g_side[dev];
+  Side& sd = g_side[dev][i];
   if (!sd.s) {
     SLORA_CUDA(cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking));
     SLORA_CUDA(cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming));
@@ -179,20 +182,48 @@ slora_status side_for(Side** out) {
   *out = &sd;
   return SLORA_OK;
 }
+// The pool entry of stream `side` on the current device.
+slora_status side_of(cudaStream_t side, Side** out) {
+  int dev = -1;
+  SLORA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kSideDevices)
+    SLORA_FAIL(SLORA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kSideDevices);
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  for (int i = 0; i < kSidePool; ++i)
+    if (g_side[dev][i].s == side && side) {
+      *out = &g_side[dev][i];
+      return SLORA_OK;
+    }
+  SLORA_FAIL(SLORA_ERR_INVALID_ARG, "internal error: stream is not a library side stream");
+}
 }  // namespace
 
-slora_status side_stream(cudaStream_t* side) {
+slora_status side_stream(cudaStream_t* side) { return side_stream_at(0, side); }
+
+slora_status side_stream_at(int i, cudaStream_t* side) {
   Side* sd = nullptr;
-  SLORA_TRY(side_for(&sd));
+  SLORA_TRY(side_for(i, &sd));
   *side = sd->s;
   return SLORA_OK;
+}
+
+bool side_pool_ready(int n) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSideDevices || n > kSidePool) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  for (int i = 1; i < n; ++i)
+    if (!g_side[dev][i].s) return false;
+  return true;
 }
 
 // The record and the wait happen under the lock, so calls from several host
 // threads cannot interleave on the shared events.
 slora_status fork_side(cudaStream_t st, cudaStream_t side) {
   Side* sd = nullptr;
-  SLORA_TRY(side_for(&sd));
+  SLORA_TRY(side_of(side, &sd));
   std::lock_guard<std::mutex> lock(g_side_mu);
   SLORA_CUDA(cudaEventRecord(sd->fork, st));
   SLORA_CUDA(cudaStreamWaitEvent(side, sd->fork, 0));
@@ -201,7 +232,7 @@ slora_status fork_side(cudaStream_t st, cudaStream_t side) {
 
 slora_status join_side(cudaStream_t st, cudaStream_t side) {
   Side* sd = nullptr;
-  SLORA_TRY(side_for(&sd));
+  SLORA_TRY(side_of(side, &sd));
   std::lock_guard<std::mutex> lock(g_side_mu);
   SLORA_CUDA(cudaEventRecord(sd->join, side));
   SLORA_CUDA(cudaStreamWaitEvent(st, sd->join, 0));

@@ -71,3 +71,77 @@ def test_ffn_per_sequence_sets(L, bf16):
                         per_sequence=True)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
+
+
+def test_ffn_per_sequence_lanes_match_single_sequence_calls(L):
+    """Six sequences run in four concurrent lanes (two lanes take two
+    sequences each, reusing their sub-workspace): every sequence's output
+    rows, input gradient and index list equal, bit for bit, a separate call
+    on that sequence alone; the LoRA gradients equal the sequence-ordered sum
+    of the separate calls' gradients; and a CUDA-graph replay of the call
+    reproduces the eager result exactly."""
+    B, seq, d, F, r = 6, 64, 128, 344, 8
+    tok = synth.Tokens(B, seq, np.array([48, 64, 30, 0, 57, 41], np.int32))
+    case = synth.ffn_case(tok, d=d, d_ff=F, r_svd=8, r_lora=r, sparsity=0.5, bf16=True,
+                          workload=0, layer=13)
+    dt = torch.bfloat16
+    t = {k: dev(getattr(case, k), dt) for k in ("Ag", "Bg", "Au", "Bu", "Ad", "Bd")}
+    W = {"Wg": dev(case.Wg.W, dt), "Wu": dev(case.Wu.W, dt), "Wd_t": dev(case.Wd.W.T.copy(), dt)}
+    fac = {}
+    fac["Lg"], fac["Ug"] = (dev(a, torch.float32) for a in O.svd_prepare(case.Wg.W, 8))
+    fac["Lu"], fac["Uu"] = (dev(a, torch.float32) for a in O.svd_prepare(case.Wu.W, 8))
+    layer = L.ffn_layer_struct(d, F, 8, r, case.lora_scale, W["Wg"], W["Wu"], W["Wd_t"], t["Ag"],
+                               t["Bg"], t["Au"], t["Bu"], t["Ad"], t["Bd"], fac["Lg"], fac["Ug"],
+                               fac["Lu"], fac["Uu"])
+    X, dOut = dev(case.X, dt), dev(case.dOut, dt)
+    shapes = (("dAg", (r, d)), ("dBg", (F, r)), ("dAu", (r, d)), ("dBu", (F, r)),
+              ("dAd", (r, F)), ("dBd", (d, r)))
+
+    def run(per_seq_tok, Xs, dOs, graph=False):
+        T = Xs.shape[0]
+        out = torch.zeros(T, d, dtype=dt, device="cuda")
+        dX = torch.zeros(T, d, dtype=dt, device="cuda")
+        g = {k: torch.zeros(sh, device="cuda") for k, sh in shapes}
+        grads = L.ffn_grads_struct(*(g[k] for k, _ in shapes))
+        idx = torch.full((per_seq_tok.batch * F,), -1, dtype=torch.int32, device="cuda")
+        call = lambda: L.slora_ffn_fwd_bwd(layer, per_seq_tok.batch, per_seq_tok.seq,
+                                           per_seq_tok.ctx_len, 0.5, Xs, dOs, out, dX, grads,
+                                           idx, per_sequence=True)
+        k = call()
+        if graph:
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                cg = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(cg, stream=s):
+                    call()
+            res = []
+            for _ in range(2):
+                for v in g.values():
+                    v.zero_()
+                cg.replay()
+                torch.cuda.synchronize()
+                res.append((out.clone(), dX.clone(), {n: v.clone() for n, v in g.items()}))
+            return k, idx, res
+        torch.cuda.synchronize()
+        return k, idx, (out, dX, g)
+
+    k, idx, (out, dX, g) = run(tok, X, dOut)
+    acc = {n: torch.zeros(sh, device="cuda") for n, sh in shapes}
+    for b in range(B):
+        rows = slice(b * seq, (b + 1) * seq)
+        tb = synth.Tokens(1, seq, tok.ctx_len[b:b + 1].copy())
+        kb, ib, (ob, xb, gb) = run(tb, X[rows].contiguous(), dOut[rows].contiguous())
+        assert kb == k
+        assert torch.equal(idx[b * F:b * F + k], ib[:k]), f"sequence {b} selection"
+        assert torch.equal(out[rows], ob), f"sequence {b} output"
+        assert torch.equal(dX[rows], xb), f"sequence {b} input gradient"
+        for n in acc:
+            acc[n] += gb[n]
+    for n in acc:
+        torch.testing.assert_close(g[n], acc[n], rtol=1e-5, atol=1e-6)
+    _, _, res = run(tok, X, dOut, graph=True)
+    for o2, x2, g2 in res:
+        assert torch.equal(o2, out) and torch.equal(x2, dX)
+        for n in g:
+            assert torch.equal(g2[n], g[n]), n
