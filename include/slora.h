@@ -391,7 +391,13 @@ slora_status slora_ffn_bwd(slora_dtype dt, const slora_ffn_layer* layer, const s
  *             (ascending) at idx_out + b*d_ff.
  *   idx_force optional device int32 [batch x k_force]: sequence b's forced set
  *             at idx_force + b*k_force.
- *   The workspace holds one set of LoRA gradients per sequence.
+ *   The workspace holds one set of LoRA gradients per sequence and one
+ *   per-sequence working area for each of up to four lanes. The sequences run
+ *   in those lanes at once: lane 0 on `stream`, the others on library-owned
+ *   streams that fork from `stream` and join it before the call returns in
+ *   stream order. The result does not depend on the lanes. The first call on
+ *   a device creates the lane streams; a call captured into a CUDA graph
+ *   before that runs one lane.
  */
 slora_status slora_ffn_fwd_bwd_per_seq(slora_dtype dt, const slora_ffn_layer* layer,
                                        const slora_tokens* tok, double sparsity, const void* X,
