@@ -60,17 +60,64 @@ class _Call:
         L._check(self.name, self.fn(*self.args, ws_ptr, ctypes.byref(ws_bytes), stream))
 
 
+class _Par:
+    """Independent call lists issued at once: the first runs on the runner's
+    stream and workspace, list i > 0 on the runner's branch stream i - 1 with
+    its own branch workspace.  The branches fork from the runner's stream
+    and are joined back into it (events, so this holds inside a CUDA-graph
+    capture too).  The lists must not share any buffer they write."""
+
+    def __init__(self, *branches):
+        self.branches = [list(b) for b in branches]
+        self.fork = torch.cuda.Event()
+        self.joins = [torch.cuda.Event() for _ in self.branches[1:]]
+
+
 class _Runner:
     calls: list
+    _bstreams: list = []
+    _bws: list = []
+
+    def _main_calls(self):
+        for c in self.calls:
+            if isinstance(c, _Par):
+                yield from c.branches[0]
+            else:
+                yield c
 
     def workspace_bytes(self) -> int:
-        return max([c.need() for c in self.calls if c.own_ws is None] + [16])
+        return max([c.need() for c in self._main_calls() if c.own_ws is None] + [16])
+
+    def _setup_branches(self):
+        """Streams and workspaces of the branches of the _Par groups."""
+        pars = [c for c in self.calls if isinstance(c, _Par)]
+        nb = max([len(c.branches) for c in pars] + [1])
+        self._bstreams = [torch.cuda.Stream() for _ in range(nb - 1)]
+        self._bws = []
+        for i in range(1, nb):
+            need = max([16] + [x.need() for c in pars if len(c.branches) > i
+                               for x in c.branches[i]])
+            self._bws.append(torch.empty(need, dtype=torch.uint8, device="cuda"))
 
     def step(self, ws: torch.Tensor, stream=None):
-        st = (stream or torch.cuda.current_stream()).cuda_stream
+        cur = stream or torch.cuda.current_stream()
+        st = cur.cuda_stream
         ptr, nb = ws.data_ptr(), L.c_sz(ws.numel())
         for c in self.calls:
-            c(ptr, nb, st)
+            if not isinstance(c, _Par):
+                c(ptr, nb, st)
+                continue
+            c.fork.record(cur)
+            for i, br in enumerate(c.branches[1:]):
+                bs, bw = self._bstreams[i], self._bws[i]
+                bs.wait_event(c.fork)
+                for x in br:
+                    x(bw.data_ptr(), L.c_sz(bw.numel()), bs.cuda_stream)
+                c.joins[i].record(bs)
+            for x in c.branches[0]:
+                x(ptr, nb, st)
+            for e in c.joins:
+                cur.wait_event(e)
 
 
 class FfnLayer(_Runner):
@@ -442,7 +489,9 @@ class DecoderStack(_Runner):
             o_b = _Call("slora_linear_bwd", obase + [L.ptr(S_["O"]), None, L.ptr(S_["XAo"]),
                                                      L.ptr(dh), None, L.ptr(dO_att), None,
                                                      L.ptr(G["dAo"]), L.ptr(G["dBo"])])
-            calls += [proj["q"][0], proj["k"][0], v_f, proj["q"][1], proj["k"][1], att_f, o_f]
+            # q, k and v (with the rotary packing of q and k) run at once
+            calls += [_Par([proj["q"][0], proj["q"][1]], [proj["k"][0], proj["k"][1]], [v_f]),
+                      att_f, o_f]
             # -- residual + second normalisation, FFN forward (its own selection)
             calls.append(_Call("slora_rmsnorm_fwd", [L.BF16, T, d, L.c_f32(eps),
                                                      L.ptr(self.x[l]), L.ptr(a_out),
@@ -488,8 +537,8 @@ class DecoderStack(_Runner):
             calls.append(_Call("slora_rmsnorm_bwd", [L.BF16, T, d, L.ptr(S_["h"]),
                                                      L.ptr(S_["r2"]), L.ptr(w["g2"]), L.ptr(dn2),
                                                      None, None, L.ptr(dx_cur), L.ptr(dh)]))
-            calls += [B["o_b"], B["att_b"], B["q"][2], B["k"][2], B["q"][3], B["k"][3],
-                      B["v_b"]]
+            calls += [B["o_b"], B["att_b"],
+                      _Par([B["q"][2], B["q"][3]], [B["k"][2], B["k"][3]], [B["v_b"]])]
             calls.append(_Call("slora_rmsnorm_bwd", [L.BF16, T, d, L.ptr(self.x[l]),
                                                      L.ptr(S_["r1"]), L.ptr(w["g1"]), L.ptr(dxq),
                                                      L.ptr(dxk), L.ptr(dxv), L.ptr(dh),
@@ -497,3 +546,4 @@ class DecoderStack(_Runner):
             dx_cur = dx_next
         self.dX = dx_cur
         self.calls = calls
+        self._setup_branches()
