@@ -77,6 +77,10 @@ class _Runner:
     calls: list
     _bstreams: list = []
     _bws: list = []
+    # serial: the branches of each _Par group run one after another on the
+    # runner's stream (each still on its own workspace); for per-launch
+    # timings that must not include other branches' work
+    serial = False
 
     def _main_calls(self):
         for c in self.calls:
@@ -106,6 +110,14 @@ class _Runner:
         for c in self.calls:
             if not isinstance(c, _Par):
                 c(ptr, nb, st)
+                continue
+            if self.serial:
+                for x in c.branches[0]:
+                    x(ptr, nb, st)
+                for i, br in enumerate(c.branches[1:]):
+                    bw = self._bws[i]
+                    for x in br:
+                        x(bw.data_ptr(), L.c_sz(bw.numel()), st)
                 continue
             c.fork.record(cur)
             for i, br in enumerate(c.branches[1:]):
@@ -305,9 +317,11 @@ class AttnLinears(_Runner):
                        grads["dBo"])
             fwds.append(f)
             bwds.append(b)
-        # step: estimators, forwards (q, k, v, o), backwards in reverse order
-        self.calls = calls + fwds + bwds[::-1]
+        # step: estimators, then the four forwards at once, then the four
+        # backwards at once (each projection writes only its own buffers)
+        self.calls = calls + [_Par(*([f] for f in fwds)), _Par(*([b] for b in bwds[::-1]))]
         self.X, self.attn_out, self.dY_o = X, attn_out, dY_o
+        self._setup_branches()
 
 
 class DecoderStack(_Runner):

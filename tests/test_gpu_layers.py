@@ -65,8 +65,19 @@ def test_attention_linears_step(L, H, KV, pairs, vo):
                       _bf(X), _bf(attn), _bf(dYo), _bf(dq), _bf(dk), _bf(dv), pairs=pairs,
                       vo_sparsity=vo)
     ws = torch.empty(run.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    # the four projections run as parallel branches; issued one after another
+    # (the profiling mode) they must give the same bits
+    run.serial = True
     run.step(ws)
     torch.cuda.synchronize()
+    serial = [host(t).copy() for t in run.dX.values()] + [host(run.gflat).copy()]
+    run.serial = False
+    run.gflat.zero_()
+    run.step(ws)
+    torch.cuda.synchronize()
+    par = [host(t) for t in run.dX.values()] + [host(run.gflat)]
+    for a, b in zip(serial, par):
+        assert np.array_equal(a, b), "parallel branches changed the result"
     C, Orow = O.context_rows(tok.batch, tok.seq, tok.ctx_len)
     # q/k selection against the oracle's
     est = O.estimate_select_qk_pairs if pairs else O.estimate_select_qk
