@@ -317,9 +317,12 @@ class AttnLinears(_Runner):
                        grads["dBo"])
             fwds.append(f)
             bwds.append(b)
-        # step: estimators, then the four forwards at once, then the four
-        # backwards at once (each projection writes only its own buffers)
-        self.calls = calls + [_Par(*([f] for f in fwds)), _Par(*([b] for b in bwds[::-1]))]
+        # step: estimators; q, k and v forwards at once (each writes only its
+        # own buffers), then o, whose input in a layer is the attention output
+        # over q, k, v; backward: o first (its input gradient feeds the
+        # attention backward), then q, k and v at once
+        self.calls = calls + [_Par([fwds[0]], [fwds[1]], [fwds[2]]), fwds[3], bwds[3],
+                              _Par([bwds[2]], [bwds[1]], [bwds[0]])]
         self.X, self.attn_out, self.dY_o = X, attn_out, dY_o
         self._setup_branches()
 
