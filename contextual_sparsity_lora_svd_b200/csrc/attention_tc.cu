@@ -631,11 +631,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) attn_fwd_tc_kernel(const __grid
 //       tensor-memory A operand and K_j MN-major.  dQ = scale dQ, fp32.
 //   attn_bwd_dkv_tc_kernel  per (key block, key/value head, sequence): K
 //       and V stay in shared memory; for every query head of the group and
-//       query tile at or after the block, S^T = K Q^T and dP^T = V dO^T; the
-//       softmax warps (key rows) form P^T and dS^T and write them (bf16
-//       pairs) over the half rows of S^T and dP^T they have read; dV +=
-//       P^T dO and dK += dS^T Q (Q and dO MN-major).  dK = scale dK (fp32),
-//       dV bf16.
+//       64-query tile at or after the block, S^T = K Q^T and dP^T = V dO^T
+//       into one of two tensor-memory buffers; the softmax warps (key rows)
+//       form P^T and dS^T and write them (bf16 pairs) over the half rows of
+//       S^T and dP^T they have read; dV += P^T dO and dK += dS^T Q (Q and
+//       dO MN-major).  dK = scale dK (fp32), dV bf16.
 struct TcBwdP {
   CUtensorMap mq, mk, mv, mdo;  // Q, dO [T x H 128]; K, V [T x KV 128]; boxes 64 x 128
   CUtensorMap mq64, mdo64;      // Q, dO with boxes of 64 columns x 64 rows
